@@ -1,0 +1,477 @@
+#!/usr/bin/env python
+"""Benchmark of the HHR decode step on B200.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--impl hhr|reference]
+                    [--workload NAME]
+
+One step = one decode token of the workload: hhr_decode_step on every layer
+in order (32 layers of Llama-3.1-8B shape at 128K context by default),
+captured in one CUDA graph.  Inputs are resident in HBM before timing; the
+KV cache (17.5 GB) is far larger than L2, so every layer's bytes are evicted
+by the other 31 layers before they are read again (no L2 flush needed).
+
+Rank 0 prints one JSON line.  Under torchrun every rank runs its own replica
+of the workload (independent sequences, no collective on the data path);
+`value` counts the tokens of all ranks over the slowest rank's time.
+`--impl reference` times the fp64 CPU oracle instead (bounded sample).
+"""
+from __future__ import annotations
+
+import argparse
+import json
+import math
+import os
+import statistics
+import subprocess
+import sys
+import threading
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+if ROOT not in sys.path:
+    sys.path.insert(0, ROOT)
+
+METRIC = "HHR decode-attention tokens/s at 128K ctx; achieved HBM GB/s vs ~8 TB/s peak"
+
+
+def parse_args(argv=None):
+    p = argparse.ArgumentParser()
+    p.add_argument("--gpus", type=int, default=1)
+    p.add_argument("--steps", type=int, default=200)
+    p.add_argument("--warmup", type=int, default=10)
+    p.add_argument("--impl", choices=["hhr", "reference"], default="hhr")
+    p.add_argument("--workload", default="llama_32l_128k")
+    p.add_argument("--layers", type=int, default=None, help="fewer layers (profiling runs only)")
+    p.add_argument("--no-dense", action="store_true")
+    p.add_argument("--no-cpu-baseline", action="store_true")
+    p.add_argument("--cpu-seconds", type=float, default=12.0)
+    p.add_argument("--soak-seconds", type=float, default=1.0)
+    return p.parse_args(argv)
+
+
+# ---------------------------------------------------------------------------
+# distributed plumbing (host side; CPU-testable with gloo)
+# ---------------------------------------------------------------------------
+
+def dist_env():
+    return int(os.environ.get("RANK", 0)), int(os.environ.get("LOCAL_RANK", 0)), int(os.environ.get("WORLD_SIZE", 1))
+
+
+def dist_init(backend: str):
+    import datetime
+    import torch.distributed as dist
+    rank, _, world = dist_env()
+    if world > 1 and not dist.is_initialized():
+        dist.init_process_group(backend, timeout=datetime.timedelta(seconds=120))
+    return rank, world
+
+
+def max_over_ranks(x: float, world: int, device=None) -> float:
+    if world <= 1:
+        return x
+    import torch
+    import torch.distributed as dist
+    t = torch.tensor([x], dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def barrier(world: int, device=None):
+    if world > 1:
+        import torch.distributed as dist
+        if device is not None and device.type == "cuda":
+            dist.barrier(device_ids=[device.index])
+        else:
+            dist.barrier()
+
+
+def whole_job_throughput(units_per_rank: float, world: int, max_seconds: float) -> float:
+    """Units processed by all ranks divided by the slowest rank's time."""
+    return units_per_rank * world / max_seconds
+
+
+# ---------------------------------------------------------------------------
+# algorithmic bytes (what the method must touch per decode step)
+# ---------------------------------------------------------------------------
+
+def hhr_bytes_per_head(L: int, P: int, N: int, k: int, G: int, nb: int, d: int = 128) -> dict:
+    """Bytes one (sequence, KV head) decode must move: page metadata, codes of
+    the candidate rows, the kept K'/V rows, q and out, and R_h, W_h."""
+    np_ = -(-L // P)
+    Neff = min(N, np_)
+    # candidate rows: exact when every kept page is full (L a multiple of P, or
+    # the partial last page not kept); otherwise over by fewer than P rows
+    cand = min(Neff * P, L)
+    keff = min(k, cand)
+    return dict(meta=np_ * 2 * d * 2, codes=cand * (nb // 8), gather=keff * 2 * d * 2,
+                qo=G * (d * 2 + d * 4), rw=d * d * 4 + nb * d * 2, cand=cand, keff=keff, pages=Neff)
+
+
+def dense_bytes_per_head(L: int, G: int, d: int = 128) -> int:
+    return L * 2 * d * 2 + G * (d * 2 + d * 4) + d * d * 4
+
+
+# ---------------------------------------------------------------------------
+# clocks sampled during the timed region
+# ---------------------------------------------------------------------------
+
+class ClockSampler:
+    FIELDS = ("clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.hw_slowdown,"
+              "clocks_event_reasons.hw_thermal_slowdown,clocks_event_reasons.sw_thermal_slowdown,"
+              "clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, gpu_id: str):
+        self.gpu_id = gpu_id
+        self.proc = None
+        self.lines = []
+
+    def start(self):
+        try:
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", f"--id={self.gpu_id}", f"--query-gpu={self.FIELDS}", "--format=csv,noheader,nounits",
+                 "-lms", "100"], stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+            self.thread = threading.Thread(target=self._read, daemon=True)
+            self.thread.start()
+        except (OSError, FileNotFoundError):
+            self.proc = None
+
+    def _read(self):
+        for line in self.proc.stdout:
+            self.lines.append(line.strip())
+
+    def stop(self) -> dict:
+        if self.proc is None:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["nvidia-smi unavailable"], "samples": 0}
+        self.proc.terminate()
+        try:
+            self.proc.wait(timeout=5)
+        except subprocess.TimeoutExpired:
+            self.proc.kill()
+        self.thread.join(timeout=2)
+        sm, smax, reasons = [], [], set()
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        for ln in self.lines:
+            parts = [x.strip() for x in ln.split(",")]
+            if len(parts) < 7:
+                continue
+            try:
+                sm.append(float(parts[0]))
+                smax.append(float(parts[1]))
+            except ValueError:
+                continue
+            for n, v in zip(names, parts[3:7]):
+                if v.lower() == "active":
+                    reasons.add(n)
+        return {"sm_mhz": statistics.median(sm) if sm else None, "sm_max_mhz": max(smax) if smax else None,
+                "reasons": sorted(reasons), "samples": len(sm)}
+
+
+def peaks() -> dict:
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(path):
+        with open(path) as f:
+            pk = json.load(f)
+        return {"hbm_gbs": float(pk["hbm_gbs"]), "source": "measured"}
+    return {"hbm_gbs": 6650.0, "source": "fallback"}
+
+
+# ---------------------------------------------------------------------------
+# CPU oracle (baseline leg and reference arm)
+# ---------------------------------------------------------------------------
+
+def oracle_units(w, n_heads: int, layer: int = 0):
+    """Oracle-built caches of the first n_heads KV heads of one layer (sequence 0)."""
+    import numpy as np
+    import torch
+    from hash_sparse_attention_b200.synth import make_layer
+    from oracle import hhr_oracle as O
+    li = make_layer(w, layer=layer, device="cuda" if torch.cuda.is_available() else "cpu")
+    L = int(li.seq_lens[0])
+    G, P = w.group, w.page_size
+    R32 = li.R.double().cpu().numpy()
+    Wn = li.W.double().cpu().numpy()
+    units = []
+    for h in range(n_heads):
+        K = (li.K_logical if w.paged else li.K)[0, h, :L].double().cpu().numpy()
+        V = (li.V_logical if w.paged else li.V)[0, h, :L].double().cpu().numpy()
+        Q = li.q[0, h * G:(h + 1) * G].double().cpu().numpy()
+        Kp, mn, mx, codes = O.build_head(K, R32[h], Wn[h], L, P)
+        units.append(dict(Q=Q, R=R32[h], W=Wn[h], Kp=Kp, V=V, mn=mn, mx=mx, codes=codes, L=L, P=P,
+                          N=int(li.n_keep[0]), k=int(li.top_k[0])))
+    del li
+    return units
+
+
+def oracle_decode_unit(u):
+    from oracle import hhr_oracle as O
+    return O.decode_head(u["Q"], u["R"], u["W"], u["Kp"], u["V"], u["mn"], u["mx"], u["codes"], u["L"], u["P"],
+                         u["N"], u["k"])
+
+
+def cpu_baseline(w, seconds: float) -> dict:
+    """Times the fp64 oracle's decode on whole (layer, KV head) units, one thread."""
+    from threadpoolctl import threadpool_limits
+    units = oracle_units(w, min(2, w.num_kv_heads))
+    heads_per_token = w.layers * w.num_kv_heads * w.batch
+    done = 0
+    with threadpool_limits(1):
+        t0 = time.perf_counter()
+        while True:
+            oracle_decode_unit(units[done % len(units)])
+            done += 1
+            el = time.perf_counter() - t0
+            if el >= seconds:
+                break
+    tok_s = (done / heads_per_token) / el
+    return {"value": tok_s, "unit": "tokens/s", "cores": 1, "kind": "oracle",
+            "sample": f"{done} (layer 0, KV head) decode units of {heads_per_token} per token, "
+                      f"{el:.1f} s of fp64 CPU work, one thread; cache build untimed"}
+
+
+# ---------------------------------------------------------------------------
+# the HHR arm
+# ---------------------------------------------------------------------------
+
+def run_hhr(args, rank, world):
+    import torch
+    from hash_sparse_attention_b200 import hhr
+    from hash_sparse_attention_b200.synth import WORKLOADS, make_layer, scaled
+
+    _, local_rank, _ = dist_env()
+    dev = torch.device("cuda", local_rank)
+    torch.cuda.set_device(dev)
+    w = WORKLOADS[args.workload]
+    if args.layers is not None:
+        w = scaled(w, layers=args.layers)
+    B, Hq, Hkv, d, P = w.batch, w.num_q_heads, w.num_kv_heads, w.head_dim, w.page_size
+
+    # ---- setup: every layer's cache built in place by the library ----
+    layers = []
+    q_all = None
+    for l in range(w.layers):
+        li = make_layer(w, layer=l, device=dev)
+        if w.paged:
+            cfg = hhr.make_config(B, Hq, Hkv, P, w.hash_bits, w.context, paged=True, num_blocks=li.K.shape[0],
+                                  max_blocks_per_seq=li.block_table.shape[1])
+        else:
+            cfg = hhr.make_config(B, Hq, Hkv, P, w.hash_bits, w.context)
+        cache = hhr.alloc_cache(cfg, dev, Krot=li.K, V=li.V)
+        hhr.build_cache(cfg, li.K, li.V, li.R, li.W, li.seq_lens, li.block_table, cache)
+        if q_all is None:
+            q_all = torch.empty(w.layers, B, Hq, d, dtype=torch.bfloat16, device=dev)
+            out_all = torch.empty(w.layers, B, Hq, d, dtype=torch.float32, device=dev)
+            dense_all = torch.empty(w.layers, B, Hq, d, dtype=torch.float32, device=dev)
+        q_all[l].copy_(li.q)
+        layers.append(dict(cfg=cfg, cache=cache, R=li.R, W=li.W, seq=li.seq_lens, table=li.block_table,
+                           n_keep=li.n_keep, top_k=li.top_k, lens=[int(x) for x in li.seq_lens.cpu()],
+                           nk=[int(x) for x in li.n_keep.cpu()], tk=[int(x) for x in li.top_k.cpu()]))
+        li.K_logical = li.V_logical = None
+        del li
+    torch.cuda.synchronize()
+    cfg0 = layers[0]["cfg"]
+    Nmax = max(max(L["nk"]) for L in layers)
+    Kmax = max(max(L["tk"]) for L in layers)
+    ws = hhr.decode_workspace(cfg0, Nmax, Kmax, dev)
+    dws = hhr.dense_workspace(cfg0, dev)
+    status = torch.zeros(1, dtype=torch.int32, device=dev)
+
+    def step():
+        for l, L in enumerate(layers):
+            hhr.decode_step(L["cfg"], q_all[l], L["R"], L["W"], L["cache"], L["seq"], L["table"], L["n_keep"],
+                            L["top_k"], Nmax, Kmax, out_all[l], ws, status=status)
+
+    def dense_step():
+        for l, L in enumerate(layers):
+            hhr.dense_decode(L["cfg"], q_all[l], L["R"], L["cache"], L["seq"], L["table"], dense_all[l], dws,
+                             status=status)
+
+    # eager once (and check status), then capture
+    step()
+    torch.cuda.synchronize()
+    assert int(status.item()) == 0, f"device status {int(status.item())}"
+    s = torch.cuda.Stream(device=dev)
+    s.wait_stream(torch.cuda.current_stream())
+    with torch.cuda.stream(s):
+        for _ in range(2):
+            step()
+    torch.cuda.current_stream().wait_stream(s)
+    graph = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(graph):
+        step()
+    dgraph = None
+    if not args.no_dense:
+        dense_step()
+        dgraph = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(dgraph):
+            dense_step()
+    torch.cuda.synchronize()
+
+    props = torch.cuda.get_device_properties(dev)
+    sampler = ClockSampler(str(getattr(props, "uuid", local_rank)) if getattr(props, "uuid", None) else str(local_rank))
+    if getattr(props, "uuid", None) is not None:
+        u = str(props.uuid)
+        sampler.gpu_id = u if u.startswith("GPU-") else f"GPU-{u}"
+    sampler.start()
+    st = torch.cuda.current_stream()
+
+    def timed(g, steps):
+        barrier(world, dev)
+        torch.cuda.synchronize()
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record(st)
+        for _ in range(steps):
+            g.replay()
+        e1.record(st)
+        e1.synchronize()
+        torch.cuda.synchronize()
+        barrier(world, dev)
+        return e0.elapsed_time(e1) / 1e3
+
+    # warm-up, plus a short soak so that clocks settle under load
+    for _ in range(max(3, args.warmup)):
+        graph.replay()
+    t_end = time.time() + args.soak_seconds
+    while time.time() < t_end:
+        graph.replay()
+        torch.cuda.synchronize()
+    secs = timed(graph, args.steps)
+    clocks = sampler.stop()
+    secs_max = max_over_ranks(secs, world, dev)
+
+    # dense comparison (same context, same library)
+    dense = None
+    if dgraph is not None:
+        for _ in range(3):
+            dgraph.replay()
+        dsecs = max_over_ranks(timed(dgraph, max(3, args.steps // 8)), world, dev)
+        dsteps = max(3, args.steps // 8)
+        dbytes = sum(dense_bytes_per_head(Lb, w.group) for L in layers for Lb in L["lens"] for _ in range(Hkv))
+        dense = {"value": whole_job_throughput(B * dsteps, world, dsecs), "unit": "tokens/s",
+                 "ms_per_step": dsecs / dsteps * 1e3,
+                 "achieved_gbs": dbytes / (dsecs / dsteps) / 1e9}
+
+    # e2e: q from pinned host memory, out back to pinned host memory, every step
+    q_host = q_all.cpu().pin_memory()
+    out_host = torch.empty(out_all.shape, dtype=out_all.dtype).pin_memory()
+    for _ in range(3):
+        q_all.copy_(q_host, non_blocking=True)
+        graph.replay()
+        out_host.copy_(out_all, non_blocking=True)
+    barrier(world, dev)
+    torch.cuda.synchronize()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record(st)
+    for _ in range(args.steps):
+        q_all.copy_(q_host, non_blocking=True)
+        graph.replay()
+        out_host.copy_(out_all, non_blocking=True)
+    e1.record(st)
+    e1.synchronize()
+    e2e_secs = max_over_ranks(e0.elapsed_time(e1) / 1e3, world, dev)
+    assert int(status.item()) == 0, f"device status {int(status.item())}"
+
+    # ---- algorithmic bytes ----
+    per_layer_bytes = []
+    for L in layers:
+        tot = 0
+        for b, Lb in enumerate(L["lens"]):
+            hb = hhr_bytes_per_head(Lb, P, min(L["nk"][b], Nmax), min(L["tk"][b], Kmax), w.group, w.hash_bits)
+            tot += Hkv * (hb["meta"] + hb["codes"] + hb["gather"] + hb["qo"])
+        tot += Hkv * (d * d * 4 + w.hash_bits * d * 2)
+        per_layer_bytes.append(tot)
+    step_bytes = sum(per_layer_bytes)
+    t_step = secs_max / args.steps
+    pk = peaks()
+    # the timed graph holds only the per-layer decode launches, back to back:
+    # the average duration of one layer's launch is the timed region / layers
+    mean_layer_s = t_step / len(layers)
+    achieved = statistics.mean(per_layer_bytes) / mean_layer_s / 1e9
+    roofline = {"bound": "hbm", "achieved": achieved, "peak": pk["hbm_gbs"], "unit": "GB/s",
+                "frac": achieved / pk["hbm_gbs"], "traffic": None,
+                "kernel": "hhr_decode_step (one layer: prep_query, gkr_scan_select, lhp_score_select, attn_split)",
+                "peak_source": pk["source"],
+                "step_gbs": step_bytes / t_step / 1e9, "step_frac": step_bytes / t_step / 1e9 / pk["hbm_gbs"]}
+    launches_per_step = 4 * len(layers)
+    result = {
+        "metric": METRIC,
+        "value": whole_job_throughput(B * args.steps, world, secs_max),
+        "unit": "tokens/s",
+        "n_gpus": world,
+        "steps": args.steps,
+        "warmup": args.warmup,
+        "ms_per_step": t_step * 1e3,
+        "higher_is_better": True,
+        "scaling": "weak",
+        "vs_baseline": None,
+        "dtype": "f32",
+        "data": "synthetic",
+        "config": {"workload": w.name, "batch": B, "q_heads": Hq, "kv_heads": Hkv, "head_dim": d,
+                   "context": w.context, "layers": len(layers), "page_size": P, "hash_bits": w.hash_bits,
+                   "keep_pages": Nmax, "top_k": Kmax, "kv_dtype": "bf16",
+                   "parallelism": f"replicas x{world}" if world > 1 else "single",
+                   "l2": "not flushed: the KV cache (all layers) is far larger than L2 and each layer's bytes "
+                         "are evicted by the other layers before reuse",
+                   "bytes_per_step": step_bytes},
+        "e2e": {"value": whole_job_throughput(B * args.steps, world, e2e_secs), "unit": "tokens/s",
+                "h2d_bytes_per_step": q_host.numel() * q_host.element_size(),
+                "d2h_bytes_per_step": out_host.numel() * out_host.element_size()},
+        "gpu_launches": launches_per_step * args.steps,
+        "roofline": roofline,
+        "clocks": clocks,
+        "dense": dense,
+        "achieved_gbs": step_bytes / t_step / 1e9,
+    }
+    return result, w
+
+
+def run_reference(args, rank, world):
+    """fp64 CPU oracle, rank 0 only: each step decodes one (layer 0, KV head) unit."""
+    from threadpoolctl import threadpool_limits
+    from hash_sparse_attention_b200.synth import WORKLOADS
+    w = WORKLOADS[args.workload]
+    units = oracle_units(w, min(2, w.num_kv_heads))
+    heads_per_token = w.layers * w.num_kv_heads * w.batch
+    with threadpool_limits(1):
+        for i in range(max(3, args.warmup)):
+            oracle_decode_unit(units[i % len(units)])
+        t0 = time.perf_counter()
+        for i in range(args.steps):
+            oracle_decode_unit(units[i % len(units)])
+        el = time.perf_counter() - t0
+    value = (args.steps / heads_per_token) / el
+    return {
+        "metric": METRIC, "value": value, "unit": "tokens/s", "n_gpus": world, "steps": args.steps,
+        "warmup": args.warmup, "ms_per_step": el / args.steps * 1e3, "higher_is_better": True, "scaling": "weak",
+        "vs_baseline": None, "dtype": "f64", "data": "synthetic", "impl": "reference",
+        "config": {"workload": w.name, "batch": w.batch, "context": w.context, "layers": w.layers,
+                   "note": "each step is one (layer, KV head) unit of the oracle; value scales by the "
+                           f"{heads_per_token} units of one token"},
+        "cpu_baseline": {"value": value, "unit": "tokens/s", "cores": 1, "kind": "oracle",
+                         "sample": f"{args.steps} timed (layer 0, KV head) decode units, one thread"},
+        "e2e": {"value": value, "unit": "tokens/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+    }
+
+
+def main(argv=None):
+    args = parse_args(argv)
+    rank, local_rank, world = dist_env()
+    if args.impl == "reference":
+        if rank != 0:
+            return 0
+        print(json.dumps(run_reference(args, rank, 1)))
+        return 0
+    import torch
+    rank, world = dist_init("nccl" if torch.cuda.is_available() else "gloo")
+    result, w = run_hhr(args, rank, world)
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        result["cpu_baseline"] = cpu_baseline(w, args.cpu_seconds)
+    if rank == 0:
+        print(json.dumps(result))
+    if world > 1:
+        import torch.distributed as dist
+        dist.destroy_process_group()
+    return 0
+
+
+if __name__ == "__main__":
+    sys.exit(main())

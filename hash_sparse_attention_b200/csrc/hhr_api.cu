@@ -1,0 +1,292 @@
+// C ABI of libhhr.so: argument validation, workspace carve-out and launches.
+// The kernels live in hhr_build.cuh and hhr_decode.cuh.
+#include <algorithm>
+#include <cstdarg>
+#include <cstdio>
+#include <cstring>
+
+#include "hhr_launch.h"
+
+using namespace hhr;
+
+namespace {
+
+thread_local char g_err[512] = {0};
+
+hhr_status fail(hhr_status s, const char* fmt, ...) {
+  va_list ap;
+  va_start(ap, fmt);
+  vsnprintf(g_err, sizeof(g_err), fmt, ap);
+  va_end(ap);
+  return s;
+}
+
+hhr_status ok() {
+  g_err[0] = 0;
+  return HHR_OK;
+}
+
+bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+hhr_status check_cuda(const char* what) {
+  const cudaError_t e = cudaGetLastError();
+  if (e != cudaSuccess) return fail(HHR_ERR_CUDA, "%s: %s", what, cudaGetErrorString(e));
+  return HHR_OK;
+}
+
+// Validates the configuration and fills the kernel-side dimensions.
+hhr_status make_dims(const hhr_config* cfg, Dims* dm) {
+  if (!cfg) return fail(HHR_ERR_INVALID_ARG, "cfg is NULL");
+  if (cfg->head_dim != D) return fail(HHR_ERR_UNSUPPORTED, "head_dim %d (only 128)", cfg->head_dim);
+  if (cfg->batch < 1 || cfg->num_kv_heads < 1 || cfg->num_q_heads < 1 || cfg->max_seq_len < 1)
+    return fail(HHR_ERR_INVALID_ARG, "batch, heads and max_seq_len must be >= 1");
+  if (cfg->num_q_heads % cfg->num_kv_heads != 0)
+    return fail(HHR_ERR_INVALID_ARG, "num_q_heads %d not a multiple of num_kv_heads %d", cfg->num_q_heads,
+                cfg->num_kv_heads);
+  const int G = cfg->num_q_heads / cfg->num_kv_heads;
+  if (G > 8) return fail(HHR_ERR_UNSUPPORTED, "group size %d (1..8)", G);
+  if (cfg->page_size != 16 && cfg->page_size != 32)
+    return fail(HHR_ERR_UNSUPPORTED, "page_size %d (16 or 32)", cfg->page_size);
+  if (cfg->hash_bits != 64 && cfg->hash_bits != 128 && cfg->hash_bits != 256)
+    return fail(HHR_ERR_UNSUPPORTED, "hash_bits %d (64, 128 or 256)", cfg->hash_bits);
+  const long long np_max = ((long long)cfg->max_seq_len + cfg->page_size - 1) / cfg->page_size;
+  if (np_max > MAX_SELECT_PAGES)
+    return fail(HHR_ERR_UNSUPPORTED, "%lld pages per sequence (at most %d)", np_max, MAX_SELECT_PAGES);
+  if (cfg->paged) {
+    if (cfg->num_blocks < 1) return fail(HHR_ERR_INVALID_ARG, "paged: num_blocks must be >= 1");
+    if (cfg->max_blocks_per_seq < np_max)
+      return fail(HHR_ERR_INVALID_ARG, "paged: max_blocks_per_seq %d < ceil(max_seq_len / page_size) %lld",
+                  cfg->max_blocks_per_seq, np_max);
+  }
+  dm->B = cfg->batch;
+  dm->Hq = cfg->num_q_heads;
+  dm->Hkv = cfg->num_kv_heads;
+  dm->G = G;
+  dm->P = cfg->page_size;
+  dm->nb = cfg->hash_bits;
+  dm->words = cfg->hash_bits / 64;
+  dm->T = cfg->max_seq_len;
+  dm->np_max = (int)np_max;
+  dm->paged = cfg->paged ? 1 : 0;
+  dm->num_blocks = cfg->paged ? cfg->num_blocks : 0;
+  dm->max_blocks = cfg->paged ? cfg->max_blocks_per_seq : 0;
+  return HHR_OK;
+}
+
+size_t align256(size_t x) { return (x + 255) & ~size_t(255); }
+
+// Carves the workspace; with base == nullptr only the size is computed.
+size_t carve(const Dims& dm, int Nmax, int Kmax, int keys_per_split, int nsplit, char* base, Work* wk) {
+  const size_t BH = (size_t)dm.B * dm.Hkv;
+  const int hist_stride = (int)((dm.G * dm.nb + 1 + 63) / 64 * 64);
+  size_t off = 0;
+  auto take = [&](size_t bytes) {
+    char* p = base ? base + off : nullptr;
+    off += align256(bytes);
+    return p;
+  };
+  Work w{};
+  w.qrot = reinterpret_cast<float*>(take(sizeof(float) * dm.B * dm.Hq * D));
+  w.qcodes = reinterpret_cast<uint64_t*>(take(sizeof(uint64_t) * dm.B * dm.Hq * dm.words));
+  w.U = reinterpret_cast<float*>(take(sizeof(float) * BH * dm.np_max));
+  w.sel_pages = reinterpret_cast<int*>(take(sizeof(int) * BH * Nmax));
+  w.n_sel = reinterpret_cast<int*>(take(sizeof(int) * BH));
+  w.scores = reinterpret_cast<int*>(take(sizeof(int) * BH * Nmax * dm.P));
+  w.hist = reinterpret_cast<int*>(take(sizeof(int) * BH * hist_stride));
+  w.sel_keys = reinterpret_cast<int*>(take(sizeof(int) * BH * Kmax));
+  w.n_keys = reinterpret_cast<int*>(take(sizeof(int) * BH));
+  w.part = reinterpret_cast<float*>(take(sizeof(float) * BH * nsplit * dm.G * (D + 2)));
+  w.tickets = reinterpret_cast<unsigned*>(take(sizeof(unsigned) * BH * 4));
+  w.Nmax = Nmax;
+  w.Kmax = Kmax;
+  w.hist_stride = hist_stride;
+  w.nsplit = nsplit;
+  w.keys_per_split = keys_per_split;
+  if (wk) *wk = w;
+  return off;
+}
+
+int sparse_nsplit(const Dims& dm, int Nmax, int Kmax) {
+  const long long kcap = std::min<long long>(Kmax, (long long)Nmax * dm.P);
+  return (int)std::max<long long>(1, (kcap + ATT_SPLIT - 1) / ATT_SPLIT);
+}
+
+int dense_nsplit(const Dims& dm) { return (dm.T + DENSE_SPLIT - 1) / DENSE_SPLIT; }
+
+// ---- group-size dispatch -------------------------------------------------
+#define HHR_DISPATCH_G(G_, ...)                          \
+  switch (G_) {                                          \
+    case 1: { constexpr int GG = 1; __VA_ARGS__; } break; \
+    case 2: { constexpr int GG = 2; __VA_ARGS__; } break; \
+    case 3: { constexpr int GG = 3; __VA_ARGS__; } break; \
+    case 4: { constexpr int GG = 4; __VA_ARGS__; } break; \
+    case 5: { constexpr int GG = 5; __VA_ARGS__; } break; \
+    case 6: { constexpr int GG = 6; __VA_ARGS__; } break; \
+    case 7: { constexpr int GG = 7; __VA_ARGS__; } break; \
+    case 8: { constexpr int GG = 8; __VA_ARGS__; } break; \
+    default: break;                                      \
+  }
+
+}  // namespace
+
+extern "C" {
+
+const char* hhr_status_string(hhr_status s) {
+  switch (s) {
+    case HHR_OK: return "HHR_OK";
+    case HHR_ERR_INVALID_ARG: return "HHR_ERR_INVALID_ARG";
+    case HHR_ERR_UNSUPPORTED: return "HHR_ERR_UNSUPPORTED";
+    case HHR_ERR_WORKSPACE: return "HHR_ERR_WORKSPACE";
+    case HHR_ERR_CUDA: return "HHR_ERR_CUDA";
+    case HHR_ERR_TIMEOUT: return "HHR_ERR_TIMEOUT";
+    case HHR_ERR_BAD_BLOCK: return "HHR_ERR_BAD_BLOCK";
+  }
+  return "HHR_ERR_UNKNOWN";
+}
+
+const char* hhr_last_error(void) { return g_err; }
+
+hhr_status hhr_build_cache(const hhr_config* cfg, const void* K, const void* V, const float* R, const void* W,
+                           const int32_t* seq_lens, const int32_t* block_table, void* Krot, void* Vcache,
+                           void* page_min, void* page_max, uint64_t* codes, hhr_stream_t stream) {
+  Dims dm;
+  hhr_status s = make_dims(cfg, &dm);
+  if (s != HHR_OK) return s;
+  if (!K || !V || !R || !W || !seq_lens || !Krot || !Vcache || !page_min || !page_max || !codes)
+    return fail(HHR_ERR_INVALID_ARG, "hhr_build_cache: NULL tensor pointer");
+  if (dm.paged && !block_table) return fail(HHR_ERR_INVALID_ARG, "hhr_build_cache: paged needs block_table");
+  const void* al[] = {K, V, R, W, Krot, Vcache, page_min, page_max, codes};
+  for (const void* p : al)
+    if (!aligned16(p)) return fail(HHR_ERR_INVALID_ARG, "hhr_build_cache: tensor not 16-byte aligned");
+  cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+  if (V != Vcache) {
+    const size_t bytes = dm.paged ? (size_t)dm.num_blocks * dm.Hkv * dm.P * D * 2
+                                  : (size_t)dm.B * dm.Hkv * dm.T * D * 2;
+    if (cudaMemcpyAsync(Vcache, V, bytes, cudaMemcpyDeviceToDevice, st) != cudaSuccess)
+      return check_cuda("hhr_build_cache: V copy");
+  }
+  const cudaError_t e = launch_build(dm, static_cast<const __nv_bfloat16*>(K), R, static_cast<const __nv_bfloat16*>(W),
+                                     seq_lens, block_table, static_cast<__nv_bfloat16*>(Krot),
+                                     static_cast<__nv_bfloat16*>(page_min), static_cast<__nv_bfloat16*>(page_max), codes,
+                                     nullptr, st);
+  if (e != cudaSuccess) return fail(HHR_ERR_CUDA, "hhr_build_cache: %s", cudaGetErrorString(e));
+  return ok();
+}
+
+size_t hhr_decode_workspace_size(const hhr_config* cfg, int32_t max_keep_pages, int32_t max_top_k) {
+  Dims dm;
+  if (make_dims(cfg, &dm) != HHR_OK || max_keep_pages < 1 || max_top_k < 1) return 0;
+  const int Nmax = std::min(max_keep_pages, dm.np_max);
+  return carve(dm, Nmax, max_top_k, ATT_SPLIT, sparse_nsplit(dm, Nmax, max_top_k), nullptr, nullptr);
+}
+
+hhr_status hhr_workspace_init(void* workspace, size_t workspace_bytes, hhr_stream_t stream) {
+  if (!workspace) return fail(HHR_ERR_INVALID_ARG, "hhr_workspace_init: NULL workspace");
+  if (cudaMemsetAsync(workspace, 0, workspace_bytes, reinterpret_cast<cudaStream_t>(stream)) != cudaSuccess)
+    return check_cuda("hhr_workspace_init");
+  return ok();
+}
+
+hhr_status hhr_decode_step(const hhr_config* cfg, const void* q, const float* R, const void* W, const void* Krot,
+                           const void* Vcache, const void* page_min, const void* page_max, const uint64_t* codes,
+                           const int32_t* seq_lens, const int32_t* block_table, const int32_t* n_keep_pages,
+                           const int32_t* top_k, int32_t max_keep_pages, int32_t max_top_k, float sm_scale,
+                           float* out, const hhr_debug* dbg, void* workspace, size_t workspace_bytes,
+                           int32_t* device_status, hhr_stream_t stream) {
+  Dims dm;
+  hhr_status s = make_dims(cfg, &dm);
+  if (s != HHR_OK) return s;
+  if (!q || !R || !W || !Krot || !Vcache || !page_min || !page_max || !codes || !seq_lens || !n_keep_pages ||
+      !top_k || !out || !workspace)
+    return fail(HHR_ERR_INVALID_ARG, "hhr_decode_step: NULL pointer");
+  if (dm.paged && !block_table) return fail(HHR_ERR_INVALID_ARG, "hhr_decode_step: paged needs block_table");
+  const void* al[] = {R, W, Krot, Vcache, page_min, page_max, codes};
+  for (const void* p : al)
+    if (!aligned16(p)) return fail(HHR_ERR_INVALID_ARG, "hhr_decode_step: tensor not 16-byte aligned");
+  if ((reinterpret_cast<uintptr_t>(workspace) & 255u) != 0)
+    return fail(HHR_ERR_INVALID_ARG, "hhr_decode_step: workspace not 256-byte aligned");
+  if (max_keep_pages < 1 || max_top_k < 1)
+    return fail(HHR_ERR_INVALID_ARG, "hhr_decode_step: max_keep_pages and max_top_k must be >= 1");
+  if (!(sm_scale > 0.f)) return fail(HHR_ERR_INVALID_ARG, "hhr_decode_step: sm_scale must be > 0");
+  const int Nmax = std::min(max_keep_pages, dm.np_max);
+  const int nsplit = sparse_nsplit(dm, Nmax, max_top_k);
+  const size_t need = carve(dm, Nmax, max_top_k, ATT_SPLIT, nsplit, nullptr, nullptr);
+  if (workspace_bytes < need)
+    return fail(HHR_ERR_WORKSPACE, "hhr_decode_step: workspace %zu bytes < %zu", workspace_bytes, need);
+  Work wk;
+  carve(dm, Nmax, max_top_k, ATT_SPLIT, nsplit, static_cast<char*>(workspace), &wk);
+
+  DecodeArgs a = {};
+  a.dm = dm;
+  a.wk = wk;
+  a.q = static_cast<const __nv_bfloat16*>(q);
+  a.R = R;
+  a.W = static_cast<const __nv_bfloat16*>(W);
+  a.Kr = static_cast<const __nv_bfloat16*>(Krot);
+  a.Vc = static_cast<const __nv_bfloat16*>(Vcache);
+  a.pmin = static_cast<const __nv_bfloat16*>(page_min);
+  a.pmax = static_cast<const __nv_bfloat16*>(page_max);
+  a.codes = codes;
+  a.seq_lens = seq_lens;
+  a.table = block_table;
+  a.n_keep = n_keep_pages;
+  a.top_k = top_k;
+  a.sm_scale = sm_scale;
+  a.out = out;
+  if (dbg) a.dbg = *dbg;
+  a.status = device_status;
+  a.stream = reinterpret_cast<cudaStream_t>(stream);
+  cudaError_t e = cudaErrorInvalidValue;
+  HHR_DISPATCH_G(dm.G, e = launch_decode<GG>(a));
+  if (e != cudaSuccess) return fail(HHR_ERR_CUDA, "hhr_decode_step: launch failed: %s", cudaGetErrorString(e));
+  return ok();
+}
+
+size_t hhr_dense_workspace_size(const hhr_config* cfg) {
+  Dims dm;
+  if (make_dims(cfg, &dm) != HHR_OK) return 0;
+  return carve(dm, 1, 1, DENSE_SPLIT, dense_nsplit(dm), nullptr, nullptr);
+}
+
+hhr_status hhr_dense_decode(const hhr_config* cfg, const void* q, const float* R, const void* Krot,
+                            const void* Vcache, const int32_t* seq_lens, const int32_t* block_table, float sm_scale,
+                            float* out, void* workspace, size_t workspace_bytes, int32_t* device_status,
+                            hhr_stream_t stream) {
+  Dims dm;
+  hhr_status s = make_dims(cfg, &dm);
+  if (s != HHR_OK) return s;
+  if (!q || !R || !Krot || !Vcache || !seq_lens || !out || !workspace)
+    return fail(HHR_ERR_INVALID_ARG, "hhr_dense_decode: NULL pointer");
+  if (dm.paged && !block_table) return fail(HHR_ERR_INVALID_ARG, "hhr_dense_decode: paged needs block_table");
+  const void* al[] = {R, Krot, Vcache};
+  for (const void* p : al)
+    if (!aligned16(p)) return fail(HHR_ERR_INVALID_ARG, "hhr_dense_decode: tensor not 16-byte aligned");
+  if ((reinterpret_cast<uintptr_t>(workspace) & 255u) != 0)
+    return fail(HHR_ERR_INVALID_ARG, "hhr_dense_decode: workspace not 256-byte aligned");
+  if (!(sm_scale > 0.f)) return fail(HHR_ERR_INVALID_ARG, "hhr_dense_decode: sm_scale must be > 0");
+  const int nsplit = dense_nsplit(dm);
+  const size_t need = carve(dm, 1, 1, DENSE_SPLIT, nsplit, nullptr, nullptr);
+  if (workspace_bytes < need)
+    return fail(HHR_ERR_WORKSPACE, "hhr_dense_decode: workspace %zu bytes < %zu", workspace_bytes, need);
+  Work wk;
+  carve(dm, 1, 1, DENSE_SPLIT, nsplit, static_cast<char*>(workspace), &wk);
+  DecodeArgs a = {};
+  a.dm = dm;
+  a.wk = wk;
+  a.q = static_cast<const __nv_bfloat16*>(q);
+  a.R = R;
+  a.Kr = static_cast<const __nv_bfloat16*>(Krot);
+  a.Vc = static_cast<const __nv_bfloat16*>(Vcache);
+  a.seq_lens = seq_lens;
+  a.table = block_table;
+  a.sm_scale = sm_scale;
+  a.out = out;
+  a.status = device_status;
+  a.stream = reinterpret_cast<cudaStream_t>(stream);
+  cudaError_t e = cudaErrorInvalidValue;
+  HHR_DISPATCH_G(dm.G, e = launch_dense<GG>(a));
+  if (e != cudaSuccess) return fail(HHR_ERR_CUDA, "hhr_dense_decode: launch failed: %s", cudaGetErrorString(e));
+  return ok();
+}
+
+}  // extern "C"

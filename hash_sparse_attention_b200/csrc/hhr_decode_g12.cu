@@ -1,0 +1,7 @@
+// Decode kernels instantiated for group sizes 1 and 2.
+#include "hhr_decode.cuh"
+
+namespace hhr {
+HHR_INSTANTIATE_DECODE(1)
+HHR_INSTANTIATE_DECODE(2)
+}  // namespace hhr

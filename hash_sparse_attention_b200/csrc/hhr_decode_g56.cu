@@ -1,0 +1,7 @@
+// Decode kernels instantiated for group sizes 5 and 6.
+#include "hhr_decode.cuh"
+
+namespace hhr {
+HHR_INSTANTIATE_DECODE(5)
+HHR_INSTANTIATE_DECODE(6)
+}  // namespace hhr

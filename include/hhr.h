@@ -1,0 +1,196 @@
+/*
+ * hhr.h -- C ABI of the HHR decode-path library (libhhr.so), sm_100a.
+ *
+ * HHR ("HHR: Hierarchical Hash Retrieval for Efficient LLM Generation",
+ * paper card, Abstract) retrieves keys for one decode step in two stages
+ * before attention (rit.work explainer, section "Два уровня маршрутизации
+ * решают разные ошибки"):
+ *   GKR  keys are stored rotated by a per-KV-head orthogonal R_h (q.k is
+ *        unchanged); pages of P neighbouring keys keep channel min/max; each
+ *        page gets a logit upper bound and only the top-N pages survive.
+ *   LHP  keys of surviving pages are ranked by the Hamming distance between
+ *        sign codes of W_h k and W_h q; the top-k keys are kept.
+ *   Then exact softmax attention runs over the kept keys only.
+ *
+ * Conventions shared by every entry point
+ *   - All tensor pointers are DEVICE pointers owned by the caller.  The
+ *     library never allocates or frees device memory and never synchronises;
+ *     every call is enqueued on `stream` and returns immediately.
+ *   - The return value reports host-side validation and launch errors only.
+ *     Device-side problems (a block-table entry outside the pool, a bounded
+ *     wait that ran out) are written to `device_status` (an int32 the caller
+ *     zeroes and reads after synchronising); kernels never trap.
+ *   - bf16 tensors and uint64 codes must be 16-byte aligned (vector loads).
+ *   - head_dim must be 128; num_q_heads must be a multiple of num_kv_heads
+ *     with a group size G = num_q_heads / num_kv_heads of 1..8; page_size 16
+ *     or 32; hash_bits 64, 128 or 256.
+ *   - No C++ exception crosses this boundary.
+ *
+ * Layouts (row-major, innermost last).  d = head_dim, T = max_seq_len,
+ * np = ceil(T / page_size), w = hash_bits / 64, Bk = num_blocks.
+ *   contiguous (paged == 0)        paged (paged == 1, block = one page)
+ *   K, Krot, V : [B, Hkv, T, d]    [Bk, Hkv, P, d]
+ *   page_min/max: [B, Hkv, np, d]  [Bk, Hkv, d]
+ *   codes       : [B, Hkv, T, w]   [Bk, Hkv, P, w]
+ *   block_table : unused (NULL)    int32 [B, max_blocks_per_seq]; logical
+ *                                  page p of sequence b lives in block
+ *                                  block_table[b * max_blocks_per_seq + p]
+ *   q : bf16 [B, Hq, d];  R : fp32 [Hkv, d, d] with k' = R_h k (row i of
+ *   R_h gives channel i);  W : bf16 [Hkv, hash_bits, d];  out : fp32 [B, Hq, d].
+ *   Query head hq belongs to KV head hq / G.
+ */
+#ifndef HHR_H_
+#define HHR_H_
+
+#include <stddef.h>
+#include <stdint.h>
+
+#if defined(__GNUC__)
+#define HHR_API __attribute__((visibility("default")))
+#else
+#define HHR_API
+#endif
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+/* Same type as cudaStream_t; NULL means the legacy default stream. */
+typedef struct CUstream_st* hhr_stream_t;
+
+typedef enum {
+  HHR_OK = 0,
+  HHR_ERR_INVALID_ARG = 1,  /* null / misaligned pointer, bad size or shape  */
+  HHR_ERR_UNSUPPORTED = 2,  /* head_dim, group size, bits or page size       */
+  HHR_ERR_WORKSPACE = 3,    /* workspace too small for the requested budgets */
+  HHR_ERR_CUDA = 4,         /* a CUDA launch or copy failed                  */
+  HHR_ERR_TIMEOUT = 5,      /* (device_status only) a bounded wait ran out   */
+  HHR_ERR_BAD_BLOCK = 6     /* (device_status only) block id outside the pool */
+} hhr_status;
+
+typedef struct {
+  int32_t batch;              /* B                                            */
+  int32_t num_q_heads;        /* Hq                                           */
+  int32_t num_kv_heads;       /* Hkv                                          */
+  int32_t head_dim;           /* d, must be 128                               */
+  int32_t page_size;          /* P: 16 or 32 (the block size when paged)      */
+  int32_t hash_bits;          /* 64, 128 or 256                               */
+  int32_t max_seq_len;        /* T: capacity of one sequence                  */
+  int32_t paged;              /* 0 contiguous, 1 block pool + block table     */
+  int32_t num_blocks;         /* Bk: blocks in the pool (paged only)          */
+  int32_t max_blocks_per_seq; /* row length of block_table (paged only)       */
+} hhr_config;
+
+/* Optional stage outputs of hhr_decode_step (any pointer may be NULL). They
+ * expose each stage's result so that it can be checked on its own.
+ * np_max = ceil(T / P), Nmax = max_keep_pages, Kmax = max_top_k.            */
+typedef struct {
+  float* q_rot;          /* [B, Hq, d]        q' = R_h q                        */
+  float* page_ub;        /* [B, Hq, np_max]   per query head page bound          */
+  float* page_U;         /* [B, Hkv, np_max]  max of page_ub over the group      */
+  int32_t* sel_pages;    /* [B, Hkv, Nmax]    kept pages, ascending              */
+  int32_t* n_sel_pages;  /* [B, Hkv]                                             */
+  uint64_t* q_codes;     /* [B, Hq, w]        query sign codes                   */
+  int32_t* key_scores;   /* [B, Hkv, Nmax*P]  group Hamming distance per candidate
+                                              (candidate order: kept pages
+                                              ascending, rows ascending; rows past
+                                              the sequence end hold INT32_MAX)   */
+  int32_t* n_cand;       /* [B, Hkv]          valid candidates                   */
+  int32_t* sel_keys;     /* [B, Hkv, Kmax]    kept token ids, ascending          */
+  int32_t* n_sel_keys;   /* [B, Hkv]                                             */
+} hhr_debug;
+
+/* Human-readable name of a status code (static storage). */
+HHR_API const char* hhr_status_string(hhr_status s);
+
+/* Message describing the last host-side validation failure on this thread
+ * (static thread-local storage; empty when the last call succeeded). */
+HHR_API const char* hhr_last_error(void);
+
+/*
+ * hhr_build_cache -- cache build for one layer (prefill side of HHR).
+ *
+ * GKR stores keys in the basis of the head-wise orthogonal transform, which
+ * leaves every query-key product unchanged (paper card, Abstract; rit.work,
+ * two-level routing section); pages keep what their bound needs; LHP keys
+ * get sign codes (paper page, Figure 2 caption: projection then sign).
+ * For every sequence b, KV head h and row t < seq_lens[b]:
+ *   Krot[t] = bf16_rne(R_h K[t])                 (fp32 accumulation)
+ *   codes[t] bit j = [ (W_h K[t])_j > 0 ]        (unrotated K; bit j in word
+ *                                                 j/64 at position j%64; the
+ *                                                 sign is exact: near-zero
+ *                                                 projections are recomputed
+ *                                                 in fp64)
+ *   page_min/max[p] = channel min/max of the stored Krot rows of page p that
+ *                     lie below seq_lens[b]
+ *   Vcache = V (copied unless Vcache == V).
+ * Rows at or past seq_lens[b] and pages past the last valid one are left
+ * untouched.  Krot may alias K (in place).  seq_lens is a device array [B].
+ */
+HHR_API hhr_status hhr_build_cache(const hhr_config* cfg, const void* K, const void* V,
+                           const float* R, const void* W, const int32_t* seq_lens,
+                           const int32_t* block_table, void* Krot, void* Vcache,
+                           void* page_min, void* page_max, uint64_t* codes,
+                           hhr_stream_t stream);
+
+/* Bytes of workspace hhr_decode_step needs for these budgets. */
+HHR_API size_t hhr_decode_workspace_size(const hhr_config* cfg, int32_t max_keep_pages,
+                                 int32_t max_top_k);
+
+/* Zero a workspace before its first use (the decode step keeps its arrival
+ * counters at zero between calls).  Enqueued on `stream`. */
+HHR_API hhr_status hhr_workspace_init(void* workspace, size_t workspace_bytes, hhr_stream_t stream);
+
+/*
+ * hhr_decode_step -- one HHR decode step of one layer for all sequences.
+ *
+ * For each sequence b with L = seq_lens[b], np = ceil(L / P), each KV head h
+ * and its query heads g (hq = h*G + g):
+ *  1. q'_g = R_h q_g (fp32).                      GKR rotation (Abstract)
+ *  2. ub[g,p] = sum_i max(q'_gi mn_pi, q'_gi mx_pi); U_p = max_g ub[g,p].
+ *                                                 page logit bound (Abstract)
+ *  3. keep N = min(clamp(n_keep_pages[b], 1, max_keep_pages), np) pages with
+ *     the largest U_p; equal bounds go to the lower page index.  Coarse
+ *     pruning of whole pages (rit.work, two-level routing section).
+ *  4. query codes: bit j = [ (W_h q_g)_j > 0 ] (exact sign, fp64 fallback).
+ *  5. for the valid rows of kept pages: S = sum_g popcount(code_g ^ code_row).
+ *  6. keep k = min(clamp(top_k[b], 1, max_top_k), #candidates) rows with the
+ *     smallest S; equal scores go to the lower token index.
+ *  7. out[b, hq] = sum_j softmax_j(sm_scale * q'_g . Krot_j) V_j over the kept
+ *     rows (fp32 accumulation, fp32 output).  L == 0 gives a zero output.
+ * n_keep_pages and top_k are device arrays [B]; max_keep_pages and max_top_k
+ * are their host-side upper bounds and size the workspace.  `dbg` may be
+ * NULL.  `workspace` must be at least hhr_decode_workspace_size() bytes,
+ * 256-byte aligned, zeroed once with hhr_workspace_init(), and not shared by
+ * calls that may run concurrently.  `device_status` may be NULL.
+ */
+HHR_API hhr_status hhr_decode_step(const hhr_config* cfg, const void* q, const float* R, const void* W,
+                           const void* Krot, const void* Vcache, const void* page_min,
+                           const void* page_max, const uint64_t* codes,
+                           const int32_t* seq_lens, const int32_t* block_table,
+                           const int32_t* n_keep_pages, const int32_t* top_k,
+                           int32_t max_keep_pages, int32_t max_top_k, float sm_scale,
+                           float* out, const hhr_debug* dbg, void* workspace,
+                           size_t workspace_bytes, int32_t* device_status,
+                           hhr_stream_t stream);
+
+/* Bytes of workspace hhr_dense_decode needs. */
+HHR_API size_t hhr_dense_workspace_size(const hhr_config* cfg);
+
+/*
+ * hhr_dense_decode -- full decode attention over all L = seq_lens[b] keys of
+ * the same cache (the "Full Attention" comparison row of the paper's tables):
+ *   out[b, hq] = sum_{t<L} softmax_t(sm_scale * (R_h q) . Krot_t) V_t
+ * Same layouts, workspace and status rules as hhr_decode_step.
+ */
+HHR_API hhr_status hhr_dense_decode(const hhr_config* cfg, const void* q, const float* R,
+                            const void* Krot, const void* Vcache, const int32_t* seq_lens,
+                            const int32_t* block_table, float sm_scale, float* out,
+                            void* workspace, size_t workspace_bytes, int32_t* device_status,
+                            hhr_stream_t stream);
+
+#ifdef __cplusplus
+}  /* extern "C" */
+#endif
+
+#endif  /* HHR_H_ */
