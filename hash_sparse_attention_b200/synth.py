@@ -262,15 +262,17 @@ def to_pool(X: torch.Tensor, table: torch.Tensor, lens: list[int], P: int, nbloc
 
 
 def from_pool(pool: torch.Tensor, table: torch.Tensor, lens: list[int], T: int) -> torch.Tensor:
-    """Gather a block pool back into per-sequence rows [B, H, T, d] (zeros past each length)."""
-    nblocks, H, P, d = pool.shape
+    """Gather a block pool [nblocks, H, P, ...] back into per-sequence rows [B, H, T, ...]
+    (zeros past each length)."""
+    nblocks, H, P = pool.shape[:3]
+    rest = tuple(pool.shape[3:])
     B = table.shape[0]
-    out = torch.zeros(B, H, T, d, dtype=pool.dtype, device=pool.device)
+    out = torch.zeros((B, H, T) + rest, dtype=pool.dtype, device=pool.device)
     for b, L in enumerate(lens):
         nb_ = -(-L // P)
         if nb_ == 0:
             continue
-        rows = pool[table[b, :nb_].long().to(pool.device)].permute(1, 0, 2, 3).reshape(H, nb_ * P, d)
+        rows = pool[table[b, :nb_].long().to(pool.device)].transpose(0, 1).reshape((H, nb_ * P) + rest)
         out[b, :, :L] = rows[:, :L]
     return out
 
@@ -286,4 +288,4 @@ def l2_flush_bytes() -> int:
 
 
 __all__ = ["Workload", "WORKLOADS", "LayerInputs", "make_layer", "scaled", "to_pool",
-           "from_pool", "num_pages", "orthogonal_from_gaussian", "l2_flush_bytes", "math"]
+           "from_pool", "num_pages", "orthogonal_from_gaussian", "l2_flush_bytes"]

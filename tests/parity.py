@@ -10,7 +10,8 @@ within tolerance where the selections agree.
 Tolerances and exemptions (readings of the pages):
   * attention output: per query head max|o - o^| / max|o^| <= 2e-3
   * page bounds: |ub - ub^| <= 2e-3 * sum_i |q'_i| max(|mn_i|, |mx_i|)
-  * K': within one bf16 ulp of the fp64-rounded value
+  * K': within one bf16 ulp of the fp64-rounded value plus the fp32
+    accumulation bound 2^-16 * sum_j |R_ij k_j|
   * a hash bit is exempt when |fp64 projection| < 1e-5 |x|; a page is exempt
     when |U_p - thr| <= 1e-4 |thr| (thr = the N-th largest fp64 bound)
 """
@@ -103,7 +104,7 @@ def run_gpu(w: Workload, li: LayerInputs, max_keep: int | None = None, max_topk:
     if w.paged:
         Kr = from_pool(cache.Krot, table, lens, w.context)
         Vl = from_pool(cache.V, table, lens, w.context)
-        cd = from_pool(cache.codes.view(*cache.codes.shape, 1), table, lens, w.context)[..., 0]
+        cd = from_pool(cache.codes, table, lens, w.context)
         pmn = _logical_meta(cache.page_min, table, lens, P, np_max)
         pmx = _logical_meta(cache.page_max, table, lens, P, np_max)
     else:
@@ -162,7 +163,11 @@ def check_build(w: Workload, li: LayerInputs, g: GpuRun, rep: Report, heads=None
             diff = Kp != Kp_ref
             rep.kprime_flips += int(diff.sum())
             rep.kprime_elems += diff.size
-            assert np.all(np.abs(Kp - Kp_ref) <= _bf16_ulp(Kp_ref) * 1.0000001), "K' off by more than one bf16 ulp"
+            # fp32 accumulation: the unrounded value may be off by gamma_128 * sum|R_ij k_j|
+            # (about 2^-17 of it), then rounding to bf16 adds at most one ulp
+            acc_err = 2.0 ** -16 * (np.abs(Kx) @ np.abs(R32[h]).T)
+            assert np.all(np.abs(Kp - Kp_ref) <= _bf16_ulp(Kp_ref) * 1.0000001 + acc_err), \
+                "K' off by more than one bf16 ulp plus the fp32 accumulation bound"
             # page metadata: stage-wise on the GPU's stored K'
             mn, mx = O.page_minmax(Kp, L, P)
             n = mn.shape[0]
