@@ -19,6 +19,7 @@ HHR_ERR_WORKSPACE = 3
 HHR_ERR_CUDA = 4
 HHR_ERR_TIMEOUT = 5
 HHR_ERR_BAD_BLOCK = 6
+NOALLOC_SCRATCH_BYTES = 16 << 20  # HHR_NOALLOC_SCRATCH_BYTES in include/hhr.h
 
 
 class HHRConfig(ctypes.Structure):
@@ -51,6 +52,8 @@ SIGNATURES = {
     "hhr_decode_step": (_i32, [_cfgp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp,
                                _i32, _i32, ctypes.c_float, _vp, ctypes.POINTER(HHRDebug), _vp, _sz,
                                _vp, _vp]),
+    "hhr_decode_step_noalloc": (_i32, [_cfgp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp,
+                                       _i32, _i32, ctypes.c_float, _vp, ctypes.POINTER(HHRDebug), _vp, _vp]),
     "hhr_dense_workspace_size": (_sz, [_cfgp]),
     "hhr_dense_decode": (_i32, [_cfgp, _vp, _vp, _vp, _vp, _vp, _vp, ctypes.c_float, _vp, _vp, _sz,
                                 _vp, _vp]),

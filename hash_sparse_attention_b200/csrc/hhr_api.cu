@@ -129,6 +129,12 @@ int dense_nsplit(const Dims& dm) { return (dm.T + DENSE_SPLIT - 1) / DENSE_SPLIT
 
 }  // namespace
 
+namespace hhr {
+// Records a host-side error message for hhr_last_error() (used by entry
+// points defined in other translation units).
+hhr_status record_error(hhr_status s, const char* msg) { return fail(s, "%s", msg); }
+}  // namespace hhr
+
 extern "C" {
 
 const char* hhr_status_string(hhr_status s) {

@@ -44,6 +44,8 @@ struct DecodeArgs {
   cudaStream_t stream;
 };
 
+hhr_status record_error(hhr_status s, const char* msg);
+
 template <int G> cudaError_t launch_decode(const DecodeArgs& a);
 template <int G> cudaError_t launch_dense(const DecodeArgs& a);
 

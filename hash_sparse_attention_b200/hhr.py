@@ -15,7 +15,7 @@ import torch
 from ._lib import HHRConfig, HHRDebug, check, lib
 
 __all__ = ["HHRConfig", "HHRDebug", "make_config", "Cache", "alloc_cache", "build_cache",
-           "decode_workspace", "dense_workspace", "decode_step", "dense_decode", "DebugOutputs",
+           "decode_workspace", "dense_workspace", "decode_step", "decode_step_noalloc", "dense_decode", "DebugOutputs",
            "alloc_debug"]
 
 
@@ -158,6 +158,28 @@ def decode_step(cfg: HHRConfig, q: torch.Tensor, R: torch.Tensor, W: torch.Tenso
         max_keep_pages, max_top_k, sm_scale, _ptr(out), ctypes.byref(d) if d is not None else None,
         _ptr(workspace), workspace.numel(), _ptr(status), _stream(stream))
     check(st, "hhr_decode_step")
+    return out
+
+
+def decode_step_noalloc(cfg: HHRConfig, q: torch.Tensor, R: torch.Tensor, W: torch.Tensor, cache: Cache,
+                        seq_lens: torch.Tensor, block_table: torch.Tensor | None, n_keep: torch.Tensor,
+                        top_k: torch.Tensor, max_keep_pages: int, max_top_k: int, out: torch.Tensor,
+                        sm_scale: float | None = None, dbg: DebugOutputs | None = None,
+                        status: torch.Tensor | None = None,
+                        stream: torch.cuda.Stream | None = None) -> torch.Tensor:
+    """decode_step without a workspace tensor: the library's built-in device
+    scratch is used instead (see hhr_decode_step_noalloc in include/hhr.h)."""
+    _expect(q, torch.bfloat16, (cfg.batch, cfg.num_q_heads, cfg.head_dim), "q")
+    _expect(out, torch.float32, (cfg.batch, cfg.num_q_heads, cfg.head_dim), "out")
+    if sm_scale is None:
+        sm_scale = 1.0 / math.sqrt(cfg.head_dim)
+    d = dbg.struct() if dbg is not None else None
+    st = lib().hhr_decode_step_noalloc(
+        ctypes.byref(cfg), _ptr(q), _ptr(R), _ptr(W), _ptr(cache.Krot), _ptr(cache.V), _ptr(cache.page_min),
+        _ptr(cache.page_max), _ptr(cache.codes), _ptr(seq_lens), _ptr(block_table), _ptr(n_keep), _ptr(top_k),
+        max_keep_pages, max_top_k, sm_scale, _ptr(out), ctypes.byref(d) if d is not None else None,
+        _ptr(status), _stream(stream))
+    check(st, "hhr_decode_step_noalloc")
     return out
 
 

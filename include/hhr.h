@@ -174,6 +174,44 @@ HHR_API hhr_status hhr_decode_step(const hhr_config* cfg, const void* q, const f
                            size_t workspace_bytes, int32_t* device_status,
                            hhr_stream_t stream);
 
+/* Size of the scratch array behind hhr_decode_step_noalloc (16 MiB). */
+#define HHR_NOALLOC_SCRATCH_BYTES (16u << 20)
+
+/*
+ * hhr_decode_step_noalloc -- hhr_decode_step without a caller workspace.
+ *
+ * (The paper has no counterpart; this is a library convenience.)  Some
+ * callers cannot call cudaMalloc at all: code that runs while another
+ * framework is capturing a CUDA graph (allocation is not a capturable
+ * operation and may break the capture), plugins of inference runtimes that
+ * must draw every byte from the host runtime's own memory pool, and
+ * latency-critical serving loops where an allocation (and the implicit
+ * synchronisation it can bring) is not allowed.  Such callers still pass
+ * every input and output, but the scratch comes from a fixed
+ * HHR_NOALLOC_SCRATCH_BYTES array in the library's device memory, which
+ * every GPU that loads the library holds until the process exits.
+ *   - Same arguments and results as hhr_decode_step, minus the workspace.
+ *   - Sizes whose workspace (hhr_decode_workspace_size) exceeds the array are
+ *     rejected with HHR_ERR_WORKSPACE and a message; nothing is launched.
+ *   - Allocates nothing: no cudaMalloc, cudaFree or allocating library call.
+ *   - The first call on a device looks up the array's device address with
+ *     that device current (cudaGetSymbolAddress) and caches it; make that
+ *     first call before any stream capture.
+ *   - Every call clears the part of the array it uses (one cudaMemsetAsync on
+ *     `stream`) and then runs the decode step in it.  All calls share the one
+ *     array, so calls that may overlap on the GPU (other streams, other host
+ *     threads) race with each other: serialise them.
+ */
+HHR_API hhr_status hhr_decode_step_noalloc(const hhr_config* cfg, const void* q, const float* R,
+                                           const void* W, const void* Krot, const void* Vcache,
+                                           const void* page_min, const void* page_max,
+                                           const uint64_t* codes, const int32_t* seq_lens,
+                                           const int32_t* block_table, const int32_t* n_keep_pages,
+                                           const int32_t* top_k, int32_t max_keep_pages,
+                                           int32_t max_top_k, float sm_scale, float* out,
+                                           const hhr_debug* dbg, int32_t* device_status,
+                                           hhr_stream_t stream);
+
 /* Bytes of workspace hhr_dense_decode needs. */
 HHR_API size_t hhr_dense_workspace_size(const hhr_config* cfg);
 
