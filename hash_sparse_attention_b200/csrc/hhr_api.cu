@@ -1,5 +1,5 @@
 // C ABI of libhhr.so: argument validation, workspace carve-out and launches.
-// The kernels live in hhr_build.cuh and hhr_decode.cuh.
+// The kernels live in hhr_build.cuh and hhr_fused.cuh.
 #include <algorithm>
 #include <cstdarg>
 #include <cstdio>
@@ -75,10 +75,26 @@ hhr_status make_dims(const hhr_config* cfg, Dims* dm) {
 
 size_t align256(size_t x) { return (x + 255) & ~size_t(255); }
 
+int ceil_div(long long a, long long b) { return (int)((a + b - 1) / b); }
+
+// Chunk counts of the fused kernel: scan chunks and gather chunks per unit.
+void chunk_counts(const Dims& dm, int Nmax, int Kmax, bool dense, int* C1, int* C3) {
+  if (dense) {
+    *C1 = 0;
+    *C3 = ceil_div(dm.T, FUSED_ROWS);
+  } else {
+    *C1 = ceil_div(dm.np_max, FUSED_ROWS);
+    const long long kcap = std::min<long long>(Kmax, (long long)Nmax * dm.P);
+    *C3 = std::max(1, ceil_div(kcap, FUSED_ROWS));
+  }
+}
+
 // Carves the workspace; with base == nullptr only the size is computed.
-size_t carve(const Dims& dm, int Nmax, int Kmax, int keys_per_split, int nsplit, char* base, Work* wk) {
+size_t carve(const Dims& dm, int Nmax, int Kmax, bool dense, char* base, Work* wk) {
   const size_t BH = (size_t)dm.B * dm.Hkv;
-  const int hist_stride = (int)((dm.G * dm.nb + 1 + 63) / 64 * 64);
+  int C1, C3;
+  chunk_counts(dm, Nmax, Kmax, dense, &C1, &C3);
+  const int part_cap = std::min(C3, MAX_GRID);
   size_t off = 0;
   auto take = [&](size_t bytes) {
     char* p = base ? base + off : nullptr;
@@ -86,32 +102,36 @@ size_t carve(const Dims& dm, int Nmax, int Kmax, int keys_per_split, int nsplit,
     return p;
   };
   Work w{};
+  w.ctrl = reinterpret_cast<unsigned*>(take(sizeof(unsigned) * (4 + BH * 8)));
   w.qrot = reinterpret_cast<float*>(take(sizeof(float) * dm.B * dm.Hq * D));
   w.qcodes = reinterpret_cast<uint64_t*>(take(sizeof(uint64_t) * dm.B * dm.Hq * dm.words));
-  w.U = reinterpret_cast<float*>(take(sizeof(float) * BH * dm.np_max));
-  w.sel_pages = reinterpret_cast<int*>(take(sizeof(int) * BH * Nmax));
-  w.n_sel = reinterpret_cast<int*>(take(sizeof(int) * BH));
-  w.scores = reinterpret_cast<int*>(take(sizeof(int) * BH * Nmax * dm.P));
-  w.hist = reinterpret_cast<int*>(take(sizeof(int) * BH * hist_stride));
-  w.sel_keys = reinterpret_cast<int*>(take(sizeof(int) * BH * Kmax));
-  w.n_keys = reinterpret_cast<int*>(take(sizeof(int) * BH));
-  w.part = reinterpret_cast<float*>(take(sizeof(float) * BH * nsplit * dm.G * (D + 2)));
-  w.tickets = reinterpret_cast<unsigned*>(take(sizeof(unsigned) * BH * 4));
+  w.part = reinterpret_cast<float*>(take(sizeof(float) * BH * part_cap * dm.G * (D + 2)));
+  if (!dense) {
+    w.U = reinterpret_cast<float*>(take(sizeof(float) * BH * dm.np_max));
+    w.sel_pages = reinterpret_cast<int*>(take(sizeof(int) * BH * Nmax));
+    w.sel_keys = reinterpret_cast<int*>(take(sizeof(int) * BH * Kmax));
+  }
   w.Nmax = Nmax;
   w.Kmax = Kmax;
-  w.hist_stride = hist_stride;
-  w.nsplit = nsplit;
-  w.keys_per_split = keys_per_split;
+  w.C1 = C1;
+  w.C3 = C3;
+  w.part_cap = part_cap;
   if (wk) *wk = w;
   return off;
 }
 
-int sparse_nsplit(const Dims& dm, int Nmax, int Kmax) {
-  const long long kcap = std::min<long long>(Kmax, (long long)Nmax * dm.P);
-  return (int)std::max<long long>(1, (kcap + ATT_SPLIT - 1) / ATT_SPLIT);
+// SMs of the current device (cached per device), at most MAX_GRID.
+int device_sms() {
+  static int cache[64] = {0};
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return 0;
+  if (cache[dev] == 0) {
+    int n = 0;
+    if (cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess || n <= 0) return 0;
+    cache[dev] = std::min(n, MAX_GRID);
+  }
+  return cache[dev];
 }
-
-int dense_nsplit(const Dims& dm) { return (dm.T + DENSE_SPLIT - 1) / DENSE_SPLIT; }
 
 // ---- group-size dispatch -------------------------------------------------
 #define HHR_DISPATCH_G(G_, ...)                          \
@@ -183,7 +203,8 @@ size_t hhr_decode_workspace_size(const hhr_config* cfg, int32_t max_keep_pages, 
   Dims dm;
   if (make_dims(cfg, &dm) != HHR_OK || max_keep_pages < 1 || max_top_k < 1) return 0;
   const int Nmax = std::min(max_keep_pages, dm.np_max);
-  return carve(dm, Nmax, max_top_k, ATT_SPLIT, sparse_nsplit(dm, Nmax, max_top_k), nullptr, nullptr);
+  if (Nmax > MAX_KEEP_PAGES || (long long)Nmax * dm.P > MAX_CANDIDATES) return 0;
+  return carve(dm, Nmax, max_top_k, false, nullptr, nullptr);
 }
 
 hhr_status hhr_workspace_init(void* workspace, size_t workspace_bytes, hhr_stream_t stream) {
@@ -206,7 +227,7 @@ hhr_status hhr_decode_step(const hhr_config* cfg, const void* q, const float* R,
       !top_k || !out || !workspace)
     return fail(HHR_ERR_INVALID_ARG, "hhr_decode_step: NULL pointer");
   if (dm.paged && !block_table) return fail(HHR_ERR_INVALID_ARG, "hhr_decode_step: paged needs block_table");
-  const void* al[] = {R, W, Krot, Vcache, page_min, page_max, codes};
+  const void* al[] = {q, R, W, Krot, Vcache, page_min, page_max, codes};
   for (const void* p : al)
     if (!aligned16(p)) return fail(HHR_ERR_INVALID_ARG, "hhr_decode_step: tensor not 16-byte aligned");
   if ((reinterpret_cast<uintptr_t>(workspace) & 255u) != 0)
@@ -215,12 +236,18 @@ hhr_status hhr_decode_step(const hhr_config* cfg, const void* q, const float* R,
     return fail(HHR_ERR_INVALID_ARG, "hhr_decode_step: max_keep_pages and max_top_k must be >= 1");
   if (!(sm_scale > 0.f)) return fail(HHR_ERR_INVALID_ARG, "hhr_decode_step: sm_scale must be > 0");
   const int Nmax = std::min(max_keep_pages, dm.np_max);
-  const int nsplit = sparse_nsplit(dm, Nmax, max_top_k);
-  const size_t need = carve(dm, Nmax, max_top_k, ATT_SPLIT, nsplit, nullptr, nullptr);
+  if (Nmax > MAX_KEEP_PAGES)
+    return fail(HHR_ERR_UNSUPPORTED, "hhr_decode_step: max_keep_pages %d (at most %d)", Nmax, MAX_KEEP_PAGES);
+  if ((long long)Nmax * dm.P > MAX_CANDIDATES)
+    return fail(HHR_ERR_UNSUPPORTED, "hhr_decode_step: max_keep_pages x page_size = %lld candidates (at most %d)",
+                (long long)Nmax * dm.P, MAX_CANDIDATES);
+  const size_t need = carve(dm, Nmax, max_top_k, false, nullptr, nullptr);
   if (workspace_bytes < need)
     return fail(HHR_ERR_WORKSPACE, "hhr_decode_step: workspace %zu bytes < %zu", workspace_bytes, need);
   Work wk;
-  carve(dm, Nmax, max_top_k, ATT_SPLIT, nsplit, static_cast<char*>(workspace), &wk);
+  carve(dm, Nmax, max_top_k, false, static_cast<char*>(workspace), &wk);
+  const int sms = device_sms();
+  if (sms <= 0) return fail(HHR_ERR_CUDA, "hhr_decode_step: cannot query the device");
 
   DecodeArgs a = {};
   a.dm = dm;
@@ -242,6 +269,7 @@ hhr_status hhr_decode_step(const hhr_config* cfg, const void* q, const float* R,
   if (dbg) a.dbg = *dbg;
   a.status = device_status;
   a.stream = reinterpret_cast<cudaStream_t>(stream);
+  a.num_sms = sms;
   cudaError_t e = cudaErrorInvalidValue;
   HHR_DISPATCH_G(dm.G, e = launch_decode<GG>(a));
   if (e != cudaSuccess) return fail(HHR_ERR_CUDA, "hhr_decode_step: launch failed: %s", cudaGetErrorString(e));
@@ -251,7 +279,7 @@ hhr_status hhr_decode_step(const hhr_config* cfg, const void* q, const float* R,
 size_t hhr_dense_workspace_size(const hhr_config* cfg) {
   Dims dm;
   if (make_dims(cfg, &dm) != HHR_OK) return 0;
-  return carve(dm, 1, 1, DENSE_SPLIT, dense_nsplit(dm), nullptr, nullptr);
+  return carve(dm, 1, 1, true, nullptr, nullptr);
 }
 
 hhr_status hhr_dense_decode(const hhr_config* cfg, const void* q, const float* R, const void* Krot,
@@ -264,18 +292,19 @@ hhr_status hhr_dense_decode(const hhr_config* cfg, const void* q, const float* R
   if (!q || !R || !Krot || !Vcache || !seq_lens || !out || !workspace)
     return fail(HHR_ERR_INVALID_ARG, "hhr_dense_decode: NULL pointer");
   if (dm.paged && !block_table) return fail(HHR_ERR_INVALID_ARG, "hhr_dense_decode: paged needs block_table");
-  const void* al[] = {R, Krot, Vcache};
+  const void* al[] = {q, R, Krot, Vcache};
   for (const void* p : al)
     if (!aligned16(p)) return fail(HHR_ERR_INVALID_ARG, "hhr_dense_decode: tensor not 16-byte aligned");
   if ((reinterpret_cast<uintptr_t>(workspace) & 255u) != 0)
     return fail(HHR_ERR_INVALID_ARG, "hhr_dense_decode: workspace not 256-byte aligned");
   if (!(sm_scale > 0.f)) return fail(HHR_ERR_INVALID_ARG, "hhr_dense_decode: sm_scale must be > 0");
-  const int nsplit = dense_nsplit(dm);
-  const size_t need = carve(dm, 1, 1, DENSE_SPLIT, nsplit, nullptr, nullptr);
+  const size_t need = carve(dm, 1, 1, true, nullptr, nullptr);
   if (workspace_bytes < need)
     return fail(HHR_ERR_WORKSPACE, "hhr_dense_decode: workspace %zu bytes < %zu", workspace_bytes, need);
   Work wk;
-  carve(dm, 1, 1, DENSE_SPLIT, nsplit, static_cast<char*>(workspace), &wk);
+  carve(dm, 1, 1, true, static_cast<char*>(workspace), &wk);
+  const int sms = device_sms();
+  if (sms <= 0) return fail(HHR_ERR_CUDA, "hhr_dense_decode: cannot query the device");
   DecodeArgs a = {};
   a.dm = dm;
   a.wk = wk;
@@ -289,6 +318,7 @@ hhr_status hhr_dense_decode(const hhr_config* cfg, const void* q, const float* R
   a.out = out;
   a.status = device_status;
   a.stream = reinterpret_cast<cudaStream_t>(stream);
+  a.num_sms = sms;
   cudaError_t e = cudaErrorInvalidValue;
   HHR_DISPATCH_G(dm.G, e = launch_dense<GG>(a));
   if (e != cudaSuccess) return fail(HHR_ERR_CUDA, "hhr_dense_decode: launch failed: %s", cudaGetErrorString(e));

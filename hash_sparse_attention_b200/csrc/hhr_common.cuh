@@ -17,21 +17,20 @@ struct Dims {
 };
 
 // Workspace carve-out of one decode step (device pointers).
-// `tickets` and `hist` are kept at zero between calls by the kernels that
-// use them; everything else is overwritten by every call.
+// `ctrl` holds the work-queue counter, the exit counter and per-unit flags and
+// counters; the kernel keeps it at zero between calls (the last CTA to leave
+// resets it).  Everything else is overwritten by every call.
 struct Work {
-  float* qrot;         // [B, Hq, D]
-  uint64_t* qcodes;    // [B, Hq, w]
-  float* U;            // [B, Hkv, np_max]
-  int* sel_pages;      // [B, Hkv, Nmax]
-  int* n_sel;          // [B, Hkv]
-  int* scores;         // [B, Hkv, Nmax * P]
-  int* hist;           // [B, Hkv, hist_stride]
-  int* sel_keys;       // [B, Hkv, Kmax]
-  int* n_keys;         // [B, Hkv]
-  float* part;         // [B, Hkv, nsplit, G * (D + 2)]
-  unsigned* tickets;   // [B, Hkv, 4]
-  int Nmax, Kmax, hist_stride, nsplit, keys_per_split;
+  float* qrot;         // [B, Hq, D]        q' = R_h q
+  uint64_t* qcodes;    // [B, Hq, w]        query sign codes
+  float* U;            // [B, Hkv, np_max]  page bounds (group max)
+  int* sel_pages;      // [B, Hkv, Nmax]    kept pages, ascending
+  int* sel_keys;       // [B, Hkv, Kmax]    kept rows, ascending
+  float* part;         // [B, Hkv, part_cap, G * (D + 2)] attention partials
+  unsigned* ctrl;      // [4 + B * Hkv * 8]
+  int Nmax, Kmax;      // budgets the workspace was sized for
+  int C1, C3;          // scan chunks and gather chunks per unit
+  int part_cap;        // partial slots per unit
 };
 
 // --- bf16 ---------------------------------------------------------------

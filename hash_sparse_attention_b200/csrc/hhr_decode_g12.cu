@@ -1,5 +1,5 @@
 // Decode kernels instantiated for group sizes 1 and 2.
-#include "hhr_decode.cuh"
+#include "hhr_fused.cuh"
 
 namespace hhr {
 HHR_INSTANTIATE_DECODE(1)

@@ -11,16 +11,11 @@
 
 namespace hhr {
 
-constexpr int PREP_THREADS = 256;
-constexpr int SCAN_THREADS = 512;
-constexpr int SCAN_PAGES = 128;          // pages per scan CTA: 4 per half-warp
-constexpr int SEL_KPT = 32;              // keys per thread in the page select
-constexpr int MAX_SELECT_PAGES = SCAN_THREADS * SEL_KPT;  // 16384 pages
-constexpr int LHP_THREADS = 256;         // one candidate row per thread
-constexpr int LHP_KPT = 16;              // candidates per thread per compaction tile
-constexpr int ATT_THREADS = 128;         // 8 half-warps
-constexpr int ATT_SPLIT = 128;           // kept rows per attention CTA
-constexpr int DENSE_SPLIT = 1024;        // rows per dense-attention CTA
+constexpr int MAX_SELECT_PAGES = 16384;  // pages of one sequence (page select keys in registers)
+constexpr int MAX_KEEP_PAGES = 2048;     // kept pages per sequence
+constexpr int MAX_CANDIDATES = 16384;    // kept pages x page size (scores in shared memory)
+constexpr int FUSED_ROWS = 128;          // pages per scan item, rows per gather item
+constexpr int MAX_GRID = 160;            // CTAs of the fused kernel (one per SM)
 
 struct DecodeArgs {
   Dims dm;
@@ -42,6 +37,7 @@ struct DecodeArgs {
   hhr_debug dbg;
   int* status;
   cudaStream_t stream;
+  int num_sms;
 };
 
 hhr_status record_error(hhr_status s, const char* msg);
