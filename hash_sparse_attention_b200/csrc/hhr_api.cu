@@ -94,7 +94,7 @@ size_t carve(const Dims& dm, int Nmax, int Kmax, bool dense, char* base, Work* w
   const size_t BH = (size_t)dm.B * dm.Hkv;
   int C1, C3;
   chunk_counts(dm, Nmax, Kmax, dense, &C1, &C3);
-  const int part_cap = std::min(C3, MAX_GRID);
+  const int max_groups = ceil_div(C3, FUSED_GROUP);
   size_t off = 0;
   auto take = [&](size_t bytes) {
     char* p = base ? base + off : nullptr;
@@ -102,10 +102,11 @@ size_t carve(const Dims& dm, int Nmax, int Kmax, bool dense, char* base, Work* w
     return p;
   };
   Work w{};
-  w.ctrl = reinterpret_cast<unsigned*>(take(sizeof(unsigned) * (4 + BH * 8)));
+  w.ctrl = reinterpret_cast<unsigned*>(take(sizeof(unsigned) * (4 + BH * (8 + max_groups))));
   w.qrot = reinterpret_cast<float*>(take(sizeof(float) * dm.B * dm.Hq * D));
   w.qcodes = reinterpret_cast<uint64_t*>(take(sizeof(uint64_t) * dm.B * dm.Hq * dm.words));
-  w.part = reinterpret_cast<float*>(take(sizeof(float) * BH * part_cap * dm.G * (D + 2)));
+  w.part = reinterpret_cast<float*>(take(sizeof(float) * BH * C3 * dm.G * (D + 2)));
+  w.gpart = reinterpret_cast<float*>(take(sizeof(float) * BH * max_groups * dm.G * (D + 2)));
   if (!dense) {
     w.U = reinterpret_cast<float*>(take(sizeof(float) * BH * dm.np_max));
     w.sel_pages = reinterpret_cast<int*>(take(sizeof(int) * BH * Nmax));
@@ -115,7 +116,7 @@ size_t carve(const Dims& dm, int Nmax, int Kmax, bool dense, char* base, Work* w
   w.Kmax = Kmax;
   w.C1 = C1;
   w.C3 = C3;
-  w.part_cap = part_cap;
+  w.max_groups = max_groups;
   if (wk) *wk = w;
   return off;
 }
@@ -298,6 +299,8 @@ hhr_status hhr_dense_decode(const hhr_config* cfg, const void* q, const float* R
   if ((reinterpret_cast<uintptr_t>(workspace) & 255u) != 0)
     return fail(HHR_ERR_INVALID_ARG, "hhr_dense_decode: workspace not 256-byte aligned");
   if (!(sm_scale > 0.f)) return fail(HHR_ERR_INVALID_ARG, "hhr_dense_decode: sm_scale must be > 0");
+  if (ceil_div(ceil_div(dm.T, FUSED_ROWS), FUSED_GROUP) > MAX_GATHER_GROUPS)
+    return fail(HHR_ERR_UNSUPPORTED, "hhr_dense_decode: max_seq_len %d too long", dm.T);
   const size_t need = carve(dm, 1, 1, true, nullptr, nullptr);
   if (workspace_bytes < need)
     return fail(HHR_ERR_WORKSPACE, "hhr_dense_decode: workspace %zu bytes < %zu", workspace_bytes, need);

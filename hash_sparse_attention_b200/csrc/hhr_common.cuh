@@ -26,11 +26,12 @@ struct Work {
   float* U;            // [B, Hkv, np_max]  page bounds (group max)
   int* sel_pages;      // [B, Hkv, Nmax]    kept pages, ascending
   int* sel_keys;       // [B, Hkv, Kmax]    kept rows, ascending
-  float* part;         // [B, Hkv, part_cap, G * (D + 2)] attention partials
-  unsigned* ctrl;      // [4 + B * Hkv * 8]
+  float* part;         // [B, Hkv, C3, G * (D + 2)] attention partial of every gather chunk
+  float* gpart;        // [B, Hkv, max_groups, G * (D + 2)] merged groups of chunks
+  unsigned* ctrl;      // [4 + B * Hkv * (8 + max_groups)] queue, flags, counters
   int Nmax, Kmax;      // budgets the workspace was sized for
   int C1, C3;          // scan chunks and gather chunks per unit
-  int part_cap;        // partial slots per unit
+  int max_groups;      // groups of 16 gather chunks per unit
 };
 
 // --- bf16 ---------------------------------------------------------------

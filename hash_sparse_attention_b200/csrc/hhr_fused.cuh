@@ -224,7 +224,7 @@ __device__ void fz_producer(const FzParams& p, const FzShared& s) {
   const Dims& dm = p.dm;
   const int U = dm.B * dm.Hkv;
   const int C1 = p.wk.C1, C3 = p.wk.C3;
-  const int prep_slots = 4 + dm.nb / 64;
+  const int prep_slots = DENSE ? 4 : 4 + dm.nb / 64;  // R_h, then W_h (not needed without hashing)
   unsigned nslot = 0, ndesc = 0, armed = 0;
   while (true) {
     int item = 0;
@@ -288,6 +288,15 @@ __device__ void fz_producer(const FzParams& p, const FzShared& s) {
       qsrc = p.wk.qrot + ((long long)x.b * dm.Hq + x.h * G) * D;
     }
     unsigned char* qdst = s.qbuf + d * FZ_QBUF;
+    // kept-row ids of a sparse gather chunk: lane holds rows lane + 32 i
+    int rid[4] = {0, 0, 0, 0};
+    if (!DENSE && kind == IT_GATHER) {
+#pragma unroll
+      for (int i = 0; i < 4; ++i) {
+        const int jj = lane + 32 * i;
+        if (jj < n) rid[i] = __ldcg(p.wk.sel_keys + (long long)u * p.wk.Kmax + (long long)c * FZ_ROWS + jj);
+      }
+    }
     bool aborted = false;
     for (int k = 0; k < nslots; ++k) {
       const unsigned gs = nslot + k;
@@ -350,8 +359,8 @@ __device__ void fz_producer(const FzParams& p, const FzShared& s) {
           for (int i = 0; i < 2; ++i) {
             const int j = lane + 32 * i;
             if (j < rows) {
-              const int t = DENSE ? c * FZ_ROWS + j0 + j
-                                  : __ldcg(p.wk.sel_keys + (long long)u * p.wk.Kmax + (long long)c * FZ_ROWS + j0 + j);
+              // row j0 + j = lane + 32 (2 (k & 1) + i): its id is rid[2 (k & 1) + i]
+              const int t = DENSE ? c * FZ_ROWS + j0 + j : (((k & 1) == 0) ? rid[i] : rid[2 + i]);
               const long long off = kv_row(dm, p.table, x.b, x.h, t, p.status);
               if (off >= 0) {
                 bulk_g2s(dst + j * 256, base + off, 256, &s.full[slot]);
@@ -447,7 +456,7 @@ __device__ __forceinline__ int cons_excl_scan(int v, int* red, int* total) {
 }
 
 // ---- PREP ------------------------------------------------------------------
-template <int G>
+template <int G, bool DENSE>
 __device__ void fz_prep(const FzParams& p, const FzShared& s, const Unit& x, int d, int s0) {
   const Dims& dm = p.dm;
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
@@ -484,6 +493,7 @@ __device__ void fz_prep(const FzParams& p, const FzShared& s, const Unit& x, int
       }
     }
   }
+  if constexpr (DENSE) return;  // full attention needs no codes (and has no W_h)
   // query codes: bit j = [ (W_h q)_j > 0 ]; products of bf16 values are exact
   // in fp32; the 128-term fp32 sum errs by at most 127 * 2^-24 * sum|w q|, so
   // below 2^-14 * sum|w q| the sign is taken from an fp64 recompute
@@ -840,30 +850,23 @@ __device__ void fz_select(const FzParams& p, const FzShared& s, const Unit& x) {
   (void)warp;
 }
 
-// ---- GATHER: running softmax attention over one chunk of kept rows ----------
-// Per-thread state for the V accumulation: channel pair cp = tid & 63 of
-// every head, over rows of key group kg = tid >> 6 (32 of each 128-row chunk).
+// ---- GATHER: softmax attention over one chunk of kept rows ---------------------
+// Writes the chunk's partial (unnormalised output, max and sum of weights per
+// head, in log2 units) to its fixed slot part[u][c].
 template <int G>
-struct GatherState {
-  float2 o[G];
-  float m[G];  // running max (log2 units), uniform over the CTA
-  float l[G];  // running sum of weights, uniform over the CTA
-  int unit;    // unit being accumulated, -1 when empty
-  int chunks;  // chunks accumulated since the last flush
-};
-
-template <int G>
-__device__ void fz_gather(const FzParams& p, const FzShared& s, GatherState<G>& st, int n, int d, int s0) {
+__device__ void fz_gather(const FzParams& p, const FzShared& s, const Unit& x, int c, int n, int d, int s0) {
   constexpr int GP = G <= 4 ? 4 : 8;  // heads padded to a power of two
   constexpr int CH = GP == 4 ? 8 : 4; // rows per half-warp per pass
   constexpr int NPASS = FZ_ROWS / (16 * CH);
   constexpr int NV = CH * GP;         // partial logits per lane
   constexpr int KPL = NV / 16;        // logits a lane keeps after the reduction
   constexpr int HS = GP / 2;          // heads per softmax thread (two head slots)
+  constexpr int NKG = FZ_CONS / 64;   // key groups of the V accumulation
   const int tid = threadIdx.x, hw = tid >> 4, ln = tid & 15, lane = tid & 31, warp = tid >> 5;
   float* S = reinterpret_cast<float*>(s.work);                  // [128][GP] logits (log2 units)
   float2* PP = reinterpret_cast<float2*>(s.work + 4096);        // [128][GP] (p, p)
   float* red = reinterpret_cast<float*>(s.work + 4096 + 8192);  // [8 warps][HS]
+  float2* OR = reinterpret_cast<float2*>(s.work + 16384);       // [NKG][G][64]
   const float* qs = reinterpret_cast<const float*>(s.qbuf + d * FZ_QBUF);
   const float qscale = p.sm_scale * 1.4426950408889634f;
   // ---- logits: pass r, half-warp hw takes rows 16 CH r + CH hw + kk; lane owns 8 channels ----
@@ -910,7 +913,7 @@ __device__ void fz_gather(const FzParams& p, const FzShared& s, GatherState<G>& 
     }
   }
   cons_sync();
-  // ---- chunk max per head, then weights relative to the new running max ----
+  // ---- chunk max per head, weights, sums ----
   // thread t: row j = t & 127, head slot gsl = t >> 7; heads gsl + 2e, e < HS
   const int j = tid & 127, gsl = tid >> 7;
   float sv[HS];
@@ -923,28 +926,24 @@ __device__ void fz_gather(const FzParams& p, const FzShared& s, GatherState<G>& 
     if (lane == 0) red[warp * HS + e] = m;
   }
   cons_sync();
-  float mnew[G], alpha[G];
+  float mh[GP];
 #pragma unroll
-  for (int g = 0; g < G; ++g) {
+  for (int g = 0; g < GP; ++g) {
     const int sl = g & 1, e = g >> 1;
     float cm = -INFINITY;
 #pragma unroll
     for (int w = 0; w < 4; ++w) cm = fmaxf(cm, red[(sl * 4 + w) * HS + e]);
-    mnew[g] = fmaxf(st.m[g], cm);
-    alpha[g] = (st.m[g] == -INFINITY) ? 0.f : exp2f(st.m[g] - mnew[g]);
+    mh[g] = cm;
   }
   float ps[HS];
 #pragma unroll
   for (int e = 0; e < HS; ++e) {
     const int g = gsl + 2 * e;
-    float pv = 0.f;
-    if (g < G && j < n) {
-      float mg = mnew[0];
+    float mg = mh[0];
 #pragma unroll
-      for (int gg = 1; gg < G; ++gg)
-        if (gg == g) mg = mnew[gg];
-      pv = exp2f(sv[e] - mg);
-    }
+    for (int gg = 1; gg < GP; ++gg)
+      if (gg == g) mg = mh[gg];
+    const float pv = (g < G && j < n) ? exp2f(sv[e] - mg) : 0.f;
     PP[j * GP + g] = make_float2(pv, pv);
     float t = pv;
 #pragma unroll
@@ -956,60 +955,35 @@ __device__ void fz_gather(const FzParams& p, const FzShared& s, GatherState<G>& 
 #pragma unroll
     for (int e = 0; e < HS; ++e) red[warp * HS + e] = ps[e];
   }
-#pragma unroll
-  for (int g = 0; g < G; ++g) {
-    st.o[g].x *= alpha[g];
-    st.o[g].y *= alpha[g];
-  }
   cons_sync();  // weights and sums complete
   // ---- V accumulation: channel pair cp of every head, rows of key group kg ----
   const int cp = tid & 63, kg = tid >> 6;
+  float2 o2[G];
+#pragma unroll
+  for (int g = 0; g < G; ++g) o2[g] = make_float2(0.f, 0.f);
+  constexpr int RPG = FZ_ROWS / NKG;  // rows per key group
 #pragma unroll 4
-  for (int r = 0; r < 32; ++r) {
-    const int jr = kg * 32 + r;
+  for (int r = 0; r < RPG; ++r) {
+    const int jr = kg * RPG + r;
     if (jr < n) {
       const uint32_t vw = *reinterpret_cast<const uint32_t*>(
           s.ring + (size_t)((s0 + 2 + jr / 64) % FZ_NSLOT) * FZ_SLOT + (jr % 64) * 256 + cp * 4);
       const float2 v2 = make_float2(bf_lo(vw), bf_hi(vw));
 #pragma unroll
-      for (int g = 0; g < G; ++g) st.o[g] = __ffma2_rn(PP[jr * GP + g], v2, st.o[g]);
+      for (int g = 0; g < G; ++g) o2[g] = __ffma2_rn(PP[jr * GP + g], v2, o2[g]);
     }
   }
 #pragma unroll
-  for (int g = 0; g < G; ++g) {
-    const int sl = g & 1, e = g >> 1;
-    float cs = 0.f;
-#pragma unroll
-    for (int w = 0; w < 4; ++w) cs += red[(sl * 4 + w) * HS + e];
-    st.l[g] = st.l[g] * alpha[g] + cs;
-    st.m[g] = mnew[g];
-  }
-}
-
-// Writes the accumulated partial of st.unit (sum over key groups) and, if it
-// completes the unit, merges all of the unit's partials into the output.
-template <int G>
-__device__ void fz_flush(const FzParams& p, const FzShared& s, GatherState<G>& st) {
-  const Dims& dm = p.dm;
-  const int tid = threadIdx.x;
-  const int u = st.unit;
-  constexpr int NKG = FZ_CONS / 64;                         // key groups
-  float2* OR = reinterpret_cast<float2*>(s.work + 16384);  // [NKG][G][64]
-  int* bc = reinterpret_cast<int*>(s.work + 16384 + NKG * 8 * 64 * 8);
-  const int cp = tid & 63, kg = tid >> 6;
-  cons_sync();  // the work area is free (previous users done)
-#pragma unroll
-  for (int g = 0; g < G; ++g) OR[(kg * G + g) * 64 + cp] = st.o[g];
-  if (tid == 0) bc[0] = (int)atomicAdd(unit_ctrl(p, u) + CU_NPART, 1u);
+  for (int g = 0; g < G; ++g) OR[(kg * G + g) * 64 + cp] = o2[g];
   cons_sync();
-  const int slot = bc[0];
+  // ---- the chunk's partial: key groups summed in order ----
   const int PS = G * (D + 2);
-  float* part = p.wk.part + ((long long)u * p.wk.part_cap + slot) * PS;
+  float* part = p.wk.part + ((long long)x.u * p.wk.C3 + c) * PS;
   for (int e = tid; e < G * 64; e += FZ_CONS) {
     const int g = e / 64, c2 = e % 64;
-    float2 a = make_float2(0.f, 0.f);
+    float2 a = OR[(0 * G + g) * 64 + c2];
 #pragma unroll
-    for (int k = 0; k < NKG; ++k) {
+    for (int k = 1; k < NKG; ++k) {
       const float2 v = OR[(k * G + g) * 64 + c2];
       a.x += v.x;
       a.y += v.y;
@@ -1017,75 +991,136 @@ __device__ void fz_flush(const FzParams& p, const FzShared& s, GatherState<G>& s
     *reinterpret_cast<float2*>(part + g * D + 2 * c2) = a;
   }
   if (tid < G) {
-    part[G * D + tid] = st.m[tid];
-    part[G * D + G + tid] = st.l[tid];
+    const int sl = tid & 1, e = tid >> 1;
+    float cs = 0.f;
+#pragma unroll
+    for (int w = 0; w < 4; ++w) cs += red[(sl * 4 + w) * HS + e];
+    part[G * D + tid] = mh[0];
+#pragma unroll
+    for (int gg = 1; gg < G; ++gg)
+      if (gg == tid) part[G * D + tid] = mh[gg];
+    part[G * D + G + tid] = cs;
   }
+}
+
+// Merges K partials src[0 .. K) (stride G (D + 2) floats) in index order:
+// M = max m_k, w_k = 2^(m_k - M), L = sum w_k l_k, O = sum w_k o_k.  With
+// dst, the merged partial (O, M, L) is written there; otherwise out = O / L.
+// K <= 256.  Loads are issued in batches so that a merge costs a few L2
+// round trips, not one per partial.
+template <int G>
+__device__ void fz_merge(const FzShared& s, const float* src, int K, float* dst, float* out) {
+  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+  const int PS = G * (D + 2);
+  float* wsm = reinterpret_cast<float*>(s.work + 32768);  // [256][G] weights, then M[8], L[8]
+  float* MH = wsm + 256 * G;
+  float* LH = MH + 8;
+  cons_sync();  // the work area's previous readers are done
+  if (warp < G) {
+    const int g = warp;
+    float mk[8], lk[8];
+#pragma unroll
+    for (int i = 0; i < 8; ++i) {
+      const int k = lane + 32 * i;
+      mk[i] = (k < K) ? __ldcg(src + (long long)k * PS + G * D + g) : -INFINITY;
+      lk[i] = (k < K) ? __ldcg(src + (long long)k * PS + G * D + G + g) : 0.f;
+    }
+    float M = mk[0];
+#pragma unroll
+    for (int i = 1; i < 8; ++i) M = fmaxf(M, mk[i]);
+#pragma unroll
+    for (int o = 16; o >= 1; o >>= 1) M = fmaxf(M, __shfl_xor_sync(0xffffffffu, M, o));
+    float L = 0.f;
+#pragma unroll
+    for (int i = 0; i < 8; ++i) {
+      const int k = lane + 32 * i;
+      const float w = (mk[i] == -INFINITY) ? 0.f : exp2f(mk[i] - M);
+      if (k < K) wsm[k * G + g] = w;
+      L = fmaf(lk[i], w, L);
+    }
+#pragma unroll
+    for (int o = 16; o >= 1; o >>= 1) L += __shfl_xor_sync(0xffffffffu, L, o);
+    if (lane == 0) {
+      MH[g] = M;
+      LH[g] = L;
+    }
+  }
+  cons_sync();
+  for (int f = tid; f < 32 * G; f += FZ_CONS) {
+    const int g = f >> 5, c4 = f & 31;
+    float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
+    for (int k0 = 0; k0 < K; k0 += 8) {
+      float4 v[8];
+#pragma unroll
+      for (int i = 0; i < 8; ++i)
+        v[i] = (k0 + i < K) ? __ldcg(reinterpret_cast<const float4*>(src + (long long)(k0 + i) * PS + g * D) + c4)
+                            : make_float4(0.f, 0.f, 0.f, 0.f);
+#pragma unroll
+      for (int i = 0; i < 8; ++i) {
+        const float w = (k0 + i < K) ? wsm[(k0 + i) * G + g] : 0.f;
+        acc.x = fmaf(v[i].x, w, acc.x);
+        acc.y = fmaf(v[i].y, w, acc.y);
+        acc.z = fmaf(v[i].z, w, acc.z);
+        acc.w = fmaf(v[i].w, w, acc.w);
+      }
+    }
+    if (dst) {
+      *reinterpret_cast<float4*>(dst + g * D + 4 * c4) = acc;
+    } else {
+      const float L = LH[g];
+      const float r = L > 0.f ? 1.f / L : 0.f;
+      *reinterpret_cast<float4*>(out + g * D + 4 * c4) = make_float4(acc.x * r, acc.y * r, acc.z * r, acc.w * r);
+    }
+  }
+  if (dst && tid < G) {
+    dst[G * D + tid] = MH[tid];
+    dst[G * D + G + tid] = LH[tid];
+  }
+}
+
+// After a chunk's partial is written: the last chunk of its group of
+// FZ_GROUP chunks merges the group (in chunk order) into gpart[u][group];
+// the last group of the unit merges the groups (in order) into the output.
+constexpr int FZ_GROUP = FUSED_GROUP;
+
+template <int G>
+__device__ void fz_gather_done(const FzParams& p, const FzShared& s, const Unit& x, int c) {
+  const int tid = threadIdx.x;
+  const int PS = G * (D + 2);
+  int* bc = reinterpret_cast<int*>(s.work + FZ_WORK - 64);
+  const unsigned nk = __ldcg(unit_ctrl(p, x.u) + CU_NKEYS);
+  const int nchunks = (int)((nk + FZ_ROWS - 1) / FZ_ROWS);
+  const int ngroups = (nchunks + FZ_GROUP - 1) / FZ_GROUP;
+  const int grp = c / FZ_GROUP;
+  const int gsize = min(FZ_GROUP, nchunks - grp * FZ_GROUP);
   __threadfence();
   cons_sync();
   if (tid == 0) {
-    const unsigned done = atomicAdd(unit_ctrl(p, u) + CU_GATHER, (unsigned)st.chunks) + (unsigned)st.chunks;
-    const unsigned nk = __ldcg(unit_ctrl(p, u) + CU_NKEYS);
-    const unsigned nchunks = (nk + FZ_ROWS - 1) / FZ_ROWS;
-    bc[1] = (done == nchunks) ? 1 : 0;
+    unsigned* gc = p.wk.ctrl + 4 + (p.dm.B * p.dm.Hkv) * CU_STRIDE + x.u * p.wk.max_groups + grp;
+    bc[0] = (atomicAdd(gc, 1u) + 1u == (unsigned)gsize) ? 1 : 0;
   }
   cons_sync();
-  const bool last = bc[1] != 0;
-  // reset the state
-#pragma unroll
-  for (int g = 0; g < G; ++g) {
-    st.o[g] = make_float2(0.f, 0.f);
-    st.m[g] = -INFINITY;
-    st.l[g] = 0.f;
-  }
-  st.unit = -1;
-  st.chunks = 0;
-  if (!last) return;
+  if (!bc[0]) return;
   __threadfence();
-  // ---- merge every partial of unit u ----
-  const int nparts = (int)__ldcg(unit_ctrl(p, u) + CU_NPART);
-  float* wsm = reinterpret_cast<float*>(s.work + 16384);  // [nparts][G] weights, then [G] M, [G] L
-  const float* pb = p.wk.part + (long long)u * p.wk.part_cap * PS;
-  float* Mh = wsm + p.wk.part_cap * G;
-  float* Lh = Mh + G;
-  if (tid < G) {
-    float M = -INFINITY;
-    for (int q = 0; q < nparts; ++q) M = fmaxf(M, __ldcg(pb + (long long)q * PS + G * D + tid));
-    float Ls = 0.f;
-    for (int q = 0; q < nparts; ++q) {
-      const float mq = __ldcg(pb + (long long)q * PS + G * D + tid);
-      const float w = (mq == -INFINITY) ? 0.f : exp2f(mq - M);
-      wsm[q * G + tid] = w;
-      Ls = fmaf(__ldcg(pb + (long long)q * PS + G * D + G + tid), w, Ls);
-    }
-    Mh[tid] = M;
-    Lh[tid] = Ls;
-  }
+  const float* chunk_parts = p.wk.part + ((long long)x.u * p.wk.C3 + grp * FZ_GROUP) * PS;
+  float* gp = p.wk.gpart + ((long long)x.u * p.wk.max_groups + grp) * PS;
+  fz_merge<G>(s, chunk_parts, gsize, gp, nullptr);
+  __threadfence();
   cons_sync();
-  const Unit x = unit_of(p, u);
-  for (int e = tid; e < G * D; e += FZ_CONS) {
-    const int g = e / D, c = e % D;
-    float O = 0.f;
-    for (int q = 0; q < nparts; ++q) O = fmaf(__ldcg(pb + (long long)q * PS + g * D + c), wsm[q * G + g], O);
-    const float Ls = Lh[g];
-    p.out[((long long)x.b * dm.Hq + x.h * G + g) * D + c] = Ls > 0.f ? O / Ls : 0.f;
-  }
+  if (tid == 0) bc[1] = (atomicAdd(unit_ctrl(p, x.u) + CU_GATHER, 1u) + 1u == (unsigned)ngroups) ? 1 : 0;
+  cons_sync();
+  if (!bc[1]) return;
+  __threadfence();
+  fz_merge<G>(s, p.wk.gpart + (long long)x.u * p.wk.max_groups * PS, ngroups, nullptr,
+              p.out + ((long long)x.b * p.dm.Hq + x.h * G) * D);
 }
 
 template <int G, int WORDS, bool DENSE>
 __device__ void fz_consumer(const FzParams& p, const FzShared& s) {
   const Dims& dm = p.dm;
   const int tid = threadIdx.x, lane = tid & 31;
-  const int prep_slots = 4 + dm.nb / 64;
+  const int prep_slots = DENSE ? 4 : 4 + dm.nb / 64;  // R_h, then W_h (not needed without hashing)
   unsigned nslot = 0, ndesc = 0;
-  GatherState<G> st;
-#pragma unroll
-  for (int g = 0; g < G; ++g) {
-    st.o[g] = make_float2(0.f, 0.f);
-    st.m[g] = -INFINITY;
-    st.l[g] = 0.f;
-  }
-  st.unit = -1;
-  st.chunks = 0;
   int* dec = reinterpret_cast<int*>(s.work + FZ_WORK - 32);  // wait decisions of thread 0
   while (true) {
     const int d = (int)(ndesc % FZ_NDESC);
@@ -1097,9 +1132,6 @@ __device__ void fz_consumer(const FzParams& p, const FzShared& s) {
     mbar_confirm(&s.dfull[d], (ndesc / FZ_NDESC) & 1);
     const FzDesc ds = s.desc[d];
     cons_sync();  // everyone holds the descriptor before dec is written again
-    if (ds.kind == IT_GATHER || ds.kind == IT_END) {
-      if (st.unit >= 0 && (ds.kind == IT_END || ds.unit != st.unit)) fz_flush<G>(p, s, st);
-    }
     if (ds.kind == IT_END) break;
     const int nslots = ds.kind == IT_PREP ? prep_slots : 4;
     const int s0 = (int)(nslot % FZ_NSLOT);
@@ -1119,13 +1151,11 @@ __device__ void fz_consumer(const FzParams& p, const FzShared& s) {
     }
     const Unit x = unit_of(p, ds.unit);
     if (ds.kind == IT_PREP) {
-      fz_prep<G>(p, s, x, d, s0);
+      fz_prep<G, DENSE>(p, s, x, d, s0);
     } else if (ds.kind == IT_SCAN) {
       if constexpr (!DENSE) fz_scan<G>(p, s, x, ds.chunk, ds.n, d, s0);
     } else {
-      if (st.unit < 0) st.unit = ds.unit;
-      fz_gather<G>(p, s, st, ds.n, d, s0);
-      ++st.chunks;
+      fz_gather<G>(p, s, x, ds.chunk, ds.n, d, s0);
     }
     // release the slots and the descriptor (one arrival per consumer warp)
     __syncwarp();
@@ -1153,6 +1183,8 @@ __device__ void fz_consumer(const FzParams& p, const FzShared& s) {
         st_release(unit_ctrl(p, x.u) + CU_PREP, 1u);
         if (DENSE || x.L == 0) st_release(unit_ctrl(p, x.u) + CU_SEL, 1u);
       }
+    } else if (ds.kind == IT_GATHER) {
+      fz_gather_done<G>(p, s, x, ds.chunk);
     } else if (ds.kind == IT_SCAN) {
       __threadfence();
       cons_sync();
@@ -1221,7 +1253,7 @@ __global__ void __launch_bounds__(FZ_THREADS, 1) hhr_fused_kernel(FzParams p) {
   if (s_last) {
     __threadfence();
     const int U = p.dm.B * p.dm.Hkv;
-    for (int i = tid; i < U * CU_STRIDE; i += blockDim.x) p.wk.ctrl[4 + i] = 0u;
+    for (int i = tid; i < U * (CU_STRIDE + p.wk.max_groups); i += blockDim.x) p.wk.ctrl[4 + i] = 0u;
     if (tid == 0) {
       p.wk.ctrl[0] = 0u;
       p.wk.ctrl[1] = 0u;

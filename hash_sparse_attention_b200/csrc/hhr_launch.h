@@ -16,6 +16,8 @@ constexpr int MAX_KEEP_PAGES = 2048;     // kept pages per sequence
 constexpr int MAX_CANDIDATES = 16384;    // kept pages x page size (scores in shared memory)
 constexpr int FUSED_ROWS = 128;          // pages per scan item, rows per gather item
 constexpr int MAX_GRID = 160;            // CTAs of the fused kernel (one per SM)
+constexpr int FUSED_GROUP = 16;          // gather chunks merged together first
+constexpr int MAX_GATHER_GROUPS = 256;   // groups per unit (final merge width)
 
 struct DecodeArgs {
   Dims dm;
