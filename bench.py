@@ -388,10 +388,11 @@ def run_hhr(args, rank, world):
     achieved = statistics.mean(per_layer_bytes) / mean_layer_s / 1e9
     roofline = {"bound": "hbm", "achieved": achieved, "peak": pk["hbm_gbs"], "unit": "GB/s",
                 "frac": achieved / pk["hbm_gbs"], "traffic": None,
-                "kernel": "hhr_decode_step (one layer: prep_query, gkr_scan_select, lhp_score_select, attn_split)",
+                "kernel": "hhr_fused_kernel (one launch per layer: query prep, page scan, page and key select, "
+                          "sparse attention, partial merges)",
                 "peak_source": pk["source"],
                 "step_gbs": step_bytes / t_step / 1e9, "step_frac": step_bytes / t_step / 1e9 / pk["hbm_gbs"]}
-    launches_per_step = 4 * len(layers)
+    launches_per_step = len(layers)  # one hhr_fused_kernel launch per layer
     result = {
         "metric": METRIC,
         "value": whole_job_throughput(B * args.steps, world, secs_max),

@@ -50,8 +50,8 @@ hhr_status make_dims(const hhr_config* cfg, Dims* dm) {
   if (cfg->hash_bits != 64 && cfg->hash_bits != 128 && cfg->hash_bits != 256)
     return fail(HHR_ERR_UNSUPPORTED, "hash_bits %d (64, 128 or 256)", cfg->hash_bits);
   const long long np_max = ((long long)cfg->max_seq_len + cfg->page_size - 1) / cfg->page_size;
-  if (np_max > MAX_SELECT_PAGES)
-    return fail(HHR_ERR_UNSUPPORTED, "%lld pages per sequence (at most %d)", np_max, MAX_SELECT_PAGES);
+  if (np_max > MAX_DENSE_PAGES)
+    return fail(HHR_ERR_UNSUPPORTED, "%lld pages per sequence (at most %d)", np_max, MAX_DENSE_PAGES);
   if (cfg->paged) {
     if (cfg->num_blocks < 1) return fail(HHR_ERR_INVALID_ARG, "paged: num_blocks must be >= 1");
     if (cfg->max_blocks_per_seq < np_max)
@@ -105,8 +105,8 @@ size_t carve(const Dims& dm, int Nmax, int Kmax, bool dense, char* base, Work* w
   w.ctrl = reinterpret_cast<unsigned*>(take(sizeof(unsigned) * (4 + BH * (8 + max_groups))));
   w.qrot = reinterpret_cast<float*>(take(sizeof(float) * dm.B * dm.Hq * D));
   w.qcodes = reinterpret_cast<uint64_t*>(take(sizeof(uint64_t) * dm.B * dm.Hq * dm.words));
-  w.part = reinterpret_cast<float*>(take(sizeof(float) * BH * C3 * dm.G * (D + 2)));
-  w.gpart = reinterpret_cast<float*>(take(sizeof(float) * BH * max_groups * dm.G * (D + 2)));
+  w.part = reinterpret_cast<float*>(take(sizeof(float) * BH * C3 * (dm.G * D + 16)));
+  w.gpart = reinterpret_cast<float*>(take(sizeof(float) * BH * max_groups * (dm.G * D + 16)));
   if (!dense) {
     w.U = reinterpret_cast<float*>(take(sizeof(float) * BH * dm.np_max));
     w.sel_pages = reinterpret_cast<int*>(take(sizeof(int) * BH * Nmax));
@@ -204,7 +204,7 @@ size_t hhr_decode_workspace_size(const hhr_config* cfg, int32_t max_keep_pages, 
   Dims dm;
   if (make_dims(cfg, &dm) != HHR_OK || max_keep_pages < 1 || max_top_k < 1) return 0;
   const int Nmax = std::min(max_keep_pages, dm.np_max);
-  if (Nmax > MAX_KEEP_PAGES || (long long)Nmax * dm.P > MAX_CANDIDATES) return 0;
+  if (dm.np_max > MAX_SELECT_PAGES || Nmax > MAX_KEEP_PAGES || (long long)Nmax * dm.P > MAX_CANDIDATES) return 0;
   return carve(dm, Nmax, max_top_k, false, nullptr, nullptr);
 }
 
@@ -224,6 +224,9 @@ hhr_status hhr_decode_step(const hhr_config* cfg, const void* q, const float* R,
   Dims dm;
   hhr_status s = make_dims(cfg, &dm);
   if (s != HHR_OK) return s;
+  if (dm.np_max > MAX_SELECT_PAGES)
+    return fail(HHR_ERR_UNSUPPORTED, "hhr_decode_step: %d pages per sequence (at most %d)", dm.np_max,
+                MAX_SELECT_PAGES);
   if (!q || !R || !W || !Krot || !Vcache || !page_min || !page_max || !codes || !seq_lens || !n_keep_pages ||
       !top_k || !out || !workspace)
     return fail(HHR_ERR_INVALID_ARG, "hhr_decode_step: NULL pointer");

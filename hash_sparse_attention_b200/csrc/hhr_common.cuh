@@ -26,8 +26,8 @@ struct Work {
   float* U;            // [B, Hkv, np_max]  page bounds (group max)
   int* sel_pages;      // [B, Hkv, Nmax]    kept pages, ascending
   int* sel_keys;       // [B, Hkv, Kmax]    kept rows, ascending
-  float* part;         // [B, Hkv, C3, G * (D + 2)] attention partial of every gather chunk
-  float* gpart;        // [B, Hkv, max_groups, G * (D + 2)] merged groups of chunks
+  float* part;         // [B, Hkv, C3, G * D + 16] attention partial of every gather chunk
+  float* gpart;        // [B, Hkv, max_groups, G * D + 16] merged groups of chunks
   unsigned* ctrl;      // [4 + B * Hkv * (8 + max_groups)] queue, flags, counters
   int Nmax, Kmax;      // budgets the workspace was sized for
   int C1, C3;          // scan chunks and gather chunks per unit

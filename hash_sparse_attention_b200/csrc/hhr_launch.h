@@ -11,7 +11,8 @@
 
 namespace hhr {
 
-constexpr int MAX_SELECT_PAGES = 16384;  // pages of one sequence (page select keys in registers)
+constexpr int MAX_SELECT_PAGES = 8192;   // pages of one sequence in the page select (shared memory)
+constexpr int MAX_DENSE_PAGES = 16384;   // pages of one sequence elsewhere
 constexpr int MAX_KEEP_PAGES = 2048;     // kept pages per sequence
 constexpr int MAX_CANDIDATES = 16384;    // kept pages x page size (scores in shared memory)
 constexpr int FUSED_ROWS = 128;          // pages per scan item, rows per gather item

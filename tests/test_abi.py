@@ -78,7 +78,8 @@ def test_workspace_size_is_host_arithmetic(L):
     (dict(num_q_heads=30), _lib.HHR_ERR_INVALID_ARG),    # not a multiple
     (dict(page_size=8), _lib.HHR_ERR_UNSUPPORTED),
     (dict(hash_bits=96), _lib.HHR_ERR_UNSUPPORTED),
-    (dict(max_seq_len=1 << 20), _lib.HHR_ERR_UNSUPPORTED),  # more pages than one select holds
+    (dict(max_seq_len=1 << 20), _lib.HHR_ERR_UNSUPPORTED),  # more pages than supported
+    (dict(max_seq_len=1 << 18), _lib.HHR_ERR_UNSUPPORTED),  # more pages than the page select holds
     (dict(paged=1, num_blocks=0), _lib.HHR_ERR_INVALID_ARG),
     (dict(paged=1, num_blocks=10, max_blocks_per_seq=3), _lib.HHR_ERR_INVALID_ARG),
 ])

@@ -66,9 +66,9 @@ def test_noalloc_rejects_sizes_beyond_the_scratch():
     if not torch.cuda.is_available():
         pytest.skip("no CUDA device")
     cfg = hhr.make_config(64, 32, 8, 16, 256, 131072)
-    need = _lib.lib().hhr_decode_workspace_size(ctypes.byref(cfg), 8192, 131072)
+    need = _lib.lib().hhr_decode_workspace_size(ctypes.byref(cfg), 1024, 13108)
     assert need > _lib.NOALLOC_SCRATCH_BYTES
     fake = [0x10000 + 256 * i for i in range(12)]
-    st = _lib.lib().hhr_decode_step_noalloc(ctypes.byref(cfg), *fake, 8192, 131072, 0.1, 0x90000, None, None, None)
+    st = _lib.lib().hhr_decode_step_noalloc(ctypes.byref(cfg), *fake, 1024, 13108, 0.1, 0x90000, None, None, None)
     assert st == _lib.HHR_ERR_WORKSPACE
     assert b"scratch" in _lib.lib().hhr_last_error()
