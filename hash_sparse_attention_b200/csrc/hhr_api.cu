@@ -78,12 +78,14 @@ size_t align256(size_t x) { return (x + 255) & ~size_t(255); }
 int ceil_div(long long a, long long b) { return (int)((a + b - 1) / b); }
 
 // Chunk counts of the fused kernel: scan chunks and gather chunks per unit.
-void chunk_counts(const Dims& dm, int Nmax, int Kmax, bool dense, int* C1, int* C3) {
+void chunk_counts(const Dims& dm, int Nmax, int Kmax, bool dense, int* C1, int* C2, int* C3) {
   if (dense) {
     *C1 = 0;
+    *C2 = 0;
     *C3 = ceil_div(dm.T, FUSED_ROWS);
   } else {
     *C1 = ceil_div(dm.np_max, FUSED_ROWS);
+    *C2 = ceil_div((long long)Nmax * dm.P, FUSED_SCORE);
     const long long kcap = std::min<long long>(Kmax, (long long)Nmax * dm.P);
     *C3 = std::max(1, ceil_div(kcap, FUSED_ROWS));
   }
@@ -92,8 +94,8 @@ void chunk_counts(const Dims& dm, int Nmax, int Kmax, bool dense, int* C1, int* 
 // Carves the workspace; with base == nullptr only the size is computed.
 size_t carve(const Dims& dm, int Nmax, int Kmax, bool dense, char* base, Work* wk) {
   const size_t BH = (size_t)dm.B * dm.Hkv;
-  int C1, C3;
-  chunk_counts(dm, Nmax, Kmax, dense, &C1, &C3);
+  int C1, C2, C3;
+  chunk_counts(dm, Nmax, Kmax, dense, &C1, &C2, &C3);
   const int max_groups = ceil_div(C3, FUSED_GROUP);
   size_t off = 0;
   auto take = [&](size_t bytes) {
@@ -107,14 +109,23 @@ size_t carve(const Dims& dm, int Nmax, int Kmax, bool dense, char* base, Work* w
   w.qcodes = reinterpret_cast<uint64_t*>(take(sizeof(uint64_t) * dm.B * dm.Hq * dm.words));
   w.part = reinterpret_cast<float*>(take(sizeof(float) * BH * C3 * (dm.G * D + 16)));
   w.gpart = reinterpret_cast<float*>(take(sizeof(float) * BH * max_groups * (dm.G * D + 16)));
+  const int Ustride = (dm.np_max + 31) / 32 * 32;
+  const int Cmax = Nmax * dm.P;
+  const int HB = (dm.G * dm.nb + 1 + 7) / 8 * 8;
   if (!dense) {
-    w.U = reinterpret_cast<float*>(take(sizeof(float) * BH * dm.np_max));
+    w.U = reinterpret_cast<float*>(take(sizeof(float) * BH * Ustride));
     w.sel_pages = reinterpret_cast<int*>(take(sizeof(int) * BH * Nmax));
     w.sel_keys = reinterpret_cast<int*>(take(sizeof(int) * BH * Kmax));
+    w.kscore = reinterpret_cast<uint16_t*>(take(sizeof(uint16_t) * BH * Cmax));
+    w.khist = reinterpret_cast<int*>(take(sizeof(int) * BH * HB));
   }
   w.Nmax = Nmax;
   w.Kmax = Kmax;
+  w.Cmax = Cmax;
+  w.HB = HB;
+  w.Ustride = Ustride;
   w.C1 = C1;
+  w.C2 = C2;
   w.C3 = C3;
   w.max_groups = max_groups;
   if (wk) *wk = w;

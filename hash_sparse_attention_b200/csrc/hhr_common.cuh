@@ -23,14 +23,19 @@ struct Dims {
 struct Work {
   float* qrot;         // [B, Hq, D]        q' = R_h q
   uint64_t* qcodes;    // [B, Hq, w]        query sign codes
-  float* U;            // [B, Hkv, np_max]  page bounds (group max)
+  float* U;            // [B, Hkv, Ustride] page bounds (group max)
   int* sel_pages;      // [B, Hkv, Nmax]    kept pages, ascending
   int* sel_keys;       // [B, Hkv, Kmax]    kept rows, ascending
   float* part;         // [B, Hkv, C3, G * D + 16] attention partial of every gather chunk
   float* gpart;        // [B, Hkv, max_groups, G * D + 16] merged groups of chunks
+  uint16_t* kscore;    // [B, Hkv, Cmax]    Hamming score of every candidate row
+  int* khist;          // [B, Hkv, HB]      score histogram (kept at zero between calls)
   unsigned* ctrl;      // [4 + B * Hkv * (8 + max_groups)] queue, flags, counters
   int Nmax, Kmax;      // budgets the workspace was sized for
-  int C1, C3;          // scan chunks and gather chunks per unit
+  int Cmax;            // Nmax * page size: candidate rows per unit
+  int HB;              // histogram stride (>= G * hash bits + 1)
+  int Ustride;         // row stride of U (np_max rounded up to 32)
+  int C1, C2, C3;      // scan, score and gather chunks per unit
   int max_groups;      // groups of 16 gather chunks per unit
 };
 

@@ -2,27 +2,31 @@
 //
 // Work is a queue of items claimed in order by the CTAs (one CTA per SM).
 // For units u = (sequence b, KV head h) the queue holds, in this order:
-//   PREP(u)        for every unit: q' = R_h q, then the query codes
-//   SCAN(u, c)     for every unit in turn: page bounds of pages
-//                  [128c, 128c + 128)
-//   GATHER(u, c)   for every unit in turn: softmax attention over kept rows
-//                  [128c, 128c + 128), written as a partial per chunk
-// Three more steps run as local tasks of the CTA that completes their
-// inputs (it sees its own counter increment reach the target):
-//   SELECT(u)      after the last scan chunk and the query codes of u: page
-//                  top-N, Hamming scores of the kept pages' rows, key top-k
-//   GMERGE(u, g)   after the 16 chunks of group g: their partials, merged
-//   MERGE(u)       after the last group: the groups, merged into the output
-// So no CTA ever waits for another CTA's consumers; only the producer waits,
-// for q' (scan) or the selection (gather) of a unit claimed before.  The
-// queue is unit-major, so late units are scanned while early units are
-// selected and gathered.
+//   PREP(u)        for every unit: q' = R_h q, then the query sign codes
+//   SCAN(u, c)     page bounds of pages [128c, 128c + 128)
+//   SCORE(u, c)    Hamming scores of candidates [1024c, 1024c + 1024) (the
+//                  rows of the kept pages, in page order) and their histogram
+//   GATHER(u, c)   softmax attention over kept rows [128c, 128c + 128),
+//                  written as a partial per chunk
+// Four more steps run as local tasks of the CTA whose counter increment
+// completes their inputs:
+//   PSEL(u)        after the last scan chunk of u: page top-N
+//   KSEL(u)        after the last score chunk of u: key top-k from the
+//                  score histogram, kept rows compacted in index order
+//   GMERGE(u, g)   after the 16 gather chunks of group g: their partials merged
+//   MERGE(u)       after the last group: the groups merged into the output
+// No CTA ever waits for another CTA's consumers; only the producer waits, for
+// q' (scan), the kept pages and query codes (score) or the kept rows (gather)
+// of a unit claimed before.
 //
-// Warps 0-7 consume; warp 8 (producer) claims items and moves their bytes
-// (R_h, W_h, q or q', page metadata rows, K'/V rows) into a ring of shared
-// memory slots with cp.async.bulk, each slot completing on an mbarrier;
-// warp 9 (finisher) publishes completions (a gpu-scope fence, then an
-// acquire-release counter increment) and posts the tasks that become ready.
+// Warps 0-15 consume; warp 16 (producer) claims items and moves their bytes
+// (R_h, W_h, q or q', page metadata rows, code rows, K'/V rows) into a ring
+// of shared memory slots with cp.async.bulk, each slot completing on an
+// mbarrier; warp 17 (finisher) publishes completions (a gpu-scope fence, then
+// an acquire-release counter increment) and posts the tasks that become ready.
+// Inside an item every consumer lane owns 4 channels of a 128-channel row, so
+// each warp reads whole 256-byte rows from shared memory without conflicts
+// and reduces dot products with one transposed butterfly.
 //
 // Every wait (mbarrier, shared flag or global counter) is bounded by a clock
 // budget; on expiry the kernel records HHR_ERR_TIMEOUT in the status word,
@@ -89,9 +93,10 @@ __device__ __forceinline__ void fence_proxy_async_global() {
 // ---------------------------------------------------------------------------
 // parameters
 // ---------------------------------------------------------------------------
-constexpr int FZ_CONS = 256;                 // consumer threads (warps 0-7)
-constexpr int FZ_PRODUCER_WARP = 8;
-constexpr int FZ_FINISHER_WARP = 9;
+constexpr int FZ_CONS = 512;                 // consumer threads (warps 0-15)
+constexpr int FZ_CWARPS = FZ_CONS / 32;
+constexpr int FZ_PRODUCER_WARP = FZ_CWARPS;
+constexpr int FZ_FINISHER_WARP = FZ_CWARPS + 1;
 constexpr int FZ_THREADS = FZ_CONS + 64;
 constexpr int FZ_NSLOT = 8;                  // ring slots
 constexpr int FZ_SLOT = 16384;               // bytes per slot (64 rows of 256 B)
@@ -100,8 +105,11 @@ constexpr int FZ_NFIN = 8;                   // finisher ring
 constexpr int FZ_NTASK = 16;                 // local task ring
 constexpr int FZ_QBUF = 4096;                // q (bf16) or q' (fp32) of one unit
 constexpr int FZ_ROWS = FUSED_ROWS;          // pages per SCAN item, rows per GATHER item
+constexpr int FZ_CS = FUSED_SCORE;           // candidates per SCORE item
 constexpr int FZ_GROUP = FUSED_GROUP;        // gather chunks per group merge
-constexpr int FZ_WORK = 57344;               // consumer scratch (select, softmax, merges)
+constexpr int FZ_WORK = 83200;               // consumer scratch
+constexpr int FZ_HIST_OFF = 73728;           // score histogram: zero between SCORE items, used by nothing else
+constexpr int FZ_HIST_BINS = 2052;           // >= 8 heads x 256 bits + 1
 constexpr long long FZ_WAIT_CYCLES = 4000000000ll;  // ~2 s at 1.9 GHz
 
 constexpr size_t FZ_OFF_RING = 0;
@@ -113,9 +121,11 @@ constexpr size_t FZ_OFF_TASK = FZ_OFF_FINQ + FZ_NFIN * 32;
 constexpr size_t FZ_OFF_BAR = FZ_OFF_TASK + FZ_NTASK * 16;
 constexpr size_t FZ_OFF_MISC = FZ_OFF_BAR + 8 * (2 * FZ_NSLOT + 2 * FZ_NDESC + 2 * FZ_NFIN);
 constexpr size_t FZ_SMEM = FZ_OFF_MISC + 256;
+static_assert(FZ_SMEM <= 232448, "shared memory of the fused kernel");
+static_assert(FZ_HIST_OFF + 4 * FZ_HIST_BINS <= FZ_WORK, "score histogram");
 
-enum : int { IT_PREP = 0, IT_SCAN = 1, IT_SELECT = 2, IT_GATHER = 3, IT_GMERGE = 4, IT_MERGE = 5, IT_END = 6 };
-// (SELECT, GMERGE and MERGE are local tasks, never queue items)
+enum : int { IT_PREP = 0, IT_SCAN = 1, IT_SCORE = 2, IT_GATHER = 3, IT_END = 4 };
+enum : int { TK_PSEL = 10, TK_KSEL = 11, TK_GMERGE = 12, TK_MERGE = 13 };
 
 struct __align__(16) FzDesc {
   int kind, unit, chunk, n;
@@ -138,10 +148,13 @@ struct __align__(16) FzTask {
 // per-unit control words (kept at zero between calls; the last CTA resets them)
 enum : int {
   CU_PREP = 0,    // q' published
-  CU_SEL = 2,     // kept rows published (sel_keys, n_keys)
-  CU_SCAN = 3,    // scan chunks finished + query codes finished
+  CU_CODES = 1,   // query codes published
+  CU_SEL = 2,     // kept rows published (sel_keys, CU_NKEYS)
+  CU_SCAN = 3,    // scan chunks finished
   CU_MERGED = 4,  // groups merged
   CU_NKEYS = 5,   // kept rows
+  CU_PSEL = 6,    // kept pages published
+  CU_SCORE = 7,   // score chunks finished
   CU_STRIDE = 8
 };
 
@@ -165,6 +178,7 @@ struct FzParams {
   hhr_debug dbg;
   int* status;
   int items_per_unit_scan;    // C1 (sparse) or 0 (dense)
+  int items_per_unit_score;   // C2 (sparse) or 0 (dense)
   int items_per_unit_gather;  // C3
   int total_items;
 };
@@ -183,7 +197,8 @@ struct FzShared {
   uint64_t* ffull;
   uint64_t* fempty;
   int* misc;  // [0] abort, [1] consumed slots, [2] tasks posted, [3] tasks taken,
-              // [4] armed slots, [5] finisher requests done, [6] consumers finished
+              // [4] armed slots, [5] finisher requests done, [6] consumers finished,
+              // [16..23] consumer broadcasts
 };
 
 __device__ __forceinline__ FzShared fz_shared(unsigned char* base) {
@@ -207,8 +222,8 @@ __device__ __forceinline__ FzShared fz_shared(unsigned char* base) {
 
 __device__ __forceinline__ volatile int* abort_flag(const FzShared& s) { return s.misc; }
 
-// barrier among the 256 consumer threads only
-__device__ __forceinline__ void cons_sync() { asm volatile("bar.sync 1, 256;" ::: "memory"); }
+// barrier among the consumer threads only
+__device__ __forceinline__ void cons_sync() { asm volatile("bar.sync 1, %0;" ::"n"(FZ_CONS) : "memory"); }
 
 // Bounded wait on an mbarrier phase; false (and the abort flag) on expiry.
 __device__ __forceinline__ bool fz_wait(const FzShared& s, uint64_t* bar, uint32_t parity, int* status) {
@@ -263,6 +278,15 @@ __device__ __forceinline__ Unit unit_of(const FzParams& p, int u) {
   return x;
 }
 
+// kept pages N of a unit: n_keep clamped to [1, Nmax] and to the page count
+__device__ __forceinline__ int keep_pages(const FzParams& p, const Unit& x) {
+  if (x.np == 0) return 0;
+  return min(min(max(__ldg(p.n_keep + x.b), 1), p.wk.Nmax), x.np);
+}
+__device__ __forceinline__ int score_items(const FzParams& p, const Unit& x) {
+  return (keep_pages(p, x) * p.dm.P + FZ_CS - 1) / FZ_CS;
+}
+
 __device__ __forceinline__ unsigned* unit_ctrl(const FzParams& p, int u) { return p.wk.ctrl + 4 + u * CU_STRIDE; }
 __device__ __forceinline__ unsigned* group_ctrl(const FzParams& p, int u, int g) {
   return p.wk.ctrl + 4 + p.dm.B * p.dm.Hkv * CU_STRIDE + u * p.wk.max_groups + g;
@@ -280,30 +304,38 @@ __device__ __forceinline__ void decode_item(const FzParams& p, int item, int& ki
     return;
   }
   item -= U;
-  if (item < U * p.items_per_unit_scan) {
-    kind = IT_SCAN;
-    u = item / p.items_per_unit_scan;
-    c = item - u * p.items_per_unit_scan;
-    return;
-  }
-  item -= U * p.items_per_unit_scan;
-  if (item < U * p.items_per_unit_gather) {
-    kind = IT_GATHER;
-    u = item / p.items_per_unit_gather;
-    c = item - u * p.items_per_unit_gather;
-    return;
+  const int per[3] = {p.items_per_unit_scan, p.items_per_unit_score, p.items_per_unit_gather};
+  const int kinds[3] = {IT_SCAN, IT_SCORE, IT_GATHER};
+#pragma unroll
+  for (int k = 0; k < 3; ++k) {
+    if (item < U * per[k]) {
+      kind = kinds[k];
+      u = item / per[k];
+      c = item - u * per[k];
+      return;
+    }
+    item -= U * per[k];
   }
   kind = IT_END;
 }
 
+// Zeroes `bytes` (a multiple of 16) of shared memory: the stand-in for a row
+// whose block id is outside the pool (the status word records the error).
+__device__ __forceinline__ void zero_row(unsigned char* dst, int bytes) {
+  for (int e = 0; e < bytes; e += 16) *reinterpret_cast<uint4*>(dst + e) = make_uint4(0u, 0u, 0u, 0u);
+}
+
 // ---------------------------------------------------------------------------
-// producer (warp 8): claims items and fills slots
+// producer (warp 16): claims items and fills slots
 // ---------------------------------------------------------------------------
 template <int G, int WORDS, bool DENSE>
 __device__ void fz_producer(const FzParams& p, const FzShared& s) {
   const int lane = threadIdx.x & 31;
   const Dims& dm = p.dm;
   const int prep_slots = DENSE ? 4 : 4 + dm.nb / 64;  // R_h, then W_h (not needed without hashing)
+  const int page_bytes = dm.P * WORDS * 8;            // codes of one page
+  const int pps = FZ_SLOT / page_bytes;               // pages per slot
+  constexpr int score_slots = (FZ_CS * WORDS * 8 + FZ_SLOT - 1) / FZ_SLOT;
   unsigned nslot = 0, ndesc = 0, armed = 0;
   while (true) {
     int item = 0;
@@ -317,6 +349,15 @@ __device__ void fz_producer(const FzParams& p, const FzShared& s) {
     if (kind == IT_SCAN) {
       n = min(FZ_ROWS, x.np - c * FZ_ROWS);
       if (n <= 0) continue;
+    } else if (kind == IT_SCORE) {
+      n = min(FZ_CS, keep_pages(p, x) * dm.P - c * FZ_CS);
+      if (n <= 0) continue;
+      bool ok = true;
+      if (lane == 0)
+        ok = fz_wait_count(s, unit_ctrl(p, u) + CU_PSEL, 1u, p.status) &&
+             fz_wait_count(s, unit_ctrl(p, u) + CU_CODES, 1u, p.status);
+      if (__shfl_sync(0xffffffffu, (int)ok, 0) == 0) break;
+      (void)ld_acquire(unit_ctrl(p, u) + CU_PSEL);  // every lane reads the kept pages
     } else if (kind == IT_GATHER) {
       bool ok = true;
       if (lane == 0) ok = fz_wait_count(s, unit_ctrl(p, u) + CU_SEL, 1u, p.status);
@@ -334,7 +375,9 @@ __device__ void fz_producer(const FzParams& p, const FzShared& s) {
       if (lane == 0) ok = fz_wait(s, &s.dempty[d], ((ndesc / FZ_NDESC) - 1) & 1, p.status);
       if (__shfl_sync(0xffffffffu, (int)ok, 0) == 0) break;
     }
-    const int nslots = kind == IT_PREP ? prep_slots : ((kind == IT_SCAN || kind == IT_GATHER) ? 4 : 0);
+    const int nslots = kind == IT_PREP ? prep_slots
+                       : (kind == IT_SCAN || kind == IT_GATHER) ? 4
+                       : kind == IT_SCORE ? score_slots : 0;
     // the unit's q or q' goes to the descriptor's q buffer, completing on the first slot
     uint32_t qbytes = 0;
     const void* qsrc = nullptr;
@@ -378,6 +421,7 @@ __device__ void fz_producer(const FzParams& p, const FzShared& s) {
       // warp's byte total (the phase cannot complete before that arrival,
       // whichever order the copies land in).
       uint32_t mine = 0;
+      bool plain = false;  // bytes stored by the lanes themselves (seen through lane 0's arrival)
       if (kind == IT_PREP) {
         if (lane == 0) {
           const void* src = (k < 4) ? (const void*)(p.R + (long long)x.h * D * D + (long long)k * 32 * D)
@@ -407,8 +451,36 @@ __device__ void fz_producer(const FzParams& p, const FzShared& s) {
                 mine += 256;
               } else {
                 set_status(p.status, HHR_ERR_BAD_BLOCK);
+                zero_row(dst + j * 256, 256);
+                plain = true;
               }
             }
+          }
+        }
+      } else if (kind == IT_SCORE) {
+        // whole pages of codes, in kept-page order: page j of the item at j * page_bytes
+        const int npg = (n + dm.P - 1) / dm.P;
+        const int pfirst = c * (FZ_CS / dm.P);
+        const int cnt = min(pps, npg - k * pps);
+        for (int jj = lane; jj < cnt; jj += 32) {
+          const int j = k * pps + jj;
+          const int pg = __ldcg(p.wk.sel_pages + (long long)u * p.wk.Nmax + pfirst + j);
+          const long long off = code_row(dm, p.table, x.b, x.h, pg * dm.P, p.status);
+          if (off >= 0) {
+            const uint64_t* src = p.codes + off;
+            if ((reinterpret_cast<uintptr_t>(src) & 15u) == 0) {
+              bulk_g2s(dst + jj * page_bytes, src, (uint32_t)page_bytes, &s.full[slot]);
+              mine += page_bytes;
+            } else {
+              // one code word per row and an odd row count per head: the page
+              // starts 8 bytes off a 16-byte boundary, so it is copied by hand
+              uint64_t* d64 = reinterpret_cast<uint64_t*>(dst + jj * page_bytes);
+              for (int e = 0; e < page_bytes / 8; ++e) d64[e] = __ldg(src + e);
+              plain = true;
+            }
+          } else {
+            zero_row(dst + jj * page_bytes, page_bytes);
+            plain = true;
           }
         }
       } else {  // IT_GATHER
@@ -432,6 +504,9 @@ __device__ void fz_producer(const FzParams& p, const FzShared& s) {
               if (off >= 0) {
                 bulk_g2s(dst + j * 256, base + off, 256, &s.full[slot]);
                 mine += 256;
+              } else {
+                zero_row(dst + j * 256, 256);
+                plain = true;
               }
             }
           }
@@ -443,6 +518,10 @@ __device__ void fz_producer(const FzParams& p, const FzShared& s) {
       }
 #pragma unroll
       for (int o = 16; o >= 1; o >>= 1) mine += __shfl_xor_sync(0xffffffffu, mine, o);
+      if (__any_sync(0xffffffffu, plain)) {
+        asm volatile("fence.proxy.async.shared::cta;" ::: "memory");  // before later bulk copies into the slot
+        __syncwarp();  // the lanes' stores happen before lane 0's arrival
+      }
       if (lane == 0) mbar_arrive_expect_tx(&s.full[slot], mine);
       __syncwarp();
       armed = gs + 1;
@@ -467,7 +546,7 @@ __device__ void fz_producer(const FzParams& p, const FzShared& s) {
 }
 
 // ---------------------------------------------------------------------------
-// finisher (warp 9): gpu-scope fence, the counter increment, task posting
+// finisher (warp 17): gpu-scope fence, the counter increment, task posting
 // ---------------------------------------------------------------------------
 static __device__ void fz_finisher(const FzParams& p, const FzShared& s) {
   const int lane = threadIdx.x & 31;
@@ -540,41 +619,29 @@ __device__ __forceinline__ bool fz_finish(const FzShared& s, unsigned& nfin, uns
 // consumer helpers
 // ---------------------------------------------------------------------------
 
-// One halving round of a transposed butterfly over WIDTH lanes: the lane
+// One halving round of a transposed butterfly over the 32 lanes: the lane
 // keeps the half of its N values selected by bit `o` of its lane index and
 // adds the partner's copy of that half.
-template <int N, int WIDTH>
-__device__ __forceinline__ void halving_round(float* v, int ln, int o) {
-  const bool up = (ln & o) != 0;
+template <int N>
+__device__ __forceinline__ void halving_round(float* v, int lane, int o) {
+  const bool up = (lane & o) != 0;
 #pragma unroll
   for (int i = 0; i < N / 2; ++i) {
     const float send = up ? v[i] : v[i + N / 2];
     const float keep = up ? v[i + N / 2] : v[i];
-    v[i] = keep + __shfl_xor_sync(0xffffffffu, send, o, WIDTH);
+    v[i] = keep + __shfl_xor_sync(0xffffffffu, send, o);
   }
-}
-
-// Sums NV per-lane values over the 16 lanes of a half-warp.  With NV >= 16
-// lane l ends with the sums of values [ (NV/16) l, (NV/16)(l+1) ) in
-// v[0 .. NV/16); with NV < 16 every lane ends with value index
-// l >> (4 - log2 NV) in v[0] (the last rounds are plain butterflies).
-template <int NV>
-__device__ __forceinline__ void half_reduce(float* v, int ln) {
-  if constexpr (NV >= 2) halving_round<NV, 16>(v, ln, 8); else v[0] += __shfl_xor_sync(0xffffffffu, v[0], 8, 16);
-  if constexpr (NV >= 4) halving_round<NV / 2, 16>(v, ln, 4); else v[0] += __shfl_xor_sync(0xffffffffu, v[0], 4, 16);
-  if constexpr (NV >= 8) halving_round<NV / 4, 16>(v, ln, 2); else v[0] += __shfl_xor_sync(0xffffffffu, v[0], 2, 16);
-  if constexpr (NV >= 16) halving_round<NV / 8, 16>(v, ln, 1); else v[0] += __shfl_xor_sync(0xffffffffu, v[0], 1, 16);
 }
 
 // Sums NV (>= 32) per-lane values over the 32 lanes of a warp; lane l ends
 // with the sums of values [ (NV/32) l, (NV/32)(l+1) ) in v[0 .. NV/32).
 template <int NV>
 __device__ __forceinline__ void warp_reduce_t(float* v, int lane) {
-  halving_round<NV, 32>(v, lane, 16);
-  halving_round<NV / 2, 32>(v, lane, 8);
-  halving_round<NV / 4, 32>(v, lane, 4);
-  halving_round<NV / 8, 32>(v, lane, 2);
-  halving_round<NV / 16, 32>(v, lane, 1);
+  halving_round<NV>(v, lane, 16);
+  halving_round<NV / 2>(v, lane, 8);
+  halving_round<NV / 4>(v, lane, 4);
+  halving_round<NV / 8>(v, lane, 2);
+  halving_round<NV / 16>(v, lane, 1);
 }
 
 // Exclusive scan of one int over the consumer threads; `red` holds 33 ints.
@@ -589,7 +656,7 @@ __device__ __forceinline__ int cons_excl_scan(int v, int* red, int* total) {
   if (lane == 31) red[warp] = x;
   cons_sync();
   if (warp == 0) {
-    int t = lane < FZ_CONS / 32 ? red[lane] : 0;
+    int t = lane < FZ_CWARPS ? red[lane] : 0;
 #pragma unroll
     for (int o = 1; o < 32; o <<= 1) {
       const int y = __shfl_up_sync(0xffffffffu, t, o);
@@ -599,14 +666,44 @@ __device__ __forceinline__ int cons_excl_scan(int v, int* red, int* total) {
   }
   cons_sync();
   const int before = (warp > 0 ? red[warp - 1] : 0) + x - v;
-  *total = red[FZ_CONS / 32 - 1];
+  *total = red[FZ_CWARPS - 1];
   cons_sync();
   return before;
 }
 
+// Block-wide min and max of one value per consumer thread (scratch: 32 floats).
+__device__ __forceinline__ void cons_minmax(float& lo, float& hi, float* wr) {
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+#pragma unroll
+  for (int o = 16; o >= 1; o >>= 1) {
+    lo = fminf(lo, __shfl_xor_sync(0xffffffffu, lo, o));
+    hi = fmaxf(hi, __shfl_xor_sync(0xffffffffu, hi, o));
+  }
+  if (lane == 0) {
+    wr[warp * 2 + 0] = lo;
+    wr[warp * 2 + 1] = hi;
+  }
+  cons_sync();
+  lo = wr[0];
+  hi = wr[1];
+#pragma unroll
+  for (int w = 1; w < FZ_CWARPS; ++w) {
+    lo = fminf(lo, wr[w * 2 + 0]);
+    hi = fmaxf(hi, wr[w * 2 + 1]);
+  }
+  cons_sync();
+}
+
+__device__ __forceinline__ float dot4(const float4& a, const float* b) {
+  float r = a.x * b[0];
+  r = fmaf(a.y, b[1], r);
+  r = fmaf(a.z, b[2], r);
+  return fmaf(a.w, b[3], r);
+}
+
 // ---- PREP: q' = R_h q, then the query codes --------------------------------
 template <int G, bool DENSE>
-__device__ void fz_prep(const FzParams& p, const FzShared& s, const Unit& x, int d, int s0, unsigned& nfin) {
+__device__ void fz_prep(const FzParams& p, const FzShared& s, const Unit& x, int d, int s0) {
   constexpr int GP = G <= 4 ? 4 : 8;
   const Dims& dm = p.dm;
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
@@ -623,36 +720,26 @@ __device__ void fz_prep(const FzParams& p, const FzShared& s, const Unit& x, int
     const float4 t = *reinterpret_cast<const float4*>(qf + g * D + 4 * lane);
     qv[g][0] = t.x; qv[g][1] = t.y; qv[g][2] = t.z; qv[g][3] = t.w;
   }
-  // q'_i = sum_j R_h[i][j] q_j: warp w takes rows 16w .. 16w+15 in blocks of
-  // RB rows; the RB x GP partial sums are reduced together (transposed)
-  constexpr int RB = GP == 4 ? 16 : 8;
-  for (int rb = 0; rb < 16; rb += RB) {
-    float v[RB * GP];
+  // q'_i = sum_j R_h[i][j] q_j: warp w takes rows 8w .. 8w+7; the 8 x GP
+  // partial sums are reduced together (transposed)
+  {
+    constexpr int NV = 8 * GP, KP = NV / 32;
+    float v[NV];
 #pragma unroll
-    for (int r = 0; r < RB; ++r) {
-      const int i = warp * 16 + rb + r;
+    for (int r = 0; r < 8; ++r) {
+      const int i = warp * 8 + r;
       const float4 rr = *reinterpret_cast<const float4*>(
           s.ring + (size_t)((s0 + i / 32) % FZ_NSLOT) * FZ_SLOT + (i % 32) * 512 + lane * 16);
 #pragma unroll
-      for (int g = 0; g < GP; ++g) {
-        float a = 0.f;
-        if (g < G) {
-          a = rr.x * qv[g][0];
-          a = fmaf(rr.y, qv[g][1], a);
-          a = fmaf(rr.z, qv[g][2], a);
-          a = fmaf(rr.w, qv[g][3], a);
-        }
-        v[r * GP + g] = a;
-      }
+      for (int g = 0; g < GP; ++g) v[r * GP + g] = (g < G) ? dot4(rr, qv[g]) : 0.f;
     }
-    warp_reduce_t<RB * GP>(v, lane);
-    // lane holds values [2 lane, 2 lane + 2): row (2 lane + e) / GP, head (2 lane + e) % GP
+    warp_reduce_t<NV>(v, lane);
 #pragma unroll
-    for (int e = 0; e < 2; ++e) {
-      const int vi = 2 * lane + e;
+    for (int e = 0; e < KP; ++e) {
+      const int vi = KP * lane + e;
       const int r = vi / GP, g = vi % GP;
       if (g < G) {
-        const int i = warp * 16 + rb + r;
+        const int i = warp * 8 + r;
         const long long idx = ((long long)x.b * dm.Hq + x.h * G + g) * D + i;
         p.wk.qrot[idx] = v[e];
         if (p.dbg.q_rot) p.dbg.q_rot[idx] = v[e];
@@ -667,19 +754,23 @@ __device__ void fz_prep(const FzParams& p, const FzShared& s, const Unit& x, int
   // Query codes: bit j = [ (W_h q)_j > 0 ].  Products of bf16 values are exact
   // in fp32; the 128-term fp32 sum errs by at most 127 * 2^-24 * sum|w q|, so
   // below 2^-14 * sum|w q| the sign is taken from an fp64 recompute.  Warp w
-  // takes bits [w nb/8, (w+1) nb/8) in blocks of NBB bits; after the
+  // takes bits [w nb/16, (w+1) nb/16) in blocks of NBB bits; after the
   // transposed reduction lane l holds (sum, magnitude) of bit l / GP of the
   // block and head l % GP.
   constexpr int NBB = 32 / GP;  // 8 (GP 4) or 4 (GP 8) bits per block
-  const int bits_per_warp = dm.nb / (FZ_CONS / 32);
-  for (int jb = 0; jb < bits_per_warp; jb += NBB) {
+  const int bpw = dm.nb / FZ_CWARPS;
+  for (int jb = 0; jb < bpw; jb += NBB) {
     float v[2 * NBB * GP];  // [bit][head][sum, magnitude]
 #pragma unroll
     for (int bb = 0; bb < NBB; ++bb) {
-      const int j = warp * bits_per_warp + jb + bb;
-      const uint2 wv = *reinterpret_cast<const uint2*>(s.ring + (size_t)((s0 + 4 + j / 64) % FZ_NSLOT) * FZ_SLOT +
-                                                       (j % 64) * 256 + lane * 8);
-      const float w4[4] = {bf_lo(wv.x), bf_hi(wv.x), bf_lo(wv.y), bf_hi(wv.y)};
+      const int j = warp * bpw + jb + bb;
+      const bool live = jb + bb < bpw;
+      float w4[4] = {0.f, 0.f, 0.f, 0.f};
+      if (live) {
+        const uint2 wv = *reinterpret_cast<const uint2*>(s.ring + (size_t)((s0 + 4 + j / 64) % FZ_NSLOT) * FZ_SLOT +
+                                                         (j % 64) * 256 + lane * 8);
+        w4[0] = bf_lo(wv.x); w4[1] = bf_hi(wv.x); w4[2] = bf_lo(wv.y); w4[3] = bf_hi(wv.y);
+      }
 #pragma unroll
       for (int g = 0; g < GP; ++g) {
         float a = 0.f, m = 0.f;
@@ -697,19 +788,21 @@ __device__ void fz_prep(const FzParams& p, const FzShared& s, const Unit& x, int
     }
     warp_reduce_t<2 * NBB * GP>(v, lane);
     const int bb = lane / GP, g = lane % GP;
-    const int j = warp * bits_per_warp + jb + bb;
-    bool bit = v[0] > 0.f;
-    if (g < G && fabsf(v[0]) <= ldexpf(v[1], -14)) {
-      double ad = 0.0;
-      const unsigned char* wrow = s.ring + (size_t)((s0 + 4 + j / 64) % FZ_NSLOT) * FZ_SLOT + (j % 64) * 256;
-      for (int c = 0; c < D; c += 2) {
-        const uint32_t w2 = *reinterpret_cast<const uint32_t*>(wrow + c * 2);
-        ad += (double)bf_lo(w2) * (double)qf[g * D + c];
-        ad += (double)bf_hi(w2) * (double)qf[g * D + c + 1];
+    const int j = warp * bpw + jb + bb;
+    if (g < G && jb + bb < bpw) {
+      bool bit = v[0] > 0.f;
+      if (fabsf(v[0]) <= ldexpf(v[1], -14)) {
+        double ad = 0.0;
+        const unsigned char* wrow = s.ring + (size_t)((s0 + 4 + j / 64) % FZ_NSLOT) * FZ_SLOT + (j % 64) * 256;
+        for (int c = 0; c < D; c += 2) {
+          const uint32_t w2 = *reinterpret_cast<const uint32_t*>(wrow + c * 2);
+          ad += (double)bf_lo(w2) * (double)qf[g * D + c];
+          ad += (double)bf_hi(w2) * (double)qf[g * D + c + 1];
+        }
+        bit = ad > 0.0;
       }
-      bit = ad > 0.0;
+      if (bit) atomicOr(&qc[g * 8 + j / 32], 1u << (j % 32));
     }
-    if (g < G && bit) atomicOr(&qc[g * 8 + j / 32], 1u << (j % 32));
   }
   cons_sync();
   const int w32 = dm.words * 2;
@@ -719,110 +812,101 @@ __device__ void fz_prep(const FzParams& p, const FzShared& s, const Unit& x, int
     reinterpret_cast<uint32_t*>(p.wk.qcodes)[o] = qc[g * 8 + k];
     if (p.dbg.q_codes) reinterpret_cast<uint32_t*>(p.dbg.q_codes)[o] = qc[g * 8 + k];
   }
+  __threadfence();
   cons_sync();
-  // the query codes count like one more scan chunk toward the unit's select
-  const unsigned nscan = (unsigned)((x.np + FZ_ROWS - 1) / FZ_ROWS);
-  fz_finish(s, nfin, unit_ctrl(p, x.u) + CU_SCAN, 1u, x.np > 0 ? nscan + 1u : 0u, IT_SELECT, x.u, 0, p.status);
+  if (tid == 0) st_release(unit_ctrl(p, x.u) + CU_CODES, 1u);
 }
 
 // ---- SCAN: page bounds of one chunk ------------------------------------------
+// ub_g(page) = sum_i max(q'_gi mn_i, q'_gi mx_i) = q'+_g . mx + q'-_g . mn with
+// q'+ = max(q', 0) and q'- = min(q', 0) (the same products, summed); the
+// unit's page score is U = max_g ub_g.  Warp w takes pages 8w .. 8w+7.
 template <int G>
 __device__ void fz_scan(const FzParams& p, const FzShared& s, const Unit& x, int c, int n, int d, int s0) {
   constexpr int GP = G <= 4 ? 4 : 8;
+  constexpr bool SPLIT = G <= 4;          // q'+ and q'- in registers (else q' and a select)
+  constexpr int PB = GP == 4 ? 8 : 4;     // pages per batch
+  constexpr int NBT = 8 / PB;             // batches
+  constexpr int NV = PB * GP;             // 32 partial bounds per lane
   const Dims& dm = p.dm;
-  const int tid = threadIdx.x, hw = tid >> 4, ln = tid & 15;
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
   const float* qs = reinterpret_cast<const float*>(s.qbuf + d * FZ_QBUF);
-  // channels 8 ln .. 8 ln + 7 of each head, as channel pairs.  For G <= 4
-  // the positive and negative parts of q' are kept apart so that the bound
-  // is two packed FMAs per channel pair; for larger groups q' itself is kept
-  // and each channel picks min or max by the sign of q'.
-  constexpr int QS = G <= 4 ? 2 : 1;
-  float2 qh[QS][G][4];
+  float2 qa[G][2], qb[G][2];
 #pragma unroll
   for (int g = 0; g < G; ++g) {
-#pragma unroll
-    for (int k = 0; k < 4; ++k) {
-      const float2 v = *reinterpret_cast<const float2*>(qs + g * D + ln * 8 + 2 * k);
-      if constexpr (QS == 2) {
-        qh[0][g][k] = make_float2(fmaxf(v.x, 0.f), fmaxf(v.y, 0.f));
-        qh[QS - 1][g][k] = make_float2(fminf(v.x, 0.f), fminf(v.y, 0.f));
-      } else {
-        qh[0][g][k] = v;
-      }
+    const float4 t = *reinterpret_cast<const float4*>(qs + g * D + 4 * lane);
+    if constexpr (SPLIT) {
+      qa[g][0] = make_float2(fmaxf(t.x, 0.f), fmaxf(t.y, 0.f));
+      qa[g][1] = make_float2(fmaxf(t.z, 0.f), fmaxf(t.w, 0.f));
+      qb[g][0] = make_float2(fminf(t.x, 0.f), fminf(t.y, 0.f));
+      qb[g][1] = make_float2(fminf(t.z, 0.f), fminf(t.w, 0.f));
+    } else {
+      qa[g][0] = make_float2(t.x, t.y);
+      qa[g][1] = make_float2(t.z, t.w);
     }
   }
-  // Two pages per half-warp step: values [page][head].  After the reduction
-  // lane ln holds value index ln >> HSH, i.e. page pl and head hidx below.
-  constexpr int NV = 2 * GP;
-  constexpr int HSH = GP == 4 ? 1 : 0;
-  const int vi = ln >> HSH;
-  const int pl = vi / GP, hidx = vi % GP;
-#pragma unroll 1
-  for (int r = 0; r < 4; ++r) {
-    float a[NV];
+  // after the reduction lane l holds page l / GP of the batch, head l % GP
+  const int pl = lane / GP, hidx = lane % GP;
 #pragma unroll
-    for (int pp = 0; pp < 2; ++pp) {
-      const int j = hw + 16 * (2 * r + pp);  // page within the chunk
-      const size_t off = (size_t)(j % 64) * 256 + ln * 16;
-      const uint4 mnv = *reinterpret_cast<const uint4*>(s.ring + (size_t)((s0 + j / 64) % FZ_NSLOT) * FZ_SLOT + off);
-      const uint4 mxv = *reinterpret_cast<const uint4*>(s.ring + (size_t)((s0 + 2 + j / 64) % FZ_NSLOT) * FZ_SLOT + off);
-      const uint32_t mw[4] = {mnv.x, mnv.y, mnv.z, mnv.w};
-      const uint32_t xw[4] = {mxv.x, mxv.y, mxv.z, mxv.w};
+  for (int bt = 0; bt < NBT; ++bt) {
+    float v[NV];
+#pragma unroll
+    for (int pp = 0; pp < PB; ++pp) {
+      const int j = warp * 8 + bt * PB + pp;  // page within the chunk
+      const size_t off = (size_t)(j % 64) * 256 + lane * 8;
+      const uint2 mnv = *reinterpret_cast<const uint2*>(s.ring + (size_t)((s0 + j / 64) % FZ_NSLOT) * FZ_SLOT + off);
+      const uint2 mxv = *reinterpret_cast<const uint2*>(s.ring + (size_t)((s0 + 2 + j / 64) % FZ_NSLOT) * FZ_SLOT + off);
+      const float2 mn0 = make_float2(bf_lo(mnv.x), bf_hi(mnv.x)), mn1 = make_float2(bf_lo(mnv.y), bf_hi(mnv.y));
+      const float2 mx0 = make_float2(bf_lo(mxv.x), bf_hi(mxv.x)), mx1 = make_float2(bf_lo(mxv.y), bf_hi(mxv.y));
 #pragma unroll
       for (int g = 0; g < GP; ++g) {
         float sum = 0.f;
         if (g < G) {
-          float2 acc = make_float2(0.f, 0.f);
-#pragma unroll
-          for (int k = 0; k < 4; ++k) {
-            const float2 hi2 = make_float2(bf_lo(xw[k]), bf_hi(xw[k]));
-            const float2 lo2 = make_float2(bf_lo(mw[k]), bf_hi(mw[k]));
-            if constexpr (QS == 2) {
-              acc = __ffma2_rn(qh[0][g][k], hi2, acc);
-              acc = __ffma2_rn(qh[QS - 1][g][k], lo2, acc);
-            } else {
-              const float2 q2 = qh[0][g][k];
-              acc = __ffma2_rn(q2, make_float2(q2.x >= 0.f ? hi2.x : lo2.x, q2.y >= 0.f ? hi2.y : lo2.y), acc);
-            }
+          float2 acc;
+          if constexpr (SPLIT) {
+            acc = __fmul2_rn(qa[g][0], mx0);
+            acc = __ffma2_rn(qb[g][0], mn0, acc);
+            acc = __ffma2_rn(qa[g][1], mx1, acc);
+            acc = __ffma2_rn(qb[g][1], mn1, acc);
+          } else {
+            const float2 q0 = qa[g][0], q1 = qa[g][1];
+            acc = __fmul2_rn(q0, make_float2(q0.x >= 0.f ? mx0.x : mn0.x, q0.y >= 0.f ? mx0.y : mn0.y));
+            acc = __ffma2_rn(q1, make_float2(q1.x >= 0.f ? mx1.x : mn1.x, q1.y >= 0.f ? mx1.y : mn1.y), acc);
           }
           sum = acc.x + acc.y;
         }
-        a[pp * GP + g] = sum;
+        v[pp * GP + g] = sum;
       }
     }
-    half_reduce<NV>(a, ln);
-    // U = max over the real heads of the lane's page (the 8 lanes of that page)
-    float U = hidx < G ? a[0] : -INFINITY;
+    warp_reduce_t<NV>(v, lane);
+    // U = max over the real heads of the lane's page (GP adjacent lanes)
+    float U = hidx < G ? v[0] : -INFINITY;
 #pragma unroll
-    for (int o = 1 << HSH; o < 8; o <<= 1) U = fmaxf(U, __shfl_xor_sync(0xffffffffu, U, o, 16));
-    const int j = hw + 16 * (2 * r + pl);
+    for (int o = 1; o < GP; o <<= 1) U = fmaxf(U, __shfl_xor_sync(0xffffffffu, U, o));
+    const int j = warp * 8 + bt * PB + pl;
     if (j < n) {
       const int pg = c * FZ_ROWS + j;
-      if ((ln & 7) == 0) {
-        p.wk.U[(long long)x.u * dm.np_max + pg] = U;
+      if (hidx == 0) {
+        p.wk.U[(long long)x.u * p.wk.Ustride + pg] = U;
         if (p.dbg.page_U) p.dbg.page_U[(long long)x.u * dm.np_max + pg] = U;
       }
-      if (p.dbg.page_ub && hidx < G && (ln & ((1 << HSH) - 1)) == 0)
-        p.dbg.page_ub[((long long)x.b * dm.Hq + x.h * G + hidx) * dm.np_max + pg] = a[0];
+      if (p.dbg.page_ub && hidx < G)
+        p.dbg.page_ub[((long long)x.b * dm.Hq + x.h * G + hidx) * dm.np_max + pg] = v[0];
     }
   }
 }
 
-// ---- SELECT: page top-N, Hamming scores, key top-k --------------------------
-// Shared scratch of the select (byte offsets into the work area).
-constexpr int SEL_US = 0;                      // float [np + np/32] bounds, later uint16 scores (padded)
-constexpr int SEL_HIST = 33792;                // int [2112]
-constexpr int SEL_SPAGE = SEL_HIST + 8448;     // int [2048] kept pages
-constexpr int SEL_CAND = SEL_SPAGE + 8192;     // int [512] members of the threshold bin
-constexpr int SEL_FLAG = SEL_CAND + 2048;      // u32 [256] bitmap of kept threshold-bin members
-constexpr int SEL_RED = SEL_FLAG + 1024;       // int [48] scan scratch and broadcasts
-constexpr int SEL_CQ = SEL_RED + 192;          // u64 [G * WORDS]
-constexpr int SEL_NBIN = 1024;                 // value bins of the page select
+// ---- PSEL: page top-N (larger bound first, ties to the lower page) ------------
+constexpr int PS_HIST = 0;                // int [2048] value bins
+constexpr int PS_CAND = 8192;             // int [512] members of the threshold bin
+constexpr int PS_CANDV = PS_CAND + 2048;  // float [512] their bounds
+constexpr int PS_FLAG = PS_CANDV + 2048;  // u32 [256] bitmap of kept members
+constexpr int PS_RED = PS_FLAG + 1024;    // int [48] scan scratch and broadcasts
+constexpr int PS_WR = PS_RED + 256;       // float [32] min / max scratch
+constexpr int SEL_NBIN = 2048;
 constexpr int SEL_MAX_CAND = 512;
-
-// padded index: one spare word per 32 so that blocked per-thread ranges read
-// shared memory without bank conflicts
-__device__ __forceinline__ int pad32(int i) { return i + (i >> 5); }
+constexpr int PS_PER = MAX_SELECT_PAGES / FZ_CONS;  // 16 pages per thread
+static_assert(PS_PER == 16, "page select layout");
 
 // Bin of a bound: monotone non-decreasing in the value, so the N-th largest
 // lies in one bin and every larger bin is kept whole.
@@ -831,86 +915,51 @@ __device__ __forceinline__ int value_bin(float v, float lo, float scale) {
   return min(SEL_NBIN - 1, max(0, (int)t));
 }
 
-// Block-wide min and max of one value per consumer thread (scratch: 16 floats).
-__device__ __forceinline__ void cons_minmax(float& lo, float& hi, float* wr) {
-  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
-#pragma unroll
-  for (int o = 16; o >= 1; o >>= 1) {
-    lo = fminf(lo, __shfl_xor_sync(0xffffffffu, lo, o));
-    hi = fmaxf(hi, __shfl_xor_sync(0xffffffffu, hi, o));
-  }
-  if (lane == 0) {
-    wr[warp * 2 + 0] = lo;
-    wr[warp * 2 + 1] = hi;
-  }
-  cons_sync();
-  lo = wr[0];
-  hi = wr[1];
-#pragma unroll
-  for (int w = 1; w < FZ_CONS / 32; ++w) {
-    lo = fminf(lo, wr[w * 2 + 0]);
-    hi = fmaxf(hi, wr[w * 2 + 1]);
-  }
-  cons_sync();
-}
-
-template <int G, int WORDS>
-__device__ void fz_select(const FzParams& p, const FzShared& s, const Unit& x) {
-  const Dims& dm = p.dm;
+static __device__ void fz_psel(const FzParams& p, const FzShared& s, const Unit& x) {
   const Work& wk = p.wk;
-  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
-  float* Us = reinterpret_cast<float*>(s.work + SEL_US);
-  int* hist = reinterpret_cast<int*>(s.work + SEL_HIST);
-  int* spage = reinterpret_cast<int*>(s.work + SEL_SPAGE);
-  int* cand = reinterpret_cast<int*>(s.work + SEL_CAND);
-  unsigned* flag = reinterpret_cast<unsigned*>(s.work + SEL_FLAG);
-  int* red = reinterpret_cast<int*>(s.work + SEL_RED);
+  const int tid = threadIdx.x;
+  int* hist = reinterpret_cast<int*>(s.work + PS_HIST);
+  int* cand = reinterpret_cast<int*>(s.work + PS_CAND);
+  float* candv = reinterpret_cast<float*>(s.work + PS_CANDV);
+  unsigned* flag = reinterpret_cast<unsigned*>(s.work + PS_FLAG);
+  int* red = reinterpret_cast<int*>(s.work + PS_RED);
   int* bc = red + 36;  // broadcasts [0..11]
-  uint64_t* cq = reinterpret_cast<uint64_t*>(s.work + SEL_CQ);
-  float* wr = reinterpret_cast<float*>(hist + 2048);  // 16 floats of min / max scratch
+  float* wr = reinterpret_cast<float*>(s.work + PS_WR);
   const int np = x.np;
-  const int N = min(min(max(__ldg(p.n_keep + x.b), 1), wk.Nmax), np);
+  const int N = keep_pages(p, x);
   int* gsel = wk.sel_pages + (long long)x.u * wk.Nmax;
   int* dsel = p.dbg.sel_pages ? p.dbg.sel_pages + (long long)x.u * wk.Nmax : nullptr;
-
   if (N >= np) {
     for (int i = tid; i < np; i += FZ_CONS) {
-      spage[i] = i;
       gsel[i] = i;
       if (dsel) dsel[i] = i;
     }
-    cons_sync();
   } else {
-    // ---- bounds into shared memory (coalesced, 8 loads in flight per thread) ----
-    const float* Ug = wk.U + (long long)x.u * dm.np_max;
-    float lo = INFINITY, hi = -INFINITY;
-    for (int base = 0; base < np; base += FZ_CONS * 8) {
-      float v[8];
+    // ---- the bounds of pages [16 t, 16 t + 16) into registers ----
+    const float* Ug = wk.U + (long long)x.u * wk.Ustride;
+    const int i0 = tid * PS_PER;
+    float v[PS_PER];
 #pragma unroll
-      for (int r = 0; r < 8; ++r) {
-        const int i = base + r * FZ_CONS + tid;
-        v[r] = i < np ? __ldcg(Ug + i) : 0.f;
-      }
-#pragma unroll
-      for (int r = 0; r < 8; ++r) {
-        const int i = base + r * FZ_CONS + tid;
-        if (i < np) {
-          Us[pad32(i)] = v[r];
-          lo = fminf(lo, v[r]);
-          hi = fmaxf(hi, v[r]);
-        }
-      }
+    for (int k4 = 0; k4 < PS_PER / 4; ++k4) {
+      const float4 t = i0 + 4 * k4 < np ? __ldcg(reinterpret_cast<const float4*>(Ug + i0) + k4)
+                                        : make_float4(0.f, 0.f, 0.f, 0.f);
+      v[4 * k4 + 0] = t.x; v[4 * k4 + 1] = t.y; v[4 * k4 + 2] = t.z; v[4 * k4 + 3] = t.w;
     }
+    const int cnt = max(0, min(PS_PER, np - i0));
+    unsigned member = (1u << cnt) - 1u;
+    float lo = INFINITY, hi = -INFINITY;
+#pragma unroll
+    for (int k = 0; k < PS_PER; ++k)
+      if ((member >> k) & 1u) {
+        lo = fminf(lo, v[k]);
+        hi = fmaxf(hi, v[k]);
+      }
     cons_minmax(lo, hi, wr);
-    // ---- threshold by value bins.  Each thread owns a blocked range of at
-    // most 32 pages; `member` marks pages still undecided, `keep` the kept.
-    // A level bins the members over their value range (bins are monotone in
-    // the value), keeps every bin above the one holding the need-th largest
-    // member and descends into that bin; a small bin is then ranked exactly,
-    // a bin of equal values is taken in index order. ----
-    const int kpt = (np + FZ_CONS - 1) / FZ_CONS;
-    const int i0 = min(np, tid * kpt), cnt = min(np, i0 + kpt) - i0;
-    unsigned member = cnt >= 32 ? 0xffffffffu : ((1u << cnt) - 1u);
+    // ---- threshold by value bins.  `member` marks pages still undecided,
+    // `keep` the kept.  A level bins the members over their value range,
+    // keeps every bin above the one holding the need-th largest member and
+    // descends into that bin; a small bin is then ranked exactly, a bin of
+    // equal values is taken in index order. ----
     unsigned keep = 0u;
     int need = N, nbin = 0;
     bool tie = false;
@@ -921,28 +970,31 @@ __device__ void fz_select(const FzParams& p, const FzShared& s, const Unit& x) {
       const float scale = (float)SEL_NBIN / (hi - lo);
       for (int i = tid; i < SEL_NBIN; i += FZ_CONS) hist[i] = 0;
       cons_sync();
-      for (int k = 0; k < cnt; ++k)
-        if ((member >> k) & 1u) atomicAdd(&hist[value_bin(Us[pad32(i0 + k)], lo, scale)], 1);
+#pragma unroll
+      for (int k = 0; k < PS_PER; ++k)
+        if ((member >> k) & 1u) atomicAdd(&hist[value_bin(v[k], lo, scale)], 1);
       cons_sync();
       {
         constexpr int BPT = SEL_NBIN / FZ_CONS;  // 4 bins per thread, counted from the top
+        int hv[BPT];
         int c4 = 0;
 #pragma unroll
-        for (int e = 0; e < BPT; ++e) c4 += hist[SEL_NBIN - 1 - (tid * BPT + e)];
+        for (int e = 0; e < BPT; ++e) {
+          hv[e] = hist[SEL_NBIN - 1 - (tid * BPT + e)];
+          c4 += hv[e];
+        }
         int tot;
         const int before = cons_excl_scan(c4, red, &tot);
         if (before < need && before + c4 >= need) {
           int run = before;
 #pragma unroll
           for (int e = 0; e < BPT; ++e) {
-            const int bi = SEL_NBIN - 1 - (tid * BPT + e);
-            if (run + hist[bi] >= need) {
-              bc[0] = bi;
+            if (run < need && run + hv[e] >= need) {
+              bc[0] = SEL_NBIN - 1 - (tid * BPT + e);
               bc[1] = need - run;
-              bc[2] = hist[bi];
-              break;
+              bc[2] = hv[e];
             }
-            run += hist[bi];
+            run += hv[e];
           }
         }
         cons_sync();
@@ -951,18 +1003,18 @@ __device__ void fz_select(const FzParams& p, const FzShared& s, const Unit& x) {
       need = bc[1];
       nbin = bc[2];
       float nlo = INFINITY, nhi = -INFINITY;
-      for (int k = 0; k < cnt; ++k) {
+#pragma unroll
+      for (int k = 0; k < PS_PER; ++k) {
         if (!((member >> k) & 1u)) continue;
-        const float v = Us[pad32(i0 + k)];
-        const int bn = value_bin(v, lo, scale);
+        const int bn = value_bin(v[k], lo, scale);
         if (bn > bstar) {
           keep |= 1u << k;
           member &= ~(1u << k);
         } else if (bn < bstar) {
           member &= ~(1u << k);
         } else {
-          nlo = fminf(nlo, v);
-          nhi = fmaxf(nhi, v);
+          nlo = fminf(nlo, v[k]);
+          nhi = fmaxf(nhi, v[k]);
         }
       }
       if (nbin <= SEL_MAX_CAND) break;
@@ -972,12 +1024,13 @@ __device__ void fz_select(const FzParams& p, const FzShared& s, const Unit& x) {
     }
     if (tie || nbin > SEL_MAX_CAND) {
       // equal values (or still crowded): members in index order, the first `need`
-      int m = __popc(member);
+      const int m = __popc(member);
       int tot;
       const int mb = cons_excl_scan(m, red, &tot);
       int take = max(0, min(m, need - mb));
-      for (int k = 0; k < cnt && take > 0; ++k) {
-        if ((member >> k) & 1u) {
+#pragma unroll
+      for (int k = 0; k < PS_PER; ++k) {
+        if (((member >> k) & 1u) && take > 0) {
           keep |= 1u << k;
           --take;
         }
@@ -985,168 +1038,213 @@ __device__ void fz_select(const FzParams& p, const FzShared& s, const Unit& x) {
     } else {
       // exact ranking of the (few) members: larger value first, then lower index
       if (tid == 0) bc[4] = 0;
-      for (int i = tid; i < (np + 31) / 32; i += FZ_CONS) flag[i] = 0u;
+      if (tid < MAX_SELECT_PAGES / 32) flag[tid] = 0u;
       cons_sync();
-      for (int k = 0; k < cnt; ++k)
-        if ((member >> k) & 1u) cand[atomicAdd(&bc[4], 1)] = i0 + k;
+#pragma unroll
+      for (int k = 0; k < PS_PER; ++k)
+        if ((member >> k) & 1u) {
+          const int at = atomicAdd(&bc[4], 1);
+          cand[at] = i0 + k;
+          candv[at] = v[k];
+        }
       cons_sync();
       for (int a = tid; a < nbin; a += FZ_CONS) {
         const int ia = cand[a];
-        const float va = Us[pad32(ia)];
+        const float va = candv[a];
         int rank = 0;
         for (int b2 = 0; b2 < nbin; ++b2) {
           const int ib = cand[b2];
-          const float vb = Us[pad32(ib)];
+          const float vb = candv[b2];
           rank += (vb > va) || (vb == va && ib < ia);
         }
         if (rank < need) atomicOr(&flag[ia >> 5], 1u << (ia & 31));
       }
       cons_sync();
-      for (int k = 0; k < cnt; ++k) {
-        const int i = i0 + k;
-        if (((member >> k) & 1u) && ((flag[i >> 5] >> (i & 31)) & 1u)) keep |= 1u << k;
-      }
+      const unsigned fw = flag[i0 >> 5] >> (i0 & 31);  // the thread's 16 pages share one flag word
+      keep |= member & fw & 0xffffu;
     }
     // ---- kept pages in index order ----
     int tot;
     int pos = cons_excl_scan(__popc(keep), red, &tot);
-    for (int k = 0; k < cnt; ++k) {
+#pragma unroll
+    for (int k = 0; k < PS_PER; ++k) {
       if ((keep >> k) & 1u) {
-        const int i = i0 + k;
-        spage[pos] = i;
-        gsel[pos] = i;
-        if (dsel) dsel[pos] = i;
+        gsel[pos] = i0 + k;
+        if (dsel) dsel[pos] = i0 + k;
         ++pos;
       }
     }
-    cons_sync();
   }
   if (tid == 0 && p.dbg.n_sel_pages) p.dbg.n_sel_pages[x.u] = N;
-  // ---- Hamming scores of the kept pages' rows (candidate ci = round * 256 + tid) ----
-  const int nbins = G * dm.nb + 1;
-  for (int i = tid; i < nbins; i += FZ_CONS) hist[i] = 0;
-  if (tid < G * WORDS) cq[tid] = __ldcg(wk.qcodes + ((long long)x.b * dm.Hq + x.h * G) * WORDS + tid);
-  cons_sync();
-  unsigned short* sc = reinterpret_cast<unsigned short*>(s.work + SEL_US);
-  const int ncs = N * dm.P;
+}
+
+// ---- SCORE: Hamming scores of one chunk of candidates ------------------------
+// S = sum over the group's heads g of popcount(code(q_g) XOR code(k)); the
+// chunk's scores go to kscore (uint16, 0xFFFF for rows past the sequence end)
+// and their histogram is added to the unit's global histogram.
+template <int G, int WORDS>
+__device__ void fz_score(const FzParams& p, const FzShared& s, const Unit& x, int c, int n, int s0) {
+  const Dims& dm = p.dm;
+  const Work& wk = p.wk;
+  const int tid = threadIdx.x;
+  int* hist = reinterpret_cast<int*>(s.work + FZ_HIST_OFF);
+  (void)ld_acquire(unit_ctrl(p, x.u) + CU_CODES);
+  uint64_t cq[G][WORDS];
+#pragma unroll
+  for (int g = 0; g < G; ++g)
+#pragma unroll
+    for (int w2 = 0; w2 < WORDS; ++w2) cq[g][w2] = __ldcg(wk.qcodes + ((long long)x.b * dm.Hq + x.h * G + g) * WORDS + w2);
+  (void)ld_acquire(unit_ctrl(p, x.u) + CU_PSEL);
+  const int pfirst = c * (FZ_CS / dm.P);
+  const int* gsel = wk.sel_pages + (long long)x.u * wk.Nmax;
   int* dsc = p.dbg.key_scores ? p.dbg.key_scores + (long long)x.u * wk.Nmax * dm.P : nullptr;
-  constexpr int RB = WORDS >= 4 ? 4 : 8;  // rows per thread in flight
-  for (int base = 0; base < ncs; base += FZ_CONS * RB) {
-    uint64_t cw[RB][WORDS];
-    bool valid[RB];
+  uint16_t* ks = wk.kscore + (long long)x.u * wk.Cmax;
+  constexpr int CPS = FZ_SLOT / (WORDS * 8);  // candidates per slot
 #pragma unroll
-    for (int r = 0; r < RB; ++r) {
-      const int ci = base + r * FZ_CONS + tid;
-      valid[r] = false;
+  for (int r = 0; r < FZ_CS / FZ_CONS; ++r) {
+    const int j = r * FZ_CONS + tid;
+    if (j < n) {
+      const unsigned char* src = s.ring + (size_t)((s0 + j / CPS) % FZ_NSLOT) * FZ_SLOT + (size_t)(j % CPS) * WORDS * 8;
+      uint64_t cw[WORDS];
+      if constexpr (WORDS == 1) {
+        cw[0] = *reinterpret_cast<const uint64_t*>(src);
+      } else {
 #pragma unroll
-      for (int w2 = 0; w2 < WORDS; ++w2) cw[r][w2] = 0ull;
-      if (ci < ncs) {
-        const int slot = ci / dm.P;
-        const int t = spage[slot] * dm.P + (ci - slot * dm.P);
-        if (t < x.L) {
-          const long long off = code_row(dm, p.table, x.b, x.h, t, p.status);
-          if (off >= 0) {
-            valid[r] = true;
-            if constexpr (WORDS == 1) {
-              cw[r][0] = __ldg(p.codes + off);
-            } else {
-#pragma unroll
-              for (int w2 = 0; w2 < WORDS; w2 += 2) {
-                const ulonglong2 v = __ldg(reinterpret_cast<const ulonglong2*>(p.codes + off + w2));
-                cw[r][w2] = v.x;
-                cw[r][w2 + 1] = v.y;
-              }
-            }
-          }
+        for (int w2 = 0; w2 < WORDS; w2 += 2) {
+          const ulonglong2 t = *reinterpret_cast<const ulonglong2*>(src + w2 * 8);
+          cw[w2] = t.x;
+          cw[w2 + 1] = t.y;
         }
       }
-    }
+      const int pg = __ldcg(gsel + pfirst + j / dm.P);
+      const int t = pg * dm.P + (j % dm.P);
+      const bool valid = t < x.L;
+      int S = 0;
 #pragma unroll
-    for (int r = 0; r < RB; ++r) {
-      const int ci = base + r * FZ_CONS + tid;
-      if (ci < ncs) {
-        int S = 0;
+      for (int g = 0; g < G; ++g)
 #pragma unroll
-        for (int g = 0; g < G; ++g)
-#pragma unroll
-          for (int w2 = 0; w2 < WORDS; ++w2) S += __popcll(cq[g * WORDS + w2] ^ cw[r][w2]);
-        sc[ci] = valid[r] ? (unsigned short)S : (unsigned short)0xFFFFu;
-        if (dsc) dsc[ci] = valid[r] ? S : INT_MAX;
-        if (valid[r]) atomicAdd(&hist[S], 1);
-      }
+        for (int w2 = 0; w2 < WORDS; ++w2) S += __popcll(cq[g][w2] ^ cw[w2]);
+      const int ci = c * FZ_CS + j;
+      ks[ci] = valid ? (uint16_t)S : (uint16_t)0xFFFFu;
+      if (dsc) dsc[ci] = valid ? S : INT_MAX;
+      if (valid) atomicAdd(&hist[S], 1);
     }
   }
   cons_sync();
-  // ---- key top-k: counting select on the score histogram ----
-  const int bpt = (nbins + FZ_CONS - 1) / FZ_CONS;
+  const int nbins = G * dm.nb + 1;
+  int* gh = wk.khist + (long long)x.u * wk.HB;
+  for (int b = tid; b < nbins; b += FZ_CONS) {
+    const int h = hist[b];
+    if (h) {
+      atomicAdd(gh + b, h);
+      hist[b] = 0;
+    }
+  }
+}
+
+// ---- KSEL: key top-k (smaller score first, ties to the lower row) ------------
+constexpr int KS_SPAGE = 0;      // int [2048] kept pages
+constexpr int KS_WCNT = 8192;    // int [32 rounds x 16 warps] packed counts
+constexpr int KS_RED = 8192 + 2048 + 64;
+static_assert(MAX_KEEP_PAGES <= 2048 && MAX_CANDIDATES <= 32 * FZ_CONS, "key select layout");
+
+template <int G>
+__device__ void fz_ksel(const FzParams& p, const FzShared& s, const Unit& x) {
+  const Dims& dm = p.dm;
+  const Work& wk = p.wk;
+  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+  int* spage = reinterpret_cast<int*>(s.work + KS_SPAGE);
+  int* wcnt = reinterpret_cast<int*>(s.work + KS_WCNT);
+  int* red = reinterpret_cast<int*>(s.work + KS_RED);
+  int* bc = red + 36;
+  const int N = keep_pages(p, x);
+  const int ncs = N * dm.P;
+  const int nbins = G * dm.nb + 1;
+  for (int i = tid; i < N; i += FZ_CONS) spage[i] = __ldcg(wk.sel_pages + (long long)x.u * wk.Nmax + i);
+  // ---- histogram (blocked bins per thread) -> threshold T and ties taken ----
+  int* gh = wk.khist + (long long)x.u * wk.HB;
+  const int bpt = (nbins + FZ_CONS - 1) / FZ_CONS;  // <= 5
+  int hv[5];
   int local = 0;
-  for (int e = 0; e < bpt; ++e) {
+#pragma unroll
+  for (int e = 0; e < 5; ++e) {
     const int bi = tid * bpt + e;
-    if (bi < nbins) local += hist[bi];
+    hv[e] = (e < bpt && bi < nbins) ? __ldcg(gh + bi) : 0;
+    local += hv[e];
   }
   int n_cand;
   const int before = cons_excl_scan(local, red, &n_cand);
   const int keff = min(min(max(__ldg(p.top_k + x.b), 1), wk.Kmax), n_cand);
   if (keff > 0 && before < keff && before + local >= keff) {
     int run = before;
-    for (int e = 0; e < bpt; ++e) {
-      const int bi = tid * bpt + e;
-      const int c2 = bi < nbins ? hist[bi] : 0;
-      if (run + c2 >= keff) {
-        bc[2] = bi;
+#pragma unroll
+    for (int e = 0; e < 5; ++e) {
+      if (run < keff && run + hv[e] >= keff) {
+        bc[2] = tid * bpt + e;
         bc[3] = keff - run;
-        break;
       }
-      run += c2;
+      run += hv[e];
     }
+  }
+  // the histogram is kept at zero between calls
+#pragma unroll
+  for (int e = 0; e < 5; ++e) {
+    const int bi = tid * bpt + e;
+    if (e < bpt && bi < nbins && hv[e]) gh[bi] = 0;
   }
   cons_sync();
   if (keff > 0) {
     // Kept rows in candidate order, written coalesced: candidates go in
-    // rounds of 256 (thread t takes candidate round * 256 + t); per round
+    // rounds of 512 (thread t takes candidate round * 512 + t); per round
     // and warp the counts of S < T and S == T are scanned once, then each
     // warp places its rows with ballots.
     const int T = bc[2], need_eq = bc[3];
-    const int rounds = (ncs + FZ_CONS - 1) / FZ_CONS;  // <= 64
-    int* wcnt = reinterpret_cast<int*>(s.work + SEL_CAND);  // [rounds][8] packed (lt << 16 | eq)
+    const int rounds = (ncs + FZ_CONS - 1) / FZ_CONS;  // <= 32
+    const uint16_t* ks = wk.kscore + (long long)x.u * wk.Cmax;
     const unsigned lanemask_lt = (1u << lane) - 1u;
-    for (int r = 0; r < rounds; ++r) {
+    int sv[32];
+#pragma unroll
+    for (int r = 0; r < 32; ++r) {
       const int ci = r * FZ_CONS + tid;
-      const int v = ci < ncs ? sc[ci] : 0xFFFF;
-      const unsigned blt = __ballot_sync(0xffffffffu, v < T);
-      const unsigned beq = __ballot_sync(0xffffffffu, v == T);
-      if (lane == 0) wcnt[r * 8 + warp] = (__popc(blt) << 16) | __popc(beq);
+      sv[r] = (r < rounds && ci < ncs) ? (int)__ldcg(ks + ci) : 0xFFFF;
+    }
+#pragma unroll
+    for (int r = 0; r < 32; ++r) {
+      if (r < rounds) {
+        const unsigned blt = __ballot_sync(0xffffffffu, sv[r] < T);
+        const unsigned beq = __ballot_sync(0xffffffffu, sv[r] == T);
+        if (lane == 0) wcnt[r * FZ_CWARPS + warp] = (__popc(blt) << 16) | __popc(beq);
+      }
     }
     cons_sync();
-    // exclusive scan over the rounds * 8 packed counts (2 per thread)
     {
-      const int n2 = rounds * 8;
-      const int a0 = 2 * tid, a1 = 2 * tid + 1;
-      const int c0 = a0 < n2 ? wcnt[a0] : 0, c1 = a1 < n2 ? wcnt[a1] : 0;
+      const int n2 = rounds * FZ_CWARPS;  // <= 512: one count per thread
+      const int c0 = tid < n2 ? wcnt[tid] : 0;
       int tot;
-      const int bsum = cons_excl_scan(c0 + c1, red, &tot);
-      if (a0 < n2) wcnt[a0] = bsum;
-      if (a1 < n2) wcnt[a1] = bsum + c0;
+      const int bsum = cons_excl_scan(c0, red, &tot);
+      if (tid < n2) wcnt[tid] = bsum;
       cons_sync();
     }
     int* out = wk.sel_keys + (long long)x.u * wk.Kmax;
     int* dout = p.dbg.sel_keys ? p.dbg.sel_keys + (long long)x.u * wk.Kmax : nullptr;
-    for (int r = 0; r < rounds; ++r) {
-      const int ci = r * FZ_CONS + tid;
-      const int v = ci < ncs ? sc[ci] : 0xFFFF;
-      const bool lt = v < T, eq = v == T;
-      const unsigned beq = __ballot_sync(0xffffffffu, eq);
-      const int base2 = wcnt[r * 8 + warp];
-      const int lt_before = base2 >> 16, eq_before = base2 & 0xffff;
-      const int eq_rank = eq_before + __popc(beq & lanemask_lt);
-      const bool take = lt || (eq && eq_rank < need_eq);
-      const unsigned btake = __ballot_sync(0xffffffffu, take);
-      const int pos = lt_before + min(eq_before, need_eq) + __popc(btake & lanemask_lt);
-      if (take) {
-        const int slot = ci / dm.P;
-        const int t = spage[slot] * dm.P + (ci - slot * dm.P);
-        out[pos] = t;
-        if (dout) dout[pos] = t;
+#pragma unroll
+    for (int r = 0; r < 32; ++r) {
+      if (r < rounds) {
+        const int ci = r * FZ_CONS + tid;
+        const bool lt = sv[r] < T, eq = sv[r] == T;
+        const unsigned beq = __ballot_sync(0xffffffffu, eq);
+        const int base2 = wcnt[r * FZ_CWARPS + warp];
+        const int lt_before = base2 >> 16, eq_before = base2 & 0xffff;
+        const int eq_rank = eq_before + __popc(beq & lanemask_lt);
+        const bool take = lt || (eq && eq_rank < need_eq);
+        const unsigned btake = __ballot_sync(0xffffffffu, take);
+        const int pos = lt_before + min(eq_before, need_eq) + __popc(btake & lanemask_lt);
+        if (take) {
+          const int slot = ci / dm.P;
+          const int t = spage[slot] * dm.P + (ci - slot * dm.P);
+          out[pos] = t;
+          if (dout) dout[pos] = t;
+        }
       }
     }
   }
@@ -1158,180 +1256,183 @@ __device__ void fz_select(const FzParams& p, const FzShared& s, const Unit& x) {
 }
 
 // ---- GATHER: softmax attention over one chunk of kept rows ---------------------
-// Writes the chunk's partial (unnormalised output, max and sum of weights per
-// head, in log2 units) to its fixed slot part[u][c].
+// Warp w takes rows 8w .. 8w+7: logits, the warp's max and weights per head,
+// and the weighted V sum of those rows (lane: channels 4l .. 4l+3).  One
+// barrier later the 16 warp partials are combined in warp order into the
+// chunk's partial (unnormalised output, max and sum of weights per head, in
+// log2 units) at its fixed slot part[u][c].
+constexpr int GA_OB = 0;                  // float [16 warps][G][128] warp outputs
+constexpr int GA_PB = 65536;              // float [16 warps][8 rows][GP] weights
+constexpr int GA_MB = GA_PB + 4096;       // float [16][8] warp maxima
+constexpr int GA_LB = GA_MB + 512;        // float [16][8] warp sums
+static_assert(GA_LB + 512 <= FZ_HIST_OFF, "gather scratch");
+
 template <int G>
 __device__ void fz_gather(const FzParams& p, const FzShared& s, const Unit& x, int c, int n, int d, int s0) {
-  constexpr int GP = G <= 4 ? 4 : 8;  // heads padded to a power of two
-  constexpr int CH = GP == 4 ? 8 : 4; // rows per half-warp per pass
-  constexpr int NPASS = FZ_ROWS / (16 * CH);
-  constexpr int NV = CH * GP;         // partial logits per lane
-  constexpr int KPL = NV / 16;        // logits a lane keeps after the reduction
-  constexpr int HS = GP / 2;          // heads per softmax thread (two head slots)
-  constexpr int NKG = FZ_CONS / 64;   // key groups of the V accumulation
-  const int tid = threadIdx.x, hw = tid >> 4, ln = tid & 15, lane = tid & 31, warp = tid >> 5;
-  float* S = reinterpret_cast<float*>(s.work);                  // [128][GP] logits (log2 units)
-  float2* PP = reinterpret_cast<float2*>(s.work + 4096);        // [128][GP] (p, p)
-  float* red = reinterpret_cast<float*>(s.work + 4096 + 8192);  // [8 warps][HS]
-  float2* OR = reinterpret_cast<float2*>(s.work + 16384);       // [NKG][G][64]
+  constexpr int GP = G <= 4 ? 4 : 8;   // heads padded to a power of two
+  constexpr int RB = GP == 4 ? 8 : 4;  // rows per logit batch
+  constexpr int NBT = 8 / RB;          // batches
+  constexpr int NV = RB * GP;          // 32 partial logits per lane per batch
+  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+  float* OB = reinterpret_cast<float*>(s.work + GA_OB);
+  float* PB = reinterpret_cast<float*>(s.work + GA_PB) + warp * 8 * GP;
+  float* MB = reinterpret_cast<float*>(s.work + GA_MB);
+  float* LB = reinterpret_cast<float*>(s.work + GA_LB);
   const float* qs = reinterpret_cast<const float*>(s.qbuf + d * FZ_QBUF);
   const float qscale = p.sm_scale * 1.4426950408889634f;
-  // ---- logits: pass r, half-warp hw takes rows 16 CH r + CH hw + kk; lane owns 8 channels ----
+  // ---- logits; after the reduction lane l holds head l / RB, row l % RB of the batch ----
+  const int gl = lane / RB, rl = lane % RB;
+  float sv[NBT];
   {
-    float2 qv[G][4];
+    float qv[G][4];
 #pragma unroll
-    for (int g = 0; g < G; ++g)
+    for (int g = 0; g < G; ++g) {
+      const float4 t = *reinterpret_cast<const float4*>(qs + g * D + 4 * lane);
+      qv[g][0] = t.x * qscale; qv[g][1] = t.y * qscale; qv[g][2] = t.z * qscale; qv[g][3] = t.w * qscale;
+    }
 #pragma unroll
-      for (int k = 0; k < 4; ++k) {
-        const float2 v = *reinterpret_cast<const float2*>(qs + g * D + ln * 8 + 2 * k);
-        qv[g][k] = make_float2(v.x * qscale, v.y * qscale);
-      }
-#pragma unroll 1
-    for (int pass = 0; pass < NPASS; ++pass) {
-      const int row0 = pass * 16 * CH + CH * hw;
-      float val[NV];
+    for (int bt = 0; bt < NBT; ++bt) {
+      float v[NV];
 #pragma unroll
-      for (int kk = 0; kk < CH; ++kk) {
-        const int j = row0 + kk;
-        const uint4 kv = *reinterpret_cast<const uint4*>(s.ring + (size_t)((s0 + j / 64) % FZ_NSLOT) * FZ_SLOT +
-                                                         (j % 64) * 256 + ln * 16);
-        const uint32_t kw[4] = {kv.x, kv.y, kv.z, kv.w};
+      for (int r = 0; r < RB; ++r) {
+        const int j = warp * 8 + bt * RB + r;
+        const uint2 kv = *reinterpret_cast<const uint2*>(s.ring + (size_t)((s0 + j / 64) % FZ_NSLOT) * FZ_SLOT +
+                                                         (j % 64) * 256 + lane * 8);
+        const float kf[4] = {bf_lo(kv.x), bf_hi(kv.x), bf_lo(kv.y), bf_hi(kv.y)};
 #pragma unroll
         for (int g = 0; g < GP; ++g) {
           float a = 0.f;
           if (g < G) {
-            float2 acc = make_float2(0.f, 0.f);
-#pragma unroll
-            for (int k = 0; k < 4; ++k) acc = __ffma2_rn(qv[g][k], make_float2(bf_lo(kw[k]), bf_hi(kw[k])), acc);
-            a = acc.x + acc.y;
+            a = qv[g][0] * kf[0];
+            a = fmaf(qv[g][1], kf[1], a);
+            a = fmaf(qv[g][2], kf[2], a);
+            a = fmaf(qv[g][3], kf[3], a);
           }
-          val[g * CH + kk] = a;
+          v[g * RB + r] = a;
         }
       }
-      half_reduce<NV>(val, ln);
-      // lane holds values [KPL ln, KPL ln + KPL): head (KPL ln) / CH, rows (KPL ln) % CH + i
+      warp_reduce_t<NV>(v, lane);
+      const int j = warp * 8 + bt * RB + rl;
+      sv[bt] = (gl < G && j < n) ? v[0] : -INFINITY;
+    }
+  }
+  // ---- the warp's max and weights per head (the RB lanes of head gl) ----
+  float m = sv[0];
 #pragma unroll
-      for (int i = 0; i < KPL; ++i) {
-        const int vi = KPL * ln + i;
-        const int g = vi / CH, kk = vi % CH;
-        const int j = row0 + kk;
-        S[j * GP + g] = (j < n) ? val[i] : -INFINITY;
+  for (int bt = 1; bt < NBT; ++bt) m = fmaxf(m, sv[bt]);
+#pragma unroll
+  for (int o = 1; o < RB; o <<= 1) m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, o));
+  float l = 0.f;
+#pragma unroll
+  for (int bt = 0; bt < NBT; ++bt) {
+    const float pv = (sv[bt] == -INFINITY) ? 0.f : exp2f(sv[bt] - m);
+    PB[(bt * RB + rl) * GP + gl] = pv;
+    l += pv;
+  }
+#pragma unroll
+  for (int o = 1; o < RB; o <<= 1) l += __shfl_xor_sync(0xffffffffu, l, o);
+  if (rl == 0 && gl < G) {
+    MB[warp * 8 + gl] = m;
+    LB[warp * 8 + gl] = l;
+  }
+  __syncwarp();
+  // ---- weighted V sum of the warp's rows ----
+  float2 o2[G][2];
+#pragma unroll
+  for (int g = 0; g < G; ++g) o2[g][0] = o2[g][1] = make_float2(0.f, 0.f);
+#pragma unroll
+  for (int r = 0; r < 8; ++r) {
+    const int j = warp * 8 + r;
+    if (j < n) {
+      const uint2 vv = *reinterpret_cast<const uint2*>(s.ring + (size_t)((s0 + 2 + j / 64) % FZ_NSLOT) * FZ_SLOT +
+                                                       (j % 64) * 256 + lane * 8);
+      const float2 v0 = make_float2(bf_lo(vv.x), bf_hi(vv.x)), v1 = make_float2(bf_lo(vv.y), bf_hi(vv.y));
+      float pr[GP];
+#pragma unroll
+      for (int g4 = 0; g4 < GP; g4 += 4) {
+        const float4 t = *reinterpret_cast<const float4*>(PB + r * GP + g4);
+        pr[g4] = t.x; pr[g4 + 1] = t.y; pr[g4 + 2] = t.z; pr[g4 + 3] = t.w;
+      }
+#pragma unroll
+      for (int g = 0; g < G; ++g) {
+        const float2 pp = make_float2(pr[g], pr[g]);
+        o2[g][0] = __ffma2_rn(pp, v0, o2[g][0]);
+        o2[g][1] = __ffma2_rn(pp, v1, o2[g][1]);
       }
     }
   }
+#pragma unroll
+  for (int g = 0; g < G; ++g)
+    *reinterpret_cast<float4*>(OB + (warp * G + g) * D + 4 * lane) =
+        make_float4(o2[g][0].x, o2[g][0].y, o2[g][1].x, o2[g][1].y);
   cons_sync();
-  // ---- chunk max per head, weights, sums ----
-  // thread t: row j = t & 127, head slot gsl = t >> 7; heads gsl + 2e, e < HS
-  const int j = tid & 127, gsl = tid >> 7;
-  float sv[HS];
+  // ---- the chunk's partial: warps combined in order (thread: head g, channels 4 c4 ..) ----
+  if (tid < G * 32) {
+    const int g = warp, c4 = lane;  // warp-uniform head
+    const float mw = MB[(lane & 15) * 8 + g];
+    float M = mw;
 #pragma unroll
-  for (int e = 0; e < HS; ++e) {
-    sv[e] = S[j * GP + gsl + 2 * e];
-    float m = sv[e];
+    for (int o = 1; o < 16; o <<= 1) M = fmaxf(M, __shfl_xor_sync(0xffffffffu, M, o));
+    const float sc = (mw == -INFINITY) ? 0.f : exp2f(mw - M);  // lane l: scale of warp l & 15
+    float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
+    float L = 0.f;
 #pragma unroll
-    for (int o = 16; o >= 1; o >>= 1) m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, o));
-    if (lane == 0) red[warp * HS + e] = m;
-  }
-  cons_sync();
-  float mh[GP];
-#pragma unroll
-  for (int g = 0; g < GP; ++g) {
-    const int sl = g & 1, e = g >> 1;
-    float cm = -INFINITY;
-#pragma unroll
-    for (int w = 0; w < 4; ++w) cm = fmaxf(cm, red[(sl * 4 + w) * HS + e]);
-    mh[g] = cm;
-  }
-  float ps[HS];
-#pragma unroll
-  for (int e = 0; e < HS; ++e) {
-    const int g = gsl + 2 * e;
-    float mg = mh[0];
-#pragma unroll
-    for (int gg = 1; gg < GP; ++gg)
-      if (gg == g) mg = mh[gg];
-    const float pv = (g < G && j < n) ? exp2f(sv[e] - mg) : 0.f;
-    PP[j * GP + g] = make_float2(pv, pv);
-    float t = pv;
-#pragma unroll
-    for (int o = 16; o >= 1; o >>= 1) t += __shfl_xor_sync(0xffffffffu, t, o);
-    ps[e] = t;
-  }
-  cons_sync();  // every thread has read the maxima before red is reused for sums
-  if (lane == 0) {
-#pragma unroll
-    for (int e = 0; e < HS; ++e) red[warp * HS + e] = ps[e];
-  }
-  cons_sync();  // weights and sums complete
-  // ---- V accumulation: channel pair cp of every head, rows of key group kg ----
-  const int cp = tid & 63, kg = tid >> 6;
-  float2 o2[G];
-#pragma unroll
-  for (int g = 0; g < G; ++g) o2[g] = make_float2(0.f, 0.f);
-  constexpr int RPG = FZ_ROWS / NKG;  // rows per key group
-#pragma unroll 4
-  for (int r = 0; r < RPG; ++r) {
-    const int jr = kg * RPG + r;
-    if (jr < n) {
-      const uint32_t vw = *reinterpret_cast<const uint32_t*>(
-          s.ring + (size_t)((s0 + 2 + jr / 64) % FZ_NSLOT) * FZ_SLOT + (jr % 64) * 256 + cp * 4);
-      const float2 v2 = make_float2(bf_lo(vw), bf_hi(vw));
-#pragma unroll
-      for (int g = 0; g < G; ++g) o2[g] = __ffma2_rn(PP[jr * GP + g], v2, o2[g]);
+    for (int w = 0; w < FZ_CWARPS; ++w) {
+      const float scw = __shfl_sync(0xffffffffu, sc, w);
+      const float4 a = *reinterpret_cast<const float4*>(OB + (w * G + g) * D + 4 * c4);
+      acc.x = fmaf(scw, a.x, acc.x);
+      acc.y = fmaf(scw, a.y, acc.y);
+      acc.z = fmaf(scw, a.z, acc.z);
+      acc.w = fmaf(scw, a.w, acc.w);
+      L = fmaf(scw, LB[w * 8 + g], L);
     }
-  }
-#pragma unroll
-  for (int g = 0; g < G; ++g) OR[(kg * G + g) * 64 + cp] = o2[g];
-  cons_sync();
-  // ---- the chunk's partial: key groups summed in order ----
-  const int PS = G * D + 16;  // partial: o[G][D], m at G D, l at G D + 8 (16-byte rows)
-  float* part = p.wk.part + ((long long)x.u * p.wk.C3 + c) * PS;
-  for (int e = tid; e < G * 64; e += FZ_CONS) {
-    const int g = e / 64, c2 = e % 64;
-    float2 a = OR[(0 * G + g) * 64 + c2];
-#pragma unroll
-    for (int k = 1; k < NKG; ++k) {
-      const float2 v = OR[(k * G + g) * 64 + c2];
-      a.x += v.x;
-      a.y += v.y;
+    const int PS = G * D + 16;  // partial: o[G][D], m at G D, l at G D + 8 (16-byte rows)
+    float* part = p.wk.part + ((long long)x.u * p.wk.C3 + c) * PS;
+    *reinterpret_cast<float4*>(part + g * D + 4 * c4) = acc;
+    if (c4 == 0) {
+      part[G * D + g] = M;
+      part[G * D + 8 + g] = L;
     }
-    *reinterpret_cast<float2*>(part + g * D + 2 * c2) = a;
-  }
-  if (tid < G) {
-    const int sl = tid & 1, e = tid >> 1;
-    float cs = 0.f;
-#pragma unroll
-    for (int w = 0; w < 4; ++w) cs += red[(sl * 4 + w) * HS + e];
-    float mt = mh[0];
-#pragma unroll
-    for (int gg = 1; gg < GP; ++gg)
-      if (gg == tid) mt = mh[gg];
-    part[G * D + tid] = mt;
-    part[G * D + 8 + tid] = cs;
   }
 }
 
 // Merges K partials src[0 .. K) (stride G D + 16 floats) in index order:
 // M = max m_k, w_k = 2^(m_k - M), L = sum w_k l_k, O = sum w_k o_k.  With
 // dst, the merged partial (O, M, L) is written there; otherwise out = O / L.
-// K <= 256.  Loads are issued in batches so that a merge costs a few L2
-// round trips, not one per partial.
+// K <= 256.  The output float4s are split over NPART groups of threads, each
+// taking every NPART-th partial (loads issued before the weights are known);
+// the group sums are then added in group order.
 template <int G>
 __device__ void fz_merge(const FzShared& s, const float* src, int K, float* dst, float* out) {
+  constexpr int NOUT = G * 32;  // float4 outputs
+  constexpr int NPART = FZ_CONS / NOUT >= 4 ? 4 : FZ_CONS / NOUT;
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
   const int PS = G * D + 16;
-  float* wsm = reinterpret_cast<float*>(s.work + 32768);  // [256][G] weights, then M[8], L[8]
-  float* MH = wsm + 256 * G;
-  float* LH = MH + 8;
+  float* wsm = reinterpret_cast<float*>(s.work);            // [256][G] weights
+  float* MH = reinterpret_cast<float*>(s.work + 8192);      // [8]
+  float* LH = MH + 8;                                        // [8]
+  float4* psum = reinterpret_cast<float4*>(s.work + 16384);  // [NPART][NOUT]
   cons_sync();  // the work area's previous readers are done
+  const int f = tid % NOUT, part = tid / NOUT;
+  const int g = f >> 5, c4 = f & 31;
+  const bool active = part < NPART;
+  // prefetch the first batch of this thread's partials
+  constexpr int PF = 8;
+  float4 pv[PF];
+#pragma unroll
+  for (int i = 0; i < PF; ++i) {
+    const int k = part + NPART * i;
+    pv[i] = (active && k < K) ? __ldcg(reinterpret_cast<const float4*>(src + (long long)k * PS + g * D) + c4)
+                              : make_float4(0.f, 0.f, 0.f, 0.f);
+  }
   if (warp < G) {
-    const int g = warp;
+    const int gg = warp;
     float mk[8], lk[8];
 #pragma unroll
     for (int i = 0; i < 8; ++i) {
       const int k = lane + 32 * i;
-      mk[i] = (k < K) ? __ldcg(src + (long long)k * PS + G * D + g) : -INFINITY;
-      lk[i] = (k < K) ? __ldcg(src + (long long)k * PS + G * D + 8 + g) : 0.f;
+      mk[i] = (k < K) ? __ldcg(src + (long long)k * PS + G * D + gg) : -INFINITY;
+      lk[i] = (k < K) ? __ldcg(src + (long long)k * PS + G * D + 8 + gg) : 0.f;
     }
     float M = mk[0];
 #pragma unroll
@@ -1343,41 +1444,57 @@ __device__ void fz_merge(const FzShared& s, const float* src, int K, float* dst,
     for (int i = 0; i < 8; ++i) {
       const int k = lane + 32 * i;
       const float w = (mk[i] == -INFINITY) ? 0.f : exp2f(mk[i] - M);
-      if (k < K) wsm[k * G + g] = w;
+      if (k < K) wsm[k * G + gg] = w;
       L = fmaf(lk[i], w, L);
     }
 #pragma unroll
     for (int o = 16; o >= 1; o >>= 1) L += __shfl_xor_sync(0xffffffffu, L, o);
     if (lane == 0) {
-      MH[g] = M;
-      LH[g] = L;
+      MH[gg] = M;
+      LH[gg] = L;
     }
   }
   cons_sync();
-  for (int f = tid; f < 32 * G; f += FZ_CONS) {
-    const int g = f >> 5, c4 = f & 31;
+  if (active) {
     float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
-    for (int k0 = 0; k0 < K; k0 += 8) {
-      float4 v[8];
+    for (int k0 = 0; k0 < K; k0 += NPART * PF) {
+      if (k0 > 0) {
 #pragma unroll
-      for (int i = 0; i < 8; ++i)
-        v[i] = (k0 + i < K) ? __ldcg(reinterpret_cast<const float4*>(src + (long long)(k0 + i) * PS + g * D) + c4)
-                            : make_float4(0.f, 0.f, 0.f, 0.f);
+        for (int i = 0; i < PF; ++i) {
+          const int k = k0 + part + NPART * i;
+          pv[i] = (k < K) ? __ldcg(reinterpret_cast<const float4*>(src + (long long)k * PS + g * D) + c4)
+                          : make_float4(0.f, 0.f, 0.f, 0.f);
+        }
+      }
 #pragma unroll
-      for (int i = 0; i < 8; ++i) {
-        const float w = (k0 + i < K) ? wsm[(k0 + i) * G + g] : 0.f;
-        acc.x = fmaf(v[i].x, w, acc.x);
-        acc.y = fmaf(v[i].y, w, acc.y);
-        acc.z = fmaf(v[i].z, w, acc.z);
-        acc.w = fmaf(v[i].w, w, acc.w);
+      for (int i = 0; i < PF; ++i) {
+        const int k = k0 + part + NPART * i;
+        const float w = (k < K) ? wsm[k * G + g] : 0.f;
+        acc.x = fmaf(pv[i].x, w, acc.x);
+        acc.y = fmaf(pv[i].y, w, acc.y);
+        acc.z = fmaf(pv[i].z, w, acc.z);
+        acc.w = fmaf(pv[i].w, w, acc.w);
       }
     }
+    psum[part * NOUT + f] = acc;
+  }
+  cons_sync();
+  if (tid < NOUT) {
+    float4 a = psum[tid];
+#pragma unroll
+    for (int q = 1; q < NPART; ++q) {
+      const float4 b = psum[q * NOUT + tid];
+      a.x += b.x;
+      a.y += b.y;
+      a.z += b.z;
+      a.w += b.w;
+    }
     if (dst) {
-      *reinterpret_cast<float4*>(dst + g * D + 4 * c4) = acc;
+      *reinterpret_cast<float4*>(dst + g * D + 4 * c4) = a;
     } else {
       const float L = LH[g];
       const float r = L > 0.f ? 1.f / L : 0.f;
-      *reinterpret_cast<float4*>(out + g * D + 4 * c4) = make_float4(acc.x * r, acc.y * r, acc.z * r, acc.w * r);
+      *reinterpret_cast<float4*>(out + g * D + 4 * c4) = make_float4(a.x * r, a.y * r, a.z * r, a.w * r);
     }
   }
   if (dst && tid < G) {
@@ -1387,7 +1504,7 @@ __device__ void fz_merge(const FzShared& s, const float* src, int K, float* dst,
 }
 
 // ---------------------------------------------------------------------------
-// consumer loop (warps 0-7)
+// consumer loop (warps 0-15)
 // ---------------------------------------------------------------------------
 template <int G, int WORDS, bool DENSE>
 __device__ void fz_run_task(const FzParams& p, const FzShared& s, int kind, int u, int arg, unsigned& nfin) {
@@ -1395,29 +1512,31 @@ __device__ void fz_run_task(const FzParams& p, const FzShared& s, int kind, int 
   const int PS = G * D + 16;
   const Unit x = unit_of(p, u);
   // every thread acquires what the counted CTAs wrote before reading it
-  if (kind == IT_SELECT) (void)ld_acquire(unit_ctrl(p, u) + CU_SCAN);
-  else if (kind == IT_GMERGE) (void)ld_acquire(group_ctrl(p, u, arg));
+  if (kind == TK_PSEL) (void)ld_acquire(unit_ctrl(p, u) + CU_SCAN);
+  else if (kind == TK_KSEL) (void)ld_acquire(unit_ctrl(p, u) + CU_SCORE);
+  else if (kind == TK_GMERGE) (void)ld_acquire(group_ctrl(p, u, arg));
   else (void)ld_acquire(unit_ctrl(p, u) + CU_MERGED);
-  if (kind == IT_SELECT) {
+  if (kind == TK_PSEL || kind == TK_KSEL) {
     if constexpr (!DENSE) {
-      fz_select<G, WORDS>(p, s, x);
+      if (kind == TK_PSEL) fz_psel(p, s, x);
+      else fz_ksel<G>(p, s, x);
       __threadfence();
       cons_sync();
-      if (tid == 0) st_release(unit_ctrl(p, u) + CU_SEL, 1u);
+      if (tid == 0) st_release(unit_ctrl(p, u) + (kind == TK_PSEL ? CU_PSEL : CU_SEL), 1u);
     }
     return;
   }
   const unsigned nk = __ldcg(unit_ctrl(p, u) + CU_NKEYS);
   const int nch = nchunks_of(nk);
   const int ngroups = (nch + FZ_GROUP - 1) / FZ_GROUP;
-  if (kind == IT_GMERGE) {
+  if (kind == TK_GMERGE) {
     const int gsize = min(FZ_GROUP, nch - arg * FZ_GROUP);
     const float* src = p.wk.part + ((long long)u * p.wk.C3 + (long long)arg * FZ_GROUP) * PS;
     float* gp = p.wk.gpart + ((long long)u * p.wk.max_groups + arg) * PS;
     fz_merge<G>(s, src, gsize, gp, nullptr);
     cons_sync();
-    fz_finish(s, nfin, unit_ctrl(p, u) + CU_MERGED, 1u, (unsigned)ngroups, IT_MERGE, u, 0, p.status);
-  } else if (kind == IT_MERGE) {
+    fz_finish(s, nfin, unit_ctrl(p, u) + CU_MERGED, 1u, (unsigned)ngroups, TK_MERGE, u, 0, p.status);
+  } else if (kind == TK_MERGE) {
     fz_merge<G>(s, p.wk.gpart + (long long)u * p.wk.max_groups * PS, ngroups, nullptr,
                 p.out + ((long long)x.b * p.dm.Hq + x.h * G) * D);
     cons_sync();
@@ -1512,9 +1631,11 @@ __device__ void fz_consumer(const FzParams& p, const FzShared& s) {
     }
     const Unit x = unit_of(p, ds.unit);
     if (ds.kind == IT_PREP) {
-      fz_prep<G, DENSE>(p, s, x, d, s0, nfin);
+      fz_prep<G, DENSE>(p, s, x, d, s0);
     } else if (ds.kind == IT_SCAN) {
       if constexpr (!DENSE) fz_scan<G>(p, s, x, ds.chunk, ds.n, d, s0);
+    } else if (ds.kind == IT_SCORE) {
+      if constexpr (!DENSE) fz_score<G, WORDS>(p, s, x, ds.chunk, ds.n, s0);
     } else if (ds.kind == IT_GATHER) {
       fz_gather<G>(p, s, x, ds.chunk, ds.n, d, s0);
     }
@@ -1545,13 +1666,17 @@ __device__ void fz_consumer(const FzParams& p, const FzShared& s) {
     } else if (ds.kind == IT_SCAN) {
       cons_sync();
       const unsigned nscan = (unsigned)((x.np + FZ_ROWS - 1) / FZ_ROWS);
-      fz_finish(s, nfin, unit_ctrl(p, x.u) + CU_SCAN, 1u, nscan + 1u, IT_SELECT, x.u, 0, p.status);
+      fz_finish(s, nfin, unit_ctrl(p, x.u) + CU_SCAN, 1u, nscan, TK_PSEL, x.u, 0, p.status);
+    } else if (ds.kind == IT_SCORE) {
+      cons_sync();
+      fz_finish(s, nfin, unit_ctrl(p, x.u) + CU_SCORE, 1u, (unsigned)score_items(p, x), TK_KSEL, x.u, 0,
+                p.status);
     } else if (ds.kind == IT_GATHER) {
       cons_sync();
       const int nch = nchunks_of((unsigned)ds.pad0);
       const int g = ds.chunk / FZ_GROUP;
       const int gsize = min(FZ_GROUP, nch - g * FZ_GROUP);
-      fz_finish(s, nfin, group_ctrl(p, x.u, g), 1u, (unsigned)gsize, IT_GMERGE, x.u, g, p.status);
+      fz_finish(s, nfin, group_ctrl(p, x.u, g), 1u, (unsigned)gsize, TK_GMERGE, x.u, g, p.status);
     }
   }
   if (tid == 0) {
@@ -1569,11 +1694,11 @@ __global__ void __launch_bounds__(FZ_THREADS, 1) hhr_fused_kernel(FzParams p) {
   if (tid == 0) {
     for (int i = 0; i < FZ_NSLOT; ++i) {
       mbar_init(&s.full[i], 1);
-      mbar_init(&s.empty[i], FZ_CONS / 32);
+      mbar_init(&s.empty[i], FZ_CWARPS);
     }
     for (int i = 0; i < FZ_NDESC; ++i) {
       mbar_init(&s.dfull[i], 1);
-      mbar_init(&s.dempty[i], FZ_CONS / 32);
+      mbar_init(&s.dempty[i], FZ_CWARPS);
     }
     for (int i = 0; i < FZ_NFIN; ++i) {
       mbar_init(&s.ffull[i], 1);
@@ -1582,6 +1707,8 @@ __global__ void __launch_bounds__(FZ_THREADS, 1) hhr_fused_kernel(FzParams p) {
     for (int i = 0; i < 8; ++i) s.misc[i] = 0;
     fence_mbar_init();
   }
+  int* hist = reinterpret_cast<int*>(s.work + FZ_HIST_OFF);
+  for (int i = tid; i < FZ_HIST_BINS; i += blockDim.x) hist[i] = 0;
   __syncthreads();
   const int warp = tid >> 5;
   if (warp == FZ_PRODUCER_WARP) {
@@ -1661,8 +1788,9 @@ static FzParams make_params(const DecodeArgs& a, bool dense) {
   prm.status = a.status;
   const int U = a.dm.B * a.dm.Hkv;
   prm.items_per_unit_scan = dense ? 0 : a.wk.C1;
+  prm.items_per_unit_score = dense ? 0 : a.wk.C2;
   prm.items_per_unit_gather = a.wk.C3;
-  prm.total_items = U * (1 + prm.items_per_unit_scan + prm.items_per_unit_gather);
+  prm.total_items = U * (1 + prm.items_per_unit_scan + prm.items_per_unit_score + prm.items_per_unit_gather);
   return prm;
 }
 

@@ -18,6 +18,7 @@ constexpr int MAX_CANDIDATES = 16384;    // kept pages x page size (scores in sh
 constexpr int FUSED_ROWS = 128;          // pages per scan item, rows per gather item
 constexpr int MAX_GRID = 160;            // CTAs of the fused kernel (one per SM)
 constexpr int FUSED_GROUP = 16;          // gather chunks merged together first
+constexpr int FUSED_SCORE = 1024;        // candidate rows per score item
 constexpr int MAX_GATHER_GROUPS = 256;   // groups per unit (final merge width)
 
 struct DecodeArgs {
