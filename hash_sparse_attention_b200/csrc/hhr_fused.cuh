@@ -66,6 +66,15 @@ __device__ __forceinline__ bool mbar_try_wait(uint64_t* bar, uint32_t parity) {
       : "memory");
   return ok != 0;
 }
+__device__ __forceinline__ bool mbar_test_wait(uint64_t* bar, uint32_t parity) {
+  uint32_t ok;
+  asm volatile(
+      "{\n .reg .pred p;\n mbarrier.test_wait.parity.shared::cta.b64 p, [%1], %2;\n selp.u32 %0, 1, 0, p;\n}\n"
+      : "=r"(ok)
+      : "r"(smem_u32(bar)), "r"(parity)
+      : "memory");
+  return ok != 0;
+}
 // 1-D bulk copy global -> shared (16-byte aligned, size a multiple of 16)
 __device__ __forceinline__ void bulk_g2s(void* dst, const void* src, uint32_t bytes, uint64_t* bar) {
   asm volatile("cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];" ::"r"(
@@ -73,6 +82,29 @@ __device__ __forceinline__ void bulk_g2s(void* dst, const void* src, uint32_t by
                "l"(src), "r"(bytes), "r"(smem_u32(bar))
                : "memory");
 }
+// the same for bytes read once: marked first to leave L2 (code, queue words and
+// partials stay resident while the cache streams through)
+__device__ __forceinline__ void bulk_g2s_stream(void* dst, const void* src, uint32_t bytes, uint64_t* bar,
+                                                uint64_t policy) {
+  asm volatile(
+      "cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes.L2::cache_hint [%0], [%1], %2, [%3], %4;" ::"r"(
+          smem_u32(dst)),
+      "l"(src), "r"(bytes), "r"(smem_u32(bar)), "l"(policy)
+      : "memory");
+}
+__device__ __forceinline__ uint64_t evict_first_policy() {
+  uint64_t pol;
+  asm volatile("createpolicy.fractional.L2::evict_first.b64 %0, 1.0;" : "=l"(pol));
+  return pol;
+}
+// 16-byte asynchronous copy global -> shared through L2 only (the rows that
+// consumer threads gather themselves), and its group bookkeeping
+__device__ __forceinline__ void cp_async16(void* dst, const void* src) {
+  asm volatile("cp.async.cg.shared.global [%0], [%1], 16;" ::"r"(smem_u32(dst)), "l"(src) : "memory");
+}
+__device__ __forceinline__ void cp_async_commit() { asm volatile("cp.async.commit_group;" ::: "memory"); }
+template <int N>
+__device__ __forceinline__ void cp_async_wait() { asm volatile("cp.async.wait_group %0;" ::"n"(N) : "memory"); }
 __device__ __forceinline__ void st_release(unsigned* p, unsigned v) {
   asm volatile("st.release.gpu.global.u32 [%0], %1;" ::"l"(p), "r"(v) : "memory");
 }
@@ -107,29 +139,35 @@ constexpr int FZ_QBUF = 4096;                // q (bf16) or q' (fp32) of one uni
 constexpr int FZ_ROWS = FUSED_ROWS;          // pages per SCAN item, rows per GATHER item
 constexpr int FZ_CS = FUSED_SCORE;           // candidates per SCORE item
 constexpr int FZ_GROUP = FUSED_GROUP;        // gather chunks per group merge
-constexpr int FZ_WORK = 83200;               // consumer scratch
-constexpr int FZ_HIST_OFF = 73728;           // score histogram: zero between SCORE items, used by nothing else
+constexpr int FZ_WORK = 74752;               // consumer scratch
+constexpr int FZ_SEQ = 256;                  // sequences whose length, n_keep and top_k sit in shared memory
 constexpr int FZ_HIST_BINS = 2052;           // >= 8 heads x 256 bits + 1
 constexpr long long FZ_WAIT_CYCLES = 4000000000ll;  // ~2 s at 1.9 GHz
 
 constexpr size_t FZ_OFF_RING = 0;
 constexpr size_t FZ_OFF_QBUF = FZ_OFF_RING + (size_t)FZ_NSLOT * FZ_SLOT;
 constexpr size_t FZ_OFF_WORK = FZ_OFF_QBUF + (size_t)FZ_NDESC * FZ_QBUF;
-constexpr size_t FZ_OFF_DESC = FZ_OFF_WORK + FZ_WORK;
+constexpr size_t FZ_OFF_SEQP = FZ_OFF_WORK + FZ_WORK;
+constexpr size_t FZ_OFF_RIDX = FZ_OFF_SEQP + 3 * FZ_SEQ * 4;
+constexpr size_t FZ_OFF_DESC = FZ_OFF_RIDX + FZ_NDESC * FZ_ROWS * 4;
 constexpr size_t FZ_OFF_FINQ = FZ_OFF_DESC + FZ_NDESC * 32;
 constexpr size_t FZ_OFF_TASK = FZ_OFF_FINQ + FZ_NFIN * 32;
 constexpr size_t FZ_OFF_BAR = FZ_OFF_TASK + FZ_NTASK * 16;
 constexpr size_t FZ_OFF_MISC = FZ_OFF_BAR + 8 * (2 * FZ_NSLOT + 2 * FZ_NDESC + 2 * FZ_NFIN);
 constexpr size_t FZ_SMEM = FZ_OFF_MISC + 256;
 static_assert(FZ_SMEM <= 232448, "shared memory of the fused kernel");
-static_assert(FZ_HIST_OFF + 4 * FZ_HIST_BINS <= FZ_WORK, "score histogram");
+static_assert(4 * FZ_HIST_BINS <= FZ_WORK, "score histogram");
 
 enum : int { IT_PREP = 0, IT_SCAN = 1, IT_SCORE = 2, IT_GATHER = 3, IT_END = 4 };
 enum : int { TK_PSEL = 10, TK_KSEL = 11, TK_GMERGE = 12, TK_MERGE = 13 };
 
+// A descriptor with `gather` set names rows that the consumer threads copy
+// themselves (16-byte cp.async): ridx[j] is the 256-byte row number of row j
+// in the item's first tensor and second tensor alike (K' and V, or the page
+// minima and maxima), -1 for a row whose block id is bad.
 struct __align__(16) FzDesc {
   int kind, unit, chunk, n;
-  int nslots, pad0, pad1, pad2;
+  int nslots, pad0, gather, pad2;
 };
 
 // finisher request: after a gpu-scope fence add `value` to `counter`; if the
@@ -196,6 +234,8 @@ struct FzShared {
   uint64_t* dempty;
   uint64_t* ffull;
   uint64_t* fempty;
+  int* seqp;  // [3][FZ_SEQ]: clamped sequence length, n_keep, top_k of the first FZ_SEQ sequences
+  int* ridx;  // [FZ_NDESC][FZ_ROWS]: row numbers of a descriptor (see FzDesc)
   int* misc;  // [0] abort, [1] consumed slots, [2] tasks posted, [3] tasks taken,
               // [4] armed slots, [5] finisher requests done, [6] consumers finished,
               // [16..23] consumer broadcasts
@@ -206,6 +246,8 @@ __device__ __forceinline__ FzShared fz_shared(unsigned char* base) {
   s.ring = base + FZ_OFF_RING;
   s.qbuf = base + FZ_OFF_QBUF;
   s.work = base + FZ_OFF_WORK;
+  s.seqp = reinterpret_cast<int*>(base + FZ_OFF_SEQP);
+  s.ridx = reinterpret_cast<int*>(base + FZ_OFF_RIDX);
   s.desc = reinterpret_cast<FzDesc*>(base + FZ_OFF_DESC);
   s.finq = reinterpret_cast<FzFin*>(base + FZ_OFF_FINQ);
   s.tasks = reinterpret_cast<FzTask*>(base + FZ_OFF_TASK);
@@ -240,15 +282,6 @@ __device__ __forceinline__ bool fz_wait(const FzShared& s, uint64_t* bar, uint32
   }
 }
 
-// Acquires a phase another thread of the CTA has already seen complete (so the
-// slot's bytes are visible to this thread too); bounded like every wait.
-__device__ __forceinline__ void mbar_confirm(uint64_t* bar, uint32_t parity) {
-  const long long t0 = clock64();
-  while (!mbar_try_wait(bar, parity)) {
-    if (clock64() - t0 > FZ_WAIT_CYCLES) break;
-  }
-}
-
 // Bounded wait until a global counter reaches `target` (acquire).
 __device__ __forceinline__ bool fz_wait_count(const FzShared& s, const unsigned* ctr, unsigned target, int* status) {
   if (ld_acquire(ctr) >= target) return true;
@@ -268,23 +301,24 @@ __device__ __forceinline__ bool fz_wait_count(const FzShared& s, const unsigned*
 struct Unit {
   int u, b, h, L, np;
 };
-__device__ __forceinline__ Unit unit_of(const FzParams& p, int u) {
+__device__ __forceinline__ Unit unit_of(const FzParams& p, const FzShared& s, int u) {
   Unit x;
   x.u = u;
   x.b = u / p.dm.Hkv;
   x.h = u - x.b * p.dm.Hkv;
-  x.L = seq_len_of(p.dm, p.seq_lens, x.b);
+  x.L = x.b < FZ_SEQ ? s.seqp[x.b] : seq_len_of(p.dm, p.seq_lens, x.b);
   x.np = (x.L + p.dm.P - 1) / p.dm.P;
   return x;
 }
 
 // kept pages N of a unit: n_keep clamped to [1, Nmax] and to the page count
-__device__ __forceinline__ int keep_pages(const FzParams& p, const Unit& x) {
+__device__ __forceinline__ int keep_pages(const FzParams& p, const FzShared& s, const Unit& x) {
   if (x.np == 0) return 0;
-  return min(min(max(__ldg(p.n_keep + x.b), 1), p.wk.Nmax), x.np);
+  const int nk = x.b < FZ_SEQ ? s.seqp[FZ_SEQ + x.b] : __ldg(p.n_keep + x.b);
+  return min(min(max(nk, 1), p.wk.Nmax), x.np);
 }
-__device__ __forceinline__ int score_items(const FzParams& p, const Unit& x) {
-  return (keep_pages(p, x) * p.dm.P + FZ_CS - 1) / FZ_CS;
+__device__ __forceinline__ int score_items(const FzParams& p, const FzShared& s, const Unit& x) {
+  return (keep_pages(p, s, x) * p.dm.P + FZ_CS - 1) / FZ_CS;
 }
 
 __device__ __forceinline__ unsigned* unit_ctrl(const FzParams& p, int u) { return p.wk.ctrl + 4 + u * CU_STRIDE; }
@@ -319,23 +353,16 @@ __device__ __forceinline__ void decode_item(const FzParams& p, int item, int& ki
   kind = IT_END;
 }
 
-// Zeroes `bytes` (a multiple of 16) of shared memory: the stand-in for a row
-// whose block id is outside the pool (the status word records the error).
-__device__ __forceinline__ void zero_row(unsigned char* dst, int bytes) {
-  for (int e = 0; e < bytes; e += 16) *reinterpret_cast<uint4*>(dst + e) = make_uint4(0u, 0u, 0u, 0u);
-}
-
 // ---------------------------------------------------------------------------
-// producer (warp 16): claims items and fills slots
+// producer (warp 16): claims items, moves contiguous blocks with bulk copies
+// and lists the rows that the consumers gather themselves
 // ---------------------------------------------------------------------------
 template <int G, int WORDS, bool DENSE>
 __device__ void fz_producer(const FzParams& p, const FzShared& s) {
   const int lane = threadIdx.x & 31;
   const Dims& dm = p.dm;
   const int prep_slots = DENSE ? 4 : 4 + dm.nb / 64;  // R_h, then W_h (not needed without hashing)
-  const int page_bytes = dm.P * WORDS * 8;            // codes of one page
-  const int pps = FZ_SLOT / page_bytes;               // pages per slot
-  constexpr int score_slots = (FZ_CS * WORDS * 8 + FZ_SLOT - 1) / FZ_SLOT;
+  const uint64_t ef = evict_first_policy();
   unsigned nslot = 0, ndesc = 0, armed = 0;
   while (true) {
     int item = 0;
@@ -343,14 +370,14 @@ __device__ void fz_producer(const FzParams& p, const FzShared& s) {
     item = __shfl_sync(0xffffffffu, item, 0);
     int kind, u, c;
     decode_item(p, item, kind, u, c);
-    const Unit x = unit_of(p, u);
+    const Unit x = unit_of(p, s, u);
     int n = 0;
     unsigned nk = 0;
     if (kind == IT_SCAN) {
       n = min(FZ_ROWS, x.np - c * FZ_ROWS);
       if (n <= 0) continue;
     } else if (kind == IT_SCORE) {
-      n = min(FZ_CS, keep_pages(p, x) * dm.P - c * FZ_CS);
+      n = min(FZ_CS, keep_pages(p, s, x) * dm.P - c * FZ_CS);
       if (n <= 0) continue;
       bool ok = true;
       if (lane == 0)
@@ -375,9 +402,41 @@ __device__ void fz_producer(const FzParams& p, const FzShared& s) {
       if (lane == 0) ok = fz_wait(s, &s.dempty[d], ((ndesc / FZ_NDESC) - 1) & 1, p.status);
       if (__shfl_sync(0xffffffffu, (int)ok, 0) == 0) break;
     }
-    const int nslots = kind == IT_PREP ? prep_slots
-                       : (kind == IT_SCAN || kind == IT_GATHER) ? 4
-                       : kind == IT_SCORE ? score_slots : 0;
+    // rows at scattered addresses (paged metadata, kept or paged K'/V rows)
+    // are gathered by the consumers: here only their row numbers
+    const bool gather = (kind == IT_SCAN && dm.paged) || (kind == IT_GATHER && !(DENSE && !dm.paged));
+    const int nslots = kind == IT_PREP ? prep_slots : (kind == IT_SCAN || kind == IT_GATHER) ? 4 : 0;
+    int* ridx = s.ridx + d * FZ_ROWS;
+    if (gather) {
+#pragma unroll
+      for (int i = 0; i < FZ_ROWS / 32; ++i) {
+        const int j = lane + 32 * i;
+        if (j < n) {
+          int r = -1;
+          if (kind == IT_SCAN) {
+            const int blk = __ldg(p.table + (long long)x.b * dm.max_blocks + c * FZ_ROWS + j);
+            if ((unsigned)blk < (unsigned)dm.num_blocks) r = blk * dm.Hkv + x.h;
+            else set_status(p.status, HHR_ERR_BAD_BLOCK);
+          } else {
+            const int t = DENSE ? c * FZ_ROWS + j
+                                : __ldcg(p.wk.sel_keys + (long long)u * p.wk.Kmax + (long long)c * FZ_ROWS + j);
+            const long long off = kv_row(dm, p.table, x.b, x.h, t, p.status);
+            if (off >= 0) r = (int)(off / D);
+          }
+          ridx[j] = r;
+        }
+      }
+    } else if (kind == IT_SCORE) {
+      // pages of the item: code word offset, then the page's rows inside the sequence
+      const int npg = (n + dm.P - 1) / dm.P;
+      const int pfirst = c * (FZ_CS / dm.P);
+      for (int jp = lane; jp < npg; jp += 32) {
+        const int pg = __ldcg(p.wk.sel_pages + (long long)u * p.wk.Nmax + pfirst + jp);
+        const long long off = code_row(dm, p.table, x.b, x.h, pg * dm.P, p.status);
+        ridx[jp] = off >= 0 ? (int)off : -1;
+        ridx[FZ_ROWS / 2 + jp] = min(dm.P, x.L - pg * dm.P);
+      }
+    }
     // the unit's q or q' goes to the descriptor's q buffer, completing on the first slot
     uint32_t qbytes = 0;
     const void* qsrc = nullptr;
@@ -395,15 +454,6 @@ __device__ void fz_producer(const FzParams& p, const FzShared& s) {
       qsrc = p.wk.qrot + ((long long)x.b * dm.Hq + x.h * G) * D;
     }
     unsigned char* qdst = s.qbuf + d * FZ_QBUF;
-    // kept-row ids of a sparse gather chunk: lane holds rows lane + 32 i
-    int rid[4] = {0, 0, 0, 0};
-    if (!DENSE && kind == IT_GATHER) {
-#pragma unroll
-      for (int i = 0; i < 4; ++i) {
-        const int jj = lane + 32 * i;
-        if (jj < n) rid[i] = __ldcg(p.wk.sel_keys + (long long)u * p.wk.Kmax + (long long)c * FZ_ROWS + jj);
-      }
-    }
     bool aborted = false;
     for (int k = 0; k < nslots; ++k) {
       const unsigned gs = nslot + k;
@@ -416,117 +466,37 @@ __device__ void fz_producer(const FzParams& p, const FzShared& s) {
           break;
         }
       }
-      unsigned char* dst = s.ring + (size_t)slot * FZ_SLOT;
-      // Each lane issues its own copies; lane 0 then arms the barrier with the
-      // warp's byte total (the phase cannot complete before that arrival,
-      // whichever order the copies land in).
-      uint32_t mine = 0;
-      bool plain = false;  // bytes stored by the lanes themselves (seen through lane 0's arrival)
-      if (kind == IT_PREP) {
-        if (lane == 0) {
+      if (lane == 0) {
+        unsigned char* dst = s.ring + (size_t)slot * FZ_SLOT;
+        uint32_t bytes = 0;
+        if (kind == IT_PREP) {
           const void* src = (k < 4) ? (const void*)(p.R + (long long)x.h * D * D + (long long)k * 32 * D)
                                     : (const void*)(p.W + ((long long)x.h * dm.nb + (long long)(k - 4) * 64) * D);
           bulk_g2s(dst, src, FZ_SLOT, &s.full[slot]);
-          mine += FZ_SLOT;
-        }
-      } else if (kind == IT_SCAN) {
-        const __nv_bfloat16* base = (k < 2) ? p.pmin : p.pmax;
-        const int j0 = (k & 1) * 64;  // first page of this slot within the chunk
-        const int rows = max(0, min(64, n - j0));
-        if (!dm.paged) {
-          if (lane == 0 && rows > 0) {
-            bulk_g2s(dst, base + ((long long)(x.b * dm.Hkv + x.h) * dm.np_max + (long long)c * FZ_ROWS + j0) * D,
-                     rows * 256, &s.full[slot]);
-            mine += rows * 256;
-          }
-        } else {
-#pragma unroll
-          for (int i = 0; i < 2; ++i) {
-            const int j = lane + 32 * i;
-            if (j < rows) {
-              const int pg = c * FZ_ROWS + j0 + j;
-              const int blk = __ldg(p.table + (long long)x.b * dm.max_blocks + pg);
-              if ((unsigned)blk < (unsigned)dm.num_blocks) {
-                bulk_g2s(dst + j * 256, base + ((long long)blk * dm.Hkv + x.h) * D, 256, &s.full[slot]);
-                mine += 256;
-              } else {
-                set_status(p.status, HHR_ERR_BAD_BLOCK);
-                zero_row(dst + j * 256, 256);
-                plain = true;
-              }
-            }
+          bytes = FZ_SLOT;
+        } else if (!gather) {
+          // contiguous rows: page minima / maxima of the scan, or K'/V of dense attention
+          const __nv_bfloat16* base = kind == IT_SCAN ? ((k < 2) ? p.pmin : p.pmax) : ((k < 2) ? p.Kr : p.Vc);
+          const long long rows_per_head = kind == IT_SCAN ? dm.np_max : dm.T;
+          const int j0 = (k & 1) * 64;
+          const int rows = max(0, min(64, n - j0));
+          if (rows > 0) {
+            bulk_g2s_stream(dst, base + ((long long)(x.b * dm.Hkv + x.h) * rows_per_head + (long long)c * FZ_ROWS + j0) * D,
+                            rows * 256, &s.full[slot], ef);
+            bytes = rows * 256;
           }
         }
-      } else if (kind == IT_SCORE) {
-        // whole pages of codes, in kept-page order: page j of the item at j * page_bytes
-        const int npg = (n + dm.P - 1) / dm.P;
-        const int pfirst = c * (FZ_CS / dm.P);
-        const int cnt = min(pps, npg - k * pps);
-        for (int jj = lane; jj < cnt; jj += 32) {
-          const int j = k * pps + jj;
-          const int pg = __ldcg(p.wk.sel_pages + (long long)u * p.wk.Nmax + pfirst + j);
-          const long long off = code_row(dm, p.table, x.b, x.h, pg * dm.P, p.status);
-          if (off >= 0) {
-            const uint64_t* src = p.codes + off;
-            if ((reinterpret_cast<uintptr_t>(src) & 15u) == 0) {
-              bulk_g2s(dst + jj * page_bytes, src, (uint32_t)page_bytes, &s.full[slot]);
-              mine += page_bytes;
-            } else {
-              // one code word per row and an odd row count per head: the page
-              // starts 8 bytes off a 16-byte boundary, so it is copied by hand
-              uint64_t* d64 = reinterpret_cast<uint64_t*>(dst + jj * page_bytes);
-              for (int e = 0; e < page_bytes / 8; ++e) d64[e] = __ldg(src + e);
-              plain = true;
-            }
-          } else {
-            zero_row(dst + jj * page_bytes, page_bytes);
-            plain = true;
-          }
+        if (k == 0 && qbytes) {
+          bulk_g2s(qdst, qsrc, qbytes, &s.full[slot]);
+          bytes += qbytes;
         }
-      } else {  // IT_GATHER
-        const __nv_bfloat16* base = (k < 2) ? p.Kr : p.Vc;
-        const int j0 = (k & 1) * 64;
-        const int rows = max(0, min(64, n - j0));
-        if (DENSE && !dm.paged) {
-          if (lane == 0 && rows > 0) {
-            bulk_g2s(dst, base + ((long long)(x.b * dm.Hkv + x.h) * dm.T + (long long)c * FZ_ROWS + j0) * D,
-                     rows * 256, &s.full[slot]);
-            mine += rows * 256;
-          }
-        } else {
-#pragma unroll
-          for (int i = 0; i < 2; ++i) {
-            const int j = lane + 32 * i;
-            if (j < rows) {
-              // row j0 + j = lane + 32 (2 (k & 1) + i): its id is rid[2 (k & 1) + i]
-              const int t = DENSE ? c * FZ_ROWS + j0 + j : (((k & 1) == 0) ? rid[i] : rid[2 + i]);
-              const long long off = kv_row(dm, p.table, x.b, x.h, t, p.status);
-              if (off >= 0) {
-                bulk_g2s(dst + j * 256, base + off, 256, &s.full[slot]);
-                mine += 256;
-              } else {
-                zero_row(dst + j * 256, 256);
-                plain = true;
-              }
-            }
-          }
-        }
+        mbar_arrive_expect_tx(&s.full[slot], bytes);
       }
-      if (k == 0 && lane == 0 && qbytes) {
-        bulk_g2s(qdst, qsrc, qbytes, &s.full[slot]);
-        mine += qbytes;
-      }
-#pragma unroll
-      for (int o = 16; o >= 1; o >>= 1) mine += __shfl_xor_sync(0xffffffffu, mine, o);
-      if (__any_sync(0xffffffffu, plain)) {
-        asm volatile("fence.proxy.async.shared::cta;" ::: "memory");  // before later bulk copies into the slot
-        __syncwarp();  // the lanes' stores happen before lane 0's arrival
-      }
-      if (lane == 0) mbar_arrive_expect_tx(&s.full[slot], mine);
       __syncwarp();
       armed = gs + 1;
     }
     if (aborted) break;
+    __syncwarp();  // the row lists are written before the descriptor is published
     if (lane == 0) {
       FzDesc& ds = s.desc[d];
       ds.kind = kind;
@@ -535,6 +505,7 @@ __device__ void fz_producer(const FzParams& p, const FzShared& s) {
       ds.n = n;
       ds.nslots = nslots;
       ds.pad0 = (int)nk;  // gather: the unit's kept rows
+      ds.gather = gather ? 1 : 0;
       mbar_arrive(&s.dfull[d]);
     }
     __syncwarp();
@@ -543,6 +514,33 @@ __device__ void fz_producer(const FzParams& p, const FzShared& s) {
     if (kind == IT_END) break;
   }
   if (lane == 0) s.misc[4] = (int)armed;  // slots armed with copies (drained at exit)
+}
+
+// Consumers copy the rows of a gathering descriptor into its slots: warp w
+// takes rows 8w .. 8w+7 (the rows it computes on), two rows per instruction,
+// 16 bytes per lane, from both tensors; a bad row reads as zeros.  One
+// cp.async group per call.
+__device__ __forceinline__ void gather_rows(const FzShared& s, const int* ridx, int n, int sbase,
+                                            const __nv_bfloat16* first, const __nv_bfloat16* second) {
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+  const int q = lane & 15;
+#pragma unroll
+  for (int i = 0; i < 4; ++i) {
+    const int j = warp * 8 + 2 * i + (lane >> 4);
+    if (j < n) {
+      const int r = ridx[j];
+      unsigned char* d1 = s.ring + (size_t)((sbase + j / 64) % FZ_NSLOT) * FZ_SLOT + (j % 64) * 256 + q * 16;
+      unsigned char* d2 = s.ring + (size_t)((sbase + 2 + j / 64) % FZ_NSLOT) * FZ_SLOT + (j % 64) * 256 + q * 16;
+      if (r >= 0) {
+        cp_async16(d1, first + (long long)r * D + q * 8);
+        cp_async16(d2, second + (long long)r * D + q * 8);
+      } else {
+        *reinterpret_cast<uint4*>(d1) = make_uint4(0u, 0u, 0u, 0u);
+        *reinterpret_cast<uint4*>(d2) = make_uint4(0u, 0u, 0u, 0u);
+      }
+    }
+  }
+  cp_async_commit();
 }
 
 // ---------------------------------------------------------------------------
@@ -746,10 +744,13 @@ __device__ void fz_prep(const FzParams& p, const FzShared& s, const Unit& x, int
       }
     }
   }
-  // publish q' now: the scans of this unit need only q'
-  __threadfence();
+  // publish q' now: the scans of this unit need only q'.  (The barrier orders
+  // every consumer's writes before thread 0's gpu-scope fence and release.)
   cons_sync();
-  if (tid == 0) st_release(unit_ctrl(p, x.u) + CU_PREP, 1u);
+  if (tid == 0) {
+    __threadfence();
+    st_release(unit_ctrl(p, x.u) + CU_PREP, 1u);
+  }
   if constexpr (DENSE) return;  // full attention needs no codes (and has no W_h)
   // Query codes: bit j = [ (W_h q)_j > 0 ].  Products of bf16 values are exact
   // in fp32; the 128-term fp32 sum errs by at most 127 * 2^-24 * sum|w q|, so
@@ -812,78 +813,123 @@ __device__ void fz_prep(const FzParams& p, const FzShared& s, const Unit& x, int
     reinterpret_cast<uint32_t*>(p.wk.qcodes)[o] = qc[g * 8 + k];
     if (p.dbg.q_codes) reinterpret_cast<uint32_t*>(p.dbg.q_codes)[o] = qc[g * 8 + k];
   }
-  __threadfence();
   cons_sync();
-  if (tid == 0) st_release(unit_ctrl(p, x.u) + CU_CODES, 1u);
+  if (tid == 0) {
+    __threadfence();
+    st_release(unit_ctrl(p, x.u) + CU_CODES, 1u);
+  }
 }
 
 // ---- SCAN: page bounds of one chunk ------------------------------------------
 // ub_g(page) = sum_i max(q'_gi mn_i, q'_gi mx_i) = q'+_g . mx + q'-_g . mn with
 // q'+ = max(q', 0) and q'- = min(q', 0) (the same products, summed); the
-// unit's page score is U = max_g ub_g.  Warp w takes pages 8w .. 8w+7.
+// unit's page score is U = max_g ub_g.  Warp w takes pages 8w .. 8w+7, half
+// a warp per page (lane: channels 8l .. 8l+7 of the half-warp's pages).
+
+// One halving round of a transposed butterfly among the lanes that differ in
+// bit `o`: the lane keeps the half of its N values selected by that bit and
+// adds the partner's copy of that half.
+template <int N>
+__device__ __forceinline__ void halving_round_o(float* v, int lane, int o) {
+  const bool up = (lane & o) != 0;
+#pragma unroll
+  for (int i = 0; i < N / 2; ++i) {
+    const float send = up ? v[i] : v[i + N / 2];
+    const float keep = up ? v[i + N / 2] : v[i];
+    v[i] = keep + __shfl_xor_sync(0xffffffffu, send, o);
+  }
+}
+// Sums NV per-lane values over groups of W lanes (W = 8 or 16, NV >= W);
+// lane l of a group ends with the sums of values [(NV/W) l, (NV/W)(l+1)).
+template <int NV, int W>
+__device__ __forceinline__ void group_reduce_t(float* v, int lane) {
+  if constexpr (W == 16) halving_round_o<NV>(v, lane, 8);
+  halving_round_o<(W == 16 ? NV / 2 : NV)>(v, lane, 4);
+  halving_round_o<(W == 16 ? NV / 4 : NV / 2)>(v, lane, 2);
+  halving_round_o<(W == 16 ? NV / 8 : NV / 4)>(v, lane, 1);
+}
+
 template <int G>
 __device__ void fz_scan(const FzParams& p, const FzShared& s, const Unit& x, int c, int n, int d, int s0) {
   constexpr int GP = G <= 4 ? 4 : 8;
   constexpr bool SPLIT = G <= 4;          // q'+ and q'- in registers (else q' and a select)
-  constexpr int PB = GP == 4 ? 8 : 4;     // pages per batch
-  constexpr int NBT = 8 / PB;             // batches
-  constexpr int NV = PB * GP;             // 32 partial bounds per lane
+  constexpr int PB = GP == 4 ? 4 : 2;     // pages per half-warp per batch
+  constexpr int NBT = 4 / PB;             // batches (4 pages per half-warp)
+  constexpr int NV = PB * GP;             // 16 partial bounds per lane
   const Dims& dm = p.dm;
   const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+  const int hw = lane >> 4, li = lane & 15;
   const float* qs = reinterpret_cast<const float*>(s.qbuf + d * FZ_QBUF);
-  float2 qa[G][2], qb[G][2];
+  float2 qa[G][4], qb[G][4];
 #pragma unroll
   for (int g = 0; g < G; ++g) {
-    const float4 t = *reinterpret_cast<const float4*>(qs + g * D + 4 * lane);
-    if constexpr (SPLIT) {
-      qa[g][0] = make_float2(fmaxf(t.x, 0.f), fmaxf(t.y, 0.f));
-      qa[g][1] = make_float2(fmaxf(t.z, 0.f), fmaxf(t.w, 0.f));
-      qb[g][0] = make_float2(fminf(t.x, 0.f), fminf(t.y, 0.f));
-      qb[g][1] = make_float2(fminf(t.z, 0.f), fminf(t.w, 0.f));
-    } else {
-      qa[g][0] = make_float2(t.x, t.y);
-      qa[g][1] = make_float2(t.z, t.w);
+#pragma unroll
+    for (int k = 0; k < 2; ++k) {
+      const float4 t = *reinterpret_cast<const float4*>(qs + g * D + 8 * li + 4 * k);
+      if constexpr (SPLIT) {
+        qa[g][2 * k] = make_float2(fmaxf(t.x, 0.f), fmaxf(t.y, 0.f));
+        qa[g][2 * k + 1] = make_float2(fmaxf(t.z, 0.f), fmaxf(t.w, 0.f));
+        qb[g][2 * k] = make_float2(fminf(t.x, 0.f), fminf(t.y, 0.f));
+        qb[g][2 * k + 1] = make_float2(fminf(t.z, 0.f), fminf(t.w, 0.f));
+      } else {
+        qa[g][2 * k] = make_float2(t.x, t.y);
+        qa[g][2 * k + 1] = make_float2(t.z, t.w);
+      }
     }
   }
-  // after the reduction lane l holds page l / GP of the batch, head l % GP
-  const int pl = lane / GP, hidx = lane % GP;
+  // after the reduction lane l of a half-warp holds page l / GP of the batch, head l % GP
+  const int pl = li / GP, hidx = li % GP;
 #pragma unroll
   for (int bt = 0; bt < NBT; ++bt) {
     float v[NV];
 #pragma unroll
     for (int pp = 0; pp < PB; ++pp) {
-      const int j = warp * 8 + bt * PB + pp;  // page within the chunk
-      const size_t off = (size_t)(j % 64) * 256 + lane * 8;
-      const uint2 mnv = *reinterpret_cast<const uint2*>(s.ring + (size_t)((s0 + j / 64) % FZ_NSLOT) * FZ_SLOT + off);
-      const uint2 mxv = *reinterpret_cast<const uint2*>(s.ring + (size_t)((s0 + 2 + j / 64) % FZ_NSLOT) * FZ_SLOT + off);
-      const float2 mn0 = make_float2(bf_lo(mnv.x), bf_hi(mnv.x)), mn1 = make_float2(bf_lo(mnv.y), bf_hi(mnv.y));
-      const float2 mx0 = make_float2(bf_lo(mxv.x), bf_hi(mxv.x)), mx1 = make_float2(bf_lo(mxv.y), bf_hi(mxv.y));
+      const int j = warp * 8 + hw * 4 + bt * PB + pp;  // page within the chunk
+      const size_t off = (size_t)(j % 64) * 256 + li * 16;
+      const uint4 mnv = *reinterpret_cast<const uint4*>(s.ring + (size_t)((s0 + j / 64) % FZ_NSLOT) * FZ_SLOT + off);
+      const uint4 mxv = *reinterpret_cast<const uint4*>(s.ring + (size_t)((s0 + 2 + j / 64) % FZ_NSLOT) * FZ_SLOT + off);
+      const uint32_t mw[4] = {mnv.x, mnv.y, mnv.z, mnv.w};
+      const uint32_t xw[4] = {mxv.x, mxv.y, mxv.z, mxv.w};
+      float2 mn[4], mx[4];
+#pragma unroll
+      for (int k = 0; k < 4; ++k) {
+        mn[k] = make_float2(bf_lo(mw[k]), bf_hi(mw[k]));
+        mx[k] = make_float2(bf_lo(xw[k]), bf_hi(xw[k]));
+      }
 #pragma unroll
       for (int g = 0; g < GP; ++g) {
         float sum = 0.f;
         if (g < G) {
-          float2 acc;
+          float2 a0, a1;
           if constexpr (SPLIT) {
-            acc = __fmul2_rn(qa[g][0], mx0);
-            acc = __ffma2_rn(qb[g][0], mn0, acc);
-            acc = __ffma2_rn(qa[g][1], mx1, acc);
-            acc = __ffma2_rn(qb[g][1], mn1, acc);
+            a0 = __fmul2_rn(qa[g][0], mx[0]);
+            a1 = __fmul2_rn(qb[g][0], mn[0]);
+#pragma unroll
+            for (int k = 1; k < 4; ++k) {
+              a0 = __ffma2_rn(qa[g][k], mx[k], a0);
+              a1 = __ffma2_rn(qb[g][k], mn[k], a1);
+            }
           } else {
-            const float2 q0 = qa[g][0], q1 = qa[g][1];
-            acc = __fmul2_rn(q0, make_float2(q0.x >= 0.f ? mx0.x : mn0.x, q0.y >= 0.f ? mx0.y : mn0.y));
-            acc = __ffma2_rn(q1, make_float2(q1.x >= 0.f ? mx1.x : mn1.x, q1.y >= 0.f ? mx1.y : mn1.y), acc);
+            float2 sel[4];
+#pragma unroll
+            for (int k = 0; k < 4; ++k)
+              sel[k] = make_float2(qa[g][k].x >= 0.f ? mx[k].x : mn[k].x, qa[g][k].y >= 0.f ? mx[k].y : mn[k].y);
+            a0 = __fmul2_rn(qa[g][0], sel[0]);
+            a1 = __fmul2_rn(qa[g][1], sel[1]);
+            a0 = __ffma2_rn(qa[g][2], sel[2], a0);
+            a1 = __ffma2_rn(qa[g][3], sel[3], a1);
           }
-          sum = acc.x + acc.y;
+          sum = (a0.x + a0.y) + (a1.x + a1.y);
         }
         v[pp * GP + g] = sum;
       }
     }
-    warp_reduce_t<NV>(v, lane);
+    group_reduce_t<NV, 16>(v, lane);
     // U = max over the real heads of the lane's page (GP adjacent lanes)
     float U = hidx < G ? v[0] : -INFINITY;
 #pragma unroll
     for (int o = 1; o < GP; o <<= 1) U = fmaxf(U, __shfl_xor_sync(0xffffffffu, U, o));
-    const int j = warp * 8 + bt * PB + pl;
+    const int j = warp * 8 + hw * 4 + bt * PB + pl;
     if (j < n) {
       const int pg = c * FZ_ROWS + j;
       if (hidx == 0) {
@@ -926,7 +972,7 @@ static __device__ void fz_psel(const FzParams& p, const FzShared& s, const Unit&
   int* bc = red + 36;  // broadcasts [0..11]
   float* wr = reinterpret_cast<float*>(s.work + PS_WR);
   const int np = x.np;
-  const int N = keep_pages(p, x);
+  const int N = keep_pages(p, s, x);
   int* gsel = wk.sel_pages + (long long)x.u * wk.Nmax;
   int* dsel = p.dbg.sel_pages ? p.dbg.sel_pages + (long long)x.u * wk.Nmax : nullptr;
   if (N >= np) {
@@ -1083,62 +1129,69 @@ static __device__ void fz_psel(const FzParams& p, const FzShared& s, const Unit&
 // chunk's scores go to kscore (uint16, 0xFFFF for rows past the sequence end)
 // and their histogram is added to the unit's global histogram.
 template <int G, int WORDS>
-__device__ void fz_score(const FzParams& p, const FzShared& s, const Unit& x, int c, int n, int s0) {
+__device__ void fz_score(const FzParams& p, const FzShared& s, const Unit& x, int c, int n, int d) {
   const Dims& dm = p.dm;
   const Work& wk = p.wk;
   const int tid = threadIdx.x;
-  int* hist = reinterpret_cast<int*>(s.work + FZ_HIST_OFF);
+  int* hist = reinterpret_cast<int*>(s.work);
+  const int nbins = G * dm.nb + 1;
+  for (int b = tid; b < nbins; b += FZ_CONS) hist[b] = 0;
+  const int* ridx = s.ridx + d * FZ_ROWS;  // per page: code word offset, then rows inside the sequence
+  // the candidates' code words (two per thread), straight from global memory
+  constexpr int NR = FZ_CS / FZ_CONS;
+  uint64_t cw[NR][WORDS];
+  bool valid[NR];
+#pragma unroll
+  for (int r = 0; r < NR; ++r) {
+    const int j = r * FZ_CONS + tid;
+    const int jp = j / dm.P, jr = j - jp * dm.P;
+    const int woff = j < n ? ridx[jp] : -1;
+    valid[r] = woff >= 0 && jr < ridx[FZ_ROWS / 2 + jp];
+#pragma unroll
+    for (int w2 = 0; w2 < WORDS; ++w2) cw[r][w2] = 0ull;
+    if (valid[r]) {
+      const uint64_t* src = p.codes + (long long)woff + (long long)jr * WORDS;
+      if constexpr (WORDS == 1) {
+        cw[r][0] = __ldg(src);
+      } else {
+#pragma unroll
+        for (int w2 = 0; w2 < WORDS; w2 += 2) {
+          const ulonglong2 t = __ldg(reinterpret_cast<const ulonglong2*>(src + w2));
+          cw[r][w2] = t.x;
+          cw[r][w2 + 1] = t.y;
+        }
+      }
+    }
+  }
   (void)ld_acquire(unit_ctrl(p, x.u) + CU_CODES);
   uint64_t cq[G][WORDS];
 #pragma unroll
   for (int g = 0; g < G; ++g)
 #pragma unroll
     for (int w2 = 0; w2 < WORDS; ++w2) cq[g][w2] = __ldcg(wk.qcodes + ((long long)x.b * dm.Hq + x.h * G + g) * WORDS + w2);
-  (void)ld_acquire(unit_ctrl(p, x.u) + CU_PSEL);
-  const int pfirst = c * (FZ_CS / dm.P);
-  const int* gsel = wk.sel_pages + (long long)x.u * wk.Nmax;
+  cons_sync();  // the histogram is zero
   int* dsc = p.dbg.key_scores ? p.dbg.key_scores + (long long)x.u * wk.Nmax * dm.P : nullptr;
   uint16_t* ks = wk.kscore + (long long)x.u * wk.Cmax;
-  constexpr int CPS = FZ_SLOT / (WORDS * 8);  // candidates per slot
 #pragma unroll
-  for (int r = 0; r < FZ_CS / FZ_CONS; ++r) {
+  for (int r = 0; r < NR; ++r) {
     const int j = r * FZ_CONS + tid;
     if (j < n) {
-      const unsigned char* src = s.ring + (size_t)((s0 + j / CPS) % FZ_NSLOT) * FZ_SLOT + (size_t)(j % CPS) * WORDS * 8;
-      uint64_t cw[WORDS];
-      if constexpr (WORDS == 1) {
-        cw[0] = *reinterpret_cast<const uint64_t*>(src);
-      } else {
-#pragma unroll
-        for (int w2 = 0; w2 < WORDS; w2 += 2) {
-          const ulonglong2 t = *reinterpret_cast<const ulonglong2*>(src + w2 * 8);
-          cw[w2] = t.x;
-          cw[w2 + 1] = t.y;
-        }
-      }
-      const int pg = __ldcg(gsel + pfirst + j / dm.P);
-      const int t = pg * dm.P + (j % dm.P);
-      const bool valid = t < x.L;
       int S = 0;
 #pragma unroll
       for (int g = 0; g < G; ++g)
 #pragma unroll
-        for (int w2 = 0; w2 < WORDS; ++w2) S += __popcll(cq[g][w2] ^ cw[w2]);
+        for (int w2 = 0; w2 < WORDS; ++w2) S += __popcll(cq[g][w2] ^ cw[r][w2]);
       const int ci = c * FZ_CS + j;
-      ks[ci] = valid ? (uint16_t)S : (uint16_t)0xFFFFu;
-      if (dsc) dsc[ci] = valid ? S : INT_MAX;
-      if (valid) atomicAdd(&hist[S], 1);
+      ks[ci] = valid[r] ? (uint16_t)S : (uint16_t)0xFFFFu;
+      if (dsc) dsc[ci] = valid[r] ? S : INT_MAX;
+      if (valid[r]) atomicAdd(&hist[S], 1);
     }
   }
   cons_sync();
-  const int nbins = G * dm.nb + 1;
   int* gh = wk.khist + (long long)x.u * wk.HB;
   for (int b = tid; b < nbins; b += FZ_CONS) {
     const int h = hist[b];
-    if (h) {
-      atomicAdd(gh + b, h);
-      hist[b] = 0;
-    }
+    if (h) atomicAdd(gh + b, h);
   }
 }
 
@@ -1146,7 +1199,9 @@ __device__ void fz_score(const FzParams& p, const FzShared& s, const Unit& x, in
 constexpr int KS_SPAGE = 0;      // int [2048] kept pages
 constexpr int KS_WCNT = 8192;    // int [32 rounds x 16 warps] packed counts
 constexpr int KS_RED = 8192 + 2048 + 64;
-static_assert(MAX_KEEP_PAGES <= 2048 && MAX_CANDIDATES <= 32 * FZ_CONS, "key select layout");
+constexpr int KS_SC = 12288;     // uint16 [16384] candidate scores
+static_assert(MAX_KEEP_PAGES <= 2048 && MAX_CANDIDATES <= 32 * FZ_CONS && KS_SC + 2 * MAX_CANDIDATES <= FZ_WORK,
+              "key select layout");
 
 template <int G>
 __device__ void fz_ksel(const FzParams& p, const FzShared& s, const Unit& x) {
@@ -1157,7 +1212,7 @@ __device__ void fz_ksel(const FzParams& p, const FzShared& s, const Unit& x) {
   int* wcnt = reinterpret_cast<int*>(s.work + KS_WCNT);
   int* red = reinterpret_cast<int*>(s.work + KS_RED);
   int* bc = red + 36;
-  const int N = keep_pages(p, x);
+  const int N = keep_pages(p, s, x);
   const int ncs = N * dm.P;
   const int nbins = G * dm.nb + 1;
   for (int i = tid; i < N; i += FZ_CONS) spage[i] = __ldcg(wk.sel_pages + (long long)x.u * wk.Nmax + i);
@@ -1174,7 +1229,8 @@ __device__ void fz_ksel(const FzParams& p, const FzShared& s, const Unit& x) {
   }
   int n_cand;
   const int before = cons_excl_scan(local, red, &n_cand);
-  const int keff = min(min(max(__ldg(p.top_k + x.b), 1), wk.Kmax), n_cand);
+  const int tk = x.b < FZ_SEQ ? s.seqp[2 * FZ_SEQ + x.b] : __ldg(p.top_k + x.b);
+  const int keff = min(min(max(tk, 1), wk.Kmax), n_cand);
   if (keff > 0 && before < keff && before + local >= keff) {
     int run = before;
 #pragma unroll
@@ -1200,21 +1256,23 @@ __device__ void fz_ksel(const FzParams& p, const FzShared& s, const Unit& x) {
     // warp places its rows with ballots.
     const int T = bc[2], need_eq = bc[3];
     const int rounds = (ncs + FZ_CONS - 1) / FZ_CONS;  // <= 32
-    const uint16_t* ks = wk.kscore + (long long)x.u * wk.Cmax;
     const unsigned lanemask_lt = (1u << lane) - 1u;
-    int sv[32];
-#pragma unroll
-    for (int r = 0; r < 32; ++r) {
-      const int ci = r * FZ_CONS + tid;
-      sv[r] = (r < rounds && ci < ncs) ? (int)__ldcg(ks + ci) : 0xFFFF;
+    // the scores into shared memory (ncs is a multiple of the page size: whole 16-byte vectors)
+    uint16_t* scs = reinterpret_cast<uint16_t*>(s.work + KS_SC);
+    {
+      const uint4* src = reinterpret_cast<const uint4*>(wk.kscore + (long long)x.u * wk.Cmax);
+      const int n16 = ncs / 8;
+#pragma unroll 4
+      for (int i = tid; i < n16; i += FZ_CONS) reinterpret_cast<uint4*>(scs)[i] = __ldcg(src + i);
     }
-#pragma unroll
-    for (int r = 0; r < 32; ++r) {
-      if (r < rounds) {
-        const unsigned blt = __ballot_sync(0xffffffffu, sv[r] < T);
-        const unsigned beq = __ballot_sync(0xffffffffu, sv[r] == T);
-        if (lane == 0) wcnt[r * FZ_CWARPS + warp] = (__popc(blt) << 16) | __popc(beq);
-      }
+    cons_sync();
+#pragma unroll 2
+    for (int r = 0; r < rounds; ++r) {
+      const int ci = r * FZ_CONS + tid;
+      const int v = ci < ncs ? (int)scs[ci] : 0xFFFF;
+      const unsigned blt = __ballot_sync(0xffffffffu, v < T);
+      const unsigned beq = __ballot_sync(0xffffffffu, v == T);
+      if (lane == 0) wcnt[r * FZ_CWARPS + warp] = (__popc(blt) << 16) | __popc(beq);
     }
     cons_sync();
     {
@@ -1227,24 +1285,23 @@ __device__ void fz_ksel(const FzParams& p, const FzShared& s, const Unit& x) {
     }
     int* out = wk.sel_keys + (long long)x.u * wk.Kmax;
     int* dout = p.dbg.sel_keys ? p.dbg.sel_keys + (long long)x.u * wk.Kmax : nullptr;
-#pragma unroll
-    for (int r = 0; r < 32; ++r) {
-      if (r < rounds) {
-        const int ci = r * FZ_CONS + tid;
-        const bool lt = sv[r] < T, eq = sv[r] == T;
-        const unsigned beq = __ballot_sync(0xffffffffu, eq);
-        const int base2 = wcnt[r * FZ_CWARPS + warp];
-        const int lt_before = base2 >> 16, eq_before = base2 & 0xffff;
-        const int eq_rank = eq_before + __popc(beq & lanemask_lt);
-        const bool take = lt || (eq && eq_rank < need_eq);
-        const unsigned btake = __ballot_sync(0xffffffffu, take);
-        const int pos = lt_before + min(eq_before, need_eq) + __popc(btake & lanemask_lt);
-        if (take) {
-          const int slot = ci / dm.P;
-          const int t = spage[slot] * dm.P + (ci - slot * dm.P);
-          out[pos] = t;
-          if (dout) dout[pos] = t;
-        }
+#pragma unroll 2
+    for (int r = 0; r < rounds; ++r) {
+      const int ci = r * FZ_CONS + tid;
+      const int v = ci < ncs ? (int)scs[ci] : 0xFFFF;
+      const bool lt = v < T, eq = v == T;
+      const unsigned beq = __ballot_sync(0xffffffffu, eq);
+      const int base2 = wcnt[r * FZ_CWARPS + warp];
+      const int lt_before = base2 >> 16, eq_before = base2 & 0xffff;
+      const int eq_rank = eq_before + __popc(beq & lanemask_lt);
+      const bool take = lt || (eq && eq_rank < need_eq);
+      const unsigned btake = __ballot_sync(0xffffffffu, take);
+      const int pos = lt_before + min(eq_before, need_eq) + __popc(btake & lanemask_lt);
+      if (take) {
+        const int slot = ci / dm.P;
+        const int t = spage[slot] * dm.P + (ci - slot * dm.P);
+        out[pos] = t;
+        if (dout) dout[pos] = t;
       }
     }
   }
@@ -1256,82 +1313,107 @@ __device__ void fz_ksel(const FzParams& p, const FzShared& s, const Unit& x) {
 }
 
 // ---- GATHER: softmax attention over one chunk of kept rows ---------------------
-// Warp w takes rows 8w .. 8w+7: logits, the warp's max and weights per head,
-// and the weighted V sum of those rows (lane: channels 4l .. 4l+3).  One
-// barrier later the 16 warp partials are combined in warp order into the
-// chunk's partial (unnormalised output, max and sum of weights per head, in
-// log2 units) at its fixed slot part[u][c].
+// Warp w takes rows 8w .. 8w+7.  Logits: groups of LPR lanes share a row (a
+// lane holds 16 or 8 of its channels), so a dot product is reduced over LPR
+// lanes only.  Then the warp's max and weights per head, and the weighted V
+// sum of its rows (lane: channels 4l .. 4l+3).  One barrier later the 16 warp
+// partials are combined in warp order into the chunk's partial (unnormalised
+// output, max and sum of weights per head, in log2 units) at part[u][c].
 constexpr int GA_OB = 0;                  // float [16 warps][G][128] warp outputs
-constexpr int GA_PB = 65536;              // float [16 warps][8 rows][GP] weights
-constexpr int GA_MB = GA_PB + 4096;       // float [16][8] warp maxima
+constexpr int GA_PB = 65536;              // float2 [16 warps][8 rows][GP] weights as (p, p)
+constexpr int GA_MB = GA_PB + 8192;       // float [16][8] warp maxima
 constexpr int GA_LB = GA_MB + 512;        // float [16][8] warp sums
-static_assert(GA_LB + 512 <= FZ_HIST_OFF, "gather scratch");
+static_assert(GA_LB + 512 <= FZ_WORK, "gather scratch");
 
 template <int G>
 __device__ void fz_gather(const FzParams& p, const FzShared& s, const Unit& x, int c, int n, int d, int s0) {
-  constexpr int GP = G <= 4 ? 4 : 8;   // heads padded to a power of two
-  constexpr int RB = GP == 4 ? 8 : 4;  // rows per logit batch
-  constexpr int NBT = 8 / RB;          // batches
-  constexpr int NV = RB * GP;          // 32 partial logits per lane per batch
+  constexpr int GP = G <= 4 ? 4 : 8;     // heads padded to a power of two
+  constexpr int LPR = GP == 4 ? 8 : 16;  // lanes per row in the logits
+  constexpr int NCK = 128 / LPR / 8;     // 16-byte chunks per lane and row (2 or 1)
+  constexpr int RPG = LPR / 4;           // rows per lane group (2 or 4; 8 rows per warp)
+  constexpr int NV = RPG * GP;           // partial logits per lane (8 or 32)
+  constexpr int KP = NV / LPR;           // logits per lane after the reduction (1 or 2)
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+  const int grp = lane / LPR, li = lane % LPR;
   float* OB = reinterpret_cast<float*>(s.work + GA_OB);
-  float* PB = reinterpret_cast<float*>(s.work + GA_PB) + warp * 8 * GP;
+  float2* PB = reinterpret_cast<float2*>(s.work + GA_PB) + warp * 8 * GP;
   float* MB = reinterpret_cast<float*>(s.work + GA_MB);
   float* LB = reinterpret_cast<float*>(s.work + GA_LB);
   const float* qs = reinterpret_cast<const float*>(s.qbuf + d * FZ_QBUF);
   const float qscale = p.sm_scale * 1.4426950408889634f;
-  // ---- logits; after the reduction lane l holds head l / RB, row l % RB of the batch ----
-  const int gl = lane / RB, rl = lane % RB;
-  float sv[NBT];
+  // ---- logits: lane holds channels 8 (LPR k + li) .. +7 for chunks k < NCK ----
+  float sv[KP];
   {
-    float qv[G][4];
+    float2 q2[G][4 * NCK];
 #pragma unroll
-    for (int g = 0; g < G; ++g) {
-      const float4 t = *reinterpret_cast<const float4*>(qs + g * D + 4 * lane);
-      qv[g][0] = t.x * qscale; qv[g][1] = t.y * qscale; qv[g][2] = t.z * qscale; qv[g][3] = t.w * qscale;
-    }
+    for (int g = 0; g < G; ++g)
 #pragma unroll
-    for (int bt = 0; bt < NBT; ++bt) {
-      float v[NV];
+      for (int k = 0; k < NCK; ++k)
 #pragma unroll
-      for (int r = 0; r < RB; ++r) {
-        const int j = warp * 8 + bt * RB + r;
-        const uint2 kv = *reinterpret_cast<const uint2*>(s.ring + (size_t)((s0 + j / 64) % FZ_NSLOT) * FZ_SLOT +
-                                                         (j % 64) * 256 + lane * 8);
-        const float kf[4] = {bf_lo(kv.x), bf_hi(kv.x), bf_lo(kv.y), bf_hi(kv.y)};
-#pragma unroll
-        for (int g = 0; g < GP; ++g) {
-          float a = 0.f;
-          if (g < G) {
-            a = qv[g][0] * kf[0];
-            a = fmaf(qv[g][1], kf[1], a);
-            a = fmaf(qv[g][2], kf[2], a);
-            a = fmaf(qv[g][3], kf[3], a);
-          }
-          v[g * RB + r] = a;
+        for (int h = 0; h < 2; ++h) {
+          const float4 t = *reinterpret_cast<const float4*>(qs + g * D + 8 * (LPR * k + li) + 4 * h);
+          q2[g][4 * k + 2 * h] = make_float2(t.x * qscale, t.y * qscale);
+          q2[g][4 * k + 2 * h + 1] = make_float2(t.z * qscale, t.w * qscale);
         }
+    float v[NV];  // [head][row of the group]
+#pragma unroll
+    for (int r = 0; r < RPG; ++r) {
+      const int j = warp * 8 + grp * RPG + r;
+      const unsigned char* row = s.ring + (size_t)((s0 + j / 64) % FZ_NSLOT) * FZ_SLOT + (j % 64) * 256;
+      float2 kf[4 * NCK];
+#pragma unroll
+      for (int k = 0; k < NCK; ++k) {
+        const uint4 kv = *reinterpret_cast<const uint4*>(row + 16 * (LPR * k + li));
+        kf[4 * k] = make_float2(bf_lo(kv.x), bf_hi(kv.x));
+        kf[4 * k + 1] = make_float2(bf_lo(kv.y), bf_hi(kv.y));
+        kf[4 * k + 2] = make_float2(bf_lo(kv.z), bf_hi(kv.z));
+        kf[4 * k + 3] = make_float2(bf_lo(kv.w), bf_hi(kv.w));
       }
-      warp_reduce_t<NV>(v, lane);
-      const int j = warp * 8 + bt * RB + rl;
-      sv[bt] = (gl < G && j < n) ? v[0] : -INFINITY;
+#pragma unroll
+      for (int g = 0; g < GP; ++g) {
+        float a = 0.f;
+        if (g < G) {
+          float2 a0 = __fmul2_rn(q2[g][0], kf[0]);
+          float2 a1 = __fmul2_rn(q2[g][1], kf[1]);
+#pragma unroll
+          for (int k = 2; k < 4 * NCK; k += 2) {
+            a0 = __ffma2_rn(q2[g][k], kf[k], a0);
+            a1 = __ffma2_rn(q2[g][k + 1], kf[k + 1], a1);
+          }
+          a = (a0.x + a0.y) + (a1.x + a1.y);
+        }
+        v[g * RPG + r] = a;
+      }
+    }
+    group_reduce_t<NV, LPR>(v, lane);
+    // lane li holds values [KP li, KP li + KP): head (KP li) / RPG = li / 2, rows KP li % RPG + e
+#pragma unroll
+    for (int e = 0; e < KP; ++e) {
+      const int r = (KP * li + e) % RPG;
+      const int j = warp * 8 + grp * RPG + r;
+      sv[e] = ((li >> 1) < G && j < n) ? v[e] : -INFINITY;
     }
   }
-  // ---- the warp's max and weights per head (the RB lanes of head gl) ----
+  const int gl = li >> 1;  // the lane's head
+  // ---- the warp's max and weights per head: lanes 2 gl, 2 gl + 1 of every group ----
   float m = sv[0];
 #pragma unroll
-  for (int bt = 1; bt < NBT; ++bt) m = fmaxf(m, sv[bt]);
+  for (int e = 1; e < KP; ++e) m = fmaxf(m, sv[e]);
+  m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, 1));
 #pragma unroll
-  for (int o = 1; o < RB; o <<= 1) m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, o));
+  for (int o = LPR; o < 32; o <<= 1) m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, o));
   float l = 0.f;
 #pragma unroll
-  for (int bt = 0; bt < NBT; ++bt) {
-    const float pv = (sv[bt] == -INFINITY) ? 0.f : exp2f(sv[bt] - m);
-    PB[(bt * RB + rl) * GP + gl] = pv;
+  for (int e = 0; e < KP; ++e) {
+    const float pv = (sv[e] == -INFINITY) ? 0.f : exp2f(sv[e] - m);
+    const int r = (KP * li + e) % RPG;
+    PB[(grp * RPG + r) * GP + gl] = make_float2(pv, pv);
     l += pv;
   }
+  l += __shfl_xor_sync(0xffffffffu, l, 1);
 #pragma unroll
-  for (int o = 1; o < RB; o <<= 1) l += __shfl_xor_sync(0xffffffffu, l, o);
-  if (rl == 0 && gl < G) {
+  for (int o = LPR; o < 32; o <<= 1) l += __shfl_xor_sync(0xffffffffu, l, o);
+  if (lane < LPR && (li & 1) == 0 && gl < G) {
     MB[warp * 8 + gl] = m;
     LB[warp * 8 + gl] = l;
   }
@@ -1347,17 +1429,17 @@ __device__ void fz_gather(const FzParams& p, const FzShared& s, const Unit& x, i
       const uint2 vv = *reinterpret_cast<const uint2*>(s.ring + (size_t)((s0 + 2 + j / 64) % FZ_NSLOT) * FZ_SLOT +
                                                        (j % 64) * 256 + lane * 8);
       const float2 v0 = make_float2(bf_lo(vv.x), bf_hi(vv.x)), v1 = make_float2(bf_lo(vv.y), bf_hi(vv.y));
-      float pr[GP];
+      float2 pr[GP];
 #pragma unroll
-      for (int g4 = 0; g4 < GP; g4 += 4) {
-        const float4 t = *reinterpret_cast<const float4*>(PB + r * GP + g4);
-        pr[g4] = t.x; pr[g4 + 1] = t.y; pr[g4 + 2] = t.z; pr[g4 + 3] = t.w;
+      for (int g2 = 0; g2 < G; g2 += 2) {
+        const float4 t = *reinterpret_cast<const float4*>(PB + r * GP + g2);
+        pr[g2] = make_float2(t.x, t.y);
+        pr[g2 + 1] = make_float2(t.z, t.w);
       }
 #pragma unroll
       for (int g = 0; g < G; ++g) {
-        const float2 pp = make_float2(pr[g], pr[g]);
-        o2[g][0] = __ffma2_rn(pp, v0, o2[g][0]);
-        o2[g][1] = __ffma2_rn(pp, v1, o2[g][1]);
+        o2[g][0] = __ffma2_rn(pr[g], v0, o2[g][0]);
+        o2[g][1] = __ffma2_rn(pr[g], v1, o2[g][1]);
       }
     }
   }
@@ -1510,7 +1592,7 @@ template <int G, int WORDS, bool DENSE>
 __device__ void fz_run_task(const FzParams& p, const FzShared& s, int kind, int u, int arg, unsigned& nfin) {
   const int tid = threadIdx.x;
   const int PS = G * D + 16;
-  const Unit x = unit_of(p, u);
+  const Unit x = unit_of(p, s, u);
   // every thread acquires what the counted CTAs wrote before reading it
   if (kind == TK_PSEL) (void)ld_acquire(unit_ctrl(p, u) + CU_SCAN);
   else if (kind == TK_KSEL) (void)ld_acquire(unit_ctrl(p, u) + CU_SCORE);
@@ -1520,9 +1602,11 @@ __device__ void fz_run_task(const FzParams& p, const FzShared& s, int kind, int 
     if constexpr (!DENSE) {
       if (kind == TK_PSEL) fz_psel(p, s, x);
       else fz_ksel<G>(p, s, x);
-      __threadfence();
       cons_sync();
-      if (tid == 0) st_release(unit_ctrl(p, u) + (kind == TK_PSEL ? CU_PSEL : CU_SEL), 1u);
+      if (tid == 0) {
+        __threadfence();
+        st_release(unit_ctrl(p, u) + (kind == TK_PSEL ? CU_PSEL : CU_SEL), 1u);
+      }
     }
     return;
   }
@@ -1550,6 +1634,7 @@ __device__ void fz_consumer(const FzParams& p, const FzShared& s) {
   volatile int* misc = s.misc;
   unsigned nslot = 0, ndesc = 0, nfin = 0;
   bool ended = false;
+  bool pref = false;  // the rows of the next descriptor were gathered during the previous item
   int* dec = s.misc + 16;  // decisions broadcast by thread 0 (outside every scratch area)
   while (true) {
     const int d = (int)(ndesc % FZ_NDESC);
@@ -1572,8 +1657,12 @@ __device__ void fz_consumer(const FzParams& p, const FzShared& s) {
           break;
         }
         if (!ended) {
-          if (mbar_try_wait(&s.dfull[d], dpar)) {
+          if (mbar_test_wait(&s.dfull[d], dpar)) {
             res = 2;
+            // is the descriptor after it published already, with rows to gather?
+            const unsigned n1 = ndesc + 1;
+            const int d1 = (int)(n1 % FZ_NDESC);
+            dec[3] = (mbar_test_wait(&s.dfull[d1], (n1 / FZ_NDESC) & 1) && s.desc[d1].gather) ? 1 : 0;
             break;
           }
         } else if (misc[5] == (int)nfin) {
@@ -1601,18 +1690,32 @@ __device__ void fz_consumer(const FzParams& p, const FzShared& s) {
       fz_run_task<G, WORDS, DENSE>(p, s, kind, u, arg, nfin);
       continue;
     }
-    mbar_confirm(&s.dfull[d], dpar);
+    // Thread 0 saw the descriptor's phase (and below, the slots' phases)
+    // complete; the consumer barrier orders every other thread after it.
     const FzDesc ds = s.desc[d];
     cons_sync();  // everyone holds the descriptor before dec is written again
     if (ds.kind == IT_END) {
       ended = true;
-      __syncwarp();
-      if (lane == 0) mbar_arrive(&s.dempty[d]);
+      if (tid == 0) mbar_arrive(&s.dempty[d]);
       ++ndesc;
       continue;
     }
     const int nslots = ds.nslots;
     const int s0 = (int)(nslot % FZ_NSLOT);
+    // Rows this item gathers (unless already requested during the previous
+    // item), then the rows of the next descriptor, so that its copies run
+    // while this item computes.
+    const bool pn = dec[3] != 0;
+    if (ds.gather && !pref)
+      gather_rows(s, s.ridx + d * FZ_ROWS, ds.n, s0, ds.kind == IT_SCAN ? p.pmin : p.Kr,
+                  ds.kind == IT_SCAN ? p.pmax : p.Vc);
+    if (pn) {
+      const int d1 = (int)((ndesc + 1) % FZ_NDESC);
+      const FzDesc nx = s.desc[d1];
+      gather_rows(s, s.ridx + d1 * FZ_ROWS, nx.n, (int)((nslot + nslots) % FZ_NSLOT), nx.kind == IT_SCAN ? p.pmin : p.Kr,
+                  nx.kind == IT_SCAN ? p.pmax : p.Vc);
+    }
+    pref = pn;
     if (nslots > 0) {
       if (tid == 0) {
         bool ok = true;
@@ -1624,24 +1727,28 @@ __device__ void fz_consumer(const FzParams& p, const FzShared& s) {
       }
       cons_sync();
       if (!dec[2]) break;
-      for (int k = 0; k < nslots; ++k) {
-        const unsigned gs = nslot + k;
-        mbar_confirm(&s.full[gs % FZ_NSLOT], (gs / FZ_NSLOT) & 1);
-      }
     }
-    const Unit x = unit_of(p, ds.unit);
+    if (ds.gather) {
+      // this thread's copies of this item have landed (the next item's may still fly);
+      // every warp computes on the rows it copied itself
+      if (pn) cp_async_wait<1>();
+      else cp_async_wait<0>();
+      __syncwarp();
+    }
+    const Unit x = unit_of(p, s, ds.unit);
     if (ds.kind == IT_PREP) {
       fz_prep<G, DENSE>(p, s, x, d, s0);
     } else if (ds.kind == IT_SCAN) {
       if constexpr (!DENSE) fz_scan<G>(p, s, x, ds.chunk, ds.n, d, s0);
     } else if (ds.kind == IT_SCORE) {
-      if constexpr (!DENSE) fz_score<G, WORDS>(p, s, x, ds.chunk, ds.n, s0);
+      if constexpr (!DENSE) fz_score<G, WORDS>(p, s, x, ds.chunk, ds.n, d);
     } else if (ds.kind == IT_GATHER) {
       fz_gather<G>(p, s, x, ds.chunk, ds.n, d, s0);
     }
-    // release the slots and the descriptor (one arrival per consumer warp)
-    __syncwarp();
-    if (lane == 0) {
+    // every consumer thread is done with the slots: release them and the descriptor
+    cons_sync();
+    if (tid == 0) {
+      if (ds.gather) asm volatile("fence.proxy.async.shared::cta;" ::: "memory");  // before later bulk copies into the slots
       for (int k = 0; k < nslots; ++k) mbar_arrive(&s.empty[(nslot + k) % FZ_NSLOT]);
       mbar_arrive(&s.dempty[d]);
     }
@@ -1658,21 +1765,20 @@ __device__ void fz_consumer(const FzParams& p, const FzShared& s) {
         }
       }
       if (DENSE || x.L == 0) {
-        if (tid == 0) unit_ctrl(p, x.u)[CU_NKEYS] = DENSE ? (unsigned)x.L : 0u;
-        __threadfence();
         cons_sync();
-        if (tid == 0) st_release(unit_ctrl(p, x.u) + CU_SEL, 1u);
+        if (tid == 0) {
+          unit_ctrl(p, x.u)[CU_NKEYS] = DENSE ? (unsigned)x.L : 0u;
+          __threadfence();
+          st_release(unit_ctrl(p, x.u) + CU_SEL, 1u);
+        }
       }
     } else if (ds.kind == IT_SCAN) {
-      cons_sync();
       const unsigned nscan = (unsigned)((x.np + FZ_ROWS - 1) / FZ_ROWS);
       fz_finish(s, nfin, unit_ctrl(p, x.u) + CU_SCAN, 1u, nscan, TK_PSEL, x.u, 0, p.status);
     } else if (ds.kind == IT_SCORE) {
-      cons_sync();
-      fz_finish(s, nfin, unit_ctrl(p, x.u) + CU_SCORE, 1u, (unsigned)score_items(p, x), TK_KSEL, x.u, 0,
+      fz_finish(s, nfin, unit_ctrl(p, x.u) + CU_SCORE, 1u, (unsigned)score_items(p, s, x), TK_KSEL, x.u, 0,
                 p.status);
     } else if (ds.kind == IT_GATHER) {
-      cons_sync();
       const int nch = nchunks_of((unsigned)ds.pad0);
       const int g = ds.chunk / FZ_GROUP;
       const int gsize = min(FZ_GROUP, nch - g * FZ_GROUP);
@@ -1694,11 +1800,11 @@ __global__ void __launch_bounds__(FZ_THREADS, 1) hhr_fused_kernel(FzParams p) {
   if (tid == 0) {
     for (int i = 0; i < FZ_NSLOT; ++i) {
       mbar_init(&s.full[i], 1);
-      mbar_init(&s.empty[i], FZ_CWARPS);
+      mbar_init(&s.empty[i], 1);
     }
     for (int i = 0; i < FZ_NDESC; ++i) {
       mbar_init(&s.dfull[i], 1);
-      mbar_init(&s.dempty[i], FZ_CWARPS);
+      mbar_init(&s.dempty[i], 1);
     }
     for (int i = 0; i < FZ_NFIN; ++i) {
       mbar_init(&s.ffull[i], 1);
@@ -1707,8 +1813,13 @@ __global__ void __launch_bounds__(FZ_THREADS, 1) hhr_fused_kernel(FzParams p) {
     for (int i = 0; i < 8; ++i) s.misc[i] = 0;
     fence_mbar_init();
   }
-  int* hist = reinterpret_cast<int*>(s.work + FZ_HIST_OFF);
-  for (int i = tid; i < FZ_HIST_BINS; i += blockDim.x) hist[i] = 0;
+  for (int b = tid; b < min(p.dm.B, FZ_SEQ); b += blockDim.x) {
+    s.seqp[b] = seq_len_of(p.dm, p.seq_lens, b);
+    if constexpr (!DENSE) {  // full attention has no budgets
+      s.seqp[FZ_SEQ + b] = __ldg(p.n_keep + b);
+      s.seqp[2 * FZ_SEQ + b] = __ldg(p.top_k + b);
+    }
+  }
   __syncthreads();
   const int warp = tid >> 5;
   if (warp == FZ_PRODUCER_WARP) {
