@@ -129,7 +129,11 @@ constexpr int FZ_CONS = 512;                 // consumer threads (warps 0-15)
 constexpr int FZ_CWARPS = FZ_CONS / 32;
 constexpr int FZ_PRODUCER_WARP = FZ_CWARPS;
 constexpr int FZ_FINISHER_WARP = FZ_CWARPS + 1;
-constexpr int FZ_THREADS = FZ_CONS + 64;
+constexpr int FZ_THREADS = FZ_CONS + 128;    // + one warpgroup: producer, finisher, two idle warps
+// Registers: the block starts with 96 per thread (20 warps); the last
+// warpgroup gives most of its share to the consumers.
+constexpr int FZ_REGS_CONS = 104, FZ_REGS_AUX = 64;
+static_assert(FZ_CONS * FZ_REGS_CONS + 128 * FZ_REGS_AUX <= FZ_THREADS * 96, "register split");
 constexpr int FZ_NSLOT = 8;                  // ring slots
 constexpr int FZ_SLOT = 16384;               // bytes per slot (64 rows of 256 B)
 constexpr int FZ_NDESC = 4;                  // descriptor ring
@@ -149,7 +153,9 @@ constexpr size_t FZ_OFF_QBUF = FZ_OFF_RING + (size_t)FZ_NSLOT * FZ_SLOT;
 constexpr size_t FZ_OFF_WORK = FZ_OFF_QBUF + (size_t)FZ_NDESC * FZ_QBUF;
 constexpr size_t FZ_OFF_SEQP = FZ_OFF_WORK + FZ_WORK;
 constexpr size_t FZ_OFF_RIDX = FZ_OFF_SEQP + 3 * FZ_SEQ * 4;
-constexpr size_t FZ_OFF_DESC = FZ_OFF_RIDX + FZ_NDESC * FZ_ROWS * 4;
+constexpr int FZ_UCACHE = 512;               // units whose readiness the producer remembers
+constexpr size_t FZ_OFF_UCACHE = FZ_OFF_RIDX + FZ_NDESC * FZ_ROWS * 4;
+constexpr size_t FZ_OFF_DESC = FZ_OFF_UCACHE + FZ_UCACHE * 4;
 constexpr size_t FZ_OFF_FINQ = FZ_OFF_DESC + FZ_NDESC * 32;
 constexpr size_t FZ_OFF_TASK = FZ_OFF_FINQ + FZ_NFIN * 32;
 constexpr size_t FZ_OFF_BAR = FZ_OFF_TASK + FZ_NTASK * 16;
@@ -236,6 +242,7 @@ struct FzShared {
   uint64_t* fempty;
   int* seqp;  // [3][FZ_SEQ]: clamped sequence length, n_keep, top_k of the first FZ_SEQ sequences
   int* ridx;  // [FZ_NDESC][FZ_ROWS]: row numbers of a descriptor (see FzDesc)
+  unsigned* ucache;  // [FZ_UCACHE] producer only: readiness flags seen (UC_*) and the kept rows
   int* misc;  // [0] abort, [1] consumed slots, [2] tasks posted, [3] tasks taken,
               // [4] armed slots, [5] finisher requests done, [6] consumers finished,
               // [16..23] consumer broadcasts
@@ -248,6 +255,7 @@ __device__ __forceinline__ FzShared fz_shared(unsigned char* base) {
   s.work = base + FZ_OFF_WORK;
   s.seqp = reinterpret_cast<int*>(base + FZ_OFF_SEQP);
   s.ridx = reinterpret_cast<int*>(base + FZ_OFF_RIDX);
+  s.ucache = reinterpret_cast<unsigned*>(base + FZ_OFF_UCACHE);
   s.desc = reinterpret_cast<FzDesc*>(base + FZ_OFF_DESC);
   s.finq = reinterpret_cast<FzFin*>(base + FZ_OFF_FINQ);
   s.tasks = reinterpret_cast<FzTask*>(base + FZ_OFF_TASK);
@@ -353,6 +361,38 @@ __device__ __forceinline__ void decode_item(const FzParams& p, int item, int& ki
   kind = IT_END;
 }
 
+// producer-side memory of a unit's readiness: flags seen and the kept rows
+enum : unsigned { UC_PREP = 1u << 31, UC_SEL = 1u << 30, UC_SCORE = 1u << 29, UC_NKEYS = (1u << 24) - 1u };
+
+// The producer warp waits (bounded) until unit u is ready for an item kind:
+// q' published (UC_PREP), kept rows published (UC_SEL; their count is
+// remembered), or kept pages and query codes published (UC_SCORE).  The
+// first time, every lane acquires what the publishing CTA wrote and orders
+// later bulk copies (async proxy) after it; later items of the unit reuse
+// that.  False after a timeout or an abort.
+__device__ __forceinline__ bool fz_unit_ready(const FzParams& p, const FzShared& s, int u, unsigned flag, int lane) {
+  if (u < FZ_UCACHE && (s.ucache[u] & flag)) return true;
+  unsigned* uc = unit_ctrl(p, u);
+  bool ok = true;
+  if (lane == 0) {
+    if (flag == UC_PREP) ok = fz_wait_count(s, uc + CU_PREP, 1u, p.status);
+    else if (flag == UC_SEL) ok = fz_wait_count(s, uc + CU_SEL, 1u, p.status);
+    else ok = fz_wait_count(s, uc + CU_PSEL, 1u, p.status) && fz_wait_count(s, uc + CU_CODES, 1u, p.status);
+  }
+  if (__shfl_sync(0xffffffffu, (int)ok, 0) == 0) return false;
+  (void)ld_acquire(uc + (flag == UC_PREP ? CU_PREP : flag == UC_SEL ? CU_SEL : CU_PSEL));
+  if (flag == UC_SCORE) (void)ld_acquire(uc + CU_CODES);
+  fence_proxy_async_global();  // q' was written by another CTA with ordinary stores
+  if (u < FZ_UCACHE) {
+    unsigned v = 0;
+    if (flag == UC_SEL) v = min(__ldcg(uc + CU_NKEYS), UC_NKEYS);
+    __syncwarp();
+    if (lane == 0) s.ucache[u] |= flag | v;
+    __syncwarp();
+  }
+  return true;
+}
+
 // ---------------------------------------------------------------------------
 // producer (warp 16): claims items, moves contiguous blocks with bulk copies
 // and lists the rows that the consumers gather themselves
@@ -364,10 +404,13 @@ __device__ void fz_producer(const FzParams& p, const FzShared& s) {
   const int prep_slots = DENSE ? 4 : 4 + dm.nb / 64;  // R_h, then W_h (not needed without hashing)
   const uint64_t ef = evict_first_policy();
   unsigned nslot = 0, ndesc = 0, armed = 0;
+  // The next item is claimed one item ahead (the atomic's round trip overlaps
+  // the current item); a unit's readiness, once seen, is remembered.
+  int next = 0;
+  if (lane == 0) next = (int)atomicAdd(p.wk.ctrl + 0, 1u);
   while (true) {
-    int item = 0;
-    if (lane == 0) item = (int)atomicAdd(p.wk.ctrl + 0, 1u);
-    item = __shfl_sync(0xffffffffu, item, 0);
+    const int item = __shfl_sync(0xffffffffu, next, 0);
+    if (lane == 0) next = (int)atomicAdd(p.wk.ctrl + 0, 1u);
     int kind, u, c;
     decode_item(p, item, kind, u, c);
     const Unit x = unit_of(p, s, u);
@@ -379,18 +422,10 @@ __device__ void fz_producer(const FzParams& p, const FzShared& s) {
     } else if (kind == IT_SCORE) {
       n = min(FZ_CS, keep_pages(p, s, x) * dm.P - c * FZ_CS);
       if (n <= 0) continue;
-      bool ok = true;
-      if (lane == 0)
-        ok = fz_wait_count(s, unit_ctrl(p, u) + CU_PSEL, 1u, p.status) &&
-             fz_wait_count(s, unit_ctrl(p, u) + CU_CODES, 1u, p.status);
-      if (__shfl_sync(0xffffffffu, (int)ok, 0) == 0) break;
-      (void)ld_acquire(unit_ctrl(p, u) + CU_PSEL);  // every lane reads the kept pages
+      if (!fz_unit_ready(p, s, u, UC_SCORE, lane)) break;
     } else if (kind == IT_GATHER) {
-      bool ok = true;
-      if (lane == 0) ok = fz_wait_count(s, unit_ctrl(p, u) + CU_SEL, 1u, p.status);
-      if (__shfl_sync(0xffffffffu, (int)ok, 0) == 0) break;
-      (void)ld_acquire(unit_ctrl(p, u) + CU_SEL);  // every lane reads what the selecting CTA wrote
-      nk = __ldcg(unit_ctrl(p, u) + CU_NKEYS);
+      if (!fz_unit_ready(p, s, u, UC_SEL, lane)) break;
+      nk = u < FZ_UCACHE ? (s.ucache[u] & UC_NKEYS) : __ldcg(unit_ctrl(p, u) + CU_NKEYS);
       n = min(FZ_ROWS, (int)nk - c * FZ_ROWS);
       if (n <= 0) continue;
     } else if (kind == IT_PREP) {
@@ -444,12 +479,7 @@ __device__ void fz_producer(const FzParams& p, const FzShared& s) {
       qbytes = G * D * 2;
       qsrc = p.q + ((long long)x.b * dm.Hq + x.h * G) * D;
     } else if (kind == IT_SCAN || kind == IT_GATHER) {
-      if (kind == IT_SCAN) {
-        bool ok = true;
-        if (lane == 0) ok = fz_wait_count(s, unit_ctrl(p, u) + CU_PREP, 1u, p.status);
-        if (__shfl_sync(0xffffffffu, (int)ok, 0) == 0) break;
-      }
-      fence_proxy_async_global();  // q' was written by another CTA with ordinary stores
+      if (kind == IT_SCAN && !fz_unit_ready(p, s, u, UC_PREP, lane)) break;
       qbytes = G * D * 4;
       qsrc = p.wk.qrot + ((long long)x.b * dm.Hq + x.h * G) * D;
     }
@@ -513,7 +543,12 @@ __device__ void fz_producer(const FzParams& p, const FzShared& s) {
     ++ndesc;
     if (kind == IT_END) break;
   }
-  if (lane == 0) s.misc[4] = (int)armed;  // slots armed with copies (drained at exit)
+  if (lane == 0) {
+    s.misc[4] = (int)armed;  // slots armed with copies (drained at exit)
+    // the claim issued ahead has returned before the CTA reports its exit
+    // (the last CTA then resets the queue counter)
+    asm volatile("" ::"r"(next));
+  }
 }
 
 // Consumers copy the rows of a gathering descriptor into its slots: warp w
@@ -692,6 +727,14 @@ __device__ __forceinline__ void cons_minmax(float& lo, float& hi, float* wr) {
   cons_sync();
 }
 
+// q' of a head is stored with its channel quads (4 channels) reordered:
+// quad 2m + b at position m + 16 b.  The scan's and the gather's lanes then
+// read 8 consecutive 16-byte vectors per wavefront (no bank conflicts).
+__device__ __forceinline__ int qpos(int c) {
+  const int q = c >> 2;
+  return 4 * ((q >> 1) + ((q & 1) << 4)) + (c & 3);
+}
+
 __device__ __forceinline__ float dot4(const float4& a, const float* b) {
   float r = a.x * b[0];
   r = fmaf(a.y, b[1], r);
@@ -738,9 +781,9 @@ __device__ void fz_prep(const FzParams& p, const FzShared& s, const Unit& x, int
       const int r = vi / GP, g = vi % GP;
       if (g < G) {
         const int i = warp * 8 + r;
-        const long long idx = ((long long)x.b * dm.Hq + x.h * G + g) * D + i;
-        p.wk.qrot[idx] = v[e];
-        if (p.dbg.q_rot) p.dbg.q_rot[idx] = v[e];
+        const long long idx = ((long long)x.b * dm.Hq + x.h * G + g) * D;
+        p.wk.qrot[idx + qpos(i)] = v[e];
+        if (p.dbg.q_rot) p.dbg.q_rot[idx + i] = v[e];
       }
     }
   }
@@ -865,7 +908,7 @@ __device__ void fz_scan(const FzParams& p, const FzShared& s, const Unit& x, int
   for (int g = 0; g < G; ++g) {
 #pragma unroll
     for (int k = 0; k < 2; ++k) {
-      const float4 t = *reinterpret_cast<const float4*>(qs + g * D + 8 * li + 4 * k);
+      const float4 t = *reinterpret_cast<const float4*>(qs + g * D + 4 * (li + 16 * k));  // channels 8 li + 4 k ..
       if constexpr (SPLIT) {
         qa[g][2 * k] = make_float2(fmaxf(t.x, 0.f), fmaxf(t.y, 0.f));
         qa[g][2 * k + 1] = make_float2(fmaxf(t.z, 0.f), fmaxf(t.w, 0.f));
@@ -1297,7 +1340,7 @@ __device__ void fz_ksel(const FzParams& p, const FzShared& s, const Unit& x) {
       const bool take = lt || (eq && eq_rank < need_eq);
       const unsigned btake = __ballot_sync(0xffffffffu, take);
       const int pos = lt_before + min(eq_before, need_eq) + __popc(btake & lanemask_lt);
-      if (take) {
+      if (take && pos < keff) {  // (always true; keeps the stores inside the list)
         const int slot = ci / dm.P;
         const int t = spage[slot] * dm.P + (ci - slot * dm.P);
         out[pos] = t;
@@ -1351,7 +1394,8 @@ __device__ void fz_gather(const FzParams& p, const FzShared& s, const Unit& x, i
       for (int k = 0; k < NCK; ++k)
 #pragma unroll
         for (int h = 0; h < 2; ++h) {
-          const float4 t = *reinterpret_cast<const float4*>(qs + g * D + 8 * (LPR * k + li) + 4 * h);
+          // channels 8 (LPR k + li) + 4 h .. (stored in quad order, see qpos)
+          const float4 t = *reinterpret_cast<const float4*>(qs + g * D + 4 * (LPR * k + li + 16 * h));
           q2[g][4 * k + 2 * h] = make_float2(t.x * qscale, t.y * qscale);
           q2[g][4 * k + 2 * h + 1] = make_float2(t.z * qscale, t.w * qscale);
         }
@@ -1374,13 +1418,9 @@ __device__ void fz_gather(const FzParams& p, const FzShared& s, const Unit& x, i
         float a = 0.f;
         if (g < G) {
           float2 a0 = __fmul2_rn(q2[g][0], kf[0]);
-          float2 a1 = __fmul2_rn(q2[g][1], kf[1]);
 #pragma unroll
-          for (int k = 2; k < 4 * NCK; k += 2) {
-            a0 = __ffma2_rn(q2[g][k], kf[k], a0);
-            a1 = __ffma2_rn(q2[g][k + 1], kf[k + 1], a1);
-          }
-          a = (a0.x + a0.y) + (a1.x + a1.y);
+          for (int k = 1; k < 4 * NCK; ++k) a0 = __ffma2_rn(q2[g][k], kf[k], a0);
+          a = a0.x + a0.y;
         }
         v[g * RPG + r] = a;
       }
@@ -1658,8 +1698,14 @@ __device__ void fz_consumer(const FzParams& p, const FzShared& s) {
         }
         if (!ended) {
           if (mbar_test_wait(&s.dfull[d], dpar)) {
+            // the descriptor's bulk copies (bounded wait), then: is the
+            // descriptor after it published already, with rows to gather?
             res = 2;
-            // is the descriptor after it published already, with rows to gather?
+            const int ns = s.desc[d].nslots;
+            for (int k = 0; k < ns && res; ++k) {
+              const unsigned gs = nslot + k;
+              if (!fz_wait(s, &s.full[gs % FZ_NSLOT], (gs / FZ_NSLOT) & 1, p.status)) res = 0;
+            }
             const unsigned n1 = ndesc + 1;
             const int d1 = (int)(n1 % FZ_NDESC);
             dec[3] = (mbar_test_wait(&s.dfull[d1], (n1 / FZ_NDESC) & 1) && s.desc[d1].gather) ? 1 : 0;
@@ -1690,10 +1736,10 @@ __device__ void fz_consumer(const FzParams& p, const FzShared& s) {
       fz_run_task<G, WORDS, DENSE>(p, s, kind, u, arg, nfin);
       continue;
     }
-    // Thread 0 saw the descriptor's phase (and below, the slots' phases)
-    // complete; the consumer barrier orders every other thread after it.
+    // Thread 0 saw the descriptor's phase and its slots' phases complete; the
+    // consumer barrier above orders every other thread after it.  (The
+    // descriptor stays put until this item releases it.)
     const FzDesc ds = s.desc[d];
-    cons_sync();  // everyone holds the descriptor before dec is written again
     if (ds.kind == IT_END) {
       ended = true;
       if (tid == 0) mbar_arrive(&s.dempty[d]);
@@ -1716,18 +1762,6 @@ __device__ void fz_consumer(const FzParams& p, const FzShared& s) {
                   nx.kind == IT_SCAN ? p.pmax : p.Vc);
     }
     pref = pn;
-    if (nslots > 0) {
-      if (tid == 0) {
-        bool ok = true;
-        for (int k = 0; k < nslots && ok; ++k) {
-          const unsigned gs = nslot + k;
-          ok = fz_wait(s, &s.full[gs % FZ_NSLOT], (gs / FZ_NSLOT) & 1, p.status);
-        }
-        dec[2] = ok ? 1 : 0;
-      }
-      cons_sync();
-      if (!dec[2]) break;
-    }
     if (ds.gather) {
       // this thread's copies of this item have landed (the next item's may still fly);
       // every warp computes on the rows it copied itself
@@ -1813,6 +1847,7 @@ __global__ void __launch_bounds__(FZ_THREADS, 1) hhr_fused_kernel(FzParams p) {
     for (int i = 0; i < 8; ++i) s.misc[i] = 0;
     fence_mbar_init();
   }
+  for (int i = tid; i < FZ_UCACHE; i += blockDim.x) s.ucache[i] = 0u;
   for (int b = tid; b < min(p.dm.B, FZ_SEQ); b += blockDim.x) {
     s.seqp[b] = seq_len_of(p.dm, p.seq_lens, b);
     if constexpr (!DENSE) {  // full attention has no budgets
@@ -1822,11 +1857,12 @@ __global__ void __launch_bounds__(FZ_THREADS, 1) hhr_fused_kernel(FzParams p) {
   }
   __syncthreads();
   const int warp = tid >> 5;
-  if (warp == FZ_PRODUCER_WARP) {
-    fz_producer<G, WORDS, DENSE>(p, s);
-  } else if (warp == FZ_FINISHER_WARP) {
-    fz_finisher(p, s);
+  if (warp >= FZ_CWARPS) {
+    asm volatile("setmaxnreg.dec.sync.aligned.u32 %0;" ::"n"(FZ_REGS_AUX));
+    if (warp == FZ_PRODUCER_WARP) fz_producer<G, WORDS, DENSE>(p, s);
+    else if (warp == FZ_FINISHER_WARP) fz_finisher(p, s);
   } else {
+    asm volatile("setmaxnreg.inc.sync.aligned.u32 %0;" ::"n"(FZ_REGS_CONS));
     fz_consumer<G, WORDS, DENSE>(p, s);
   }
   __syncthreads();
