@@ -109,6 +109,10 @@ size_t carve(const Dims& dm, int Nmax, int Kmax, bool dense, char* base, Work* w
   w.qcodes = reinterpret_cast<uint64_t*>(take(sizeof(uint64_t) * dm.B * dm.Hq * dm.words));
   w.part = reinterpret_cast<float*>(take(sizeof(float) * BH * C3 * (dm.G * D + 16)));
   w.gpart = reinterpret_cast<float*>(take(sizeof(float) * BH * max_groups * (dm.G * D + 16)));
+  // grid-wide tasks per unit: page select, key select, the final merge
+  const int tq_cap = (int)(BH * 3);
+  w.tq = reinterpret_cast<int4*>(take(sizeof(int4) * tq_cap));
+  w.tq_cap = tq_cap;
   const int Ustride = (dm.np_max + 31) / 32 * 32;
   const int Cmax = Nmax * dm.P;
   const int HB = (dm.G * dm.nb + 1 + 7) / 8 * 8;

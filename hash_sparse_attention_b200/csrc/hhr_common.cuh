@@ -30,13 +30,15 @@ struct Work {
   float* gpart;        // [B, Hkv, max_groups, G * D + 16] merged groups of chunks
   uint16_t* kscore;    // [B, Hkv, Cmax]    Hamming score of every candidate row
   int* khist;          // [B, Hkv, HB]      score histogram (kept at zero between calls)
-  unsigned* ctrl;      // [4 + B * Hkv * (8 + max_groups)] queue, flags, counters
+  int4* tq;            // [tq_cap]          task queue: (kind, unit, arg, sequence + 1), zero between calls
+  unsigned* ctrl;      // [4 + B * Hkv * (8 + max_groups)] item queue, exit count, task queue head / tail, flags, counters
   int Nmax, Kmax;      // budgets the workspace was sized for
   int Cmax;            // Nmax * page size: candidate rows per unit
   int HB;              // histogram stride (>= G * hash bits + 1)
   int Ustride;         // row stride of U (np_max rounded up to 32)
   int C1, C2, C3;      // scan, score and gather chunks per unit
   int max_groups;      // groups of 16 gather chunks per unit
+  int tq_cap;          // task queue entries (every task of one call fits)
 };
 
 // --- bf16 ---------------------------------------------------------------

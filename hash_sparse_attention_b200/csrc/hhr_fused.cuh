@@ -8,8 +8,10 @@
 //                  rows of the kept pages, in page order) and their histogram
 //   GATHER(u, c)   softmax attention over kept rows [128c, 128c + 128),
 //                  written as a partial per chunk
-// Four more steps run as local tasks of the CTA whose counter increment
-// completes their inputs:
+// Four more steps are tasks, made by the CTA whose counter increment completes
+// their inputs.  Group merges stay in that CTA; the others join a grid-wide
+// queue and the first CTA whose consumers are free (they look at the queue
+// before every item) runs them:
 //   PSEL(u)        after the last scan chunk of u: page top-N
 //   KSEL(u)        after the last score chunk of u: key top-k from the
 //                  score histogram, kept rows compacted in index order
@@ -19,14 +21,16 @@
 // q' (scan), the kept pages and query codes (score) or the kept rows (gather)
 // of a unit claimed before.
 //
-// Warps 0-15 consume; warp 16 (producer) claims items and moves their bytes
-// (R_h, W_h, q or q', page metadata rows, code rows, K'/V rows) into a ring
-// of shared memory slots with cp.async.bulk, each slot completing on an
-// mbarrier; warp 17 (finisher) publishes completions (a gpu-scope fence, then
-// an acquire-release counter increment) and posts the tasks that become ready.
-// Inside an item every consumer lane owns 4 channels of a 128-channel row, so
-// each warp reads whole 256-byte rows from shared memory without conflicts
-// and reduces dot products with one transposed butterfly.
+// Warps 0-15 consume; warp 16 (producer) claims items, moves contiguous
+// blocks (R_h, W_h, q or q', page metadata, dense K'/V) into a ring of shared
+// memory slots with cp.async.bulk, each slot completing on an mbarrier, and
+// lists the rows at scattered addresses (kept or paged K'/V rows, paged
+// metadata, code pages), which the consumer warps copy themselves one item
+// ahead; warp 17 (finisher) publishes completions (a gpu-scope fence, then an
+// acquire-release counter increment) and queues the tasks that become ready.
+// In the scan and the gather a group of 8 or 16 lanes shares a 128-channel
+// row, each lane holding 16 or 8 channels, so a dot product is reduced over
+// that group only; the rest of the warp's work is warp-local.
 //
 // Every wait (mbarrier, shared flag or global counter) is bounded by a clock
 // budget; on expiry the kernel records HHR_ERR_TIMEOUT in the status word,
@@ -113,6 +117,11 @@ __device__ __forceinline__ unsigned ld_acquire(const unsigned* p) {
   asm volatile("ld.acquire.gpu.global.u32 %0, [%1];" : "=r"(v) : "l"(p) : "memory");
   return v;
 }
+__device__ __forceinline__ unsigned ld_relaxed(const unsigned* p) {
+  unsigned v;
+  asm volatile("ld.relaxed.gpu.global.u32 %0, [%1];" : "=r"(v) : "l"(p) : "memory");
+  return v;
+}
 __device__ __forceinline__ unsigned atom_add_acq_rel(unsigned* p, unsigned v) {
   unsigned old;
   asm volatile("atom.acq_rel.gpu.global.add.u32 %0, [%1], %2;" : "=r"(old) : "l"(p), "r"(v) : "memory");
@@ -138,7 +147,7 @@ constexpr int FZ_NSLOT = 8;                  // ring slots
 constexpr int FZ_SLOT = 16384;               // bytes per slot (64 rows of 256 B)
 constexpr int FZ_NDESC = 4;                  // descriptor ring
 constexpr int FZ_NFIN = 8;                   // finisher ring
-constexpr int FZ_NTASK = 16;                 // local task ring
+constexpr int FZ_NTASK = 16;                 // local task ring (group merges)
 constexpr int FZ_QBUF = 4096;                // q (bf16) or q' (fp32) of one unit
 constexpr int FZ_ROWS = FUSED_ROWS;          // pages per SCAN item, rows per GATHER item
 constexpr int FZ_CS = FUSED_SCORE;           // candidates per SCORE item
@@ -184,6 +193,7 @@ struct __align__(16) FzFin {
   unsigned target;  // 0: no task
   int kind, unit, arg, pad;
 };
+
 
 struct __align__(16) FzTask {
   int kind, unit, arg, pad;
@@ -243,7 +253,7 @@ struct FzShared {
   int* seqp;  // [3][FZ_SEQ]: clamped sequence length, n_keep, top_k of the first FZ_SEQ sequences
   int* ridx;  // [FZ_NDESC][FZ_ROWS]: row numbers of a descriptor (see FzDesc)
   unsigned* ucache;  // [FZ_UCACHE] producer only: readiness flags seen (UC_*) and the kept rows
-  int* misc;  // [0] abort, [1] consumed slots, [2] tasks posted, [3] tasks taken,
+  int* misc;  // [0] abort, [1] consumed slots, [2] local tasks posted, [3] local tasks taken,
               // [4] armed slots, [5] finisher requests done, [6] consumers finished,
               // [16..23] consumer broadcasts
 };
@@ -604,7 +614,8 @@ static __device__ void fz_finisher(const FzParams& p, const FzShared& s) {
     mbar_arrive(&s.fempty[f]);  // the request has been read
     __threadfence();  // the consumers' writes (ordered before by their barrier) become visible first
     const unsigned old = atom_add_acq_rel(r.counter, r.value);
-    if (r.target != 0u && old + r.value == r.target) {
+    if (r.target != 0u && old + r.value == r.target && r.kind == TK_GMERGE) {
+      // group merges (many, off the critical path) stay in this CTA
       const long long t1 = clock64();
       while (misc[2] - misc[3] >= FZ_NTASK) {  // ring full: wait for the consumers (bounded)
         if (misc[0] || clock64() - t1 > FZ_WAIT_CYCLES) {
@@ -620,6 +631,19 @@ static __device__ void fz_finisher(const FzParams& p, const FzShared& s) {
       tk.arg = r.arg;
       __threadfence_block();
       misc[2] = t + 1;
+    } else if (r.target != 0u && old + r.value == r.target) {
+      // selects and final merges join the grid-wide queue: whichever CTA is free first runs them
+      const unsigned t = atomicAdd(p.wk.ctrl + 3, 1u);
+      if (t < (unsigned)p.wk.tq_cap) {
+        int4* e = p.wk.tq + t;
+        e->x = r.kind;
+        e->y = r.unit;
+        e->z = r.arg;
+        st_release(reinterpret_cast<unsigned*>(&e->w), t + 1u);
+      } else {
+        set_status(p.status, HHR_ERR_WORKSPACE);  // cannot happen: the queue holds every task of a call
+        misc[0] = 1;
+      }
     }
     __threadfence_block();
     misc[5] = misc[5] + 1;
@@ -702,6 +726,29 @@ __device__ __forceinline__ int cons_excl_scan(int v, int* red, int* total) {
   *total = red[FZ_CWARPS - 1];
   cons_sync();
   return before;
+}
+
+// Exclusive scan of one int over the consumer threads with one barrier:
+// `red` holds FZ_CWARPS ints and must not be reused before the next barrier.
+__device__ __forceinline__ int cons_scan1(int v, int* red, int* total) {
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+  int x = v;
+#pragma unroll
+  for (int o = 1; o < 32; o <<= 1) {
+    const int y = __shfl_up_sync(0xffffffffu, x, o);
+    if (lane >= o) x += y;
+  }
+  if (lane == 31) red[warp] = x;
+  cons_sync();
+  int before = 0, tot = 0;
+#pragma unroll
+  for (int w = 0; w < FZ_CWARPS; ++w) {
+    const int r = red[w];
+    before += w < warp ? r : 0;
+    tot += r;
+  }
+  *total = tot;
+  return before + x - v;
 }
 
 // Block-wide min and max of one value per consumer thread (scratch: 32 floats).
@@ -990,8 +1037,8 @@ constexpr int PS_HIST = 0;                // int [2048] value bins
 constexpr int PS_CAND = 8192;             // int [512] members of the threshold bin
 constexpr int PS_CANDV = PS_CAND + 2048;  // float [512] their bounds
 constexpr int PS_FLAG = PS_CANDV + 2048;  // u32 [256] bitmap of kept members
-constexpr int PS_RED = PS_FLAG + 1024;    // int [48] scan scratch and broadcasts
-constexpr int PS_WR = PS_RED + 256;       // float [32] min / max scratch
+constexpr int PS_RED = PS_FLAG + 1024;    // int [128]: four scan buffers of 16 and broadcasts
+constexpr int PS_WR = PS_RED + 512;       // float [32] min / max scratch
 constexpr int SEL_NBIN = 2048;
 constexpr int SEL_MAX_CAND = 512;
 constexpr int PS_PER = MAX_SELECT_PAGES / FZ_CONS;  // 16 pages per thread
@@ -1006,13 +1053,13 @@ __device__ __forceinline__ int value_bin(float v, float lo, float scale) {
 
 static __device__ void fz_psel(const FzParams& p, const FzShared& s, const Unit& x) {
   const Work& wk = p.wk;
-  const int tid = threadIdx.x;
+  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
   int* hist = reinterpret_cast<int*>(s.work + PS_HIST);
   int* cand = reinterpret_cast<int*>(s.work + PS_CAND);
   float* candv = reinterpret_cast<float*>(s.work + PS_CANDV);
   unsigned* flag = reinterpret_cast<unsigned*>(s.work + PS_FLAG);
-  int* red = reinterpret_cast<int*>(s.work + PS_RED);
-  int* bc = red + 36;  // broadcasts [0..11]
+  int* red = reinterpret_cast<int*>(s.work + PS_RED);  // scans: [0, 32) levels, [64, 80) ties, [80, 96) kept pages
+  int* bc = red + 48;                                  // broadcasts [0..11]
   float* wr = reinterpret_cast<float*>(s.work + PS_WR);
   const int np = x.np;
   const int N = keep_pages(p, s, x);
@@ -1024,7 +1071,7 @@ static __device__ void fz_psel(const FzParams& p, const FzShared& s, const Unit&
       if (dsel) dsel[i] = i;
     }
   } else {
-    // ---- the bounds of pages [16 t, 16 t + 16) into registers ----
+    // ---- the bounds of pages [16 t, 16 t + 16) into registers; hist zeroed meanwhile ----
     const float* Ug = wk.U + (long long)x.u * wk.Ustride;
     const int i0 = tid * PS_PER;
     float v[PS_PER];
@@ -1034,6 +1081,9 @@ static __device__ void fz_psel(const FzParams& p, const FzShared& s, const Unit&
                                         : make_float4(0.f, 0.f, 0.f, 0.f);
       v[4 * k4 + 0] = t.x; v[4 * k4 + 1] = t.y; v[4 * k4 + 2] = t.z; v[4 * k4 + 3] = t.w;
     }
+    for (int i = tid; i < SEL_NBIN; i += FZ_CONS) hist[i] = 0;
+    if (tid < MAX_SELECT_PAGES / 32) flag[tid] = 0u;
+    if (tid == 0) bc[4] = 0;
     const int cnt = max(0, min(PS_PER, np - i0));
     unsigned member = (1u << cnt) - 1u;
     float lo = INFINITY, hi = -INFINITY;
@@ -1043,7 +1093,21 @@ static __device__ void fz_psel(const FzParams& p, const FzShared& s, const Unit&
         lo = fminf(lo, v[k]);
         hi = fmaxf(hi, v[k]);
       }
-    cons_minmax(lo, hi, wr);
+#pragma unroll
+    for (int o = 16; o >= 1; o >>= 1) {
+      lo = fminf(lo, __shfl_xor_sync(0xffffffffu, lo, o));
+      hi = fmaxf(hi, __shfl_xor_sync(0xffffffffu, hi, o));
+    }
+    if (lane == 0) {
+      wr[2 * warp] = lo;
+      wr[2 * warp + 1] = hi;
+    }
+    cons_sync();
+#pragma unroll
+    for (int w = 0; w < FZ_CWARPS; ++w) {
+      lo = fminf(lo, wr[2 * w]);
+      hi = fmaxf(hi, wr[2 * w + 1]);
+    }
     // ---- threshold by value bins.  `member` marks pages still undecided,
     // `keep` the kept.  A level bins the members over their value range,
     // keeps every bin above the one holding the need-th largest member and
@@ -1057,11 +1121,16 @@ static __device__ void fz_psel(const FzParams& p, const FzShared& s, const Unit&
       tie = !(hi > lo);
       if (tie) break;
       const float scale = (float)SEL_NBIN / (hi - lo);
-      for (int i = tid; i < SEL_NBIN; i += FZ_CONS) hist[i] = 0;
-      cons_sync();
+      if (level > 0) {
+        for (int i = tid; i < SEL_NBIN; i += FZ_CONS) hist[i] = 0;
+        cons_sync();
+      }
+      int bn[PS_PER];
 #pragma unroll
-      for (int k = 0; k < PS_PER; ++k)
-        if ((member >> k) & 1u) atomicAdd(&hist[value_bin(v[k], lo, scale)], 1);
+      for (int k = 0; k < PS_PER; ++k) {
+        bn[k] = value_bin(v[k], lo, scale);
+        if ((member >> k) & 1u) atomicAdd(&hist[bn[k]], 1);
+      }
       cons_sync();
       {
         constexpr int BPT = SEL_NBIN / FZ_CONS;  // 4 bins per thread, counted from the top
@@ -1073,7 +1142,7 @@ static __device__ void fz_psel(const FzParams& p, const FzShared& s, const Unit&
           c4 += hv[e];
         }
         int tot;
-        const int before = cons_excl_scan(c4, red, &tot);
+        const int before = cons_scan1(c4, red + 16 * (level & 1), &tot);
         if (before < need && before + c4 >= need) {
           int run = before;
 #pragma unroll
@@ -1094,17 +1163,12 @@ static __device__ void fz_psel(const FzParams& p, const FzShared& s, const Unit&
       float nlo = INFINITY, nhi = -INFINITY;
 #pragma unroll
       for (int k = 0; k < PS_PER; ++k) {
-        if (!((member >> k) & 1u)) continue;
-        const int bn = value_bin(v[k], lo, scale);
-        if (bn > bstar) {
-          keep |= 1u << k;
-          member &= ~(1u << k);
-        } else if (bn < bstar) {
-          member &= ~(1u << k);
-        } else {
-          nlo = fminf(nlo, v[k]);
-          nhi = fmaxf(nhi, v[k]);
-        }
+        const bool m = (member >> k) & 1u;
+        const bool above = m && bn[k] > bstar, at = m && bn[k] == bstar;
+        keep |= above ? 1u << k : 0u;
+        member &= at ? ~0u : ~(1u << k);
+        nlo = at ? fminf(nlo, v[k]) : nlo;
+        nhi = at ? fmaxf(nhi, v[k]) : nhi;
       }
       if (nbin <= SEL_MAX_CAND) break;
       cons_minmax(nlo, nhi, wr);
@@ -1115,7 +1179,7 @@ static __device__ void fz_psel(const FzParams& p, const FzShared& s, const Unit&
       // equal values (or still crowded): members in index order, the first `need`
       const int m = __popc(member);
       int tot;
-      const int mb = cons_excl_scan(m, red, &tot);
+      const int mb = cons_scan1(m, red + 64, &tot);
       int take = max(0, min(m, need - mb));
 #pragma unroll
       for (int k = 0; k < PS_PER; ++k) {
@@ -1126,9 +1190,6 @@ static __device__ void fz_psel(const FzParams& p, const FzShared& s, const Unit&
       }
     } else {
       // exact ranking of the (few) members: larger value first, then lower index
-      if (tid == 0) bc[4] = 0;
-      if (tid < MAX_SELECT_PAGES / 32) flag[tid] = 0u;
-      cons_sync();
 #pragma unroll
       for (int k = 0; k < PS_PER; ++k)
         if ((member >> k) & 1u) {
@@ -1154,7 +1215,7 @@ static __device__ void fz_psel(const FzParams& p, const FzShared& s, const Unit&
     }
     // ---- kept pages in index order ----
     int tot;
-    int pos = cons_excl_scan(__popc(keep), red, &tot);
+    int pos = cons_scan1(__popc(keep), red + 80, &tot);
 #pragma unroll
     for (int k = 0; k < PS_PER; ++k) {
       if ((keep >> k) & 1u) {
@@ -1240,10 +1301,9 @@ __device__ void fz_score(const FzParams& p, const FzShared& s, const Unit& x, in
 
 // ---- KSEL: key top-k (smaller score first, ties to the lower row) ------------
 constexpr int KS_SPAGE = 0;      // int [2048] kept pages
-constexpr int KS_WCNT = 8192;    // int [32 rounds x 16 warps] packed counts
-constexpr int KS_RED = 8192 + 2048 + 64;
-constexpr int KS_SC = 12288;     // uint16 [16384] candidate scores
-static_assert(MAX_KEEP_PAGES <= 2048 && MAX_CANDIDATES <= 32 * FZ_CONS && KS_SC + 2 * MAX_CANDIDATES <= FZ_WORK,
+constexpr int KS_RED = 8192;     // int [64] scan scratch and broadcasts
+constexpr int KS_SC = 8448;      // uint16 [32 rounds x 512] staged candidate scores
+static_assert(MAX_KEEP_PAGES <= 2048 && MAX_CANDIDATES <= 32 * FZ_CONS && KS_SC + 2 * 32 * FZ_CONS <= FZ_WORK,
               "key select layout");
 
 template <int G>
@@ -1252,14 +1312,14 @@ __device__ void fz_ksel(const FzParams& p, const FzShared& s, const Unit& x) {
   const Work& wk = p.wk;
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
   int* spage = reinterpret_cast<int*>(s.work + KS_SPAGE);
-  int* wcnt = reinterpret_cast<int*>(s.work + KS_WCNT);
   int* red = reinterpret_cast<int*>(s.work + KS_RED);
-  int* bc = red + 36;
+  int* bc = red + 48;
+  uint16_t* scs = reinterpret_cast<uint16_t*>(s.work + KS_SC);
   const int N = keep_pages(p, s, x);
   const int ncs = N * dm.P;
   const int nbins = G * dm.nb + 1;
   for (int i = tid; i < N; i += FZ_CONS) spage[i] = __ldcg(wk.sel_pages + (long long)x.u * wk.Nmax + i);
-  // ---- histogram (blocked bins per thread) -> threshold T and ties taken ----
+  // ---- histogram (blocked bins per thread) -> threshold T and the ties taken ----
   int* gh = wk.khist + (long long)x.u * wk.HB;
   const int bpt = (nbins + FZ_CONS - 1) / FZ_CONS;  // <= 5
   int hv[5];
@@ -1271,7 +1331,7 @@ __device__ void fz_ksel(const FzParams& p, const FzShared& s, const Unit& x) {
     local += hv[e];
   }
   int n_cand;
-  const int before = cons_excl_scan(local, red, &n_cand);
+  const int before = cons_scan1(local, red, &n_cand);
   const int tk = x.b < FZ_SEQ ? s.seqp[2 * FZ_SEQ + x.b] : __ldg(p.top_k + x.b);
   const int keff = min(min(max(tk, 1), wk.Kmax), n_cand);
   if (keff > 0 && before < keff && before + local >= keff) {
@@ -1279,8 +1339,8 @@ __device__ void fz_ksel(const FzParams& p, const FzShared& s, const Unit& x) {
 #pragma unroll
     for (int e = 0; e < 5; ++e) {
       if (run < keff && run + hv[e] >= keff) {
-        bc[2] = tid * bpt + e;
-        bc[3] = keff - run;
+        bc[0] = tid * bpt + e;
+        bc[1] = keff - run;
       }
       run += hv[e];
     }
@@ -1291,61 +1351,52 @@ __device__ void fz_ksel(const FzParams& p, const FzShared& s, const Unit& x) {
     const int bi = tid * bpt + e;
     if (e < bpt && bi < nbins && hv[e]) gh[bi] = 0;
   }
-  cons_sync();
+  cons_sync();  // bc, spage
   if (keff > 0) {
-    // Kept rows in candidate order, written coalesced: candidates go in
-    // rounds of 512 (thread t takes candidate round * 512 + t); per round
-    // and warp the counts of S < T and S == T are scanned once, then each
-    // warp places its rows with ballots.
-    const int T = bc[2], need_eq = bc[3];
-    const int rounds = (ncs + FZ_CONS - 1) / FZ_CONS;  // <= 32
+    // Kept rows in candidate order: count S < T and S == T over this
+    // thread's run, one scan, then each thread writes its kept rows.
+    // Kept rows in candidate order.  Warp w owns candidates
+    // [w nbw, (w + 1) nbw) in rounds of 32 (lane l: candidate 32 r + l).
+    // Pass 1 stages the scores and counts S < T and S == T per warp; one
+    // scan over the warp totals; pass 2 places the kept rows with ballots
+    // (coalesced stores).
+    const int T = bc[0], need_eq = bc[1];
+    const int rounds = (ncs + 32 * FZ_CWARPS - 1) / (32 * FZ_CWARPS);  // <= 32
+    const int cw0 = warp * rounds * 32;
+    const uint16_t* ks = wk.kscore + (long long)x.u * wk.Cmax;
     const unsigned lanemask_lt = (1u << lane) - 1u;
-    // the scores into shared memory (ncs is a multiple of the page size: whole 16-byte vectors)
-    uint16_t* scs = reinterpret_cast<uint16_t*>(s.work + KS_SC);
-    {
-      const uint4* src = reinterpret_cast<const uint4*>(wk.kscore + (long long)x.u * wk.Cmax);
-      const int n16 = ncs / 8;
-#pragma unroll 4
-      for (int i = tid; i < n16; i += FZ_CONS) reinterpret_cast<uint4*>(scs)[i] = __ldcg(src + i);
-    }
-    cons_sync();
-#pragma unroll 2
+    int lt_w = 0, eq_w = 0;
+#pragma unroll 8
     for (int r = 0; r < rounds; ++r) {
-      const int ci = r * FZ_CONS + tid;
-      const int v = ci < ncs ? (int)scs[ci] : 0xFFFF;
-      const unsigned blt = __ballot_sync(0xffffffffu, v < T);
-      const unsigned beq = __ballot_sync(0xffffffffu, v == T);
-      if (lane == 0) wcnt[r * FZ_CWARPS + warp] = (__popc(blt) << 16) | __popc(beq);
+      const int ci = cw0 + 32 * r + lane;
+      const int S = ci < ncs ? (int)__ldcg(ks + ci) : 0xFFFF;
+      scs[ci] = (uint16_t)S;
+      lt_w += __popc(__ballot_sync(0xffffffffu, S < T));
+      eq_w += __popc(__ballot_sync(0xffffffffu, S == T));
     }
-    cons_sync();
-    {
-      const int n2 = rounds * FZ_CWARPS;  // <= 512: one count per thread
-      const int c0 = tid < n2 ? wcnt[tid] : 0;
-      int tot;
-      const int bsum = cons_excl_scan(c0, red, &tot);
-      if (tid < n2) wcnt[tid] = bsum;
-      cons_sync();
-    }
+    int tot;
+    const int pk = cons_scan1(lane == 0 ? (lt_w << 16) | eq_w : 0, red + 16, &tot);
+    int lt_b = __shfl_sync(0xffffffffu, pk, 0) >> 16, eq_b = __shfl_sync(0xffffffffu, pk, 0) & 0xFFFF;
+    __syncwarp();  // the warp's staged scores
     int* out = wk.sel_keys + (long long)x.u * wk.Kmax;
     int* dout = p.dbg.sel_keys ? p.dbg.sel_keys + (long long)x.u * wk.Kmax : nullptr;
-#pragma unroll 2
+#pragma unroll 4
     for (int r = 0; r < rounds; ++r) {
-      const int ci = r * FZ_CONS + tid;
-      const int v = ci < ncs ? (int)scs[ci] : 0xFFFF;
-      const bool lt = v < T, eq = v == T;
-      const unsigned beq = __ballot_sync(0xffffffffu, eq);
-      const int base2 = wcnt[r * FZ_CWARPS + warp];
-      const int lt_before = base2 >> 16, eq_before = base2 & 0xffff;
-      const int eq_rank = eq_before + __popc(beq & lanemask_lt);
-      const bool take = lt || (eq && eq_rank < need_eq);
-      const unsigned btake = __ballot_sync(0xffffffffu, take);
-      const int pos = lt_before + min(eq_before, need_eq) + __popc(btake & lanemask_lt);
-      if (take && pos < keff) {  // (always true; keeps the stores inside the list)
+      const int ci = cw0 + 32 * r + lane;
+      const int S = scs[ci];
+      const bool lt = S < T, eq = S == T;
+      const unsigned blt = __ballot_sync(0xffffffffu, lt), beq = __ballot_sync(0xffffffffu, eq);
+      const int eq_before = eq_b + __popc(beq & lanemask_lt);
+      const bool take = lt || (eq && eq_before < need_eq);
+      const int pos = lt_b + __popc(blt & lanemask_lt) + min(eq_before, need_eq);
+      if (take && pos < keff) {  // (pos < keff always holds; keeps the stores inside the list)
         const int slot = ci / dm.P;
         const int t = spage[slot] * dm.P + (ci - slot * dm.P);
         out[pos] = t;
         if (dout) dout[pos] = t;
       }
+      lt_b += __popc(blt);
+      eq_b += __popc(beq);
     }
   }
   if (tid == 0) {
@@ -1676,6 +1727,7 @@ __device__ void fz_consumer(const FzParams& p, const FzShared& s) {
   bool ended = false;
   bool pref = false;  // the rows of the next descriptor were gathered during the previous item
   int* dec = s.misc + 16;  // decisions broadcast by thread 0 (outside every scratch area)
+  unsigned qhead = 0, qtail = 0;  // thread 0: the task queue as last read
   while (true) {
     const int d = (int)(ndesc % FZ_NDESC);
     const uint32_t dpar = (ndesc / FZ_NDESC) & 1;
@@ -1685,8 +1737,9 @@ __device__ void fz_consumer(const FzParams& p, const FzShared& s) {
     if (tid == 0) {
       int res = 0;
       const long long t0 = clock64();
+      unsigned spins = 0;
       while (true) {
-        if (misc[3] != misc[2]) {
+        if (misc[3] != misc[2]) {  // a group merge of this CTA
           __threadfence_block();
           const FzTask tk = s.tasks[misc[3] % FZ_NTASK];
           dec[4] = tk.kind;
@@ -1695,6 +1748,31 @@ __device__ void fz_consumer(const FzParams& p, const FzShared& s) {
           misc[3] = misc[3] + 1;
           res = 1;
           break;
+        }
+        // the grid-wide task queue (head and tail read before the last release, then fresh)
+        if (spins++ > 0) {
+          qhead = ld_relaxed(p.wk.ctrl + 2);
+          qtail = ld_relaxed(p.wk.ctrl + 3);
+        }
+        if (qhead < qtail) {
+          if (atomicCAS(p.wk.ctrl + 2, qhead, qhead + 1u) == qhead) {
+            int4* e = p.wk.tq + qhead;
+            const long long t1 = clock64();
+            while (ld_acquire(reinterpret_cast<const unsigned*>(&e->w)) != qhead + 1u) {
+              if (misc[0] || clock64() - t1 > FZ_WAIT_CYCLES) {
+                set_status(p.status, HHR_ERR_TIMEOUT);
+                misc[0] = 1;
+                break;
+              }
+            }
+            dec[4] = e->x;
+            dec[5] = e->y;
+            dec[6] = e->z;
+            e->w = 0;  // the queue is clean for the next call
+            res = misc[0] ? 0 : 1;
+            break;
+          }
+          continue;
         }
         if (!ended) {
           if (mbar_test_wait(&s.dfull[d], dpar)) {
@@ -1712,10 +1790,13 @@ __device__ void fz_consumer(const FzParams& p, const FzShared& s) {
             break;
           }
         } else if (misc[5] == (int)nfin) {
-          // every request handled; a task posted by the last one is visible
-          // now (the finisher posts before it counts the request)
+          // Every request of this CTA is handled (tasks it made are in the
+          // queue).  Done when the queue is empty; a task posted later by
+          // another CTA is run there, at the latest by that CTA itself.
           __threadfence_block();
-          if (misc[3] == misc[2]) break;  // none pending: done
+          if (misc[3] != misc[2]) continue;
+          const unsigned h2 = ld_acquire(p.wk.ctrl + 2), t2 = ld_acquire(p.wk.ctrl + 3);
+          if (h2 >= t2) break;
           continue;
         }
         if (misc[0]) break;
@@ -1780,6 +1861,10 @@ __device__ void fz_consumer(const FzParams& p, const FzShared& s) {
       fz_gather<G>(p, s, x, ds.chunk, ds.n, d, s0);
     }
     // every consumer thread is done with the slots: release them and the descriptor
+    if (tid == 0) {  // the task queue's state, read now so the next poll need not wait for it
+      qhead = ld_relaxed(p.wk.ctrl + 2);
+      qtail = ld_relaxed(p.wk.ctrl + 3);
+    }
     cons_sync();
     if (tid == 0) {
       if (ds.gather) asm volatile("fence.proxy.async.shared::cta;" ::: "memory");  // before later bulk copies into the slots
@@ -1891,6 +1976,8 @@ __global__ void __launch_bounds__(FZ_THREADS, 1) hhr_fused_kernel(FzParams p) {
     if (tid == 0) {
       p.wk.ctrl[0] = 0u;
       p.wk.ctrl[1] = 0u;
+      p.wk.ctrl[2] = 0u;
+      p.wk.ctrl[3] = 0u;
     }
   }
 }
