@@ -63,6 +63,7 @@ hhr_status make_dims(const hhr_config* cfg, Dims* dm) {
   dm->Hkv = cfg->num_kv_heads;
   dm->G = G;
   dm->P = cfg->page_size;
+  dm->lgP = cfg->page_size == 16 ? 4 : 5;
   dm->nb = cfg->hash_bits;
   dm->words = cfg->hash_bits / 64;
   dm->T = cfg->max_seq_len;

@@ -14,6 +14,7 @@ constexpr int D = 128;  // head_dim: the only supported value
 // Problem dimensions passed by value to every kernel.
 struct Dims {
   int B, Hq, Hkv, G, P, nb, words, T, np_max, paged, num_blocks, max_blocks;
+  int lgP;  // log2 of the page size (a power of two)
 };
 
 // Workspace carve-out of one decode step (device pointers).
@@ -94,9 +95,9 @@ __device__ __forceinline__ int seq_len_of(const Dims& dm, const int* __restrict_
 __device__ __forceinline__ long long kv_row(const Dims& dm, const int* __restrict__ table,
                                             int b, int h, int t, int* status) {
   if (!dm.paged) return ((long long)(b * dm.Hkv + h) * dm.T + t) * D;
-  const int blk = __ldg(table + (long long)b * dm.max_blocks + t / dm.P);
+  const int blk = __ldg(table + (long long)b * dm.max_blocks + (t >> dm.lgP));
   if ((unsigned)blk >= (unsigned)dm.num_blocks) { set_status(status, HHR_ERR_BAD_BLOCK); return -1; }
-  return (((long long)blk * dm.Hkv + h) * dm.P + (t % dm.P)) * D;
+  return (((long long)blk * dm.Hkv + h) * dm.P + (t & (dm.P - 1))) * D;
 }
 
 // Element offset of page p's metadata row (page_min / page_max).
@@ -112,9 +113,9 @@ __device__ __forceinline__ long long meta_row(const Dims& dm, const int* __restr
 __device__ __forceinline__ long long code_row(const Dims& dm, const int* __restrict__ table,
                                               int b, int h, int t, int* status) {
   if (!dm.paged) return ((long long)(b * dm.Hkv + h) * dm.T + t) * dm.words;
-  const int blk = __ldg(table + (long long)b * dm.max_blocks + t / dm.P);
+  const int blk = __ldg(table + (long long)b * dm.max_blocks + (t >> dm.lgP));
   if ((unsigned)blk >= (unsigned)dm.num_blocks) { set_status(status, HHR_ERR_BAD_BLOCK); return -1; }
-  return (((long long)blk * dm.Hkv + h) * dm.P + (t % dm.P)) * dm.words;
+  return (((long long)blk * dm.Hkv + h) * dm.P + (t & (dm.P - 1))) * dm.words;
 }
 
 // --- block-wide exclusive scan of one int (blockDim multiple of 32, <= 1024) --

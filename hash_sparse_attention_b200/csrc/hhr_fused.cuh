@@ -325,7 +325,7 @@ __device__ __forceinline__ Unit unit_of(const FzParams& p, const FzShared& s, in
   x.b = u / p.dm.Hkv;
   x.h = u - x.b * p.dm.Hkv;
   x.L = x.b < FZ_SEQ ? s.seqp[x.b] : seq_len_of(p.dm, p.seq_lens, x.b);
-  x.np = (x.L + p.dm.P - 1) / p.dm.P;
+  x.np = (x.L + p.dm.P - 1) >> p.dm.lgP;
   return x;
 }
 
@@ -1047,8 +1047,10 @@ static_assert(PS_PER == 16, "page select layout");
 // Bin of a bound: monotone non-decreasing in the value, so the N-th largest
 // lies in one bin and every larger bin is kept whole.
 __device__ __forceinline__ int value_bin(float v, float lo, float scale) {
-  const float t = (v - lo) * scale;
-  return min(SEL_NBIN - 1, max(0, (int)t));
+  // nearest integer by the 1.5 * 2^23 addition (monotone, and cheaper than a
+  // conversion instruction; members lie in [0, SEL_NBIN])
+  const float t = fminf(fmaxf((v - lo) * scale, 0.f), (float)(SEL_NBIN - 1));
+  return __float_as_int(t + 12582912.0f) - 0x4B400000;
 }
 
 static __device__ void fz_psel(const FzParams& p, const FzShared& s, const Unit& x) {
@@ -1248,7 +1250,7 @@ __device__ void fz_score(const FzParams& p, const FzShared& s, const Unit& x, in
 #pragma unroll
   for (int r = 0; r < NR; ++r) {
     const int j = r * FZ_CONS + tid;
-    const int jp = j / dm.P, jr = j - jp * dm.P;
+    const int jp = j >> dm.lgP, jr = j & (dm.P - 1);
     const int woff = j < n ? ridx[jp] : -1;
     valid[r] = woff >= 0 && jr < ridx[FZ_ROWS / 2 + jp];
 #pragma unroll
@@ -1390,8 +1392,7 @@ __device__ void fz_ksel(const FzParams& p, const FzShared& s, const Unit& x) {
       const bool take = lt || (eq && eq_before < need_eq);
       const int pos = lt_b + __popc(blt & lanemask_lt) + min(eq_before, need_eq);
       if (take && pos < keff) {  // (pos < keff always holds; keeps the stores inside the list)
-        const int slot = ci / dm.P;
-        const int t = spage[slot] * dm.P + (ci - slot * dm.P);
+        const int t = (spage[ci >> dm.lgP] << dm.lgP) + (ci & (dm.P - 1));
         out[pos] = t;
         if (dout) dout[pos] = t;
       }
