@@ -166,6 +166,38 @@ class ClockSampler:
                 "reasons": sorted(reasons), "samples": len(sm)}
 
 
+def kernel_source_hash() -> str:
+    """sha256 over the CUDA sources of the library (any edit changes it)."""
+    import hashlib
+    csrc = os.path.join(ROOT, "hash_sparse_attention_b200", "csrc")
+    h = hashlib.sha256()
+    for name in sorted(os.listdir(csrc)):
+        if name.endswith((".cu", ".cuh", ".h")):
+            with open(os.path.join(csrc, name), "rb") as f:
+                h.update(name.encode() + b"\0" + f.read())
+    return h.hexdigest()
+
+
+def profiled_traffic(workload: str):
+    """DRAM bytes per hhr_fused_kernel launch from the committed ncu summary,
+    when that summary was taken on the current sources (else None)."""
+    path = os.path.join(ROOT, "profiles", "hhr_fused_kernel_llama_32l_128k.md")
+    if not os.path.exists(path):
+        return None
+    fields = {}
+    with open(path) as f:
+        for line in f:
+            if line.startswith("- ") and ": " in line:
+                k, v = line[2:].split(": ", 1)
+                fields[k.strip()] = v.strip().strip("`")
+    try:
+        if fields.get("sources_sha256") != kernel_source_hash() or fields.get("workload") != workload:
+            return None
+        return float(fields["dram_bytes_per_launch"])
+    except (KeyError, ValueError):
+        return None
+
+
 def peaks() -> dict:
     path = os.path.join(ROOT, "MEASURED_PEAKS.json")
     if os.path.exists(path):
@@ -387,7 +419,8 @@ def run_hhr(args, rank, world):
     mean_layer_s = t_step / len(layers)
     achieved = statistics.mean(per_layer_bytes) / mean_layer_s / 1e9
     roofline = {"bound": "hbm", "achieved": achieved, "peak": pk["hbm_gbs"], "unit": "GB/s",
-                "frac": achieved / pk["hbm_gbs"], "traffic": None,
+                "frac": achieved / pk["hbm_gbs"], "traffic": profiled_traffic(w.name),
+                "algorithmic_bytes_per_launch": statistics.mean(per_layer_bytes),
                 "kernel": "hhr_fused_kernel (one launch per layer: query prep, page scan, page and key select, "
                           "sparse attention, partial merges)",
                 "peak_source": pk["source"],
