@@ -179,9 +179,9 @@ def kernel_source_hash() -> str:
 
 
 def profiled_traffic(workload: str):
-    """DRAM bytes per hhr_fused_kernel launch from the committed ncu summary,
+    """DRAM bytes per hhr_group_kernel launch from the committed ncu summary,
     when that summary was taken on the current sources (else None)."""
-    path = os.path.join(ROOT, "profiles", "hhr_fused_kernel_llama_32l_128k.md")
+    path = os.path.join(ROOT, "profiles", "hhr_group_kernel_llama_32l_128k.md")
     if not os.path.exists(path):
         return None
     fields = {}
@@ -421,11 +421,11 @@ def run_hhr(args, rank, world):
     roofline = {"bound": "hbm", "achieved": achieved, "peak": pk["hbm_gbs"], "unit": "GB/s",
                 "frac": achieved / pk["hbm_gbs"], "traffic": profiled_traffic(w.name),
                 "algorithmic_bytes_per_launch": statistics.mean(per_layer_bytes),
-                "kernel": "hhr_fused_kernel (one launch per layer: query prep, page scan, page and key select, "
-                          "sparse attention, partial merges)",
+                "kernel": "hhr_group_kernel (one launch per layer; one group of CTAs per KV head: query prep, "
+                          "page scan, distributed page and key select, sparse attention, chunk-partial merge)",
                 "peak_source": pk["source"],
                 "step_gbs": step_bytes / t_step / 1e9, "step_frac": step_bytes / t_step / 1e9 / pk["hbm_gbs"]}
-    launches_per_step = len(layers)  # one hhr_fused_kernel launch per layer
+    launches_per_step = len(layers)  # one hhr_group_kernel launch per layer
     result = {
         "metric": METRIC,
         "value": whole_job_throughput(B * args.steps, world, secs_max),

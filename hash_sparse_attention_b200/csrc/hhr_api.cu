@@ -1,5 +1,5 @@
 // C ABI of libhhr.so: argument validation, workspace carve-out and launches.
-// The kernels live in hhr_build.cuh and hhr_fused.cuh.
+// The kernels live in hhr_build.cuh, hhr_fused.cuh (dense) and hhr_group.cuh (decode step).
 #include <algorithm>
 #include <cstdarg>
 #include <cstdio>
@@ -118,6 +118,9 @@ size_t carve(const Dims& dm, int Nmax, int Kmax, bool dense, char* base, Work* w
   const int Cmax = Nmax * dm.P;
   const int HB = (dm.G * dm.nb + 1 + 7) / 8 * 8;
   if (!dense) {
+    // group kernel: per-unit exchange areas
+    w.gx_stride = (GROUP_GX_FIXED_WORDS + HB + 3) / 4 * 4;
+    w.gx = reinterpret_cast<unsigned*>(take(sizeof(unsigned) * BH * w.gx_stride));
     w.U = reinterpret_cast<float*>(take(sizeof(float) * BH * Ustride));
     w.sel_pages = reinterpret_cast<int*>(take(sizeof(int) * BH * Nmax));
     w.sel_keys = reinterpret_cast<int*>(take(sizeof(int) * BH * Kmax));

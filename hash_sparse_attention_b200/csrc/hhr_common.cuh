@@ -32,6 +32,7 @@ struct Work {
   uint16_t* kscore;    // [B, Hkv, Cmax]    Hamming score of every candidate row
   int* khist;          // [B, Hkv, HB]      score histogram (kept at zero between calls)
   int4* tq;            // [tq_cap]          task queue: (kind, unit, arg, sequence + 1), zero between calls
+  unsigned* gx;        // [B * Hkv, gx_stride] per-unit exchange areas of the CTA groups
   unsigned* ctrl;      // [4 + B * Hkv * (8 + max_groups)] item queue, exit count, task queue head / tail, flags, counters
   int Nmax, Kmax;      // budgets the workspace was sized for
   int Cmax;            // Nmax * page size: candidate rows per unit
@@ -40,6 +41,7 @@ struct Work {
   int C1, C2, C3;      // scan, score and gather chunks per unit
   int max_groups;      // groups of 16 gather chunks per unit
   int tq_cap;          // task queue entries (every task of one call fits)
+  int gx_stride;       // 32-bit words per unit exchange area
 };
 
 // --- bf16 ---------------------------------------------------------------

@@ -235,6 +235,7 @@ struct FzParams {
   int items_per_unit_score;   // C2 (sparse) or 0 (dense)
   int items_per_unit_gather;  // C3
   int total_items;
+  int gsize, ngroups;         // group kernel: CTAs per group, groups
 };
 
 struct FzShared {
@@ -1577,15 +1578,15 @@ __device__ void fz_gather(const FzParams& p, const FzShared& s, const Unit& x, i
 // taking every NPART-th partial (loads issued before the weights are known);
 // the group sums are then added in group order.
 template <int G>
-__device__ void fz_merge(const FzShared& s, const float* src, int K, float* dst, float* out) {
+__device__ void merge_partials(unsigned char* work, const float* src, int K, float* dst, float* out) {
   constexpr int NOUT = G * 32;  // float4 outputs
   constexpr int NPART = FZ_CONS / NOUT >= 4 ? 4 : FZ_CONS / NOUT;
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
   const int PS = G * D + 16;
-  float* wsm = reinterpret_cast<float*>(s.work);            // [256][G] weights
-  float* MH = reinterpret_cast<float*>(s.work + 8192);      // [8]
-  float* LH = MH + 8;                                        // [8]
-  float4* psum = reinterpret_cast<float4*>(s.work + 16384);  // [NPART][NOUT]
+  float* wsm = reinterpret_cast<float*>(work);            // [256][G] weights
+  float* MH = reinterpret_cast<float*>(work + 8192);      // [8]
+  float* LH = MH + 8;                                      // [8]
+  float4* psum = reinterpret_cast<float4*>(work + 16384);  // [NPART][NOUT]
   cons_sync();  // the work area's previous readers are done
   const int f = tid % NOUT, part = tid / NOUT;
   const int g = f >> 5, c4 = f & 31;
@@ -1675,6 +1676,10 @@ __device__ void fz_merge(const FzShared& s, const float* src, int K, float* dst,
     dst[G * D + tid] = MH[tid];
     dst[G * D + 8 + tid] = LH[tid];
   }
+}
+template <int G>
+__device__ __forceinline__ void fz_merge(const FzShared& s, const float* src, int K, float* dst, float* out) {
+  merge_partials<G>(s.work, src, K, dst, out);
 }
 
 // ---------------------------------------------------------------------------
@@ -2027,18 +2032,6 @@ static FzParams make_params(const DecodeArgs& a, bool dense) {
   prm.items_per_unit_gather = a.wk.C3;
   prm.total_items = U * (1 + prm.items_per_unit_scan + prm.items_per_unit_score + prm.items_per_unit_gather);
   return prm;
-}
-
-template <int G>
-cudaError_t launch_decode(const DecodeArgs& a) {
-  const FzParams prm = make_params(a, false);
-  const int grid = std::min(a.num_sms, prm.total_items);
-  switch (a.dm.words) {
-    case 1: return launch_fused_t<G, 1, false>(prm, grid, a.stream);
-    case 2: return launch_fused_t<G, 2, false>(prm, grid, a.stream);
-    case 4: return launch_fused_t<G, 4, false>(prm, grid, a.stream);
-  }
-  return cudaErrorInvalidValue;
 }
 
 template <int G>

@@ -1,0 +1,1236 @@
+// HHR decode step with CTA groups: one group of S CTAs per unit (sequence b,
+// KV head h), every CTA of a group owning a contiguous share of the unit's
+// pages and, after the selects, a balanced share of its kept rows (sm_100a).
+//
+// Per unit, CTA r of the group:
+//   1. computes q' = R_h q and the query sign codes itself (R_h, W_h and q are
+//      read by every CTA of the group; the copies after the first hit L2),
+//      while its producer warp already streams the page metadata of its share
+//      into the shared-memory ring;
+//   2. scans its pages: U = max over the group's heads of the page bound;
+//   3. page top-N, distributed: the group agrees on the global value range,
+//      bins its bounds (2048 bins per level, counts added in L2), descends
+//      into the bin that holds the N-th largest and ranks that bin's members
+//      exactly (larger bound first, then the lower page);
+//   4. scores the rows of the pages it kept (Hamming distance summed over the
+//      group's heads), adds their histogram in L2; the threshold score and the
+//      ties every CTA may take follow from the histogram and the per-CTA
+//      counts (CTAs own ascending page ranges, so CTA order is row order);
+//   5. writes its kept rows at their place in the unit's row list and, after
+//      one more group barrier, gathers the K'/V rows of its share of that
+//      list's chunks of 128 rows (cp.async by the consumer warps, one chunk
+//      ahead), one softmax partial per chunk;
+//   6. the last CTA of the group to arrive merges the chunk partials in chunk
+//      order into the output and clears the unit's counters (the result does
+//      not depend on the number of CTAs per group).
+// A group barrier is an acquire-release counter in the workspace: every CTA
+// adds 1 after a CTA barrier, then waits (bounded) for S per barrier passed.
+// All of a group's CTAs are resident at once (one CTA per SM, grid <= SMs).
+#pragma once
+
+#include "hhr_fused.cuh"
+
+namespace hhr {
+
+constexpr int GP_WORK = 90112;                 // consumer scratch
+constexpr int GP_SMAX = MAX_GRID;              // CTAs per group at most
+constexpr int GP_LEVELS = 4;                   // page select levels
+constexpr int GP_PAGES_PER_SLOT = 32;          // a ring slot: 32 pages of minima, then their maxima
+constexpr size_t GP_OFF_RING = 0;
+constexpr size_t GP_OFF_WORK = GP_OFF_RING + (size_t)FZ_NSLOT * FZ_SLOT;
+constexpr size_t GP_OFF_QS = GP_OFF_WORK + GP_WORK;   // q' fp32 [8][128] (quad-permuted)
+constexpr size_t GP_OFF_QC = GP_OFF_QS + 8 * D * 4;   // query codes u32 [8][8]
+constexpr size_t GP_OFF_RIDX = GP_OFF_QC + 256;       // row numbers of two gather steps [2][128]
+constexpr size_t GP_OFF_BAR = GP_OFF_RIDX + 2 * FZ_ROWS * 4;
+constexpr size_t GP_OFF_MISC = GP_OFF_BAR + 8 * (2 * FZ_NSLOT);
+constexpr size_t GP_SMEM = GP_OFF_MISC + 256;
+static_assert(GP_SMEM <= 232448, "shared memory of the group kernel");
+
+// consumer scratch during the scan and the selects (the gather reuses it all)
+constexpr int GW_US = 0;                       // float [8192] bounds of the CTA's pages
+constexpr int GW_HIST = 32768;                 // int [2056] value bins / score histogram
+constexpr int GW_CAND = GW_HIST + 8448;        // int2 [512] members of the threshold bin
+constexpr int GW_FLAG = GW_CAND + 4096;        // u32 [256] kept members (bitmap over local pages)
+constexpr int GW_RED = GW_FLAG + 1024;         // int [256] scan scratch and broadcasts
+constexpr int GW_KP = GW_RED + 1024;           // int [2048] kept pages (ascending)
+constexpr int GW_SC = GW_KP + 8192;            // uint16 [16384] scores of the candidate rows
+static_assert(GW_SC + 2 * MAX_CANDIDATES <= GP_WORK, "group kernel scratch");
+static_assert(MAX_SELECT_PAGES * 4 <= GW_HIST && FZ_HIST_BINS * 4 <= 8448, "group kernel scratch");
+static_assert(GA_LB + 512 <= GP_WORK, "gather scratch");
+
+// Per-unit exchange area in the workspace (32-bit words).  The counters and
+// histograms are zero between units (the merging CTA clears them); the rest
+// is written before it is read.
+enum : int {
+  GX_BAR = 0,     // group barrier arrivals
+  GX_ARRIVE = 1,  // partials published
+  GX_CCOUNT = 2,  // members in the candidate list
+  GX_MM = 4,                                        // float2 [levels][SMAX] member range per CTA
+  GX_PUB4 = GX_MM + 2 * GP_LEVELS * GP_SMAX,        // int2 [SMAX] kept pages, valid candidates
+  GX_PUB5 = GX_PUB4 + 2 * GP_SMAX,                  // int2 [SMAX] rows below the threshold, ties
+  GX_PUBT = GX_PUB5 + 2 * GP_SMAX,                  // int [SMAX] members (equal bounds)
+  GX_HIST = GX_PUBT + GP_SMAX,                      // int [levels][2048]
+  GX_CAND = GX_HIST + GP_LEVELS * SEL_NBIN,         // int2 [512] (bound bits, page)
+  GX_KHIST = GX_CAND + 2 * SEL_MAX_CAND,            // int [HB] score histogram
+};
+// words of one unit's area before the partials (the score histogram is HB long)
+__host__ __device__ constexpr int gx_head_words(int HB) { return (GX_KHIST + HB + 3) / 4 * 4; }
+
+struct GpShared {
+  unsigned char* ring;
+  unsigned char* work;
+  float* qs;
+  unsigned* qc;
+  int* ridx;
+  uint64_t* full;
+  uint64_t* empty;
+  int* misc;        // [0] abort, [1] slots consumed, [2] slots armed, [17], [18] broadcasts,
+                    // [20] units whose ring use the consumers have finished
+};
+
+__device__ __forceinline__ GpShared gp_shared(unsigned char* base) {
+  GpShared s;
+  s.ring = base + GP_OFF_RING;
+  s.work = base + GP_OFF_WORK;
+  s.qs = reinterpret_cast<float*>(base + GP_OFF_QS);
+  s.qc = reinterpret_cast<unsigned*>(base + GP_OFF_QC);
+  s.ridx = reinterpret_cast<int*>(base + GP_OFF_RIDX);
+  uint64_t* bars = reinterpret_cast<uint64_t*>(base + GP_OFF_BAR);
+  s.full = bars;
+  s.empty = bars + FZ_NSLOT;
+  s.misc = reinterpret_cast<int*>(base + GP_OFF_MISC);
+  return s;
+}
+
+// Bounded mbarrier wait for the group kernel (abort flag in misc[0]).
+__device__ __forceinline__ bool gp_wait(const GpShared& s, uint64_t* bar, uint32_t parity, int* status) {
+  if (mbar_try_wait(bar, parity)) return true;
+  const long long t0 = clock64();
+  while (true) {
+    if (mbar_try_wait(bar, parity)) return true;
+    if (*reinterpret_cast<volatile int*>(s.misc)) return false;
+    if (clock64() - t0 > FZ_WAIT_CYCLES) {
+      set_status(status, HHR_ERR_TIMEOUT);
+      *reinterpret_cast<volatile int*>(s.misc) = 1;
+      return false;
+    }
+  }
+}
+
+__device__ __forceinline__ void red_release_add(unsigned* p, unsigned v) {
+  asm volatile("red.release.gpu.global.add.u32 [%0], %1;" ::"l"(p), "r"(v) : "memory");
+}
+
+// Group of unit u's CTAs: the unit's exchange area.
+__device__ __forceinline__ unsigned* gx_of(const FzParams& p, int u) { return p.wk.gx + (long long)u * p.wk.gx_stride; }
+
+// Pages [p0, p1) of CTA r among S for a unit of np pages.
+__device__ __forceinline__ void share_of(int n, int S, int r, int& a, int& b) {
+  a = (int)(((long long)n * r) / S);
+  b = (int)(((long long)n * (r + 1)) / S);
+}
+
+
+// Group barrier among the consumer threads of the group's S CTAs.  Every
+// consumer thread calls it; writes made before it by any thread of the group
+// are visible after it (read them with ld.global.cg: L1 is not coherent).
+// False after a timeout or an abort (then every thread of the CTA sees false).
+__device__ __forceinline__ bool gp_sync(const FzParams& p, const GpShared& s, unsigned* gx, unsigned& epoch) {
+  cons_sync();
+  if (p.gsize == 1) return *reinterpret_cast<volatile int*>(s.misc) == 0;  // a CTA barrier suffices
+  epoch += (unsigned)p.gsize;
+  if (threadIdx.x == 0) {
+    volatile int* ab = s.misc;
+    red_release_add(gx + GX_BAR, 1u);
+    if (ld_acquire(gx + GX_BAR) < epoch) {
+      const long long t0 = clock64();
+      while (ld_acquire(gx + GX_BAR) < epoch) {
+        if (*ab) break;
+        if (clock64() - t0 > FZ_WAIT_CYCLES) {
+          set_status(p.status, HHR_ERR_TIMEOUT);
+          *ab = 1;
+          break;
+        }
+      }
+    }
+  }
+  cons_sync();
+  return *reinterpret_cast<volatile int*>(s.misc) == 0;
+}
+
+// ---------------------------------------------------------------------------
+// producer (warp 16): streams the page metadata of the CTA's share of every
+// unit of its group into the ring, 32 pages per slot (minima, then maxima)
+// ---------------------------------------------------------------------------
+static __device__ void gp_producer(const FzParams& p, const GpShared& s, int g, int r) {
+  const int lane = threadIdx.x & 31;
+  const Dims& dm = p.dm;
+  const int U = dm.B * dm.Hkv, S = p.gsize;
+  const uint64_t ef = evict_first_policy();
+  unsigned nslot = 0, nunit = 0;
+  for (int u = g; u < U; u += p.ngroups, ++nunit) {
+    if (nunit > 0) {  // the consumers are done with the ring (gather of the previous unit)
+      bool ok = true;
+      if (lane == 0) {
+        volatile int* rel = s.misc + 20;  // units the consumers have released
+        if (*rel < (int)nunit) {
+          const long long t0 = clock64();
+          while (*rel < (int)nunit) {
+            if (*reinterpret_cast<volatile int*>(s.misc)) {
+              ok = false;
+              break;
+            }
+            if (clock64() - t0 > FZ_WAIT_CYCLES) {
+              set_status(p.status, HHR_ERR_TIMEOUT);
+              *reinterpret_cast<volatile int*>(s.misc) = 1;
+              ok = false;
+              break;
+            }
+          }
+        }
+      }
+      if (__shfl_sync(0xffffffffu, (int)ok, 0) == 0) break;
+    }
+    const int b = u / dm.Hkv, h = u - b * dm.Hkv;
+    const int L = seq_len_of(dm, p.seq_lens, b);
+    const int np = (L + dm.P - 1) >> dm.lgP;
+    int p0, p1;
+    share_of(np, S, r, p0, p1);
+    bool aborted = false;
+    for (int j0 = p0; j0 < p1; j0 += GP_PAGES_PER_SLOT) {
+      const int n = min(GP_PAGES_PER_SLOT, p1 - j0);
+      const int slot = (int)(nslot % FZ_NSLOT);
+      if (nslot >= FZ_NSLOT) {
+        bool ok = true;
+        if (lane == 0) ok = gp_wait(s, &s.empty[slot], ((nslot / FZ_NSLOT) - 1) & 1, p.status);
+        if (__shfl_sync(0xffffffffu, (int)ok, 0) == 0) {
+          aborted = true;
+          break;
+        }
+      }
+      unsigned char* dst = s.ring + (size_t)slot * FZ_SLOT;
+      if (!dm.paged) {
+        if (lane == 0) {
+          const long long off = ((long long)(b * dm.Hkv + h) * dm.np_max + j0) * D;
+          mbar_arrive_expect_tx(&s.full[slot], (uint32_t)(2 * n * 256));
+          bulk_g2s_stream(dst, p.pmin + off, (uint32_t)(n * 256), &s.full[slot], ef);
+          bulk_g2s_stream(dst + FZ_SLOT / 2, p.pmax + off, (uint32_t)(n * 256), &s.full[slot], ef);
+        }
+      } else {
+        // one page per lane; a bad block id reads as zero rows
+        int blk = -1;
+        bool ok = false;
+        if (lane < n) {
+          blk = __ldg(p.table + (long long)b * dm.max_blocks + j0 + lane);
+          ok = (unsigned)blk < (unsigned)dm.num_blocks;
+          if (!ok) {
+            set_status(p.status, HHR_ERR_BAD_BLOCK);
+            uint4* z0 = reinterpret_cast<uint4*>(dst + lane * 256);
+            uint4* z1 = reinterpret_cast<uint4*>(dst + FZ_SLOT / 2 + lane * 256);
+#pragma unroll
+            for (int i = 0; i < 16; ++i) z0[i] = z1[i] = make_uint4(0u, 0u, 0u, 0u);
+          }
+        }
+        const unsigned okm = __ballot_sync(0xffffffffu, ok);
+        if (lane == 0) mbar_arrive_expect_tx(&s.full[slot], (uint32_t)(__popc(okm) * 512));
+        __syncwarp();
+        if (ok) {
+          const long long off = ((long long)blk * dm.Hkv + h) * D;
+          bulk_g2s_stream(dst + lane * 256, p.pmin + off, 256u, &s.full[slot], ef);
+          bulk_g2s_stream(dst + FZ_SLOT / 2 + lane * 256, p.pmax + off, 256u, &s.full[slot], ef);
+        }
+      }
+      __syncwarp();
+      ++nslot;
+      if (lane == 0) s.misc[2] = (int)nslot;  // slots armed (drained at exit after an abort)
+    }
+    if (aborted) break;
+  }
+}
+
+// ---- PREP: q' = R_h q and the query codes, read straight from global memory ----
+// Same arithmetic as the fused kernel's query preparation: q' rows reduced by
+// a transposed butterfly; code bits from fp32 sums with an fp64 recompute
+// whenever |sum| <= 2^-14 sum |w q| (the sign is then exact).
+template <int G>
+__device__ void gp_prep(const FzParams& p, const GpShared& s, const Unit& x, bool write_dbg) {
+  constexpr int GP = G <= 4 ? 4 : 8;
+  const Dims& dm = p.dm;
+  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+  float* qf = reinterpret_cast<float*>(s.work);  // [G][128] q in natural order
+  const __nv_bfloat16* qg = p.q + ((long long)x.b * dm.Hq + x.h * G) * D;
+  // R_h rows 8w .. 8w+7 of this warp (lane: channels 4l .. 4l+3), issued first
+  const float* Rh = p.R + (long long)x.h * D * D;
+  float4 rr[8];
+#pragma unroll
+  for (int k = 0; k < 8; ++k) rr[k] = __ldg(reinterpret_cast<const float4*>(Rh + (long long)(warp * 8 + k) * D) + lane);
+  for (int i = tid; i < G * D; i += FZ_CONS) qf[i] = __bfloat162float(qg[i]);
+  if (tid < 64) s.qc[tid] = 0u;
+  cons_sync();
+  float qv[G][4];
+#pragma unroll
+  for (int g = 0; g < G; ++g) {
+    const float4 t = *reinterpret_cast<const float4*>(qf + g * D + 4 * lane);
+    qv[g][0] = t.x; qv[g][1] = t.y; qv[g][2] = t.z; qv[g][3] = t.w;
+  }
+  {
+    constexpr int NV = 8 * GP, KP = NV / 32;
+    float v[NV];
+#pragma unroll
+    for (int k = 0; k < 8; ++k)
+#pragma unroll
+      for (int g = 0; g < GP; ++g) v[k * GP + g] = (g < G) ? dot4(rr[k], qv[g]) : 0.f;
+    warp_reduce_t<NV>(v, lane);
+#pragma unroll
+    for (int e = 0; e < KP; ++e) {
+      const int vi = KP * lane + e;
+      const int k = vi / GP, g = vi % GP;
+      if (g < G) {
+        const int i = warp * 8 + k;
+        s.qs[g * D + qpos(i)] = v[e];
+        if (write_dbg && p.dbg.q_rot) p.dbg.q_rot[((long long)x.b * dm.Hq + x.h * G + g) * D + i] = v[e];
+      }
+    }
+  }
+  // query codes: warp w takes bits [w nb/16, (w+1) nb/16) in blocks of NBB
+  constexpr int NBB = 32 / GP;
+  const int bpw = dm.nb / FZ_CWARPS;
+  const __nv_bfloat16* Wh = p.W + (long long)x.h * dm.nb * D;
+  for (int jb = 0; jb < bpw; jb += NBB) {
+    float v[2 * NBB * GP];
+    uint2 wv[NBB];
+#pragma unroll
+    for (int bb = 0; bb < NBB; ++bb) {
+      const int j = warp * bpw + jb + bb;
+      wv[bb] = (jb + bb < bpw) ? __ldg(reinterpret_cast<const uint2*>(Wh + (long long)j * D) + lane) : make_uint2(0u, 0u);
+    }
+#pragma unroll
+    for (int bb = 0; bb < NBB; ++bb) {
+      const float w4[4] = {bf_lo(wv[bb].x), bf_hi(wv[bb].x), bf_lo(wv[bb].y), bf_hi(wv[bb].y)};
+#pragma unroll
+      for (int g = 0; g < GP; ++g) {
+        float a = 0.f, m = 0.f;
+        if (g < G) {
+#pragma unroll
+          for (int e = 0; e < 4; ++e) {
+            const float pe = w4[e] * qv[g][e];
+            a += pe;
+            m += fabsf(pe);
+          }
+        }
+        v[(bb * GP + g) * 2 + 0] = a;
+        v[(bb * GP + g) * 2 + 1] = m;
+      }
+    }
+    warp_reduce_t<2 * NBB * GP>(v, lane);
+    const int bb = lane / GP, g = lane % GP;
+    const int j = warp * bpw + jb + bb;
+    if (g < G && jb + bb < bpw) {
+      bool bit = v[0] > 0.f;
+      if (fabsf(v[0]) <= ldexpf(v[1], -14)) {
+        double ad = 0.0;
+        const __nv_bfloat16* wrow = Wh + (long long)j * D;
+        for (int c = 0; c < D; ++c) ad += (double)__bfloat162float(wrow[c]) * (double)qf[g * D + c];
+        bit = ad > 0.0;
+      }
+      if (bit) atomicOr(&s.qc[g * 8 + j / 32], 1u << (j % 32));
+    }
+  }
+  cons_sync();
+  if (write_dbg && p.dbg.q_codes) {
+    const int w32 = dm.words * 2;
+    if (tid < G * w32) {
+      const int g = tid / w32, k = tid - g * w32;
+      reinterpret_cast<uint32_t*>(p.dbg.q_codes)[((long long)x.b * dm.Hq + x.h * G + g) * w32 + k] = s.qc[g * 8 + k];
+    }
+  }
+}
+
+// ---- SCAN: bounds of up to 128 pages of the CTA's share ----
+// As the fused kernel's scan (half a warp per page, lane: 8 channels), with
+// the ring layout of the group kernel: page j of the step in slot
+// sb + j / 32, its minima at row j % 32 and its maxima half a slot further.
+template <int G>
+__device__ void gp_scan(const FzParams& p, const GpShared& s, const Unit& x, int pg0, int n, int sb, float* Us) {
+  constexpr int GP = G <= 4 ? 4 : 8;
+  constexpr bool SPLIT = G <= 4;
+  constexpr int PB = GP == 4 ? 4 : 2;
+  constexpr int NBT = 4 / PB;
+  constexpr int NV = PB * GP;
+  const Dims& dm = p.dm;
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+  const int hw = lane >> 4, li = lane & 15;
+  float2 qa[G][4], qb[G][4];
+#pragma unroll
+  for (int g = 0; g < G; ++g) {
+#pragma unroll
+    for (int k = 0; k < 2; ++k) {
+      const float4 t = *reinterpret_cast<const float4*>(s.qs + g * D + 4 * (li + 16 * k));
+      if constexpr (SPLIT) {
+        qa[g][2 * k] = make_float2(fmaxf(t.x, 0.f), fmaxf(t.y, 0.f));
+        qa[g][2 * k + 1] = make_float2(fmaxf(t.z, 0.f), fmaxf(t.w, 0.f));
+        qb[g][2 * k] = make_float2(fminf(t.x, 0.f), fminf(t.y, 0.f));
+        qb[g][2 * k + 1] = make_float2(fminf(t.z, 0.f), fminf(t.w, 0.f));
+      } else {
+        qa[g][2 * k] = make_float2(t.x, t.y);
+        qa[g][2 * k + 1] = make_float2(t.z, t.w);
+      }
+    }
+  }
+  const int pl = li / GP, hidx = li % GP;
+#pragma unroll
+  for (int bt = 0; bt < NBT; ++bt) {
+    float v[NV];
+#pragma unroll
+    for (int pp = 0; pp < PB; ++pp) {
+      const int j = warp * 8 + hw * 4 + bt * PB + pp;
+      const unsigned char* slot = s.ring + (size_t)((sb + j / GP_PAGES_PER_SLOT) % FZ_NSLOT) * FZ_SLOT;
+      const size_t off = (size_t)(j % GP_PAGES_PER_SLOT) * 256 + li * 16;
+      const uint4 mnv = *reinterpret_cast<const uint4*>(slot + off);
+      const uint4 mxv = *reinterpret_cast<const uint4*>(slot + FZ_SLOT / 2 + off);
+      const uint32_t mw[4] = {mnv.x, mnv.y, mnv.z, mnv.w};
+      const uint32_t xw[4] = {mxv.x, mxv.y, mxv.z, mxv.w};
+      float2 mn[4], mx[4];
+#pragma unroll
+      for (int k = 0; k < 4; ++k) {
+        mn[k] = make_float2(bf_lo(mw[k]), bf_hi(mw[k]));
+        mx[k] = make_float2(bf_lo(xw[k]), bf_hi(xw[k]));
+      }
+#pragma unroll
+      for (int g = 0; g < GP; ++g) {
+        float sum = 0.f;
+        if (g < G) {
+          float2 a0, a1;
+          if constexpr (SPLIT) {
+            a0 = __fmul2_rn(qa[g][0], mx[0]);
+            a1 = __fmul2_rn(qb[g][0], mn[0]);
+#pragma unroll
+            for (int k = 1; k < 4; ++k) {
+              a0 = __ffma2_rn(qa[g][k], mx[k], a0);
+              a1 = __ffma2_rn(qb[g][k], mn[k], a1);
+            }
+          } else {
+            float2 sel[4];
+#pragma unroll
+            for (int k = 0; k < 4; ++k)
+              sel[k] = make_float2(qa[g][k].x >= 0.f ? mx[k].x : mn[k].x, qa[g][k].y >= 0.f ? mx[k].y : mn[k].y);
+            a0 = __fmul2_rn(qa[g][0], sel[0]);
+            a1 = __fmul2_rn(qa[g][1], sel[1]);
+            a0 = __ffma2_rn(qa[g][2], sel[2], a0);
+            a1 = __ffma2_rn(qa[g][3], sel[3], a1);
+          }
+          sum = (a0.x + a0.y) + (a1.x + a1.y);
+        }
+        v[pp * GP + g] = sum;
+      }
+    }
+    group_reduce_t<NV, 16>(v, lane);
+    float U = hidx < G ? v[0] : -INFINITY;
+#pragma unroll
+    for (int o = 1; o < GP; o <<= 1) U = fmaxf(U, __shfl_xor_sync(0xffffffffu, U, o));
+    const int j = warp * 8 + hw * 4 + bt * PB + pl;
+    if (j < n) {
+      const int pg = pg0 + j;
+      if (hidx == 0) {
+        Us[j] = U;
+        if (p.dbg.page_U) p.dbg.page_U[(long long)x.u * dm.np_max + pg] = U;
+      }
+      if (p.dbg.page_ub && hidx < G)
+        p.dbg.page_ub[((long long)x.b * dm.Hq + x.h * G + hidx) * dm.np_max + pg] = v[0];
+    }
+  }
+}
+
+
+// ---- page top-N over the group (larger bound first, ties to the lower page) ----
+// Thread t holds the bounds of local pages [16 t, 16 t + 16).  A level agrees
+// on the members' value range (one group barrier), bins the members into
+// 2048 bins whose counts are added in L2 (one more), keeps every bin above
+// the one holding the need-th largest and descends into that bin.  A bin of
+// at most 512 members is ranked exactly against the whole group's members; a
+// bin of equal bounds (or one still crowded after four levels) is taken in
+// page order.  Returns the CTA's kept pages (ascending, in GW_KP).
+static __device__ int gp_psel(const FzParams& p, const GpShared& s, const Unit& x, int r, int p0, int nr, int N,
+                       unsigned* gx, unsigned& epoch, bool& ok) {
+  const int tid = threadIdx.x;
+  const int S = p.gsize;
+  unsigned char* w = s.work;
+  const float* Us = reinterpret_cast<const float*>(w + GW_US);
+  int* hist = reinterpret_cast<int*>(w + GW_HIST);
+  int2* cand = reinterpret_cast<int2*>(w + GW_CAND);
+  unsigned* flag = reinterpret_cast<unsigned*>(w + GW_FLAG);
+  int* red = reinterpret_cast<int*>(w + GW_RED);  // scan buffers of 16 at 0, 16, 32, 48, 64; broadcasts at 128
+  int* bc = red + 128;
+  float* wr = reinterpret_cast<float*>(red + 160);
+  int* kp = reinterpret_cast<int*>(w + GW_KP);
+  const int i0 = tid * PS_PER;
+  const int cnt = max(0, min(PS_PER, nr - i0));
+  unsigned member = (1u << cnt) - 1u;
+  float v[PS_PER];
+#pragma unroll
+  for (int k = 0; k < PS_PER; ++k) v[k] = k < cnt ? Us[i0 + k] : 0.f;
+  unsigned keep = 0u;
+  if (N >= x.np) {
+    keep = member;
+  } else {
+    int need = N, nbin = 0;
+    bool tie = false;
+#pragma unroll 1
+    for (int level = 0; level < GP_LEVELS; ++level) {
+      float lo = INFINITY, hi = -INFINITY;
+#pragma unroll
+      for (int k = 0; k < PS_PER; ++k)
+        if ((member >> k) & 1u) {
+          lo = fminf(lo, v[k]);
+          hi = fmaxf(hi, v[k]);
+        }
+      cons_minmax(lo, hi, wr);
+      float2* mm = reinterpret_cast<float2*>(gx + GX_MM) + level * GP_SMAX;
+      if (tid == 0) mm[r] = make_float2(lo, hi);
+      if (!gp_sync(p, s, gx, epoch)) {
+        ok = false;
+        return 0;
+      }
+      lo = INFINITY;
+      hi = -INFINITY;
+      if (tid < S) {
+        const float2 t = __ldcg(mm + tid);
+        lo = t.x;
+        hi = t.y;
+      }
+      cons_minmax(lo, hi, wr);
+      tie = !(hi > lo);
+      if (tie) break;
+      const float scale = (float)SEL_NBIN / (hi - lo);
+      for (int i = tid; i < SEL_NBIN; i += FZ_CONS) hist[i] = 0;
+      cons_sync();
+      int bn[PS_PER];
+#pragma unroll
+      for (int k = 0; k < PS_PER; ++k) {
+        bn[k] = value_bin(v[k], lo, scale);
+        if ((member >> k) & 1u) atomicAdd(&hist[bn[k]], 1);
+      }
+      cons_sync();
+      int* gh = reinterpret_cast<int*>(gx + GX_HIST) + level * SEL_NBIN;
+      for (int i = tid; i < SEL_NBIN; i += FZ_CONS) {
+        const int h = hist[i];
+        if (h) atomicAdd(gh + i, h);
+      }
+      if (!gp_sync(p, s, gx, epoch)) {
+        ok = false;
+        return 0;
+      }
+      {
+        constexpr int BPT = SEL_NBIN / FZ_CONS;  // 4 bins per thread, counted from the top
+        int hv[BPT];
+        int c4 = 0;
+#pragma unroll
+        for (int e = 0; e < BPT; ++e) {
+          hv[e] = __ldcg(gh + SEL_NBIN - 1 - (tid * BPT + e));
+          c4 += hv[e];
+        }
+        int tot;
+        const int before = cons_scan1(c4, red + 16 * (level & 1), &tot);
+        if (before < need && before + c4 >= need) {
+          int run = before;
+#pragma unroll
+          for (int e = 0; e < BPT; ++e) {
+            if (run < need && run + hv[e] >= need) {
+              bc[0] = SEL_NBIN - 1 - (tid * BPT + e);
+              bc[1] = need - run;
+              bc[2] = hv[e];
+            }
+            run += hv[e];
+          }
+        }
+        cons_sync();
+      }
+      const int bstar = bc[0];
+      need = bc[1];
+      nbin = bc[2];
+#pragma unroll
+      for (int k = 0; k < PS_PER; ++k) {
+        const bool m = (member >> k) & 1u;
+        keep |= (m && bn[k] > bstar) ? 1u << k : 0u;
+        member &= (m && bn[k] == bstar) ? ~0u : ~(1u << k);
+      }
+      if (nbin <= SEL_MAX_CAND) break;
+    }
+    if (tie || nbin > SEL_MAX_CAND) {
+      // equal bounds (or still crowded): members in page order, the first `need`
+      const int m = __popc(member);
+      int mt;
+      const int mb = cons_scan1(m, red + 32, &mt);
+      int* pubt = reinterpret_cast<int*>(gx + GX_PUBT);
+      if (tid == 0) pubt[r] = mt;
+      if (!gp_sync(p, s, gx, epoch)) {
+        ok = false;
+        return 0;
+      }
+      int tt;
+      const int bt = cons_scan1(tid < S ? __ldcg(pubt + tid) : 0, red + 48, &tt);
+      if (tid == r) bc[3] = bt;
+      cons_sync();
+      int take = max(0, min(m, need - bc[3] - mb));
+#pragma unroll
+      for (int k = 0; k < PS_PER; ++k) {
+        if (((member >> k) & 1u) && take > 0) {
+          keep |= 1u << k;
+          --take;
+        }
+      }
+    } else {
+      // exact ranking of the threshold bin's members across the group
+      int2* gc = reinterpret_cast<int2*>(gx + GX_CAND);
+      for (int i = tid; i < MAX_SELECT_PAGES / 32; i += FZ_CONS) flag[i] = 0u;
+#pragma unroll
+      for (int k = 0; k < PS_PER; ++k)
+        if ((member >> k) & 1u) {
+          const unsigned at = atomicAdd(gx + GX_CCOUNT, 1u);
+          if (at < (unsigned)SEL_MAX_CAND) gc[at] = make_int2(__float_as_int(v[k]), p0 + i0 + k);
+        }
+      if (!gp_sync(p, s, gx, epoch)) {
+        ok = false;
+        return 0;
+      }
+      for (int a = tid; a < nbin; a += FZ_CONS) cand[a] = __ldcg(gc + a);
+      cons_sync();
+      for (int a = tid; a < nbin; a += FZ_CONS) {
+        const int2 ea = cand[a];
+        const int pa = ea.y - p0;
+        if (pa >= 0 && pa < nr) {
+          const float va = __int_as_float(ea.x);
+          int rank = 0;
+          for (int b2 = 0; b2 < nbin; ++b2) {
+            const int2 eb = cand[b2];
+            const float vb = __int_as_float(eb.x);
+            rank += (vb > va) || (vb == va && eb.y < ea.y);
+          }
+          if (rank < need) atomicOr(&flag[pa >> 5], 1u << (pa & 31));
+        }
+      }
+      cons_sync();
+      const unsigned fw = flag[i0 >> 5] >> (i0 & 31);  // the thread's 16 pages share one flag word
+      keep |= member & fw & 0xffffu;
+    }
+  }
+  int nkp;
+  int pos = cons_scan1(__popc(keep), red + 64, &nkp);
+#pragma unroll
+  for (int k = 0; k < PS_PER; ++k)
+    if ((keep >> k) & 1u) kp[pos++] = p0 + i0 + k;
+  cons_sync();
+  return nkp;
+}
+
+
+// ---- Hamming scores of the CTA's candidate rows, key top-k over the group ----
+// (smaller score first, ties to the lower row).  Candidates are the rows of
+// the CTA's kept pages in page order; the group histogram of the integer
+// scores gives the threshold T and the ties taken; per-CTA counts of rows
+// below T and at T, published and scanned in CTA order (= row order), give
+// each CTA its ties and its place in the unit's row list.  Returns k_eff; the
+// list is complete when it returns (group barrier).
+template <int G, int WORDS>
+__device__ int gp_ksel(const FzParams& p, const GpShared& s, const Unit& x, int r, int nkp, unsigned* gx,
+                       unsigned& epoch, bool& ok) {
+  const Dims& dm = p.dm;
+  const Work& wk = p.wk;
+  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+  const int S = p.gsize;
+  unsigned char* w = s.work;
+  int* hist = reinterpret_cast<int*>(w + GW_HIST);
+  int* red = reinterpret_cast<int*>(w + GW_RED);
+  int* bc = red + 128;
+  const int* kp = reinterpret_cast<const int*>(w + GW_KP);
+  uint16_t* sc = reinterpret_cast<uint16_t*>(w + GW_SC);
+  const int nbins = G * dm.nb + 1;
+  const int ncs = nkp << dm.lgP;
+  for (int i = tid; i < nbins; i += FZ_CONS) hist[i] = 0;
+  uint64_t cq[G][WORDS];
+#pragma unroll
+  for (int g = 0; g < G; ++g)
+#pragma unroll
+    for (int w2 = 0; w2 < WORDS; ++w2)
+      cq[g][w2] = (uint64_t)s.qc[g * 8 + 2 * w2] | ((uint64_t)s.qc[g * 8 + 2 * w2 + 1] << 32);
+  // ---- scores (four rows per thread in flight) ----
+  int nval = 0;
+  for (int j0 = 0; j0 < ncs; j0 += 4 * FZ_CONS) {
+    uint64_t cw[4][WORDS];
+    bool valid[4];
+#pragma unroll
+    for (int e = 0; e < 4; ++e) {
+      const int j = j0 + e * FZ_CONS + tid;
+      valid[e] = false;
+#pragma unroll
+      for (int w2 = 0; w2 < WORDS; ++w2) cw[e][w2] = 0ull;
+      if (j < ncs) {
+        const int t = (kp[j >> dm.lgP] << dm.lgP) + (j & (dm.P - 1));
+        if (t < x.L) {
+          const long long woff = code_row(dm, p.table, x.b, x.h, t, p.status);
+          if (woff >= 0) {
+            valid[e] = true;
+            const uint64_t* src = p.codes + woff;
+            if constexpr (WORDS == 1) {
+              cw[e][0] = __ldg(src);
+            } else {
+#pragma unroll
+              for (int w2 = 0; w2 < WORDS; w2 += 2) {
+                const ulonglong2 tt = __ldg(reinterpret_cast<const ulonglong2*>(src + w2));
+                cw[e][w2] = tt.x;
+                cw[e][w2 + 1] = tt.y;
+              }
+            }
+          }
+        }
+      }
+    }
+#pragma unroll
+    for (int e = 0; e < 4; ++e) {
+      const int j = j0 + e * FZ_CONS + tid;
+      if (j < ncs) {
+        int sv = 0;
+#pragma unroll
+        for (int g = 0; g < G; ++g)
+#pragma unroll
+          for (int w2 = 0; w2 < WORDS; ++w2) sv += __popcll(cq[g][w2] ^ cw[e][w2]);
+        sc[j] = valid[e] ? (uint16_t)sv : (uint16_t)0xFFFFu;
+        nval += valid[e] ? 1 : 0;
+      }
+    }
+  }
+  cons_sync();  // scores complete, histogram zero
+  for (int j = tid; j < ncs; j += FZ_CONS) {
+    const int sv = sc[j];
+    if (sv != 0xFFFF) atomicAdd(&hist[sv], 1);
+  }
+  int cval;
+  (void)cons_scan1(nval, red, &cval);  // (its barrier also completes the histogram)
+  int* gh = reinterpret_cast<int*>(gx + GX_KHIST);
+  for (int i = tid; i < nbins; i += FZ_CONS) {
+    const int h = hist[i];
+    if (h) atomicAdd(gh + i, h);
+  }
+  int2* pub4 = reinterpret_cast<int2*>(gx + GX_PUB4);
+  if (tid == 0) pub4[r] = make_int2(nkp, cval);
+  if (!gp_sync(p, s, gx, epoch)) {
+    ok = false;
+    return 0;
+  }
+  // ---- threshold T from the group histogram; the CTAs' page offsets ----
+  const int bpt = (nbins + FZ_CONS - 1) / FZ_CONS;  // <= 5
+  int hv[5];
+  int local = 0;
+#pragma unroll
+  for (int e = 0; e < 5; ++e) {
+    const int bi = tid * bpt + e;
+    hv[e] = (e < bpt && bi < nbins) ? __ldcg(gh + bi) : 0;
+    local += hv[e];
+  }
+  if (tid == 0) {
+    bc[0] = -1;  // no candidate: nothing is kept
+    bc[1] = 0;
+  }
+  int n_cand;
+  const int before = cons_scan1(local, red + 16, &n_cand);
+  const int tk = __ldg(p.top_k + x.b);
+  const int keff = min(min(max(tk, 1), wk.Kmax), n_cand);
+  if (keff > 0 && before < keff && before + local >= keff) {
+    int run = before;
+#pragma unroll
+    for (int e = 0; e < 5; ++e) {
+      if (run < keff && run + hv[e] >= keff) {
+        bc[0] = tid * bpt + e;
+        bc[1] = keff - run;
+      }
+      run += hv[e];
+    }
+  }
+  const int2 q4 = tid < S ? __ldcg(pub4 + tid) : make_int2(0, 0);
+  int totp;
+  const int pb = cons_scan1(q4.x, red + 32, &totp);
+  if (tid == r) bc[2] = pb;
+  cons_sync();
+  const int T = bc[0], need_eq = bc[1], poff = bc[2];
+  // ---- this CTA's rows below T and at T ----
+  int lt = 0, eq = 0;
+  for (int j = tid; j < ncs; j += FZ_CONS) {
+    const int sv = sc[j];
+    lt += sv < T ? 1 : 0;
+    eq += sv == T ? 1 : 0;
+  }
+  int tot5;
+  (void)cons_scan1((lt << 16) | eq, red + 48, &tot5);
+  int2* pub5 = reinterpret_cast<int2*>(gx + GX_PUB5);
+  if (tid == 0) pub5[r] = make_int2(tot5 >> 16, tot5 & 0xFFFF);
+  // the stage's outputs: scores in candidate order, kept pages, counts
+  if (p.dbg.key_scores) {
+    int* dsc = p.dbg.key_scores + (long long)x.u * wk.Nmax * dm.P + ((long long)poff << dm.lgP);
+    for (int j = tid; j < ncs; j += FZ_CONS) {
+      const int sv = sc[j];
+      dsc[j] = sv == 0xFFFF ? INT_MAX : sv;
+    }
+  }
+  if (p.dbg.sel_pages)
+    for (int i = tid; i < nkp; i += FZ_CONS) p.dbg.sel_pages[(long long)x.u * wk.Nmax + poff + i] = kp[i];
+  if (r == 0 && tid == 0) {
+    if (p.dbg.n_sel_pages) p.dbg.n_sel_pages[x.u] = totp;
+    if (p.dbg.n_cand) p.dbg.n_cand[x.u] = n_cand;
+    if (p.dbg.n_sel_keys) p.dbg.n_sel_keys[x.u] = keff;
+  }
+  if (!gp_sync(p, s, gx, epoch)) {
+    ok = false;
+    return 0;
+  }
+  // ---- ties go to the lower CTAs; each CTA's place in the row list ----
+  const int2 q5 = tid < S ? __ldcg(pub5 + tid) : make_int2(0, 0);
+  int tt;
+  const int tb = cons_scan1(q5.y, red + 64, &tt);
+  const int take_t = max(0, min(q5.y, need_eq - tb));
+  int tsel;
+  const int ob = cons_scan1(q5.x + take_t, red + 80, &tsel);
+  if (tid == r) {
+    bc[3] = ob;
+    bc[4] = take_t;
+  }
+  cons_sync();
+  const int off = bc[3], take = bc[4];
+  // ---- kept rows in candidate order: warp w owns candidates [w nbw, (w+1) nbw)
+  // in rounds of 32; counts per warp, one scan, then ballots place the rows ----
+  const int rounds = (ncs + 32 * FZ_CWARPS - 1) / (32 * FZ_CWARPS);
+  const int cw0 = warp * rounds * 32;
+  const unsigned lanemask_lt = (1u << lane) - 1u;
+  int lt_w = 0, eq_w = 0;
+  for (int rr = 0; rr < rounds; ++rr) {
+    const int ci = cw0 + 32 * rr + lane;
+    const int sv = ci < ncs ? (int)sc[ci] : 0xFFFF;
+    lt_w += __popc(__ballot_sync(0xffffffffu, sv < T));
+    eq_w += __popc(__ballot_sync(0xffffffffu, sv == T));
+  }
+  int totw;
+  const int pk = cons_scan1(lane == 0 ? (lt_w << 16) | eq_w : 0, red + 96, &totw);
+  int lt_b = __shfl_sync(0xffffffffu, pk, 0) >> 16, eq_b = __shfl_sync(0xffffffffu, pk, 0) & 0xFFFF;
+  int* out = wk.sel_keys + (long long)x.u * wk.Kmax + off;
+  int* dout = p.dbg.sel_keys ? p.dbg.sel_keys + (long long)x.u * wk.Kmax + off : nullptr;
+  const int room = keff - off;
+  for (int rr = 0; rr < rounds; ++rr) {
+    const int ci = cw0 + 32 * rr + lane;
+    const int sv = ci < ncs ? (int)sc[ci] : 0xFFFF;
+    const bool l1 = sv < T, e1 = sv == T;
+    const unsigned blt = __ballot_sync(0xffffffffu, l1), beq = __ballot_sync(0xffffffffu, e1);
+    const int eq_before = eq_b + __popc(beq & lanemask_lt);
+    const bool tk1 = l1 || (e1 && eq_before < take);
+    const int pos = lt_b + __popc(blt & lanemask_lt) + min(eq_before, take);
+    if (tk1 && pos < room) {
+      const int t = (kp[ci >> dm.lgP] << dm.lgP) + (ci & (dm.P - 1));
+      out[pos] = t;
+      if (dout) dout[pos] = t;
+    }
+    lt_b += __popc(blt);
+    eq_b += __popc(beq);
+  }
+  if (!gp_sync(p, s, gx, epoch)) {
+    ok = false;
+    return 0;
+  }
+  return keff;
+}
+
+
+// Consumers copy the K'/V rows of one gather step into four ring slots:
+// warp w the rows 8w .. 8w+7 it computes on (K' row j in slot sb + j / 64,
+// V row j two slots further); a bad row reads as zeros.  One cp.async group.
+__device__ __forceinline__ void gp_gather_rows(unsigned char* ring, const int* ridx, int n, int sb,
+                                               const __nv_bfloat16* K, const __nv_bfloat16* V) {
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+  const int q = lane & 15;
+#pragma unroll
+  for (int i = 0; i < 4; ++i) {
+    const int j = warp * 8 + 2 * i + (lane >> 4);
+    if (j < n) {
+      const int r = ridx[j];
+      unsigned char* d1 = ring + (size_t)(sb + j / 64) * FZ_SLOT + (j % 64) * 256 + q * 16;
+      unsigned char* d2 = ring + (size_t)(sb + 2 + j / 64) * FZ_SLOT + (j % 64) * 256 + q * 16;
+      if (r >= 0) {
+        cp_async16(d1, K + (long long)r * D + q * 8);
+        cp_async16(d2, V + (long long)r * D + q * 8);
+      } else {
+        *reinterpret_cast<uint4*>(d1) = make_uint4(0u, 0u, 0u, 0u);
+        *reinterpret_cast<uint4*>(d2) = make_uint4(0u, 0u, 0u, 0u);
+      }
+    }
+  }
+  cp_async_commit();
+}
+
+// ---- one gather step: softmax attention over one chunk of 128 kept rows ----
+// The arithmetic of the fused kernel's gather (logits by groups of LPR lanes,
+// warp-local softmax and P.V, 16 warp partials combined in warp order); the
+// chunk's partial (unnormalised output, max and sum of weights per head, in
+// log2 units) goes to `part`.  A chunk's partial depends only on its rows, so
+// results do not depend on how many CTAs share the unit.
+template <int G>
+__device__ void gp_gather_step(const FzParams& p, const GpShared& s, int n, int sb, float* part) {
+  constexpr int GP = G <= 4 ? 4 : 8;
+  constexpr int LPR = GP == 4 ? 8 : 16;
+  constexpr int NCK = 128 / LPR / 8;
+  constexpr int RPG = LPR / 4;
+  constexpr int NV = RPG * GP;
+  constexpr int KP = NV / LPR;
+  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+  const int grp = lane / LPR, li = lane % LPR;
+  float* OB = reinterpret_cast<float*>(s.work + GA_OB);
+  float2* PB = reinterpret_cast<float2*>(s.work + GA_PB) + warp * 8 * GP;
+  float* MB = reinterpret_cast<float*>(s.work + GA_MB);
+  float* LB = reinterpret_cast<float*>(s.work + GA_LB);
+  const float* qs = s.qs;
+  const float qscale = p.sm_scale * 1.4426950408889634f;
+  float sv[KP];
+  {
+    float2 q2[G][4 * NCK];
+#pragma unroll
+    for (int g = 0; g < G; ++g)
+#pragma unroll
+      for (int k = 0; k < NCK; ++k)
+#pragma unroll
+        for (int h = 0; h < 2; ++h) {
+          const float4 t = *reinterpret_cast<const float4*>(qs + g * D + 4 * (LPR * k + li + 16 * h));
+          q2[g][4 * k + 2 * h] = make_float2(t.x * qscale, t.y * qscale);
+          q2[g][4 * k + 2 * h + 1] = make_float2(t.z * qscale, t.w * qscale);
+        }
+    float v[NV];
+#pragma unroll
+    for (int r = 0; r < RPG; ++r) {
+      const int j = warp * 8 + grp * RPG + r;
+      const unsigned char* row = s.ring + (size_t)(sb + j / 64) * FZ_SLOT + (j % 64) * 256;
+      float2 kf[4 * NCK];
+#pragma unroll
+      for (int k = 0; k < NCK; ++k) {
+        const uint4 kv = *reinterpret_cast<const uint4*>(row + 16 * (LPR * k + li));
+        kf[4 * k] = make_float2(bf_lo(kv.x), bf_hi(kv.x));
+        kf[4 * k + 1] = make_float2(bf_lo(kv.y), bf_hi(kv.y));
+        kf[4 * k + 2] = make_float2(bf_lo(kv.z), bf_hi(kv.z));
+        kf[4 * k + 3] = make_float2(bf_lo(kv.w), bf_hi(kv.w));
+      }
+#pragma unroll
+      for (int g = 0; g < GP; ++g) {
+        float a = 0.f;
+        if (g < G) {
+          float2 a0 = __fmul2_rn(q2[g][0], kf[0]);
+#pragma unroll
+          for (int k = 1; k < 4 * NCK; ++k) a0 = __ffma2_rn(q2[g][k], kf[k], a0);
+          a = a0.x + a0.y;
+        }
+        v[g * RPG + r] = a;
+      }
+    }
+    group_reduce_t<NV, LPR>(v, lane);
+#pragma unroll
+    for (int e = 0; e < KP; ++e) {
+      const int r = (KP * li + e) % RPG;
+      const int j = warp * 8 + grp * RPG + r;
+      sv[e] = ((li >> 1) < G && j < n) ? v[e] : -INFINITY;
+    }
+  }
+  const int gl = li >> 1;
+  float m = sv[0];
+#pragma unroll
+  for (int e = 1; e < KP; ++e) m = fmaxf(m, sv[e]);
+  m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, 1));
+#pragma unroll
+  for (int o = LPR; o < 32; o <<= 1) m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, o));
+  float l = 0.f;
+#pragma unroll
+  for (int e = 0; e < KP; ++e) {
+    const float pv = (sv[e] == -INFINITY) ? 0.f : exp2f(sv[e] - m);
+    const int r = (KP * li + e) % RPG;
+    PB[(grp * RPG + r) * GP + gl] = make_float2(pv, pv);
+    l += pv;
+  }
+  l += __shfl_xor_sync(0xffffffffu, l, 1);
+#pragma unroll
+  for (int o = LPR; o < 32; o <<= 1) l += __shfl_xor_sync(0xffffffffu, l, o);
+  if (lane < LPR && (li & 1) == 0 && gl < G) {
+    MB[warp * 8 + gl] = m;
+    LB[warp * 8 + gl] = l;
+  }
+  __syncwarp();
+  float2 o2[G][2];
+#pragma unroll
+  for (int g = 0; g < G; ++g) o2[g][0] = o2[g][1] = make_float2(0.f, 0.f);
+#pragma unroll
+  for (int r = 0; r < 8; ++r) {
+    const int j = warp * 8 + r;
+    if (j < n) {
+      const uint2 vv = *reinterpret_cast<const uint2*>(s.ring + (size_t)(sb + 2 + j / 64) * FZ_SLOT + (j % 64) * 256 +
+                                                       lane * 8);
+      const float2 v0 = make_float2(bf_lo(vv.x), bf_hi(vv.x)), v1 = make_float2(bf_lo(vv.y), bf_hi(vv.y));
+      float2 pr[GP];
+#pragma unroll
+      for (int g2 = 0; g2 < G; g2 += 2) {
+        const float4 t = *reinterpret_cast<const float4*>(PB + r * GP + g2);
+        pr[g2] = make_float2(t.x, t.y);
+        pr[g2 + 1] = make_float2(t.z, t.w);
+      }
+#pragma unroll
+      for (int g = 0; g < G; ++g) {
+        o2[g][0] = __ffma2_rn(pr[g], v0, o2[g][0]);
+        o2[g][1] = __ffma2_rn(pr[g], v1, o2[g][1]);
+      }
+    }
+  }
+#pragma unroll
+  for (int g = 0; g < G; ++g)
+    *reinterpret_cast<float4*>(OB + (warp * G + g) * D + 4 * lane) =
+        make_float4(o2[g][0].x, o2[g][0].y, o2[g][1].x, o2[g][1].y);
+  cons_sync();
+  if (tid < G * 32) {
+    const int g = warp, c4 = lane;
+    const float mw = MB[(lane & 15) * 8 + g];
+    float M = mw;
+#pragma unroll
+    for (int o = 1; o < 16; o <<= 1) M = fmaxf(M, __shfl_xor_sync(0xffffffffu, M, o));
+    const float sc = (mw == -INFINITY) ? 0.f : exp2f(mw - M);
+    float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
+    float L = 0.f;
+#pragma unroll
+    for (int w = 0; w < FZ_CWARPS; ++w) {
+      const float scw = __shfl_sync(0xffffffffu, sc, w);
+      const float4 a = *reinterpret_cast<const float4*>(OB + (w * G + g) * D + 4 * c4);
+      acc.x = fmaf(scw, a.x, acc.x);
+      acc.y = fmaf(scw, a.y, acc.y);
+      acc.z = fmaf(scw, a.z, acc.z);
+      acc.w = fmaf(scw, a.w, acc.w);
+      L = fmaf(scw, LB[w * 8 + g], L);
+    }
+    *reinterpret_cast<float4*>(part + g * D + 4 * c4) = acc;
+    if (c4 == 0) {
+      part[G * D + g] = M;
+      part[G * D + 8 + g] = L;
+    }
+  }
+  cons_sync();  // the step's scratch and slots are free
+}
+
+
+// ---------------------------------------------------------------------------
+// consumer warps 0-15: the units of the group, one after another
+// ---------------------------------------------------------------------------
+template <int G, int WORDS>
+__device__ void gp_consumer(const FzParams& p, const GpShared& s, int g, int r) {
+  const Dims& dm = p.dm;
+  const Work& wk = p.wk;
+  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+  const int U = dm.B * dm.Hkv, S = p.gsize;
+  const int PS = G * D + 16;
+  volatile int* misc = s.misc;
+  unsigned nslot = 0, nunit = 0;
+  for (int u = g; u < U; u += p.ngroups) {
+    Unit x;
+    x.u = u;
+    x.b = u / dm.Hkv;
+    x.h = u - x.b * dm.Hkv;
+    x.L = seq_len_of(dm, p.seq_lens, x.b);
+    x.np = (x.L + dm.P - 1) >> dm.lgP;
+    unsigned* gx = gx_of(p, u);
+    unsigned epoch = 0;
+    bool ok = true;
+    gp_prep<G>(p, s, x, r == 0);  // (q' and the query codes are stage outputs even for an empty sequence)
+    if (x.L == 0) {
+      if (r == 0) {
+        for (int e = tid; e < G * D; e += FZ_CONS) p.out[((long long)x.b * dm.Hq + x.h * G) * D + e] = 0.f;
+        if (tid == 0) {
+          if (p.dbg.n_sel_pages) p.dbg.n_sel_pages[x.u] = 0;
+          if (p.dbg.n_sel_keys) p.dbg.n_sel_keys[x.u] = 0;
+          if (p.dbg.n_cand) p.dbg.n_cand[x.u] = 0;
+        }
+      }
+    } else {
+      // ---- scan of the CTA's pages, 128 per step ----
+      int p0, p1;
+      share_of(x.np, S, r, p0, p1);
+      const int nr = p1 - p0;
+      float* Us = reinterpret_cast<float*>(s.work + GW_US);
+      for (int j = 0; j < nr; j += FZ_ROWS) {
+        const int n = min(FZ_ROWS, nr - j), nsl = (n + GP_PAGES_PER_SLOT - 1) / GP_PAGES_PER_SLOT;
+        if (tid == 0) {
+          int good = 1;
+          for (int k = 0; k < nsl && good; ++k) {
+            const unsigned gs = nslot + k;
+            if (!gp_wait(s, &s.full[gs % FZ_NSLOT], (gs / FZ_NSLOT) & 1, p.status)) good = 0;
+          }
+          misc[17] = good;
+        }
+        cons_sync();
+        if (!misc[17]) {
+          ok = false;
+          break;
+        }
+        gp_scan<G>(p, s, x, p0 + j, n, (int)(nslot % FZ_NSLOT), Us + j);
+        cons_sync();
+        if (tid == 0)
+          for (int k = 0; k < nsl; ++k) mbar_arrive(&s.empty[(nslot + k) % FZ_NSLOT]);
+        nslot += nsl;
+      }
+      // ---- selects ----
+      int nkp = 0, keff = 0;
+      if (ok) {
+        const int N = min(min(max(__ldg(p.n_keep + x.b), 1), wk.Nmax), x.np);
+        nkp = gp_psel(p, s, x, r, p0, nr, N, gx, epoch, ok);
+      }
+      if (ok) keff = gp_ksel<G, WORDS>(p, s, x, r, nkp, gx, epoch, ok);
+      if (ok) {
+        // ---- attention over the CTA's chunks of 128 kept rows ----
+        const int nch = (keff + FZ_ROWS - 1) / FZ_ROWS;
+        int c0, c1;
+        share_of(nch, S, r, c0, c1);
+        const int k0 = c0 * FZ_ROWS;
+        const int nrow = min(keff, c1 * FZ_ROWS) - k0, nst = c1 - c0;
+        const int* keys = wk.sel_keys + (long long)x.u * wk.Kmax + k0;
+        float* parts = wk.part + (long long)x.u * wk.C3 * PS;
+        // row numbers of step i, warp w: rows 8w .. 8w+7 (the rows it copies)
+        auto rows_of = [&](int i, int* rx) {
+          if (lane < 8) {
+            const int j = warp * 8 + lane, jj = i * FZ_ROWS + j;
+            if (jj < nrow) {
+              const int t = __ldcg(keys + jj);
+              const long long off = kv_row(dm, p.table, x.b, x.h, t, p.status);
+              rx[j] = off >= 0 ? (int)(off / D) : -1;
+            }
+          }
+          __syncwarp();
+        };
+        if (nst > 0) {
+          rows_of(0, s.ridx);
+          gp_gather_rows(s.ring, s.ridx, min(FZ_ROWS, nrow), 0, p.Kr, p.Vc);
+        }
+        for (int i = 0; i < nst; ++i) {
+          const int n = min(FZ_ROWS, nrow - i * FZ_ROWS);
+          if (i + 1 < nst) {
+            int* rx = s.ridx + ((i + 1) & 1) * FZ_ROWS;
+            rows_of(i + 1, rx);
+            gp_gather_rows(s.ring, rx, min(FZ_ROWS, nrow - (i + 1) * FZ_ROWS), 4 * ((i + 1) & 1), p.Kr, p.Vc);
+            cp_async_wait<1>();
+          } else {
+            cp_async_wait<0>();
+          }
+          __syncwarp();
+          gp_gather_step<G>(p, s, n, 4 * (i & 1), parts + (long long)(c0 + i) * PS);
+        }
+        // ---- the last CTA of the group merges the unit's chunk partials in chunk order ----
+        if (tid == 0) {
+          int last = 1;
+          if (S > 1) last = atom_add_acq_rel(gx + GX_ARRIVE, 1u) == (unsigned)(S - 1);
+          misc[18] = last;
+        }
+        cons_sync();
+        if (misc[18]) {
+          merge_partials<G>(s.work, parts, nch, nullptr, p.out + ((long long)x.b * dm.Hq + x.h * G) * D);
+          // the unit's counters and histograms are zero again
+          uint4* z = reinterpret_cast<uint4*>(gx + GX_HIST);
+          for (int i = tid; i < GP_LEVELS * SEL_NBIN / 4; i += FZ_CONS) z[i] = make_uint4(0u, 0u, 0u, 0u);
+          uint4* zk = reinterpret_cast<uint4*>(gx + GX_KHIST);
+          for (int i = tid; i < wk.HB / 4; i += FZ_CONS) zk[i] = make_uint4(0u, 0u, 0u, 0u);
+          if (tid == 0) {
+            gx[GX_BAR] = 0u;
+            gx[GX_ARRIVE] = 0u;
+            gx[GX_CCOUNT] = 0u;
+          }
+        }
+      }
+    }
+    if (!ok) break;
+    // the ring is free for the producer's next unit
+    cons_sync();
+    ++nunit;
+    if (tid == 0) {
+      asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+      misc[20] = (int)nunit;
+    }
+  }
+  cp_async_wait<0>();
+  if (tid == 0) misc[1] = (int)nslot;
+}
+
+template <int G, int WORDS>
+__global__ void __launch_bounds__(FZ_THREADS, 1) hhr_group_kernel(FzParams p) {
+  extern __shared__ __align__(128) unsigned char gp_smem[];
+  const GpShared s = gp_shared(gp_smem);
+  const int tid = threadIdx.x;
+  if (tid == 0) {
+    for (int i = 0; i < FZ_NSLOT; ++i) {
+      mbar_init(&s.full[i], 1);
+      mbar_init(&s.empty[i], 1);
+    }
+    for (int i = 0; i < 32; ++i) s.misc[i] = 0;
+    fence_mbar_init();
+  }
+  __syncthreads();
+  const int g = blockIdx.x / p.gsize, r = blockIdx.x - g * p.gsize;
+  const int warp = tid >> 5;
+  if (warp >= FZ_CWARPS) {
+    asm volatile("setmaxnreg.dec.sync.aligned.u32 %0;" ::"n"(FZ_REGS_AUX));
+    if (warp == FZ_PRODUCER_WARP) gp_producer(p, s, g, r);
+  } else {
+    asm volatile("setmaxnreg.inc.sync.aligned.u32 %0;" ::"n"(FZ_REGS_CONS));
+    gp_consumer<G, WORDS>(p, s, g, r);
+  }
+  __syncthreads();
+  // drain metadata copies that were armed but never consumed (only after an abort)
+  if (tid == 0) {
+    const unsigned armed = (unsigned)s.misc[2], consumed = (unsigned)s.misc[1];
+    for (unsigned gs = consumed; gs < armed; ++gs) {
+      const long long t0 = clock64();
+      while (!mbar_try_wait(&s.full[gs % FZ_NSLOT], (gs / FZ_NSLOT) & 1)) {
+        if (clock64() - t0 > FZ_WAIT_CYCLES) break;
+      }
+    }
+  }
+}
+
+template <int G, int WORDS>
+static cudaError_t launch_group_t(const FzParams& prm, int grid, cudaStream_t st) {
+  static bool configured[64] = {false};  // the attribute is per function and device
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return cudaErrorInvalidDevice;
+  if (!configured[dev]) {
+    const cudaError_t e =
+        cudaFuncSetAttribute(hhr_group_kernel<G, WORDS>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)GP_SMEM);
+    if (e != cudaSuccess) return e;
+    configured[dev] = true;
+  }
+  hhr_group_kernel<G, WORDS><<<grid, FZ_THREADS, GP_SMEM, st>>>(prm);
+  return cudaGetLastError();
+}
+
+// CTAs per group: the SMs shared out over the units, at most one CTA per 64
+// pages of the longest sequence (a short unit gains nothing from more).
+inline void group_shape(const Dims& dm, int sms, int* S, int* ngroups) {
+  const int U = dm.B * dm.Hkv;
+  sms = std::max(1, std::min(sms, (int)GP_SMAX));
+  int s = std::max(1, sms / U);
+  s = std::min(s, std::max(1, dm.np_max / 64));
+  *S = s;
+  *ngroups = std::max(1, std::min(U, sms / s));
+}
+
+
+static_assert(GX_KHIST == GROUP_GX_FIXED_WORDS, "exchange area layout");
+
+template <int G>
+cudaError_t launch_decode(const DecodeArgs& a) {
+  FzParams prm = make_params(a, false);
+  int S = 1, ngroups = 1;
+  group_shape(a.dm, a.num_sms, &S, &ngroups);
+  prm.gsize = S;
+  prm.ngroups = ngroups;
+  const int grid = S * ngroups;
+  switch (a.dm.words) {
+    case 1: return launch_group_t<G, 1>(prm, grid, a.stream);
+    case 2: return launch_group_t<G, 2>(prm, grid, a.stream);
+    case 4: return launch_group_t<G, 4>(prm, grid, a.stream);
+  }
+  return cudaErrorInvalidValue;
+}
+
+}  // namespace hhr
