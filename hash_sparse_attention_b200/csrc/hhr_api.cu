@@ -118,14 +118,14 @@ size_t carve(const Dims& dm, int Nmax, int Kmax, bool dense, char* base, Work* w
   const int Cmax = Nmax * dm.P;
   const int HB = (dm.G * dm.nb + 1 + 7) / 8 * 8;
   if (!dense) {
-    // group kernel: per-unit exchange areas
-    w.gx_stride = (GROUP_GX_FIXED_WORDS + HB + 3) / 4 * 4;
+    // group kernel: per-unit counters
+    w.gx_stride = GROUP_GX_WORDS;
     w.gx = reinterpret_cast<unsigned*>(take(sizeof(unsigned) * BH * w.gx_stride));
     w.U = reinterpret_cast<float*>(take(sizeof(float) * BH * Ustride));
     w.sel_pages = reinterpret_cast<int*>(take(sizeof(int) * BH * Nmax));
     w.sel_keys = reinterpret_cast<int*>(take(sizeof(int) * BH * Kmax));
     w.kscore = reinterpret_cast<uint16_t*>(take(sizeof(uint16_t) * BH * Cmax));
-    w.khist = reinterpret_cast<int*>(take(sizeof(int) * BH * HB));
+    w.khist = reinterpret_cast<int*>(take(sizeof(int) * std::max<size_t>(BH, MAX_GRID) * HB));
   }
   w.Nmax = Nmax;
   w.Kmax = Kmax;

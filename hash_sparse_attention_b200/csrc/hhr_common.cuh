@@ -30,7 +30,8 @@ struct Work {
   float* part;         // [B, Hkv, C3, G * D + 16] attention partial of every gather chunk
   float* gpart;        // [B, Hkv, max_groups, G * D + 16] merged groups of chunks
   uint16_t* kscore;    // [B, Hkv, Cmax]    Hamming score of every candidate row
-  int* khist;          // [B, Hkv, HB]      score histogram (kept at zero between calls)
+  int* khist;          // [max(B Hkv, grid), HB] score histograms: per unit (fused kernel, zero between
+                       // calls) or per CTA (group kernel, rewritten every unit)
   int4* tq;            // [tq_cap]          task queue: (kind, unit, arg, sequence + 1), zero between calls
   unsigned* gx;        // [B * Hkv, gx_stride] per-unit exchange areas of the CTA groups
   unsigned* ctrl;      // [4 + B * Hkv * (8 + max_groups)] item queue, exit count, task queue head / tail, flags, counters

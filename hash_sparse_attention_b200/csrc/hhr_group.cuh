@@ -41,7 +41,9 @@ constexpr size_t GP_OFF_WORK = GP_OFF_RING + (size_t)FZ_NSLOT * FZ_SLOT;
 constexpr size_t GP_OFF_QS = GP_OFF_WORK + GP_WORK;   // q' fp32 [8][128] (quad-permuted)
 constexpr size_t GP_OFF_QC = GP_OFF_QS + 8 * D * 4;   // query codes u32 [8][8]
 constexpr size_t GP_OFF_RIDX = GP_OFF_QC + 256;       // row numbers of two gather steps [2][128]
-constexpr size_t GP_OFF_BAR = GP_OFF_RIDX + 2 * FZ_ROWS * 4;
+constexpr int GP_PF_MAX = 512;                 // pages in the producer's prefetch list
+constexpr size_t GP_OFF_PF = GP_OFF_RIDX + 2 * FZ_ROWS * 4;  // int [GP_PF_MAX]
+constexpr size_t GP_OFF_BAR = GP_OFF_PF + GP_PF_MAX * 4;
 constexpr size_t GP_OFF_MISC = GP_OFF_BAR + 8 * (2 * FZ_NSLOT);
 constexpr size_t GP_SMEM = GP_OFF_MISC + 256;
 static_assert(GP_SMEM <= 232448, "shared memory of the group kernel");
@@ -58,23 +60,22 @@ static_assert(GW_SC + 2 * MAX_CANDIDATES <= GP_WORK, "group kernel scratch");
 static_assert(MAX_SELECT_PAGES * 4 <= GW_HIST && FZ_HIST_BINS * 4 <= 8448, "group kernel scratch");
 static_assert(GA_LB + 512 <= GP_WORK, "gather scratch");
 
-// Per-unit exchange area in the workspace (32-bit words).  The counters and
-// histograms are zero between units (the merging CTA clears them); the rest
-// is written before it is read.
+// Per-unit counters in the workspace (32-bit words), zero between calls (the
+// merging CTA resets them).
 enum : int {
   GX_BAR = 0,     // group barrier arrivals
-  GX_ARRIVE = 1,  // partials published
-  GX_CCOUNT = 2,  // members in the candidate list
-  GX_MM = 4,                                        // float2 [levels][SMAX] member range per CTA
-  GX_PUB4 = GX_MM + 2 * GP_LEVELS * GP_SMAX,        // int2 [SMAX] kept pages, valid candidates
-  GX_PUB5 = GX_PUB4 + 2 * GP_SMAX,                  // int2 [SMAX] rows below the threshold, ties
-  GX_PUBT = GX_PUB5 + 2 * GP_SMAX,                  // int [SMAX] members (equal bounds)
-  GX_HIST = GX_PUBT + GP_SMAX,                      // int [levels][2048]
-  GX_CAND = GX_HIST + GP_LEVELS * SEL_NBIN,         // int2 [512] (bound bits, page)
-  GX_KHIST = GX_CAND + 2 * SEL_MAX_CAND,            // int [HB] score histogram
+  GX_ARRIVE = 1,  // CTAs done with the unit (the last one merges)
+  GX_WORDS = 4,
 };
-// words of one unit's area before the partials (the score histogram is HB long)
-__host__ __device__ constexpr int gx_head_words(int HB) { return (GX_KHIST + HB + 3) / 4 * 4; }
+
+__device__ __forceinline__ int ld_relaxed32(const int* w) {
+  int v;
+  asm volatile("ld.relaxed.gpu.global.s32 %0, [%1];" : "=r"(v) : "l"(w) : "memory");
+  return v;
+}
+__device__ __forceinline__ void prefetch_l2(const void* p, unsigned bytes) {
+  asm volatile("cp.async.bulk.prefetch.L2.global [%0], %1;" ::"l"(p), "r"(bytes) : "memory");
+}
 
 struct GpShared {
   unsigned char* ring;
@@ -82,10 +83,13 @@ struct GpShared {
   float* qs;
   unsigned* qc;
   int* ridx;
+  int* pf;          // pages whose code (then K'/V) rows the producer prefetches to L2
+  const int* kpw;   // kept pages of the unit (consumer scratch)
   uint64_t* full;
   uint64_t* empty;
   int* misc;        // [0] abort, [1] slots consumed, [2] slots armed, [17], [18] broadcasts,
-                    // [20] units whose ring use the consumers have finished
+                    // [20] units whose ring use the consumers have finished, [21] units whose
+                    // prefetch list is ready, [22], [23] its code and K'/V page counts
 };
 
 __device__ __forceinline__ GpShared gp_shared(unsigned char* base) {
@@ -95,6 +99,8 @@ __device__ __forceinline__ GpShared gp_shared(unsigned char* base) {
   s.qs = reinterpret_cast<float*>(base + GP_OFF_QS);
   s.qc = reinterpret_cast<unsigned*>(base + GP_OFF_QC);
   s.ridx = reinterpret_cast<int*>(base + GP_OFF_RIDX);
+  s.pf = reinterpret_cast<int*>(base + GP_OFF_PF);
+  s.kpw = reinterpret_cast<const int*>(base + GP_OFF_WORK + GW_KP);
   uint64_t* bars = reinterpret_cast<uint64_t*>(base + GP_OFF_BAR);
   s.full = bars;
   s.empty = bars + FZ_NSLOT;
@@ -245,6 +251,51 @@ static __device__ void gp_producer(const FzParams& p, const GpShared& s, int g, 
       if (lane == 0) s.misc[2] = (int)nslot;  // slots armed (drained at exit after an abort)
     }
     if (aborted) break;
+    if (L > 0) {
+      // L2 prefetches from the consumers' list, once the kept pages are known:
+      // code rows (trimmed to 16-byte boundaries), then K'/V rows of pages
+      bool ok = true;
+      if (lane == 0) {
+        volatile int* rdy = s.misc + 21;
+        if (*rdy < (int)nunit + 1) {
+          const long long t0 = clock64();
+          while (*rdy < (int)nunit + 1) {
+            if (*reinterpret_cast<volatile int*>(s.misc)) {
+              ok = false;
+              break;
+            }
+            if (clock64() - t0 > FZ_WAIT_CYCLES) {
+              set_status(p.status, HHR_ERR_TIMEOUT);
+              *reinterpret_cast<volatile int*>(s.misc) = 1;
+              ok = false;
+              break;
+            }
+          }
+        }
+      }
+      if (__shfl_sync(0xffffffffu, (int)ok, 0) == 0) break;
+      const int n1 = reinterpret_cast<volatile int*>(s.misc)[22], n2 = reinterpret_cast<volatile int*>(s.misc)[23];
+      for (int i = lane; i < n1 + n2; i += 32) {
+        const int pg = reinterpret_cast<volatile int*>(s.pf)[i];
+        const int t0 = pg << dm.lgP;
+        if (i < n1) {
+          const long long co = code_row(dm, p.table, b, h, t0, p.status);
+          if (co >= 0) {
+            const uintptr_t a0 = reinterpret_cast<uintptr_t>(p.codes + co);
+            const uintptr_t a1 = a0 + (uintptr_t)(dm.P * dm.words * 8);
+            const uintptr_t c0 = (a0 + 15) & ~(uintptr_t)15, c1 = a1 & ~(uintptr_t)15;
+            if (c1 > c0) prefetch_l2(reinterpret_cast<const void*>(c0), (unsigned)(c1 - c0));
+          }
+        } else {
+          const long long ro = kv_row(dm, p.table, b, h, t0, p.status);
+          if (ro >= 0) {
+            prefetch_l2(p.Kr + ro, (unsigned)(dm.P * D * 2));
+            prefetch_l2(p.Vc + ro, (unsigned)(dm.P * D * 2));
+          }
+        }
+      }
+      __syncwarp();
+    }
   }
 }
 
@@ -261,9 +312,19 @@ __device__ void gp_prep(const FzParams& p, const GpShared& s, const Unit& x, boo
   const __nv_bfloat16* qg = p.q + ((long long)x.b * dm.Hq + x.h * G) * D;
   // R_h rows 8w .. 8w+7 of this warp (lane: channels 4l .. 4l+3), issued first
   const float* Rh = p.R + (long long)x.h * D * D;
+  constexpr int NBB = 32 / GP;  // code bits per block (see below)
+  const int bpw = dm.nb / FZ_CWARPS;
+  const __nv_bfloat16* Wh = p.W + (long long)x.h * dm.nb * D;
+  // every load of the first round is issued before any is used: R_h rows, the
+  // first block of W_h rows, q
   float4 rr[8];
+  uint2 wv[NBB];
 #pragma unroll
   for (int k = 0; k < 8; ++k) rr[k] = __ldg(reinterpret_cast<const float4*>(Rh + (long long)(warp * 8 + k) * D) + lane);
+#pragma unroll
+  for (int bb = 0; bb < NBB; ++bb)
+    wv[bb] = bb < bpw ? __ldg(reinterpret_cast<const uint2*>(Wh + (long long)(warp * bpw + bb) * D) + lane)
+                      : make_uint2(0u, 0u);
   for (int i = tid; i < G * D; i += FZ_CONS) qf[i] = __bfloat162float(qg[i]);
   if (tid < 64) s.qc[tid] = 0u;
   cons_sync();
@@ -293,16 +354,15 @@ __device__ void gp_prep(const FzParams& p, const GpShared& s, const Unit& x, boo
     }
   }
   // query codes: warp w takes bits [w nb/16, (w+1) nb/16) in blocks of NBB
-  constexpr int NBB = 32 / GP;
-  const int bpw = dm.nb / FZ_CWARPS;
-  const __nv_bfloat16* Wh = p.W + (long long)x.h * dm.nb * D;
   for (int jb = 0; jb < bpw; jb += NBB) {
     float v[2 * NBB * GP];
-    uint2 wv[NBB];
+    if (jb > 0) {
 #pragma unroll
-    for (int bb = 0; bb < NBB; ++bb) {
-      const int j = warp * bpw + jb + bb;
-      wv[bb] = (jb + bb < bpw) ? __ldg(reinterpret_cast<const uint2*>(Wh + (long long)j * D) + lane) : make_uint2(0u, 0u);
+      for (int bb = 0; bb < NBB; ++bb) {
+        const int j = warp * bpw + jb + bb;
+        wv[bb] = (jb + bb < bpw) ? __ldg(reinterpret_cast<const uint2*>(Wh + (long long)j * D) + lane)
+                                 : make_uint2(0u, 0u);
+      }
     }
 #pragma unroll
     for (int bb = 0; bb < NBB; ++bb) {
@@ -351,7 +411,7 @@ __device__ void gp_prep(const FzParams& p, const GpShared& s, const Unit& x, boo
 // the ring layout of the group kernel: page j of the step in slot
 // sb + j / 32, its minima at row j % 32 and its maxima half a slot further.
 template <int G>
-__device__ void gp_scan(const FzParams& p, const GpShared& s, const Unit& x, int pg0, int n, int sb, float* Us) {
+__device__ void gp_scan(const FzParams& p, const GpShared& s, const Unit& x, int pg0, int n, int sb) {
   constexpr int GP = G <= 4 ? 4 : 8;
   constexpr bool SPLIT = G <= 4;
   constexpr int PB = GP == 4 ? 4 : 2;
@@ -432,7 +492,7 @@ __device__ void gp_scan(const FzParams& p, const GpShared& s, const Unit& x, int
     if (j < n) {
       const int pg = pg0 + j;
       if (hidx == 0) {
-        Us[j] = U;
+        p.wk.U[(long long)x.u * p.wk.Ustride + pg] = U;
         if (p.dbg.page_U) p.dbg.page_U[(long long)x.u * dm.np_max + pg] = U;
       }
       if (p.dbg.page_ub && hidx < G)
@@ -442,68 +502,66 @@ __device__ void gp_scan(const FzParams& p, const GpShared& s, const Unit& x, int
 }
 
 
-// ---- page top-N over the group (larger bound first, ties to the lower page) ----
-// Thread t holds the bounds of local pages [16 t, 16 t + 16).  A level agrees
-// on the members' value range (one group barrier), bins the members into
-// 2048 bins whose counts are added in L2 (one more), keeps every bin above
-// the one holding the need-th largest and descends into that bin.  A bin of
-// at most 512 members is ranked exactly against the whole group's members; a
-// bin of equal bounds (or one still crowded after four levels) is taken in
-// page order.  Returns the CTA's kept pages (ascending, in GW_KP).
-static __device__ int gp_psel(const FzParams& p, const GpShared& s, const Unit& x, int r, int p0, int nr, int N,
-                       unsigned* gx, unsigned& epoch, bool& ok) {
-  const int tid = threadIdx.x;
-  const int S = p.gsize;
+// ---- page top-N of the unit (larger bound first, ties to the lower page) ----
+// Every CTA of the group runs the same select on the unit's bounds (written
+// by the group's scans, read from L2), so all of them know every kept page
+// without another exchange.  Thread t holds the bounds of pages
+// [16 t, 16 t + 16) in registers.  A level bins the undecided pages over
+// their value range into 2048 bins (monotone bin), keeps every bin above the
+// one holding the need-th largest and descends into that bin; a bin of at
+// most 512 pages is ranked exactly (larger bound first, then the lower page),
+// a bin of equal bounds (or one still crowded after four levels) is taken in
+// page order.  Writes the kept pages (ascending) to GW_KP; returns N.
+static __device__ int gp_psel_all(const FzParams& p, const GpShared& s, const Unit& x, int N, bool write_dbg) {
+  const Work& wk = p.wk;
+  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
   unsigned char* w = s.work;
-  const float* Us = reinterpret_cast<const float*>(w + GW_US);
   int* hist = reinterpret_cast<int*>(w + GW_HIST);
-  int2* cand = reinterpret_cast<int2*>(w + GW_CAND);
+  int* cand = reinterpret_cast<int*>(w + GW_CAND);              // int [512]
+  float* candv = reinterpret_cast<float*>(w + GW_CAND + 2048);  // float [512]
   unsigned* flag = reinterpret_cast<unsigned*>(w + GW_FLAG);
   int* red = reinterpret_cast<int*>(w + GW_RED);  // scan buffers of 16 at 0, 16, 32, 48, 64; broadcasts at 128
   int* bc = red + 128;
   float* wr = reinterpret_cast<float*>(red + 160);
   int* kp = reinterpret_cast<int*>(w + GW_KP);
+  const int np = x.np;
   const int i0 = tid * PS_PER;
-  const int cnt = max(0, min(PS_PER, nr - i0));
+  const int cnt = max(0, min(PS_PER, np - i0));
   unsigned member = (1u << cnt) - 1u;
-  float v[PS_PER];
-#pragma unroll
-  for (int k = 0; k < PS_PER; ++k) v[k] = k < cnt ? Us[i0 + k] : 0.f;
   unsigned keep = 0u;
-  if (N >= x.np) {
+  if (N >= np) {
     keep = member;
   } else {
+    const float* Ug = wk.U + (long long)x.u * wk.Ustride;
+    float v[PS_PER];
+#pragma unroll
+    for (int k4 = 0; k4 < PS_PER / 4; ++k4) {
+      const float4 t = i0 + 4 * k4 < np ? __ldcg(reinterpret_cast<const float4*>(Ug + i0) + k4)
+                                        : make_float4(0.f, 0.f, 0.f, 0.f);
+      v[4 * k4 + 0] = t.x; v[4 * k4 + 1] = t.y; v[4 * k4 + 2] = t.z; v[4 * k4 + 3] = t.w;
+    }
+    for (int i = tid; i < SEL_NBIN; i += FZ_CONS) hist[i] = 0;
+    if (tid < MAX_SELECT_PAGES / 32) flag[tid] = 0u;
+    if (tid == 0) bc[4] = 0;
+    float lo = INFINITY, hi = -INFINITY;
+#pragma unroll
+    for (int k = 0; k < PS_PER; ++k)
+      if ((member >> k) & 1u) {
+        lo = fminf(lo, v[k]);
+        hi = fmaxf(hi, v[k]);
+      }
+    cons_minmax(lo, hi, wr);
     int need = N, nbin = 0;
     bool tie = false;
 #pragma unroll 1
     for (int level = 0; level < GP_LEVELS; ++level) {
-      float lo = INFINITY, hi = -INFINITY;
-#pragma unroll
-      for (int k = 0; k < PS_PER; ++k)
-        if ((member >> k) & 1u) {
-          lo = fminf(lo, v[k]);
-          hi = fmaxf(hi, v[k]);
-        }
-      cons_minmax(lo, hi, wr);
-      float2* mm = reinterpret_cast<float2*>(gx + GX_MM) + level * GP_SMAX;
-      if (tid == 0) mm[r] = make_float2(lo, hi);
-      if (!gp_sync(p, s, gx, epoch)) {
-        ok = false;
-        return 0;
-      }
-      lo = INFINITY;
-      hi = -INFINITY;
-      if (tid < S) {
-        const float2 t = __ldcg(mm + tid);
-        lo = t.x;
-        hi = t.y;
-      }
-      cons_minmax(lo, hi, wr);
       tie = !(hi > lo);
       if (tie) break;
       const float scale = (float)SEL_NBIN / (hi - lo);
-      for (int i = tid; i < SEL_NBIN; i += FZ_CONS) hist[i] = 0;
-      cons_sync();
+      if (level > 0) {
+        for (int i = tid; i < SEL_NBIN; i += FZ_CONS) hist[i] = 0;
+        cons_sync();
+      }
       int bn[PS_PER];
 #pragma unroll
       for (int k = 0; k < PS_PER; ++k) {
@@ -511,22 +569,13 @@ static __device__ int gp_psel(const FzParams& p, const GpShared& s, const Unit& 
         if ((member >> k) & 1u) atomicAdd(&hist[bn[k]], 1);
       }
       cons_sync();
-      int* gh = reinterpret_cast<int*>(gx + GX_HIST) + level * SEL_NBIN;
-      for (int i = tid; i < SEL_NBIN; i += FZ_CONS) {
-        const int h = hist[i];
-        if (h) atomicAdd(gh + i, h);
-      }
-      if (!gp_sync(p, s, gx, epoch)) {
-        ok = false;
-        return 0;
-      }
       {
         constexpr int BPT = SEL_NBIN / FZ_CONS;  // 4 bins per thread, counted from the top
         int hv[BPT];
         int c4 = 0;
 #pragma unroll
         for (int e = 0; e < BPT; ++e) {
-          hv[e] = __ldcg(gh + SEL_NBIN - 1 - (tid * BPT + e));
+          hv[e] = hist[SEL_NBIN - 1 - (tid * BPT + e)];
           c4 += hv[e];
         }
         int tot;
@@ -548,30 +597,27 @@ static __device__ int gp_psel(const FzParams& p, const GpShared& s, const Unit& 
       const int bstar = bc[0];
       need = bc[1];
       nbin = bc[2];
+      float nlo = INFINITY, nhi = -INFINITY;
 #pragma unroll
       for (int k = 0; k < PS_PER; ++k) {
         const bool m = (member >> k) & 1u;
+        const bool at = m && bn[k] == bstar;
         keep |= (m && bn[k] > bstar) ? 1u << k : 0u;
-        member &= (m && bn[k] == bstar) ? ~0u : ~(1u << k);
+        member &= at ? ~0u : ~(1u << k);
+        nlo = at ? fminf(nlo, v[k]) : nlo;
+        nhi = at ? fmaxf(nhi, v[k]) : nhi;
       }
       if (nbin <= SEL_MAX_CAND) break;
+      cons_minmax(nlo, nhi, wr);
+      lo = nlo;
+      hi = nhi;
     }
     if (tie || nbin > SEL_MAX_CAND) {
       // equal bounds (or still crowded): members in page order, the first `need`
       const int m = __popc(member);
-      int mt;
-      const int mb = cons_scan1(m, red + 32, &mt);
-      int* pubt = reinterpret_cast<int*>(gx + GX_PUBT);
-      if (tid == 0) pubt[r] = mt;
-      if (!gp_sync(p, s, gx, epoch)) {
-        ok = false;
-        return 0;
-      }
-      int tt;
-      const int bt = cons_scan1(tid < S ? __ldcg(pubt + tid) : 0, red + 48, &tt);
-      if (tid == r) bc[3] = bt;
-      cons_sync();
-      int take = max(0, min(m, need - bc[3] - mb));
+      int tot;
+      const int mb = cons_scan1(m, red + 32, &tot);
+      int take = max(0, min(m, need - mb));
 #pragma unroll
       for (int k = 0; k < PS_PER; ++k) {
         if (((member >> k) & 1u) && take > 0) {
@@ -580,34 +626,24 @@ static __device__ int gp_psel(const FzParams& p, const GpShared& s, const Unit& 
         }
       }
     } else {
-      // exact ranking of the threshold bin's members across the group
-      int2* gc = reinterpret_cast<int2*>(gx + GX_CAND);
-      for (int i = tid; i < MAX_SELECT_PAGES / 32; i += FZ_CONS) flag[i] = 0u;
+      // exact ranking of the (few) members: larger bound first, then lower page
 #pragma unroll
       for (int k = 0; k < PS_PER; ++k)
         if ((member >> k) & 1u) {
-          const unsigned at = atomicAdd(gx + GX_CCOUNT, 1u);
-          if (at < (unsigned)SEL_MAX_CAND) gc[at] = make_int2(__float_as_int(v[k]), p0 + i0 + k);
+          const int at = atomicAdd(&bc[4], 1);
+          cand[at] = i0 + k;
+          candv[at] = v[k];
         }
-      if (!gp_sync(p, s, gx, epoch)) {
-        ok = false;
-        return 0;
-      }
-      for (int a = tid; a < nbin; a += FZ_CONS) cand[a] = __ldcg(gc + a);
       cons_sync();
       for (int a = tid; a < nbin; a += FZ_CONS) {
-        const int2 ea = cand[a];
-        const int pa = ea.y - p0;
-        if (pa >= 0 && pa < nr) {
-          const float va = __int_as_float(ea.x);
-          int rank = 0;
-          for (int b2 = 0; b2 < nbin; ++b2) {
-            const int2 eb = cand[b2];
-            const float vb = __int_as_float(eb.x);
-            rank += (vb > va) || (vb == va && eb.y < ea.y);
-          }
-          if (rank < need) atomicOr(&flag[pa >> 5], 1u << (pa & 31));
+        const int ia = cand[a];
+        const float va = candv[a];
+        int rank = 0;
+        for (int b2 = 0; b2 < nbin; ++b2) {
+          const float vb = candv[b2];
+          rank += (vb > va) || (vb == va && cand[b2] < ia);
         }
+        if (rank < need) atomicOr(&flag[ia >> 5], 1u << (ia & 31));
       }
       cons_sync();
       const unsigned fw = flag[i0 >> 5] >> (i0 & 31);  // the thread's 16 pages share one flag word
@@ -616,21 +652,31 @@ static __device__ int gp_psel(const FzParams& p, const GpShared& s, const Unit& 
   }
   int nkp;
   int pos = cons_scan1(__popc(keep), red + 64, &nkp);
+  int* dsel = (write_dbg && p.dbg.sel_pages) ? p.dbg.sel_pages + (long long)x.u * wk.Nmax : nullptr;
 #pragma unroll
   for (int k = 0; k < PS_PER; ++k)
-    if ((keep >> k) & 1u) kp[pos++] = p0 + i0 + k;
+    if ((keep >> k) & 1u) {
+      kp[pos] = i0 + k;
+      if (dsel) dsel[pos] = i0 + k;
+      ++pos;
+    }
+  if (write_dbg && tid == 0 && p.dbg.n_sel_pages) p.dbg.n_sel_pages[x.u] = nkp;
+  (void)lane;
+  (void)warp;
   cons_sync();
   return nkp;
 }
 
-
-// ---- Hamming scores of the CTA's candidate rows, key top-k over the group ----
-// (smaller score first, ties to the lower row).  Candidates are the rows of
-// the CTA's kept pages in page order; the group histogram of the integer
-// scores gives the threshold T and the ties taken; per-CTA counts of rows
-// below T and at T, published and scanned in CTA order (= row order), give
-// each CTA its ties and its place in the unit's row list.  Returns k_eff; the
-// list is complete when it returns (group barrier).
+// ---- Hamming scores and key top-k of the unit (smaller score first, ties
+// to the lower row), one group barrier ----
+// Candidates are the rows of the kept pages in page order; CTA r scores the
+// balanced share [cs0, cs1) and publishes the histogram of its integer scores
+// (G nb + 1 bins).  After the barrier every CTA reads the S histograms: their
+// sum gives the threshold T and the ties taken at T; the histograms of the
+// CTAs before r give r's place in the row list (rows below T of lower CTAs,
+// plus their ties, which go to the lower rows first).  The CTA writes its kept
+// rows there as row + 1 (0 = not yet written), so that the gather of a chunk
+// polls only the entries it needs.  Returns k_eff.
 template <int G, int WORDS>
 __device__ int gp_ksel(const FzParams& p, const GpShared& s, const Unit& x, int r, int nkp, unsigned* gx,
                        unsigned& epoch, bool& ok) {
@@ -644,8 +690,14 @@ __device__ int gp_ksel(const FzParams& p, const GpShared& s, const Unit& x, int 
   int* bc = red + 128;
   const int* kp = reinterpret_cast<const int*>(w + GW_KP);
   uint16_t* sc = reinterpret_cast<uint16_t*>(w + GW_SC);
+  int* hm = reinterpret_cast<int*>(s.ring);         // the S histograms [S][HB] (the ring is idle here)
+  int* ltc = reinterpret_cast<int*>(w + GW_CAND);   // [S] rows below T per CTA
   const int nbins = G * dm.nb + 1;
+  const int HB = wk.HB;
   const int ncs = nkp << dm.lgP;
+  int cs0, cs1;
+  share_of(ncs, S, r, cs0, cs1);
+  const int nmy = cs1 - cs0;
   for (int i = tid; i < nbins; i += FZ_CONS) hist[i] = 0;
   uint64_t cq[G][WORDS];
 #pragma unroll
@@ -653,9 +705,8 @@ __device__ int gp_ksel(const FzParams& p, const GpShared& s, const Unit& x, int 
 #pragma unroll
     for (int w2 = 0; w2 < WORDS; ++w2)
       cq[g][w2] = (uint64_t)s.qc[g * 8 + 2 * w2] | ((uint64_t)s.qc[g * 8 + 2 * w2 + 1] << 32);
-  // ---- scores (four rows per thread in flight) ----
-  int nval = 0;
-  for (int j0 = 0; j0 < ncs; j0 += 4 * FZ_CONS) {
+  // ---- scores of the CTA's share (four rows per thread in flight) ----
+  for (int j0 = 0; j0 < nmy; j0 += 4 * FZ_CONS) {
     uint64_t cw[4][WORDS];
     bool valid[4];
 #pragma unroll
@@ -664,8 +715,9 @@ __device__ int gp_ksel(const FzParams& p, const GpShared& s, const Unit& x, int 
       valid[e] = false;
 #pragma unroll
       for (int w2 = 0; w2 < WORDS; ++w2) cw[e][w2] = 0ull;
-      if (j < ncs) {
-        const int t = (kp[j >> dm.lgP] << dm.lgP) + (j & (dm.P - 1));
+      if (j < nmy) {
+        const int ci = cs0 + j;
+        const int t = (kp[ci >> dm.lgP] << dm.lgP) + (ci & (dm.P - 1));
         if (t < x.L) {
           const long long woff = code_row(dm, p.table, x.b, x.h, t, p.status);
           if (woff >= 0) {
@@ -688,48 +740,61 @@ __device__ int gp_ksel(const FzParams& p, const GpShared& s, const Unit& x, int 
 #pragma unroll
     for (int e = 0; e < 4; ++e) {
       const int j = j0 + e * FZ_CONS + tid;
-      if (j < ncs) {
+      if (j < nmy) {
         int sv = 0;
 #pragma unroll
         for (int g = 0; g < G; ++g)
 #pragma unroll
           for (int w2 = 0; w2 < WORDS; ++w2) sv += __popcll(cq[g][w2] ^ cw[e][w2]);
         sc[j] = valid[e] ? (uint16_t)sv : (uint16_t)0xFFFFu;
-        nval += valid[e] ? 1 : 0;
       }
     }
   }
   cons_sync();  // scores complete, histogram zero
-  for (int j = tid; j < ncs; j += FZ_CONS) {
+  for (int j = tid; j < nmy; j += FZ_CONS) {
     const int sv = sc[j];
     if (sv != 0xFFFF) atomicAdd(&hist[sv], 1);
   }
-  int cval;
-  (void)cons_scan1(nval, red, &cval);  // (its barrier also completes the histogram)
-  int* gh = reinterpret_cast<int*>(gx + GX_KHIST);
-  for (int i = tid; i < nbins; i += FZ_CONS) {
-    const int h = hist[i];
-    if (h) atomicAdd(gh + i, h);
+  cons_sync();
+  // publish the CTA's histogram (one slot per CTA of the grid)
+  int* myh = wk.khist + (long long)blockIdx.x * HB;
+  for (int i = tid; i < nbins; i += FZ_CONS) myh[i] = hist[i];
+  if (p.dbg.key_scores) {
+    int* dsc = p.dbg.key_scores + (long long)x.u * wk.Nmax * dm.P + cs0;
+    for (int j = tid; j < nmy; j += FZ_CONS) {
+      const int sv = sc[j];
+      dsc[j] = sv == 0xFFFF ? INT_MAX : sv;
+    }
   }
-  int2* pub4 = reinterpret_cast<int2*>(gx + GX_PUB4);
-  if (tid == 0) pub4[r] = make_int2(nkp, cval);
   if (!gp_sync(p, s, gx, epoch)) {
     ok = false;
     return 0;
   }
-  // ---- threshold T from the group histogram; the CTAs' page offsets ----
+  // ---- the group's histograms: sum, threshold T, ties ----
+  const int* gh0 = wk.khist + (long long)(blockIdx.x - r) * HB;
+  for (int i = tid; i < S * nbins; i += FZ_CONS) {
+    const int rr = i / nbins, b = i - rr * nbins;
+    hm[rr * HB + b] = __ldcg(gh0 + (long long)rr * HB + b);
+  }
+  cons_sync();
+  for (int b = tid; b < nbins; b += FZ_CONS) {
+    int t = 0;
+    for (int rr = 0; rr < S; ++rr) t += hm[rr * HB + b];
+    hist[b] = t;
+  }
+  if (tid == 0) {
+    bc[0] = -1;  // no candidate: nothing is kept
+    bc[1] = 0;
+  }
+  cons_sync();
   const int bpt = (nbins + FZ_CONS - 1) / FZ_CONS;  // <= 5
   int hv[5];
   int local = 0;
 #pragma unroll
   for (int e = 0; e < 5; ++e) {
     const int bi = tid * bpt + e;
-    hv[e] = (e < bpt && bi < nbins) ? __ldcg(gh + bi) : 0;
+    hv[e] = (e < bpt && bi < nbins) ? hist[bi] : 0;
     local += hv[e];
-  }
-  if (tid == 0) {
-    bc[0] = -1;  // no candidate: nothing is kept
-    bc[1] = 0;
   }
   int n_cand;
   const int before = cons_scan1(local, red + 16, &n_cand);
@@ -746,64 +811,43 @@ __device__ int gp_ksel(const FzParams& p, const GpShared& s, const Unit& x, int 
       run += hv[e];
     }
   }
-  const int2 q4 = tid < S ? __ldcg(pub4 + tid) : make_int2(0, 0);
-  int totp;
-  const int pb = cons_scan1(q4.x, red + 32, &totp);
-  if (tid == r) bc[2] = pb;
   cons_sync();
-  const int T = bc[0], need_eq = bc[1], poff = bc[2];
-  // ---- this CTA's rows below T and at T ----
-  int lt = 0, eq = 0;
-  for (int j = tid; j < ncs; j += FZ_CONS) {
-    const int sv = sc[j];
-    lt += sv < T ? 1 : 0;
-    eq += sv == T ? 1 : 0;
+  const int T = bc[0], need_eq = bc[1];
+  // rows below T of each CTA (warp w: CTAs w, w + 16, ...)
+  for (int rr = warp; rr < S; rr += FZ_CWARPS) {
+    int c = 0;
+    for (int b = lane; b < T; b += 32) c += hm[rr * HB + b];
+#pragma unroll
+    for (int o = 16; o >= 1; o >>= 1) c += __shfl_xor_sync(0xffffffffu, c, o);
+    if (lane == 0) ltc[rr] = c;
   }
-  int tot5;
-  (void)cons_scan1((lt << 16) | eq, red + 48, &tot5);
-  int2* pub5 = reinterpret_cast<int2*>(gx + GX_PUB5);
-  if (tid == 0) pub5[r] = make_int2(tot5 >> 16, tot5 & 0xFFFF);
-  // the stage's outputs: scores in candidate order, kept pages, counts
-  if (p.dbg.key_scores) {
-    int* dsc = p.dbg.key_scores + (long long)x.u * wk.Nmax * dm.P + ((long long)poff << dm.lgP);
-    for (int j = tid; j < ncs; j += FZ_CONS) {
-      const int sv = sc[j];
-      dsc[j] = sv == 0xFFFF ? INT_MAX : sv;
+  cons_sync();
+  if (tid == 0) {
+    int lt_before = 0, eq_before = 0;
+    for (int rr = 0; rr < r; ++rr) {
+      lt_before += ltc[rr];
+      eq_before += T >= 0 ? hm[rr * HB + T] : 0;
     }
+    bc[3] = lt_before + min(need_eq, eq_before);     // the CTA's first place in the list
+    bc[4] = max(0, need_eq - eq_before);             // ties it may take
   }
-  if (p.dbg.sel_pages)
-    for (int i = tid; i < nkp; i += FZ_CONS) p.dbg.sel_pages[(long long)x.u * wk.Nmax + poff + i] = kp[i];
   if (r == 0 && tid == 0) {
-    if (p.dbg.n_sel_pages) p.dbg.n_sel_pages[x.u] = totp;
+    if (p.dbg.n_sel_pages) p.dbg.n_sel_pages[x.u] = nkp;
     if (p.dbg.n_cand) p.dbg.n_cand[x.u] = n_cand;
     if (p.dbg.n_sel_keys) p.dbg.n_sel_keys[x.u] = keff;
   }
-  if (!gp_sync(p, s, gx, epoch)) {
-    ok = false;
-    return 0;
-  }
-  // ---- ties go to the lower CTAs; each CTA's place in the row list ----
-  const int2 q5 = tid < S ? __ldcg(pub5 + tid) : make_int2(0, 0);
-  int tt;
-  const int tb = cons_scan1(q5.y, red + 64, &tt);
-  const int take_t = max(0, min(q5.y, need_eq - tb));
-  int tsel;
-  const int ob = cons_scan1(q5.x + take_t, red + 80, &tsel);
-  if (tid == r) {
-    bc[3] = ob;
-    bc[4] = take_t;
-  }
   cons_sync();
   const int off = bc[3], take = bc[4];
-  // ---- kept rows in candidate order: warp w owns candidates [w nbw, (w+1) nbw)
-  // in rounds of 32; counts per warp, one scan, then ballots place the rows ----
-  const int rounds = (ncs + 32 * FZ_CWARPS - 1) / (32 * FZ_CWARPS);
+  // ---- the CTA's kept rows in candidate order: warp w owns candidates
+  // [w nbw, (w+1) nbw) of the share in rounds of 32; counts per warp, one
+  // scan, then ballots place the rows ----
+  const int rounds = (nmy + 32 * FZ_CWARPS - 1) / (32 * FZ_CWARPS);
   const int cw0 = warp * rounds * 32;
   const unsigned lanemask_lt = (1u << lane) - 1u;
   int lt_w = 0, eq_w = 0;
   for (int rr = 0; rr < rounds; ++rr) {
-    const int ci = cw0 + 32 * rr + lane;
-    const int sv = ci < ncs ? (int)sc[ci] : 0xFFFF;
+    const int j = cw0 + 32 * rr + lane;
+    const int sv = j < nmy ? (int)sc[j] : 0xFFFF;
     lt_w += __popc(__ballot_sync(0xffffffffu, sv < T));
     eq_w += __popc(__ballot_sync(0xffffffffu, sv == T));
   }
@@ -814,28 +858,24 @@ __device__ int gp_ksel(const FzParams& p, const GpShared& s, const Unit& x, int 
   int* dout = p.dbg.sel_keys ? p.dbg.sel_keys + (long long)x.u * wk.Kmax + off : nullptr;
   const int room = keff - off;
   for (int rr = 0; rr < rounds; ++rr) {
-    const int ci = cw0 + 32 * rr + lane;
-    const int sv = ci < ncs ? (int)sc[ci] : 0xFFFF;
+    const int j = cw0 + 32 * rr + lane;
+    const int sv = j < nmy ? (int)sc[j] : 0xFFFF;
     const bool l1 = sv < T, e1 = sv == T;
     const unsigned blt = __ballot_sync(0xffffffffu, l1), beq = __ballot_sync(0xffffffffu, e1);
     const int eq_before = eq_b + __popc(beq & lanemask_lt);
     const bool tk1 = l1 || (e1 && eq_before < take);
     const int pos = lt_b + __popc(blt & lanemask_lt) + min(eq_before, take);
     if (tk1 && pos < room) {
+      const int ci = cs0 + j;
       const int t = (kp[ci >> dm.lgP] << dm.lgP) + (ci & (dm.P - 1));
-      out[pos] = t;
+      out[pos] = t + 1;
       if (dout) dout[pos] = t;
     }
     lt_b += __popc(blt);
     eq_b += __popc(beq);
   }
-  if (!gp_sync(p, s, gx, epoch)) {
-    ok = false;
-    return 0;
-  }
   return keff;
 }
-
 
 // Consumers copy the K'/V rows of one gather step into four ring slots:
 // warp w the rows 8w .. 8w+7 it computes on (K' row j in slot sb + j / 64,
@@ -1050,7 +1090,6 @@ __device__ void gp_consumer(const FzParams& p, const GpShared& s, int g, int r) 
       int p0, p1;
       share_of(x.np, S, r, p0, p1);
       const int nr = p1 - p0;
-      float* Us = reinterpret_cast<float*>(s.work + GW_US);
       for (int j = 0; j < nr; j += FZ_ROWS) {
         const int n = min(FZ_ROWS, nr - j), nsl = (n + GP_PAGES_PER_SLOT - 1) / GP_PAGES_PER_SLOT;
         if (tid == 0) {
@@ -1066,35 +1105,87 @@ __device__ void gp_consumer(const FzParams& p, const GpShared& s, int g, int r) 
           ok = false;
           break;
         }
-        gp_scan<G>(p, s, x, p0 + j, n, (int)(nslot % FZ_NSLOT), Us + j);
+        gp_scan<G>(p, s, x, p0 + j, n, (int)(nslot % FZ_NSLOT));
         cons_sync();
         if (tid == 0)
           for (int k = 0; k < nsl; ++k) mbar_arrive(&s.empty[(nslot + k) % FZ_NSLOT]);
         nslot += nsl;
       }
-      // ---- selects ----
-      int nkp = 0, keff = 0;
+      // ---- the group's bounds are complete: one group barrier ----
+      if (ok) ok = gp_sync(p, s, gx, epoch);
+      // ---- selects, the same in every CTA of the group ----
+      int nkp = 0, keff = 0, k0 = 0, k1 = 0;
       if (ok) {
         const int N = min(min(max(__ldg(p.n_keep + x.b), 1), wk.Nmax), x.np);
-        nkp = gp_psel(p, s, x, r, p0, nr, N, gx, epoch, ok);
-      }
-      if (ok) keff = gp_ksel<G, WORDS>(p, s, x, r, nkp, gx, epoch, ok);
-      if (ok) {
-        // ---- attention over the CTA's chunks of 128 kept rows ----
+        nkp = gp_psel_all(p, s, x, N, r == 0);
+        // L2 prefetches for the producer warp: this CTA's share of the kept
+        // pages' code rows, and (when every candidate row will be kept) the
+        // K'/V rows of the pages its own chunks will gather
+        const bool pf_kv = min(max(__ldg(p.top_k + x.b), 1), wk.Kmax) >= nkp * dm.P;
+        if (tid == 0) {
+          int a0, a1;
+          share_of(nkp, S, r, a0, a1);
+          const int n1 = min(a1 - a0, GP_PF_MAX);
+          int n2 = 0, b0 = 0;
+          if (pf_kv) {
+            const int nch = (nkp * dm.P + FZ_ROWS - 1) / FZ_ROWS;
+            int c0, c1;
+            share_of(nch, S, r, c0, c1);
+            b0 = (c0 * FZ_ROWS) >> dm.lgP;
+            n2 = min(min(nkp, (c1 * FZ_ROWS) >> dm.lgP) - b0, GP_PF_MAX - n1);
+            n2 = max(n2, 0);
+          }
+          misc[22] = n1;
+          misc[23] = n2;
+          misc[24] = a0;
+          misc[25] = b0;
+        }
+        cons_sync();
+        {
+          const int n1 = misc[22], n2 = misc[23], a0 = misc[24], b0 = misc[25];
+          for (int i = tid; i < n1 + n2; i += FZ_CONS) s.pf[i] = i < n1 ? s.kpw[a0 + i] : s.kpw[b0 + i - n1];
+        }
+        cons_sync();
+        if (tid == 0) {
+          __threadfence_block();
+          misc[21] = (int)nunit + 1;
+        }
+        keff = gp_ksel<G, WORDS>(p, s, x, r, nkp, gx, epoch, ok);
         const int nch = (keff + FZ_ROWS - 1) / FZ_ROWS;
         int c0, c1;
         share_of(nch, S, r, c0, c1);
-        const int k0 = c0 * FZ_ROWS;
-        const int nrow = min(keff, c1 * FZ_ROWS) - k0, nst = c1 - c0;
+        k0 = c0 * FZ_ROWS;
+        k1 = min(keff, c1 * FZ_ROWS);
+      }
+      if (ok) {
+        // ---- attention over the CTA's chunks of 128 kept rows ----
+        const int nch = (keff + FZ_ROWS - 1) / FZ_ROWS;
+        const int c0 = k0 / FZ_ROWS;
+        const int nrow = k1 - k0, nst = (nrow + FZ_ROWS - 1) / FZ_ROWS;
         const int* keys = wk.sel_keys + (long long)x.u * wk.Kmax + k0;
         float* parts = wk.part + (long long)x.u * wk.C3 * PS;
-        // row numbers of step i, warp w: rows 8w .. 8w+7 (the rows it copies)
+        // row numbers of step i, warp w: rows 8w .. 8w+7 (the rows it copies).
+        // A list entry holds row + 1 once written (polled, bounded); it is
+        // cleared after reading for the next call.
         auto rows_of = [&](int i, int* rx) {
           if (lane < 8) {
             const int j = warp * 8 + lane, jj = i * FZ_ROWS + j;
             if (jj < nrow) {
-              const int t = __ldcg(keys + jj);
-              const long long off = kv_row(dm, p.table, x.b, x.h, t, p.status);
+              int* e = const_cast<int*>(keys) + jj;
+              int t1 = ld_relaxed32(e);
+              if (t1 == 0) {
+                const long long w0 = clock64();
+                while ((t1 = ld_relaxed32(e)) == 0) {
+                  if (misc[0]) break;
+                  if (clock64() - w0 > FZ_WAIT_CYCLES) {
+                    set_status(p.status, HHR_ERR_TIMEOUT);
+                    misc[0] = 1;
+                    break;
+                  }
+                }
+              }
+              *e = 0;
+              const long long off = t1 > 0 ? kv_row(dm, p.table, x.b, x.h, t1 - 1, p.status) : -1;
               rx[j] = off >= 0 ? (int)(off / D) : -1;
             }
           }
@@ -1126,15 +1217,10 @@ __device__ void gp_consumer(const FzParams& p, const GpShared& s, int g, int r) 
         cons_sync();
         if (misc[18]) {
           merge_partials<G>(s.work, parts, nch, nullptr, p.out + ((long long)x.b * dm.Hq + x.h * G) * D);
-          // the unit's counters and histograms are zero again
-          uint4* z = reinterpret_cast<uint4*>(gx + GX_HIST);
-          for (int i = tid; i < GP_LEVELS * SEL_NBIN / 4; i += FZ_CONS) z[i] = make_uint4(0u, 0u, 0u, 0u);
-          uint4* zk = reinterpret_cast<uint4*>(gx + GX_KHIST);
-          for (int i = tid; i < wk.HB / 4; i += FZ_CONS) zk[i] = make_uint4(0u, 0u, 0u, 0u);
+          // the unit's counters are zero again for the next call
           if (tid == 0) {
             gx[GX_BAR] = 0u;
             gx[GX_ARRIVE] = 0u;
-            gx[GX_CCOUNT] = 0u;
           }
         }
       }
@@ -1204,18 +1290,22 @@ static cudaError_t launch_group_t(const FzParams& prm, int grid, cudaStream_t st
 }
 
 // CTAs per group: the SMs shared out over the units, at most one CTA per 64
-// pages of the longest sequence (a short unit gains nothing from more).
+// pages of the longest sequence (a short unit gains nothing from more), and
+// no more than the ring holds score histograms of.
 inline void group_shape(const Dims& dm, int sms, int* S, int* ngroups) {
   const int U = dm.B * dm.Hkv;
   sms = std::max(1, std::min(sms, (int)GP_SMAX));
   int s = std::max(1, sms / U);
   s = std::min(s, std::max(1, dm.np_max / 64));
+  // the key select holds the group's S score histograms in the ring
+  const int HB = (dm.G * dm.nb + 1 + 7) / 8 * 8;
+  s = std::min(s, std::max(1, (FZ_NSLOT * FZ_SLOT / 4) / HB));
   *S = s;
   *ngroups = std::max(1, std::min(U, sms / s));
 }
 
 
-static_assert(GX_KHIST == GROUP_GX_FIXED_WORDS, "exchange area layout");
+static_assert(GX_WORDS == GROUP_GX_WORDS, "exchange area layout");
 
 template <int G>
 cudaError_t launch_decode(const DecodeArgs& a) {

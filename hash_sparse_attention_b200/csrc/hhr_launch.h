@@ -20,7 +20,7 @@ constexpr int MAX_GRID = 160;            // CTAs of the fused kernel (one per SM
 constexpr int FUSED_GROUP = 16;          // gather chunks merged together first
 constexpr int FUSED_SCORE = 1024;        // candidate rows per score item
 constexpr int MAX_GATHER_GROUPS = 256;   // groups per unit (final merge width)
-constexpr int GROUP_GX_FIXED_WORDS = 11300;  // per-unit exchange area of the group kernel, before the score histogram
+constexpr int GROUP_GX_WORDS = 4;       // per-unit counters of the group kernel
 
 struct DecodeArgs {
   Dims dm;
