@@ -35,6 +35,7 @@ namespace hhr {
 constexpr int GP_WORK = 90112;                 // consumer scratch
 constexpr int GP_SMAX = MAX_GRID;              // CTAs per group at most
 constexpr int GP_LEVELS = 4;                   // page select levels
+constexpr int SEL_RANK_SMALL = 32;             // threshold-bin size ranked without another level
 constexpr int GP_PAGES_PER_SLOT = 32;          // a ring slot: 32 pages of minima, then their maxima
 constexpr size_t GP_OFF_RING = 0;
 constexpr size_t GP_OFF_WORK = GP_OFF_RING + (size_t)FZ_NSLOT * FZ_SLOT;
@@ -182,6 +183,7 @@ static __device__ void gp_producer(const FzParams& p, const GpShared& s, int g, 
         if (*rel < (int)nunit) {
           const long long t0 = clock64();
           while (*rel < (int)nunit) {
+            __nanosleep(256);  // (a tight spin would take issue slots from the consumer warps)
             if (*reinterpret_cast<volatile int*>(s.misc)) {
               ok = false;
               break;
@@ -260,6 +262,7 @@ static __device__ void gp_producer(const FzParams& p, const GpShared& s, int g, 
         if (*rdy < (int)nunit + 1) {
           const long long t0 = clock64();
           while (*rdy < (int)nunit + 1) {
+            __nanosleep(128);
             if (*reinterpret_cast<volatile int*>(s.misc)) {
               ok = false;
               break;
@@ -607,7 +610,8 @@ static __device__ int gp_psel_all(const FzParams& p, const GpShared& s, const Un
         nlo = at ? fminf(nlo, v[k]) : nlo;
         nhi = at ? fmaxf(nhi, v[k]) : nhi;
       }
-      if (nbin <= SEL_MAX_CAND) break;
+      // a small bin is ranked exactly; a larger one is refined (ranking costs nbin^2)
+      if (nbin <= SEL_RANK_SMALL || (nbin <= SEL_MAX_CAND && level == GP_LEVELS - 1)) break;
       cons_minmax(nlo, nhi, wr);
       lo = nlo;
       hi = nhi;
@@ -705,50 +709,43 @@ __device__ int gp_ksel(const FzParams& p, const GpShared& s, const Unit& x, int 
 #pragma unroll
     for (int w2 = 0; w2 < WORDS; ++w2)
       cq[g][w2] = (uint64_t)s.qc[g * 8 + 2 * w2] | ((uint64_t)s.qc[g * 8 + 2 * w2 + 1] << 32);
-  // ---- scores of the CTA's share (four rows per thread in flight) ----
-  for (int j0 = 0; j0 < nmy; j0 += 4 * FZ_CONS) {
-    uint64_t cw[4][WORDS];
-    bool valid[4];
+  // ---- scores of the CTA's share: the code rows are staged in the (idle)
+  // ring by cp.async, all in flight at once, then scored from shared memory ----
+  const int cap = (FZ_NSLOT * FZ_SLOT) / (WORDS * 8);
+  unsigned char* cstage = s.ring;
+  for (int jb = 0; jb < nmy; jb += cap) {
+    const int nbt = min(cap, nmy - jb);
+    for (int j = tid; j < nbt; j += FZ_CONS) {
+      const int ci = cs0 + jb + j;
+      const int t = (kp[ci >> dm.lgP] << dm.lgP) + (ci & (dm.P - 1));
+      const long long woff = t < x.L ? code_row(dm, p.table, x.b, x.h, t, p.status) : -1;
+      sc[jb + j] = woff >= 0 ? 0 : 0xFFFF;
+      if (woff >= 0) {
+        const uint64_t* src = p.codes + woff;
+        if constexpr (WORDS == 1) {
+          asm volatile("cp.async.ca.shared.global [%0], [%1], 8;" ::"r"(smem_u32(cstage + j * 8)), "l"(src) : "memory");
+        } else {
 #pragma unroll
-    for (int e = 0; e < 4; ++e) {
-      const int j = j0 + e * FZ_CONS + tid;
-      valid[e] = false;
-#pragma unroll
-      for (int w2 = 0; w2 < WORDS; ++w2) cw[e][w2] = 0ull;
-      if (j < nmy) {
-        const int ci = cs0 + j;
-        const int t = (kp[ci >> dm.lgP] << dm.lgP) + (ci & (dm.P - 1));
-        if (t < x.L) {
-          const long long woff = code_row(dm, p.table, x.b, x.h, t, p.status);
-          if (woff >= 0) {
-            valid[e] = true;
-            const uint64_t* src = p.codes + woff;
-            if constexpr (WORDS == 1) {
-              cw[e][0] = __ldg(src);
-            } else {
-#pragma unroll
-              for (int w2 = 0; w2 < WORDS; w2 += 2) {
-                const ulonglong2 tt = __ldg(reinterpret_cast<const ulonglong2*>(src + w2));
-                cw[e][w2] = tt.x;
-                cw[e][w2 + 1] = tt.y;
-              }
-            }
-          }
+          for (int w2 = 0; w2 < WORDS; w2 += 2) cp_async16(cstage + (j * WORDS + w2) * 8, src + w2);
         }
       }
     }
+    cp_async_commit();
+    cp_async_wait<0>();
+    cons_sync();
+    for (int j = tid; j < nbt; j += FZ_CONS) {
+      if (sc[jb + j] == 0xFFFF) continue;
+      const uint64_t* cw = reinterpret_cast<const uint64_t*>(cstage + j * WORDS * 8);
+      int sv = 0;
 #pragma unroll
-    for (int e = 0; e < 4; ++e) {
-      const int j = j0 + e * FZ_CONS + tid;
-      if (j < nmy) {
-        int sv = 0;
+      for (int w2 = 0; w2 < WORDS; ++w2) {
+        const uint64_t c = cw[w2];
 #pragma unroll
-        for (int g = 0; g < G; ++g)
-#pragma unroll
-          for (int w2 = 0; w2 < WORDS; ++w2) sv += __popcll(cq[g][w2] ^ cw[e][w2]);
-        sc[j] = valid[e] ? (uint16_t)sv : (uint16_t)0xFFFFu;
+        for (int g = 0; g < G; ++g) sv += __popcll(c ^ cq[g][w2]);
       }
+      sc[jb + j] = (uint16_t)sv;
     }
+    cons_sync();
   }
   cons_sync();  // scores complete, histogram zero
   for (int j = tid; j < nmy; j += FZ_CONS) {
@@ -772,10 +769,9 @@ __device__ int gp_ksel(const FzParams& p, const GpShared& s, const Unit& x, int 
   }
   // ---- the group's histograms: sum, threshold T, ties ----
   const int* gh0 = wk.khist + (long long)(blockIdx.x - r) * HB;
-  for (int i = tid; i < S * nbins; i += FZ_CONS) {
-    const int rr = i / nbins, b = i - rr * nbins;
-    hm[rr * HB + b] = __ldcg(gh0 + (long long)rr * HB + b);
-  }
+  for (int i = tid; i < S * HB / 4; i += FZ_CONS) cp_async16(hm + 4 * i, gh0 + 4 * i);  // all in flight
+  cp_async_commit();
+  cp_async_wait<0>();
   cons_sync();
   for (int b = tid; b < nbins; b += FZ_CONS) {
     int t = 0;
@@ -1075,6 +1071,8 @@ __device__ void gp_consumer(const FzParams& p, const GpShared& s, int g, int r) 
     unsigned* gx = gx_of(p, u);
     unsigned epoch = 0;
     bool ok = true;
+    // the unit's budgets, loaded now (their latency hides behind the prep and the scan)
+    const int nk_b = __ldg(p.n_keep + x.b), tk_b = __ldg(p.top_k + x.b);
     gp_prep<G>(p, s, x, r == 0);  // (q' and the query codes are stage outputs even for an empty sequence)
     if (x.L == 0) {
       if (r == 0) {
@@ -1116,12 +1114,12 @@ __device__ void gp_consumer(const FzParams& p, const GpShared& s, int g, int r) 
       // ---- selects, the same in every CTA of the group ----
       int nkp = 0, keff = 0, k0 = 0, k1 = 0;
       if (ok) {
-        const int N = min(min(max(__ldg(p.n_keep + x.b), 1), wk.Nmax), x.np);
+        const int N = min(min(max(nk_b, 1), wk.Nmax), x.np);
         nkp = gp_psel_all(p, s, x, N, r == 0);
         // L2 prefetches for the producer warp: this CTA's share of the kept
         // pages' code rows, and (when every candidate row will be kept) the
         // K'/V rows of the pages its own chunks will gather
-        const bool pf_kv = min(max(__ldg(p.top_k + x.b), 1), wk.Kmax) >= nkp * dm.P;
+        const bool pf_kv = min(max(tk_b, 1), wk.Kmax) >= nkp * dm.P;
         if (tid == 0) {
           int a0, a1;
           share_of(nkp, S, r, a0, a1);
