@@ -1592,7 +1592,7 @@ __device__ void merge_partials(unsigned char* work, const float* src, int K, flo
   const int g = f >> 5, c4 = f & 31;
   const bool active = part < NPART;
   // prefetch the first batch of this thread's partials
-  constexpr int PF = 8;
+  constexpr int PF = G <= 4 ? 16 : 8;  // (G <= 4: up to 64 partials in one round of loads)
   float4 pv[PF];
 #pragma unroll
   for (int i = 0; i < PF; ++i) {

@@ -1165,9 +1165,12 @@ __device__ void gp_consumer(const FzParams& p, const GpShared& s, int g, int r) 
         // row numbers of step i, warp w: rows 8w .. 8w+7 (the rows it copies).
         // A list entry holds row + 1 once written (polled, bounded); it is
         // cleared after reading for the next call.
-        auto rows_of = [&](int i, int* rx) {
-          if (lane < 8) {
-            const int j = warp * 8 + lane, jj = i * FZ_ROWS + j;
+        // (with two steps, lanes 8-15 poll the entries of step i + 1 into rx + FZ_ROWS at once)
+        auto rows_of = [&](int i, int* rx, bool two) {
+          if (lane < (two ? 16 : 8)) {
+            const int st = lane >> 3;
+            const int j = warp * 8 + (lane & 7), jj = (i + st) * FZ_ROWS + j;
+            if (st) rx = s.ridx + ((i + 1) & 1) * FZ_ROWS;
             if (jj < nrow) {
               int* e = const_cast<int*>(keys) + jj;
               int t1 = ld_relaxed32(e);
@@ -1189,16 +1192,19 @@ __device__ void gp_consumer(const FzParams& p, const GpShared& s, int g, int r) 
           }
           __syncwarp();
         };
-        if (nst > 0) {
-          rows_of(0, s.ridx);
+        if (nst > 0) {  // the first two steps' row lists are polled together
+          rows_of(0, s.ridx, nst > 1);
           gp_gather_rows(s.ring, s.ridx, min(FZ_ROWS, nrow), 0, p.Kr, p.Vc);
+          if (nst > 1) gp_gather_rows(s.ring, s.ridx + FZ_ROWS, min(FZ_ROWS, nrow - FZ_ROWS), 4, p.Kr, p.Vc);
         }
         for (int i = 0; i < nst; ++i) {
           const int n = min(FZ_ROWS, nrow - i * FZ_ROWS);
           if (i + 1 < nst) {
-            int* rx = s.ridx + ((i + 1) & 1) * FZ_ROWS;
-            rows_of(i + 1, rx);
-            gp_gather_rows(s.ring, rx, min(FZ_ROWS, nrow - (i + 1) * FZ_ROWS), 4 * ((i + 1) & 1), p.Kr, p.Vc);
+            if (i >= 1) {
+              int* rx = s.ridx + ((i + 1) & 1) * FZ_ROWS;
+              rows_of(i + 1, rx, false);
+              gp_gather_rows(s.ring, rx, min(FZ_ROWS, nrow - (i + 1) * FZ_ROWS), 4 * ((i + 1) & 1), p.Kr, p.Vc);
+            }
             cp_async_wait<1>();
           } else {
             cp_async_wait<0>();
