@@ -874,8 +874,11 @@ __device__ int gp_ksel(const FzParams& p, const GpShared& s, const Unit& x, int 
 }
 
 // Consumers copy the K'/V rows of one gather step into four ring slots:
-// warp w the rows 8w .. 8w+7 it computes on (K' row j in slot sb + j / 64,
-// V row j two slots further); a bad row reads as zeros.  One cp.async group.
+// warp w the rows 8w .. 8w+7 (K' row j in slot sb + j / 64, V row j two
+// slots further).  The 16-byte chunk q of row j goes to chunk q ^ (j & 7) of
+// its 256-byte row, so that eight consecutive rows' same chunk fall in
+// distinct banks for ldmatrix.  Rows at or past n and bad rows read as zeros
+// (the tensor-core products then stay finite).  One cp.async group.
 __device__ __forceinline__ void gp_gather_rows(unsigned char* ring, const int* ridx, int n, int sb,
                                                const __nv_bfloat16* K, const __nv_bfloat16* V) {
   const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
@@ -883,171 +886,242 @@ __device__ __forceinline__ void gp_gather_rows(unsigned char* ring, const int* r
 #pragma unroll
   for (int i = 0; i < 4; ++i) {
     const int j = warp * 8 + 2 * i + (lane >> 4);
-    if (j < n) {
-      const int r = ridx[j];
-      unsigned char* d1 = ring + (size_t)(sb + j / 64) * FZ_SLOT + (j % 64) * 256 + q * 16;
-      unsigned char* d2 = ring + (size_t)(sb + 2 + j / 64) * FZ_SLOT + (j % 64) * 256 + q * 16;
-      if (r >= 0) {
-        cp_async16(d1, K + (long long)r * D + q * 8);
-        cp_async16(d2, V + (long long)r * D + q * 8);
-      } else {
-        *reinterpret_cast<uint4*>(d1) = make_uint4(0u, 0u, 0u, 0u);
-        *reinterpret_cast<uint4*>(d2) = make_uint4(0u, 0u, 0u, 0u);
-      }
+    const int off = (j % 64) * 256 + ((q ^ (j & 7)) * 16);
+    unsigned char* d1 = ring + (size_t)(sb + j / 64) * FZ_SLOT + off;
+    unsigned char* d2 = ring + (size_t)(sb + 2 + j / 64) * FZ_SLOT + off;
+    const int r = j < n ? ridx[j] : -1;
+    if (r >= 0) {
+      cp_async16(d1, K + (long long)r * D + q * 8);
+      cp_async16(d2, V + (long long)r * D + q * 8);
+    } else {
+      *reinterpret_cast<uint4*>(d1) = make_uint4(0u, 0u, 0u, 0u);
+      *reinterpret_cast<uint4*>(d2) = make_uint4(0u, 0u, 0u, 0u);
     }
   }
   cp_async_commit();
 }
 
-// ---- one gather step: softmax attention over one chunk of 128 kept rows ----
-// The arithmetic of the fused kernel's gather (logits by groups of LPR lanes,
-// warp-local softmax and P.V, 16 warp partials combined in warp order); the
-// chunk's partial (unnormalised output, max and sum of weights per head, in
-// log2 units) goes to `part`.  A chunk's partial depends only on its rows, so
-// results do not depend on how many CTAs share the unit.
-template <int G>
-__device__ void gp_gather_step(const FzParams& p, const GpShared& s, int n, int sb, float* part) {
-  constexpr int GP = G <= 4 ? 4 : 8;
-  constexpr int LPR = GP == 4 ? 8 : 16;
-  constexpr int NCK = 128 / LPR / 8;
-  constexpr int RPG = LPR / 4;
-  constexpr int NV = RPG * GP;
-  constexpr int KP = NV / LPR;
-  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
-  const int grp = lane / LPR, li = lane % LPR;
-  float* OB = reinterpret_cast<float*>(s.work + GA_OB);
-  float2* PB = reinterpret_cast<float2*>(s.work + GA_PB) + warp * 8 * GP;
-  float* MB = reinterpret_cast<float*>(s.work + GA_MB);
-  float* LB = reinterpret_cast<float*>(s.work + GA_LB);
-  const float* qs = s.qs;
-  const float qscale = p.sm_scale * 1.4426950408889634f;
-  float sv[KP];
-  {
-    float2 q2[G][4 * NCK];
-#pragma unroll
-    for (int g = 0; g < G; ++g)
-#pragma unroll
-      for (int k = 0; k < NCK; ++k)
-#pragma unroll
-        for (int h = 0; h < 2; ++h) {
-          const float4 t = *reinterpret_cast<const float4*>(qs + g * D + 4 * (LPR * k + li + 16 * h));
-          q2[g][4 * k + 2 * h] = make_float2(t.x * qscale, t.y * qscale);
-          q2[g][4 * k + 2 * h + 1] = make_float2(t.z * qscale, t.w * qscale);
-        }
-    float v[NV];
-#pragma unroll
-    for (int r = 0; r < RPG; ++r) {
-      const int j = warp * 8 + grp * RPG + r;
-      const unsigned char* row = s.ring + (size_t)(sb + j / 64) * FZ_SLOT + (j % 64) * 256;
-      float2 kf[4 * NCK];
-#pragma unroll
-      for (int k = 0; k < NCK; ++k) {
-        const uint4 kv = *reinterpret_cast<const uint4*>(row + 16 * (LPR * k + li));
-        kf[4 * k] = make_float2(bf_lo(kv.x), bf_hi(kv.x));
-        kf[4 * k + 1] = make_float2(bf_lo(kv.y), bf_hi(kv.y));
-        kf[4 * k + 2] = make_float2(bf_lo(kv.z), bf_hi(kv.z));
-        kf[4 * k + 3] = make_float2(bf_lo(kv.w), bf_hi(kv.w));
-      }
-#pragma unroll
-      for (int g = 0; g < GP; ++g) {
-        float a = 0.f;
-        if (g < G) {
-          float2 a0 = __fmul2_rn(q2[g][0], kf[0]);
-#pragma unroll
-          for (int k = 1; k < 4 * NCK; ++k) a0 = __ffma2_rn(q2[g][k], kf[k], a0);
-          a = a0.x + a0.y;
-        }
-        v[g * RPG + r] = a;
-      }
-    }
-    group_reduce_t<NV, LPR>(v, lane);
-#pragma unroll
-    for (int e = 0; e < KP; ++e) {
-      const int r = (KP * li + e) % RPG;
-      const int j = warp * 8 + grp * RPG + r;
-      sv[e] = ((li >> 1) < G && j < n) ? v[e] : -INFINITY;
-    }
-  }
-  const int gl = li >> 1;
-  float m = sv[0];
-#pragma unroll
-  for (int e = 1; e < KP; ++e) m = fmaxf(m, sv[e]);
-  m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, 1));
-#pragma unroll
-  for (int o = LPR; o < 32; o <<= 1) m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, o));
-  float l = 0.f;
-#pragma unroll
-  for (int e = 0; e < KP; ++e) {
-    const float pv = (sv[e] == -INFINITY) ? 0.f : exp2f(sv[e] - m);
-    const int r = (KP * li + e) % RPG;
-    PB[(grp * RPG + r) * GP + gl] = make_float2(pv, pv);
-    l += pv;
-  }
-  l += __shfl_xor_sync(0xffffffffu, l, 1);
-#pragma unroll
-  for (int o = LPR; o < 32; o <<= 1) l += __shfl_xor_sync(0xffffffffu, l, o);
-  if (lane < LPR && (li & 1) == 0 && gl < G) {
-    MB[warp * 8 + gl] = m;
-    LB[warp * 8 + gl] = l;
-  }
-  __syncwarp();
-  float2 o2[G][2];
-#pragma unroll
-  for (int g = 0; g < G; ++g) o2[g][0] = o2[g][1] = make_float2(0.f, 0.f);
-#pragma unroll
-  for (int r = 0; r < 8; ++r) {
-    const int j = warp * 8 + r;
-    if (j < n) {
-      const uint2 vv = *reinterpret_cast<const uint2*>(s.ring + (size_t)(sb + 2 + j / 64) * FZ_SLOT + (j % 64) * 256 +
-                                                       lane * 8);
-      const float2 v0 = make_float2(bf_lo(vv.x), bf_hi(vv.x)), v1 = make_float2(bf_lo(vv.y), bf_hi(vv.y));
-      float2 pr[GP];
-#pragma unroll
-      for (int g2 = 0; g2 < G; g2 += 2) {
-        const float4 t = *reinterpret_cast<const float4*>(PB + r * GP + g2);
-        pr[g2] = make_float2(t.x, t.y);
-        pr[g2 + 1] = make_float2(t.z, t.w);
-      }
-#pragma unroll
-      for (int g = 0; g < G; ++g) {
-        o2[g][0] = __ffma2_rn(pr[g], v0, o2[g][0]);
-        o2[g][1] = __ffma2_rn(pr[g], v1, o2[g][1]);
-      }
-    }
-  }
-#pragma unroll
-  for (int g = 0; g < G; ++g)
-    *reinterpret_cast<float4*>(OB + (warp * G + g) * D + 4 * lane) =
-        make_float4(o2[g][0].x, o2[g][0].y, o2[g][1].x, o2[g][1].y);
-  cons_sync();
-  if (tid < G * 32) {
-    const int g = warp, c4 = lane;
-    const float mw = MB[(lane & 15) * 8 + g];
-    float M = mw;
-#pragma unroll
-    for (int o = 1; o < 16; o <<= 1) M = fmaxf(M, __shfl_xor_sync(0xffffffffu, M, o));
-    const float sc = (mw == -INFINITY) ? 0.f : exp2f(mw - M);
-    float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
-    float L = 0.f;
-#pragma unroll
-    for (int w = 0; w < FZ_CWARPS; ++w) {
-      const float scw = __shfl_sync(0xffffffffu, sc, w);
-      const float4 a = *reinterpret_cast<const float4*>(OB + (w * G + g) * D + 4 * c4);
-      acc.x = fmaf(scw, a.x, acc.x);
-      acc.y = fmaf(scw, a.y, acc.y);
-      acc.z = fmaf(scw, a.z, acc.z);
-      acc.w = fmaf(scw, a.w, acc.w);
-      L = fmaf(scw, LB[w * 8 + g], L);
-    }
-    *reinterpret_cast<float4*>(part + g * D + 4 * c4) = acc;
-    if (c4 == 0) {
-      part[G * D + g] = M;
-      part[G * D + 8 + g] = L;
-    }
-  }
-  cons_sync();  // the step's scratch and slots are free
+// ---- tensor-core helpers (mma.sync m16n8k16, bf16 in, fp32 accumulate) ----
+__device__ __forceinline__ void ldsm_x4(uint32_t (&r)[4], const void* p) {
+  asm volatile("ldmatrix.sync.aligned.m8n8.x4.shared.b16 {%0,%1,%2,%3}, [%4];"
+               : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]) : "r"(smem_u32(p)));
+}
+__device__ __forceinline__ void ldsm_x4_t(uint32_t (&r)[4], const void* p) {
+  asm volatile("ldmatrix.sync.aligned.m8n8.x4.trans.shared.b16 {%0,%1,%2,%3}, [%4];"
+               : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]) : "r"(smem_u32(p)));
+}
+__device__ __forceinline__ void ldsm_x2(uint32_t (&r)[2], const void* p) {
+  asm volatile("ldmatrix.sync.aligned.m8n8.x2.shared.b16 {%0,%1}, [%2];" : "=r"(r[0]), "=r"(r[1]) : "r"(smem_u32(p)));
+}
+__device__ __forceinline__ void mma_bf16(float (&d)[4], const uint32_t (&a)[4], const uint32_t (&b)[2]) {
+  asm volatile("mma.sync.aligned.m16n8k16.row.col.f32.bf16.bf16.f32 {%0,%1,%2,%3}, {%4,%5,%6,%7}, {%8,%9}, "
+               "{%0,%1,%2,%3};"
+               : "+f"(d[0]), "+f"(d[1]), "+f"(d[2]), "+f"(d[3])
+               : "r"(a[0]), "r"(a[1]), "r"(a[2]), "r"(a[3]), "r"(b[0]), "r"(b[1]));
+}
+// x as bf16 hi + lo (hi = RNE(x), lo = RNE(x - hi)): |x - hi - lo| <= 2^-17 |x|
+__device__ __forceinline__ void split_bf16(float x, __nv_bfloat16& hi, __nv_bfloat16& lo) {
+  hi = __float2bfloat16_rn(x);
+  lo = __float2bfloat16_rn(x - __bfloat162float(hi));
 }
 
+// gather scratch (consumer work area)
+constexpr int GM_QB = 0;                 // bf16 [16 cols][136] q'^T operand (hi, lo), rows 272 B apart
+constexpr int GM_PB = GM_QB + 16 * 272;  // bf16 [16 cols][136] P^T operand (hi, lo)
+constexpr int GM_MX = GM_PB + 16 * 272;  // float [8 warps][8 heads] row-block maxima
+constexpr int GM_LS = GM_MX + 256;       // float [8][8] row-block sums of weights
+constexpr int GM_OB = GM_LS + 256;       // float [2 row halves][128 ch][16 cols] P.V partials
+static_assert(GM_OB + 2 * 128 * 16 * 4 <= GP_WORK, "gather scratch");
+
+// Column layout of the two operands: NT = 1 (G <= 4): columns 0-3 the heads'
+// hi parts, 4-7 their lo parts; NT = 2 (G <= 8): 0-7 hi, 8-15 lo.
+template <int G>
+struct GCols {
+  static constexpr int NT = G <= 4 ? 1 : 2;
+  static constexpr int HP = 4 * NT;  // heads padded
+  __device__ static int hi(int h) { return h; }
+  __device__ static int lo(int h) { return HP + h; }
+};
+
+// q' of the unit, scaled to log2 units, as the hi/lo bf16 operand of the logits.
+template <int G>
+__device__ void gp_build_qb(const FzParams& p, const GpShared& s) {
+  using C = GCols<G>;
+  const float qscale = p.sm_scale * 1.4426950408889634f;
+  __nv_bfloat16* qb = reinterpret_cast<__nv_bfloat16*>(s.work + GM_QB);
+  for (int e = threadIdx.x; e < C::HP * D; e += FZ_CONS) {
+    const int h = e / D, c = e - h * D;
+    const float v = h < G ? s.qs[h * D + qpos(c)] * qscale : 0.f;
+    __nv_bfloat16 hi, lo;
+    split_bf16(v, hi, lo);
+    qb[C::hi(h) * 136 + c] = hi;
+    qb[C::lo(h) * 136 + c] = lo;
+  }
+}
+
+// ---- one gather step: softmax attention over one chunk of up to 128 kept rows ----
+// Logits S = K' (q' hi + lo)^T on tensor cores (warps 0-7, 16 rows each),
+// the chunk's maximum and weights per head in fp32, then O^T = V^T (P hi + lo)^T
+// on tensor cores (warp w: channels 16 (w & 7) .. +15 over rows 64 (w >> 3) .. +63),
+// the two row halves added in order.  The chunk's partial (unnormalised output,
+// maximum and sum of weights per head, in log2 units) goes to `part`; it depends
+// only on the chunk's rows.
+template <int G>
+__device__ void gp_gather_step(const FzParams& p, const GpShared& s, int n, int sb, float* part) {
+  using C = GCols<G>;
+  constexpr int NT = C::NT, HP = C::HP;
+  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+  const int g = lane >> 2, t = lane & 3;
+  unsigned char* w = s.work;
+  const unsigned char* qb = w + GM_QB;
+  __nv_bfloat16* pb = reinterpret_cast<__nv_bfloat16*>(w + GM_PB);
+  float* mx = reinterpret_cast<float*>(w + GM_MX);
+  float* ls = reinterpret_cast<float*>(w + GM_LS);
+  float* ob = reinterpret_cast<float*>(w + GM_OB);
+  cons_sync();  // every warp's rows have landed (each thread waited for its own copies)
+  // ---- logits: warp w < 8 takes rows 16w .. 16w+15 ----
+  float sv[2][2];  // [row g / g+8][head pair element]
+  int h0 = 0;      // first head of this thread's pair
+  if (warp < 8) {
+    float acc[NT][4];
+#pragma unroll
+    for (int nt = 0; nt < NT; ++nt) acc[nt][0] = acc[nt][1] = acc[nt][2] = acc[nt][3] = 0.f;
+    const int r0 = warp * 16;
+    const int arow = r0 + (lane & 7) + ((lane >> 3) & 1) * 8;  // A: this lane's row address
+    const unsigned char* krow = s.ring + (size_t)(sb + arow / 64) * FZ_SLOT + (arow % 64) * 256;
+#pragma unroll
+    for (int ks = 0; ks < 8; ++ks) {
+      uint32_t af[4];
+      ldsm_x4(af, krow + (((2 * ks + (lane >> 4)) ^ (arow & 7)) * 16));
+#pragma unroll
+      for (int nt = 0; nt < NT; ++nt) {
+        uint32_t bf[2];
+        ldsm_x2(bf, qb + (nt * 8 + (lane & 7)) * 272 + (2 * ks + ((lane >> 3) & 1)) * 16);
+        mma_bf16(acc[nt], af, bf);
+      }
+    }
+    // hi + lo of the same heads: NT = 1 pairs columns 2t, 2t+1 with 2t+4, 2t+5
+    // (lane t ^ 2); NT = 2 holds them in its two n-tiles
+    float v0 = acc[0][0], v1 = acc[0][1], v2 = acc[0][2], v3 = acc[0][3];
+    if constexpr (NT == 1) {
+      v0 += __shfl_xor_sync(0xffffffffu, v0, 2);
+      v1 += __shfl_xor_sync(0xffffffffu, v1, 2);
+      v2 += __shfl_xor_sync(0xffffffffu, v2, 2);
+      v3 += __shfl_xor_sync(0xffffffffu, v3, 2);
+      h0 = 2 * (t & 1);
+    } else {
+      v0 += acc[NT - 1][0];
+      v1 += acc[NT - 1][1];
+      v2 += acc[NT - 1][2];
+      v3 += acc[NT - 1][3];
+      h0 = 2 * t;
+    }
+    const bool rg = r0 + g < n, rg8 = r0 + g + 8 < n;
+    sv[0][0] = (rg && h0 < G) ? v0 : -INFINITY;
+    sv[0][1] = (rg && h0 + 1 < G) ? v1 : -INFINITY;
+    sv[1][0] = (rg8 && h0 < G) ? v2 : -INFINITY;
+    sv[1][1] = (rg8 && h0 + 1 < G) ? v3 : -INFINITY;
+    float m0 = fmaxf(sv[0][0], sv[1][0]), m1 = fmaxf(sv[0][1], sv[1][1]);
+#pragma unroll
+    for (int o = 4; o < 32; o <<= 1) {
+      m0 = fmaxf(m0, __shfl_xor_sync(0xffffffffu, m0, o));
+      m1 = fmaxf(m1, __shfl_xor_sync(0xffffffffu, m1, o));
+    }
+    if (g == 0 && (NT == 2 || t < 2)) {
+      mx[warp * 8 + h0] = m0;
+      mx[warp * 8 + h0 + 1] = m1;
+    }
+  }
+  cons_sync();
+  // ---- weights p = 2^(s - M) per head, their sums, P^T as hi / lo ----
+  if (warp < 8) {
+    const int r0 = warp * 16;
+    float M0 = -INFINITY, M1 = -INFINITY;
+#pragma unroll
+    for (int w2 = 0; w2 < 8; ++w2) {
+      M0 = fmaxf(M0, mx[w2 * 8 + h0]);
+      M1 = fmaxf(M1, mx[w2 * 8 + h0 + 1]);
+    }
+    float pw[2][2];
+#pragma unroll
+    for (int rr = 0; rr < 2; ++rr) {
+      pw[rr][0] = sv[rr][0] == -INFINITY ? 0.f : exp2f(sv[rr][0] - M0);
+      pw[rr][1] = sv[rr][1] == -INFINITY ? 0.f : exp2f(sv[rr][1] - M1);
+    }
+    float l0 = pw[0][0] + pw[1][0], l1 = pw[0][1] + pw[1][1];
+#pragma unroll
+    for (int o = 4; o < 32; o <<= 1) {
+      l0 += __shfl_xor_sync(0xffffffffu, l0, o);
+      l1 += __shfl_xor_sync(0xffffffffu, l1, o);
+    }
+    if (NT == 2 || t < 2) {
+      if (g == 0) {
+        ls[warp * 8 + h0] = l0;
+        ls[warp * 8 + h0 + 1] = l1;
+      }
+#pragma unroll
+      for (int rr = 0; rr < 2; ++rr) {
+        const int row = r0 + g + 8 * rr;
+#pragma unroll
+        for (int e = 0; e < 2; ++e) {
+          __nv_bfloat16 hi, lo;
+          split_bf16(pw[rr][e], hi, lo);
+          pb[C::hi(h0 + e) * 136 + row] = hi;
+          pb[C::lo(h0 + e) * 136 + row] = lo;
+        }
+      }
+    }
+  }
+  cons_sync();
+  // ---- O^T = V^T P^T: warp w: channels 16 (w & 7) .., rows 64 (w >> 3) .. ----
+  {
+    const int mt = warp & 7, kh = warp >> 3;
+    float oacc[NT][4];
+#pragma unroll
+    for (int nt = 0; nt < NT; ++nt) oacc[nt][0] = oacc[nt][1] = oacc[nt][2] = oacc[nt][3] = 0.f;
+#pragma unroll
+    for (int ks = 0; ks < 4; ++ks) {
+      const int k0 = kh * 64 + ks * 16;
+      const int vrow = k0 + (lane & 7) + 8 * (lane >> 4);  // matrices 2, 3: rows k0 + 8 ..
+      const int vch = 2 * mt + ((lane >> 3) & 1);           // matrices 1, 3: channels + 8
+      uint32_t af[4];
+      ldsm_x4_t(af, s.ring + (size_t)(sb + 2 + vrow / 64) * FZ_SLOT + (vrow % 64) * 256 + ((vch ^ (vrow & 7)) * 16));
+#pragma unroll
+      for (int nt = 0; nt < NT; ++nt) {
+        uint32_t bf[2];
+        ldsm_x2(bf, reinterpret_cast<const unsigned char*>(pb) + (nt * 8 + (lane & 7)) * 272 +
+                        (k0 / 8 + ((lane >> 3) & 1)) * 16);
+        mma_bf16(oacc[nt], af, bf);
+      }
+    }
+    // rows 16 mt + g (+8) are channels; columns 8 nt + 2t, +1
+#pragma unroll
+    for (int nt = 0; nt < NT; ++nt) {
+      const int c0 = 16 * mt + g, col = 8 * nt + 2 * t;
+      *reinterpret_cast<float2*>(ob + ((kh * 128 + c0) * 16 + col)) = make_float2(oacc[nt][0], oacc[nt][1]);
+      *reinterpret_cast<float2*>(ob + ((kh * 128 + c0 + 8) * 16 + col)) = make_float2(oacc[nt][2], oacc[nt][3]);
+    }
+  }
+  cons_sync();
+  // ---- the chunk's partial: o[h][c] = sum over the row halves of hi + lo columns ----
+  for (int e = tid; e < G * D; e += FZ_CONS) {
+    const int h = e / D, c = e - h * D;
+    const float* o0 = ob + c * 16;
+    const float* o1 = ob + (128 + c) * 16;
+    part[h * D + c] = (o0[C::hi(h)] + o0[C::lo(h)]) + (o1[C::hi(h)] + o1[C::lo(h)]);
+  }
+  if (tid < G) {
+    float M = -INFINITY, L = 0.f;
+#pragma unroll
+    for (int w2 = 0; w2 < 8; ++w2) M = fmaxf(M, mx[w2 * 8 + tid]);
+#pragma unroll
+    for (int w2 = 0; w2 < 8; ++w2) L += ls[w2 * 8 + tid];
+    part[G * D + tid] = M;
+    part[G * D + 8 + tid] = L;
+  }
+  (void)HP;
+  cons_sync();  // the step's scratch and slots are free
+}
 
 // ---------------------------------------------------------------------------
 // consumer warps 0-15: the units of the group, one after another
@@ -1192,6 +1266,7 @@ __device__ void gp_consumer(const FzParams& p, const GpShared& s, int g, int r) 
           }
           __syncwarp();
         };
+        gp_build_qb<G>(p, s);  // (ordered before the first step by its barrier)
         if (nst > 0) {  // the first two steps' row lists are polled together
           rows_of(0, s.ridx, nst > 1);
           gp_gather_rows(s.ring, s.ridx, min(FZ_ROWS, nrow), 0, p.Kr, p.Vc);
