@@ -191,3 +191,28 @@ def test_bad_block_id_sets_status_without_fault():
     torch.cuda.synchronize()
     assert int(status.item()) == 6  # HHR_ERR_BAD_BLOCK
     assert torch.isfinite(out).all()
+
+
+def test_more_units_than_sms():
+    """160 (sequence, KV head) units on a grid of at most one CTA per SM: some
+    CTA groups decode several units one after another (the shared-memory ring,
+    the slot counts and the per-unit counters carry over).  Three calls on one
+    workspace (its counters reset by the kernel) give identical results."""
+    _cuda()
+    w = scaled(WORKLOADS["llama_layer_32k"], context=3000, batch=20, seed=21)
+    li = make_layer(w)
+    g, rep = _run_and_check(w, li, e2e=False)
+    r = parity.run_gpu(w, li, to_host=False)
+    assert r.status == 0
+    cache, ws = r.extra["cache"], r.extra["ws"]
+    dev = torch.device("cuda")
+    q, R, W = li.q.to(dev), li.R.to(dev), li.W.to(dev)
+    seq, nk, tk = li.seq_lens.to(dev), li.n_keep.to(dev), li.top_k.to(dev)
+    status = torch.zeros(1, dtype=torch.int32, device=dev)
+    for _ in range(2):
+        out = torch.full_like(r.out, float("nan"))
+        hhr.decode_step(r.cfg, q, R, W, cache, seq, None, nk, tk, r.Nmax, r.Kmax, out, ws, status=status)
+        torch.cuda.synchronize()
+        assert int(status.item()) == 0
+        assert torch.equal(out, r.out)
+    assert np.array_equal(g.out, r.out.cpu().numpy().astype(np.float64))
