@@ -422,7 +422,8 @@ def run_hhr(args, rank, world):
                 "frac": achieved / pk["hbm_gbs"], "traffic": profiled_traffic(w.name),
                 "algorithmic_bytes_per_launch": statistics.mean(per_layer_bytes),
                 "kernel": "hhr_group_kernel (one launch per layer; one group of CTAs per KV head: query prep, "
-                          "page scan, distributed page and key select, sparse attention, chunk-partial merge)",
+                          "page scan, page select, distributed key select, tensor-core sparse attention, "
+                          "chunk-partial merge)",
                 "peak_source": pk["source"],
                 "step_gbs": step_bytes / t_step / 1e9, "step_frac": step_bytes / t_step / 1e9 / pk["hbm_gbs"]}
     launches_per_step = len(layers)  # one hhr_group_kernel launch per layer
