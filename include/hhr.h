@@ -163,6 +163,16 @@ HHR_API hhr_status hhr_workspace_init(void* workspace, size_t workspace_bytes, h
  * NULL.  `workspace` must be at least hhr_decode_workspace_size() bytes,
  * 256-byte aligned, zeroed once with hhr_workspace_init(), and not shared by
  * calls that may run concurrently.  `device_status` may be NULL.
+ *
+ * One kernel launch, at most one CTA per SM; the CTAs of a group that shares
+ * a (sequence, KV head) wait for one another, so the launch expects the SMs
+ * it was sized for (a kernel occupying SMs on another stream only delays
+ * it).  Every device-side wait is bounded: on expiry the launch records
+ * HHR_ERR_TIMEOUT in `device_status` and returns.  After any call whose
+ * status is not HHR_OK, zero the workspace again (hhr_workspace_init) before
+ * the next call: its counters and row list may be left mid-use.  Results are
+ * deterministic and do not depend on the batch composition or on the layout
+ * (contiguous or paged).
  */
 HHR_API hhr_status hhr_decode_step(const hhr_config* cfg, const void* q, const float* R, const void* W,
                            const void* Krot, const void* Vcache, const void* page_min,
