@@ -65,3 +65,29 @@ def test_max_over_ranks_gloo_two_ranks():
         assert p.exitcode == 0
     got = sorted(q.get(timeout=10) for _ in range(2))
     assert got == [(0, 2.0), (1, 2.0)]
+
+
+def test_build_report_counts_rows_bytes_and_fma():
+    """The cache-build line: median over layers after the first, fp32 FMA and
+    HBM ceilings from the unit counts (no GPU needed)."""
+    import bench
+    from hash_sparse_attention_b200.synth import WORKLOADS
+
+    class Ev:
+        def __init__(self, t):
+            self.t = t
+
+        def elapsed_time(self, other):
+            return other.t - self.t
+
+    w = WORKLOADS["llama_32l_128k"]
+    ev = [(Ev(0.0), Ev(9.0)), (Ev(0.0), Ev(4.0)), (Ev(0.0), Ev(2.0)), (Ev(0.0), Ev(3.0))]
+    r = bench.build_report(w, [{"lens": [131072]}], ev, {"sm_max_mhz": 2000.0}, 100, {"hbm_gbs": 1000.0})
+    assert r["ms_per_layer"] == 3.0  # median of 4, 2, 3 (the first layer is left out)
+    rows = 8 * 131072
+    assert r["rows_per_layer"] == rows
+    assert r["fma_per_layer"] == rows * 128 * (128 + 128)
+    pages = 8 * 131072 // 16
+    assert r["algorithmic_bytes_per_layer"] == rows * (512 + 16) + pages * 512 + 8 * (128 * 128 * 4 + 128 * 128 * 2)
+    assert abs(r["peak"] - 100 * 128 * 2000e6 / 1e12) < 1e-9
+    assert abs(r["frac"] - r["fma_per_layer"] / 3e-3 / (100 * 128 * 2000e6)) < 1e-12
