@@ -26,7 +26,7 @@ struct Work {
   uint64_t* qcodes;    // [B, Hq, w]        query sign codes
   float* U;            // [B, Hkv, Ustride] page bounds (group max)
   int* sel_pages;      // [B, Hkv, Nmax]    kept pages, ascending
-  int* sel_keys;       // [B, Hkv, Kmax]    kept rows, ascending
+  int* sel_keys;       // [B, Hkv, Kmax]    kept rows, ascending (group kernel: row + 1, cleared after reading)
   float* part;         // [B, Hkv, C3, G * D + 16] attention partial of every gather chunk
   float* gpart;        // [B, Hkv, max_groups, G * D + 16] merged groups of chunks
   uint16_t* kscore;    // [B, Hkv, Cmax]    Hamming score of every candidate row

@@ -1,4 +1,8 @@
 // HHR decode step as one persistent, warp-specialised kernel per layer (sm_100a).
+// The library launches it for the dense comparison (DENSE = 1: every row, no
+// selects); the sparse decode step runs in hhr_group.cuh, which also uses the
+// device helpers of this file (mbarriers, bulk copies, scans, reductions, the
+// partial merge).  The sparse items below are not instantiated.
 //
 // Work is a queue of items claimed in order by the CTAs (one CTA per SM).
 // For units u = (sequence b, KV head h) the queue holds, in this order:

@@ -1,25 +1,27 @@
 // HHR decode step with CTA groups: one group of S CTAs per unit (sequence b,
 // KV head h), every CTA of a group owning a contiguous share of the unit's
-// pages and, after the selects, a balanced share of its kept rows (sm_100a).
+// pages and, after the selects, a share of the chunks of its kept rows (sm_100a).
 //
 // Per unit, CTA r of the group:
 //   1. computes q' = R_h q and the query sign codes itself (R_h, W_h and q are
 //      read by every CTA of the group; the copies after the first hit L2),
 //      while its producer warp already streams the page metadata of its share
 //      into the shared-memory ring;
-//   2. scans its pages: U = max over the group's heads of the page bound;
-//   3. page top-N, distributed: the group agrees on the global value range,
-//      bins its bounds (2048 bins per level, counts added in L2), descends
-//      into the bin that holds the N-th largest and ranks that bin's members
-//      exactly (larger bound first, then the lower page);
-//   4. scores the rows of the pages it kept (Hamming distance summed over the
-//      group's heads), adds their histogram in L2; the threshold score and the
-//      ties every CTA may take follow from the histogram and the per-CTA
-//      counts (CTAs own ascending page ranges, so CTA order is row order);
-//   5. writes its kept rows at their place in the unit's row list and, after
-//      one more group barrier, gathers the K'/V rows of its share of that
-//      list's chunks of 128 rows (cp.async by the consumer warps, one chunk
-//      ahead), one softmax partial per chunk;
+//   2. scans its pages: U = max over the group's heads of the page bound,
+//      written to the workspace; one group barrier;
+//   3. runs the page top-N on all the unit's bounds (read from L2), the same
+//      in every CTA of the group: value-bin histograms, refined while the
+//      threshold bin is crowded, then an exact ranking (larger bound first,
+//      then the lower page), so every CTA knows every kept page;
+//   4. scores its balanced share of the candidate rows (the rows of the kept
+//      pages in page order; Hamming distance summed over the group's heads)
+//      and publishes the histogram of its scores; one group barrier; the S
+//      histograms give the threshold, the ties taken and the CTA's place in
+//      the unit's row list (CTA order is row order);
+//   5. writes its kept rows there (row + 1; readers poll the entries) and
+//      gathers the K'/V rows of its share of that list's chunks of 128 rows
+//      (cp.async by the consumer warps, one chunk ahead; logits and P.V on
+//      tensor cores), one softmax partial per chunk;
 //   6. the last CTA of the group to arrive merges the chunk partials in chunk
 //      order into the output and clears the unit's counters (the result does
 //      not depend on the number of CTAs per group).
