@@ -91,3 +91,29 @@ def test_build_report_counts_rows_bytes_and_fma():
     assert r["algorithmic_bytes_per_layer"] == rows * (512 + 16) + pages * 512 + 8 * (128 * 128 * 4 + 128 * 128 * 2)
     assert abs(r["peak"] - 100 * 128 * 2000e6 / 1e12) < 1e-9
     assert abs(r["frac"] - r["fma_per_layer"] / 3e-3 / (100 * 128 * 2000e6)) < 1e-12
+
+
+def test_profiled_traffic_only_for_matching_sources_and_workload(tmp_path, monkeypatch):
+    """roofline.traffic comes from the committed profile summary only when it
+    was taken on the current kernel sources and the same workload."""
+    import bench
+
+    prof = tmp_path / "profiles"
+    prof.mkdir()
+    f = prof / "hhr_group_kernel_llama_32l_128k.md"
+    monkeypatch.setattr(bench, "ROOT", str(tmp_path))
+    assert bench.profiled_traffic("llama_32l_128k") is None  # no summary
+    monkeypatch.setattr(bench, "kernel_source_hash", lambda: "abc123")
+    f.write_text("- workload: `llama_32l_128k`\n- dram_bytes_per_launch: `1234`\n- sources_sha256: `abc123`\n")
+    assert bench.profiled_traffic("llama_32l_128k") == 1234.0
+    assert bench.profiled_traffic("qwen_gqa7_128k") is None  # another workload
+    f.write_text("- workload: `llama_32l_128k`\n- dram_bytes_per_launch: `1234`\n- sources_sha256: `def456`\n")
+    assert bench.profiled_traffic("llama_32l_128k") is None  # sources changed since the capture
+    f.write_text("- workload: `llama_32l_128k`\n- sources_sha256: `abc123`\n")
+    assert bench.profiled_traffic("llama_32l_128k") is None  # no figure
+
+
+def test_kernel_source_hash_tracks_the_sources():
+    import bench
+    h1 = bench.kernel_source_hash()
+    assert len(h1) == 64 and h1 == bench.kernel_source_hash()
