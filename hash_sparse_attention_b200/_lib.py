@@ -46,6 +46,7 @@ _cfgp = ctypes.POINTER(HHRConfig)
 SIGNATURES = {
     "hhr_status_string": (ctypes.c_char_p, [_i32]),
     "hhr_last_error": (ctypes.c_char_p, []),
+    "hhr_set_wait_limit": (None, [ctypes.c_int64]),
     "hhr_build_cache": (_i32, [_cfgp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp]),
     "hhr_decode_workspace_size": (_sz, [_cfgp, _i32, _i32]),
     "hhr_workspace_init": (_i32, [_vp, _sz, _vp]),

@@ -1,17 +1,20 @@
 // C ABI of libhhr.so: argument validation, workspace carve-out and launches.
-// The kernels live in hhr_build.cuh, hhr_fused.cuh (dense) and hhr_group.cuh (decode step).
+// The kernels live in hhr_build.cuh (cache build), hhr_decode.cuh (decode
+// step) and hhr_dense.cuh (dense comparison).
 #include <algorithm>
+#include <atomic>
 #include <cstdarg>
 #include <cstdio>
 #include <cstring>
 
-#include "hhr_launch.h"
+#include "hhr_api_internal.h"
 
 using namespace hhr;
 
 namespace {
 
 thread_local char g_err[512] = {0};
+std::atomic<long long> g_wait_cycles{DEFAULT_WAIT_CYCLES};
 
 hhr_status fail(hhr_status s, const char* fmt, ...) {
   va_list ap;
@@ -34,111 +37,9 @@ hhr_status check_cuda(const char* what) {
   return HHR_OK;
 }
 
-// Validates the configuration and fills the kernel-side dimensions.
-hhr_status make_dims(const hhr_config* cfg, Dims* dm) {
-  if (!cfg) return fail(HHR_ERR_INVALID_ARG, "cfg is NULL");
-  if (cfg->head_dim != D) return fail(HHR_ERR_UNSUPPORTED, "head_dim %d (only 128)", cfg->head_dim);
-  if (cfg->batch < 1 || cfg->num_kv_heads < 1 || cfg->num_q_heads < 1 || cfg->max_seq_len < 1)
-    return fail(HHR_ERR_INVALID_ARG, "batch, heads and max_seq_len must be >= 1");
-  if (cfg->num_q_heads % cfg->num_kv_heads != 0)
-    return fail(HHR_ERR_INVALID_ARG, "num_q_heads %d not a multiple of num_kv_heads %d", cfg->num_q_heads,
-                cfg->num_kv_heads);
-  const int G = cfg->num_q_heads / cfg->num_kv_heads;
-  if (G > 8) return fail(HHR_ERR_UNSUPPORTED, "group size %d (1..8)", G);
-  if (cfg->page_size != 16 && cfg->page_size != 32)
-    return fail(HHR_ERR_UNSUPPORTED, "page_size %d (16 or 32)", cfg->page_size);
-  if (cfg->hash_bits != 64 && cfg->hash_bits != 128 && cfg->hash_bits != 256)
-    return fail(HHR_ERR_UNSUPPORTED, "hash_bits %d (64, 128 or 256)", cfg->hash_bits);
-  const long long np_max = ((long long)cfg->max_seq_len + cfg->page_size - 1) / cfg->page_size;
-  if (np_max > MAX_DENSE_PAGES)
-    return fail(HHR_ERR_UNSUPPORTED, "%lld pages per sequence (at most %d)", np_max, MAX_DENSE_PAGES);
-  if (cfg->paged) {
-    if (cfg->num_blocks < 1) return fail(HHR_ERR_INVALID_ARG, "paged: num_blocks must be >= 1");
-    if (cfg->max_blocks_per_seq < np_max)
-      return fail(HHR_ERR_INVALID_ARG, "paged: max_blocks_per_seq %d < ceil(max_seq_len / page_size) %lld",
-                  cfg->max_blocks_per_seq, np_max);
-  }
-  dm->B = cfg->batch;
-  dm->Hq = cfg->num_q_heads;
-  dm->Hkv = cfg->num_kv_heads;
-  dm->G = G;
-  dm->P = cfg->page_size;
-  dm->lgP = cfg->page_size == 16 ? 4 : 5;
-  dm->nb = cfg->hash_bits;
-  dm->words = cfg->hash_bits / 64;
-  dm->T = cfg->max_seq_len;
-  dm->np_max = (int)np_max;
-  dm->paged = cfg->paged ? 1 : 0;
-  dm->num_blocks = cfg->paged ? cfg->num_blocks : 0;
-  dm->max_blocks = cfg->paged ? cfg->max_blocks_per_seq : 0;
-  return HHR_OK;
-}
-
 size_t align256(size_t x) { return (x + 255) & ~size_t(255); }
 
 int ceil_div(long long a, long long b) { return (int)((a + b - 1) / b); }
-
-// Chunk counts of the fused kernel: scan chunks and gather chunks per unit.
-void chunk_counts(const Dims& dm, int Nmax, int Kmax, bool dense, int* C1, int* C2, int* C3) {
-  if (dense) {
-    *C1 = 0;
-    *C2 = 0;
-    *C3 = ceil_div(dm.T, FUSED_ROWS);
-  } else {
-    *C1 = ceil_div(dm.np_max, FUSED_ROWS);
-    *C2 = ceil_div((long long)Nmax * dm.P, FUSED_SCORE);
-    const long long kcap = std::min<long long>(Kmax, (long long)Nmax * dm.P);
-    *C3 = std::max(1, ceil_div(kcap, FUSED_ROWS));
-  }
-}
-
-// Carves the workspace; with base == nullptr only the size is computed.
-size_t carve(const Dims& dm, int Nmax, int Kmax, bool dense, char* base, Work* wk) {
-  const size_t BH = (size_t)dm.B * dm.Hkv;
-  int C1, C2, C3;
-  chunk_counts(dm, Nmax, Kmax, dense, &C1, &C2, &C3);
-  const int max_groups = ceil_div(C3, FUSED_GROUP);
-  size_t off = 0;
-  auto take = [&](size_t bytes) {
-    char* p = base ? base + off : nullptr;
-    off += align256(bytes);
-    return p;
-  };
-  Work w{};
-  w.ctrl = reinterpret_cast<unsigned*>(take(sizeof(unsigned) * (4 + BH * (8 + max_groups))));
-  w.qrot = reinterpret_cast<float*>(take(sizeof(float) * dm.B * dm.Hq * D));
-  w.qcodes = reinterpret_cast<uint64_t*>(take(sizeof(uint64_t) * dm.B * dm.Hq * dm.words));
-  w.part = reinterpret_cast<float*>(take(sizeof(float) * BH * C3 * (dm.G * D + 16)));
-  w.gpart = reinterpret_cast<float*>(take(sizeof(float) * BH * max_groups * (dm.G * D + 16)));
-  // grid-wide tasks per unit: page select, key select, the final merge
-  const int tq_cap = (int)(BH * 3);
-  w.tq = reinterpret_cast<int4*>(take(sizeof(int4) * tq_cap));
-  w.tq_cap = tq_cap;
-  const int Ustride = (dm.np_max + 31) / 32 * 32;
-  const int Cmax = Nmax * dm.P;
-  const int HB = (dm.G * dm.nb + 1 + 7) / 8 * 8;
-  if (!dense) {
-    // group kernel: per-unit counters
-    w.gx_stride = GROUP_GX_WORDS;
-    w.gx = reinterpret_cast<unsigned*>(take(sizeof(unsigned) * BH * w.gx_stride));
-    w.U = reinterpret_cast<float*>(take(sizeof(float) * BH * Ustride));
-    w.sel_pages = reinterpret_cast<int*>(take(sizeof(int) * BH * Nmax));
-    w.sel_keys = reinterpret_cast<int*>(take(sizeof(int) * BH * Kmax));
-    w.kscore = reinterpret_cast<uint16_t*>(take(sizeof(uint16_t) * BH * Cmax));
-    w.khist = reinterpret_cast<int*>(take(sizeof(int) * std::max<size_t>(BH, MAX_GRID) * HB));
-  }
-  w.Nmax = Nmax;
-  w.Kmax = Kmax;
-  w.Cmax = Cmax;
-  w.HB = HB;
-  w.Ustride = Ustride;
-  w.C1 = C1;
-  w.C2 = C2;
-  w.C3 = C3;
-  w.max_groups = max_groups;
-  if (wk) *wk = w;
-  return off;
-}
 
 // SMs of the current device (cached per device), at most MAX_GRID.
 int device_sms() {
@@ -170,9 +71,174 @@ int device_sms() {
 }  // namespace
 
 namespace hhr {
+
 // Records a host-side error message for hhr_last_error() (used by entry
 // points defined in other translation units).
 hhr_status record_error(hhr_status s, const char* msg) { return fail(s, "%s", msg); }
+
+long long wait_limit_cycles() { return g_wait_cycles.load(std::memory_order_relaxed); }
+
+void dense_split(const Dims& dm, int sms, int* nsplit, int* rows) {
+  const int U = dm.B * dm.Hkv;
+  int ns = std::max(1, std::min(MAX_GRID, sms / U));
+  ns = std::min(ns, ceil_div(dm.T, GATHER_ROWS));
+  const int r = ceil_div(ceil_div(dm.T, ns), GATHER_ROWS) * GATHER_ROWS;
+  *rows = r;
+  *nsplit = ceil_div(dm.T, r);
+}
+
+// Validates the configuration and fills the kernel-side dimensions.
+hhr_status make_dims(const hhr_config* cfg, Dims* dm) {
+  if (!cfg) return fail(HHR_ERR_INVALID_ARG, "cfg is NULL");
+  if (cfg->head_dim != D) return fail(HHR_ERR_UNSUPPORTED, "head_dim %d (only 128)", cfg->head_dim);
+  if (cfg->batch < 1 || cfg->num_kv_heads < 1 || cfg->num_q_heads < 1 || cfg->max_seq_len < 1)
+    return fail(HHR_ERR_INVALID_ARG, "batch, heads and max_seq_len must be >= 1");
+  if (cfg->num_q_heads % cfg->num_kv_heads != 0)
+    return fail(HHR_ERR_INVALID_ARG, "num_q_heads %d not a multiple of num_kv_heads %d", cfg->num_q_heads,
+                cfg->num_kv_heads);
+  const int G = cfg->num_q_heads / cfg->num_kv_heads;
+  if (G > 8) return fail(HHR_ERR_UNSUPPORTED, "group size %d (1..8)", G);
+  if (cfg->page_size != 16 && cfg->page_size != 32)
+    return fail(HHR_ERR_UNSUPPORTED, "page_size %d (16 or 32)", cfg->page_size);
+  if (cfg->hash_bits != 64 && cfg->hash_bits != 128 && cfg->hash_bits != 256)
+    return fail(HHR_ERR_UNSUPPORTED, "hash_bits %d (64, 128 or 256)", cfg->hash_bits);
+  const long long np_max = ((long long)cfg->max_seq_len + cfg->page_size - 1) / cfg->page_size;
+  if (np_max > MAX_DENSE_PAGES)
+    return fail(HHR_ERR_UNSUPPORTED, "%lld pages per sequence (at most %d)", np_max, MAX_DENSE_PAGES);
+  if ((long long)cfg->batch * cfg->num_kv_heads * cfg->max_seq_len * D >= (1ll << 31) * D)
+    return fail(HHR_ERR_UNSUPPORTED, "cache of %lld rows (at most 2^31)",
+                (long long)cfg->batch * cfg->num_kv_heads * cfg->max_seq_len);
+  if (cfg->paged) {
+    if (cfg->num_blocks < 1) return fail(HHR_ERR_INVALID_ARG, "paged: num_blocks must be >= 1");
+    if (cfg->max_blocks_per_seq < np_max)
+      return fail(HHR_ERR_INVALID_ARG, "paged: max_blocks_per_seq %d < ceil(max_seq_len / page_size) %lld",
+                  cfg->max_blocks_per_seq, np_max);
+    if ((long long)cfg->num_blocks * cfg->num_kv_heads * cfg->page_size >= (1ll << 31))
+      return fail(HHR_ERR_UNSUPPORTED, "block pool of %lld rows (at most 2^31)",
+                  (long long)cfg->num_blocks * cfg->num_kv_heads * cfg->page_size);
+  }
+  dm->B = cfg->batch;
+  dm->Hq = cfg->num_q_heads;
+  dm->Hkv = cfg->num_kv_heads;
+  dm->G = G;
+  dm->P = cfg->page_size;
+  dm->lgP = cfg->page_size == 16 ? 4 : 5;
+  dm->nb = cfg->hash_bits;
+  dm->words = cfg->hash_bits / 64;
+  dm->T = cfg->max_seq_len;
+  dm->np_max = (int)np_max;
+  dm->paged = cfg->paged ? 1 : 0;
+  dm->num_blocks = cfg->paged ? cfg->num_blocks : 0;
+  dm->max_blocks = cfg->paged ? cfg->max_blocks_per_seq : 0;
+  return HHR_OK;
+}
+
+// Carves the workspace; with base == nullptr only the size is computed.
+// Sparse: per-unit counters, page bounds, the kept-row list, one partial per
+// gather chunk, one score histogram per CTA.  Dense: counters and one
+// partial per split.
+size_t carve(const Dims& dm, int Nmax, int Kmax, bool dense, char* base, Work* wk) {
+  const size_t BH = (size_t)dm.B * dm.Hkv;
+  size_t off = 0;
+  auto take = [&](size_t bytes) {
+    char* p = base ? base + off : nullptr;
+    off += align256(bytes);
+    return p;
+  };
+  Work w{};
+  w.gx_stride = GX_STRIDE;
+  w.gx = reinterpret_cast<unsigned*>(take(sizeof(unsigned) * BH * GX_STRIDE));
+  const size_t PS = (size_t)dm.G * D + 16;
+  if (dense) {
+    w.C3 = std::min(MAX_GRID, ceil_div(dm.T, GATHER_ROWS));
+    w.part = reinterpret_cast<float*>(take(sizeof(float) * BH * w.C3 * PS));
+  } else {
+    const long long kcap = std::min<long long>(Kmax, (long long)Nmax * dm.P);
+    w.C3 = std::max(1, ceil_div(kcap, GATHER_ROWS));
+    w.Ustride = (dm.np_max + 31) / 32 * 32;
+    w.HB = (dm.G * dm.nb + 1 + 7) / 8 * 8;
+    w.U = reinterpret_cast<float*>(take(sizeof(float) * BH * w.Ustride));
+    w.sel_keys = reinterpret_cast<int*>(take(sizeof(int) * BH * Kmax));
+    w.part = reinterpret_cast<float*>(take(sizeof(float) * BH * w.C3 * PS));
+    w.khist = reinterpret_cast<int*>(take(sizeof(int) * (size_t)MAX_GRID * w.HB));
+  }
+  w.Nmax = Nmax;
+  w.Kmax = Kmax;
+  if (wk) *wk = w;
+  return off;
+}
+
+hhr_status decode_check(const hhr_config* cfg, const void* q, const float* R, const void* W, const void* Krot,
+                        const void* Vcache, const void* page_min, const void* page_max, const uint64_t* codes,
+                        const int32_t* seq_lens, const int32_t* block_table, const int32_t* n_keep_pages,
+                        const int32_t* top_k, int32_t max_keep_pages, int32_t max_top_k, float sm_scale,
+                        const float* out, const char* who, Dims* dm, int* Nmax, size_t* need) {
+  hhr_status s = make_dims(cfg, dm);
+  if (s != HHR_OK) return s;
+  if (dm->np_max > MAX_SELECT_PAGES)
+    return fail(HHR_ERR_UNSUPPORTED, "%s: %d pages per sequence (at most %d)", who, dm->np_max, MAX_SELECT_PAGES);
+  if (!q || !R || !W || !Krot || !Vcache || !page_min || !page_max || !codes || !seq_lens || !n_keep_pages ||
+      !top_k || !out)
+    return fail(HHR_ERR_INVALID_ARG, "%s: NULL pointer", who);
+  if (dm->paged && !block_table) return fail(HHR_ERR_INVALID_ARG, "%s: paged needs block_table", who);
+  const void* al[] = {q, R, W, Krot, Vcache, page_min, page_max, codes};
+  for (const void* p : al)
+    if (!aligned16(p)) return fail(HHR_ERR_INVALID_ARG, "%s: tensor not 16-byte aligned", who);
+  if (max_keep_pages < 1 || max_top_k < 1)
+    return fail(HHR_ERR_INVALID_ARG, "%s: max_keep_pages and max_top_k must be >= 1", who);
+  if (!(sm_scale > 0.f)) return fail(HHR_ERR_INVALID_ARG, "%s: sm_scale must be > 0", who);
+  const int nm = std::min(max_keep_pages, dm->np_max);
+  if (nm > MAX_KEEP_PAGES)
+    return fail(HHR_ERR_UNSUPPORTED, "%s: max_keep_pages %d (at most %d)", who, nm, MAX_KEEP_PAGES);
+  if ((long long)nm * dm->P > MAX_CANDIDATES)
+    return fail(HHR_ERR_UNSUPPORTED, "%s: max_keep_pages x page_size = %lld candidates (at most %d)", who,
+                (long long)nm * dm->P, MAX_CANDIDATES);
+  *Nmax = nm;
+  *need = carve(*dm, nm, max_top_k, false, nullptr, nullptr);
+  return HHR_OK;
+}
+
+hhr_status decode_launch(const Dims& dm, int Nmax, int32_t max_top_k, const void* q, const float* R, const void* W,
+                         const void* Krot, const void* Vcache, const void* page_min, const void* page_max,
+                         const uint64_t* codes, const int32_t* seq_lens, const int32_t* block_table,
+                         const int32_t* n_keep_pages, const int32_t* top_k, float sm_scale, float* out,
+                         const hhr_debug* dbg, void* workspace, int32_t* device_status, hhr_stream_t stream,
+                         const char* who) {
+  Work wk;
+  carve(dm, Nmax, max_top_k, false, static_cast<char*>(workspace), &wk);
+  const int sms = device_sms();
+  if (sms <= 0) return fail(HHR_ERR_CUDA, "%s: cannot query the device", who);
+  DecodeArgs a = {};
+  a.dm = dm;
+  a.wk = wk;
+  a.q = static_cast<const __nv_bfloat16*>(q);
+  a.R = R;
+  a.W = static_cast<const __nv_bfloat16*>(W);
+  a.Kr = static_cast<const __nv_bfloat16*>(Krot);
+  a.Vc = static_cast<const __nv_bfloat16*>(Vcache);
+  a.pmin = static_cast<const __nv_bfloat16*>(page_min);
+  a.pmax = static_cast<const __nv_bfloat16*>(page_max);
+  a.codes = codes;
+  a.seq_lens = seq_lens;
+  a.table = block_table;
+  a.n_keep = n_keep_pages;
+  a.top_k = top_k;
+  a.sm_scale = sm_scale;
+  a.out = out;
+  if (dbg) a.dbg = *dbg;
+  a.status = device_status;
+  a.stream = reinterpret_cast<cudaStream_t>(stream);
+  a.num_sms = sms;
+  a.wait_limit = wait_limit_cycles();
+  cudaError_t e = cudaErrorInvalidValue;
+  HHR_DISPATCH_G(dm.G, e = launch_decode<GG>(a));
+  if (e != cudaSuccess) {
+    cudaGetLastError();
+    return fail(HHR_ERR_CUDA, "%s: launch failed: %s", who, cudaGetErrorString(e));
+  }
+  return ok();
+}
+
 }  // namespace hhr
 
 extern "C" {
@@ -191,6 +257,10 @@ const char* hhr_status_string(hhr_status s) {
 }
 
 const char* hhr_last_error(void) { return g_err; }
+
+void hhr_set_wait_limit(int64_t cycles) {
+  g_wait_cycles.store(cycles > 0 ? (long long)cycles : DEFAULT_WAIT_CYCLES, std::memory_order_relaxed);
+}
 
 hhr_status hhr_build_cache(const hhr_config* cfg, const void* K, const void* V, const float* R, const void* W,
                            const int32_t* seq_lens, const int32_t* block_table, void* Krot, void* Vcache,
@@ -215,7 +285,10 @@ hhr_status hhr_build_cache(const hhr_config* cfg, const void* K, const void* V, 
                                      seq_lens, block_table, static_cast<__nv_bfloat16*>(Krot),
                                      static_cast<__nv_bfloat16*>(page_min), static_cast<__nv_bfloat16*>(page_max), codes,
                                      nullptr, st);
-  if (e != cudaSuccess) return fail(HHR_ERR_CUDA, "hhr_build_cache: %s", cudaGetErrorString(e));
+  if (e != cudaSuccess) {
+    cudaGetLastError();
+    return fail(HHR_ERR_CUDA, "hhr_build_cache: %s", cudaGetErrorString(e));
+  }
   return ok();
 }
 
@@ -240,63 +313,19 @@ hhr_status hhr_decode_step(const hhr_config* cfg, const void* q, const float* R,
                            const int32_t* top_k, int32_t max_keep_pages, int32_t max_top_k, float sm_scale,
                            float* out, const hhr_debug* dbg, void* workspace, size_t workspace_bytes,
                            int32_t* device_status, hhr_stream_t stream) {
+  static const char* who = "hhr_decode_step";
   Dims dm;
-  hhr_status s = make_dims(cfg, &dm);
+  int Nmax = 0;
+  size_t need = 0;
+  hhr_status s = decode_check(cfg, q, R, W, Krot, Vcache, page_min, page_max, codes, seq_lens, block_table,
+                              n_keep_pages, top_k, max_keep_pages, max_top_k, sm_scale, out, who, &dm, &Nmax, &need);
   if (s != HHR_OK) return s;
-  if (dm.np_max > MAX_SELECT_PAGES)
-    return fail(HHR_ERR_UNSUPPORTED, "hhr_decode_step: %d pages per sequence (at most %d)", dm.np_max,
-                MAX_SELECT_PAGES);
-  if (!q || !R || !W || !Krot || !Vcache || !page_min || !page_max || !codes || !seq_lens || !n_keep_pages ||
-      !top_k || !out || !workspace)
-    return fail(HHR_ERR_INVALID_ARG, "hhr_decode_step: NULL pointer");
-  if (dm.paged && !block_table) return fail(HHR_ERR_INVALID_ARG, "hhr_decode_step: paged needs block_table");
-  const void* al[] = {q, R, W, Krot, Vcache, page_min, page_max, codes};
-  for (const void* p : al)
-    if (!aligned16(p)) return fail(HHR_ERR_INVALID_ARG, "hhr_decode_step: tensor not 16-byte aligned");
+  if (!workspace) return fail(HHR_ERR_INVALID_ARG, "%s: NULL workspace", who);
   if ((reinterpret_cast<uintptr_t>(workspace) & 255u) != 0)
-    return fail(HHR_ERR_INVALID_ARG, "hhr_decode_step: workspace not 256-byte aligned");
-  if (max_keep_pages < 1 || max_top_k < 1)
-    return fail(HHR_ERR_INVALID_ARG, "hhr_decode_step: max_keep_pages and max_top_k must be >= 1");
-  if (!(sm_scale > 0.f)) return fail(HHR_ERR_INVALID_ARG, "hhr_decode_step: sm_scale must be > 0");
-  const int Nmax = std::min(max_keep_pages, dm.np_max);
-  if (Nmax > MAX_KEEP_PAGES)
-    return fail(HHR_ERR_UNSUPPORTED, "hhr_decode_step: max_keep_pages %d (at most %d)", Nmax, MAX_KEEP_PAGES);
-  if ((long long)Nmax * dm.P > MAX_CANDIDATES)
-    return fail(HHR_ERR_UNSUPPORTED, "hhr_decode_step: max_keep_pages x page_size = %lld candidates (at most %d)",
-                (long long)Nmax * dm.P, MAX_CANDIDATES);
-  const size_t need = carve(dm, Nmax, max_top_k, false, nullptr, nullptr);
-  if (workspace_bytes < need)
-    return fail(HHR_ERR_WORKSPACE, "hhr_decode_step: workspace %zu bytes < %zu", workspace_bytes, need);
-  Work wk;
-  carve(dm, Nmax, max_top_k, false, static_cast<char*>(workspace), &wk);
-  const int sms = device_sms();
-  if (sms <= 0) return fail(HHR_ERR_CUDA, "hhr_decode_step: cannot query the device");
-
-  DecodeArgs a = {};
-  a.dm = dm;
-  a.wk = wk;
-  a.q = static_cast<const __nv_bfloat16*>(q);
-  a.R = R;
-  a.W = static_cast<const __nv_bfloat16*>(W);
-  a.Kr = static_cast<const __nv_bfloat16*>(Krot);
-  a.Vc = static_cast<const __nv_bfloat16*>(Vcache);
-  a.pmin = static_cast<const __nv_bfloat16*>(page_min);
-  a.pmax = static_cast<const __nv_bfloat16*>(page_max);
-  a.codes = codes;
-  a.seq_lens = seq_lens;
-  a.table = block_table;
-  a.n_keep = n_keep_pages;
-  a.top_k = top_k;
-  a.sm_scale = sm_scale;
-  a.out = out;
-  if (dbg) a.dbg = *dbg;
-  a.status = device_status;
-  a.stream = reinterpret_cast<cudaStream_t>(stream);
-  a.num_sms = sms;
-  cudaError_t e = cudaErrorInvalidValue;
-  HHR_DISPATCH_G(dm.G, e = launch_decode<GG>(a));
-  if (e != cudaSuccess) return fail(HHR_ERR_CUDA, "hhr_decode_step: launch failed: %s", cudaGetErrorString(e));
-  return ok();
+    return fail(HHR_ERR_INVALID_ARG, "%s: workspace not 256-byte aligned", who);
+  if (workspace_bytes < need) return fail(HHR_ERR_WORKSPACE, "%s: workspace %zu bytes < %zu", who, workspace_bytes, need);
+  return decode_launch(dm, Nmax, max_top_k, q, R, W, Krot, Vcache, page_min, page_max, codes, seq_lens, block_table,
+                       n_keep_pages, top_k, sm_scale, out, dbg, workspace, device_status, stream, who);
 }
 
 size_t hhr_dense_workspace_size(const hhr_config* cfg) {
@@ -321,8 +350,6 @@ hhr_status hhr_dense_decode(const hhr_config* cfg, const void* q, const float* R
   if ((reinterpret_cast<uintptr_t>(workspace) & 255u) != 0)
     return fail(HHR_ERR_INVALID_ARG, "hhr_dense_decode: workspace not 256-byte aligned");
   if (!(sm_scale > 0.f)) return fail(HHR_ERR_INVALID_ARG, "hhr_dense_decode: sm_scale must be > 0");
-  if (ceil_div(ceil_div(dm.T, FUSED_ROWS), FUSED_GROUP) > MAX_GATHER_GROUPS)
-    return fail(HHR_ERR_UNSUPPORTED, "hhr_dense_decode: max_seq_len %d too long", dm.T);
   const size_t need = carve(dm, 1, 1, true, nullptr, nullptr);
   if (workspace_bytes < need)
     return fail(HHR_ERR_WORKSPACE, "hhr_dense_decode: workspace %zu bytes < %zu", workspace_bytes, need);
@@ -344,9 +371,15 @@ hhr_status hhr_dense_decode(const hhr_config* cfg, const void* q, const float* R
   a.status = device_status;
   a.stream = reinterpret_cast<cudaStream_t>(stream);
   a.num_sms = sms;
+  a.wait_limit = wait_limit_cycles();
+  dense_split(dm, sms, &a.dense_nsplit, &a.dense_rows);
+  if (a.dense_nsplit > wk.C3) return fail(HHR_ERR_UNSUPPORTED, "hhr_dense_decode: %d splits", a.dense_nsplit);
   cudaError_t e = cudaErrorInvalidValue;
   HHR_DISPATCH_G(dm.G, e = launch_dense<GG>(a));
-  if (e != cudaSuccess) return fail(HHR_ERR_CUDA, "hhr_dense_decode: launch failed: %s", cudaGetErrorString(e));
+  if (e != cudaSuccess) {
+    cudaGetLastError();
+    return fail(HHR_ERR_CUDA, "hhr_dense_decode: launch failed: %s", cudaGetErrorString(e));
+  }
   return ok();
 }
 

@@ -17,31 +17,19 @@ struct Dims {
   int lgP;  // log2 of the page size (a power of two)
 };
 
-// Workspace carve-out of one decode step (device pointers).
-// `ctrl` holds the work-queue counter, the exit counter and per-unit flags and
-// counters; the kernel keeps it at zero between calls (the last CTA to leave
-// resets it).  Everything else is overwritten by every call.
+// Workspace carve-out of one decode step (device pointers).  The per-unit
+// counters `gx` and the kept-row list `sel_keys` are zero between calls (the
+// kernels reset what they use); everything else is overwritten by every call.
 struct Work {
-  float* qrot;         // [B, Hq, D]        q' = R_h q
-  uint64_t* qcodes;    // [B, Hq, w]        query sign codes
-  float* U;            // [B, Hkv, Ustride] page bounds (group max)
-  int* sel_pages;      // [B, Hkv, Nmax]    kept pages, ascending
-  int* sel_keys;       // [B, Hkv, Kmax]    kept rows, ascending (group kernel: row + 1, cleared after reading)
-  float* part;         // [B, Hkv, C3, G * D + 16] attention partial of every gather chunk
-  float* gpart;        // [B, Hkv, max_groups, G * D + 16] merged groups of chunks
-  uint16_t* kscore;    // [B, Hkv, Cmax]    Hamming score of every candidate row
-  int* khist;          // [max(B Hkv, grid), HB] score histograms: per unit (fused kernel, zero between
-                       // calls) or per CTA (group kernel, rewritten every unit)
-  int4* tq;            // [tq_cap]          task queue: (kind, unit, arg, sequence + 1), zero between calls
-  unsigned* gx;        // [B * Hkv, gx_stride] per-unit exchange areas of the CTA groups
-  unsigned* ctrl;      // [4 + B * Hkv * (8 + max_groups)] item queue, exit count, task queue head / tail, flags, counters
+  float* U;            // [B Hkv, Ustride] page bounds (max over the group's query heads)
+  int* sel_keys;       // [B Hkv, Kmax] kept-row list: row + 1 while published, read and cleared
+  float* part;         // [B Hkv, C3, G D + 16] softmax partials (gather chunks, or dense splits)
+  int* khist;          // [grid, HB] score histogram of every CTA
+  unsigned* gx;        // [B Hkv, gx_stride] per-unit barrier and arrival counters
   int Nmax, Kmax;      // budgets the workspace was sized for
-  int Cmax;            // Nmax * page size: candidate rows per unit
-  int HB;              // histogram stride (>= G * hash bits + 1)
+  int HB;              // histogram stride (>= G nb + 1, a multiple of 8)
   int Ustride;         // row stride of U (np_max rounded up to 32)
-  int C1, C2, C3;      // scan, score and gather chunks per unit
-  int max_groups;      // groups of 16 gather chunks per unit
-  int tq_cap;          // task queue entries (every task of one call fits)
+  int C3;              // partials per unit
   int gx_stride;       // 32-bit words per unit exchange area
 };
 
@@ -77,10 +65,6 @@ __device__ __forceinline__ uint32_t order_key(float f) {
   if ((u << 1) == 0u) u = 0u;
   return (u & 0x80000000u) ? ~u : (u | 0x80000000u);
 }
-
-// --- programmatic dependent launch ---------------------------------------
-__device__ __forceinline__ void pdl_wait() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
-__device__ __forceinline__ void pdl_trigger() { asm volatile("griddepcontrol.launch_dependents;" ::: "memory"); }
 
 // --- status ------------------------------------------------------------------
 __device__ __forceinline__ void set_status(int* st, int code) {
@@ -119,35 +103,6 @@ __device__ __forceinline__ long long code_row(const Dims& dm, const int* __restr
   const int blk = __ldg(table + (long long)b * dm.max_blocks + (t >> dm.lgP));
   if ((unsigned)blk >= (unsigned)dm.num_blocks) { set_status(status, HHR_ERR_BAD_BLOCK); return -1; }
   return (((long long)blk * dm.Hkv + h) * dm.P + (t & (dm.P - 1))) * dm.words;
-}
-
-// --- block-wide exclusive scan of one int (blockDim multiple of 32, <= 1024) --
-// `red` needs 33 ints of shared memory.  Returns the exclusive prefix; the
-// block total is written to *total.
-__device__ __forceinline__ int block_excl_scan(int v, int* red, int* total) {
-  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5, nw = blockDim.x >> 5;
-  int x = v;
-#pragma unroll
-  for (int o = 1; o < 32; o <<= 1) {
-    int y = __shfl_up_sync(0xffffffffu, x, o);
-    if (lane >= o) x += y;
-  }
-  if (lane == 31) red[warp] = x;
-  __syncthreads();
-  if (warp == 0) {
-    int s = lane < nw ? red[lane] : 0;
-#pragma unroll
-    for (int o = 1; o < 32; o <<= 1) {
-      int y = __shfl_up_sync(0xffffffffu, s, o);
-      if (lane >= o) s += y;
-    }
-    red[lane] = s;  // inclusive over warps
-  }
-  __syncthreads();
-  const int before = (warp > 0 ? red[warp - 1] : 0) + x - v;
-  *total = red[nw - 1];
-  __syncthreads();
-  return before;
 }
 
 }  // namespace hhr

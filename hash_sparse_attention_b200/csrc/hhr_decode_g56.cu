@@ -1,5 +1,5 @@
-// Decode kernels instantiated for group sizes 5 and 6.
-#include "hhr_group.cuh"
+// Decode-step and dense kernels instantiated for group sizes 5 and 6.
+#include "hhr_dense.cuh"
 
 namespace hhr {
 HHR_INSTANTIATE_DECODE(5)

@@ -1,0 +1,165 @@
+// Device primitives shared by the HHR kernels (sm_100a): asynchronous copies,
+// acquire/release words, tensor-core fragments, block scans and the bounded
+// wait used by every spin in the library.
+#pragma once
+
+#include <climits>
+
+#include "hhr_common.cuh"
+
+namespace hhr {
+
+__device__ __forceinline__ uint32_t smem_u32(const void* p) {
+  return static_cast<uint32_t>(__cvta_generic_to_shared(p));
+}
+
+// --- cp.async (16 bytes, through L2 only) --------------------------------------
+__device__ __forceinline__ void cp_async16(void* dst, const void* src) {
+  asm volatile("cp.async.cg.shared.global [%0], [%1], 16;" ::"r"(smem_u32(dst)), "l"(src) : "memory");
+}
+__device__ __forceinline__ void cp_async_commit() { asm volatile("cp.async.commit_group;" ::: "memory"); }
+template <int N>
+__device__ __forceinline__ void cp_async_wait() { asm volatile("cp.async.wait_group %0;" ::"n"(N) : "memory"); }
+__device__ __forceinline__ void cp_async_wait_all() { asm volatile("cp.async.wait_all;" ::: "memory"); }
+
+// --- global words with gpu-scope ordering --------------------------------------
+__device__ __forceinline__ unsigned ld_acquire(const unsigned* p) {
+  unsigned v;
+  asm volatile("ld.acquire.gpu.global.u32 %0, [%1];" : "=r"(v) : "l"(p) : "memory");
+  return v;
+}
+__device__ __forceinline__ int ld_relaxed_s32(const int* p) {
+  int v;
+  asm volatile("ld.relaxed.gpu.global.s32 %0, [%1];" : "=r"(v) : "l"(p) : "memory");
+  return v;
+}
+__device__ __forceinline__ void red_release_add(unsigned* p, unsigned v) {
+  asm volatile("red.release.gpu.global.add.u32 [%0], %1;" ::"l"(p), "r"(v) : "memory");
+}
+__device__ __forceinline__ unsigned atom_add_acq_rel(unsigned* p, unsigned v) {
+  unsigned old;
+  asm volatile("atom.acq_rel.gpu.global.add.u32 %0, [%1], %2;" : "=r"(old) : "l"(p), "r"(v) : "memory");
+  return old;
+}
+
+// --- programmatic dependent launch ------------------------------------------
+// wait: every prior grid of the stream has completed and its writes are
+// visible; launch_dependents: the next grid of the stream may be scheduled.
+// Both are no-ops for a launch without the programmatic attribute.
+__device__ __forceinline__ void pdl_wait() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
+__device__ __forceinline__ void pdl_launch_dependents() { asm volatile("griddepcontrol.launch_dependents;" ::: "memory"); }
+
+// --- bounded waits -------------------------------------------------------------
+// Every spin in the library gives up after `limit` SM clock cycles (a kernel
+// parameter; about two seconds by default).  On expiry the caller records
+// HHR_ERR_TIMEOUT and raises the CTA's abort flag.
+struct Spin {
+  long long t0, limit;
+  __device__ __forceinline__ explicit Spin(long long lim) {
+    t0 = clock64();
+    limit = lim;
+  }
+  __device__ __forceinline__ bool expired() const { return clock64() - t0 > limit; }
+};
+
+// --- tensor-core fragments (mma.sync m16n8k16, bf16 in, fp32 accumulate) -------
+__device__ __forceinline__ void ldsm_x4(uint32_t (&r)[4], const void* p) {
+  asm volatile("ldmatrix.sync.aligned.m8n8.x4.shared.b16 {%0,%1,%2,%3}, [%4];"
+               : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3])
+               : "r"(smem_u32(p)));
+}
+__device__ __forceinline__ void ldsm_x4_t(uint32_t (&r)[4], const void* p) {
+  asm volatile("ldmatrix.sync.aligned.m8n8.x4.trans.shared.b16 {%0,%1,%2,%3}, [%4];"
+               : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3])
+               : "r"(smem_u32(p)));
+}
+__device__ __forceinline__ void ldsm_x2(uint32_t (&r)[2], const void* p) {
+  asm volatile("ldmatrix.sync.aligned.m8n8.x2.shared.b16 {%0,%1}, [%2];" : "=r"(r[0]), "=r"(r[1]) : "r"(smem_u32(p)));
+}
+__device__ __forceinline__ void mma_bf16(float (&d)[4], const uint32_t (&a)[4], const uint32_t (&b)[2]) {
+  asm volatile(
+      "mma.sync.aligned.m16n8k16.row.col.f32.bf16.bf16.f32 {%0,%1,%2,%3}, {%4,%5,%6,%7}, {%8,%9}, "
+      "{%0,%1,%2,%3};"
+      : "+f"(d[0]), "+f"(d[1]), "+f"(d[2]), "+f"(d[3])
+      : "r"(a[0]), "r"(a[1]), "r"(a[2]), "r"(a[3]), "r"(b[0]), "r"(b[1]));
+}
+// x as bf16 hi + lo (hi = RNE(x), lo = RNE(x - hi)): |x - hi - lo| <= 2^-17 |x|
+__device__ __forceinline__ void split_bf16(float x, __nv_bfloat16& hi, __nv_bfloat16& lo) {
+  hi = __float2bfloat16_rn(x);
+  lo = __float2bfloat16_rn(x - __bfloat162float(hi));
+}
+
+// --- block scan ----------------------------------------------------------------
+// Exclusive prefix of v over the threads of the block in thread order, and the
+// block total.  `red` holds 2 x 32 ints; `parity` alternates between calls so
+// that one barrier per call suffices.  Every thread must call it.
+__device__ __forceinline__ int block_scan_excl(int v, int* red, int parity, int* total) {
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5, nw = blockDim.x >> 5;
+  int x = v;
+#pragma unroll
+  for (int o = 1; o < 32; o <<= 1) {
+    const int y = __shfl_up_sync(0xffffffffu, x, o);
+    if (lane >= o) x += y;
+  }
+  int* r = red + 32 * (parity & 1);
+  if (lane == 31) r[warp] = x;
+  __syncthreads();
+  int before = 0, tot = 0;
+  for (int w = 0; w < nw; ++w) {
+    const int t = r[w];
+    before += w < warp ? t : 0;
+    tot += t;
+  }
+  *total = tot;
+  return before + x - v;
+}
+
+// Block-wide minimum and maximum of unsigned values (one barrier; `red` 2 x 32).
+__device__ __forceinline__ void block_minmax_u32(unsigned& lo, unsigned& hi, unsigned* red) {
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5, nw = blockDim.x >> 5;
+#pragma unroll
+  for (int o = 16; o >= 1; o >>= 1) {
+    lo = min(lo, __shfl_xor_sync(0xffffffffu, lo, o));
+    hi = max(hi, __shfl_xor_sync(0xffffffffu, hi, o));
+  }
+  if (lane == 0) {
+    red[warp] = lo;
+    red[32 + warp] = hi;
+  }
+  __syncthreads();
+  lo = 0xffffffffu;
+  hi = 0u;
+  for (int w = 0; w < nw; ++w) {
+    lo = min(lo, red[w]);
+    hi = max(hi, red[32 + w]);
+  }
+}
+
+__host__ __device__ constexpr int ilog2(int x) { return x <= 1 ? 0 : 1 + ilog2(x >> 1); }
+
+// Transposed butterfly over the NL lanes of an aligned lane group (NV, NL
+// powers of two): v[0..NV) are per-lane partial sums of NV quantities.
+// Afterwards, with NV >= NL, lane l of the group holds the group totals of
+// quantities l*(NV/NL) + e in v[e], e < NV/NL; with NV < NL it holds the total
+// of quantity l*NV/NL in v[0].  Each round halves the values a lane keeps.
+template <int NV, int NL>
+__device__ __forceinline__ void group_reduce_scatter(float (&v)[NV], int lane) {
+  static_assert((NV & (NV - 1)) == 0 && (NL & (NL - 1)) == 0 && NL <= 32, "powers of two");
+  constexpr int ROUNDS = ilog2(NV < NL ? NV : NL);
+#pragma unroll
+  for (int k = 0; k < ROUNDS; ++k) {
+    const int half = NV >> (k + 1), o = NL >> (k + 1);
+    const bool upper = (lane & o) != 0;
+#pragma unroll
+    for (int i = 0; i < half; ++i) {
+      const float send = upper ? v[i] : v[i + half];
+      const float keep = upper ? v[i + half] : v[i];
+      v[i] = keep + __shfl_xor_sync(0xffffffffu, send, o);
+    }
+  }
+  // NV < NL: the remaining lane levels add up copies of the same quantity
+#pragma unroll
+  for (int o = (NV < NL ? NL / (2 * NV) : 0); o >= 1; o >>= 1) v[0] += __shfl_xor_sync(0xffffffffu, v[0], o);
+}
+
+}  // namespace hhr

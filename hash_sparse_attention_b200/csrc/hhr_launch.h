@@ -11,16 +11,14 @@
 
 namespace hhr {
 
-constexpr int MAX_SELECT_PAGES = 8192;   // pages of one sequence in the page select (shared memory)
+constexpr int MAX_SELECT_PAGES = 8192;   // pages of one sequence in the page select (16 per thread)
 constexpr int MAX_DENSE_PAGES = 16384;   // pages of one sequence elsewhere
-constexpr int MAX_KEEP_PAGES = 2048;     // kept pages per sequence
-constexpr int MAX_CANDIDATES = 16384;    // kept pages x page size (scores in shared memory)
-constexpr int FUSED_ROWS = 128;          // pages per scan item, rows per gather item
-constexpr int MAX_GRID = 160;            // CTAs of the fused kernel (one per SM)
-constexpr int FUSED_GROUP = 16;          // gather chunks merged together first
-constexpr int FUSED_SCORE = 1024;        // candidate rows per score item
-constexpr int MAX_GATHER_GROUPS = 256;   // groups per unit (final merge width)
-constexpr int GROUP_GX_WORDS = 4;       // per-unit counters of the group kernel
+constexpr int MAX_KEEP_PAGES = 2048;     // kept pages per sequence (shared memory list)
+constexpr int MAX_CANDIDATES = 16384;    // kept pages x page size
+constexpr int MAX_GRID = 160;            // CTAs of a launch (one per SM)
+constexpr int GATHER_ROWS = 128;         // rows per gather chunk
+constexpr int GX_STRIDE = 4;             // per-unit counter words
+constexpr long long DEFAULT_WAIT_CYCLES = 4000000000ll;  // ~2 s at 1.9 GHz
 
 struct DecodeArgs {
   Dims dm;
@@ -43,9 +41,15 @@ struct DecodeArgs {
   int* status;
   cudaStream_t stream;
   int num_sms;
+  long long wait_limit;
+  int dense_nsplit, dense_rows;
 };
 
 hhr_status record_error(hhr_status s, const char* msg);
+long long wait_limit_cycles();
+
+// splits per unit and rows per split of the dense kernel
+void dense_split(const Dims& dm, int sms, int* nsplit, int* rows);
 
 template <int G> cudaError_t launch_decode(const DecodeArgs& a);
 template <int G> cudaError_t launch_dense(const DecodeArgs& a);

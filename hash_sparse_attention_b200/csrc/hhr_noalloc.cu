@@ -4,7 +4,7 @@
 #include <cstdio>
 #include <mutex>
 
-#include "hhr_launch.h"
+#include "hhr_api_internal.h"
 
 namespace {
 
@@ -47,25 +47,30 @@ extern "C" hhr_status hhr_decode_step_noalloc(
     const int32_t* block_table, const int32_t* n_keep_pages, const int32_t* top_k, int32_t max_keep_pages,
     int32_t max_top_k, float sm_scale, float* out, const hhr_debug* dbg, int32_t* device_status,
     hhr_stream_t stream) {
-  const size_t need = hhr_decode_workspace_size(cfg, max_keep_pages, max_top_k);
-  if (need == 0)
-    return hhr::record_error(HHR_ERR_INVALID_ARG,
-                             "hhr_decode_step_noalloc: invalid configuration or budgets (see hhr_decode_step)");
+  static const char* who = "hhr_decode_step_noalloc";
+  // the same checks, status codes and messages as hhr_decode_step, before any stream work
+  hhr::Dims dm;
+  int Nmax = 0;
+  size_t need = 0;
+  hhr_status s = hhr::decode_check(cfg, q, R, W, Krot, Vcache, page_min, page_max, codes, seq_lens, block_table,
+                                   n_keep_pages, top_k, max_keep_pages, max_top_k, sm_scale, out, who, &dm, &Nmax,
+                                   &need);
+  if (s != HHR_OK) return s;
   if (need > (size_t)HHR_NOALLOC_SCRATCH_BYTES) {
     char msg[256];
     snprintf(msg, sizeof(msg),
-             "hhr_decode_step_noalloc: these sizes need %zu bytes of scratch; the built-in scratch holds %zu "
+             "%s: these sizes need %zu bytes of scratch; the built-in scratch holds %zu "
              "(use hhr_decode_step with a caller-provided workspace)",
-             need, (size_t)HHR_NOALLOC_SCRATCH_BYTES);
+             who, need, (size_t)HHR_NOALLOC_SCRATCH_BYTES);
     return hhr::record_error(HHR_ERR_WORKSPACE, msg);
   }
   void* scratch = nullptr;
-  hhr_status s = scratch_address(&scratch);
+  s = scratch_address(&scratch);
   if (s != HHR_OK) return s;
   // the scratch keeps the previous call's contents: clear the part this call uses
   s = hhr_workspace_init(scratch, need, stream);
   if (s != HHR_OK) return s;
-  return hhr_decode_step(cfg, q, R, W, Krot, Vcache, page_min, page_max, codes, seq_lens, block_table,
-                         n_keep_pages, top_k, max_keep_pages, max_top_k, sm_scale, out, dbg, scratch, need,
-                         device_status, stream);
+  return hhr::decode_launch(dm, Nmax, max_top_k, q, R, W, Krot, Vcache, page_min, page_max, codes, seq_lens,
+                            block_table, n_keep_pages, top_k, sm_scale, out, dbg, scratch, device_status, stream,
+                            who);
 }

@@ -107,6 +107,14 @@ HHR_API const char* hhr_status_string(hhr_status s);
  * (static thread-local storage; empty when the last call succeeded). */
 HHR_API const char* hhr_last_error(void);
 
+/* Bound of every device-side wait of the launches that follow (a CTA waiting
+ * for the other CTAs of its group, a reader polling the kept-row list), in SM
+ * clock cycles; cycles <= 0 restores the default of 4e9 (about 2 s).  On
+ * expiry a launch records HHR_ERR_TIMEOUT in its device_status and returns
+ * (see hhr_decode_step).  The paper has no counterpart: this is a testing and
+ * watchdog aid.  Process-wide; takes effect at the next launch. */
+HHR_API void hhr_set_wait_limit(int64_t cycles);
+
 /*
  * hhr_build_cache -- cache build for one layer (prefill side of HHR).
  *
@@ -164,15 +172,23 @@ HHR_API hhr_status hhr_workspace_init(void* workspace, size_t workspace_bytes, h
  * 256-byte aligned, zeroed once with hhr_workspace_init(), and not shared by
  * calls that may run concurrently.  `device_status` may be NULL.
  *
- * One kernel launch, at most one CTA per SM; the CTAs of a group that shares
- * a (sequence, KV head) wait for one another, so the launch expects the SMs
- * it was sized for (a kernel occupying SMs on another stream only delays
- * it).  Every device-side wait is bounded: on expiry the launch records
- * HHR_ERR_TIMEOUT in `device_status` and returns.  After any call whose
- * status is not HHR_OK, zero the workspace again (hhr_workspace_init) before
- * the next call: its counters and row list may be left mid-use.  Results are
- * deterministic and do not depend on the batch composition or on the layout
- * (contiguous or paged).
+ * One kernel launch of at most one CTA per SM (the library checks on the host
+ * that a CTA fits on an SM); the CTAs of a group that shares a (sequence, KV
+ * head) wait for one another, so the launch expects the SMs it was sized for
+ * (a kernel occupying SMs on another stream only delays it).  Every
+ * device-side wait is bounded (hhr_set_wait_limit): on expiry the launch
+ * records HHR_ERR_TIMEOUT in `device_status` and returns.  After any call
+ * whose device status is not HHR_OK, zero the workspace again
+ * (hhr_workspace_init) before the next call: its counters and row list may
+ * be left mid-use.  Results are deterministic and do not depend on the batch
+ * composition or on the layout (contiguous or paged).
+ *
+ * The launch is a programmatic dependent launch: it may start while the
+ * previous kernel on `stream` is still running and then reads R and W (the
+ * learned per-head transforms) before that kernel has finished; everything
+ * else (q, the cache, lengths, budgets, the workspace, out) is read or written
+ * only after it has finished.  Do not write R or W in the kernel launched just
+ * before.
  */
 HHR_API hhr_status hhr_decode_step(const hhr_config* cfg, const void* q, const float* R, const void* W,
                            const void* Krot, const void* Vcache, const void* page_min,
@@ -191,18 +207,19 @@ HHR_API hhr_status hhr_decode_step(const hhr_config* cfg, const void* q, const f
  * hhr_decode_step_noalloc -- hhr_decode_step without a caller workspace.
  *
  * (The paper has no counterpart; this is a library convenience.)  Some
- * callers cannot call cudaMalloc at all: code that runs while another
- * framework is capturing a CUDA graph (allocation is not a capturable
- * operation and may break the capture), plugins of inference runtimes that
- * must draw every byte from the host runtime's own memory pool, and
- * latency-critical serving loops where an allocation (and the implicit
- * synchronisation it can bring) is not allowed.  Such callers still pass
- * every input and output, but the scratch comes from a fixed
- * HHR_NOALLOC_SCRATCH_BYTES array in the library's device memory, which
- * every GPU that loads the library holds until the process exits.
- *   - Same arguments and results as hhr_decode_step, minus the workspace.
+ * callers cannot call cudaMalloc at all: plugins of inference runtimes that
+ * must draw every byte of device memory from the host runtime's own pool
+ * (and may not allocate behind its back), and latency-critical serving loops
+ * in which an allocation, with the device synchronisation it can bring, is
+ * not allowed.  Such callers still pass every input and output, but the
+ * scratch comes from a fixed HHR_NOALLOC_SCRATCH_BYTES array in the
+ * library's device memory, which every GPU that loads the library holds
+ * until the process exits.
+ *   - Same arguments, checks, status codes and results as hhr_decode_step,
+ *     minus the workspace.  Every host-side check runs before anything is
+ *     enqueued on `stream`.
  *   - Sizes whose workspace (hhr_decode_workspace_size) exceeds the array are
- *     rejected with HHR_ERR_WORKSPACE and a message; nothing is launched.
+ *     rejected with HHR_ERR_WORKSPACE and a message; nothing is enqueued.
  *   - Allocates nothing: no cudaMalloc, cudaFree or allocating library call.
  *   - The first call on a device looks up the array's device address with
  *     that device current (cudaGetSymbolAddress) and caches it; make that

@@ -7,7 +7,7 @@ fp64 oracle within the tolerances below.  End-to-end: the oracle runs its own
 pipeline from the raw inputs; index differences are counted, outputs compared
 within tolerance where the selections agree.
 
-Tolerances and exemptions (readings of the pages):
+Tolerances and exemptions:
   * attention output: per query head max|o - o^| / max|o^| <= 2e-3
   * page bounds: |ub - ub^| <= 2e-3 * sum_i |q'_i| max(|mn_i|, |mx_i|)
   * K': within one bf16 ulp of the fp64-rounded value plus the fp32

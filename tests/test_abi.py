@@ -31,7 +31,8 @@ def L():
 
 def test_header_declares_the_boundary():
     fns = declared_functions()
-    assert fns == sorted(["hhr_status_string", "hhr_last_error", "hhr_build_cache", "hhr_decode_workspace_size",
+    assert fns == sorted(["hhr_status_string", "hhr_last_error", "hhr_set_wait_limit", "hhr_build_cache",
+                          "hhr_decode_workspace_size",
                           "hhr_workspace_init", "hhr_decode_step", "hhr_decode_step_noalloc",
                           "hhr_dense_workspace_size", "hhr_dense_decode"])
     # the binding declares exactly the same functions

@@ -216,3 +216,39 @@ def test_more_units_than_sms():
         assert int(status.item()) == 0
         assert torch.equal(out, r.out)
     assert np.array_equal(g.out, r.out.cpu().numpy().astype(np.float64))
+
+
+def test_bounded_wait_runs_out_and_reports_timeout():
+    """A device-side wait that runs out ends the launch with HHR_ERR_TIMEOUT in
+    the status word (no trap, no hang); after the workspace is zeroed again the
+    next call is bit-identical to a clean run.  The wait limit is cut to a few
+    hundred SM cycles, far below the skew between the CTAs of a group, so the
+    group barriers of this 8-unit layer (18 CTAs per KV head) run out."""
+    _cuda()
+    from hash_sparse_attention_b200 import _lib
+    w = scaled(WORKLOADS["llama_layer_32k"], context=8192, batch=1, seed=33)
+    li = make_layer(w)
+    clean = parity.run_gpu(w, li, to_host=False)
+    assert clean.status == 0
+    cache, ws = clean.extra["cache"], clean.extra["ws"]
+    dev = torch.device("cuda")
+    q, R, W = li.q.to(dev), li.R.to(dev), li.W.to(dev)
+    seq, nk, tk = li.seq_lens.to(dev), li.n_keep.to(dev), li.top_k.to(dev)
+    status = torch.zeros(1, dtype=torch.int32, device=dev)
+    out = torch.zeros_like(clean.out)
+    L = _lib.lib()
+    try:
+        L.hhr_set_wait_limit(300)
+        hhr.decode_step(clean.cfg, q, R, W, cache, seq, None, nk, tk, clean.Nmax, clean.Kmax, out, ws, status=status)
+        torch.cuda.synchronize()
+    finally:
+        L.hhr_set_wait_limit(0)
+    assert int(status.item()) == _lib.HHR_ERR_TIMEOUT
+    # the context is usable; zero the workspace again, then a clean call
+    ws.zero_()
+    status.zero_()
+    out2 = torch.full_like(clean.out, float("nan"))
+    hhr.decode_step(clean.cfg, q, R, W, cache, seq, None, nk, tk, clean.Nmax, clean.Kmax, out2, ws, status=status)
+    torch.cuda.synchronize()
+    assert int(status.item()) == 0
+    assert torch.equal(out2, clean.out)
