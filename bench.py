@@ -2,13 +2,16 @@
 """Benchmark of the HHR decode step on B200.
 
     python bench.py [--gpus N] [--steps K] [--warmup W] [--impl hhr|reference]
-                    [--workload NAME]
+                    [--workload NAME] [--no-extra] [--no-dense] [--no-cpu-baseline]
 
 One step = one decode token of the workload: hhr_decode_step on every layer
 in order (32 layers of Llama-3.1-8B shape at 128K context by default),
 captured in one CUDA graph.  Inputs are resident in HBM before timing; the
-KV cache (17.5 GB) is far larger than L2, so every layer's bytes are evicted
-by the other 31 layers before they are read again (no L2 flush needed).
+headline KV cache (17.5 GB) is far larger than L2, so every layer's bytes are
+evicted by the other 31 layers before they are read again (no L2 flush).
+The other workloads (`per_config`) are timed step by step with CUDA events,
+L2 flushed (a 2 x L2 write) between steps outside the timed events; their
+figure is the median over the steps.
 
 Rank 0 prints one JSON line.  Under torchrun every rank runs its own replica
 of the workload (independent sequences, no collective on the data path);
@@ -43,8 +46,11 @@ def parse_args(argv=None):
     p.add_argument("--workload", default="llama_32l_128k")
     p.add_argument("--layers", type=int, default=None, help="fewer layers (profiling runs only)")
     p.add_argument("--no-dense", action="store_true")
+    p.add_argument("--no-extra", action="store_true", help="only the headline workload")
+    p.add_argument("--extra-steps", type=int, default=60)
     p.add_argument("--no-cpu-baseline", action="store_true")
-    p.add_argument("--cpu-seconds", type=float, default=12.0)
+    p.add_argument("--cpu-seconds", type=float, default=10.0)
+    p.add_argument("--cpu-workers", type=int, default=0, help="all-cores oracle workers (0: every core, at most 64)")
     p.add_argument("--soak-seconds", type=float, default=1.0)
     return p.parse_args(argv)
 
@@ -179,9 +185,9 @@ def kernel_source_hash() -> str:
 
 
 def profiled_traffic(workload: str):
-    """DRAM bytes per hhr_group_kernel launch from the committed ncu summary,
+    """DRAM bytes per hhr_sparse_kernel launch from the committed ncu summary,
     when that summary was taken on the current sources (else None)."""
-    path = os.path.join(ROOT, "profiles", "hhr_group_kernel_llama_32l_128k.md")
+    path = os.path.join(ROOT, "profiles", f"hhr_sparse_kernel_{workload}.md")
     if not os.path.exists(path):
         return None
     fields = {}
@@ -212,21 +218,20 @@ def peaks() -> dict:
 # ---------------------------------------------------------------------------
 
 def oracle_units(w, n_heads: int, layer: int = 0):
-    """Oracle-built caches of the first n_heads KV heads of one layer (sequence 0)."""
-    import numpy as np
-    import torch
+    """Oracle-built caches of the first n_heads KV heads of one layer (sequence
+    0), generated on the CPU (the oracle's timing never touches the GPU)."""
     from hash_sparse_attention_b200.synth import make_layer
     from oracle import hhr_oracle as O
-    li = make_layer(w, layer=layer, device="cuda" if torch.cuda.is_available() else "cpu")
+    li = make_layer(w, layer=layer, device="cpu")
     L = int(li.seq_lens[0])
     G, P = w.group, w.page_size
-    R32 = li.R.double().cpu().numpy()
-    Wn = li.W.double().cpu().numpy()
+    R32 = li.R.double().numpy()
+    Wn = li.W.double().numpy()
     units = []
     for h in range(n_heads):
-        K = (li.K_logical if w.paged else li.K)[0, h, :L].double().cpu().numpy()
-        V = (li.V_logical if w.paged else li.V)[0, h, :L].double().cpu().numpy()
-        Q = li.q[0, h * G:(h + 1) * G].double().cpu().numpy()
+        K = (li.K_logical if w.paged else li.K)[0, h, :L].double().numpy()
+        V = (li.V_logical if w.paged else li.V)[0, h, :L].double().numpy()
+        Q = li.q[0, h * G:(h + 1) * G].double().numpy()
         Kp, mn, mx, codes = O.build_head(K, R32[h], Wn[h], L, P)
         units.append(dict(Q=Q, R=R32[h], W=Wn[h], Kp=Kp, V=V, mn=mn, mx=mx, codes=codes, L=L, P=P,
                           N=int(li.n_keep[0]), k=int(li.top_k[0])))
@@ -240,9 +245,63 @@ def oracle_decode_unit(u):
                          u["N"], u["k"])
 
 
-def cpu_baseline(w, seconds: float) -> dict:
-    """Times the fp64 oracle's decode on whole (layer, KV head) units, one thread."""
+def cpu_model() -> str:
+    try:
+        with open("/proc/cpuinfo") as f:
+            for line in f:
+                if line.startswith("model name"):
+                    return line.split(":", 1)[1].strip()
+    except OSError:
+        pass
+    return "unknown"
+
+
+def host_cores() -> int:
+    try:
+        return len(os.sched_getaffinity(0))
+    except AttributeError:
+        return os.cpu_count() or 1
+
+
+_ARRAYS = ("Q", "R", "W", "Kp", "V", "mn", "mx", "codes")
+
+
+def _cpu_worker(path, n_units, seconds, go, q):
+    """All-cores oracle leg: one process, one thread, decodes the shared units
+    (memory-mapped .npy files) until `seconds` have passed."""
+    import json as _json
+    import numpy as _np
     from threadpoolctl import threadpool_limits
+    with open(os.path.join(path, "meta.json")) as f:
+        meta = _json.load(f)
+    units = []
+    for i in range(n_units):
+        u = {k: _np.load(os.path.join(path, f"u{i}_{k}.npy"), mmap_mode="r") for k in _ARRAYS}
+        u.update(meta[i])
+        units.append(u)
+    with threadpool_limits(1):
+        go.wait()
+        t0 = time.perf_counter()
+        done = 0
+        while True:
+            oracle_decode_unit(units[done % n_units])
+            done += 1
+            el = time.perf_counter() - t0
+            if el >= seconds:
+                break
+    q.put((done, el))
+
+
+def cpu_baseline(w, seconds: float, workers: int = 0) -> dict:
+    """The fp64 oracle's decode step on whole (layer, KV head) units of the
+    workload, on the host cores: one thread, then one process per core (each
+    single-threaded), every unit's cache built beforehand (untimed).  Runs
+    before the GPU is touched."""
+    import multiprocessing as mp
+    import shutil
+    import tempfile
+    from threadpoolctl import threadpool_limits
+    import numpy as np
     units = oracle_units(w, min(2, w.num_kv_heads))
     heads_per_token = w.layers * w.num_kv_heads * w.batch
     done = 0
@@ -254,20 +313,207 @@ def cpu_baseline(w, seconds: float) -> dict:
             el = time.perf_counter() - t0
             if el >= seconds:
                 break
-    tok_s = (done / heads_per_token) / el
-    return {"value": tok_s, "unit": "tokens/s", "cores": 1, "kind": "oracle",
-            "sample": f"{done} (layer 0, KV head) decode units of {heads_per_token} per token, "
-                      f"{el:.1f} s of fp64 CPU work, one thread; cache build untimed"}
+    single = (done / heads_per_token) / el
+    out = {"value": single, "unit": "tokens/s", "cores": 1, "kind": "oracle",
+           "cpu_model": cpu_model(), "host_cores": host_cores(),
+           "sample": f"{done} (layer 0, KV head) decode units of {heads_per_token} per token, "
+                     f"{el:.1f} s of fp64 CPU work on one thread; cache build untimed"}
+    n = workers if workers > 0 else min(64, host_cores())
+    if n > 1:
+        base = "/dev/shm" if os.path.isdir("/dev/shm") else None
+        tmp = tempfile.mkdtemp(prefix="hhr_oracle_", dir=base)
+        try:
+            meta = []
+            for i, u in enumerate(units):
+                for k in _ARRAYS:
+                    np.save(os.path.join(tmp, f"u{i}_{k}.npy"), np.ascontiguousarray(u[k]))
+                meta.append({k: u[k] for k in ("L", "P", "N", "k")})
+            with open(os.path.join(tmp, "meta.json"), "w") as f:
+                json.dump(meta, f)
+            ctx = mp.get_context("spawn")
+            go, q = ctx.Event(), ctx.Queue()
+            procs = [ctx.Process(target=_cpu_worker, args=(tmp, len(units), seconds, go, q)) for _ in range(n)]
+            for p_ in procs:
+                p_.start()
+            time.sleep(min(20.0, 2.0 + 0.05 * n))  # workers map the units
+            go.set()
+            res = [q.get(timeout=seconds + 600) for _ in procs]
+            for p_ in procs:
+                p_.join(timeout=60)
+            total = sum(d / e for d, e in res) / heads_per_token
+            out["all_cores"] = {"value": total, "unit": "tokens/s", "cores": n, "kind": "oracle",
+                                "sample": f"{sum(d for d, _ in res)} units in {n} single-threaded processes, "
+                                          f"{seconds:.0f} s each"}
+        finally:
+            shutil.rmtree(tmp, ignore_errors=True)
+    return out
 
 
 # ---------------------------------------------------------------------------
 # the HHR arm
 # ---------------------------------------------------------------------------
 
+def _config_of(hhr, w, li):
+    if w.paged:
+        return hhr.make_config(w.batch, w.num_q_heads, w.num_kv_heads, w.page_size, w.hash_bits, w.context,
+                               paged=True, num_blocks=li.K.shape[0], max_blocks_per_seq=li.block_table.shape[1])
+    return hhr.make_config(w.batch, w.num_q_heads, w.num_kv_heads, w.page_size, w.hash_bits, w.context)
+
+
+def build_layers(w, dev):
+    """Every layer's inputs, drawn on the device, and its cache built in place
+    by the library (each build timed with CUDA events)."""
+    import torch
+    from hash_sparse_attention_b200 import hhr
+    from hash_sparse_attention_b200.synth import make_layer
+    layers, events = [], []
+    for l in range(w.layers):
+        li = make_layer(w, layer=l, device=dev)
+        cfg = _config_of(hhr, w, li)
+        cache = hhr.alloc_cache(cfg, dev, Krot=li.K, V=li.V)
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record()
+        hhr.build_cache(cfg, li.K, li.V, li.R, li.W, li.seq_lens, li.block_table, cache)
+        e1.record()
+        events.append((e0, e1))
+        lens = [int(x) for x in li.seq_lens.cpu()]
+        layers.append(dict(cfg=cfg, cache=cache, R=li.R, W=li.W, q=li.q, seq=li.seq_lens, table=li.block_table,
+                           lens=lens, n_keep=li.n_keep, top_k=li.top_k,
+                           nk=[int(x) for x in li.n_keep.cpu()], tk=[int(x) for x in li.top_k.cpu()]))
+        li.K_logical = li.V_logical = None
+        del li
+    return layers, events
+
+
+def with_budgets(w, layers, dev):
+    """The same caches with another workload's page and key budgets."""
+    import torch
+    out = []
+    for L in layers:
+        nk = [w.keep_for(x) for x in L["lens"]]
+        tk = [w.topk_for(x) for x in L["lens"]]
+        out.append(dict(L, nk=nk, tk=tk, n_keep=torch.tensor(nk, dtype=torch.int32, device=dev),
+                        top_k=torch.tensor(tk, dtype=torch.int32, device=dev)))
+    return out
+
+
+def step_bytes(w, layers, Nmax, Kmax):
+    """Algorithmic bytes of one decode step per layer (see hhr_bytes_per_head)."""
+    d, Hkv = w.head_dim, w.num_kv_heads
+    per_layer = []
+    for L in layers:
+        tot = 0
+        for b, Lb in enumerate(L["lens"]):
+            hb = hhr_bytes_per_head(Lb, w.page_size, min(L["nk"][b], Nmax), min(L["tk"][b], Kmax), w.group,
+                                    w.hash_bits)
+            tot += Hkv * (hb["meta"] + hb["codes"] + hb["gather"] + hb["qo"])
+        tot += Hkv * (d * d * 4 + w.hash_bits * d * 2)
+        per_layer.append(tot)
+    return per_layer
+
+
+def capture(fn, dev):
+    """fn warmed up on a side stream, then captured in a CUDA graph."""
+    import torch
+    fn()
+    s = torch.cuda.Stream(device=dev)
+    s.wait_stream(torch.cuda.current_stream())
+    with torch.cuda.stream(s):
+        for _ in range(2):
+            fn()
+    torch.cuda.current_stream().wait_stream(s)
+    g = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(g):
+        fn()
+    torch.cuda.synchronize()
+    return g
+
+
+def timed_steps(graph, steps, world, dev, flush=None):
+    """Replays `graph` `steps` times with an event pair around each replay on
+    the launching stream.  Without `flush` the replays run back to back and
+    the total is the span from the first start to the last end; with it, L2
+    is flushed between steps outside the events and the total is the sum.
+    Returns (total seconds, per-step milliseconds)."""
+    import torch
+    st = torch.cuda.current_stream()
+    ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(steps)]
+    barrier(world, dev)
+    torch.cuda.synchronize()
+    for e0, e1 in ev:
+        if flush is not None:
+            flush.add_(1)
+        e0.record(st)
+        graph.replay()
+        e1.record(st)
+    torch.cuda.synchronize()
+    barrier(world, dev)
+    per = [e0.elapsed_time(e1) for e0, e1 in ev]
+    total = sum(per) / 1e3 if flush is not None else ev[0][0].elapsed_time(ev[-1][1]) / 1e3
+    return total, per
+
+
+def measure_workload(w, layers, dev, args, world, flush, with_dense):
+    """Decode-step (and dense) throughput of one workload on prepared caches."""
+    import torch
+    from hash_sparse_attention_b200 import hhr
+    B, Hq, d = w.batch, w.num_q_heads, w.head_dim
+    Nmax = max(max(L["nk"]) for L in layers)
+    Kmax = max(max(L["tk"]) for L in layers)
+    cfg0 = layers[0]["cfg"]
+    ws = hhr.decode_workspace(cfg0, Nmax, Kmax, dev)
+    status = torch.zeros(1, dtype=torch.int32, device=dev)
+    out = torch.empty(len(layers), B, Hq, d, dtype=torch.float32, device=dev)
+
+    def step():
+        for l, L in enumerate(layers):
+            hhr.decode_step(L["cfg"], L["q"], L["R"], L["W"], L["cache"], L["seq"], L["table"], L["n_keep"],
+                            L["top_k"], Nmax, Kmax, out[l], ws, status=status)
+    step()
+    torch.cuda.synchronize()
+    assert int(status.item()) == 0, f"{w.name}: device status {int(status.item())}"
+    g = capture(step, dev)
+    for _ in range(max(3, args.warmup)):
+        g.replay()
+    steps = max(50, args.extra_steps)
+    total, per = timed_steps(g, steps, world, dev, flush)
+    med = statistics.median(per) / 1e3
+    per_layer = step_bytes(w, layers, Nmax, Kmax)
+    pk = peaks()
+    res = {"tokens_per_s": whole_job_throughput(B, world, max_over_ranks(med, world, dev)),
+           "ms_per_step_median": med * 1e3, "steps": steps, "layers": len(layers),
+           "bytes_per_step": sum(per_layer), "achieved_gbs": sum(per_layer) / med / 1e9,
+           "frac": sum(per_layer) / med / 1e9 / pk["hbm_gbs"],
+           "keep_pages": Nmax, "top_k": Kmax,
+           "l2": "flushed between steps" if flush is not None else "not flushed (the cache is far larger than L2)"}
+    if with_dense:
+        dws = hhr.dense_workspace(cfg0, dev)
+        dout = torch.empty_like(out)
+
+        def dstep():
+            for l, L in enumerate(layers):
+                hhr.dense_decode(L["cfg"], L["q"], L["R"], L["cache"], L["seq"], L["table"], dout[l], dws,
+                                 status=status)
+        dg = capture(dstep, dev)
+        for _ in range(3):
+            dg.replay()
+        _, dper = timed_steps(dg, max(10, steps // 4), world, dev, flush)
+        dmed = statistics.median(dper) / 1e3
+        dbytes = sum(dense_bytes_per_head(Lb, w.group) for L in layers for Lb in L["lens"] for _ in range(w.num_kv_heads))
+        res["dense"] = {"tokens_per_s": whole_job_throughput(B, world, max_over_ranks(dmed, world, dev)),
+                        "ms_per_step_median": dmed * 1e3, "achieved_gbs": dbytes / dmed / 1e9,
+                        "frac": dbytes / dmed / 1e9 / pk["hbm_gbs"]}
+        res["sparse_over_dense"] = dmed / med
+        del dg, dws
+    del g, ws
+    assert int(status.item()) == 0, f"{w.name}: device status {int(status.item())}"
+    return res
+
+
 def run_hhr(args, rank, world):
     import torch
     from hash_sparse_attention_b200 import hhr
-    from hash_sparse_attention_b200.synth import WORKLOADS, make_layer, scaled
+    from hash_sparse_attention_b200.synth import WORKLOADS, scaled
 
     _, local_rank, _ = dist_env()
     dev = torch.device("cuda", local_rank)
@@ -278,38 +524,14 @@ def run_hhr(args, rank, world):
     B, Hq, Hkv, d, P = w.batch, w.num_q_heads, w.num_kv_heads, w.head_dim, w.page_size
 
     # ---- setup: every layer's cache built in place by the library (each build timed) ----
-    layers = []
-    q_all = None
-    build_events = []
-    for l in range(w.layers):
-        li = make_layer(w, layer=l, device=dev)
-        if w.paged:
-            cfg = hhr.make_config(B, Hq, Hkv, P, w.hash_bits, w.context, paged=True, num_blocks=li.K.shape[0],
-                                  max_blocks_per_seq=li.block_table.shape[1])
-        else:
-            cfg = hhr.make_config(B, Hq, Hkv, P, w.hash_bits, w.context)
-        cache = hhr.alloc_cache(cfg, dev, Krot=li.K, V=li.V)
-        be0, be1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-        be0.record()
-        hhr.build_cache(cfg, li.K, li.V, li.R, li.W, li.seq_lens, li.block_table, cache)
-        be1.record()
-        build_events.append((be0, be1))
-        if q_all is None:
-            q_all = torch.empty(w.layers, B, Hq, d, dtype=torch.bfloat16, device=dev)
-            out_all = torch.empty(w.layers, B, Hq, d, dtype=torch.float32, device=dev)
-            dense_all = torch.empty(w.layers, B, Hq, d, dtype=torch.float32, device=dev)
-        q_all[l].copy_(li.q)
-        layers.append(dict(cfg=cfg, cache=cache, R=li.R, W=li.W, seq=li.seq_lens, table=li.block_table,
-                           n_keep=li.n_keep, top_k=li.top_k, lens=[int(x) for x in li.seq_lens.cpu()],
-                           nk=[int(x) for x in li.n_keep.cpu()], tk=[int(x) for x in li.top_k.cpu()]))
-        li.K_logical = li.V_logical = None
-        del li
+    layers, build_events = build_layers(w, dev)
     torch.cuda.synchronize()
+    q_all = torch.stack([L["q"] for L in layers])
+    out_all = torch.empty(w.layers, B, Hq, d, dtype=torch.float32, device=dev)
     cfg0 = layers[0]["cfg"]
     Nmax = max(max(L["nk"]) for L in layers)
     Kmax = max(max(L["tk"]) for L in layers)
     ws = hhr.decode_workspace(cfg0, Nmax, Kmax, dev)
-    dws = hhr.dense_workspace(cfg0, dev)
     status = torch.zeros(1, dtype=torch.int32, device=dev)
 
     def step():
@@ -317,53 +539,18 @@ def run_hhr(args, rank, world):
             hhr.decode_step(L["cfg"], q_all[l], L["R"], L["W"], L["cache"], L["seq"], L["table"], L["n_keep"],
                             L["top_k"], Nmax, Kmax, out_all[l], ws, status=status)
 
-    def dense_step():
-        for l, L in enumerate(layers):
-            hhr.dense_decode(L["cfg"], q_all[l], L["R"], L["cache"], L["seq"], L["table"], dense_all[l], dws,
-                             status=status)
-
-    # eager once (and check status), then capture
     step()
     torch.cuda.synchronize()
     assert int(status.item()) == 0, f"device status {int(status.item())}"
-    s = torch.cuda.Stream(device=dev)
-    s.wait_stream(torch.cuda.current_stream())
-    with torch.cuda.stream(s):
-        for _ in range(2):
-            step()
-    torch.cuda.current_stream().wait_stream(s)
-    graph = torch.cuda.CUDAGraph()
-    with torch.cuda.graph(graph):
-        step()
-    dgraph = None
-    if not args.no_dense:
-        dense_step()
-        dgraph = torch.cuda.CUDAGraph()
-        with torch.cuda.graph(dgraph):
-            dense_step()
-    torch.cuda.synchronize()
+    graph = capture(step, dev)
 
     props = torch.cuda.get_device_properties(dev)
-    sampler = ClockSampler(str(getattr(props, "uuid", local_rank)) if getattr(props, "uuid", None) else str(local_rank))
+    sampler = ClockSampler(str(local_rank))
     if getattr(props, "uuid", None) is not None:
         u = str(props.uuid)
         sampler.gpu_id = u if u.startswith("GPU-") else f"GPU-{u}"
     sampler.start()
     st = torch.cuda.current_stream()
-
-    def timed(g, steps):
-        barrier(world, dev)
-        torch.cuda.synchronize()
-        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-        e0.record(st)
-        for _ in range(steps):
-            g.replay()
-        e1.record(st)
-        e1.synchronize()
-        torch.cuda.synchronize()
-        barrier(world, dev)
-        return e0.elapsed_time(e1) / 1e3
-
     # warm-up, plus a short soak so that clocks settle under load
     for _ in range(max(3, args.warmup)):
         graph.replay()
@@ -371,21 +558,9 @@ def run_hhr(args, rank, world):
     while time.time() < t_end:
         graph.replay()
         torch.cuda.synchronize()
-    secs = timed(graph, args.steps)
+    secs, per_step = timed_steps(graph, args.steps, world, dev)
     clocks = sampler.stop()
     secs_max = max_over_ranks(secs, world, dev)
-
-    # dense comparison (same context, same library)
-    dense = None
-    if dgraph is not None:
-        for _ in range(3):
-            dgraph.replay()
-        dsecs = max_over_ranks(timed(dgraph, max(3, args.steps // 8)), world, dev)
-        dsteps = max(3, args.steps // 8)
-        dbytes = sum(dense_bytes_per_head(Lb, w.group) for L in layers for Lb in L["lens"] for _ in range(Hkv))
-        dense = {"value": whole_job_throughput(B * dsteps, world, dsecs), "unit": "tokens/s",
-                 "ms_per_step": dsecs / dsteps * 1e3,
-                 "achieved_gbs": dbytes / (dsecs / dsteps) / 1e9}
 
     # e2e: q from pinned host memory, out back to pinned host memory, every step
     q_host = q_all.cpu().pin_memory()
@@ -406,17 +581,11 @@ def run_hhr(args, rank, world):
     e1.synchronize()
     e2e_secs = max_over_ranks(e0.elapsed_time(e1) / 1e3, world, dev)
     assert int(status.item()) == 0, f"device status {int(status.item())}"
+    del graph
 
-    # ---- algorithmic bytes ----
-    per_layer_bytes = []
-    for L in layers:
-        tot = 0
-        for b, Lb in enumerate(L["lens"]):
-            hb = hhr_bytes_per_head(Lb, P, min(L["nk"][b], Nmax), min(L["tk"][b], Kmax), w.group, w.hash_bits)
-            tot += Hkv * (hb["meta"] + hb["codes"] + hb["gather"] + hb["qo"])
-        tot += Hkv * (d * d * 4 + w.hash_bits * d * 2)
-        per_layer_bytes.append(tot)
-    step_bytes = sum(per_layer_bytes)
+    # ---- algorithmic bytes and the roofline of the decode kernel ----
+    per_layer_bytes = step_bytes(w, layers, Nmax, Kmax)
+    step_total = sum(per_layer_bytes)
     t_step = secs_max / args.steps
     pk = peaks()
     # the timed graph holds only the per-layer decode launches, back to back:
@@ -426,14 +595,12 @@ def run_hhr(args, rank, world):
     roofline = {"bound": "hbm", "achieved": achieved, "peak": pk["hbm_gbs"], "unit": "GB/s",
                 "frac": achieved / pk["hbm_gbs"], "traffic": profiled_traffic(w.name),
                 "algorithmic_bytes_per_launch": statistics.mean(per_layer_bytes),
-                "kernel": "hhr_group_kernel (one launch per layer; one group of CTAs per KV head: query prep, "
-                          "page scan, page select, distributed key select, tensor-core sparse attention, "
-                          "chunk-partial merge)",
-                "peak_source": pk["source"],
-                "step_gbs": step_bytes / t_step / 1e9, "step_frac": step_bytes / t_step / 1e9 / pk["hbm_gbs"]}
-    launches_per_step = len(layers)  # one hhr_group_kernel launch per layer
-    build = build_report(w, layers, build_events, clocks, torch.cuda.get_device_properties(dev).multi_processor_count,
-                         pk)
+                "kernel": "hhr_sparse_kernel (one launch per layer; one group of CTAs per KV head: query prep, "
+                          "page scan, radix page select, Hamming scores and key select, tensor-core sparse "
+                          "attention, chunk-partial merge)",
+                "peak_source": pk["source"], "peak_note": "of measured" if pk["source"] == "measured" else "of fallback",
+                "step_gbs": step_total / t_step / 1e9, "step_frac": step_total / t_step / 1e9 / pk["hbm_gbs"]}
+    build = build_report(w, layers, build_events, clocks, props.multi_processor_count, pk)
     result = {
         "metric": METRIC,
         "value": whole_job_throughput(B * args.steps, world, secs_max),
@@ -442,6 +609,7 @@ def run_hhr(args, rank, world):
         "steps": args.steps,
         "warmup": args.warmup,
         "ms_per_step": t_step * 1e3,
+        "ms_per_step_median": statistics.median(per_step),
         "higher_is_better": True,
         "scaling": "weak",
         "vs_baseline": None,
@@ -453,18 +621,48 @@ def run_hhr(args, rank, world):
                    "parallelism": f"replicas x{world}" if world > 1 else "single",
                    "l2": "not flushed: the KV cache (all layers) is far larger than L2 and each layer's bytes "
                          "are evicted by the other layers before reuse",
-                   "bytes_per_step": step_bytes},
+                   "bytes_per_step": step_total},
         "e2e": {"value": whole_job_throughput(B * args.steps, world, e2e_secs), "unit": "tokens/s",
                 "h2d_bytes_per_step": q_host.numel() * q_host.element_size(),
                 "d2h_bytes_per_step": out_host.numel() * out_host.element_size()},
-        "gpu_launches": launches_per_step * args.steps,
+        "gpu_launches": len(layers) * args.steps,
         "roofline": roofline,
         "clocks": clocks,
-        "dense": dense,
         "build": build,
-        "achieved_gbs": step_bytes / t_step / 1e9,
+        "achieved_gbs": step_total / t_step / 1e9,
     }
+    del ws
+    # ---- the dense kernel at the same context, and the other workloads ----
+    flush = torch.zeros(l2_flush_elems(dev), dtype=torch.float32, device=dev)
+    if not args.no_dense:
+        m = measure_workload(w, layers, dev, args, world, None, True)
+        result["dense"] = dict(m["dense"], sparse_over_dense=m["sparse_over_dense"])
+    per_config = {}
+    if not args.no_extra and w.name == "llama_32l_128k" and args.layers is None:
+        w3b = WORKLOADS["llama_32l_128k_keep8"]
+        per_config[w3b.name] = measure_workload(w3b, with_budgets(w3b, layers, dev), dev, args, world, None,
+                                                not args.no_dense)
+    del layers, q_all, out_all
+    torch.cuda.empty_cache()
+    if not args.no_extra and args.layers is None:
+        for name in ("tiny_4k", "llama_layer_32k", "paged_b16_ragged", "qwen_gqa7_128k"):
+            if name == w.name:
+                continue
+            wx = WORKLOADS[name]
+            lx, _ = build_layers(wx, dev)
+            torch.cuda.synchronize()
+            per_config[name] = measure_workload(wx, lx, dev, args, world, flush, not args.no_dense)
+            del lx
+            torch.cuda.empty_cache()
+    if per_config:
+        result["per_config"] = per_config
     return result, w
+
+
+def l2_flush_elems(dev) -> int:
+    import torch
+    props = torch.cuda.get_device_properties(dev)
+    return 2 * int(getattr(props, "L2_cache_size", 128 << 20)) // 4
 
 
 def build_report(w, layers, build_events, clocks, sms, pk):
@@ -530,11 +728,16 @@ def main(argv=None):
             return 0
         print(json.dumps(run_reference(args, rank, 1)))
         return 0
+    from hash_sparse_attention_b200.synth import WORKLOADS, scaled
+    cpu = None
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        # the host leg first, before the GPU is touched (its processes are spawned)
+        cpu = cpu_baseline(WORKLOADS[args.workload], args.cpu_seconds, args.cpu_workers)
     import torch
     rank, world = dist_init("nccl" if torch.cuda.is_available() else "gloo")
     result, w = run_hhr(args, rank, world)
-    if rank == 0 and world == 1 and not args.no_cpu_baseline:
-        result["cpu_baseline"] = cpu_baseline(w, args.cpu_seconds)
+    if cpu is not None:
+        result["cpu_baseline"] = cpu
     if rank == 0:
         print(json.dumps(result))
     if world > 1:

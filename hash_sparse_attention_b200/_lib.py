@@ -25,7 +25,7 @@ NOALLOC_SCRATCH_BYTES = 16 << 20  # HHR_NOALLOC_SCRATCH_BYTES in include/hhr.h
 class HHRConfig(ctypes.Structure):
     _fields_ = [(n, ctypes.c_int32) for n in (
         "batch", "num_q_heads", "num_kv_heads", "head_dim", "page_size", "hash_bits",
-        "max_seq_len", "paged", "num_blocks", "max_blocks_per_seq")]
+        "max_seq_len", "paged", "num_blocks", "max_blocks_per_seq", "page_group_agg", "key_group_agg")]
 
     def as_dict(self) -> dict:
         return {n: getattr(self, n) for n, _ in self._fields_}
@@ -48,6 +48,7 @@ SIGNATURES = {
     "hhr_last_error": (ctypes.c_char_p, []),
     "hhr_set_wait_limit": (None, [ctypes.c_int64]),
     "hhr_build_cache": (_i32, [_cfgp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp]),
+    "hhr_append_cache": (_i32, [_cfgp, _vp, _vp, _vp, _vp, _vp, _vp, _i32, _vp, _vp, _vp, _vp, _vp, _vp, _vp]),
     "hhr_decode_workspace_size": (_sz, [_cfgp, _i32, _i32]),
     "hhr_workspace_init": (_i32, [_vp, _sz, _vp]),
     "hhr_decode_step": (_i32, [_cfgp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp,
@@ -56,6 +57,8 @@ SIGNATURES = {
     "hhr_decode_step_noalloc": (_i32, [_cfgp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp,
                                        _i32, _i32, ctypes.c_float, _vp, ctypes.POINTER(HHRDebug), _vp, _vp]),
     "hhr_dense_workspace_size": (_sz, [_cfgp]),
+    "hhr_exact_topk": (_i32, [_cfgp, _vp, _vp, _vp, _vp, _vp, _vp, _i32, _vp, _vp, _vp, _vp, _vp]),
+    "hhr_recall": (_i32, [_cfgp, _vp, _vp, _i32, _vp, _vp, _i32, _vp, _vp]),
     "hhr_dense_decode": (_i32, [_cfgp, _vp, _vp, _vp, _vp, _vp, _vp, ctypes.c_float, _vp, _vp, _sz,
                                 _vp, _vp]),
 }

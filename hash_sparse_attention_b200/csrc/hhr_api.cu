@@ -130,6 +130,12 @@ hhr_status make_dims(const hhr_config* cfg, Dims* dm) {
   dm->paged = cfg->paged ? 1 : 0;
   dm->num_blocks = cfg->paged ? cfg->num_blocks : 0;
   dm->max_blocks = cfg->paged ? cfg->max_blocks_per_seq : 0;
+  if (cfg->page_group_agg != 0 && cfg->page_group_agg != 1)
+    return fail(HHR_ERR_INVALID_ARG, "page_group_agg %d (0 max, 1 sum)", cfg->page_group_agg);
+  if (cfg->key_group_agg != 0 && cfg->key_group_agg != 1)
+    return fail(HHR_ERR_INVALID_ARG, "key_group_agg %d (0 sum, 1 min)", cfg->key_group_agg);
+  dm->page_sum = cfg->page_group_agg;
+  dm->key_min = cfg->key_group_agg;
   return HHR_OK;
 }
 
@@ -262,34 +268,60 @@ void hhr_set_wait_limit(int64_t cycles) {
   g_wait_cycles.store(cycles > 0 ? (long long)cycles : DEFAULT_WAIT_CYCLES, std::memory_order_relaxed);
 }
 
-hhr_status hhr_build_cache(const hhr_config* cfg, const void* K, const void* V, const float* R, const void* W,
-                           const int32_t* seq_lens, const int32_t* block_table, void* Krot, void* Vcache,
-                           void* page_min, void* page_max, uint64_t* codes, hhr_stream_t stream) {
+static hhr_status build_rows(const char* who, const hhr_config* cfg, const void* K, const void* V, const float* R,
+                             const void* W, const int32_t* starts, const int32_t* seq_lens, int32_t max_rows,
+                             const int32_t* block_table, void* Krot, void* Vcache, void* page_min, void* page_max,
+                             uint64_t* codes, hhr_stream_t stream) {
   Dims dm;
   hhr_status s = make_dims(cfg, &dm);
   if (s != HHR_OK) return s;
   if (!K || !V || !R || !W || !seq_lens || !Krot || !Vcache || !page_min || !page_max || !codes)
-    return fail(HHR_ERR_INVALID_ARG, "hhr_build_cache: NULL tensor pointer");
-  if (dm.paged && !block_table) return fail(HHR_ERR_INVALID_ARG, "hhr_build_cache: paged needs block_table");
+    return fail(HHR_ERR_INVALID_ARG, "%s: NULL tensor pointer", who);
+  if (dm.paged && !block_table) return fail(HHR_ERR_INVALID_ARG, "%s: paged needs block_table", who);
   const void* al[] = {K, V, R, W, Krot, Vcache, page_min, page_max, codes};
   for (const void* p : al)
-    if (!aligned16(p)) return fail(HHR_ERR_INVALID_ARG, "hhr_build_cache: tensor not 16-byte aligned");
-  cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
-  if (V != Vcache) {
-    const size_t bytes = dm.paged ? (size_t)dm.num_blocks * dm.Hkv * dm.P * D * 2
-                                  : (size_t)dm.B * dm.Hkv * dm.T * D * 2;
-    if (cudaMemcpyAsync(Vcache, V, bytes, cudaMemcpyDeviceToDevice, st) != cudaSuccess)
-      return check_cuda("hhr_build_cache: V copy");
-  }
-  const cudaError_t e = launch_build(dm, static_cast<const __nv_bfloat16*>(K), R, static_cast<const __nv_bfloat16*>(W),
-                                     seq_lens, block_table, static_cast<__nv_bfloat16*>(Krot),
-                                     static_cast<__nv_bfloat16*>(page_min), static_cast<__nv_bfloat16*>(page_max), codes,
-                                     nullptr, st);
+    if (!aligned16(p)) return fail(HHR_ERR_INVALID_ARG, "%s: tensor not 16-byte aligned", who);
+  if (max_rows < 1) return ok();  // nothing to build
+  BuildArgs a = {};
+  a.dm = dm;
+  a.K = static_cast<const __nv_bfloat16*>(K);
+  a.V = static_cast<const __nv_bfloat16*>(V);
+  a.R = R;
+  a.W = static_cast<const __nv_bfloat16*>(W);
+  a.starts = starts;
+  a.seq_lens = seq_lens;
+  a.table = block_table;
+  a.Krot = static_cast<__nv_bfloat16*>(Krot);
+  a.Vcache = static_cast<__nv_bfloat16*>(Vcache);
+  a.pmin = static_cast<__nv_bfloat16*>(page_min);
+  a.pmax = static_cast<__nv_bfloat16*>(page_max);
+  a.codes = codes;
+  a.status = nullptr;
+  a.max_rows = std::min(max_rows, dm.T);
+  a.stream = reinterpret_cast<cudaStream_t>(stream);
+  const cudaError_t e = launch_build(a);
   if (e != cudaSuccess) {
     cudaGetLastError();
-    return fail(HHR_ERR_CUDA, "hhr_build_cache: %s", cudaGetErrorString(e));
+    return fail(HHR_ERR_CUDA, "%s: %s", who, cudaGetErrorString(e));
   }
   return ok();
+}
+
+hhr_status hhr_build_cache(const hhr_config* cfg, const void* K, const void* V, const float* R, const void* W,
+                           const int32_t* seq_lens, const int32_t* block_table, void* Krot, void* Vcache,
+                           void* page_min, void* page_max, uint64_t* codes, hhr_stream_t stream) {
+  return build_rows("hhr_build_cache", cfg, K, V, R, W, nullptr, seq_lens, cfg ? cfg->max_seq_len : 0, block_table,
+                    Krot, Vcache, page_min, page_max, codes, stream);
+}
+
+hhr_status hhr_append_cache(const hhr_config* cfg, const void* K, const void* V, const float* R, const void* W,
+                            const int32_t* old_lens, const int32_t* new_lens, int32_t max_new,
+                            const int32_t* block_table, void* Krot, void* Vcache, void* page_min, void* page_max,
+                            uint64_t* codes, hhr_stream_t stream) {
+  if (!old_lens) return fail(HHR_ERR_INVALID_ARG, "hhr_append_cache: NULL old_lens");
+  if (max_new < 0) return fail(HHR_ERR_INVALID_ARG, "hhr_append_cache: max_new must be >= 0");
+  return build_rows("hhr_append_cache", cfg, K, V, R, W, old_lens, new_lens, max_new, block_table, Krot, Vcache,
+                    page_min, page_max, codes, stream);
 }
 
 size_t hhr_decode_workspace_size(const hhr_config* cfg, int32_t max_keep_pages, int32_t max_top_k) {

@@ -4,26 +4,26 @@
 namespace hhr {
 
 template <int NB>
-static cudaError_t launch_build_nb(const Dims& dm, const __nv_bfloat16* K, const float* R, const __nv_bfloat16* W,
-                                   const int* seq_lens, const int* table, __nv_bfloat16* Krot, __nv_bfloat16* pmin,
-                                   __nv_bfloat16* pmax, uint64_t* codes, int* status, cudaStream_t st) {
+static cudaError_t launch_build_nb(const BuildArgs& a) {
   const size_t smem = BuildSmem::bytes(NB);
   // the attribute belongs to the function; setting it again is harmless
   cudaError_t e = cudaFuncSetAttribute(build_cache_kernel<NB>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
   if (e != cudaSuccess) return e;
-  const dim3 grid((dm.T + BUILD_ROWS * BUILD_TILES - 1) / (BUILD_ROWS * BUILD_TILES), dm.Hkv, dm.B);
-  build_cache_kernel<NB><<<grid, BUILD_THREADS, smem, st>>>(dm, K, R, W, seq_lens, table, Krot, pmin, pmax, codes,
-                                                             status);
+  // rows per sequence the launch must cover: all of them, or the appended ones
+  // (they start inside a 64-row tile, hence one tile more)
+  const int span = a.max_rows + (a.starts ? BUILD_ROWS : 0);
+  const dim3 grid((span + BUILD_ROWS * BUILD_TILES - 1) / (BUILD_ROWS * BUILD_TILES), a.dm.Hkv, a.dm.B);
+  build_cache_kernel<NB><<<grid, BUILD_THREADS, smem, a.stream>>>(a.dm, a.K, a.V, a.R, a.W, a.starts, a.seq_lens,
+                                                                   a.table, a.Krot, a.Vcache, a.pmin, a.pmax,
+                                                                   a.codes, a.status);
   return cudaGetLastError();
 }
 
-cudaError_t launch_build(const Dims& dm, const __nv_bfloat16* K, const float* R, const __nv_bfloat16* W,
-                         const int* seq_lens, const int* table, __nv_bfloat16* Krot, __nv_bfloat16* pmin,
-                         __nv_bfloat16* pmax, uint64_t* codes, int* status, cudaStream_t st) {
-  switch (dm.nb) {
-    case 64: return launch_build_nb<64>(dm, K, R, W, seq_lens, table, Krot, pmin, pmax, codes, status, st);
-    case 128: return launch_build_nb<128>(dm, K, R, W, seq_lens, table, Krot, pmin, pmax, codes, status, st);
-    case 256: return launch_build_nb<256>(dm, K, R, W, seq_lens, table, Krot, pmin, pmax, codes, status, st);
+cudaError_t launch_build(const BuildArgs& a) {
+  switch (a.dm.nb) {
+    case 64: return launch_build_nb<64>(a);
+    case 128: return launch_build_nb<128>(a);
+    case 256: return launch_build_nb<256>(a);
   }
   return cudaErrorInvalidValue;
 }

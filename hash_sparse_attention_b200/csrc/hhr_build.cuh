@@ -1,13 +1,21 @@
-// HHR cache build (sm_100a), CUDA-core version.
+// HHR cache build and append (sm_100a), CUDA-core version.
 //
-// Per 64-row tile of one (sequence, KV head):
-//   K'  = bf16_rne(K R_h^T)          fp32 accumulation
+// For each sequence b the kernel (re)builds rows t in [S_b, L_b): S_b = 0 for
+// a full build, the old length for an append of new tokens.  Per 64-row tile
+// of one (sequence, KV head):
+//   K'  = bf16_rne(K R_h^T)          fp32 accumulation, in channel order j =
+//                                      0..127 for every row (the same
+//                                      arithmetic whatever the tile, so an
+//                                      append gives bit-identical rows)
 //   code bit j = [ (K W_h^T)_j > 0 ]  unrotated K; the fp32 sum of exact
 //                                      bf16 x bf16 products is trusted only
 //                                      when |sum| > 2^-14 |w_j| |k| (the fp32
 //                                      error is below 128 * 2^-24 sum|w k|),
 //                                      otherwise the sign comes from fp64
-//   page min / max over the valid stored K' rows of each page.
+//   page min / max over the valid stored K' rows of each page; a page that
+//   began before S_b merges its stored min / max with the new rows (min and
+//   max are exact, so the result equals a build over the whole page)
+//   V rows copied to the cache unless it aliases V.
 // A CTA walks BUILD_TILES consecutive tiles so that R_h and W_h are staged
 // in shared memory once per CTA.
 #pragma once
@@ -35,10 +43,10 @@ struct BuildSmem {
 
 template <int NB>
 __global__ void __launch_bounds__(BUILD_THREADS)
-build_cache_kernel(Dims dm, const __nv_bfloat16* K, const float* __restrict__ R,
-                   const __nv_bfloat16* __restrict__ W, const int* __restrict__ seq_lens,
-                   const int* __restrict__ table, __nv_bfloat16* Krot,
-                   __nv_bfloat16* __restrict__ pmin, __nv_bfloat16* __restrict__ pmax,
+build_cache_kernel(Dims dm, const __nv_bfloat16* K, const __nv_bfloat16* V, const float* __restrict__ R,
+                   const __nv_bfloat16* __restrict__ W, const int* __restrict__ starts,
+                   const int* __restrict__ seq_lens, const int* __restrict__ table, __nv_bfloat16* Krot,
+                   __nv_bfloat16* Vcache, __nv_bfloat16* __restrict__ pmin, __nv_bfloat16* __restrict__ pmax,
                    uint64_t* __restrict__ codes, int* status) {
   constexpr int NBT = NB / 16;   // bits per thread in the code product
   constexpr int WORDS = NB / 64;
@@ -53,8 +61,9 @@ build_cache_kernel(Dims dm, const __nv_bfloat16* K, const float* __restrict__ R,
 
   const int h = blockIdx.y, b = blockIdx.z, tid = threadIdx.x;
   const int L = seq_len_of(dm, seq_lens, b);
-  const int row0 = blockIdx.x * BUILD_TILES * BUILD_ROWS;
-  if (row0 >= L) return;
+  const int S0 = starts ? min(max(__ldg(starts + b), 0), L) : 0;  // first row (re)built
+  const int row0 = (S0 & ~(BUILD_ROWS - 1)) + blockIdx.x * BUILD_TILES * BUILD_ROWS;
+  if (row0 >= L || S0 >= L) return;
 
   // stage R_h^T and W_h^T, and the norms of the rows of W_h
   const float* Rh = R + (long long)h * D * D;
@@ -84,7 +93,7 @@ build_cache_kernel(Dims dm, const __nv_bfloat16* K, const float* __restrict__ R,
       const int r = e / (D / 8), v = e % (D / 8);
       const int t = t0 + r;
       float f[8] = {0, 0, 0, 0, 0, 0, 0, 0};
-      if (t < L) {
+      if (t >= S0 && t < L) {
         const long long off = kv_row(dm, table, b, h, t, status);
         if (off >= 0) unpack8(*reinterpret_cast<const uint4*>(K + off + v * 8), f);
       }
@@ -177,19 +186,22 @@ build_cache_kernel(Dims dm, const __nv_bfloat16* K, const float* __restrict__ R,
     }
     __syncthreads();
 
-    // ---- write K', codes and page min/max ----
+    // ---- write K' (and copy V), codes and page min/max ----
     for (int e = tid; e < BUILD_ROWS * (D / 8); e += BUILD_THREADS) {
       const int r = e / (D / 8), v = e % (D / 8);
       const int t = t0 + r;
-      if (t < L) {
+      if (t >= S0 && t < L) {
         const long long off = kv_row(dm, table, b, h, t, status);
-        if (off >= 0) *reinterpret_cast<uint4*>(Krot + off + v * 8) = *reinterpret_cast<const uint4*>(Ko + r * D + v * 8);
+        if (off >= 0) {
+          *reinterpret_cast<uint4*>(Krot + off + v * 8) = *reinterpret_cast<const uint4*>(Ko + r * D + v * 8);
+          if (Vcache != V) *reinterpret_cast<uint4*>(Vcache + off + v * 8) = ldg16(V + off + v * 8);
+        }
       }
     }
     for (int e = tid; e < BUILD_ROWS * WORDS; e += BUILD_THREADS) {
       const int r = e / WORDS, w = e % WORDS;
       const int t = t0 + r;
-      if (t < L) {
+      if (t >= S0 && t < L) {
         const long long off = code_row(dm, table, b, h, t, status);
         if (off >= 0) codes[off + w] = cd[r * 4 + w];
       }
@@ -198,16 +210,20 @@ build_cache_kernel(Dims dm, const __nv_bfloat16* K, const float* __restrict__ R,
     for (int e = tid; e < pages * D; e += BUILD_THREADS) {
       const int pp = e / D, c = e % D;
       const int tp = t0 + pp * dm.P;
-      if (tp >= L) continue;
-      const int rows = min(dm.P, L - tp);
+      const int r0 = max(0, S0 - tp), r1 = min(dm.P, L - tp);  // the page's rows built here
+      if (r0 >= r1) continue;
       float lo = INFINITY, hi = -INFINITY;
-      for (int r = 0; r < rows; ++r) {
+      for (int r = r0; r < r1; ++r) {
         const float x = __bfloat162float(Ko[(pp * dm.P + r) * D + c]);
         lo = fminf(lo, x);
         hi = fmaxf(hi, x);
       }
       const long long off = meta_row(dm, table, b, h, tp / dm.P, status);
       if (off >= 0) {
+        if (r0 > 0) {  // the page began before S0: merge with its stored rows
+          lo = fminf(lo, __bfloat162float(pmin[off + c]));
+          hi = fmaxf(hi, __bfloat162float(pmax[off + c]));
+        }
         pmin[off + c] = __float2bfloat16_rn(lo);
         pmax[off + c] = __float2bfloat16_rn(hi);
       }

@@ -15,6 +15,8 @@ constexpr int D = 128;  // head_dim: the only supported value
 struct Dims {
   int B, Hq, Hkv, G, P, nb, words, T, np_max, paged, num_blocks, max_blocks;
   int lgP;  // log2 of the page size (a power of two)
+  int page_sum;  // U_p: 0 max over the group's heads, 1 sum
+  int key_min;   // S_j: 0 sum over the group's heads, 1 min
 };
 
 // Workspace carve-out of one decode step (device pointers).  The per-unit

@@ -377,9 +377,16 @@ __device__ __forceinline__ void sp_scan_stage(const SpParams& p, const unsigned 
   group_reduce_scatter<NV, 16>(v, lane);
   const int q = li * NV / 16;
   const int half = q / GP, g = q % GP;
-  float U = g < G ? v[0] : -INFINITY;
+  float U;
+  if (!p.dm.page_sum) {  // max over the heads (lanes of a half hold its heads, some twice)
+    U = g < G ? v[0] : -INFINITY;
 #pragma unroll
-  for (int o = 1; o < 8; o <<= 1) U = fmaxf(U, __shfl_xor_sync(0xffffffffu, U, o));
+    for (int o = 1; o < 8; o <<= 1) U = fmaxf(U, __shfl_xor_sync(0xffffffffu, U, o));
+  } else {  // sum over the heads: one lane per head (NV = 8: even and odd lanes hold copies)
+    U = g < G ? v[0] : 0.f;
+#pragma unroll
+    for (int o = NV == 8 ? 2 : 1; o < 8; o <<= 1) U += __shfl_xor_sync(0xffffffffu, U, o);
+  }
   const int j = (tid >> 4) + 32 * half;
   const int pg = pg0 + j;
   if (pg < p1) {
@@ -810,11 +817,16 @@ __device__ int sp_keys(const SpParams& p, unsigned char* sm, const SpUnit& x, in
           cw[w2 + 1] = v2.y;
         }
       }
-      sv = 0;
+      int sum = 0, mn = INT_MAX;
 #pragma unroll
-      for (int w2 = 0; w2 < WORDS; ++w2)
+      for (int g = 0; g < G; ++g) {
+        int sg = 0;
 #pragma unroll
-        for (int g = 0; g < G; ++g) sv += __popcll(cw[w2] ^ cq[g][w2]);
+        for (int w2 = 0; w2 < WORDS; ++w2) sg += __popcll(cw[w2] ^ cq[g][w2]);
+        sum += sg;
+        mn = min(mn, sg);
+      }
+      sv = dm.key_min ? mn : sum;
       atomicAdd(&hist[sv], 1);
     }
     sc[j] = (uint16_t)sv;

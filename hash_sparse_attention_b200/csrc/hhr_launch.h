@@ -54,8 +54,26 @@ void dense_split(const Dims& dm, int sms, int* nsplit, int* rows);
 template <int G> cudaError_t launch_decode(const DecodeArgs& a);
 template <int G> cudaError_t launch_dense(const DecodeArgs& a);
 
-cudaError_t launch_build(const Dims& dm, const __nv_bfloat16* K, const float* R, const __nv_bfloat16* W,
-                         const int* seq_lens, const int* table, __nv_bfloat16* Krot, __nv_bfloat16* pmin,
-                         __nv_bfloat16* pmax, uint64_t* codes, int* status, cudaStream_t st);
+// Cache build over rows [starts[b], seq_lens[b]) of every sequence (starts
+// NULL: from row 0); max_rows bounds seq_lens[b] - starts[b].
+struct BuildArgs {
+  Dims dm;
+  const __nv_bfloat16* K;
+  const __nv_bfloat16* V;
+  const float* R;
+  const __nv_bfloat16* W;
+  const int* starts;
+  const int* seq_lens;
+  const int* table;
+  __nv_bfloat16* Krot;
+  __nv_bfloat16* Vcache;
+  __nv_bfloat16* pmin;
+  __nv_bfloat16* pmax;
+  uint64_t* codes;
+  int* status;
+  int max_rows;
+  cudaStream_t stream;
+};
+cudaError_t launch_build(const BuildArgs& a);
 
 }  // namespace hhr

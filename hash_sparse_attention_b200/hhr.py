@@ -14,16 +14,26 @@ import torch
 
 from ._lib import HHRConfig, HHRDebug, check, lib
 
-__all__ = ["HHRConfig", "HHRDebug", "make_config", "Cache", "alloc_cache", "build_cache",
+__all__ = ["HHRConfig", "HHRDebug", "make_config", "Cache", "alloc_cache", "build_cache", "append_cache",
+           "exact_topk", "recall",
            "decode_workspace", "dense_workspace", "decode_step", "decode_step_noalloc", "dense_decode", "DebugOutputs",
            "alloc_debug"]
 
 
+AGG = {"max": 0, "sum": 1, "min": 1}
+
+
 def make_config(batch: int, num_q_heads: int, num_kv_heads: int, page_size: int, hash_bits: int,
                 max_seq_len: int, paged: bool = False, num_blocks: int = 0,
-                max_blocks_per_seq: int = 0, head_dim: int = 128) -> HHRConfig:
+                max_blocks_per_seq: int = 0, head_dim: int = 128, page_agg: str = "max",
+                key_agg: str = "sum") -> HHRConfig:
+    """page_agg: "max" (default) or "sum" of the group's page bounds;
+    key_agg: "sum" (default) or "min" of the group's Hamming distances."""
+    if page_agg not in ("max", "sum") or key_agg not in ("sum", "min"):
+        raise ValueError("page_agg is 'max' or 'sum'; key_agg is 'sum' or 'min'")
     return HHRConfig(batch, num_q_heads, num_kv_heads, head_dim, page_size, hash_bits, max_seq_len,
-                     1 if paged else 0, num_blocks, max_blocks_per_seq)
+                     1 if paged else 0, num_blocks, max_blocks_per_seq, 1 if page_agg == "sum" else 0,
+                     1 if key_agg == "min" else 0)
 
 
 def _ptr(t: torch.Tensor | None) -> int | None:
@@ -94,6 +104,23 @@ def build_cache(cfg: HHRConfig, K: torch.Tensor, V: torch.Tensor, R: torch.Tenso
                                _ptr(block_table), _ptr(cache.Krot), _ptr(cache.V), _ptr(cache.page_min),
                                _ptr(cache.page_max), _ptr(cache.codes), _stream(stream))
     check(st, "hhr_build_cache")
+    return cache
+
+
+def append_cache(cfg: HHRConfig, K: torch.Tensor, V: torch.Tensor, R: torch.Tensor, W: torch.Tensor,
+                 old_lens: torch.Tensor, new_lens: torch.Tensor, max_new: int, block_table: torch.Tensor | None,
+                 cache: Cache, stream: torch.cuda.Stream | None = None) -> Cache:
+    """Builds rows [old_lens[b], new_lens[b]) of every sequence into `cache`
+    (rotation, codes, V, page min/max merged with the page's earlier rows)."""
+    sh = cache_shapes(cfg)
+    _expect(K, torch.bfloat16, sh["kv"], "K")
+    _expect(V, torch.bfloat16, sh["kv"], "V")
+    _expect(old_lens, torch.int32, (cfg.batch,), "old_lens")
+    _expect(new_lens, torch.int32, (cfg.batch,), "new_lens")
+    st = lib().hhr_append_cache(ctypes.byref(cfg), _ptr(K), _ptr(V), _ptr(R), _ptr(W), _ptr(old_lens),
+                                _ptr(new_lens), max_new, _ptr(block_table), _ptr(cache.Krot), _ptr(cache.V),
+                                _ptr(cache.page_min), _ptr(cache.page_max), _ptr(cache.codes), _stream(stream))
+    check(st, "hhr_append_cache")
     return cache
 
 
@@ -196,3 +223,32 @@ def dense_decode(cfg: HHRConfig, q: torch.Tensor, R: torch.Tensor, cache: Cache,
                                 workspace.numel(), _ptr(status), _stream(stream))
     check(st, "hhr_dense_decode")
     return out
+
+
+def exact_topk(cfg: HHRConfig, q: torch.Tensor, R: torch.Tensor, cache: Cache, seq_lens: torch.Tensor,
+               block_table: torch.Tensor | None, top_k: torch.Tensor, max_top_k: int,
+               stream: torch.cuda.Stream | None = None):
+    """The k keys with the largest max-over-the-group logit per (sequence, KV
+    head): returns (logits [B, Hkv, T] fp32, sel [B, Hkv, max_top_k], n_sel [B, Hkv])."""
+    _expect(q, torch.bfloat16, (cfg.batch, cfg.num_q_heads, cfg.head_dim), "q")
+    dev = q.device
+    logits = torch.empty(cfg.batch, cfg.num_kv_heads, cfg.max_seq_len, dtype=torch.float32, device=dev)
+    sel = torch.full((cfg.batch, cfg.num_kv_heads, max_top_k), -1, dtype=torch.int32, device=dev)
+    n_sel = torch.zeros(cfg.batch, cfg.num_kv_heads, dtype=torch.int32, device=dev)
+    st = lib().hhr_exact_topk(ctypes.byref(cfg), _ptr(q), _ptr(R), _ptr(cache.Krot), _ptr(seq_lens),
+                              _ptr(block_table), _ptr(top_k), max_top_k, _ptr(logits), _ptr(sel), _ptr(n_sel),
+                              None, _stream(stream))
+    check(st, "hhr_exact_topk")
+    return logits, sel, n_sel
+
+
+def recall(cfg: HHRConfig, sel_a: torch.Tensor, n_a: torch.Tensor, sel_b: torch.Tensor, n_b: torch.Tensor,
+           stream: torch.cuda.Stream | None = None) -> torch.Tensor:
+    """|A n B| / |B| per (sequence, KV head) for index lists [B, Hkv, *]."""
+    out = torch.empty(cfg.batch, cfg.num_kv_heads, dtype=torch.float32, device=sel_a.device)
+    st = lib().hhr_recall(ctypes.byref(cfg), _ptr(sel_a.contiguous()), _ptr(n_a.contiguous()), sel_a.shape[-1],
+                          _ptr(sel_b.contiguous()), _ptr(n_b.contiguous()), sel_b.shape[-1], _ptr(out),
+                          _stream(stream))
+    check(st, "hhr_recall")
+    return out
+

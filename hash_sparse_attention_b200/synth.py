@@ -22,6 +22,9 @@ Draw recipe, per (workload, layer):
   * a generator on the target device seeded with ``seed + 7919`` draws K,
     V and q (fp32 N(0,1), shaped [B, Hkv, T, d] / [B, Hq, d]), which are then
     scaled by the channel structure and rounded RNE to bf16.
+W_h law: "gaussian" (default) or "orthogonal" (rows of QR-orthogonalised
+Gaussian d x d matrices, the random-orthogonal-projection hash of the paper's
+Figure 2, one d x d block per d bits).
 Data laws: "outlier" = 4 channels per (layer, KV head) drawn without
 replacement, independently for K and V, multiplied by 10; "student_t3" =
 per (KV head, channel) scale |t_3| (t_3 = z / sqrt(chi2_3 / 3)), separately
@@ -52,6 +55,9 @@ class Workload:
     topk_den: int = 10            # top-k = ceil(L / topk_den) keys ...
     top_k: int | None = None      # ... unless a fixed k is given
     law: str = "outlier"          # "outlier" or "student_t3"
+    hash_law: str = "gaussian"    # W_h: "gaussian" (N(0,1)) or "orthogonal" (rows of random orthogonal matrices)
+    page_agg: str = "max"         # page bound over the group's query heads: "max" or "sum"
+    key_agg: str = "sum"          # Hamming score over the group's query heads: "sum" or "min"
     paged: bool = False
     ragged_min: int | None = None  # ragged contexts drawn uniform in [ragged_min, context]
     seed: int = 0
@@ -122,6 +128,23 @@ def orthogonal_from_gaussian(g: torch.Generator, d: int) -> np.ndarray:
     s = np.sign(np.diag(rm))
     s[s == 0] = 1.0
     return qm * s[None, :]
+
+
+def hash_projection(w: Workload, g: torch.Generator) -> torch.Tensor:
+    """W_h before rounding to bf16 (fp32, nb x d).
+
+    "gaussian": N(0,1) entries, the stand-in for the learned projection.
+    "orthogonal": the random-orthogonal-projection hash of the paper's
+    Figure 2 caption (random orthogonal projection, then sign): rows of
+    QR-orthogonalised Gaussian d x d matrices, as many blocks of d rows as nb
+    needs (256 bits at d = 128: two independent blocks)."""
+    nb, d = w.hash_bits, w.head_dim
+    if w.hash_law == "gaussian":
+        return torch.randn(nb, d, generator=g, dtype=torch.float32)
+    if w.hash_law == "orthogonal":
+        blocks = [torch.from_numpy(orthogonal_from_gaussian(g, d).T.copy()) for _ in range(-(-nb // d))]
+        return torch.cat(blocks, 0)[:nb].to(torch.float32)
+    raise ValueError(f"unknown hash law {w.hash_law!r}")
 
 
 def _channel_scales(w: Workload, g: torch.Generator) -> torch.Tensor:
@@ -199,7 +222,7 @@ def make_layer(w: Workload, layer: int = 0, device: str | torch.device = "cpu",
     vsc = torch.empty(Hkv, d, dtype=torch.float32)
     for h in range(Hkv):
         R64[h] = orthogonal_from_gaussian(g, d)
-        Wb[h] = torch.randn(nb, d, generator=g, dtype=torch.float32).to(torch.bfloat16)
+        Wb[h] = hash_projection(w, g).to(torch.bfloat16)
         ksc[h] = _channel_scales(w, g)
         vsc[h] = _channel_scales(w, g)
 
@@ -288,4 +311,4 @@ def l2_flush_bytes() -> int:
 
 
 __all__ = ["Workload", "WORKLOADS", "LayerInputs", "make_layer", "scaled", "to_pool",
-           "from_pool", "num_pages", "orthogonal_from_gaussian", "l2_flush_bytes"]
+           "from_pool", "num_pages", "orthogonal_from_gaussian", "hash_projection", "l2_flush_bytes"]

@@ -79,6 +79,10 @@ typedef struct {
   int32_t paged;              /* 0 contiguous, 1 block pool + block table     */
   int32_t num_blocks;         /* Bk: blocks in the pool (paged only)          */
   int32_t max_blocks_per_seq; /* row length of block_table (paged only)       */
+  /* How the G query heads of a KV head are combined (the paper is silent on
+   * grouped query heads; 0 selects the library's readings):                 */
+  int32_t page_group_agg;     /* page bound U_p: 0 max over the heads, 1 sum  */
+  int32_t key_group_agg;      /* key score S_j: 0 sum over the heads, 1 min   */
 } hhr_config;
 
 /* Optional stage outputs of hhr_decode_step (any pointer may be NULL). They
@@ -133,13 +137,42 @@ HHR_API void hhr_set_wait_limit(int64_t cycles);
  *                     lie below seq_lens[b]
  *   Vcache = V (copied unless Vcache == V).
  * Rows at or past seq_lens[b] and pages past the last valid one are left
- * untouched.  Krot may alias K (in place).  seq_lens is a device array [B].
+ * untouched (V rows are copied for t < seq_lens[b] only).  Krot may alias K
+ * (in place).  seq_lens is a device array [B].
  */
 HHR_API hhr_status hhr_build_cache(const hhr_config* cfg, const void* K, const void* V,
                            const float* R, const void* W, const int32_t* seq_lens,
                            const int32_t* block_table, void* Krot, void* Vcache,
                            void* page_min, void* page_max, uint64_t* codes,
                            hhr_stream_t stream);
+
+/*
+ * hhr_append_cache -- extends the cache as tokens are generated.
+ *
+ * A decode loop adds one key and value per step; GKR keeps a bound per page
+ * of neighbouring keys, so the new key must be rotated and hashed and its
+ * page's stored min/max kept current (rit.work explainer, sections "Два
+ * уровня маршрутизации решают разные ошибки": pages of neighbouring keys with
+ * a bound each, and "Когда HHR меняет планы запуска модели": the page bounds
+ * are stored with the cache).  For every sequence b, rows t in
+ * [old_lens[b], new_lens[b]) are built exactly as hhr_build_cache builds them
+ * (K'[t], codes[t], V copied unless Vcache == V), and the min/max of every page
+ * they touch is merged with that page's rows below old_lens[b] (a page that
+ * starts at t is opened).  The cache then equals, bit for bit, a
+ * hhr_build_cache over [0, new_lens[b]).
+ *   - K and V hold the new rows at their cache positions (same layouts as
+ *     hhr_build_cache); only rows >= old_lens[b] are read, so K may alias
+ *     Krot (write the raw key into Krot's row, then append).
+ *   - old_lens and new_lens are device arrays [B]; lengths are clamped to
+ *     [0, max_seq_len] and a sequence with new_lens[b] <= old_lens[b] is left
+ *     untouched.  max_new (host) bounds new_lens[b] - old_lens[b]; it sizes
+ *     the launch (rows beyond it are not built).
+ *   - Paged: the blocks of the new rows must already be in block_table.
+ */
+HHR_API hhr_status hhr_append_cache(const hhr_config* cfg, const void* K, const void* V, const float* R,
+                                    const void* W, const int32_t* old_lens, const int32_t* new_lens,
+                                    int32_t max_new, const int32_t* block_table, void* Krot, void* Vcache,
+                                    void* page_min, void* page_max, uint64_t* codes, hhr_stream_t stream);
 
 /* Bytes of workspace hhr_decode_step needs for these budgets. */
 HHR_API size_t hhr_decode_workspace_size(const hhr_config* cfg, int32_t max_keep_pages,
@@ -155,13 +188,14 @@ HHR_API hhr_status hhr_workspace_init(void* workspace, size_t workspace_bytes, h
  * For each sequence b with L = seq_lens[b], np = ceil(L / P), each KV head h
  * and its query heads g (hq = h*G + g):
  *  1. q'_g = R_h q_g (fp32).                      GKR rotation (Abstract)
- *  2. ub[g,p] = sum_i max(q'_gi mn_pi, q'_gi mx_pi); U_p = max_g ub[g,p].
- *                                                 page logit bound (Abstract)
+ *  2. ub[g,p] = sum_i max(q'_gi mn_pi, q'_gi mx_pi); U_p = max_g ub[g,p]
+ *     (sum_g with cfg->page_group_agg = 1).       page logit bound (Abstract)
  *  3. keep N = min(clamp(n_keep_pages[b], 1, max_keep_pages), np) pages with
  *     the largest U_p; equal bounds go to the lower page index.  Coarse
  *     pruning of whole pages (rit.work, two-level routing section).
  *  4. query codes: bit j = [ (W_h q_g)_j > 0 ] (exact sign, fp64 fallback).
- *  5. for the valid rows of kept pages: S = sum_g popcount(code_g ^ code_row).
+ *  5. for the valid rows of kept pages: S = sum_g popcount(code_g ^ code_row)
+ *     (min_g with cfg->key_group_agg = 1).
  *  6. keep k = min(clamp(top_k[b], 1, max_top_k), #candidates) rows with the
  *     smallest S; equal scores go to the lower token index.
  *  7. out[b, hq] = sum_j softmax_j(sm_scale * q'_g . Krot_j) V_j over the kept
@@ -238,6 +272,37 @@ HHR_API hhr_status hhr_decode_step_noalloc(const hhr_config* cfg, const void* q,
                                            int32_t max_top_k, float sm_scale, float* out,
                                            const hhr_debug* dbg, int32_t* device_status,
                                            hhr_stream_t stream);
+
+/*
+ * hhr_exact_topk -- the exact top-k keys, the reference of the recall metric
+ * ("HHR: Hierarchical Hash Retrieval for Efficient LLM Generation",
+ * thelatestinai.com page, Figure 4 caption: "Top-10% key recall").
+ *
+ * For every sequence b (L = seq_lens[b]) and KV head h, the score of key t < L
+ * is the largest logit of the group's query heads,
+ *   logits[b, h, t] = max_g (R_h q_g) . Krot[t]       (fp32, channel order),
+ * and -inf for t >= L (layout [B, Hkv, max_seq_len]).  sel[b, h, :n] holds the
+ * k = min(clamp(top_k[b], 1, max_top_k), L) keys with the largest scores,
+ * ascending (equal scores go to the lower token); n_sel[b, h] = k.
+ * top_k is a device array [B]; sel is [B, Hkv, max_top_k].  Same layouts and
+ * alignment rules as hhr_decode_step; no workspace (logits is the scratch).
+ * The paper has no kernel for this: it is the measuring stick of Figure 4.
+ */
+HHR_API hhr_status hhr_exact_topk(const hhr_config* cfg, const void* q, const float* R, const void* Krot,
+                                  const int32_t* seq_lens, const int32_t* block_table, const int32_t* top_k,
+                                  int32_t max_top_k, float* logits, int32_t* sel, int32_t* n_sel,
+                                  int32_t* device_status, hhr_stream_t stream);
+
+/*
+ * hhr_recall -- recall[u] = |A_u n B_u| / |B_u| for every unit u = b*Hkv + h,
+ * where A_u = sel_a[u*stride_a .. +n_a[u]) (e.g. the keys a decode step kept:
+ * hhr_debug.sel_keys) and B_u = sel_b[u*stride_b .. +n_b[u]) (e.g. the exact
+ * top-k of hhr_exact_topk).  Token ids outside [0, max_seq_len) are ignored.
+ * Device arrays; recall is float [B*Hkv] (0 where B_u is empty).
+ */
+HHR_API hhr_status hhr_recall(const hhr_config* cfg, const int32_t* sel_a, const int32_t* n_a, int32_t stride_a,
+                              const int32_t* sel_b, const int32_t* n_b, int32_t stride_b, float* recall,
+                              hhr_stream_t stream);
 
 /* Bytes of workspace hhr_dense_decode needs. */
 HHR_API size_t hhr_dense_workspace_size(const hhr_config* cfg);

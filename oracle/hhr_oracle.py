@@ -132,13 +132,19 @@ def page_bounds(Qr: np.ndarray, mn: np.ndarray, mx: np.ndarray) -> np.ndarray:
     return ub
 
 
-def group_bound(ub: np.ndarray) -> np.ndarray:
+def group_bound(ub: np.ndarray, mode: str = "max") -> np.ndarray:
     """U_p = max over the query heads of the group of ub[g, p].
 
     READING (pages silent on GQA): the max keeps U_p an upper bound for every
     query head that shares the KV head, so one page selection serves them all.
+    mode "sum" is the alternative aggregation: U_p = sum over the heads (a bound
+    of the group's summed logits).
     """
-    return ub.max(axis=0)
+    if mode == "max":
+        return ub.max(axis=0)
+    if mode == "sum":
+        return ub.sum(axis=0)
+    raise ValueError(mode)
 
 
 def select_pages(U: np.ndarray, N: int) -> np.ndarray:
@@ -194,16 +200,22 @@ def hash_codes(W: np.ndarray, X: np.ndarray) -> np.ndarray:
     return out
 
 
-def hamming(cq: np.ndarray, codes: np.ndarray) -> np.ndarray:
+def hamming(cq: np.ndarray, codes: np.ndarray, mode: str = "sum") -> np.ndarray:
     """S_j = sum over the group's query codes of the number of differing bits.
 
     Hamming distance counts mismatching bits (paper card Abstract; rit.work,
     first section).  READING (pages silent on GQA): the group score is the sum
     over its query heads, i.e. the distance between concatenated codes.
+    mode "min" is the alternative: the distance to the closest query head.
     cq: uint64 [G, w]; codes: uint64 [n, w] -> int64 [n].
     """
     x = np.bitwise_xor(codes[None, :, :], cq[:, None, :])  # [G, n, w]
-    return np.bitwise_count(x).astype(np.int64).sum(axis=(0, 2))
+    per_head = np.bitwise_count(x).astype(np.int64).sum(axis=2)  # [G, n]
+    if mode == "sum":
+        return per_head.sum(axis=0)
+    if mode == "min":
+        return per_head.min(axis=0)
+    raise ValueError(mode)
 
 
 def select_keys(S: np.ndarray, cand: np.ndarray, k: int) -> np.ndarray:
@@ -263,7 +275,8 @@ def build_head(K: np.ndarray, R: np.ndarray, W: np.ndarray, L: int, P: int):
 
 def decode_head(Q: np.ndarray, R: np.ndarray, W: np.ndarray, Kp: np.ndarray, V: np.ndarray,
                 mn: np.ndarray, mx: np.ndarray, codes: np.ndarray, L: int, P: int,
-                N: int, k: int, scale: float | None = None) -> dict:
+                N: int, k: int, scale: float | None = None, page_agg: str = "max",
+                key_agg: str = "sum") -> dict:
     """One decode step of HHR for the G query heads of one KV head, all stages.
 
     Q: [G, d] query rows; the other arrays as returned by build_head.
@@ -279,11 +292,11 @@ def decode_head(Q: np.ndarray, R: np.ndarray, W: np.ndarray, Kp: np.ndarray, V: 
                     q_codes=hash_codes(W, Q), cand=np.zeros(0, np.int64), scores=np.zeros(0, np.int64),
                     sel_keys=np.zeros(0, np.int64), out=np.zeros((G, d)))
     ub = page_bounds(Qr, mn, mx)
-    U = group_bound(ub)
+    U = group_bound(ub, page_agg)
     sel_p = select_pages(U, N)
     cq = hash_codes(W, Q)
     cand = candidates(sel_p, L, P)
-    S = hamming(cq, codes[cand])
+    S = hamming(cq, codes[cand], key_agg)
     sel_k = select_keys(S, cand, k)
     out = attention(Qr, Kp, V, sel_k, scale)
     return dict(q_rot=Qr, ub=ub, U=U, sel_pages=sel_p, q_codes=cq, cand=cand, scores=S,
@@ -297,3 +310,36 @@ def dense_head(Q: np.ndarray, R: np.ndarray, Kp: np.ndarray, V: np.ndarray, L: i
     if scale is None:
         scale = 1.0 / math.sqrt(d)
     return attention(rotate_query(R, Q), Kp, V, np.arange(L), scale)
+
+
+# ---------------------------------------------------------------------------
+# Exact top-k and recall (the fidelity measure of the paper's Figure 4)
+# ---------------------------------------------------------------------------
+
+def key_scores_exact(Qr: np.ndarray, Kp: np.ndarray) -> np.ndarray:
+    """z_t = max over the group's query heads of q'_g . k'_t (fp64).
+
+    "Top-10% key recall" (thelatestinai.com page, Figure 4 caption) measures
+    retrieval against the truly highest-scoring keys.  READING: with grouped
+    query heads sharing one KV head, a key's score is the largest logit of the
+    group (a key matters if any head of the group attends to it; the same
+    aggregation as the page bound's U_p)."""
+    return (np.asarray(Kp, dtype=np.float64) @ np.asarray(Qr, dtype=np.float64).T).max(axis=1)
+
+
+def exact_topk(z: np.ndarray, k: int) -> np.ndarray:
+    """The k keys with the largest score, ascending ids; READING: equal scores
+    go to the lower token, k is clamped to the number of keys."""
+    z = np.asarray(z, dtype=np.float64)
+    k = min(int(k), z.shape[0])
+    order = np.argsort(-z, kind="stable")
+    return np.sort(order[:k]).astype(np.int64)
+
+
+def recall(sel: np.ndarray, exact: np.ndarray) -> float:
+    """|sel n exact| / |exact| (0 for an empty reference)."""
+    exact = np.asarray(exact)
+    if exact.size == 0:
+        return 0.0
+    return float(np.intersect1d(np.asarray(sel), exact).size) / float(exact.size)
+

@@ -37,8 +37,10 @@ INT32_MAX = 2**31 - 1
 def config_for(w: Workload, li: LayerInputs) -> hhr.HHRConfig:
     if w.paged:
         return hhr.make_config(w.batch, w.num_q_heads, w.num_kv_heads, w.page_size, w.hash_bits, w.context,
-                               paged=True, num_blocks=li.K.shape[0], max_blocks_per_seq=li.block_table.shape[1])
-    return hhr.make_config(w.batch, w.num_q_heads, w.num_kv_heads, w.page_size, w.hash_bits, w.context)
+                               paged=True, num_blocks=li.K.shape[0], max_blocks_per_seq=li.block_table.shape[1],
+                               page_agg=w.page_agg, key_agg=w.key_agg)
+    return hhr.make_config(w.batch, w.num_q_heads, w.num_kv_heads, w.page_size, w.hash_bits, w.context,
+                           page_agg=w.page_agg, key_agg=w.key_agg)
 
 
 @dataclass
@@ -239,14 +241,18 @@ def check_decode(w: Workload, li: LayerInputs, g: GpuRun, rep: Report, heads=Non
             assert np.all(err <= tol), "page bound outside tolerance"
             rep.max_bound_err = max(rep.max_bound_err, float((err / np.maximum(tol / BOUND_RTOL, 1e-300)).max()))
             U = dg["page_U"][b, h, :np_b]
-            assert np.array_equal(U, ub.max(axis=0)), "U is not the group max of ub"
+            if w.page_agg == "max":
+                assert np.array_equal(U, ub.max(axis=0)), "U is not the group max of ub"
+            else:  # fp32 sum of G terms in the kernel's order
+                Us = ub.astype(np.float64).sum(axis=0)
+                assert np.all(np.abs(U - Us) <= 2.0 ** -21 * G * np.abs(ub).sum(axis=0)), "U is not the group sum of ub"
             # page top-N: bit exact on the GPU's bounds
             Neff = min(N, np_b)
             assert dg["n_sel_pages"][b, h] == Neff
             sel_p = dg["sel_pages"][b, h, :Neff]
             assert np.array_equal(sel_p, O.select_pages(U.astype(np.float64), Neff)), "page select differs"
             # against the fp64 bounds, outside the exempt band
-            U64 = O.group_bound(ub_ref)
+            U64 = O.group_bound(ub_ref, w.page_agg)
             ref_p = O.select_pages(U64, Neff)
             if Neff < np_b:
                 thr = np.sort(U64)[::-1][Neff - 1]
@@ -256,7 +262,7 @@ def check_decode(w: Workload, li: LayerInputs, g: GpuRun, rep: Report, heads=Non
                 rep.page_exempt_diff += len(sym)
             # Hamming on the GPU's codes of the GPU's candidates
             cand = O.candidates(sel_p, L, P)
-            S_ref = O.hamming(cq, g.codes[b, h][cand])
+            S_ref = O.hamming(cq, g.codes[b, h][cand], w.key_agg)
             assert dg["n_cand"][b, h] == len(cand)
             sc = dg["key_scores"][b, h, :Neff * P]
             slot_tok = (sel_p[:, None] * P + np.arange(P)[None]).reshape(-1)
@@ -275,7 +281,8 @@ def check_decode(w: Workload, li: LayerInputs, g: GpuRun, rep: Report, heads=Non
                 assert e <= OUT_RTOL, f"attention output rel err {e:.3g} b{b} h{h} g{gg}"
             if e2e:
                 Kp, mn_o, mx_o, codes_o = O.build_head(Klog[b, h], R32[h], Wn[h], L, P)
-                r = O.decode_head(Q, R32[h], Wn[h], Kp, Vlog[b, h, :L], mn_o, mx_o, codes_o, L, P, N, k, scale)
+                r = O.decode_head(Q, R32[h], Wn[h], Kp, Vlog[b, h, :L], mn_o, mx_o, codes_o, L, P, N, k, scale,
+                                  page_agg=w.page_agg, key_agg=w.key_agg)
                 dp = len(np.setxor1d(r["sel_pages"], sel_p))
                 dk = len(np.setxor1d(r["sel_keys"], sel_k))
                 rep.e2e_page_diff += dp

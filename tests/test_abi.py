@@ -32,6 +32,7 @@ def L():
 def test_header_declares_the_boundary():
     fns = declared_functions()
     assert fns == sorted(["hhr_status_string", "hhr_last_error", "hhr_set_wait_limit", "hhr_build_cache",
+                          "hhr_append_cache", "hhr_exact_topk", "hhr_recall",
                           "hhr_decode_workspace_size",
                           "hhr_workspace_init", "hhr_decode_step", "hhr_decode_step_noalloc",
                           "hhr_dense_workspace_size", "hhr_dense_decode"])

@@ -100,13 +100,13 @@ def test_profiled_traffic_only_for_matching_sources_and_workload(tmp_path, monke
 
     prof = tmp_path / "profiles"
     prof.mkdir()
-    f = prof / "hhr_group_kernel_llama_32l_128k.md"
+    f = prof / "hhr_sparse_kernel_llama_32l_128k.md"
     monkeypatch.setattr(bench, "ROOT", str(tmp_path))
     assert bench.profiled_traffic("llama_32l_128k") is None  # no summary
     monkeypatch.setattr(bench, "kernel_source_hash", lambda: "abc123")
     f.write_text("- workload: `llama_32l_128k`\n- dram_bytes_per_launch: `1234`\n- sources_sha256: `abc123`\n")
     assert bench.profiled_traffic("llama_32l_128k") == 1234.0
-    assert bench.profiled_traffic("qwen_gqa7_128k") is None  # another workload
+    assert bench.profiled_traffic("qwen_gqa7_128k") is None  # another workload (no summary of its own)
     f.write_text("- workload: `llama_32l_128k`\n- dram_bytes_per_launch: `1234`\n- sources_sha256: `def456`\n")
     assert bench.profiled_traffic("llama_32l_128k") is None  # sources changed since the capture
     f.write_text("- workload: `llama_32l_128k`\n- sources_sha256: `abc123`\n")
@@ -141,3 +141,17 @@ def test_reference_arm_prints_one_contract_line():
     assert d["cpu_baseline"]["kind"] == "oracle" and d["cpu_baseline"]["value"] == d["value"]
     assert d["e2e"] == {"value": d["value"], "unit": d["unit"], "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}
     assert d["config"]["workload"] == "llama_32l_128k"
+
+
+def test_cpu_baseline_single_and_all_cores():
+    """The oracle leg: one thread, then single-threaded spawned processes over
+    memory-mapped unit caches; both report tokens/s, the core count and the CPU
+    model."""
+    from hash_sparse_attention_b200.synth import WORKLOADS, scaled
+    w = scaled(WORKLOADS["tiny_4k"], context=1024)
+    out = bench.cpu_baseline(w, 0.5, workers=2)
+    assert out["kind"] == "oracle" and out["cores"] == 1 and out["value"] > 0
+    assert out["cpu_model"] and out["host_cores"] >= 1
+    ac = out["all_cores"]
+    assert ac["cores"] == 2 and ac["value"] > 0 and ac["kind"] == "oracle"
+

@@ -252,3 +252,26 @@ def test_bounded_wait_runs_out_and_reports_timeout():
     torch.cuda.synchronize()
     assert int(status.item()) == 0
     assert torch.equal(out2, clean.out)
+
+
+@pytest.mark.parametrize("bits", [64, 128, 256])
+def test_orthogonal_hash_projection(bits):
+    """The random-orthogonal-projection hash (paper page, Figure 2 caption) at
+    each code width (Figure 10's bit sweep): the same kernels, another W."""
+    _cuda()
+    w = scaled(WORKLOADS["llama_layer_32k"], context=6000, batch=2, hash_bits=bits, hash_law="orthogonal",
+               seed=90 + bits)
+    li = make_layer(w)
+    _run_and_check(w, li)
+
+
+@pytest.mark.parametrize("G,page_agg,key_agg", [(4, "sum", "sum"), (4, "max", "min"), (7, "sum", "min"),
+                                                (1, "sum", "min"), (8, "sum", "sum")])
+def test_group_aggregation_modes(G, page_agg, key_agg):
+    """The alternatives to the library's readings for grouped query heads: the
+    page bound summed over the group, the Hamming distance of the closest head."""
+    _cuda()
+    w = scaled(WORKLOADS["llama_layer_32k"], num_q_heads=2 * G, num_kv_heads=2, context=5000, batch=2,
+               page_agg=page_agg, key_agg=key_agg, seed=100 + G)
+    li = make_layer(w)
+    _run_and_check(w, li)

@@ -20,6 +20,14 @@ Each oracle function is checked against something other than itself:
   attention       torch scaled_dot_product_attention in fp64 when every key
                   is kept; one key gives v; q=0 gives the mean of V
   decode_head     the hand-derived fixture tests/golden/hhr_hand_example.json
+  key_scores_exact  rotation invariance (scores of rotated vectors equal the
+                  max over heads of the unrotated q.k, computed without the
+                  oracle) and a hand example where max and sum differ
+  exact_topk      brute-force rank definition (largest first, ties to the
+                  lower index)
+  recall          hand examples (the denominator is the reference set)
+  group_bound / hamming aggregation modes (sum of bounds, min distance):
+                  hand examples where the modes differ
 
 The last test plants plausible mistakes in copies of oracle functions and
 checks that some pin rejects each of them.
@@ -397,6 +405,64 @@ def test_rotation_spreads_outlier_channels():
 
 # ---------------------------------------------------------------------------
 # planted mistakes: each mutant must be rejected by some pin
+def pin_key_scores(key_scores_exact):
+    rng = _rng(41)
+    d, G = 16, 3
+    R = _orth(rng, d)
+    Q = rng.standard_normal((G, d))
+    K = rng.standard_normal((50, d)) * 2
+    z = key_scores_exact(Q @ R.T, K @ R.T)  # rotated query and keys (R applied by matmul)
+    ref = np.array([max(float(np.dot(Q[g], K[t])) for g in range(G)) for t in range(50)])
+    assert np.all(np.abs(z - ref) <= 1e-9 * np.linalg.norm(K, axis=1) * np.linalg.norm(Q, axis=1).max())
+    # hand example: two heads, max over heads (a sum would give [-1, 3, 0])
+    z = key_scores_exact(np.array([[1.0, 0.0], [0.0, 1.0]]), np.array([[2.0, -3.0], [-1.0, 4.0], [0.0, 0.0]]))
+    assert np.array_equal(z, [2.0, 4.0, 0.0])
+
+
+def pin_exact_topk(exact_topk):
+    rng = _rng(42)
+    for n, k in ((30, 7), (30, 30), (10, 40), (25, 1)):
+        z = rng.integers(0, 6, n).astype(np.float64)  # many ties
+        got = exact_topk(z, k)
+        keep = [t for t in range(n)
+                if sum(1 for u in range(n) if z[u] > z[t] or (z[u] == z[t] and u < t)) < min(k, n)]
+        assert np.array_equal(got, keep)
+
+
+def pin_recall(recall):
+    assert recall(np.array([1, 2, 3]), np.array([2, 3, 4, 5])) == 0.5
+    assert recall(np.array([7]), np.array([7])) == 1.0
+    assert recall(np.array([], dtype=np.int64), np.array([1])) == 0.0
+    assert recall(np.array([1, 2]), np.array([], dtype=np.int64)) == 0.0
+    assert recall(np.array([1, 2, 3, 4]), np.array([4])) == 1.0
+
+
+def pin_aggregation_modes(group_bound, hamming):
+    ub = np.array([[3.0, 1.0, -2.0], [2.0, 2.0, 1.0]])
+    assert np.array_equal(group_bound(ub, "max"), [3.0, 2.0, 1.0])
+    assert np.array_equal(group_bound(ub, "sum"), [5.0, 3.0, -1.0])
+    cq = np.array([[0b1011], [0b0000]], dtype=np.uint64)      # two heads, one word
+    codes = np.array([[0b1010], [0b1111], [0b0000]], dtype=np.uint64)
+    assert np.array_equal(hamming(cq, codes, "sum"), [1 + 2, 1 + 4, 3 + 0])
+    assert np.array_equal(hamming(cq, codes, "min"), [1, 1, 0])
+
+
+def test_aggregation_modes():
+    pin_aggregation_modes(O.group_bound, O.hamming)
+
+
+def test_key_scores_exact():
+    pin_key_scores(O.key_scores_exact)
+
+
+def test_exact_topk():
+    pin_exact_topk(O.exact_topk)
+
+
+def test_recall():
+    pin_recall(O.recall)
+
+
 # ---------------------------------------------------------------------------
 
 def _fails(fn, *args):
@@ -460,3 +526,18 @@ def test_planted_mistakes_are_caught():
     # attention without the max shift is fine numerically; without normalisation / scale it is not
     assert _fails(pin_attention, lambda Q, K, V, s, sc: np.stack([np.exp(sc * (K[s] @ q)) @ V[s] for q in Q]))
     assert _fails(pin_attention, lambda Q, K, V, s, sc: O.attention(Q, K, V, s, 1.0))
+    # key scores summed over the group instead of the max; top-k ties to the higher
+    # index; recall over the selection's size
+    assert _fails(pin_key_scores, lambda Qr, Kp: (np.asarray(Kp) @ np.asarray(Qr).T).sum(axis=1))
+    def topk_ties_high(z, k):
+        n = len(z)
+        order = np.argsort(-z[::-1], kind="stable")
+        return np.sort(n - 1 - order[:min(k, n)])
+    assert _fails(pin_exact_topk, topk_ties_high)
+    assert _fails(pin_recall, lambda a, b: float(np.intersect1d(a, b).size) / max(1, np.asarray(a).size))
+    # the modes swapped
+    assert _fails(pin_aggregation_modes, lambda ub, m="max": O.group_bound(ub, "sum" if m == "max" else "max"),
+                  O.hamming)
+    assert _fails(pin_aggregation_modes, O.group_bound,
+                  lambda cq, c, m="sum": O.hamming(cq, c, "min" if m == "sum" else "sum"))
+
