@@ -140,8 +140,8 @@ hhr_status make_dims(const hhr_config* cfg, Dims* dm) {
 }
 
 // Carves the workspace; with base == nullptr only the size is computed.
-// Sparse: per-unit counters, page bounds, the kept-row list, one partial per
-// gather chunk, one score histogram per CTA.  Dense: counters and one
+// Sparse: per-unit counters, page bounds, one attention partial per CTA of
+// the unit's group, one score histogram per CTA.  Dense: counters and one
 // partial per split.
 size_t carve(const Dims& dm, int Nmax, int Kmax, bool dense, char* base, Work* wk) {
   const size_t BH = (size_t)dm.B * dm.Hkv;
@@ -159,12 +159,13 @@ size_t carve(const Dims& dm, int Nmax, int Kmax, bool dense, char* base, Work* w
     w.C3 = std::min(MAX_GRID, ceil_div(dm.T, GATHER_ROWS));
     w.part = reinterpret_cast<float*>(take(sizeof(float) * BH * w.C3 * PS));
   } else {
+    // one partial per CTA of a unit's group: at most max(1, 160 / units) CTAs,
+    // or as many as the kept rows need (sparse_group_shape)
     const long long kcap = std::min<long long>(Kmax, (long long)Nmax * dm.P);
-    w.C3 = std::max(1, ceil_div(kcap, GATHER_ROWS));
+    w.C3 = std::max({1, MAX_GRID / (int)BH, ceil_div(kcap, MAX_KEPT_PER_CTA)});
     w.Ustride = (dm.np_max + 31) / 32 * 32;
     w.HB = (dm.G * dm.nb + 1 + 7) / 8 * 8;
     w.U = reinterpret_cast<float*>(take(sizeof(float) * BH * w.Ustride));
-    w.sel_keys = reinterpret_cast<int*>(take(sizeof(int) * BH * Kmax));
     w.part = reinterpret_cast<float*>(take(sizeof(float) * BH * w.C3 * PS));
     w.khist = reinterpret_cast<int*>(take(sizeof(int) * (size_t)MAX_GRID * w.HB));
   }

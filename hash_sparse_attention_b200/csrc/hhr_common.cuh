@@ -20,12 +20,11 @@ struct Dims {
 };
 
 // Workspace carve-out of one decode step (device pointers).  The per-unit
-// counters `gx` and the kept-row list `sel_keys` are zero between calls (the
-// kernels reset what they use); everything else is overwritten by every call.
+// counters `gx` are zero between calls (the kernels reset what they use);
+// everything else is overwritten by every call.
 struct Work {
-  float* U;            // [B Hkv, Ustride] page bounds (max over the group's query heads)
-  int* sel_keys;       // [B Hkv, Kmax] kept-row list: row + 1 while published, read and cleared
-  float* part;         // [B Hkv, C3, G D + 16] softmax partials (gather chunks, or dense splits)
+  float* U;            // [B Hkv, Ustride] page bounds (aggregated over the group's query heads)
+  float* part;         // [B Hkv, C3, G D + 16] softmax partials (CTAs of a unit's group, or dense splits)
   int* khist;          // [grid, HB] score histogram of every CTA
   unsigned* gx;        // [B Hkv, gx_stride] per-unit barrier and arrival counters
   int Nmax, Kmax;      // budgets the workspace was sized for

@@ -8,35 +8,35 @@
 // keeps the top-k, then exact attention runs over the kept keys.
 //
 // Per unit, CTA r of the group:
-//   1. issues cp.async copies of its share of the page metadata (pages
-//      [p0, p1), 64 pages per stage, five stages in flight), then computes
-//      q' = R_h q and the query sign codes (every CTA of the group; R_h and
-//      W_h of the first unit are loaded before the previous kernel on the
-//      stream has finished: programmatic dependent launch);
-//   2. scans its pages: U = max over the group's query heads of the page
-//      bound.  Every thread consumes exactly the 16-byte pieces it copied, so
-//      the scan needs no CTA barrier;
-//   3. group barrier; the page top-N on ALL the unit's bounds (read from L2),
-//      the same in every CTA: a radix select on order-preserving keys, 11
-//      bits per level starting from the keys' range, equal keys taken in page
-//      order (ties go to the lower page);
+//   1. copies the query heads and the first two of its 64-page metadata
+//      stages (cp.async; pages [p0, p1), five stages in flight), then computes
+//      q' = R_h q and the query sign codes on tensor cores (R_h and W_h of the
+//      first unit are copied to shared memory before the previous kernel on
+//      the stream has finished: programmatic dependent launch);
+//   2. scans its pages: U = the page bound aggregated over the group's query
+//      heads (max, or sum).  Every thread consumes exactly the 16-byte pieces
+//      it copied, so the scan needs no CTA barrier;
+//   3. group barrier; the page top-N on ALL the unit's bounds (read from
+//      L2), the same in every CTA: order-preserving keys in registers, a level
+//      over the keys' range, then the threshold bin's members refined 11 bits
+//      at a time; equal keys are taken in page order (ties go to the lower
+//      page);
 //   4. when the key budget covers every candidate row, starts copying the K'/V
-//      rows of its first gather chunks right away (the key select below then
-//      keeps them all); scores its balanced share of the candidate rows
-//      (Hamming distance summed over the group's heads, code words loaded
-//      straight into registers) and publishes the score histogram;
-//   5. group barrier; the S histograms give the threshold score T, the ties
-//      taken at T and the CTA's place in the unit's kept-row list; it writes
-//      its kept rows there (row + 1, polled by the readers) unless every
-//      candidate is kept (then the list is implied by the kept pages);
-//   6. gathers the K'/V rows of its share of the list's 128-row chunks
-//      (cp.async, XOR-swizzled rows, three chunks in flight) and computes each
-//      chunk's softmax partial on tensor cores (mma.sync: logits with q' as
-//      bf16 hi + lo, P.V with P as bf16 hi + lo);
-//   7. the last CTA of the group to arrive merges the chunk partials in chunk
-//      order into the output and resets the unit's counters.
-// A chunk's partial depends only on its rows and the merge order is fixed, so
-// results do not depend on S, on the batch or on the cache layout.
+//      rows of its gather share right away; scores its balanced share of the
+//      candidate rows (Hamming distance over the group's heads, summed or
+//      minimised) and publishes the score histogram;
+//   5. group barrier; the S histograms give the threshold score T and the
+//      ties taken at T (lower rows first); the CTA lists the kept rows of its
+//      own scoring share, which it then gathers (with every candidate kept,
+//      its balanced share of all candidates instead);
+//   6. eight warps gather 16-row K'/V tiles (cp.async, XOR-swizzled rows, a
+//      ring of three per warp) and run an online softmax on tensor cores
+//      (mma.sync: logits with q' as bf16 hi + lo, P.V with P as bf16 hi + lo);
+//      their partials are combined in warp order into the CTA's partial;
+//   7. the last CTA of the group to arrive merges the S partials in CTA order
+//      into the output and resets the unit's counters.
+// Every order is fixed by the launch shape, so results are deterministic for
+// a given S (they do not depend on the batch or on the cache layout).
 #pragma once
 
 #include <algorithm>
@@ -51,28 +51,35 @@ constexpr int SP_WARPS = SP_THREADS / 32;
 constexpr int SP_STAGE_PAGES = 64;                   // pages per metadata stage
 constexpr int SP_META_STAGE = SP_STAGE_PAGES * 512;  // 64 rows of minima, then 64 rows of maxima
 constexpr int SP_NST = 5;                            // metadata stages in flight
-constexpr int SP_ROWS = 128;                         // rows per gather chunk
-constexpr int SP_GSTAGE = SP_ROWS * 512;             // 128 K' rows, then 128 V rows
-constexpr int SP_NGS = 3;                            // gather chunks in flight
 
-// shared memory map (bytes).  Region A is reused by every phase.
-constexpr int SP_A_BYTES = SP_NGS * SP_GSTAGE;                // 192 KB
-constexpr int SP_PREP = SP_NST * SP_META_STAGE;               // q, q' (prep) and the page-select histograms
-constexpr int SP_PSH = SP_PREP + 8192;                        // int [2][2048] page-select histograms
-constexpr int SP_HISTS = 2 * SP_GSTAGE;                       // key select: S score histograms, then scores
+// shared memory map (bytes).  Region A is reused by every phase:
+//   prep     metadata stages 0-1 [0, 64K), R_h fp32 [64K, 128K), W_h bf16 [128K, 192K)
+//   scan     five metadata stages [0, 160K)
+//   psel     two refinement lists [0, 128K), histogram [128K, 136K), kept-page bitmap [136K, 137K)
+//   keys     tile slots 0-1 of the gathering warps [0, 128K) (copies started early when every
+//            candidate is kept), score histograms and scores [128K, 192K)
+//   gather   the warps' tile rings [0, 192K);  combine, merge: partials
+constexpr int SP_A_BYTES = 192 * 1024;                        // region A
+constexpr int SP_RS = 2 * SP_META_STAGE;                      // R_h during the prep (64 KB)
+constexpr int SP_WS = SP_RS + D * D * 4;                      // W_h during the prep (<= 64 KB)
+constexpr int SP_PLIST = MAX_SELECT_PAGES * 8;              // page select: one refinement list (keys, pages)
+constexpr int SP_PSH = 2 * SP_PLIST;                          // int [2048] page-select histogram
+constexpr int SP_BITS = SP_PSH + 2048 * 4;                    // u32 [256] kept-page bitmap
+constexpr int SP_HISTS = 128 * 1024;                          // key select: S score histograms, then scores
 constexpr int SP_QB = SP_A_BYTES;                             // bf16 [16][136] q' operand (hi, lo)
-constexpr int SP_PB = SP_QB + 16 * 272;                       // bf16 [16][136] P operand (hi, lo)
-constexpr int SP_MX = SP_PB + 16 * 272;                       // float [8 warps][8 heads] row-block maxima
-constexpr int SP_LS = SP_MX + 256;                            // float [8][8] row-block weight sums
-constexpr int SP_OB = SP_LS + 256;                            // float [128 ch][16 cols] P.V of a chunk
-constexpr int SP_KP = SP_OB + 128 * 16 * 4;                   // int [MAX_KEEP_PAGES] kept pages
+constexpr int SP_KLCAP = MAX_KEPT_PER_CTA;                    // kept rows a CTA gathers at most (see sparse_group_shape)
+constexpr int SP_OB = SP_QB + 16 * 272;                       // prep: q, q' (fp32 [2][8][128]); keys/gather: kept list
+                                                              // (u16 [SP_KLCAP]); merge: weights
+constexpr int SP_LS = SP_OB + 2 * SP_KLCAP;                   // float [8] merge: 1 / total weight
+constexpr int SP_KP = SP_LS + 256;                            // int [MAX_KEEP_PAGES] kept pages
 constexpr int SP_QC = SP_KP + MAX_KEEP_PAGES * 4;             // u32 [8 heads][8] query codes
 constexpr int SP_RED = SP_QC + 256;                           // int: [0,64) scans, [64,128) min/max, [128,160) broadcasts
 constexpr int SP_MISC = SP_RED + 640;                         // int [32] flags
 constexpr int SP_SMEM = SP_MISC + 128;
+static_assert(2 * SP_KLCAP >= 8192, "q and q' of the prep, merge weights");
 static_assert(SP_SMEM <= 232448, "shared memory of the decode kernel");
-static_assert(SP_PSH + 2 * 2048 * 4 <= SP_A_BYTES, "page-select scratch");
-static_assert(SP_PREP >= 2 * SP_GSTAGE, "page-select scratch must not overlap the first two gather stages");
+static_assert(SP_WS + 256 * D * 2 <= SP_A_BYTES, "prep scratch");
+static_assert(SP_BITS + 256 * 4 <= SP_A_BYTES, "page-select scratch");
 
 // misc flags
 enum : int { MS_ABORT = 0, MS_LAST = 1 };
@@ -124,21 +131,25 @@ __device__ __forceinline__ void sp_abort(const SpParams& p, unsigned char* sm, i
 // Group barrier: every write made before it by any thread of the group's S
 // CTAs is visible after it (read such data with .cg loads: L1 is not
 // coherent).  A release add and a bounded acquire poll on the unit's counter.
-// False after a timeout or an abort (every thread of the CTA sees the same).
-__device__ __forceinline__ bool sp_group_sync(const SpParams& p, unsigned char* sm, unsigned* gx, unsigned& epoch) {
+// Split in two: between sp_group_arrive and sp_group_wait the CTA may do work
+// that the barrier does not need to cover.  sp_group_wait is false after a
+// timeout or an abort (every thread of the CTA sees the same).
+__device__ __forceinline__ void sp_group_arrive(const SpParams& p, unsigned* gx, unsigned& epoch) {
   __syncthreads();
   if (p.gsize > 1) {
     epoch += (unsigned)p.gsize;
-    if (threadIdx.x == 0) {
-      red_release_add(gx + GX_BAR, 1u);
-      if (ld_acquire(gx + GX_BAR) < epoch) {
-        Spin sp(p.wait_limit);
-        while (ld_acquire(gx + GX_BAR) < epoch) {
-          if (sp_aborted(sm)) break;
-          if (sp.expired()) {
-            sp_abort(p, sm, HHR_ERR_TIMEOUT);
-            break;
-          }
+    if (threadIdx.x == 0) red_release_add(gx + GX_BAR, 1u);
+  }
+}
+__device__ __forceinline__ bool sp_group_wait(const SpParams& p, unsigned char* sm, unsigned* gx, unsigned epoch) {
+  if (p.gsize > 1) {
+    if (threadIdx.x == 0 && ld_acquire(gx + GX_BAR) < epoch) {
+      Spin sp(p.wait_limit);
+      while (ld_acquire(gx + GX_BAR) < epoch) {
+        if (sp_aborted(sm)) break;
+        if (sp.expired()) {
+          sp_abort(p, sm, HHR_ERR_TIMEOUT);
+          break;
         }
       }
     }
@@ -146,152 +157,159 @@ __device__ __forceinline__ bool sp_group_sync(const SpParams& p, unsigned char* 
   }
   return !sp_aborted(sm);
 }
+__device__ __forceinline__ bool sp_group_sync(const SpParams& p, unsigned char* sm, unsigned* gx, unsigned& epoch) {
+  sp_group_arrive(p, gx, epoch);
+  return sp_group_wait(p, sm, gx, epoch);
+}
 
 // ---------------------------------------------------------------------------
 // prep: q' = R_h q and the query codes
 // ---------------------------------------------------------------------------
-// Warp w takes rows 8w .. 8w+7 of R_h and bits [w nb/16, (w+1) nb/16) of W_h
-// in blocks of NBB rows; lane l holds channels 4l .. 4l+3 of each row.
-template <int G>
-struct Prep {
-  static constexpr int GP = G <= 4 ? 4 : 8;  // heads padded to a power of two
-  static constexpr int NBB = 32 / GP;        // code bits per block
-  float4 rr[8];
-  uint2 wv[NBB];
-};
-
-template <int G, bool CODES = true>
-__device__ __forceinline__ void sp_prep_load(const SpParams& p, int h, Prep<G>& pr) {
-  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+// R_h (fp32) and W_h (bf16) are staged in shared memory with cp.async, their
+// 16-byte pieces XOR-swizzled by row (piece c of row i at c ^ (i mod 32) for
+// R, c ^ (i mod 16) for W) so that the fragment reads of a warp hit distinct
+// banks.  They are weights, never written by a decode step: the first unit's
+// are copied before the previous kernel on the stream has finished.  One
+// commit group.
+static __device__ __noinline__ void sp_issue_rw(const SpParams& p, unsigned char* sm, int h) {
   const float* Rh = p.R + (long long)h * D * D;
-#pragma unroll
-  for (int k = 0; k < 8; ++k) pr.rr[k] = __ldg(reinterpret_cast<const float4*>(Rh + (long long)(warp * 8 + k) * D) + lane);
-  if constexpr (CODES) {
-    const int bpw = p.dm.nb / SP_WARPS;
-    const __nv_bfloat16* Wh = p.W + (long long)h * p.dm.nb * D;
-#pragma unroll
-    for (int bb = 0; bb < Prep<G>::NBB; ++bb)
-      pr.wv[bb] = bb < bpw ? __ldg(reinterpret_cast<const uint2*>(Wh + (long long)(warp * bpw + bb) * D) + lane)
-                           : make_uint2(0u, 0u);
+  #pragma unroll 1
+  for (int q = threadIdx.x; q < D * 32; q += blockDim.x) {  // R: 128 rows x 32 pieces
+    const int i = q >> 5, c = q & 31;
+    cp_async16(sm + SP_RS + i * 512 + ((c ^ (i & 31)) * 16), Rh + i * D + c * 4);
   }
+  const __nv_bfloat16* Wh = p.W + (long long)h * p.dm.nb * D;
+  #pragma unroll 1
+  for (int q = threadIdx.x; q < p.dm.nb * 16; q += blockDim.x) {  // W: nb rows x 16 pieces
+    const int j = q >> 4, c = q & 15;
+    cp_async16(sm + SP_WS + j * 256 + ((c ^ (j & 15)) * 16), Wh + j * D + c * 8);
+  }
+  cp_async_commit();
 }
 
-// Writes q' (fp32, natural order) to qs [G][128], the hi/lo bf16 operand of the
-// logits (q' * sm_scale * log2 e) and the query codes (SP_QC).  The sign of a
-// code bit is exact: the fp32 sum is trusted when |sum| > 2^-14 sum|w q|,
-// otherwise it is recomputed in fp64.
-template <int G, bool CODES = true>
-__device__ void sp_prep(const SpParams& p, unsigned char* sm, const SpUnit& x, Prep<G>& pr, bool write_dbg) {
-  constexpr int GP = Prep<G>::GP, NBB = Prep<G>::NBB;
+// Copies the unit's query heads (bf16, G rows of 256 bytes) to rows 0..G-1 of
+// the [8][136] bf16 buffer at SP_OB (rows G..7 are zeroed by the caller).
+// One commit group.
+static __device__ __noinline__ void sp_issue_q(const SpParams& p, unsigned char* sm, const SpUnit& x, int G) {
+  const int tid = threadIdx.x;
+  if (tid < G * 16) {
+    const int g = tid >> 4, c = tid & 15;
+    cp_async16(sm + SP_OB + g * 272 + c * 16, p.q + ((long long)x.b * p.dm.Hq + x.h * G + g) * D + c * 8);
+  }
+  cp_async_commit();
+}
+
+// On tensor cores (mma.sync m16n8k16, bf16 in, fp32 accumulate), with the
+// query heads as the 8 columns of B (q is bf16: exact; heads >= G are zero):
+//   warps 0-7   q' = R_h q, rows 16w .. 16w+15: R_h as bf16 hi + lo (two
+//               products into one accumulator; |R - hi - lo| <= 2^-17 |R|).
+//               q' goes to qs (fp32 [8][128] at SP_OB + 4096) and the Q
+//               operand of the logits (q' * sm_scale * log2 e as bf16 hi in
+//               row g and lo in row 8 + g of SP_QB);
+//   warps 8-15  the query codes: bit j of head g is [(W_h q_g)_j > 0] for bit
+//               tiles m = w - 8 and w (rows 16 m .. +15, while < nb / 16); the
+//               products are exact and the fp32 sum is trusted when |sum| >
+//               2^-14 sum|w q| (a second product, of the magnitudes), else the
+//               sign comes from fp64.
+// The caller has issued sp_issue_rw and sp_issue_q, then two more commit groups.
+template <int G>
+__device__ void sp_prep(const SpParams& p, unsigned char* sm, const SpUnit& x, bool write_dbg) {
   const Dims& dm = p.dm;
-  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
-  float* qf = reinterpret_cast<float*>(sm + SP_PREP);         // [G][128] q
-  float* qs = reinterpret_cast<float*>(sm + SP_PREP + 4096);  // [G][128] q'
+  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5, g = lane >> 2, t = lane & 3;
+  float* qs = reinterpret_cast<float*>(sm + SP_OB + 4096);
   unsigned* qc = reinterpret_cast<unsigned*>(sm + SP_QC);
-  const __nv_bfloat16* qg = p.q + ((long long)x.b * dm.Hq + x.h * G) * D;
-  for (int i = tid; i < G * D; i += SP_THREADS) qf[i] = __bfloat162float(qg[i]);
+  // B fragments q[g][16 ks + 2t, +1] and q[g][16 ks + 8 + 2t, +1]
+  const uint32_t* qrow = reinterpret_cast<const uint32_t*>(sm + SP_OB + g * 272) + t;
   if (tid < 64) qc[tid] = 0u;
+  cp_async_wait<2>();  // R, W and q (issued before the unit's first two metadata stages)
   __syncthreads();
-  float qv[GP][4];
+  if (warp < 8) {
+    const int i0 = 16 * warp + g, i1 = i0 + 8;  // the lane's two rows of R_h
+    const unsigned char* R0 = sm + SP_RS + i0 * 512;
+    const unsigned char* R1 = sm + SP_RS + i1 * 512;
+    float c[4] = {0.f, 0.f, 0.f, 0.f};
+#pragma unroll 2
+    for (int ks = 0; ks < 8; ++ks) {
+      // A: R[i][16 ks + 2t, +1] and R[i][16 ks + 8 + 2t, +1] (piece 4 ks + t/2, +2; swizzled)
+      const int pa = 4 * ks + (t >> 1), off = 8 * (t & 1);
+      const float2 rr[4] = {*reinterpret_cast<const float2*>(R0 + ((pa ^ (i0 & 31)) * 16) + off),
+                            *reinterpret_cast<const float2*>(R1 + ((pa ^ (i1 & 31)) * 16) + off),
+                            *reinterpret_cast<const float2*>(R0 + (((pa + 2) ^ (i0 & 31)) * 16) + off),
+                            *reinterpret_cast<const float2*>(R1 + (((pa + 2) ^ (i1 & 31)) * 16) + off)};
+      uint32_t ah[4], al[4];
 #pragma unroll
-  for (int g = 0; g < GP; ++g) {
-    if (g < G) {
-      const float4 t = *reinterpret_cast<const float4*>(qf + g * D + 4 * lane);
-      qv[g][0] = t.x; qv[g][1] = t.y; qv[g][2] = t.z; qv[g][3] = t.w;
-    } else {
-      qv[g][0] = qv[g][1] = qv[g][2] = qv[g][3] = 0.f;
-    }
-  }
-  {
-    // q' rows 8w + k for every head: 8 GP dot products per lane, reduced over the warp
-    constexpr int NV = 8 * GP, KP = NV / 32;
-    float v[NV];
-#pragma unroll
-    for (int k = 0; k < 8; ++k)
-#pragma unroll
-      for (int g = 0; g < GP; ++g) {
-        const float4 a = pr.rr[k];
-        float s = a.x * qv[g][0];
-        s = fmaf(a.y, qv[g][1], s);
-        s = fmaf(a.z, qv[g][2], s);
-        v[k * GP + g] = fmaf(a.w, qv[g][3], s);
+      for (int e = 0; e < 4; ++e) {
+        const __nv_bfloat162 h = __floats2bfloat162_rn(rr[e].x, rr[e].y);
+        const float2 hf = __bfloat1622float2(h);
+        const __nv_bfloat162 l = __floats2bfloat162_rn(rr[e].x - hf.x, rr[e].y - hf.y);
+        ah[e] = *reinterpret_cast<const uint32_t*>(&h);
+        al[e] = *reinterpret_cast<const uint32_t*>(&l);
       }
-    group_reduce_scatter<NV, 32>(v, lane);
-#pragma unroll
-    for (int e = 0; e < KP; ++e) {
-      const int vi = KP * lane + e, k = vi / GP, g = vi % GP;
-      if (g < G) {
-        const int i = warp * 8 + k;
-        qs[g * D + i] = v[e];
-        if (write_dbg && p.dbg.q_rot) p.dbg.q_rot[((long long)x.b * dm.Hq + x.h * G + g) * D + i] = v[e];
-      }
+      const uint32_t b[2] = {qrow[8 * ks], qrow[8 * ks + 4]};
+      mma_bf16(c, ah, b);
+      mma_bf16(c, al, b);
     }
-  }
-  // query codes: warp w takes bits [w bpw, (w+1) bpw) in blocks of NBB
-  const int bpw = CODES ? dm.nb / SP_WARPS : 0;
-  const __nv_bfloat16* Wh = p.W + (long long)x.h * dm.nb * D;
-  // (lane: channels 4l .. 4l+3 of a W row as two bf16 pairs, loaded as uint2)
-  for (int jb = 0; jb < bpw; jb += NBB) {
-    if (jb > 0) {
-#pragma unroll
-      for (int bb = 0; bb < NBB; ++bb)
-        pr.wv[bb] = jb + bb < bpw ? __ldg(reinterpret_cast<const uint2*>(Wh + (long long)(warp * bpw + jb + bb) * D) + lane)
-                                  : make_uint2(0u, 0u);
-    }
-    float v[2 * NBB * GP];
-#pragma unroll
-    for (int bb = 0; bb < NBB; ++bb) {
-      const float w4[4] = {bf_lo(pr.wv[bb].x), bf_hi(pr.wv[bb].x), bf_lo(pr.wv[bb].y), bf_hi(pr.wv[bb].y)};
-#pragma unroll
-      for (int g = 0; g < GP; ++g) {
-        float a = 0.f, m = 0.f;
-#pragma unroll
-        for (int e = 0; e < 4; ++e) {
-          const float pe = w4[e] * qv[g][e];
-          a += pe;
-          m += fabsf(pe);
-        }
-        v[(bb * GP + g) * 2 + 0] = a;
-        v[(bb * GP + g) * 2 + 1] = m;
-      }
-    }
-    group_reduce_scatter<2 * NBB * GP, 32>(v, lane);
-    const int bb = lane / GP, g = lane % GP;
-    const int j = warp * bpw + jb + bb;
-    if (g < G && jb + bb < bpw) {
-      bool bit = v[0] > 0.f;
-      if (fabsf(v[0]) <= ldexpf(v[1], -14)) {
-        double ad = 0.0;
-        const __nv_bfloat16* wrow = Wh + (long long)j * D;
-        for (int c = 0; c < D; ++c) ad += (double)__bfloat162float(wrow[c]) * (double)qf[g * D + c];
-        bit = ad > 0.0;
-      }
-      if (bit) atomicOr(&qc[g * 8 + j / 32], 1u << (j % 32));
-    }
-  }
-  __syncthreads();
-  // the logits operand: q' * sm_scale * log2(e) as bf16 hi (columns 0..HP-1) + lo (HP..2HP-1)
-  {
-    constexpr int HP = G <= 4 ? 4 : 8;
+    // c0, c1: q'[2t][i0], q'[2t+1][i0]; c2, c3: the same at i1
     const float qscale = p.sm_scale * 1.4426950408889634f;
-    __nv_bfloat16* qb = reinterpret_cast<__nv_bfloat16*>(sm + SP_QB);
-    for (int e = tid; e < HP * D; e += SP_THREADS) {
-      const int hh = e / D, c = e - hh * D;
-      const float val = hh < G ? qs[hh * D + c] * qscale : 0.f;
+    __nv_bfloat16* qo = reinterpret_cast<__nv_bfloat16*>(sm + SP_QB);
+    float* dq = (write_dbg && p.dbg.q_rot) ? p.dbg.q_rot + ((long long)x.b * dm.Hq + x.h * G) * D : nullptr;
+#pragma unroll
+    for (int e = 0; e < 4; ++e) {
+      const int n = 2 * t + (e & 1), i = (e < 2) ? i0 : i1;
+      const float v = n < G ? c[e] : 0.f;
+      qs[n * D + i] = v;
       __nv_bfloat16 hi, lo;
-      split_bf16(val, hi, lo);
-      qb[hh * 136 + c] = hi;
-      qb[(HP + hh) * 136 + c] = lo;
+      split_bf16(v * qscale, hi, lo);
+      qo[n * 136 + i] = hi;
+      qo[(8 + n) * 136 + i] = lo;
+      if (dq && n < G) dq[n * D + i] = v;
+    }
+  } else {
+#pragma unroll 1
+    for (int m = warp - 8; m < (dm.nb >> 4); m += 8) {
+      float cs[4] = {0.f, 0.f, 0.f, 0.f}, cm[4] = {0.f, 0.f, 0.f, 0.f};
+      const int j = 16 * m + (lane & 15);  // the ldmatrix row of this lane
+      const unsigned char* Wj = sm + SP_WS + j * 256;
+#pragma unroll 2
+      for (int ks = 0; ks < 8; ++ks) {
+        uint32_t a[4];
+        ldsm_x4(a, Wj + (((2 * ks + (lane >> 4)) ^ (j & 15)) * 16));
+        const uint32_t am[4] = {a[0] & 0x7fff7fffu, a[1] & 0x7fff7fffu, a[2] & 0x7fff7fffu, a[3] & 0x7fff7fffu};
+        const uint32_t b[2] = {qrow[8 * ks], qrow[8 * ks + 4]};
+        const uint32_t bm[2] = {b[0] & 0x7fff7fffu, b[1] & 0x7fff7fffu};
+        mma_bf16(cs, a, b);
+        mma_bf16(cm, am, bm);
+      }
+      // cs[e]: bit row jj = 16 m + g (+8 for e >= 2), head n = 2t + (e & 1)
+#pragma unroll
+      for (int e = 0; e < 4; ++e) {
+        const int n = 2 * t + (e & 1), jj = 16 * m + g + (e >= 2 ? 8 : 0);
+        if (n >= G) continue;
+        bool bit = cs[e] > 0.f;
+        if (fabsf(cs[e]) <= ldexpf(cm[e], -14)) {  // too close to zero for fp32: the exact sign from fp64
+          const unsigned char* Wr = sm + SP_WS + jj * 256;
+          const __nv_bfloat16* qr = reinterpret_cast<const __nv_bfloat16*>(sm + SP_OB + n * 272);
+          double ad = 0.0;
+          #pragma unroll 1
+          for (int cc = 0; cc < D; ++cc) {
+            const int pc = ((cc >> 3) ^ (jj & 15)) * 8 + (cc & 7);
+            ad += (double)__bfloat162float(reinterpret_cast<const __nv_bfloat16*>(Wr)[pc]) *
+                  (double)__bfloat162float(qr[cc]);
+          }
+          bit = ad > 0.0;
+        }
+        if (bit) atomicOr(&qc[n * 8 + (jj >> 5)], 1u << (jj & 31));
+      }
     }
   }
-  if (CODES && write_dbg && p.dbg.q_codes) {
+  __syncthreads();
+  if (write_dbg && p.dbg.q_codes) {
     const int w32 = dm.words * 2;
     if (tid < G * w32) {
-      const int g = tid / w32, k = tid - g * w32;
-      reinterpret_cast<uint32_t*>(p.dbg.q_codes)[((long long)x.b * dm.Hq + x.h * G + g) * w32 + k] = qc[g * 8 + k];
+      const int gg = tid / w32, k = tid - gg * w32;
+      reinterpret_cast<uint32_t*>(p.dbg.q_codes)[((long long)x.b * dm.Hq + x.h * G + gg) * w32 + k] = qc[gg * 8 + k];
     }
   }
-  __syncthreads();
 }
 
 // ---------------------------------------------------------------------------
@@ -300,26 +318,28 @@ __device__ void sp_prep(const SpParams& p, unsigned char* sm, const SpUnit& x, P
 // Stage s holds pages p0 + 64 s + j (j < 64): minima rows at j*256, maxima at
 // 64*256 + j*256.  Thread t copies and later reads the 16-byte piece (t & 15)
 // (channels 8(t&15) .. +7) of pages j = t/16 and j = t/16 + 32, minima and maxima.
-__device__ __forceinline__ void sp_issue_meta(const SpParams& p, unsigned char* stage, const SpUnit& x, int pg0,
-                                              int p1) {
-  const int tid = threadIdx.x, li = tid & 15;
+static __device__ __noinline__ void sp_issue_meta(const SpParams& p, unsigned char* stage, const SpUnit& x, int pg0, int p1) {
+  if (pg0 < p1) {
+    const int tid = threadIdx.x, li = tid & 15;
 #pragma unroll
-  for (int half = 0; half < 2; ++half) {
-    const int j = (tid >> 4) + 32 * half;
-    const int pg = pg0 + j;
-    unsigned char* dmin = stage + j * 256 + li * 16;
-    // every thread issues both copies: a page past the share or with a bad
-    // block id (the status records it) reads as zeros
-    const long long off = pg < p1 ? meta_row(p.dm, p.table, x.b, x.h, pg, p.status) : -1;
-    const bool ok = off >= 0;
-    const long long e = ok ? off + li * 8 : 0;
-    const unsigned nbytes = ok ? 16u : 0u;
-    asm volatile("cp.async.cg.shared.global [%0], [%1], 16, %2;" ::"r"(smem_u32(dmin)), "l"(p.pmin + e), "r"(nbytes)
-                 : "memory");
-    asm volatile("cp.async.cg.shared.global [%0], [%1], 16, %2;" ::"r"(smem_u32(dmin + SP_STAGE_PAGES * 256)),
-                 "l"(p.pmax + e), "r"(nbytes)
-                 : "memory");
+    for (int half = 0; half < 2; ++half) {
+      const int j = (tid >> 4) + 32 * half;
+      const int pg = pg0 + j;
+      unsigned char* dmin = stage + j * 256 + li * 16;
+      // every thread issues both copies: a page past the share or with a bad
+      // block id (the status records it) reads as zeros
+      const long long off = pg < p1 ? meta_row(p.dm, p.table, x.b, x.h, pg, p.status) : -1;
+      const bool ok = off >= 0;
+      const long long e = ok ? off + li * 8 : 0;
+      const unsigned nbytes = ok ? 16u : 0u;
+      asm volatile("cp.async.cg.shared.global [%0], [%1], 16, %2;" ::"r"(smem_u32(dmin)), "l"(p.pmin + e), "r"(nbytes)
+                   : "memory");
+      asm volatile("cp.async.cg.shared.global [%0], [%1], 16, %2;" ::"r"(smem_u32(dmin + SP_STAGE_PAGES * 256)),
+                   "l"(p.pmax + e), "r"(nbytes)
+                   : "memory");
+    }
   }
+  cp_async_commit();
 }
 
 // Bounds of the (up to) 64 pages of one stage.  Half-warp hw = t/16 computes
@@ -404,361 +424,431 @@ __device__ __forceinline__ void sp_scan_stage(const SpParams& p, const unsigned 
 // ---------------------------------------------------------------------------
 // page top-N (larger bound first, ties to the lower page)
 // ---------------------------------------------------------------------------
-// Thread t holds pages [16t, 16t+16) of the unit as order-preserving keys (a
-// larger bound gives a larger key; -0 folds into +0).  Each level bins the
-// remaining candidates by (key - base) >> shift into at most 2048 bins, keeps
-// every bin above the one holding the need-th largest and descends into that
-// bin; the first level's shift comes from the keys' range, each next level
-// resolves 11 more bits, and a bin of one key value (shift 0) is taken in
-// page order.  Writes the kept pages (ascending) to SP_KP; returns their count.
-static __device__ int sp_psel(const SpParams& p, unsigned char* sm, const SpUnit& x, int N, bool write_dbg) {
+// Every CTA of the group runs the same select on the unit's bounds (read
+// from L2), so all of them know every kept page without another exchange.
+// Bounds become order-preserving keys (a larger bound gives a larger key; -0
+// folds into +0).  Thread t holds the keys of pages [16t, 16t + 16) in
+// registers (np <= 8192).  Level 0 bins them by (key - min) >> shift into at
+// most 2048 bins (shift from the keys' range), keeps every page above the bin
+// holding the N-th largest and, unless that bin is kept whole or holds one key
+// value, moves its members (in page order) to a list in shared memory, where
+// each further level resolves 11 more bits the same way.  A bin of one key
+// value is taken in page order (ties go to the lower page).  Writes the kept
+// pages (ascending) to SP_KP; returns their count.
+
+// One refinement level over the list at `lst` (cnt keys, then pages, in page
+// order), binned by (key - base) >> shift; marks the kept pages in `keep`.
+// Returns the number of bin members moved (in order) to `nxt` for the next
+// level, 0 when the select is complete.
+static __device__ __noinline__ int psel_level(unsigned char* sm, const unsigned char* lst, unsigned char* nxt, int cnt,
+                                              int& need, unsigned& base, int& shift, int par) {
+  const int tid = threadIdx.x;
+  int* red = reinterpret_cast<int*>(sm + SP_RED);
+  int* bc = red + 128;
+  int* hist = reinterpret_cast<int*>(sm + SP_PSH);
+  unsigned* keep = reinterpret_cast<unsigned*>(sm + SP_BITS);
+  const uint32_t* lk = reinterpret_cast<const uint32_t*>(lst);
+  const int* lp = reinterpret_cast<const int*>(lst + SP_PLIST / 2);
+  // thread t: list elements [t c, t c + c)
+  const int c = (cnt + SP_THREADS - 1) / SP_THREADS;
+  const int e0 = min(cnt, tid * c), e1 = min(cnt, e0 + c);
+  #pragma unroll 1
+  for (int e = e0; e < e1; ++e) atomicAdd(&hist[(lk[e] - base) >> shift], 1);
+  __syncthreads();
+  int hv[4], c4 = 0;
+#pragma unroll
+  for (int q = 0; q < 4; ++q) {
+    hv[q] = hist[2047 - 4 * tid - q];
+    c4 += hv[q];
+  }
+  int tot;
+  const int before = block_scan_excl(c4, red, par, &tot);
+  if (before < need && before + c4 >= need) {
+    int run = before;
+#pragma unroll
+    for (int q = 0; q < 4; ++q) {
+      if (run < need && run + hv[q] >= need) {
+        bc[0] = 2047 - 4 * tid - q;
+        bc[1] = need - run;
+        bc[2] = hv[q];
+      }
+      run += hv[q];
+    }
+  }
+  __syncthreads();
+  const int bstar = bc[0], need_in = bc[1], cnt_in = bc[2];
+  #pragma unroll 1
+  for (int i = tid; i < 512; i += SP_THREADS) hist[4 * i] = hist[4 * i + 1] = hist[4 * i + 2] = hist[4 * i + 3] = 0;
+  // members above the bin are kept; the bin's members are counted per thread
+  int nb = 0;
+  #pragma unroll 1
+  for (int e = e0; e < e1; ++e) {
+    const int bn = (int)((lk[e] - base) >> shift);
+    if (bn > bstar) atomicOr(&keep[lp[e] >> 5], 1u << (lp[e] & 31));
+    nb += bn == bstar;
+  }
+  const bool whole = cnt_in == need_in, ties = shift == 0;
+  int nt;
+  const int pre = block_scan_excl(nb, red, par + 1, &nt);  // (its barrier also orders the clears above)
+  int* nk = reinterpret_cast<int*>(nxt);
+  int* np2 = reinterpret_cast<int*>(nxt + SP_PLIST / 2);
+  int q = pre;
+  #pragma unroll 1
+  for (int e = e0; e < e1; ++e) {
+    if ((int)((lk[e] - base) >> shift) != bstar) continue;
+    if (whole || (ties && q < need_in)) {
+      atomicOr(&keep[lp[e] >> 5], 1u << (lp[e] & 31));
+    } else if (!ties) {
+      nk[q] = lk[e];
+      np2[q] = lp[e];
+    }
+    ++q;
+  }
+  __syncthreads();
+  if (whole || ties) return 0;
+  need = need_in;
+  base += (unsigned)bstar << shift;
+  shift = shift > 11 ? shift - 11 : 0;
+  return cnt_in;
+}
+
+static __device__ __noinline__ int sp_psel(const SpParams& p, unsigned char* sm, const SpUnit& x, int N, bool write_dbg) {
   const int tid = threadIdx.x;
   int* kp = reinterpret_cast<int*>(sm + SP_KP);
   int* red = reinterpret_cast<int*>(sm + SP_RED);
   int* bc = red + 128;
-  int* hist0 = reinterpret_cast<int*>(sm + SP_PSH);
-  const int np = x.np;
-  const int i0 = tid * 16;
-  const int cnt = max(0, min(16, np - i0));
-  unsigned member = cnt >= 16 ? 0xffffu : ((1u << cnt) - 1u);
-  unsigned keep = 0u;
-  int par = 0;  // scan-buffer parity
+  int* hist = reinterpret_cast<int*>(sm + SP_PSH);
+  unsigned* keep = reinterpret_cast<unsigned*>(sm + SP_BITS);
+  const int np = x.np, i0 = tid * 16;
+  const int nv = min(16, max(0, np - i0));  // the thread's pages
+  unsigned sel = 0u;                        // bit e: page i0 + e is kept
+  int par = 0;
   if (N >= np) {
-    keep = member;
+    sel = nv >= 16 ? 0xffffu : ((1u << nv) - 1u);
   } else {
-    uint32_t key[16];
-    const float* Ug = p.wk.U + (long long)x.u * p.wk.Ustride + i0;
+    // the thread's 16 bounds: four 16-byte loads, all in flight at once (a U
+    // row is padded to a multiple of 32 pages, so they stay inside it)
+    uint32_t k[16];
+    {
+      const float4* Ug = reinterpret_cast<const float4*>(p.wk.U + (long long)x.u * p.wk.Ustride + i0);
+      float4 v[4];
 #pragma unroll
-    for (int k4 = 0; k4 < 4; ++k4) {
-      float4 t = make_float4(0.f, 0.f, 0.f, 0.f);
-      if (i0 + 4 * k4 < np) t = __ldcg(reinterpret_cast<const float4*>(Ug) + k4);
-      key[4 * k4 + 0] = order_key(t.x);
-      key[4 * k4 + 1] = order_key(t.y);
-      key[4 * k4 + 2] = order_key(t.z);
-      key[4 * k4 + 3] = order_key(t.w);
+      for (int k4 = 0; k4 < 4; ++k4) v[k4] = i0 + 4 * k4 < np ? __ldcg(Ug + k4) : make_float4(0.f, 0.f, 0.f, 0.f);
+#pragma unroll
+      for (int k4 = 0; k4 < 4; ++k4) {
+        k[4 * k4] = order_key(v[k4].x);
+        k[4 * k4 + 1] = order_key(v[k4].y);
+        k[4 * k4 + 2] = order_key(v[k4].z);
+        k[4 * k4 + 3] = order_key(v[k4].w);
+      }
     }
-    for (int i = tid; i < 2 * 2048; i += SP_THREADS) hist0[i] = 0;
     unsigned lo = 0xffffffffu, hi = 0u;
 #pragma unroll
-    for (int k = 0; k < 16; ++k)
-      if ((member >> k) & 1u) {
-        lo = min(lo, key[k]);
-        hi = max(hi, key[k]);
+    for (int e = 0; e < 16; ++e)
+      if (e < nv) {
+        lo = min(lo, k[e]);
+        hi = max(hi, k[e]);
       }
-    block_minmax_u32(lo, hi, reinterpret_cast<unsigned*>(red + 64));  // (its barrier also orders the clears)
-    int need = N;
+    reinterpret_cast<int4*>(hist)[tid] = make_int4(0, 0, 0, 0);  // 2048 bins
+    if (tid < 256) keep[tid] = 0u;
+    block_minmax_u32(lo, hi, reinterpret_cast<unsigned*>(red + 64));  // (its barrier orders the clears)
     unsigned base = lo;
     const unsigned width = hi - lo;
     int shift = width < 2048u ? 0 : (32 - __clz(width)) - 11;
-#pragma unroll 1
-    for (int level = 0;; ++level) {
-      int* hist = hist0 + 2048 * (level & 1);
-      int* hnext = hist0 + 2048 * ((level + 1) & 1);
 #pragma unroll
-      for (int k = 0; k < 16; ++k)
-        if ((member >> k) & 1u) atomicAdd(&hist[(key[k] - base) >> shift], 1);
-      __syncthreads();
-      // thread t: bins 2047-4t .. 2044-4t, counted from the top
-      int hv[4], c4 = 0;
+    for (int e = 0; e < 16; ++e)
+      if (e < nv) atomicAdd(&hist[(k[e] - base) >> shift], 1);
+    __syncthreads();
+    int hv[4], c4 = 0;
 #pragma unroll
-      for (int e = 0; e < 4; ++e) {
-        hv[e] = hist[2047 - 4 * tid - e];
-        c4 += hv[e];
-      }
-      int tot;
-      const int before = block_scan_excl(c4, red, par++, &tot);
-      if (before < need && before + c4 >= need) {
-        int run = before;
+    for (int q = 0; q < 4; ++q) {
+      hv[q] = hist[2047 - 4 * tid - q];
+      c4 += hv[q];
+    }
+    int tot;
+    const int before = block_scan_excl(c4, red, par++, &tot);
+    if (before < N && before + c4 >= N) {
+      int run = before;
 #pragma unroll
-        for (int e = 0; e < 4; ++e) {
-          if (run < need && run + hv[e] >= need) {
-            bc[0] = 2047 - 4 * tid - e;
-            bc[1] = need - run;
-            bc[2] = hv[e];
-          }
-          run += hv[e];
+      for (int q = 0; q < 4; ++q) {
+        if (run < N && run + hv[q] >= N) {
+          bc[0] = 2047 - 4 * tid - q;
+          bc[1] = N - run;
+          bc[2] = hv[q];
         }
+        run += hv[q];
       }
-      for (int i = tid; i < 2048; i += SP_THREADS) hnext[i] = 0;
-      __syncthreads();
-      const int bstar = bc[0], need_in = bc[1], cnt_in = bc[2];
-      unsigned m2 = 0u;
+    }
+    __syncthreads();
+    const int bstar = bc[0], need_in = bc[1], cnt_in = bc[2];
+    reinterpret_cast<int4*>(hist)[tid] = make_int4(0, 0, 0, 0);
+    unsigned at = 0u;
 #pragma unroll
-      for (int k = 0; k < 16; ++k)
-        if ((member >> k) & 1u) {
-          const int bn = (int)((key[k] - base) >> shift);
-          if (bn > bstar) keep |= 1u << k;
-          else if (bn == bstar) m2 |= 1u << k;
+    for (int e = 0; e < 16; ++e)
+      if (e < nv) {
+        const int bn = (int)((k[e] - base) >> shift);
+        sel |= (unsigned)(bn > bstar) << e;
+        at |= (unsigned)(bn == bstar) << e;
+      }
+    if (cnt_in == need_in) {
+      sel |= at;
+    } else {
+      // the bin's members in page order: the first need_in when they are one
+      // key value, else the list of the next level
+      int nt;
+      const int pre = block_scan_excl(__popc(at), red, par++, &nt);
+      if (shift == 0) {
+        int take = max(0, min(__popc(at), need_in - pre));
+        unsigned t = at;
+        while (take-- > 0) {
+          sel |= t & (0u - t);
+          t &= t - 1u;
         }
-      member = m2;
-      need = need_in;
-      if (cnt_in == need_in) {  // the whole bin is kept
-        keep |= member;
-        break;
-      }
-      if (shift == 0) {  // one key value: equal bounds, the first `need` in page order
-        int tot2;
-        const int mb = block_scan_excl(__popc(member), red, par++, &tot2);
-        int take = max(0, min(__popc(member), need - mb));
+      } else {
+        uint32_t* lk = reinterpret_cast<uint32_t*>(sm);
+        int* lp = reinterpret_cast<int*>(sm + SP_PLIST / 2);
+        int q = pre;
 #pragma unroll
-        for (int k = 0; k < 16; ++k)
-          if (((member >> k) & 1u) && take > 0) {
-            keep |= 1u << k;
-            --take;
+        for (int e = 0; e < 16; ++e)
+          if ((at >> e) & 1u) {
+            lk[q] = k[e];
+            lp[q] = i0 + e;
+            ++q;
           }
-        break;
+        __syncthreads();
+        int need = need_in, cnt = cnt_in;
+        base += (unsigned)bstar << shift;
+        shift = shift > 11 ? shift - 11 : 0;
+        #pragma unroll 1
+        for (int lv = 0; cnt > 0; ++lv)
+          cnt = psel_level(sm, sm + (lv & 1) * SP_PLIST, sm + ((lv + 1) & 1) * SP_PLIST, cnt, need, base, shift, 2 * lv + 2);
+        // (psel_level ends with a barrier: the keep bitmap is complete)
+        sel |= (keep[i0 >> 5] >> (i0 & 16)) & 0xffffu;
       }
-      base += (unsigned)bstar << shift;
-      shift = shift > 11 ? shift - 11 : 0;
     }
   }
+  // kept pages in ascending order
   int nkp;
-  int pos = block_scan_excl(__popc(keep), red, par++, &nkp);
+  int pos = block_scan_excl(__popc(sel), red, par & 1, &nkp);
   int* dsel = (write_dbg && p.dbg.sel_pages) ? p.dbg.sel_pages + (long long)x.u * p.wk.Nmax : nullptr;
-#pragma unroll
-  for (int k = 0; k < 16; ++k)
-    if (((keep >> k) & 1u) && pos < MAX_KEEP_PAGES) {
-      kp[pos] = i0 + k;
-      if (dsel) dsel[pos] = i0 + k;
-      ++pos;
+  unsigned t = sel;
+  while (t) {
+    const int pg = i0 + __ffs(t) - 1;
+    t &= t - 1u;
+    if (pos < MAX_KEEP_PAGES) {
+      kp[pos] = pg;
+      if (dsel) dsel[pos] = pg;
     }
+    ++pos;
+  }
   if (write_dbg && tid == 0 && p.dbg.n_sel_pages) p.dbg.n_sel_pages[x.u] = nkp;
   __syncthreads();
   return nkp;
 }
 
 // ---------------------------------------------------------------------------
-// gather: K'/V rows of a 128-row chunk, then its softmax partial
+// attention over 16-row tiles (the gather of the decode step and the dense
+// kernel): eight warps work independently, each streaming its tiles through a
+// ring of three in shared memory, with its online-softmax state in registers
 // ---------------------------------------------------------------------------
-// Row j of the chunk, 16-byte piece c: K' at stage + j*256 + ((c ^ (j & 7)) * 16),
-// V 32 KB further (eight consecutive rows' same piece fall in distinct banks
-// for ldmatrix).  Warp w copies rows 8w .. 8w+7; lane l < 8 resolves row 8w + l
-// (its element offset / 128, or -1 for a row past the chunk or a bad row).
-__device__ __forceinline__ void sp_copy_rows(const SpParams& p, unsigned char* stage, int rowidx) {
-  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
-  const int c = lane & 15;
+constexpr int TL_ROWS = 16;
+constexpr int TL_BYTES = TL_ROWS * 512;  // 16 K' rows, then 16 V rows
+constexpr int TL_WARPS = 8;
+constexpr int TL_NBUF = 3;
+static_assert(TL_NBUF * TL_WARPS * TL_BYTES == SP_A_BYTES, "tile rings fill region A");
+
+// Slot s of warp w: the three slots of all warps are interleaved so that
+// slots 0 and 1 of every warp lie in [0, 128K) and slot 2 in [128K, 192K).
+__device__ __forceinline__ unsigned char* tile_slot(unsigned char* sm, int warp, int s) {
+  return sm + (s * TL_WARPS + warp) * TL_BYTES;
+}
+
+// Copies one tile: lane l < 16 passes rowidx = element offset / 128 of the
+// tile's row l (or -1: past the end, or a bad row, which then reads as zeros).
+// Piece c of row j goes to piece c ^ (j mod 8) of its 256-byte row, so that
+// eight consecutive rows' same piece fall in distinct banks for ldmatrix.
+// One commit group per lane.
+__device__ __forceinline__ void tile_copy(const __nv_bfloat16* K, const __nv_bfloat16* V, unsigned char* slot,
+                                          int rowidx, bool live) {
+  const int lane = threadIdx.x & 31;
+  if (live) {
+#pragma unroll 1
+    for (int i = 0; i < 8; ++i) {
+      const int q = lane + 32 * i, j = q >> 4, c = q & 15;
+      const int ri = __shfl_sync(0xffffffffu, rowidx, j);
+      const long long e = ri >= 0 ? (long long)ri * D + c * 8 : 0;
+      const unsigned nbytes = ri >= 0 ? 16u : 0u;
+      unsigned char* dk = slot + j * 256 + ((c ^ (j & 7)) * 16);
+      asm volatile("cp.async.cg.shared.global [%0], [%1], 16, %2;" ::"r"(smem_u32(dk)), "l"(K + e), "r"(nbytes)
+                   : "memory");
+      asm volatile("cp.async.cg.shared.global [%0], [%1], 16, %2;" ::"r"(smem_u32(dk + TL_ROWS * 256)), "l"(V + e),
+                   "r"(nbytes)
+                   : "memory");
+    }
+  }
+  cp_async_commit();
+}
+
+// The Q operand of the logits (all eight k-steps) from the [16][136] bf16
+// layout at qb: head g's q' * sm_scale * log2 e, hi in row g, lo in row 8 + g.
+__device__ __forceinline__ void load_q_operand(const unsigned char* qb, uint32_t (&aq)[8][4]) {
+  const int lane = threadIdx.x & 31;
 #pragma unroll
-  for (int i = 0; i < 4; ++i) {
-    const int jl = 2 * i + (lane >> 4);
-    const int j = warp * 8 + jl;
-    const int ri = __shfl_sync(0xffffffffu, rowidx, jl);
-    unsigned char* dk = stage + j * 256 + ((c ^ (j & 7)) * 16);
-    // a row past the chunk or a bad row reads as zeros (the tensor-core products stay finite)
-    const long long e = ri >= 0 ? (long long)ri * D + c * 8 : 0;
-    const unsigned nbytes = ri >= 0 ? 16u : 0u;
-    asm volatile("cp.async.cg.shared.global [%0], [%1], 16, %2;" ::"r"(smem_u32(dk)), "l"(p.Kr + e), "r"(nbytes)
-                 : "memory");
-    asm volatile("cp.async.cg.shared.global [%0], [%1], 16, %2;" ::"r"(smem_u32(dk + SP_ROWS * 256)),
-                 "l"(p.Vc + e), "r"(nbytes)
-                 : "memory");
+  for (int ks = 0; ks < 8; ++ks)
+    ldsm_x4(aq[ks], qb + ((lane & 7) + ((lane >> 3) & 1) * 8) * 272 + (2 * ks + (lane >> 4)) * 16);
+}
+
+__device__ __forceinline__ uint32_t pack_bf16(float a, float b) {
+  const __nv_bfloat162 v = __floats2bfloat162_rn(a, b);
+  return *reinterpret_cast<const uint32_t*>(&v);
+}
+
+// One tile of `rows` (1..16) valid rows: on tensor cores (mma.sync m16n8k16,
+// bf16 in, fp32 accumulate) S = Q K'^T, where the 16 rows of Q are the heads'
+// hi and lo parts, so head g = lane / 4's logit is the sum of two rows held by
+// the same lane; the online softmax of head g in registers; then
+// O += P V, with P's hi and lo parts as the 16 rows of the A operand, built
+// from the lane's own logits.  O[nt] holds channels 8 nt + 2 (lane mod 4), +1
+// of head g: rows 0 (hi) and 2 (lo) of the accumulator, summed at the end.
+__device__ __forceinline__ void tile_attend(const uint32_t (&aq)[8][4], float (&o)[16][4], float& m_run,
+                                            float& l_run, const unsigned char* kt, int rows) {
+  const int lane = threadIdx.x & 31, t = lane & 3;
+  const unsigned char* vt = kt + TL_ROWS * 256;
+  float s0[4] = {0.f, 0.f, 0.f, 0.f}, s1[4] = {0.f, 0.f, 0.f, 0.f};
+  {
+    const int krow = (lane & 7) + 8 * (lane >> 4);  // matrices 0,1: rows 0-7; 2,3: rows 8-15
+    const int kp = (lane >> 3) & 1;                 // matrices 1,3: channels + 8
+#pragma unroll
+    for (int ks = 0; ks < 8; ++ks) {
+      uint32_t b[4];
+      ldsm_x4(b, kt + krow * 256 + (((2 * ks + kp) ^ (krow & 7)) * 16));
+      const uint32_t b0[2] = {b[0], b[1]}, b1[2] = {b[2], b[3]};
+      mma_bf16(s0, aq[ks], b0);
+      mma_bf16(s1, aq[ks], b1);
+    }
+  }
+  float sv[4] = {s0[0] + s0[2], s0[1] + s0[3], s1[0] + s1[2], s1[1] + s1[3]};  // rows 2t, 2t+1, 8+2t, 9+2t
+  if (2 * t >= rows) sv[0] = -INFINITY;
+  if (2 * t + 1 >= rows) sv[1] = -INFINITY;
+  if (8 + 2 * t >= rows) sv[2] = -INFINITY;
+  if (9 + 2 * t >= rows) sv[3] = -INFINITY;
+  float mt = fmaxf(fmaxf(sv[0], sv[1]), fmaxf(sv[2], sv[3]));
+  mt = fmaxf(mt, __shfl_xor_sync(0xffffffffu, mt, 1));
+  mt = fmaxf(mt, __shfl_xor_sync(0xffffffffu, mt, 2));
+  const float mn = fmaxf(m_run, mt);  // finite: row 0 of a tile is always valid
+  const float alpha = exp2f(m_run - mn);
+  float pw[4];
+#pragma unroll
+  for (int e = 0; e < 4; ++e) pw[e] = exp2f(sv[e] - mn);
+  l_run = l_run * alpha + ((pw[0] + pw[1]) + (pw[2] + pw[3]));
+  m_run = mn;
+  if (__any_sync(0xffffffffu, alpha != 1.f)) {  // (no head's maximum moved: nothing to rescale)
+#pragma unroll
+    for (int nt = 0; nt < 16; ++nt) {
+      o[nt][0] *= alpha;
+      o[nt][1] *= alpha;
+      o[nt][2] *= alpha;
+      o[nt][3] *= alpha;
+    }
+  }
+  uint32_t ap[4];
+  {
+    const float h0 = __bfloat162float(__float2bfloat16_rn(pw[0])), h1 = __bfloat162float(__float2bfloat16_rn(pw[1]));
+    const float h2 = __bfloat162float(__float2bfloat16_rn(pw[2])), h3 = __bfloat162float(__float2bfloat16_rn(pw[3]));
+    ap[0] = pack_bf16(h0, h1);
+    ap[1] = pack_bf16(pw[0] - h0, pw[1] - h1);
+    ap[2] = pack_bf16(h2, h3);
+    ap[3] = pack_bf16(pw[2] - h2, pw[3] - h3);
+  }
+  {
+    const int vrow = (lane & 7) + 8 * ((lane >> 3) & 1);  // matrices 1,3: rows 8-15
+    const int vp = lane >> 4;                             // matrices 2,3: channels + 8
+#pragma unroll
+    for (int cp = 0; cp < 8; ++cp) {
+      uint32_t b[4];
+      ldsm_x4_t(b, vt + vrow * 256 + (((2 * cp + vp) ^ (vrow & 7)) * 16));
+      const uint32_t b0[2] = {b[0], b[1]}, b1[2] = {b[2], b[3]};
+      mma_bf16(o[2 * cp], ap, b0);
+      mma_bf16(o[2 * cp + 1], ap, b1);
+    }
   }
 }
 
-// Column layout of the two mma operands: NT = 1 (G <= 4): columns 0-3 the
-// heads' hi parts, 4-7 their lo parts; NT = 2 (G <= 8): 0-7 hi, 8-15 lo.
+// The gathering warps' partials (head g: max, sum, O) combined in warp order
+// into `part` (G*128 outputs, then per head the max and the sum of weights, in
+// log2 units).  Region A is the scratch; every thread of the CTA calls it.
 template <int G>
-struct GCols {
-  static constexpr int NT = G <= 4 ? 1 : 2;
-  static constexpr int HP = 4 * NT;
-  __device__ static int hi(int h) { return h; }
-  __device__ static int lo(int h) { return HP + h; }
-};
-
-// One chunk of up to 128 kept rows: logits S = K' (q' hi + lo)^T on tensor
-// cores (warps 0-7, 16 rows each), the chunk's maximum and weights per head in
-// fp32, then O^T = V^T (P hi + lo)^T (warps 0-7, 16 channels each over all 128
-// rows).  The partial (unnormalised output, then per head the maximum and the
-// sum of weights, in log2 units) goes to `part`; it depends only on the rows.
-template <int G>
-__device__ void sp_gather_step(unsigned char* sm, const unsigned char* stage, int n, float* part) {
-  using C = GCols<G>;
-  constexpr int NT = C::NT;
-  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
-  const int g = lane >> 2, t = lane & 3;
-  const unsigned char* qb = sm + SP_QB;
-  __nv_bfloat16* pb = reinterpret_cast<__nv_bfloat16*>(sm + SP_PB);
-  float* mx = reinterpret_cast<float*>(sm + SP_MX);
-  float* ls = reinterpret_cast<float*>(sm + SP_LS);
-  float* ob = reinterpret_cast<float*>(sm + SP_OB);
-  float sv[2][2];
-  int h0 = 0;
-  if (warp < 8) {
-    float acc[NT][4];
+__device__ void tile_combine(unsigned char* sm, const float (&o)[16][4], float m_run, float l_run, bool had, float* part,
+                             bool write) {
+  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5, g = lane >> 2, t = lane & 3;
+  constexpr int WS = D + 2;
+  float* wsm = reinterpret_cast<float*>(sm);  // [8 warps][8 heads][130]
+  __syncthreads();  // every warp is done with its ring
+  if (warp < TL_WARPS) {
+    float l4 = l_run;
+    l4 += __shfl_xor_sync(0xffffffffu, l4, 1);
+    l4 += __shfl_xor_sync(0xffffffffu, l4, 2);
+    float* wr = wsm + (warp * 8 + g) * WS;
 #pragma unroll
-    for (int nt = 0; nt < NT; ++nt) acc[nt][0] = acc[nt][1] = acc[nt][2] = acc[nt][3] = 0.f;
-    const int r0 = warp * 16;
-    const int arow = r0 + (lane & 7) + ((lane >> 3) & 1) * 8;
-    const unsigned char* krow = stage + arow * 256;
-#pragma unroll
-    for (int ks = 0; ks < 8; ++ks) {
-      uint32_t af[4];
-      ldsm_x4(af, krow + (((2 * ks + (lane >> 4)) ^ (arow & 7)) * 16));
-#pragma unroll
-      for (int nt = 0; nt < NT; ++nt) {
-        uint32_t bf[2];
-        ldsm_x2(bf, qb + (nt * 8 + (lane & 7)) * 272 + (2 * ks + ((lane >> 3) & 1)) * 16);
-        mma_bf16(acc[nt], af, bf);
-      }
+    for (int nt = 0; nt < 16; ++nt) {
+      wr[8 * nt + 2 * t] = o[nt][0] + o[nt][2];
+      wr[8 * nt + 2 * t + 1] = o[nt][1] + o[nt][3];
     }
-    // hi + lo of the same heads: NT = 1 pairs columns 2t, 2t+1 with 2t+4, 2t+5
-    // (lane t ^ 2); NT = 2 holds them in its two n-tiles
-    float v0 = acc[0][0], v1 = acc[0][1], v2 = acc[0][2], v3 = acc[0][3];
-    if constexpr (NT == 1) {
-      v0 += __shfl_xor_sync(0xffffffffu, v0, 2);
-      v1 += __shfl_xor_sync(0xffffffffu, v1, 2);
-      v2 += __shfl_xor_sync(0xffffffffu, v2, 2);
-      v3 += __shfl_xor_sync(0xffffffffu, v3, 2);
-      h0 = 2 * (t & 1);
-    } else {
-      v0 += acc[NT - 1][0];
-      v1 += acc[NT - 1][1];
-      v2 += acc[NT - 1][2];
-      v3 += acc[NT - 1][3];
-      h0 = 2 * t;
-    }
-    const bool rg = r0 + g < n, rg8 = r0 + g + 8 < n;
-    sv[0][0] = (rg && h0 < G) ? v0 : -INFINITY;
-    sv[0][1] = (rg && h0 + 1 < G) ? v1 : -INFINITY;
-    sv[1][0] = (rg8 && h0 < G) ? v2 : -INFINITY;
-    sv[1][1] = (rg8 && h0 + 1 < G) ? v3 : -INFINITY;
-    float m0 = fmaxf(sv[0][0], sv[1][0]), m1 = fmaxf(sv[0][1], sv[1][1]);
-#pragma unroll
-    for (int o = 4; o < 32; o <<= 1) {
-      m0 = fmaxf(m0, __shfl_xor_sync(0xffffffffu, m0, o));
-      m1 = fmaxf(m1, __shfl_xor_sync(0xffffffffu, m1, o));
-    }
-    if (g == 0 && (NT == 2 || t < 2)) {
-      mx[warp * 8 + h0] = m0;
-      mx[warp * 8 + h0 + 1] = m1;
+    if (t == 0) {
+      wr[D] = had ? m_run : -INFINITY;
+      wr[D + 1] = had ? l4 : 0.f;
     }
   }
   __syncthreads();
-  if (warp < 8) {
-    const int r0 = warp * 16;
-    float M0 = -INFINITY, M1 = -INFINITY;
+  if (write) {
+#pragma unroll 1
+    for (int e = tid; e < G * D; e += blockDim.x) {
+      const int hh = e >> 7, c = e & (D - 1);
+      float M = -INFINITY;
 #pragma unroll
-    for (int w2 = 0; w2 < 8; ++w2) {
-      M0 = fmaxf(M0, mx[w2 * 8 + h0]);
-      M1 = fmaxf(M1, mx[w2 * 8 + h0 + 1]);
-    }
-    float pw[2][2];
+      for (int w = 0; w < TL_WARPS; ++w) M = fmaxf(M, wsm[(w * 8 + hh) * WS + D]);
+      float acc = 0.f, Ls = 0.f;
+      if (M != -INFINITY) {
 #pragma unroll
-    for (int rr = 0; rr < 2; ++rr) {
-      pw[rr][0] = sv[rr][0] == -INFINITY ? 0.f : exp2f(sv[rr][0] - M0);
-      pw[rr][1] = sv[rr][1] == -INFINITY ? 0.f : exp2f(sv[rr][1] - M1);
-    }
-    float l0 = pw[0][0] + pw[1][0], l1 = pw[0][1] + pw[1][1];
-#pragma unroll
-    for (int o = 4; o < 32; o <<= 1) {
-      l0 += __shfl_xor_sync(0xffffffffu, l0, o);
-      l1 += __shfl_xor_sync(0xffffffffu, l1, o);
-    }
-    if (NT == 2 || t < 2) {
-      if (g == 0) {
-        ls[warp * 8 + h0] = l0;
-        ls[warp * 8 + h0 + 1] = l1;
-      }
-#pragma unroll
-      for (int rr = 0; rr < 2; ++rr) {
-        const int row = r0 + g + 8 * rr;
-#pragma unroll
-        for (int e = 0; e < 2; ++e) {
-          __nv_bfloat16 hi, lo;
-          split_bf16(pw[rr][e], hi, lo);
-          pb[C::hi(h0 + e) * 136 + row] = hi;
-          pb[C::lo(h0 + e) * 136 + row] = lo;
+        for (int w = 0; w < TL_WARPS; ++w) {
+          const float* wr = wsm + (w * 8 + hh) * WS;
+          const float sc = exp2f(wr[D] - M);  // 0 for a warp without rows
+          acc = fmaf(sc, wr[c], acc);
+          Ls = fmaf(sc, wr[D + 1], Ls);
         }
       }
-    }
-  }
-  __syncthreads();
-  if (warp < 8) {  // O^T = V^T P^T: warp w: channels 16w .. 16w+15, all rows
-    float oacc[NT][4];
-#pragma unroll
-    for (int nt = 0; nt < NT; ++nt) oacc[nt][0] = oacc[nt][1] = oacc[nt][2] = oacc[nt][3] = 0.f;
-    const unsigned char* vbase = stage + SP_ROWS * 256;
-#pragma unroll
-    for (int ks = 0; ks < 8; ++ks) {
-      const int k0 = ks * 16;
-      const int vrow = k0 + (lane & 7) + 8 * (lane >> 4);  // matrices 2, 3: rows k0 + 8 ..
-      const int vch = 2 * warp + ((lane >> 3) & 1);        // matrices 1, 3: channels + 8
-      uint32_t af[4];
-      ldsm_x4_t(af, vbase + vrow * 256 + ((vch ^ (vrow & 7)) * 16));
-#pragma unroll
-      for (int nt = 0; nt < NT; ++nt) {
-        uint32_t bf[2];
-        ldsm_x2(bf, reinterpret_cast<const unsigned char*>(pb) + (nt * 8 + (lane & 7)) * 272 +
-                        (k0 / 8 + ((lane >> 3) & 1)) * 16);
-        mma_bf16(oacc[nt], af, bf);
+      part[e] = acc;
+      if (c == 0) {
+        part[G * D + hh] = M;
+        part[G * D + 8 + hh] = Ls;
       }
     }
-#pragma unroll
-    for (int nt = 0; nt < NT; ++nt) {
-      const int c0 = 16 * warp + g, col = 8 * nt + 2 * t;
-      *reinterpret_cast<float2*>(ob + (c0 * 16 + col)) = make_float2(oacc[nt][0], oacc[nt][1]);
-      *reinterpret_cast<float2*>(ob + ((c0 + 8) * 16 + col)) = make_float2(oacc[nt][2], oacc[nt][3]);
-    }
   }
   __syncthreads();
-  for (int e = tid; e < G * D; e += SP_THREADS) {
-    const int h = e / D, c = e - h * D;
-    const float* o0 = ob + c * 16;
-    part[h * D + c] = o0[C::hi(h)] + o0[C::lo(h)];
-  }
-  if (tid < G) {
-    float M = -INFINITY, Ls = 0.f;
-#pragma unroll
-    for (int w2 = 0; w2 < 8; ++w2) M = fmaxf(M, mx[w2 * 8 + tid]);
-#pragma unroll
-    for (int w2 = 0; w2 < 8; ++w2) Ls += ls[w2 * 8 + tid];
-    part[G * D + tid] = M;
-    part[G * D + 8 + tid] = Ls;
-  }
-  __syncthreads();  // the stage and the step's scratch are free
 }
 
-// Element offset / 128 of kept-list row j of the unit (the chunk's rows), or
-// -1 for j >= n_rows.  all_kept: row j is candidate j (rows of the kept pages
-// in page order); otherwise the list entry (row + 1, written by the key
-// select of some CTA of the group) is polled, bounded, and cleared.
-__device__ __forceinline__ int sp_row_of(const SpParams& p, unsigned char* sm, const SpUnit& x, int j, int n_rows,
-                                         bool all_kept) {
+// Element offset / 128 (row index into K', V) of gather row j of the CTA, or
+// -1 for j >= n_rows.  all_kept: j is a candidate slot of the unit (rows of the
+// kept pages in page order); otherwise j indexes the CTA's own kept list
+// (u16 slots relative to its candidate share, which starts at cs0).
+__device__ __forceinline__ int sp_row_of(const SpParams& p, const unsigned char* sm, const SpUnit& x, int j,
+                                         int n_rows, bool all_kept, int cs0) {
   if (j >= n_rows) return -1;
-  int t;
-  if (all_kept) {
-    const int* kp = reinterpret_cast<const int*>(sm + SP_KP);
-    t = (kp[j >> p.dm.lgP] << p.dm.lgP) + (j & (p.dm.P - 1));
-  } else {
-    int* e = p.wk.sel_keys + (long long)x.u * p.wk.Kmax + j;
-    int v = ld_relaxed_s32(e);
-    if (v == 0) {
-      Spin sp(p.wait_limit);
-      while ((v = ld_relaxed_s32(e)) == 0) {
-        if (sp_aborted(sm)) return -1;
-        if (sp.expired()) {
-          sp_abort(p, sm, HHR_ERR_TIMEOUT);
-          return -1;
-        }
-      }
-    }
-    *e = 0;  // the list is zero again for the next call
-    t = v - 1;
-  }
+  const int* kp = reinterpret_cast<const int*>(sm + SP_KP);
+  const int ci = all_kept ? j : cs0 + reinterpret_cast<const uint16_t*>(sm + SP_OB)[j];
+  const int t = (kp[ci >> p.dm.lgP] << p.dm.lgP) + (ci & (p.dm.P - 1));
   const long long off = kv_row(p.dm, p.table, x.b, x.h, t, p.status);
   return off >= 0 ? (int)(off / D) : -1;
 }
 
-// Issues the copies of chunk c into stage (c - c0) mod 3 (one commit group per
-// thread, possibly empty).
-__device__ __forceinline__ void sp_issue_chunk(const SpParams& p, unsigned char* sm, const SpUnit& x, int c, int c0,
-                                               int c1, int keff, bool all_kept) {
-  if (c < c1) {
-    const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
-    const int j = c * SP_ROWS + warp * 8 + (lane & 7);
-    const int ri = lane < 8 ? sp_row_of(p, sm, x, j, keff, all_kept) : -1;
-    sp_copy_rows(p, sm + ((c - c0) % SP_NGS) * SP_GSTAGE, ri);
-  }
-  cp_async_commit();
+// Issues tile k of gathering warp `warp` (gather rows j0 + 16 (warp + 8 k) ..
+// +15, clipped to j1) into its slot k mod 3.
+static __device__ __noinline__ void sp_issue_tile(const SpParams& p, unsigned char* sm, const SpUnit& x, int warp, int k,
+                                                  int j0, int j1, bool all_kept, int cs0, bool live) {
+  const int lane = threadIdx.x & 31;
+  const int j = j0 + TL_ROWS * (warp + TL_WARPS * k) + lane;
+  const int ri = (live && lane < TL_ROWS) ? sp_row_of(p, sm, x, j, j1, all_kept, cs0) : -1;
+  tile_copy(p.Kr, p.Vc, tile_slot(sm, warp, k % TL_NBUF), ri, live);
 }
 
 // ---------------------------------------------------------------------------
@@ -766,13 +856,52 @@ __device__ __forceinline__ void sp_issue_chunk(const SpParams& p, unsigned char*
 // ---------------------------------------------------------------------------
 // Candidates are the rows of the kept pages in page order (slot ci: page
 // kp[ci / P], row ci % P; slots past the sequence end are not candidates).
-// CTA r scores its balanced share [cs0, cs1) and publishes the histogram of
-// its integer scores; after the group barrier the S histograms give the
-// threshold T, the ties taken at T and the CTA's first place in the list.
-// Returns k_eff (0 after an abort; `ok` then false).
+// CTA r scores its balanced share [cs0, cs1) of the slots and publishes the
+// histogram of its integer scores; after the group barrier the S histograms
+// give the threshold score T and the ties taken at T (lower slots, i.e. lower
+// rows, first), and the CTA lists its own kept slots (u16, relative to cs0,
+// in slot order) at SP_OB: the rows it gathers.  Returns how many it keeps
+// (`ok` false after an abort).
+
+// Code row of slot ci (or -1: past the sequence end or a bad block).
+__device__ __forceinline__ long long sp_code_of(const SpParams& p, const int* kp, const SpUnit& x, int ci) {
+  const int t = (kp[ci >> p.dm.lgP] << p.dm.lgP) + (ci & (p.dm.P - 1));
+  return t < x.L ? code_row(p.dm, p.table, x.b, x.h, t, p.status) : -1;
+}
+
+template <int WORDS>
+__device__ __forceinline__ void sp_load_code(const uint64_t* src, uint64_t (&cw)[WORDS]) {
+  if constexpr (WORDS == 1) {
+    cw[0] = __ldg(reinterpret_cast<const unsigned long long*>(src));
+  } else {
+#pragma unroll
+    for (int w2 = 0; w2 < WORDS; w2 += 2) {
+      const ulonglong2 v2 = __ldg(reinterpret_cast<const ulonglong2*>(src + w2));
+      cw[w2] = v2.x;
+      cw[w2 + 1] = v2.y;
+    }
+  }
+}
+
+// The key's score: Hamming distance to the query codes summed (or, with
+// key_min, minimised) over the group's heads.
+template <int G, int WORDS>
+__device__ __forceinline__ int sp_score(const uint64_t (&cw)[WORDS], const uint64_t (&cq)[G][WORDS], bool key_min) {
+  int sum = 0, mn = INT_MAX;
+#pragma unroll
+  for (int g = 0; g < G; ++g) {
+    int sg = 0;
+#pragma unroll
+    for (int w2 = 0; w2 < WORDS; ++w2) sg += __popcll(cw[w2] ^ cq[g][w2]);
+    sum += sg;
+    mn = min(mn, sg);
+  }
+  return key_min ? mn : sum;
+}
+
 template <int G, int WORDS>
 __device__ int sp_keys(const SpParams& p, unsigned char* sm, const SpUnit& x, int r, int nkp, int n_cand_local,
-                       int keff, bool all_kept, unsigned* gx, unsigned& epoch, bool& ok) {
+                       int keff, unsigned* gx, unsigned& epoch, int& cs0, bool& ok) {
   const Dims& dm = p.dm;
   const Work& wk = p.wk;
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
@@ -780,15 +909,17 @@ __device__ int sp_keys(const SpParams& p, unsigned char* sm, const SpUnit& x, in
   const int nbins = G * dm.nb + 1, HB = wk.HB;
   int* hists = reinterpret_cast<int*>(sm + SP_HISTS);                          // [S][HB]
   uint16_t* sc = reinterpret_cast<uint16_t*>(sm + SP_HISTS + S * HB * 4);      // [share]
+  uint16_t* klist = reinterpret_cast<uint16_t*>(sm + SP_OB);                   // [kept]
   int* hist = hists;                                                           // the CTA's own, first
   int* red = reinterpret_cast<int*>(sm + SP_RED);
   int* bc = red + 128;
   const int* kp = reinterpret_cast<const int*>(sm + SP_KP);
   const unsigned* qcw = reinterpret_cast<const unsigned*>(sm + SP_QC);
   const int ncs = nkp << dm.lgP;
-  int cs0, cs1;
+  int cs1;
   share_of(ncs, S, r, cs0, cs1);
   const int nmy = cs1 - cs0;
+  #pragma unroll 1
   for (int i = tid; i < HB; i += SP_THREADS) hist[i] = 0;
   uint64_t cq[G][WORDS];
 #pragma unroll
@@ -798,54 +929,57 @@ __device__ int sp_keys(const SpParams& p, unsigned char* sm, const SpUnit& x, in
       cq[g][w2] = (uint64_t)qcw[g * 8 + 2 * w2] | ((uint64_t)qcw[g * 8 + 2 * w2 + 1] << 32);
   __syncthreads();
   int* dsc = p.dbg.key_scores ? p.dbg.key_scores + (long long)x.u * wk.Nmax * dm.P + cs0 : nullptr;
+  // two slots per thread and pass, both code loads in flight together
 #pragma unroll 1
-  for (int j = tid; j < nmy; j += SP_THREADS) {
-    const int ci = cs0 + j;
-    const int t = (kp[ci >> dm.lgP] << dm.lgP) + (ci & (dm.P - 1));
-    const long long woff = t < x.L ? code_row(dm, p.table, x.b, x.h, t, p.status) : -1;
-    int sv = 0xFFFF;
-    if (woff >= 0) {
-      const uint64_t* src = p.codes + woff;
-      uint64_t cw[WORDS];
-      if constexpr (WORDS == 1) {
-        cw[0] = __ldg(reinterpret_cast<const unsigned long long*>(src));
-      } else {
-#pragma unroll
-        for (int w2 = 0; w2 < WORDS; w2 += 2) {
-          const ulonglong2 v2 = __ldg(reinterpret_cast<const ulonglong2*>(src + w2));
-          cw[w2] = v2.x;
-          cw[w2 + 1] = v2.y;
-        }
-      }
-      int sum = 0, mn = INT_MAX;
-#pragma unroll
-      for (int g = 0; g < G; ++g) {
-        int sg = 0;
-#pragma unroll
-        for (int w2 = 0; w2 < WORDS; ++w2) sg += __popcll(cw[w2] ^ cq[g][w2]);
-        sum += sg;
-        mn = min(mn, sg);
-      }
-      sv = dm.key_min ? mn : sum;
-      atomicAdd(&hist[sv], 1);
+  for (int j = tid; j < nmy; j += 2 * SP_THREADS) {
+    const int j2 = j + SP_THREADS;
+    const long long w1 = sp_code_of(p, kp, x, cs0 + j);
+    const long long w2 = j2 < nmy ? sp_code_of(p, kp, x, cs0 + j2) : -1;
+    uint64_t c1[WORDS], c2[WORDS];
+    if (w1 >= 0) sp_load_code<WORDS>(p.codes + w1, c1);
+    if (w2 >= 0) sp_load_code<WORDS>(p.codes + w2, c2);
+    int s1 = 0xFFFF, s2 = 0xFFFF;
+    if (w1 >= 0) {
+      s1 = sp_score<G, WORDS>(c1, cq, dm.key_min);
+      atomicAdd(&hist[s1], 1);
     }
-    sc[j] = (uint16_t)sv;
-    if (dsc) dsc[j] = sv == 0xFFFF ? INT_MAX : sv;
+    if (w2 >= 0) {
+      s2 = sp_score<G, WORDS>(c2, cq, dm.key_min);
+      atomicAdd(&hist[s2], 1);
+    }
+    sc[j] = (uint16_t)s1;
+    if (dsc) dsc[j] = s1 == 0xFFFF ? INT_MAX : s1;
+    if (j2 < nmy) {
+      sc[j2] = (uint16_t)s2;
+      if (dsc) dsc[j2] = s2 == 0xFFFF ? INT_MAX : s2;
+    }
   }
   __syncthreads();
   int* myh = wk.khist + (long long)blockIdx.x * HB;
+  #pragma unroll 1
   for (int i = tid; i < nbins; i += SP_THREADS) myh[i] = hist[i];
   if (!sp_group_sync(p, sm, gx, epoch)) {
     ok = false;
     return 0;
   }
-  // ---- the group's S histograms (plain .cg loads: no cp.async group may be
-  // waited here, the gather's chunk copies are in flight) ----
+  // ---- the group's S histograms (plain .cg loads, four in flight per thread:
+  // no cp.async group may be waited here, tile copies may be in flight) ----
   {
     const int4* src = reinterpret_cast<const int4*>(wk.khist + (long long)(blockIdx.x - r) * HB);
     int4* dst = reinterpret_cast<int4*>(hists);
     const int n4 = S * HB / 4;
-    for (int i = tid; i < n4; i += SP_THREADS) dst[i] = __ldcg(src + i);
+#pragma unroll 1
+    for (int i0 = tid; i0 < n4; i0 += 4 * SP_THREADS) {
+      int4 v[4];
+#pragma unroll
+      for (int e = 0; e < 4; ++e) {
+        const int i = i0 + e * SP_THREADS;
+        v[e] = i < n4 ? __ldcg(src + i) : make_int4(0, 0, 0, 0);
+      }
+#pragma unroll
+      for (int e = 0; e < 4; ++e)
+        if (i0 + e * SP_THREADS < n4) dst[i0 + e * SP_THREADS] = v[e];
+    }
   }
   __syncthreads();
   // sum per bin (thread t: bins [t bpt, t bpt + bpt)), threshold from below
@@ -855,11 +989,13 @@ __device__ int sp_keys(const SpParams& p, unsigned char* sm, const SpUnit& x, in
 #pragma unroll
   for (int e = 0; e < 5; ++e) {
     const int bi = tid * bpt + e;
-    int s = 0;
-    if (e < bpt && bi < nbins)
-      for (int rr = 0; rr < S; ++rr) s += hists[rr * HB + bi];
-    hv[e] = s;
-    local += s;
+    int sum = 0;
+    if (e < bpt && bi < nbins) {
+#pragma unroll 1
+      for (int rr = 0; rr < S; ++rr) sum += hists[rr * HB + bi];
+    }
+    hv[e] = sum;
+    local += sum;
   }
   if (tid == 0) {
     bc[0] = -1;  // no candidate: nothing kept
@@ -889,11 +1025,13 @@ __device__ int sp_keys(const SpParams& p, unsigned char* sm, const SpUnit& x, in
   // rows below T and at T of the CTAs before r (warp w: CTAs w, w + 16, ...)
   int lt_before = 0, eq_before = 0;
   {
-    int* acc = reinterpret_cast<int*>(sm + SP_HISTS + S * HB * 4 + 2 * ((nmy + 15) & ~15));  // [2][32]
-    if (tid < 64) acc[tid] = 0;
+    int* acc = reinterpret_cast<int*>(sm + SP_HISTS + S * HB * 4 + 2 * ((nmy + 15) & ~15));  // [2]
+    if (tid < 2) acc[tid] = 0;
     __syncthreads();
+    #pragma unroll 1
     for (int rr = warp; rr < r; rr += SP_WARPS) {
       int c = 0;
+      #pragma unroll 1
       for (int bb = lane; bb < T; bb += 32) c += hists[rr * HB + bb];
 #pragma unroll
       for (int o = 16; o >= 1; o >>= 1) c += __shfl_xor_sync(0xffffffffu, c, o);
@@ -906,16 +1044,17 @@ __device__ int sp_keys(const SpParams& p, unsigned char* sm, const SpUnit& x, in
     lt_before = acc[0];
     eq_before = acc[1];
   }
-  const int off = lt_before + min(need_eq, eq_before);  // the CTA's first place in the list
+  const int off = lt_before + min(need_eq, eq_before);  // the CTA's first place in the unit's kept order
   const int take = max(0, need_eq - eq_before);         // ties it may take
   if (r == 0 && tid == 0) {
     if (p.dbg.n_cand) p.dbg.n_cand[x.u] = n_cand;
     if (p.dbg.n_sel_keys) p.dbg.n_sel_keys[x.u] = keff;
   }
-  // ---- kept rows in candidate order: thread t owns candidates [t m, (t+1) m) ----
+  // ---- kept slots in slot order: thread t owns slots [t m, (t+1) m) ----
   const int m = (nmy + SP_THREADS - 1) / SP_THREADS;
-  const int j0 = tid * m, j1 = min(nmy, j0 + m);
+  const int j0 = min(nmy, tid * m), j1 = min(nmy, j0 + m);
   int lt_t = 0, eq_t = 0;
+  #pragma unroll 1
   for (int j = j0; j < j1; ++j) {
     const int sv = sc[j];
     lt_t += sv < T;
@@ -924,73 +1063,79 @@ __device__ int sp_keys(const SpParams& p, unsigned char* sm, const SpUnit& x, in
   int tot2;
   const int pk = block_scan_excl((lt_t << 16) | eq_t, red, 1, &tot2);
   int lt_run = pk >> 16, eq_run = pk & 0xFFFF;
-  const int room = keff - off;
-  int* list = wk.sel_keys + (long long)x.u * wk.Kmax + off;
+  const int n_loc = min(SP_KLCAP, (tot2 >> 16) + min(tot2 & 0xFFFF, take));
   int* dout = p.dbg.sel_keys ? p.dbg.sel_keys + (long long)x.u * wk.Kmax + off : nullptr;
+  #pragma unroll 1
   for (int j = j0; j < j1; ++j) {
     const int sv = sc[j];
     const bool l1 = sv < T, e1 = sv == T;
     if (l1 || (e1 && eq_run < take)) {
       const int pos = lt_run + min(eq_run, take);
-      if (pos < room) {
-        const int ci = cs0 + j;
-        const int t = (kp[ci >> dm.lgP] << dm.lgP) + (ci & (dm.P - 1));
-        if (!all_kept) list[pos] = t + 1;
-        if (dout) dout[pos] = t;
+      if (pos < n_loc) {
+        klist[pos] = (uint16_t)j;
+        if (dout) {
+          const int ci = cs0 + j;
+          dout[pos] = (kp[ci >> dm.lgP] << dm.lgP) + (ci & (dm.P - 1));
+        }
       }
     }
     lt_run += l1;
     eq_run += e1;
   }
-  return keff;
+  __syncthreads();
+  return n_loc;
 }
 
 // ---------------------------------------------------------------------------
-// final merge of a unit's chunk partials (the last CTA of the group)
+// final merge of a unit's partials (the last CTA of the group to arrive)
 // ---------------------------------------------------------------------------
 // out[h][c] = sum_k w_k o_k[h][c] / sum_k w_k L_k[h], w_k = 2^(M_k[h] - M[h]),
-// M[h] = max_k M_k[h]; every sum in chunk order.  The partials are copied to
-// shared memory in passes (region A is free by now).
+// M[h] = max_k M_k[h], over the n partials in order (a partial without rows
+// has M = -inf and weight 0).  The partials are copied to shared memory in
+// passes (region A is free by now).
 template <int G>
-__device__ void sp_merge(const SpParams& p, unsigned char* sm, const SpUnit& x, int nch) {
+__device__ void sp_merge(const SpParams& p, unsigned char* sm, const SpUnit& x, int n) {
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
   const int PS = G * D + 16;
   const float* pt = p.wk.part + (long long)x.u * p.wk.C3 * PS;
-  float* wbuf = reinterpret_cast<float*>(sm + SP_OB);  // [nch][8] chunk weights (nch <= 256)
+  float* wbuf = reinterpret_cast<float*>(sm + SP_OB);  // [n][8] weights (n <= 256)
   float* inv = reinterpret_cast<float*>(sm + SP_LS);   // [8] 1 / total weight
-  // weights: warp h < G
-  if (warp < G) {
+  if (warp < G) {  // warp h: the weights of head h
     float M = -INFINITY;
-    for (int k = lane; k < nch; k += 32) M = fmaxf(M, __ldcg(pt + (long long)k * PS + G * D + warp));
+#pragma unroll 1
+    for (int k = lane; k < n; k += 32) M = fmaxf(M, __ldcg(pt + (long long)k * PS + G * D + warp));
 #pragma unroll
     for (int o = 16; o >= 1; o >>= 1) M = fmaxf(M, __shfl_xor_sync(0xffffffffu, M, o));
-    // sum of w_k L_k in chunk order: lanes take consecutive chunks, then a fixed tree
-    float part_l = 0.f;
-    for (int k0 = 0; k0 < nch; k0 += 32) {
+    float tot = 0.f;
+#pragma unroll 1
+    for (int k0 = 0; k0 < n; k0 += 32) {
       const int k = k0 + lane;
       float wl = 0.f;
-      if (k < nch) {
-        const float w = exp2f(__ldcg(pt + (long long)k * PS + G * D + warp) - M);
+      if (k < n) {
+        const float mk = __ldcg(pt + (long long)k * PS + G * D + warp);
+        const float w = mk == -INFINITY ? 0.f : exp2f(mk - M);
         wbuf[k * 8 + warp] = w;
         wl = w * __ldcg(pt + (long long)k * PS + G * D + 8 + warp);
       }
 #pragma unroll
       for (int o = 16; o >= 1; o >>= 1) wl += __shfl_xor_sync(0xffffffffu, wl, o);
-      part_l += wl;
+      tot += wl;
     }
-    if (lane == 0) inv[warp] = 1.f / part_l;
+    if (lane == 0) inv[warp] = 1.f / tot;
   }
-  // the partials, in passes of as many chunks as region A holds
   const int per = SP_A_BYTES / (PS * 4);
   float acc0 = 0.f, acc1 = 0.f;  // elements tid and tid + 512 (G * 128 <= 1024)
   float* sp = reinterpret_cast<float*>(sm);
-  for (int k0 = 0; k0 < nch; k0 += per) {
-    const int nk = min(per, nch - k0);
+#pragma unroll 1
+  for (int k0 = 0; k0 < n; k0 += per) {
+    const int nk = min(per, n - k0);
     const int n16 = nk * PS / 4;
+#pragma unroll 1
     for (int i = tid; i < n16; i += SP_THREADS) cp_async16(sp + 4 * i, pt + (long long)k0 * PS + 4 * i);
     cp_async_commit();
     cp_async_wait_all();
     __syncthreads();
+#pragma unroll 1
     for (int k = 0; k < nk; ++k) {
       const float* pk = sp + k * PS;
       if (tid < G * D) acc0 = fmaf(wbuf[(k0 + k) * 8 + (tid >> 7)], pk[tid], acc0);
@@ -1011,15 +1156,14 @@ __global__ void __launch_bounds__(SP_THREADS, 1) hhr_sparse_kernel(const __grid_
   extern __shared__ __align__(128) unsigned char sm[];
   const Dims& dm = p.dm;
   const Work& wk = p.wk;
-  const int tid = threadIdx.x;
+  const int tid = threadIdx.x, warp = tid >> 5;
   const int S = p.gsize;
   const int grp = blockIdx.x / S, r = blockIdx.x - grp * S;
   const int Units = dm.B * dm.Hkv;
   if (tid < 32) reinterpret_cast<volatile int*>(sm + SP_MISC)[tid] = 0;
-  // weights of the first unit: read before the previous kernel on the stream
-  // has finished (they are never written by a decode step)
-  Prep<G> pr;
-  if (grp < Units) sp_prep_load<G>(p, grp % dm.Hkv, pr);
+  // the prep's weights of the first unit: copied before the previous kernel on
+  // the stream has finished (they are never written by a decode step)
+  if (grp < Units) sp_issue_rw(p, sm, grp % dm.Hkv);
   pdl_launch_dependents();
   pdl_wait();
   __syncthreads();
@@ -1034,21 +1178,24 @@ __global__ void __launch_bounds__(SP_THREADS, 1) hhr_sparse_kernel(const __grid_
     unsigned* gx = wk.gx + (long long)u * wk.gx_stride;
     unsigned epoch = 0;
     const int nk_b = __ldg(p.n_keep + x.b), tk_b = __ldg(p.top_k + x.b);
-    if (!first) sp_prep_load<G>(p, x.h, pr);
+    if (!first) sp_issue_rw(p, sm, x.h);
     first = false;
-    // ---- metadata copies of the first stages, then the prep ----
+    // ---- the query heads, metadata copies of the first two stages, the prep, two more stages ----
+    #pragma unroll 1
+    for (int e = tid; e < (8 - G) * 68; e += SP_THREADS) reinterpret_cast<uint32_t*>(sm + SP_OB + G * 272)[e] = 0u;
+    sp_issue_q(p, sm, x, G);
     int p0, p1;
     share_of(x.np, S, r, p0, p1);
     const int nsteps = (p1 - p0 + SP_STAGE_PAGES - 1) / SP_STAGE_PAGES;
-#pragma unroll 1
-    for (int s = 0; s < SP_NST - 1; ++s) {
-      if (s < nsteps) sp_issue_meta(p, sm + s * SP_META_STAGE, x, p0 + s * SP_STAGE_PAGES, p1);
-      cp_async_commit();
-    }
-    sp_prep<G>(p, sm, x, pr, r == 0);
+    sp_issue_meta(p, sm, x, p0, p1);
+    sp_issue_meta(p, sm + SP_META_STAGE, x, p0 + SP_STAGE_PAGES, p1);
+    sp_prep<G>(p, sm, x, r == 0);
+    sp_issue_meta(p, sm + 2 * SP_META_STAGE, x, p0 + 2 * SP_STAGE_PAGES, p1);
+    sp_issue_meta(p, sm + 3 * SP_META_STAGE, x, p0 + 3 * SP_STAGE_PAGES, p1);
     if (x.L == 0) {  // empty sequence: zero output, no barrier (every CTA of the group skips alike)
       cp_async_wait_all();
       if (r == 0) {
+        #pragma unroll 1
         for (int e = tid; e < G * D; e += SP_THREADS) p.out[((long long)x.b * dm.Hq + x.h * G) * D + e] = 0.f;
         if (tid == 0) {
           if (p.dbg.n_sel_pages) p.dbg.n_sel_pages[x.u] = 0;
@@ -1062,7 +1209,7 @@ __global__ void __launch_bounds__(SP_THREADS, 1) hhr_sparse_kernel(const __grid_
     // ---- scan ----
     {
       float2 qa[G][4], qbn[G][4];
-      const float* qs = reinterpret_cast<const float*>(sm + SP_PREP + 4096);
+      const float* qs = reinterpret_cast<const float*>(sm + SP_OB + 4096);
       const int li = tid & 15;
 #pragma unroll
       for (int g = 0; g < G; ++g)
@@ -1077,12 +1224,10 @@ __global__ void __launch_bounds__(SP_THREADS, 1) hhr_sparse_kernel(const __grid_
             qbn[g][k] = t;
           }
         }
-      __syncthreads();  // (qs is read; SP_PREP is free for the page select)
 #pragma unroll 1
       for (int s = 0; s < nsteps; ++s) {
-        const int sn = s + SP_NST - 1;
-        if (sn < nsteps) sp_issue_meta(p, sm + (sn % SP_NST) * SP_META_STAGE, x, p0 + sn * SP_STAGE_PAGES, p1);
-        cp_async_commit();
+        const int sn = s + SP_NST - 1;  // (stages past the share issue no copy, only their commit group)
+        sp_issue_meta(p, sm + (sn % SP_NST) * SP_META_STAGE, x, p0 + sn * SP_STAGE_PAGES, p1);
         cp_async_wait<SP_NST - 1>();
         sp_scan_stage<G>(p, sm + (s % SP_NST) * SP_META_STAGE, x, p0 + s * SP_STAGE_PAGES, p1, qa, qbn);
       }
@@ -1098,35 +1243,57 @@ __global__ void __launch_bounds__(SP_THREADS, 1) hhr_sparse_kernel(const __grid_
     if (nkp > 0 && kp[nkp - 1] == x.np - 1) n_cand -= (x.np << dm.lgP) - x.L;
     const int keff = min(min(max(tk_b, 1), wk.Kmax), n_cand);
     const bool all_kept = keff == n_cand;
-    const int nch = (keff + SP_ROWS - 1) / SP_ROWS;
-    int c0, c1;
-    share_of(nch, S, r, c0, c1);
-    if (all_kept) {  // the chunks' rows are known now: their copies start at once
-      sp_issue_chunk(p, sm, x, c0, c0, c1, keff, true);
-      sp_issue_chunk(p, sm, x, c0 + 1, c0, c1, keff, true);
+    // gather rows of the CTA, in 16-row tiles (gathering warp w < 8 takes tiles
+    // w, w + 8, ...): with every candidate kept, its balanced share of the
+    // candidate slots, known now, so that their copies start at once (slots 0
+    // and 1); else the kept slots of its own scoring share (after the key select)
+    const bool gw = warp < TL_WARPS;
+    int j0 = 0, j1 = 0, mine = 0;
+    if (all_kept) {
+      share_of(keff, S, r, j0, j1);
+      const int ntile = (j1 - j0 + TL_ROWS - 1) / TL_ROWS;
+      mine = (gw && ntile > warp) ? (ntile - warp + TL_WARPS - 1) / TL_WARPS : 0;
+      if (gw) {
+        sp_issue_tile(p, sm, x, warp, 0, j0, j1, true, 0, mine > 0);
+        sp_issue_tile(p, sm, x, warp, 1, j0, j1, true, 0, mine > 1);
+      }
     }
     bool ok = true;
-    sp_keys<G, WORDS>(p, sm, x, r, nkp, n_cand, keff, all_kept, gx, epoch, ok);
+    int cs0 = 0;
+    const int n_loc = sp_keys<G, WORDS>(p, sm, x, r, nkp, n_cand, keff, gx, epoch, cs0, ok);
     if (!ok) break;
     if (!all_kept) {
-      sp_issue_chunk(p, sm, x, c0, c0, c1, keff, false);
-      sp_issue_chunk(p, sm, x, c0 + 1, c0, c1, keff, false);
+      j1 = n_loc;
+      const int ntile = (j1 + TL_ROWS - 1) / TL_ROWS;
+      mine = (gw && ntile > warp) ? (ntile - warp + TL_WARPS - 1) / TL_WARPS : 0;
     }
-    sp_issue_chunk(p, sm, x, c0 + 2, c0, c1, keff, all_kept);
-    // ---- gather: three chunks in flight ----
-    const int PS = G * D + 16;
-    float* parts = wk.part + (long long)x.u * wk.C3 * PS;
+    // ---- gather: the warps' tiles, three in flight ----
+    float o[16][4];
+#pragma unroll
+    for (int nt = 0; nt < 16; ++nt) o[nt][0] = o[nt][1] = o[nt][2] = o[nt][3] = 0.f;
+    float m_run = -INFINITY, l_run = 0.f;
+    if (gw) {
+      if (!all_kept) {
+        sp_issue_tile(p, sm, x, warp, 0, j0, j1, false, cs0, mine > 0);
+        sp_issue_tile(p, sm, x, warp, 1, j0, j1, false, cs0, mine > 1);
+      }
+      sp_issue_tile(p, sm, x, warp, 2, j0, j1, all_kept, cs0, mine > 2);
+      uint32_t aq[8][4];
+      load_q_operand(sm + SP_QB, aq);
 #pragma unroll 1
-    for (int c = c0; c < c1; ++c) {
-      cp_async_wait<SP_NGS - 1>();
-      __syncthreads();
-      if (sp_aborted(sm)) break;
-      sp_gather_step<G>(sm, sm + ((c - c0) % SP_NGS) * SP_GSTAGE, min(SP_ROWS, keff - c * SP_ROWS),
-                        parts + (long long)c * PS);
-      sp_issue_chunk(p, sm, x, c + SP_NGS, c0, c1, keff, all_kept);
+      for (int k = 0; k < mine; ++k) {
+        cp_async_wait<TL_NBUF - 1>();
+        __syncwarp();
+        const int tl = warp + TL_WARPS * k;
+        tile_attend(aq, o, m_run, l_run, tile_slot(sm, warp, k % TL_NBUF), min(TL_ROWS, j1 - j0 - TL_ROWS * tl));
+        __syncwarp();
+        sp_issue_tile(p, sm, x, warp, k + TL_NBUF, j0, j1, all_kept, cs0, k + TL_NBUF < mine);
+      }
     }
     cp_async_wait_all();
-    __syncthreads();
+    if (sp_aborted(sm)) break;
+    const int PS = G * D + 16;
+    tile_combine<G>(sm, o, m_run, l_run, mine > 0, wk.part + ((long long)x.u * wk.C3 + r) * PS, true);
     if (sp_aborted(sm)) break;
     // ---- the last CTA of the group merges ----
     if (tid == 0) {
@@ -1136,7 +1303,7 @@ __global__ void __launch_bounds__(SP_THREADS, 1) hhr_sparse_kernel(const __grid_
     }
     __syncthreads();
     if (reinterpret_cast<volatile int*>(sm + SP_MISC)[MS_LAST]) {
-      sp_merge<G>(p, sm, x, nch);
+      sp_merge<G>(p, sm, x, S);
       if (tid == 0) {
         gx[GX_BAR] = 0u;
         gx[GX_ARRIVE] = 0u;
@@ -1148,14 +1315,18 @@ __global__ void __launch_bounds__(SP_THREADS, 1) hhr_sparse_kernel(const __grid_
 }
 
 // CTAs per group: the SMs shared out over the units, at most one CTA per 64
-// pages of the longest sequence, and no more than the key select's scratch
-// holds score histograms and scores of.
-inline void sparse_group_shape(const Dims& dm, int sms, int Cmax, int HB, int* S, int* ngroups) {
+// pages of the longest sequence, no more than the key select's scratch holds
+// score histograms and scores of, and at least enough that a CTA's kept rows
+// (at most its share of the candidates, and at most the key budget) fit its
+// kept list.  Groups take units in a grid-stride loop.
+inline void sparse_group_shape(const Dims& dm, int sms, int Cmax, int Kmax, int HB, int* S, int* ngroups) {
   const int U = dm.B * dm.Hkv;
   sms = std::max(1, std::min(sms, MAX_GRID));
   int s = std::max(1, sms / U);
   s = std::min(s, std::max(1, dm.np_max / 64));
   while (s > 1 && (long long)s * HB * 4 + 2 * (((Cmax + s - 1) / s + 15) & ~15) + 256 > SP_A_BYTES - SP_HISTS) --s;
+  const int kcap = std::min(Kmax, Cmax);
+  s = std::max(s, (kcap + SP_KLCAP - 1) / SP_KLCAP);
   *S = s;
   *ngroups = std::max(1, std::min(U, sms / s));
 }

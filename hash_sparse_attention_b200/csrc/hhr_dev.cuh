@@ -90,11 +90,12 @@ __device__ __forceinline__ void split_bf16(float x, __nv_bfloat16& hi, __nv_bflo
 }
 
 // --- block scan ----------------------------------------------------------------
-// Exclusive prefix of v over the threads of the block in thread order, and the
-// block total.  `red` holds 2 x 32 ints; `parity` alternates between calls so
-// that one barrier per call suffices.  Every thread must call it.
-__device__ __forceinline__ int block_scan_excl(int v, int* red, int parity, int* total) {
-  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5, nw = blockDim.x >> 5;
+// Exclusive prefix of v over the threads of a 512-thread block in thread
+// order, and the block total.  `red` holds 2 x 32 ints; `parity` alternates
+// between calls so that one barrier per call suffices.  Every thread must call
+// it.  Out of line: one copy serves every call site.
+static __device__ __noinline__ int block_scan_excl(int v, int* red, int parity, int* total) {
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
   int x = v;
 #pragma unroll
   for (int o = 1; o < 32; o <<= 1) {
@@ -104,19 +105,22 @@ __device__ __forceinline__ int block_scan_excl(int v, int* red, int parity, int*
   int* r = red + 32 * (parity & 1);
   if (lane == 31) r[warp] = x;
   __syncthreads();
-  int before = 0, tot = 0;
-  for (int w = 0; w < nw; ++w) {
-    const int t = r[w];
-    before += w < warp ? t : 0;
-    tot += t;
+  // lane l < 16 holds warp l's total; a scan of the 16 totals in every warp
+  int t = lane < 16 ? r[lane] : 0;
+#pragma unroll
+  for (int o = 1; o < 16; o <<= 1) {
+    const int y = __shfl_up_sync(0xffffffffu, t, o);
+    if (lane >= o) t += y;
   }
-  *total = tot;
+  *total = __shfl_sync(0xffffffffu, t, 15);
+  const int before = warp > 0 ? __shfl_sync(0xffffffffu, t, (warp - 1) & 31) : 0;
   return before + x - v;
 }
 
-// Block-wide minimum and maximum of unsigned values (one barrier; `red` 2 x 32).
-__device__ __forceinline__ void block_minmax_u32(unsigned& lo, unsigned& hi, unsigned* red) {
-  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5, nw = blockDim.x >> 5;
+// Block-wide minimum and maximum of unsigned values over a 512-thread block
+// (one barrier; `red` 2 x 32).
+static __device__ __noinline__ void block_minmax_u32(unsigned& lo, unsigned& hi, unsigned* red) {
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
 #pragma unroll
   for (int o = 16; o >= 1; o >>= 1) {
     lo = min(lo, __shfl_xor_sync(0xffffffffu, lo, o));
@@ -127,11 +131,14 @@ __device__ __forceinline__ void block_minmax_u32(unsigned& lo, unsigned& hi, uns
     red[32 + warp] = hi;
   }
   __syncthreads();
-  lo = 0xffffffffu;
-  hi = 0u;
-  for (int w = 0; w < nw; ++w) {
-    lo = min(lo, red[w]);
-    hi = max(hi, red[32 + w]);
+  // lanes 16-31 hold the identities, so the butterfly over all 32 lanes
+  // leaves the block's result in every lane
+  lo = lane < 16 ? red[lane] : 0xffffffffu;
+  hi = lane < 16 ? red[32 + lane] : 0u;
+#pragma unroll
+  for (int o = 16; o >= 1; o >>= 1) {
+    lo = min(lo, __shfl_xor_sync(0xffffffffu, lo, o));
+    hi = max(hi, __shfl_xor_sync(0xffffffffu, hi, o));
   }
 }
 

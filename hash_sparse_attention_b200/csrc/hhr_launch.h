@@ -16,7 +16,8 @@ constexpr int MAX_DENSE_PAGES = 16384;   // pages of one sequence elsewhere
 constexpr int MAX_KEEP_PAGES = 2048;     // kept pages per sequence (shared memory list)
 constexpr int MAX_CANDIDATES = 16384;    // kept pages x page size
 constexpr int MAX_GRID = 160;            // CTAs of a launch (one per SM)
-constexpr int GATHER_ROWS = 128;         // rows per gather chunk
+constexpr int MAX_KEPT_PER_CTA = 10944;  // kept rows one CTA of a decode group gathers (shared memory list)
+constexpr int GATHER_ROWS = 128;         // rows per dense split granule
 constexpr int GX_STRIDE = 4;             // per-unit counter words
 constexpr long long DEFAULT_WAIT_CYCLES = 4000000000ll;  // ~2 s at 1.9 GHz
 

@@ -167,8 +167,12 @@ def test_batch_independence_and_determinism():
     for f in ("K", "V", "q"):
         setattr(solo, f, getattr(li, f)[1:2].clone())
     gs = parity.run_gpu(w1, solo)
-    assert np.array_equal(gs.out[0], g1.out[1])
-    assert np.array_equal(gs.dbg["sel_keys"][0], g1.dbg["sel_keys"][1])
+    # the selections are identical; the attention sum is split over a different
+    # number of CTAs per KV head alone than in the batch, so the output agrees
+    # to rounding (it is bit-identical for a given batch shape, as above)
+    for name in ("sel_pages", "sel_keys", "key_scores", "q_codes"):
+        assert np.array_equal(gs.dbg[name][0], g1.dbg[name][1]), name
+    assert np.allclose(gs.out[0], g1.out[1], rtol=0, atol=1e-6 * np.abs(g1.out[1]).max())
 
 
 def test_bad_block_id_sets_status_without_fault():
