@@ -141,8 +141,8 @@ hhr_status make_dims(const hhr_config* cfg, Dims* dm) {
 
 // Carves the workspace; with base == nullptr only the size is computed.
 // Sparse: per-unit counters, page bounds, one attention partial per CTA of
-// the unit's group, one score histogram per CTA.  Dense: counters and one
-// partial per split.
+// the unit's group, one cumulative score histogram per CTA and one score
+// histogram per unit.  Dense: counters and one partial per split.
 size_t carve(const Dims& dm, int Nmax, int Kmax, bool dense, char* base, Work* wk) {
   const size_t BH = (size_t)dm.B * dm.Hkv;
   size_t off = 0;
@@ -168,6 +168,7 @@ size_t carve(const Dims& dm, int Nmax, int Kmax, bool dense, char* base, Work* w
     w.U = reinterpret_cast<float*>(take(sizeof(float) * BH * w.Ustride));
     w.part = reinterpret_cast<float*>(take(sizeof(float) * BH * w.C3 * PS));
     w.khist = reinterpret_cast<int*>(take(sizeof(int) * (size_t)MAX_GRID * w.HB));
+    w.ktot = reinterpret_cast<int*>(take(sizeof(int) * BH * w.HB));
   }
   w.Nmax = Nmax;
   w.Kmax = Kmax;

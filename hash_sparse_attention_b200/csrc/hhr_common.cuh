@@ -20,12 +20,13 @@ struct Dims {
 };
 
 // Workspace carve-out of one decode step (device pointers).  The per-unit
-// counters `gx` are zero between calls (the kernels reset what they use);
-// everything else is overwritten by every call.
+// counters `gx` and histograms `ktot` are zero between calls (the kernels
+// reset what they use); everything else is overwritten by every call.
 struct Work {
   float* U;            // [B Hkv, Ustride] page bounds (aggregated over the group's query heads)
   float* part;         // [B Hkv, C3, G D + 16] softmax partials (CTAs of a unit's group, or dense splits)
-  int* khist;          // [grid, HB] score histogram of every CTA
+  int* khist;          // [grid, HB] cumulative score histogram of every CTA
+  int* ktot;           // [B Hkv, HB] score histogram of every unit (zero between calls)
   unsigned* gx;        // [B Hkv, gx_stride] per-unit barrier and arrival counters
   int Nmax, Kmax;      // budgets the workspace was sized for
   int HB;              // histogram stride (>= G nb + 1, a multiple of 8)

@@ -24,8 +24,9 @@
 //   4. when the key budget covers every candidate row, starts copying the K'/V
 //      rows of its gather share right away; scores its balanced share of the
 //      candidate rows (Hamming distance over the group's heads, summed or
-//      minimised) and publishes the score histogram;
-//   5. group barrier; the S histograms give the threshold score T and the
+//      minimised), adds its score histogram into the unit's and publishes
+//      its cumulative form;
+//   5. group barrier; the unit's histogram gives the threshold score T and the
 //      ties taken at T (lower rows first); the CTA lists the kept rows of its
 //      own scoring share, which it then gathers (with every candidate kept,
 //      its balanced share of all candidates instead);
@@ -57,7 +58,7 @@ constexpr int SP_NST = 5;                            // metadata stages in fligh
 //   scan     five metadata stages [0, 160K)
 //   psel     two refinement lists [0, 128K), histogram [128K, 136K), kept-page bitmap [136K, 137K)
 //   keys     tile slots 0-1 of the gathering warps [0, 128K) (copies started early when every
-//            candidate is kept), score histograms and scores [128K, 192K)
+//            candidate is kept), the CTA's score histogram and scores [128K, 192K)
 //   gather   the warps' tile rings [0, 192K);  combine, merge: partials
 constexpr int SP_A_BYTES = 192 * 1024;                        // region A
 constexpr int SP_RS = 2 * SP_META_STAGE;                      // R_h during the prep (64 KB)
@@ -65,7 +66,7 @@ constexpr int SP_WS = SP_RS + D * D * 4;                      // W_h during the 
 constexpr int SP_PLIST = MAX_SELECT_PAGES * 8;              // page select: one refinement list (keys, pages)
 constexpr int SP_PSH = 2 * SP_PLIST;                          // int [2048] page-select histogram
 constexpr int SP_BITS = SP_PSH + 2048 * 4;                    // u32 [256] kept-page bitmap
-constexpr int SP_HISTS = 128 * 1024;                          // key select: S score histograms, then scores
+constexpr int SP_HISTS = 128 * 1024;                          // key select: the CTA's score histogram, then scores
 constexpr int SP_QB = SP_A_BYTES;                             // bf16 [16][136] q' operand (hi, lo)
 constexpr int SP_KLCAP = MAX_KEPT_PER_CTA;                    // kept rows a CTA gathers at most (see sparse_group_shape)
 constexpr int SP_OB = SP_QB + 16 * 272;                       // prep: q, q' (fp32 [2][8][128]); keys/gather: kept list
@@ -616,13 +617,33 @@ static __device__ __noinline__ int sp_psel(const SpParams& p, unsigned char* sm,
             ++q;
           }
         __syncthreads();
-        int need = need_in, cnt = cnt_in;
+        int need = need_in, cnt = cnt_in, lv = 0;
         base += (unsigned)bstar << shift;
         shift = shift > 11 ? shift - 11 : 0;
         #pragma unroll 1
-        for (int lv = 0; cnt > 0; ++lv)
+        for (; cnt > 32; ++lv)
           cnt = psel_level(sm, sm + (lv & 1) * SP_PLIST, sm + ((lv + 1) & 1) * SP_PLIST, cnt, need, base, shift, 2 * lv + 2);
-        // (psel_level ends with a barrier: the keep bitmap is complete)
+        if (cnt > 0) {
+          // at most 32 members left: warp 0 ranks them directly (larger key
+          // first, then lower page) and keeps the first `need`
+          if (tid < 32) {
+            const uint32_t* lk2 = reinterpret_cast<const uint32_t*>(sm + (lv & 1) * SP_PLIST);
+            const int* lp2 = reinterpret_cast<const int*>(sm + (lv & 1) * SP_PLIST + SP_PLIST / 2);
+            const bool v = tid < cnt;
+            const uint32_t key = v ? lk2[tid] : 0u;
+            const int pg = v ? lp2[tid] : INT_MAX;
+            int rank = 0;
+#pragma unroll
+            for (int o = 0; o < 32; ++o) {
+              const uint32_t k2 = __shfl_sync(0xffffffffu, key, o);
+              const int p2 = __shfl_sync(0xffffffffu, pg, o);
+              rank += (o < cnt) && (k2 > key || (k2 == key && p2 < pg));
+            }
+            if (v && rank < need) atomicOr(&keep[pg >> 5], 1u << (pg & 31));
+          }
+          __syncthreads();
+        }
+        // (the keep bitmap is complete: psel_level and the rank step end with a barrier)
         sel |= (keep[i0 >> 5] >> (i0 & 16)) & 0xffffu;
       }
     }
@@ -857,9 +878,11 @@ static __device__ __noinline__ void sp_issue_tile(const SpParams& p, unsigned ch
 // Candidates are the rows of the kept pages in page order (slot ci: page
 // kp[ci / P], row ci % P; slots past the sequence end are not candidates).
 // CTA r scores its balanced share [cs0, cs1) of the slots and publishes the
-// histogram of its integer scores; after the group barrier the S histograms
-// give the threshold score T and the ties taken at T (lower slots, i.e. lower
-// rows, first), and the CTA lists its own kept slots (u16, relative to cs0,
+// histogram of its integer scores (added into the unit's histogram, and in
+// cumulative form); after the group barrier the unit's histogram gives the
+// threshold score T, the cumulative histograms of the CTAs before r the rows
+// below and at T that precede the CTA's (ties are taken lower slots, i.e.
+// lower rows, first), and the CTA lists its own kept slots (u16, relative to cs0,
 // in slot order) at SP_OB: the rows it gathers.  Returns how many it keeps
 // (`ok` false after an abort).
 
@@ -907,10 +930,9 @@ __device__ int sp_keys(const SpParams& p, unsigned char* sm, const SpUnit& x, in
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
   const int S = p.gsize;
   const int nbins = G * dm.nb + 1, HB = wk.HB;
-  int* hists = reinterpret_cast<int*>(sm + SP_HISTS);                          // [S][HB]
-  uint16_t* sc = reinterpret_cast<uint16_t*>(sm + SP_HISTS + S * HB * 4);      // [share]
-  uint16_t* klist = reinterpret_cast<uint16_t*>(sm + SP_OB);                   // [kept]
-  int* hist = hists;                                                           // the CTA's own, first
+  int* hist = reinterpret_cast<int*>(sm + SP_HISTS);                        // [HB] the CTA's histogram
+  uint16_t* sc = reinterpret_cast<uint16_t*>(sm + SP_HISTS + HB * 4);        // [share] scores
+  uint16_t* klist = reinterpret_cast<uint16_t*>(sm + SP_OB);                 // [kept]
   int* red = reinterpret_cast<int*>(sm + SP_RED);
   int* bc = red + 128;
   const int* kp = reinterpret_cast<const int*>(sm + SP_KP);
@@ -955,54 +977,48 @@ __device__ int sp_keys(const SpParams& p, unsigned char* sm, const SpUnit& x, in
     }
   }
   __syncthreads();
-  int* myh = wk.khist + (long long)blockIdx.x * HB;
-  #pragma unroll 1
-  for (int i = tid; i < nbins; i += SP_THREADS) myh[i] = hist[i];
+  // publish: the CTA's histogram added into the unit's, and its cumulative
+  // form (thread t: bins [t bpt, t bpt + bpt))
+  const int bpt = (nbins + SP_THREADS - 1) / SP_THREADS;  // <= 5
+  int* tot_h = wk.ktot + (long long)x.u * HB;
+  {
+    int hv[5], loc = 0;
+#pragma unroll
+    for (int e = 0; e < 5; ++e) {
+      const int bi = tid * bpt + e;
+      hv[e] = (e < bpt && bi < nbins) ? hist[bi] : 0;
+      if (hv[e]) atomicAdd(tot_h + bi, hv[e]);
+      loc += hv[e];
+    }
+    int tot0;
+    int run = block_scan_excl(loc, red, 0, &tot0);
+    int* myh = wk.khist + (long long)blockIdx.x * HB;
+#pragma unroll
+    for (int e = 0; e < 5; ++e) {
+      const int bi = tid * bpt + e;
+      run += hv[e];
+      if (e < bpt && bi < nbins) myh[bi] = run;
+    }
+  }
   if (!sp_group_sync(p, sm, gx, epoch)) {
     ok = false;
     return 0;
   }
-  // ---- the group's S histograms (plain .cg loads, four in flight per thread:
-  // no cp.async group may be waited here, tile copies may be in flight) ----
-  {
-    const int4* src = reinterpret_cast<const int4*>(wk.khist + (long long)(blockIdx.x - r) * HB);
-    int4* dst = reinterpret_cast<int4*>(hists);
-    const int n4 = S * HB / 4;
-#pragma unroll 1
-    for (int i0 = tid; i0 < n4; i0 += 4 * SP_THREADS) {
-      int4 v[4];
-#pragma unroll
-      for (int e = 0; e < 4; ++e) {
-        const int i = i0 + e * SP_THREADS;
-        v[e] = i < n4 ? __ldcg(src + i) : make_int4(0, 0, 0, 0);
-      }
-#pragma unroll
-      for (int e = 0; e < 4; ++e)
-        if (i0 + e * SP_THREADS < n4) dst[i0 + e * SP_THREADS] = v[e];
-    }
-  }
-  __syncthreads();
-  // sum per bin (thread t: bins [t bpt, t bpt + bpt)), threshold from below
-  const int bpt = (nbins + SP_THREADS - 1) / SP_THREADS;  // <= 5
+  // ---- the unit's histogram: the threshold from below ----
   int hv[5];
   int local = 0;
 #pragma unroll
   for (int e = 0; e < 5; ++e) {
     const int bi = tid * bpt + e;
-    int sum = 0;
-    if (e < bpt && bi < nbins) {
-#pragma unroll 1
-      for (int rr = 0; rr < S; ++rr) sum += hists[rr * HB + bi];
-    }
-    hv[e] = sum;
-    local += sum;
+    hv[e] = (e < bpt && bi < nbins) ? __ldcg(tot_h + bi) : 0;
+    local += hv[e];
   }
   if (tid == 0) {
     bc[0] = -1;  // no candidate: nothing kept
     bc[1] = 0;
   }
   int n_cand;
-  const int before = block_scan_excl(local, red, 0, &n_cand);
+  const int before = block_scan_excl(local, red, 1, &n_cand);
   if (n_cand != n_cand_local) {  // only a bad block id can make a candidate unreadable
     if (tid == 0) sp_abort(p, sm, HHR_ERR_BAD_BLOCK);
     __syncthreads();
@@ -1022,23 +1038,27 @@ __device__ int sp_keys(const SpParams& p, unsigned char* sm, const SpUnit& x, in
   }
   __syncthreads();
   const int T = bc[0], need_eq = bc[1];
-  // rows below T and at T of the CTAs before r (warp w: CTAs w, w + 16, ...)
+  // rows below T and at T of the CTAs before r, from their cumulative histograms
   int lt_before = 0, eq_before = 0;
   {
-    int* acc = reinterpret_cast<int*>(sm + SP_HISTS + S * HB * 4 + 2 * ((nmy + 15) & ~15));  // [2]
+    int* acc = red + 136;  // [2]
     if (tid < 2) acc[tid] = 0;
     __syncthreads();
-    #pragma unroll 1
-    for (int rr = warp; rr < r; rr += SP_WARPS) {
-      int c = 0;
-      #pragma unroll 1
-      for (int bb = lane; bb < T; bb += 32) c += hists[rr * HB + bb];
+    int lt = 0, eq = 0;
+    if (tid < r && T >= 0) {
+      const int* ch = wk.khist + (long long)(blockIdx.x - r + tid) * HB;
+      const int cT = __ldcg(ch + T), cB = T > 0 ? __ldcg(ch + T - 1) : 0;
+      lt = cB;
+      eq = cT - cB;
+    }
 #pragma unroll
-      for (int o = 16; o >= 1; o >>= 1) c += __shfl_xor_sync(0xffffffffu, c, o);
-      if (lane == 0) {
-        atomicAdd(&acc[0], c);
-        atomicAdd(&acc[1], T >= 0 ? hists[rr * HB + T] : 0);
-      }
+    for (int o = 16; o >= 1; o >>= 1) {
+      lt += __shfl_xor_sync(0xffffffffu, lt, o);
+      eq += __shfl_xor_sync(0xffffffffu, eq, o);
+    }
+    if (lane == 0 && warp * 32 < r) {
+      atomicAdd(&acc[0], lt);
+      atomicAdd(&acc[1], eq);
     }
     __syncthreads();
     lt_before = acc[0];
@@ -1100,6 +1120,15 @@ __device__ void sp_merge(const SpParams& p, unsigned char* sm, const SpUnit& x, 
   const float* pt = p.wk.part + (long long)x.u * p.wk.C3 * PS;
   float* wbuf = reinterpret_cast<float*>(sm + SP_OB);  // [n][8] weights (n <= 256)
   float* inv = reinterpret_cast<float*>(sm + SP_LS);   // [8] 1 / total weight
+  const int per = SP_A_BYTES / (PS * 4);              // partials per pass through region A
+  float* sp = reinterpret_cast<float*>(sm);
+  // the first pass's copies are in flight while the weights are computed
+  {
+    const int n16 = min(per, n) * PS / 4;
+#pragma unroll 1
+    for (int i = tid; i < n16; i += SP_THREADS) cp_async16(sp + 4 * i, pt + 4 * i);
+    cp_async_commit();
+  }
   if (warp < G) {  // warp h: the weights of head h
     float M = -INFINITY;
 #pragma unroll 1
@@ -1123,16 +1152,16 @@ __device__ void sp_merge(const SpParams& p, unsigned char* sm, const SpUnit& x, 
     }
     if (lane == 0) inv[warp] = 1.f / tot;
   }
-  const int per = SP_A_BYTES / (PS * 4);
   float acc0 = 0.f, acc1 = 0.f;  // elements tid and tid + 512 (G * 128 <= 1024)
-  float* sp = reinterpret_cast<float*>(sm);
 #pragma unroll 1
   for (int k0 = 0; k0 < n; k0 += per) {
     const int nk = min(per, n - k0);
-    const int n16 = nk * PS / 4;
+    if (k0 > 0) {
+      const int n16 = nk * PS / 4;
 #pragma unroll 1
-    for (int i = tid; i < n16; i += SP_THREADS) cp_async16(sp + 4 * i, pt + (long long)k0 * PS + 4 * i);
-    cp_async_commit();
+      for (int i = tid; i < n16; i += SP_THREADS) cp_async16(sp + 4 * i, pt + (long long)k0 * PS + 4 * i);
+      cp_async_commit();
+    }
     cp_async_wait_all();
     __syncthreads();
 #pragma unroll 1
@@ -1304,6 +1333,9 @@ __global__ void __launch_bounds__(SP_THREADS, 1) hhr_sparse_kernel(const __grid_
     __syncthreads();
     if (reinterpret_cast<volatile int*>(sm + SP_MISC)[MS_LAST]) {
       sp_merge<G>(p, sm, x, S);
+      // the unit's counters and score histogram are zero again for the next call
+      #pragma unroll 1
+      for (int i = tid; i < G * dm.nb + 1; i += SP_THREADS) wk.ktot[(long long)x.u * wk.HB + i] = 0;
       if (tid == 0) {
         gx[GX_BAR] = 0u;
         gx[GX_ARRIVE] = 0u;
@@ -1315,8 +1347,8 @@ __global__ void __launch_bounds__(SP_THREADS, 1) hhr_sparse_kernel(const __grid_
 }
 
 // CTAs per group: the SMs shared out over the units, at most one CTA per 64
-// pages of the longest sequence, no more than the key select's scratch holds
-// score histograms and scores of, and at least enough that a CTA's kept rows
+// pages of the longest sequence, few enough that the key select's scratch
+// holds a CTA's scores, and at least enough that a CTA's kept rows
 // (at most its share of the candidates, and at most the key budget) fit its
 // kept list.  Groups take units in a grid-stride loop.
 inline void sparse_group_shape(const Dims& dm, int sms, int Cmax, int Kmax, int HB, int* S, int* ngroups) {
@@ -1324,7 +1356,7 @@ inline void sparse_group_shape(const Dims& dm, int sms, int Cmax, int Kmax, int 
   sms = std::max(1, std::min(sms, MAX_GRID));
   int s = std::max(1, sms / U);
   s = std::min(s, std::max(1, dm.np_max / 64));
-  while (s > 1 && (long long)s * HB * 4 + 2 * (((Cmax + s - 1) / s + 15) & ~15) + 256 > SP_A_BYTES - SP_HISTS) --s;
+  while (s > 1 && (long long)HB * 4 + 2 * ((Cmax + s - 1) / s) > SP_A_BYTES - SP_HISTS) --s;
   const int kcap = std::min(Kmax, Cmax);
   s = std::max(s, (kcap + SP_KLCAP - 1) / SP_KLCAP);
   *S = s;

@@ -179,7 +179,8 @@ HHR_API size_t hhr_decode_workspace_size(const hhr_config* cfg, int32_t max_keep
                                  int32_t max_top_k);
 
 /* Zero a workspace before its first use (the decode step keeps its arrival
- * counters at zero between calls).  Enqueued on `stream`. */
+ * counters and per-unit score histograms at zero between calls).  Enqueued
+ * on `stream`. */
 HHR_API hhr_status hhr_workspace_init(void* workspace, size_t workspace_bytes, hhr_stream_t stream);
 
 /*
@@ -213,9 +214,11 @@ HHR_API hhr_status hhr_workspace_init(void* workspace, size_t workspace_bytes, h
  * device-side wait is bounded (hhr_set_wait_limit): on expiry the launch
  * records HHR_ERR_TIMEOUT in `device_status` and returns.  After any call
  * whose device status is not HHR_OK, zero the workspace again
- * (hhr_workspace_init) before the next call: its counters and row list may
- * be left mid-use.  Results are deterministic and do not depend on the batch
- * composition or on the layout (contiguous or paged).
+ * (hhr_workspace_init) before the next call: its counters and histograms
+ * may be left mid-use.  Results are deterministic for a given launch shape
+ * (the CTAs per unit follow from the SM count, the number of (sequence, KV
+ * head) units and the budgets) and do not depend on the layout (contiguous or
+ * paged); selections do not depend on the shape at all.
  *
  * The launch is a programmatic dependent launch: it may start while the
  * previous kernel on `stream` is still running and then reads R and W (the
