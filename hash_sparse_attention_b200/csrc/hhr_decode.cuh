@@ -75,7 +75,8 @@ constexpr int SP_LS = SP_OB + 2 * SP_KLCAP;                   // float [8] merge
 constexpr int SP_KP = SP_LS + 256;                            // int [MAX_KEEP_PAGES] kept pages
 constexpr int SP_QC = SP_KP + MAX_KEEP_PAGES * 4;             // u32 [8 heads][8] query codes
 constexpr int SP_RED = SP_QC + 256;                           // int: [0,64) scans, [64,128) min/max, [128,160) broadcasts
-constexpr int SP_MISC = SP_RED + 640;                         // int [32] flags
+constexpr int SP_MISC = SP_RED + 640;                         // int [16] flags
+constexpr int SP_MBAR = SP_MISC + 64;                         // u64 [8] barriers of the metadata stages
 constexpr int SP_SMEM = SP_MISC + 128;
 static_assert(2 * SP_KLCAP >= 8192, "q and q' of the prep, merge weights");
 static_assert(SP_SMEM <= 232448, "shared memory of the decode kernel");
@@ -212,7 +213,7 @@ static __device__ __noinline__ void sp_issue_q(const SpParams& p, unsigned char*
 //               products are exact and the fp32 sum is trusted when |sum| >
 //               2^-14 sum|w q| (a second product, of the magnitudes), else the
 //               sign comes from fp64.
-// The caller has issued sp_issue_rw and sp_issue_q, then two more commit groups.
+// The caller has issued sp_issue_rw and sp_issue_q (cp.async).
 template <int G>
 __device__ void sp_prep(const SpParams& p, unsigned char* sm, const SpUnit& x, bool write_dbg) {
   const Dims& dm = p.dm;
@@ -222,7 +223,7 @@ __device__ void sp_prep(const SpParams& p, unsigned char* sm, const SpUnit& x, b
   // B fragments q[g][16 ks + 2t, +1] and q[g][16 ks + 8 + 2t, +1]
   const uint32_t* qrow = reinterpret_cast<const uint32_t*>(sm + SP_OB + g * 272) + t;
   if (tid < 64) qc[tid] = 0u;
-  cp_async_wait<2>();  // R, W and q (issued before the unit's first two metadata stages)
+  cp_async_wait_all();  // R, W and q
   __syncthreads();
   if (warp < 8) {
     const int i0 = 16 * warp + g, i1 = i0 + 8;  // the lane's two rows of R_h
@@ -285,24 +286,34 @@ __device__ void sp_prep(const SpParams& p, unsigned char* sm, const SpUnit& x, b
 #pragma unroll
       for (int e = 0; e < 4; ++e) {
         const int n = 2 * t + (e & 1), jj = 16 * m + g + (e >= 2 ? 8 : 0);
-        if (n >= G) continue;
         bool bit = cs[e] > 0.f;
-        if (fabsf(cs[e]) <= ldexpf(cm[e], -14)) {  // too close to zero for fp32: the exact sign from fp64
-          const unsigned char* Wr = sm + SP_WS + jj * 256;
-          const __nv_bfloat16* qr = reinterpret_cast<const __nv_bfloat16*>(sm + SP_OB + n * 272);
+        // too close to zero for the fp32 sum: the whole warp recomputes it in
+        // fp64, one flagged (bit, head) at a time (the products are exact, so
+        // the sign is exact up to fp64 rounding of the sum)
+        unsigned flagged = __ballot_sync(0xffffffffu, n < G && fabsf(cs[e]) <= ldexpf(cm[e], -14));
+        while (flagged) {
+          const int src = __ffs(flagged) - 1;
+          flagged &= flagged - 1u;
+          const int jf = 16 * m + (src >> 2) + (e >= 2 ? 8 : 0), nf = 2 * (src & 3) + (e & 1);
+          const unsigned char* Wr = sm + SP_WS + jf * 256;
+          const __nv_bfloat16* qr = reinterpret_cast<const __nv_bfloat16*>(sm + SP_OB + nf * 272);
           double ad = 0.0;
-          #pragma unroll 1
-          for (int cc = 0; cc < D; ++cc) {
-            const int pc = ((cc >> 3) ^ (jj & 15)) * 8 + (cc & 7);
+#pragma unroll
+          for (int c4 = 0; c4 < 4; ++c4) {
+            const int cc = lane + 32 * c4;
+            const int pc = ((cc >> 3) ^ (jf & 15)) * 8 + (cc & 7);
             ad += (double)__bfloat162float(reinterpret_cast<const __nv_bfloat16*>(Wr)[pc]) *
                   (double)__bfloat162float(qr[cc]);
           }
-          bit = ad > 0.0;
+#pragma unroll
+          for (int o = 16; o >= 1; o >>= 1) ad += __shfl_xor_sync(0xffffffffu, ad, o);
+          if (lane == src) bit = ad > 0.0;
         }
-        if (bit) atomicOr(&qc[n * 8 + (jj >> 5)], 1u << (jj & 31));
+        if (n < G && bit) atomicOr(&qc[n * 8 + (jj >> 5)], 1u << (jj & 31));
       }
     }
   }
+  fence_proxy_async();  // (R_h and W_h's room is refilled by TMA copies next)
   __syncthreads();
   if (write_dbg && p.dbg.q_codes) {
     const int w32 = dm.words * 2;
@@ -316,31 +327,30 @@ __device__ void sp_prep(const SpParams& p, unsigned char* sm, const SpUnit& x, b
 // ---------------------------------------------------------------------------
 // scan: page bounds of the CTA's pages
 // ---------------------------------------------------------------------------
-// Stage s holds pages p0 + 64 s + j (j < 64): minima rows at j*256, maxima at
-// 64*256 + j*256.  Thread t copies and later reads the 16-byte piece (t & 15)
-// (channels 8(t&15) .. +7) of pages j = t/16 and j = t/16 + 32, minima and maxima.
-static __device__ __noinline__ void sp_issue_meta(const SpParams& p, unsigned char* stage, const SpUnit& x, int pg0, int p1) {
-  if (pg0 < p1) {
-    const int tid = threadIdx.x, li = tid & 15;
-#pragma unroll
-    for (int half = 0; half < 2; ++half) {
-      const int j = (tid >> 4) + 32 * half;
-      const int pg = pg0 + j;
-      unsigned char* dmin = stage + j * 256 + li * 16;
-      // every thread issues both copies: a page past the share or with a bad
-      // block id (the status records it) reads as zeros
-      const long long off = pg < p1 ? meta_row(p.dm, p.table, x.b, x.h, pg, p.status) : -1;
-      const bool ok = off >= 0;
-      const long long e = ok ? off + li * 8 : 0;
-      const unsigned nbytes = ok ? 16u : 0u;
-      asm volatile("cp.async.cg.shared.global [%0], [%1], 16, %2;" ::"r"(smem_u32(dmin)), "l"(p.pmin + e), "r"(nbytes)
-                   : "memory");
-      asm volatile("cp.async.cg.shared.global [%0], [%1], 16, %2;" ::"r"(smem_u32(dmin + SP_STAGE_PAGES * 256)),
-                   "l"(p.pmax + e), "r"(nbytes)
-                   : "memory");
+// Stage s holds pages p0 + 64 s + j (j < 64, clipped to p1): minima rows at
+// j*256, maxima at 64*256 + j*256, copied by TMA bulk copies that complete on
+// the stage's barrier: two copies of n rows (contiguous cache; thread 0), or
+// one 256-byte copy per row (paged cache; threads 0..2n-1; a bad block id
+// copies row 0 of the pool instead and is recorded in the status).  Thread 0
+// arms the barrier with the stage's byte count.  Thread t later reads the
+// 16-byte piece (t & 15) (channels 8(t&15) .. +7) of pages j = t/16 and
+// j = t/16 + 32, minima and maxima.
+static __device__ __noinline__ void sp_issue_meta(const SpParams& p, unsigned char* stage, uint64_t* bar,
+                                                  const SpUnit& x, int pg0, int p1) {
+  const int tid = threadIdx.x;
+  const int n = min(SP_STAGE_PAGES, p1 - pg0);  // >= 1
+  if (tid == 0) mbar_arrive_expect_tx(bar, 2u * n * 256u);
+  if (!p.dm.paged) {
+    if (tid == 0) {
+      const long long off = meta_row(p.dm, p.table, x.b, x.h, pg0, p.status);
+      bulk_g2s(stage, p.pmin + off, n * 256, bar);
+      bulk_g2s(stage + SP_STAGE_PAGES * 256, p.pmax + off, n * 256, bar);
     }
+  } else if (tid < 2 * n) {
+    const int j = tid >> 1, mx = tid & 1;
+    const long long off = meta_row(p.dm, p.table, x.b, x.h, pg0 + j, p.status);
+    bulk_g2s(stage + mx * SP_STAGE_PAGES * 256 + j * 256, (mx ? p.pmax : p.pmin) + (off >= 0 ? off : 0), 256, bar);
   }
-  cp_async_commit();
 }
 
 // Bounds of the (up to) 64 pages of one stage.  Half-warp hw = t/16 computes
@@ -1189,7 +1199,15 @@ __global__ void __launch_bounds__(SP_THREADS, 1) hhr_sparse_kernel(const __grid_
   const int S = p.gsize;
   const int grp = blockIdx.x / S, r = blockIdx.x - grp * S;
   const int Units = dm.B * dm.Hkv;
-  if (tid < 32) reinterpret_cast<volatile int*>(sm + SP_MISC)[tid] = 0;
+  if (tid < 16) reinterpret_cast<volatile int*>(sm + SP_MISC)[tid] = 0;
+  // one barrier per metadata stage slot; bit i of `ph` is the parity of slot
+  // i's next phase, bit i of `pend` marks a phase armed and not yet waited for
+  uint64_t* mbar = reinterpret_cast<uint64_t*>(sm + SP_MBAR);
+  if (tid == 0) {
+    for (int i = 0; i < SP_NST; ++i) mbar_init(mbar + i, 1);
+    mbar_fence_init();
+  }
+  unsigned ph = 0u, pend = 0u;
   // the prep's weights of the first unit: copied before the previous kernel on
   // the stream has finished (they are never written by a decode step)
   if (grp < Units) sp_issue_rw(p, sm, grp % dm.Hkv);
@@ -1216,11 +1234,18 @@ __global__ void __launch_bounds__(SP_THREADS, 1) hhr_sparse_kernel(const __grid_
     int p0, p1;
     share_of(x.np, S, r, p0, p1);
     const int nsteps = (p1 - p0 + SP_STAGE_PAGES - 1) / SP_STAGE_PAGES;
-    sp_issue_meta(p, sm, x, p0, p1);
-    sp_issue_meta(p, sm + SP_META_STAGE, x, p0 + SP_STAGE_PAGES, p1);
+    auto issue_stage = [&](int st) {  // (every thread calls it alike)
+      if (st < nsteps) {
+        const int slot = st % SP_NST;
+        sp_issue_meta(p, sm + slot * SP_META_STAGE, mbar + slot, x, p0 + st * SP_STAGE_PAGES, p1);
+        pend |= 1u << slot;
+      }
+    };
+    issue_stage(0);
+    issue_stage(1);
     sp_prep<G>(p, sm, x, r == 0);
-    sp_issue_meta(p, sm + 2 * SP_META_STAGE, x, p0 + 2 * SP_STAGE_PAGES, p1);
-    sp_issue_meta(p, sm + 3 * SP_META_STAGE, x, p0 + 3 * SP_STAGE_PAGES, p1);
+    issue_stage(2);
+    issue_stage(3);
     if (x.L == 0) {  // empty sequence: zero output, no barrier (every CTA of the group skips alike)
       cp_async_wait_all();
       if (r == 0) {
@@ -1232,6 +1257,7 @@ __global__ void __launch_bounds__(SP_THREADS, 1) hhr_sparse_kernel(const __grid_
           if (p.dbg.n_cand) p.dbg.n_cand[x.u] = 0;
         }
       }
+      fence_proxy_async();
       __syncthreads();
       continue;
     }
@@ -1255,12 +1281,16 @@ __global__ void __launch_bounds__(SP_THREADS, 1) hhr_sparse_kernel(const __grid_
         }
 #pragma unroll 1
       for (int s = 0; s < nsteps; ++s) {
-        const int sn = s + SP_NST - 1;  // (stages past the share issue no copy, only their commit group)
-        sp_issue_meta(p, sm + (sn % SP_NST) * SP_META_STAGE, x, p0 + sn * SP_STAGE_PAGES, p1);
-        cp_async_wait<SP_NST - 1>();
-        sp_scan_stage<G>(p, sm + (s % SP_NST) * SP_META_STAGE, x, p0 + s * SP_STAGE_PAGES, p1, qa, qbn);
+        if (s + SP_NST - 1 < nsteps) {
+          __syncthreads();  // every thread is done with stage s - 1, whose slot is refilled
+          issue_stage(s + SP_NST - 1);
+        }
+        const int slot = s % SP_NST;
+        if (!mbar_wait(mbar + slot, (ph >> slot) & 1u, p.wait_limit)) sp_abort(p, sm, HHR_ERR_TIMEOUT);
+        ph ^= 1u << slot;
+        pend &= ~(1u << slot);
+        sp_scan_stage<G>(p, sm + slot * SP_META_STAGE, x, p0 + s * SP_STAGE_PAGES, p1, qa, qbn);
       }
-      cp_async_wait_all();
     }
     // ---- the unit's bounds are complete ----
     if (!sp_group_sync(p, sm, gx, epoch)) break;
@@ -1341,9 +1371,14 @@ __global__ void __launch_bounds__(SP_THREADS, 1) hhr_sparse_kernel(const __grid_
         gx[GX_ARRIVE] = 0u;
       }
     }
+    fence_proxy_async();  // (region A is refilled by TMA copies in the next unit)
     __syncthreads();
   }
   cp_async_wait_all();
+  // an abort can leave metadata copies in flight: they land before the CTA exits
+  #pragma unroll 1
+  for (int i = 0; i < SP_NST; ++i)
+    if ((pend >> i) & 1u) mbar_wait(mbar + i, (ph >> i) & 1u, p.wait_limit);
 }
 
 // CTAs per group: the SMs shared out over the units, at most one CTA per 64
