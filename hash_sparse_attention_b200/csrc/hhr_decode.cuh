@@ -132,36 +132,31 @@ __device__ __forceinline__ void sp_abort(const SpParams& p, unsigned char* sm, i
 
 // Group barrier: every write made before it by any thread of the group's S
 // CTAs is visible after it (read such data with .cg loads: L1 is not
-// coherent).  A release add and a bounded acquire poll on the unit's counter.
-// Split in two: between sp_group_arrive and sp_group_wait the CTA may do work
-// that the barrier does not need to cover.  sp_group_wait is false after a
-// timeout or an abort (every thread of the CTA sees the same).
-__device__ __forceinline__ void sp_group_arrive(const SpParams& p, unsigned* gx, unsigned& epoch) {
-  __syncthreads();
+// coherent).  A release add and a bounded acquire poll on the unit's counter,
+// by the first thread of the CTA's participating warps (the whole CTA, or the
+// warp group of named barrier `bar`).  False after a timeout or an abort
+// (every participating thread sees the same).
+__device__ __forceinline__ bool sp_group_sync(const SpParams& p, unsigned char* sm, unsigned* gx, unsigned& epoch,
+                                              int tb = 0, int nthr = SP_THREADS, int bar = 0) {
+  bar_sync(bar, nthr);
   if (p.gsize > 1) {
     epoch += (unsigned)p.gsize;
-    if (threadIdx.x == 0) red_release_add(gx + GX_BAR, 1u);
-  }
-}
-__device__ __forceinline__ bool sp_group_wait(const SpParams& p, unsigned char* sm, unsigned* gx, unsigned epoch) {
-  if (p.gsize > 1) {
-    if (threadIdx.x == 0 && ld_acquire(gx + GX_BAR) < epoch) {
-      Spin sp(p.wait_limit);
-      while (ld_acquire(gx + GX_BAR) < epoch) {
-        if (sp_aborted(sm)) break;
-        if (sp.expired()) {
-          sp_abort(p, sm, HHR_ERR_TIMEOUT);
-          break;
+    if (threadIdx.x == tb) {
+      red_release_add(gx + GX_BAR, 1u);
+      if (ld_acquire(gx + GX_BAR) < epoch) {
+        Spin sp(p.wait_limit);
+        while (ld_acquire(gx + GX_BAR) < epoch) {
+          if (sp_aborted(sm)) break;
+          if (sp.expired()) {
+            sp_abort(p, sm, HHR_ERR_TIMEOUT);
+            break;
+          }
         }
       }
     }
-    __syncthreads();
+    bar_sync(bar, nthr);
   }
   return !sp_aborted(sm);
-}
-__device__ __forceinline__ bool sp_group_sync(const SpParams& p, unsigned char* sm, unsigned* gx, unsigned& epoch) {
-  sp_group_arrive(p, gx, epoch);
-  return sp_group_wait(p, sm, gx, epoch);
 }
 
 // ---------------------------------------------------------------------------
@@ -282,18 +277,24 @@ __device__ void sp_prep(const SpParams& p, unsigned char* sm, const SpUnit& x, b
         mma_bf16(cs, a, b);
         mma_bf16(cm, am, bm);
       }
-      // cs[e]: bit row jj = 16 m + g (+8 for e >= 2), head n = 2t + (e & 1)
+      // cs[e]: bit row jj = 16 m + g (+8 for e >= 2), head n = 2t + (e & 1).
+      // A sum too close to zero for fp32 is recomputed by the whole warp in
+      // fp64, one flagged (bit, head) at a time (the products are exact, so the
+      // sign is exact up to fp64 rounding of the sum).
+      unsigned bits = 0u, flag = 0u;
 #pragma unroll
       for (int e = 0; e < 4; ++e) {
-        const int n = 2 * t + (e & 1), jj = 16 * m + g + (e >= 2 ? 8 : 0);
-        bool bit = cs[e] > 0.f;
-        // too close to zero for the fp32 sum: the whole warp recomputes it in
-        // fp64, one flagged (bit, head) at a time (the products are exact, so
-        // the sign is exact up to fp64 rounding of the sum)
-        unsigned flagged = __ballot_sync(0xffffffffu, n < G && fabsf(cs[e]) <= ldexpf(cm[e], -14));
-        while (flagged) {
-          const int src = __ffs(flagged) - 1;
-          flagged &= flagged - 1u;
+        bits |= (unsigned)(cs[e] > 0.f) << e;
+        if (2 * t + (e & 1) < G && fabsf(cs[e]) <= ldexpf(cm[e], -14)) flag |= 1u << e;
+      }
+      unsigned lanes = __ballot_sync(0xffffffffu, flag != 0u);
+      while (lanes) {
+        const int src = __ffs(lanes) - 1;
+        lanes &= lanes - 1u;
+        unsigned fe = __shfl_sync(0xffffffffu, flag, src);
+        while (fe) {
+          const int e = __ffs(fe) - 1;
+          fe &= fe - 1u;
           const int jf = 16 * m + (src >> 2) + (e >= 2 ? 8 : 0), nf = 2 * (src & 3) + (e & 1);
           const unsigned char* Wr = sm + SP_WS + jf * 256;
           const __nv_bfloat16* qr = reinterpret_cast<const __nv_bfloat16*>(sm + SP_OB + nf * 272);
@@ -307,9 +308,13 @@ __device__ void sp_prep(const SpParams& p, unsigned char* sm, const SpUnit& x, b
           }
 #pragma unroll
           for (int o = 16; o >= 1; o >>= 1) ad += __shfl_xor_sync(0xffffffffu, ad, o);
-          if (lane == src) bit = ad > 0.0;
+          if (lane == src) bits = (bits & ~(1u << e)) | ((unsigned)(ad > 0.0) << e);
         }
-        if (n < G && bit) atomicOr(&qc[n * 8 + (jj >> 5)], 1u << (jj & 31));
+      }
+#pragma unroll
+      for (int e = 0; e < 4; ++e) {
+        const int n = 2 * t + (e & 1), jj = 16 * m + g + (e >= 2 ? 8 : 0);
+        if (n < G && ((bits >> e) & 1u)) atomicOr(&qc[n * 8 + (jj >> 5)], 1u << (jj & 31));
       }
     }
   }
@@ -643,7 +648,7 @@ static __device__ __noinline__ int sp_psel(const SpParams& p, unsigned char* sm,
             const uint32_t key = v ? lk2[tid] : 0u;
             const int pg = v ? lp2[tid] : INT_MAX;
             int rank = 0;
-#pragma unroll
+#pragma unroll 4
             for (int o = 0; o < 32; ++o) {
               const uint32_t k2 = __shfl_sync(0xffffffffu, key, o);
               const int p2 = __shfl_sync(0xffffffffu, pg, o);
@@ -932,17 +937,21 @@ __device__ __forceinline__ int sp_score(const uint64_t (&cw)[WORDS], const uint6
   return key_min ? mn : sum;
 }
 
+// The key select runs on the warp group [tb / 32, (tb + nthr) / 32) with named
+// barrier `bar` (the whole CTA: tb = 0, nthr = 512, bar = 0), its histogram
+// and scores at `scr`; with make_list it writes the kept list at SP_OB.
 template <int G, int WORDS>
-__device__ int sp_keys(const SpParams& p, unsigned char* sm, const SpUnit& x, int r, int nkp, int n_cand_local,
-                       int keff, unsigned* gx, unsigned& epoch, int& cs0, bool& ok) {
+__device__ __noinline__ int sp_keys(const SpParams& p, unsigned char* sm, const SpUnit& x, int r, int nkp, int n_cand_local,
+                       int keff, unsigned* gx, unsigned& epoch, int& cs0, bool& ok, int tb, int nthr, int bar,
+                       unsigned char* scr, bool make_list) {
   const Dims& dm = p.dm;
   const Work& wk = p.wk;
-  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+  const int tid = threadIdx.x - tb, lane = tid & 31, warp = tid >> 5, nw = nthr >> 5;
   const int S = p.gsize;
   const int nbins = G * dm.nb + 1, HB = wk.HB;
-  int* hist = reinterpret_cast<int*>(sm + SP_HISTS);                        // [HB] the CTA's histogram
-  uint16_t* sc = reinterpret_cast<uint16_t*>(sm + SP_HISTS + HB * 4);        // [share] scores
-  uint16_t* klist = reinterpret_cast<uint16_t*>(sm + SP_OB);                 // [kept]
+  int* hist = reinterpret_cast<int*>(scr);                            // [HB] the CTA's histogram
+  uint16_t* sc = reinterpret_cast<uint16_t*>(scr + HB * 4);           // [share] scores
+  uint16_t* klist = reinterpret_cast<uint16_t*>(sm + SP_OB);          // [kept]
   int* red = reinterpret_cast<int*>(sm + SP_RED);
   int* bc = red + 128;
   const int* kp = reinterpret_cast<const int*>(sm + SP_KP);
@@ -952,19 +961,19 @@ __device__ int sp_keys(const SpParams& p, unsigned char* sm, const SpUnit& x, in
   share_of(ncs, S, r, cs0, cs1);
   const int nmy = cs1 - cs0;
   #pragma unroll 1
-  for (int i = tid; i < HB; i += SP_THREADS) hist[i] = 0;
+  for (int i = tid; i < HB; i += nthr) hist[i] = 0;
   uint64_t cq[G][WORDS];
 #pragma unroll
   for (int g = 0; g < G; ++g)
 #pragma unroll
     for (int w2 = 0; w2 < WORDS; ++w2)
       cq[g][w2] = (uint64_t)qcw[g * 8 + 2 * w2] | ((uint64_t)qcw[g * 8 + 2 * w2 + 1] << 32);
-  __syncthreads();
+  bar_sync(bar, nthr);
   int* dsc = p.dbg.key_scores ? p.dbg.key_scores + (long long)x.u * wk.Nmax * dm.P + cs0 : nullptr;
   // two slots per thread and pass, both code loads in flight together
 #pragma unroll 1
-  for (int j = tid; j < nmy; j += 2 * SP_THREADS) {
-    const int j2 = j + SP_THREADS;
+  for (int j = tid; j < nmy; j += 2 * nthr) {
+    const int j2 = j + nthr;
     const long long w1 = sp_code_of(p, kp, x, cs0 + j);
     const long long w2 = j2 < nmy ? sp_code_of(p, kp, x, cs0 + j2) : -1;
     uint64_t c1[WORDS], c2[WORDS];
@@ -986,39 +995,39 @@ __device__ int sp_keys(const SpParams& p, unsigned char* sm, const SpUnit& x, in
       if (dsc) dsc[j2] = s2 == 0xFFFF ? INT_MAX : s2;
     }
   }
-  __syncthreads();
+  bar_sync(bar, nthr);
   // publish: the CTA's histogram added into the unit's, and its cumulative
   // form (thread t: bins [t bpt, t bpt + bpt))
-  const int bpt = (nbins + SP_THREADS - 1) / SP_THREADS;  // <= 5
+  const int bpt = (nbins + nthr - 1) / nthr;  // <= 9
   int* tot_h = wk.ktot + (long long)x.u * HB;
   {
-    int hv[5], loc = 0;
+    int hv[9], loc = 0;
 #pragma unroll
-    for (int e = 0; e < 5; ++e) {
+    for (int e = 0; e < 9; ++e) {
       const int bi = tid * bpt + e;
       hv[e] = (e < bpt && bi < nbins) ? hist[bi] : 0;
       if (hv[e]) atomicAdd(tot_h + bi, hv[e]);
       loc += hv[e];
     }
     int tot0;
-    int run = block_scan_excl(loc, red, 0, &tot0);
+    int run = block_scan_excl(loc, red, 0, &tot0, tb >> 5, nw, bar);
     int* myh = wk.khist + (long long)blockIdx.x * HB;
 #pragma unroll
-    for (int e = 0; e < 5; ++e) {
+    for (int e = 0; e < 9; ++e) {
       const int bi = tid * bpt + e;
       run += hv[e];
       if (e < bpt && bi < nbins) myh[bi] = run;
     }
   }
-  if (!sp_group_sync(p, sm, gx, epoch)) {
+  if (!sp_group_sync(p, sm, gx, epoch, tb, nthr, bar)) {
     ok = false;
     return 0;
   }
   // ---- the unit's histogram: the threshold from below ----
-  int hv[5];
+  int hv[9];
   int local = 0;
 #pragma unroll
-  for (int e = 0; e < 5; ++e) {
+  for (int e = 0; e < 9; ++e) {
     const int bi = tid * bpt + e;
     hv[e] = (e < bpt && bi < nbins) ? __ldcg(tot_h + bi) : 0;
     local += hv[e];
@@ -1028,17 +1037,17 @@ __device__ int sp_keys(const SpParams& p, unsigned char* sm, const SpUnit& x, in
     bc[1] = 0;
   }
   int n_cand;
-  const int before = block_scan_excl(local, red, 1, &n_cand);
+  const int before = block_scan_excl(local, red, 1, &n_cand, tb >> 5, nw, bar);
   if (n_cand != n_cand_local) {  // only a bad block id can make a candidate unreadable
     if (tid == 0) sp_abort(p, sm, HHR_ERR_BAD_BLOCK);
-    __syncthreads();
+    bar_sync(bar, nthr);
     ok = false;
     return 0;
   }
   if (keff > 0 && before < keff && before + local >= keff) {
     int run = before;
 #pragma unroll
-    for (int e = 0; e < 5; ++e) {
+    for (int e = 0; e < 9; ++e) {
       if (run < keff && run + hv[e] >= keff) {
         bc[0] = tid * bpt + e;
         bc[1] = keff - run;
@@ -1046,14 +1055,14 @@ __device__ int sp_keys(const SpParams& p, unsigned char* sm, const SpUnit& x, in
       run += hv[e];
     }
   }
-  __syncthreads();
+  bar_sync(bar, nthr);
   const int T = bc[0], need_eq = bc[1];
   // rows below T and at T of the CTAs before r, from their cumulative histograms
   int lt_before = 0, eq_before = 0;
   {
     int* acc = red + 136;  // [2]
     if (tid < 2) acc[tid] = 0;
-    __syncthreads();
+    bar_sync(bar, nthr);
     int lt = 0, eq = 0;
     if (tid < r && T >= 0) {
       const int* ch = wk.khist + (long long)(blockIdx.x - r + tid) * HB;
@@ -1070,7 +1079,7 @@ __device__ int sp_keys(const SpParams& p, unsigned char* sm, const SpUnit& x, in
       atomicAdd(&acc[0], lt);
       atomicAdd(&acc[1], eq);
     }
-    __syncthreads();
+    bar_sync(bar, nthr);
     lt_before = acc[0];
     eq_before = acc[1];
   }
@@ -1081,7 +1090,7 @@ __device__ int sp_keys(const SpParams& p, unsigned char* sm, const SpUnit& x, in
     if (p.dbg.n_sel_keys) p.dbg.n_sel_keys[x.u] = keff;
   }
   // ---- kept slots in slot order: thread t owns slots [t m, (t+1) m) ----
-  const int m = (nmy + SP_THREADS - 1) / SP_THREADS;
+  const int m = (nmy + nthr - 1) / nthr;
   const int j0 = min(nmy, tid * m), j1 = min(nmy, j0 + m);
   int lt_t = 0, eq_t = 0;
   #pragma unroll 1
@@ -1091,7 +1100,7 @@ __device__ int sp_keys(const SpParams& p, unsigned char* sm, const SpUnit& x, in
     eq_t += sv == T;
   }
   int tot2;
-  const int pk = block_scan_excl((lt_t << 16) | eq_t, red, 1, &tot2);
+  const int pk = block_scan_excl((lt_t << 16) | eq_t, red, 0, &tot2, tb >> 5, nw, bar);
   int lt_run = pk >> 16, eq_run = pk & 0xFFFF;
   const int n_loc = min(SP_KLCAP, (tot2 >> 16) + min(tot2 & 0xFFFF, take));
   int* dout = p.dbg.sel_keys ? p.dbg.sel_keys + (long long)x.u * wk.Kmax + off : nullptr;
@@ -1102,7 +1111,7 @@ __device__ int sp_keys(const SpParams& p, unsigned char* sm, const SpUnit& x, in
     if (l1 || (e1 && eq_run < take)) {
       const int pos = lt_run + min(eq_run, take);
       if (pos < n_loc) {
-        klist[pos] = (uint16_t)j;
+        if (make_list) klist[pos] = (uint16_t)j;
         if (dout) {
           const int ci = cs0 + j;
           dout[pos] = (kp[ci >> dm.lgP] << dm.lgP) + (ci & (dm.P - 1));
@@ -1112,7 +1121,7 @@ __device__ int sp_keys(const SpParams& p, unsigned char* sm, const SpUnit& x, in
     lt_run += l1;
     eq_run += e1;
   }
-  __syncthreads();
+  bar_sync(bar, nthr);
   return n_loc;
 }
 
@@ -1304,27 +1313,36 @@ __global__ void __launch_bounds__(SP_THREADS, 1) hhr_sparse_kernel(const __grid_
     const bool all_kept = keff == n_cand;
     // gather rows of the CTA, in 16-row tiles (gathering warp w < 8 takes tiles
     // w, w + 8, ...): with every candidate kept, its balanced share of the
-    // candidate slots, known now, so that their copies start at once (slots 0
-    // and 1); else the kept slots of its own scoring share (after the key select)
+    // candidate slots, known now; else the kept slots of its own scoring share
+    // (after the key select).  With every candidate kept and the key select's
+    // scratch small enough for region B, warps 8-15 run the key select while
+    // warps 0-7 gather (the key select then keeps every candidate).
     const bool gw = warp < TL_WARPS;
+    const int ncs = nkp << dm.lgP;
+    const bool conc = all_kept && wk.HB * 4 + 2 * ((ncs + S - 1) / S) <= 2 * SP_KLCAP;
     int j0 = 0, j1 = 0, mine = 0;
     if (all_kept) {
       share_of(keff, S, r, j0, j1);
       const int ntile = (j1 - j0 + TL_ROWS - 1) / TL_ROWS;
       mine = (gw && ntile > warp) ? (ntile - warp + TL_WARPS - 1) / TL_WARPS : 0;
-      if (gw) {
+      if (gw) {  // (their copies start at once)
         sp_issue_tile(p, sm, x, warp, 0, j0, j1, true, 0, mine > 0);
         sp_issue_tile(p, sm, x, warp, 1, j0, j1, true, 0, mine > 1);
+        if (conc) sp_issue_tile(p, sm, x, warp, 2, j0, j1, true, 0, mine > 2);
       }
     }
     bool ok = true;
     int cs0 = 0;
-    const int n_loc = sp_keys<G, WORDS>(p, sm, x, r, nkp, n_cand, keff, gx, epoch, cs0, ok);
-    if (!ok) break;
-    if (!all_kept) {
-      j1 = n_loc;
-      const int ntile = (j1 + TL_ROWS - 1) / TL_ROWS;
-      mine = (gw && ntile > warp) ? (ntile - warp + TL_WARPS - 1) / TL_WARPS : 0;
+    if (conc) {
+      if (!gw) sp_keys<G, WORDS>(p, sm, x, r, nkp, n_cand, keff, gx, epoch, cs0, ok, TL_WARPS * 32, SP_THREADS - TL_WARPS * 32, 1, sm + SP_OB, false);
+    } else {
+      const int n_loc = sp_keys<G, WORDS>(p, sm, x, r, nkp, n_cand, keff, gx, epoch, cs0, ok, 0, SP_THREADS, 0, sm + SP_HISTS, true);
+      if (!ok) break;
+      if (!all_kept) {
+        j1 = n_loc;
+        const int ntile = (j1 + TL_ROWS - 1) / TL_ROWS;
+        mine = (gw && ntile > warp) ? (ntile - warp + TL_WARPS - 1) / TL_WARPS : 0;
+      }
     }
     // ---- gather: the warps' tiles, three in flight ----
     float o[16][4];
@@ -1336,7 +1354,7 @@ __global__ void __launch_bounds__(SP_THREADS, 1) hhr_sparse_kernel(const __grid_
         sp_issue_tile(p, sm, x, warp, 0, j0, j1, false, cs0, mine > 0);
         sp_issue_tile(p, sm, x, warp, 1, j0, j1, false, cs0, mine > 1);
       }
-      sp_issue_tile(p, sm, x, warp, 2, j0, j1, all_kept, cs0, mine > 2);
+      if (!conc) sp_issue_tile(p, sm, x, warp, 2, j0, j1, all_kept, cs0, mine > 2);
       uint32_t aq[8][4];
       load_q_operand(sm + SP_QB, aq);
 #pragma unroll 1
@@ -1350,6 +1368,7 @@ __global__ void __launch_bounds__(SP_THREADS, 1) hhr_sparse_kernel(const __grid_
       }
     }
     cp_async_wait_all();
+    __syncthreads();  // (the key select of warps 8-15 may have raised the abort flag)
     if (sp_aborted(sm)) break;
     const int PS = G * D + 16;
     tile_combine<G>(sm, o, m_run, l_run, mine > 0, wk.part + ((long long)x.u * wk.C3 + r) * PS, true);

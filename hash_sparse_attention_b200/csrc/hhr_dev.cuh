@@ -130,12 +130,19 @@ __device__ __forceinline__ void split_bf16(float x, __nv_bfloat16& hi, __nv_bflo
 }
 
 // --- block scan ----------------------------------------------------------------
-// Exclusive prefix of v over the threads of a 512-thread block in thread
-// order, and the block total.  `red` holds 2 x 32 ints; `parity` alternates
-// between calls so that one barrier per call suffices.  Every thread must call
-// it.  Out of line: one copy serves every call site.
-static __device__ __noinline__ int block_scan_excl(int v, int* red, int parity, int* total) {
-  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+// Named barrier `id` over the first `n` threads that reach it (id 0 with the
+// whole block is __syncthreads).
+__device__ __forceinline__ void bar_sync(int id, int n) { asm volatile("bar.sync %0, %1;" ::"r"(id), "r"(n) : "memory"); }
+
+// Exclusive prefix of v over the threads of a group of nw consecutive warps
+// (warps wbase .. wbase + nw - 1, nw <= 16, synchronised by named barrier
+// `bar`) in thread order, and the group total.  `red` holds 2 x 32 ints;
+// `parity` alternates between calls so that one barrier per call suffices.
+// Every thread of the group must call it.  Out of line: one copy serves every
+// call site.
+static __device__ __noinline__ int block_scan_excl(int v, int* red, int parity, int* total, int wbase = 0,
+                                                   int nw = 16, int bar = 0) {
+  const int lane = threadIdx.x & 31, warp = (threadIdx.x >> 5) - wbase;
   int x = v;
 #pragma unroll
   for (int o = 1; o < 32; o <<= 1) {
@@ -144,15 +151,15 @@ static __device__ __noinline__ int block_scan_excl(int v, int* red, int parity, 
   }
   int* r = red + 32 * (parity & 1);
   if (lane == 31) r[warp] = x;
-  __syncthreads();
-  // lane l < 16 holds warp l's total; a scan of the 16 totals in every warp
-  int t = lane < 16 ? r[lane] : 0;
+  bar_sync(bar, nw * 32);
+  // lane l < nw holds warp l's total; a scan of the totals in every warp
+  int t = lane < nw ? r[lane] : 0;
 #pragma unroll
   for (int o = 1; o < 16; o <<= 1) {
     const int y = __shfl_up_sync(0xffffffffu, t, o);
     if (lane >= o) t += y;
   }
-  *total = __shfl_sync(0xffffffffu, t, 15);
+  *total = __shfl_sync(0xffffffffu, t, nw - 1);
   const int before = warp > 0 ? __shfl_sync(0xffffffffu, t, (warp - 1) & 31) : 0;
   return before + x - v;
 }
