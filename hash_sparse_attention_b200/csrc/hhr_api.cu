@@ -300,6 +300,7 @@ static hhr_status build_rows(const char* who, const hhr_config* cfg, const void*
   a.codes = codes;
   a.status = nullptr;
   a.max_rows = std::min(max_rows, dm.T);
+  a.wait_limit = wait_limit_cycles();
   a.stream = reinterpret_cast<cudaStream_t>(stream);
   const cudaError_t e = launch_build(a);
   if (e != cudaSuccess) {

@@ -10,12 +10,12 @@ static cudaError_t launch_build_nb(const BuildArgs& a) {
   cudaError_t e = cudaFuncSetAttribute(build_cache_kernel<NB>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
   if (e != cudaSuccess) return e;
   // rows per sequence the launch must cover: all of them, or the appended ones
-  // (they start inside a 64-row tile, hence one tile more)
-  const int span = a.max_rows + (a.starts ? BUILD_ROWS : 0);
-  const dim3 grid((span + BUILD_ROWS * BUILD_TILES - 1) / (BUILD_ROWS * BUILD_TILES), a.dm.Hkv, a.dm.B);
-  build_cache_kernel<NB><<<grid, BUILD_THREADS, smem, a.stream>>>(a.dm, a.K, a.V, a.R, a.W, a.starts, a.seq_lens,
-                                                                   a.table, a.Krot, a.Vcache, a.pmin, a.pmax,
-                                                                   a.codes, a.status);
+  // (they start inside a 128-row tile, hence one tile more)
+  const int span = a.max_rows + (a.starts ? BT_ROWS : 0);
+  const dim3 grid((span + BT_ROWS * BT_TILES - 1) / (BT_ROWS * BT_TILES), a.dm.Hkv, a.dm.B);
+  build_cache_kernel<NB><<<grid, BT_THREADS, smem, a.stream>>>(a.dm, a.K, a.V, a.R, a.W, a.starts, a.seq_lens, a.table,
+                                                               a.Krot, a.Vcache, a.pmin, a.pmax, a.codes, a.status,
+                                                               a.wait_limit);
   return cudaGetLastError();
 }
 

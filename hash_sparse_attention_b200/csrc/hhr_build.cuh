@@ -1,220 +1,406 @@
-// HHR cache build and append (sm_100a), CUDA-core version.
+// HHR cache build and append (sm_100a) on the 5th-generation tensor cores.
 //
 // For each sequence b the kernel (re)builds rows t in [S_b, L_b): S_b = 0 for
-// a full build, the old length for an append of new tokens.  Per 64-row tile
-// of one (sequence, KV head):
-//   K'  = bf16_rne(K R_h^T)          fp32 accumulation, in channel order j =
-//                                      0..127 for every row (the same
-//                                      arithmetic whatever the tile, so an
-//                                      append gives bit-identical rows)
-//   code bit j = [ (K W_h^T)_j > 0 ]  unrotated K; the fp32 sum of exact
-//                                      bf16 x bf16 products is trusted only
-//                                      when |sum| > 2^-14 |w_j| |k| (the fp32
-//                                      error is below 128 * 2^-24 sum|w k|),
+// a full build, the old length for an append of new tokens.  Per 128-row tile
+// of one (sequence, KV head), one tcgen05.mma chain per product, operands in
+// shared memory (no-swizzle K-major core-matrix layout), accumulators in TMEM:
+//   K'  = bf16_rne(K R_h^T)          R_h (fp32) as bf16 hi + mid + lo, the
+//                                      three products into one fp32
+//                                      accumulator (|R - hi - mid - lo| <=
+//                                      2^-26 |R|); an element whose
+//                                      accumulator lies within 2^-20 |k| of
+//                                      a bf16 rounding midpoint is recomputed
+//                                      in fp64 and rounded once, so K' is the
+//                                      correctly rounded product; every
+//                                      row gets the same arithmetic whatever
+//                                      its tile, so an append gives
+//                                      bit-identical rows
+//   code bit j = [ (K W_h^T)_j > 0 ]  unrotated K; the products are exact
+//                                      bf16 x bf16 and the fp32 sum is trusted
+//                                      only when |sum| > 2^-14 |w_j| |k|,
 //                                      otherwise the sign comes from fp64
 //   page min / max over the valid stored K' rows of each page; a page that
 //   began before S_b merges its stored min / max with the new rows (min and
 //   max are exact, so the result equals a build over the whole page)
 //   V rows copied to the cache unless it aliases V.
-// A CTA walks BUILD_TILES consecutive tiles so that R_h and W_h are staged
-// in shared memory once per CTA.
+// "HHR" paper card, Abstract (head-wise orthogonal transformation and
+// head-wise hash projection of the keys); rit.work explainer, section "Два
+// уровня маршрутизации решают разные ошибки" (pages of neighbouring keys with
+// stored per-channel bounds).
+//
+// A CTA (16 warps) walks BT_TILES consecutive tiles, so that R_h and W_h are
+// staged once.  Thread 0 issues the MMAs; in the epilogue warp w reads TMEM
+// lanes (rows) 32 (w mod 4) .. +31, columns of group w / 4 (a quarter of K'
+// and a quarter of the code bits).
 #pragma once
 
-#include "hhr_common.cuh"
+#include "hhr_dev.cuh"
 #include "hhr_launch.h"
 
 namespace hhr {
 
-constexpr int BUILD_THREADS = 256;
-constexpr int BUILD_ROWS = 64;
-constexpr int BUILD_TILES = 8;
+constexpr int BT_THREADS = 512;  // 16 warps: warp w reads TMEM lanes 32 (w mod 4) .. +31, column group w / 4
+constexpr int BT_ROWS = 128;   // rows per tile: the M of the MMA
+constexpr int BT_TILES = 16;   // tiles per CTA
+constexpr int BT_FIXCAP = 512; // K' elements per tile queued for the exact recompute
+
+// Byte offset of element (m, k) of a [rows][128] bf16 operand in the
+// no-swizzle K-major canonical layout: 8 x 8 core matrices of 128 bytes, the
+// 16 along K contiguous (leading byte offset 128), 8-row groups 2048 bytes
+// apart (stride byte offset).
+__host__ __device__ constexpr int bt_off(int m, int k) {
+  return (m >> 3) * 2048 + (k >> 3) * 128 + (m & 7) * 16 + (k & 7) * 2;
+}
+
+// Byte offset of element c of row r of the K' tile: 256-byte rows, their
+// 16-byte pieces XOR-swizzled by row (a warp's rows spread over the banks).
+__host__ __device__ constexpr int bt_koff(int r, int c) { return r * 256 + (((c >> 3) ^ (r & 15)) << 4) + (c & 7) * 2; }
 
 // dynamic shared memory layout of the build kernel
 struct BuildSmem {
-  static constexpr size_t kt = 0;                                    // float [D][64]
-  static constexpr size_t rt = kt + sizeof(float) * D * BUILD_ROWS;   // float [D][D]
-  static constexpr size_t ko = rt + sizeof(float) * D * D;            // bf16 [64][D]
-  static constexpr size_t wn = ko + 2 * BUILD_ROWS * D;               // float [256] |w_j|
-  static constexpr size_t kn = wn + sizeof(float) * 256;              // float [64]  |k|
-  static constexpr size_t cd = kn + sizeof(float) * BUILD_ROWS;       // u64 [64][4]
-  static constexpr size_t wt = cd + sizeof(uint64_t) * BUILD_ROWS * 4;  // bf16 [D][nb]
-  static size_t bytes(int nb) { return wt + 2 * (size_t)D * nb; }
+  static constexpr size_t rhi = 0;                        // R_h hi [128][128] bf16, canonical
+  static constexpr size_t rmid = rhi + 32768;             // R_h mid
+  static constexpr size_t rlo = rmid + 32768;             // R_h lo
+  static constexpr size_t a = rlo + 32768;                // K tile [128][128] bf16, canonical
+  static constexpr size_t ko = a + 32768;                 // K' tile [128][128] bf16, swizzled rows
+  static constexpr size_t wn = ko + 32768;                // float [256] |w_j|
+  static constexpr size_t bar = wn + 1024;                // u64 MMA-done barrier, u32 TMEM address, u32 count
+  static constexpr size_t fix = bar + 64;                 // u16 [BT_FIXCAP] K' elements (row << 7 | column)
+  static constexpr size_t kn = fix + 2 * BT_FIXCAP;       // float [128] |k| of the tile's rows
+  static constexpr size_t w = kn + 512;                   // W_h [nb][128] bf16, canonical
+  static size_t bytes(int nb) { return w + 256 * (size_t)nb; }
 };
 
+// --- tcgen05 (5th-generation tensor cores, accumulators in TMEM) -------------
+// Shared-memory matrix descriptor: start address, leading / stride byte
+// offsets (>> 4), descriptor version 1, no swizzle.
+__device__ __forceinline__ uint64_t bt_desc(const void* p) {
+  const uint32_t addr = smem_u32(p);
+  return (uint64_t)((addr >> 4) & 0x3FFF) | ((uint64_t)(128 >> 4) << 16) | ((uint64_t)(2048 >> 4) << 32) |
+         ((uint64_t)1 << 46);
+}
+// Instruction descriptor of kind::f16: bf16 A and B (K-major), fp32 D, M = 128.
+__host__ __device__ constexpr uint32_t bt_idesc(int n) {
+  return (1u << 4) | (1u << 7) | (1u << 10) | ((uint32_t)(n >> 3) << 17) | ((uint32_t)(128 >> 4) << 24);
+}
+__device__ __forceinline__ void bt_mma(uint32_t tmem, uint64_t da, uint64_t db, uint32_t idesc, bool acc) {
+  asm volatile(
+      "{\n .reg .pred p;\n setp.ne.b32 p, %4, 0;\n tcgen05.mma.cta_group::1.kind::f16 [%0], %1, %2, %3, p;\n}\n" ::"r"(
+          tmem),
+      "l"(da), "l"(db), "r"(idesc), "r"(acc ? 1u : 0u)
+      : "memory");
+}
+__device__ __forceinline__ void bt_commit(uint64_t* bar) {
+  asm volatile("tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%0];" ::"r"(smem_u32(bar))
+               : "memory");
+}
+__device__ __forceinline__ void tc_fence_before() { asm volatile("tcgen05.fence::before_thread_sync;" ::: "memory"); }
+__device__ __forceinline__ void tc_fence_after() { asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory"); }
+// 16 consecutive fp32 columns of the warp's 32 TMEM lanes (one lane per thread)
+__device__ __forceinline__ void tc_ld16(uint32_t taddr, float (&v)[16]) {
+  uint32_t r[16];
+  asm volatile(
+      "tcgen05.ld.sync.aligned.32x32b.x16.b32 {%0,%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15}, [%16];"
+      : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]), "=r"(r[7]), "=r"(r[8]),
+        "=r"(r[9]), "=r"(r[10]), "=r"(r[11]), "=r"(r[12]), "=r"(r[13]), "=r"(r[14]), "=r"(r[15])
+      : "r"(taddr)
+      : "memory");
+  asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory");
+#pragma unroll
+  for (int i = 0; i < 16; ++i) v[i] = __uint_as_float(r[i]);
+}
+
+// Exact sign of the dot product of K-tile row r and W_h row j (both bf16 in
+// the canonical layout), summed in fp64 (the products are exact).
+static __device__ __noinline__ bool bt_sign64(const unsigned char* A, const unsigned char* Bw, int r, int j) {
+  double s = 0.0;
+  #pragma unroll 1
+  for (int k = 0; k < D; ++k)
+    s += (double)__bfloat162float(*reinterpret_cast<const __nv_bfloat16*>(A + bt_off(r, k))) *
+         (double)__bfloat162float(*reinterpret_cast<const __nv_bfloat16*>(Bw + bt_off(j, k)));
+  return s > 0.0;
+}
+
+// K'[r][i] exactly: the fp64 dot product of K-tile row r (bf16) with R_h row i
+// (fp32; every product is exact in fp64), rounded once to bf16 (nearest, ties
+// to even).  For the rare elements whose fp32 accumulator lies too close to a
+// bf16 rounding midpoint to be sure of the rounding.
+static __device__ __noinline__ uint16_t bt_kexact(const unsigned char* A, const float* Ri, int r) {
+  double s = 0.0;
+  #pragma unroll 1
+  for (int k0 = 0; k0 < D; k0 += 32) {  // eight 16-byte loads of R in flight at a time
+    float4 rv[8];
+#pragma unroll
+    for (int q = 0; q < 8; ++q) rv[q] = __ldg(reinterpret_cast<const float4*>(Ri + k0) + q);
+#pragma unroll
+    for (int q = 0; q < 8; ++q) {
+      const float rr[4] = {rv[q].x, rv[q].y, rv[q].z, rv[q].w};
+#pragma unroll
+      for (int u = 0; u < 4; ++u)
+        s += (double)__bfloat162float(*reinterpret_cast<const __nv_bfloat16*>(A + bt_off(r, k0 + 4 * q + u))) *
+             (double)rr[u];
+    }
+  }
+  // the two bf16 values around s: its truncation toward zero and the next one away from zero
+  const float f = (float)s;
+  uint32_t c0 = __float_as_uint(f) >> 16;
+  // ((float)s may have rounded away from zero past a bf16 value: step back)
+  if (fabs((double)__uint_as_float(c0 << 16)) > fabs(s)) c0 -= 1u;
+  const uint32_t c1 = c0 + 1u;
+  const double d0 = fabs(s - (double)__uint_as_float(c0 << 16)), d1 = fabs(s - (double)__uint_as_float(c1 << 16));
+  const uint32_t c = d0 < d1 ? c0 : d1 < d0 ? c1 : ((c0 & 1u) ? c1 : c0);
+  return (uint16_t)c;
+}
+
 template <int NB>
-__global__ void __launch_bounds__(BUILD_THREADS)
+__global__ void __launch_bounds__(BT_THREADS, 1)
 build_cache_kernel(Dims dm, const __nv_bfloat16* K, const __nv_bfloat16* V, const float* __restrict__ R,
                    const __nv_bfloat16* __restrict__ W, const int* __restrict__ starts,
                    const int* __restrict__ seq_lens, const int* __restrict__ table, __nv_bfloat16* Krot,
                    __nv_bfloat16* Vcache, __nv_bfloat16* __restrict__ pmin, __nv_bfloat16* __restrict__ pmax,
-                   uint64_t* __restrict__ codes, int* status) {
-  constexpr int NBT = NB / 16;   // bits per thread in the code product
+                   uint64_t* __restrict__ codes, int* status, long long wait_limit) {
   constexpr int WORDS = NB / 64;
-  extern __shared__ __align__(16) unsigned char smem[];
-  float* Kt = reinterpret_cast<float*>(smem + BuildSmem::kt);
-  float* Rt = reinterpret_cast<float*>(smem + BuildSmem::rt);
-  __nv_bfloat16* Ko = reinterpret_cast<__nv_bfloat16*>(smem + BuildSmem::ko);
+  constexpr int TCOLS = NB <= 128 ? 256 : 512;  // TMEM columns: K' [0, 128), codes [128, 128 + NB)
+  extern __shared__ __align__(1024) unsigned char smem[];
+  unsigned char* Bh = smem + BuildSmem::rhi;
+  unsigned char* Bm = smem + BuildSmem::rmid;
+  unsigned char* Bl = smem + BuildSmem::rlo;
+  unsigned char* A = smem + BuildSmem::a;
+  unsigned char* Ko = smem + BuildSmem::ko;
   float* wn = reinterpret_cast<float*>(smem + BuildSmem::wn);
-  float* kn = reinterpret_cast<float*>(smem + BuildSmem::kn);
-  unsigned long long* cd = reinterpret_cast<unsigned long long*>(smem + BuildSmem::cd);
-  __nv_bfloat16* Wt = reinterpret_cast<__nv_bfloat16*>(smem + BuildSmem::wt);
+  uint64_t* bar = reinterpret_cast<uint64_t*>(smem + BuildSmem::bar);
+  uint32_t* tslot = reinterpret_cast<uint32_t*>(smem + BuildSmem::bar + 8);
+  int* nfix = reinterpret_cast<int*>(smem + BuildSmem::bar + 16);
+  uint16_t* fixq = reinterpret_cast<uint16_t*>(smem + BuildSmem::fix);
+  unsigned char* Bw = smem + BuildSmem::w;
 
-  const int h = blockIdx.y, b = blockIdx.z, tid = threadIdx.x;
+  const int h = blockIdx.y, b = blockIdx.z, tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   const int L = seq_len_of(dm, seq_lens, b);
   const int S0 = starts ? min(max(__ldg(starts + b), 0), L) : 0;  // first row (re)built
-  const int row0 = (S0 & ~(BUILD_ROWS - 1)) + blockIdx.x * BUILD_TILES * BUILD_ROWS;
+  const int row0 = (S0 & ~(BT_ROWS - 1)) + blockIdx.x * BT_TILES * BT_ROWS;
   if (row0 >= L || S0 >= L) return;
 
-  // stage R_h^T and W_h^T, and the norms of the rows of W_h
+  // ---- stage R_h as bf16 hi + mid + lo and W_h (canonical layout), the norms |w_j| ----
   const float* Rh = R + (long long)h * D * D;
-  for (int e = tid; e < D * D; e += BUILD_THREADS) {
-    const int i = e / D, j = e % D;
-    Rt[j * D + i] = __ldg(Rh + e);
+  #pragma unroll 4
+  for (int e = tid; e < D * 16; e += BT_THREADS) {
+    const int i = e >> 4, c = e & 15;
+    const float4 x0 = __ldg(reinterpret_cast<const float4*>(Rh + i * D + c * 8));
+    const float4 x1 = __ldg(reinterpret_cast<const float4*>(Rh + i * D + c * 8 + 4));
+    const float f[8] = {x0.x, x0.y, x0.z, x0.w, x1.x, x1.y, x1.z, x1.w};
+    uint32_t hi[4], mi[4], lo[4];
+#pragma unroll
+    for (int q = 0; q < 4; ++q) {  // (each residual is exact in fp32)
+      const __nv_bfloat162 h2 = __floats2bfloat162_rn(f[2 * q], f[2 * q + 1]);
+      const float2 hf = __bfloat1622float2(h2);
+      const float r0 = f[2 * q] - hf.x, r1 = f[2 * q + 1] - hf.y;
+      const __nv_bfloat162 m2 = __floats2bfloat162_rn(r0, r1);
+      const float2 mf = __bfloat1622float2(m2);
+      const __nv_bfloat162 l2 = __floats2bfloat162_rn(r0 - mf.x, r1 - mf.y);
+      hi[q] = *reinterpret_cast<const uint32_t*>(&h2);
+      mi[q] = *reinterpret_cast<const uint32_t*>(&m2);
+      lo[q] = *reinterpret_cast<const uint32_t*>(&l2);
+    }
+    *reinterpret_cast<uint4*>(Bh + bt_off(i, c * 8)) = make_uint4(hi[0], hi[1], hi[2], hi[3]);
+    *reinterpret_cast<uint4*>(Bm + bt_off(i, c * 8)) = make_uint4(mi[0], mi[1], mi[2], mi[3]);
+    *reinterpret_cast<uint4*>(Bl + bt_off(i, c * 8)) = make_uint4(lo[0], lo[1], lo[2], lo[3]);
   }
   const __nv_bfloat16* Wh = W + (long long)h * NB * D;
-  for (int e = tid; e < NB * D; e += BUILD_THREADS) {
-    const int bit = e / D, j = e % D;
-    Wt[j * NB + bit] = Wh[e];
+  #pragma unroll 4
+  for (int e = tid; e < NB * 16; e += BT_THREADS) {
+    const int j = e >> 4, c = e & 15;
+    *reinterpret_cast<uint4*>(Bw + bt_off(j, c * 8)) = ldg16(Wh + j * D + c * 8);
   }
   __syncthreads();
-  for (int bit = tid; bit < NB; bit += BUILD_THREADS) {
-    float s = 0.f;
-    for (int j = 0; j < D; ++j) { const float w = __bfloat162float(Wt[j * NB + bit]); s = fmaf(w, w, s); }
-    wn[bit] = sqrtf(s) * 1.0001f;  // a hair above |w_j| so the guard stays conservative
+  #pragma unroll 1
+  for (int j = tid; j < NB; j += BT_THREADS) {
+    float sq = 0.f;
+    #pragma unroll 4
+    for (int c = 0; c < 16; ++c) {
+      float f[8];
+      unpack8(*reinterpret_cast<const uint4*>(Bw + bt_off(j, c * 8)), f);
+#pragma unroll
+      for (int q = 0; q < 8; ++q) sq = fmaf(f[q], f[q], sq);
+    }
+    wn[j] = sqrtf(sq) * 1.0001f;  // a hair above |w_j| so the guard stays conservative
   }
+  if (warp == 0) {
+    asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(smem_u32(tslot)),
+                 "r"(TCOLS)
+                 : "memory");
+    asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;" ::: "memory");
+  }
+  if (tid == 0) {
+    mbar_init(bar, 1);
+    mbar_fence_init();
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = *tslot;
+  float* knr = reinterpret_cast<float*>(smem + BuildSmem::kn);
+  bool timed_out = false;
+  unsigned phase = 0u;
+  const int q = warp & 3, cg = warp >> 2;       // TMEM lane quarter, column group
+  const int r = 32 * q + lane;                  // the thread's row of the tile in the epilogue
+  const uint32_t tl = tmem + ((uint32_t)(32 * q) << 16);
 
-  const int kg = tid >> 4, cg = tid & 15;
-  for (int tile = 0; tile < BUILD_TILES; ++tile) {
-    const int t0 = row0 + tile * BUILD_ROWS;
+  #pragma unroll 1
+  for (int tile = 0; tile < BT_TILES; ++tile) {
+    const int t0 = row0 + tile * BT_ROWS;
     if (t0 >= L) break;
-    __syncthreads();
-    // ---- load the K tile (transposed, fp32); rows >= L are zero ----
-    for (int e = tid; e < BUILD_ROWS * (D / 8); e += BUILD_THREADS) {
-      const int r = e / (D / 8), v = e % (D / 8);
-      const int t = t0 + r;
-      float f[8] = {0, 0, 0, 0, 0, 0, 0, 0};
-      if (t >= S0 && t < L) {
-        const long long off = kv_row(dm, table, b, h, t, status);
-        if (off >= 0) unpack8(*reinterpret_cast<const uint4*>(K + off + v * 8), f);
-      }
-#pragma unroll
-      for (int c = 0; c < 8; ++c) Kt[(v * 8 + c) * BUILD_ROWS + r] = f[c];
-    }
-    for (int e = tid; e < BUILD_ROWS * 4; e += BUILD_THREADS) cd[e] = 0ull;
-    __syncthreads();
-    if (tid < BUILD_ROWS) {
-      float s = 0.f;
-      for (int j = 0; j < D; ++j) { const float x = Kt[j * BUILD_ROWS + tid]; s = fmaf(x, x, s); }
-      kn[tid] = sqrtf(s) * 1.0001f;
-    }
-
-    // ---- K' = K R^T: thread tile 4 rows x 8 channels ----
+    // ---- the K tile; rows outside [S0, L) read as zeros (a thread's 4 loads in flight together) ----
     {
-      float acc[4][8];
+      uint4 v[4];
 #pragma unroll
-      for (int a = 0; a < 4; ++a)
-#pragma unroll
-        for (int c = 0; c < 8; ++c) acc[a][c] = 0.f;
-#pragma unroll 4
-      for (int j = 0; j < D; ++j) {
-        const float4 kx = *reinterpret_cast<const float4*>(Kt + j * BUILD_ROWS + kg * 4);
-        const float4 r0 = *reinterpret_cast<const float4*>(Rt + j * D + cg * 8);
-        const float4 r1 = *reinterpret_cast<const float4*>(Rt + j * D + cg * 8 + 4);
-        const float kr[4] = {kx.x, kx.y, kx.z, kx.w};
-        const float rr[8] = {r0.x, r0.y, r0.z, r0.w, r1.x, r1.y, r1.z, r1.w};
-#pragma unroll
-        for (int a = 0; a < 4; ++a)
-#pragma unroll
-          for (int c = 0; c < 8; ++c) acc[a][c] = fmaf(kr[a], rr[c], acc[a][c]);
-      }
-#pragma unroll
-      for (int a = 0; a < 4; ++a) {
-        __align__(16) __nv_bfloat16 ob[8];
-#pragma unroll
-        for (int c = 0; c < 8; ++c) ob[c] = __float2bfloat16_rn(acc[a][c]);
-        *reinterpret_cast<uint4*>(Ko + (kg * 4 + a) * D + cg * 8) = *reinterpret_cast<const uint4*>(ob);
-      }
-    }
-    __syncthreads();
-
-    // ---- code bits: thread tile 4 rows x NBT bits ----
-    {
-      float acc[4][NBT];
-#pragma unroll
-      for (int a = 0; a < 4; ++a)
-#pragma unroll
-        for (int c = 0; c < NBT; ++c) acc[a][c] = 0.f;
-#pragma unroll 2
-      for (int j = 0; j < D; ++j) {
-        const float4 kx = *reinterpret_cast<const float4*>(Kt + j * BUILD_ROWS + kg * 4);
-        const float kr[4] = {kx.x, kx.y, kx.z, kx.w};
-        float wf[NBT];
-        const __nv_bfloat16* wrow = Wt + j * NB + cg * NBT;
-        if constexpr (NBT % 8 == 0) {
-#pragma unroll
-          for (int u = 0; u < NBT / 8; ++u) unpack8(*reinterpret_cast<const uint4*>(wrow + 8 * u), wf + 8 * u);
-        } else {
-          const uint2 v = *reinterpret_cast<const uint2*>(wrow);
-          wf[0] = bf_lo(v.x); wf[1] = bf_hi(v.x); wf[2] = bf_lo(v.y); wf[3] = bf_hi(v.y);
+      for (int i = 0; i < 4; ++i) {
+        const int e = tid + BT_THREADS * i, rr = e >> 4, c = e & 15, t = t0 + rr;
+        v[i] = make_uint4(0u, 0u, 0u, 0u);
+        if (t >= S0 && t < L) {
+          const long long off = kv_row(dm, table, b, h, t, status);
+          if (off >= 0) v[i] = ldg16(K + off + c * 8);
         }
-#pragma unroll
-        for (int a = 0; a < 4; ++a)
-#pragma unroll
-          for (int c = 0; c < NBT; ++c) acc[a][c] = fmaf(kr[a], wf[c], acc[a][c]);
       }
 #pragma unroll
-      for (int a = 0; a < 4; ++a) {
-        const int r = kg * 4 + a;
-        unsigned long long bits = 0ull;
+      for (int i = 0; i < 4; ++i) {
+        const int e = tid + BT_THREADS * i;
+        *reinterpret_cast<uint4*>(A + bt_off(e >> 4, (e & 15) * 8)) = v[i];
+      }
+    }
+    if (tid == 0) *nfix = 0;
+    fence_proxy_async();  // (the tensor cores read the tile through the async proxy)
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    // ---- K' = K R^T (lo, mid, then hi: the small terms first) and K W^T, one thread issues ----
+    if (tid == 0) {
+      #pragma unroll 1
+      for (int ks = 0; ks < 8; ++ks) bt_mma(tmem, bt_desc(A + ks * 256), bt_desc(Bl + ks * 256), bt_idesc(128), ks > 0);
+      #pragma unroll 1
+      for (int ks = 0; ks < 8; ++ks) bt_mma(tmem, bt_desc(A + ks * 256), bt_desc(Bm + ks * 256), bt_idesc(128), true);
+      #pragma unroll 1
+      for (int ks = 0; ks < 8; ++ks) bt_mma(tmem, bt_desc(A + ks * 256), bt_desc(Bh + ks * 256), bt_idesc(128), true);
+      #pragma unroll 1
+      for (int ks = 0; ks < 8; ++ks)
+        bt_mma(tmem + 128, bt_desc(A + ks * 256), bt_desc(Bw + ks * 256), bt_idesc(NB), ks > 0);
+      bt_commit(bar);
+    } else if (tid >= 32 && tid < 32 + BT_ROWS) {  // meanwhile |k| of every row of the tile
+      const int rr = tid - 32;
+      float sq = 0.f;
+      #pragma unroll 4
+      for (int c = 0; c < 16; ++c) {
+        float f[8];
+        unpack8(*reinterpret_cast<const uint4*>(A + bt_off(rr, c * 8)), f);
 #pragma unroll
-        for (int c = 0; c < NBT; ++c) {
-          const int bit = cg * NBT + c;
-          bool s;
-          if (fabsf(acc[a][c]) <= ldexpf(wn[bit] * kn[r], -14)) {
-            double x = 0.0;
-            for (int j = 0; j < D; ++j)
-              x += (double)Kt[j * BUILD_ROWS + r] * (double)__bfloat162float(Wt[j * NB + bit]);
-            s = x > 0.0;
-          } else {
-            s = acc[a][c] > 0.f;
+        for (int u = 0; u < 8; ++u) sq = fmaf(f[u], f[u], sq);
+      }
+      knr[rr] = sqrtf(sq) * 1.0001f;
+    }
+    if (!mbar_wait(bar, phase, wait_limit)) timed_out = true;
+    phase ^= 1u;
+    __syncthreads();  // (|k| of every row)
+    tc_fence_after();
+    // ---- epilogue: row r, K' columns [32 cg, 32 cg + 32), code bits [cg NB/4, (cg + 1) NB/4) ----
+    const float kn = knr[r];
+    const int t = t0 + r;
+    const bool live = t >= S0 && t < L;
+    // K' rounded to bf16.  The fp32 accumulator is within a few 2^-24 |k| of
+    // the exact value (|R_i| = 1); an element within 2^-20 |k| of a bf16
+    // rounding midpoint is queued for the exact recompute below.
+    const float kdelta = kn * 9.5367431640625e-07f;  // 2^-20
+#pragma unroll
+    for (int half = 0; half < 2; ++half) {
+      const int c0 = 32 * cg + 16 * half;
+      float v[16];
+      tc_ld16(tl + c0, v);
+      uint32_t pk[8];
+#pragma unroll
+      for (int qq = 0; qq < 8; ++qq) {
+        uint32_t e2[2];
+#pragma unroll
+        for (int u = 0; u < 2; ++u) {
+          const float x = v[2 * qq + u];
+          const float mid = __uint_as_float((__float_as_uint(x) & 0xffff0000u) | 0x8000u);
+          const __nv_bfloat16 hb = __float2bfloat16_rn(x);
+          e2[u] = *reinterpret_cast<const uint16_t*>(&hb);
+          if (fabsf(x - mid) < kdelta) {  // (in line if the queue is full)
+            const int c = c0 + 2 * qq + u;
+            const int slot = atomicAdd(nfix, 1);
+            if (slot < BT_FIXCAP) fixq[slot] = (uint16_t)((r << 7) | c);
+            else e2[u] = bt_kexact(A, R + ((long long)h * D + c) * D, r);
           }
-          bits |= (unsigned long long)s << c;
         }
-        const int bit0 = cg * NBT;
-        atomicOr(&cd[r * 4 + bit0 / 64], bits << (bit0 % 64));
+        pk[qq] = e2[0] | (e2[1] << 16);
       }
+      *reinterpret_cast<uint4*>(Ko + bt_koff(r, c0)) = make_uint4(pk[0], pk[1], pk[2], pk[3]);
+      *reinterpret_cast<uint4*>(Ko + bt_koff(r, c0 + 8)) = make_uint4(pk[4], pk[5], pk[6], pk[7]);
     }
-    __syncthreads();
-
-    // ---- write K' (and copy V), codes and page min/max ----
-    for (int e = tid; e < BUILD_ROWS * (D / 8); e += BUILD_THREADS) {
-      const int r = e / (D / 8), v = e % (D / 8);
-      const int t = t0 + r;
-      if (t >= S0 && t < L) {
-        const long long off = kv_row(dm, table, b, h, t, status);
-        if (off >= 0) {
-          *reinterpret_cast<uint4*>(Krot + off + v * 8) = *reinterpret_cast<const uint4*>(Ko + r * D + v * 8);
-          if (Vcache != V) *reinterpret_cast<uint4*>(Vcache + off + v * 8) = ldg16(V + off + v * 8);
+    // code bits of the group: trusted when |sum| > 2^-14 |w_j| |k|, else fp64
+    {
+      constexpr int NBQ = NB / 4;  // bits per column group (16, 32 or 64)
+      const float kg = kn * 6.103515625e-05f;  // 2^-14 |k|
+      uint64_t bits = 0ull;
+#pragma unroll
+      for (int c0 = 0; c0 < NBQ; c0 += 16) {
+        float v[16];
+        tc_ld16(tl + 128 + cg * NBQ + c0, v);
+#pragma unroll
+        for (int i = 0; i < 16; ++i) {
+          const int j = cg * NBQ + c0 + i;
+          bool sgn = v[i] > 0.f;
+          if (fabsf(v[i]) <= wn[j] * kg) sgn = bt_sign64(A, Bw, r, j);  // too close to zero for fp32
+          bits |= (uint64_t)sgn << (c0 + i);
         }
       }
-    }
-    for (int e = tid; e < BUILD_ROWS * WORDS; e += BUILD_THREADS) {
-      const int r = e / WORDS, w = e % WORDS;
-      const int t = t0 + r;
-      if (t >= S0 && t < L) {
+      if (live) {
         const long long off = code_row(dm, table, b, h, t, status);
-        if (off >= 0) codes[off + w] = cd[r * 4 + w];
+        if (off >= 0) {
+          unsigned char* dst = reinterpret_cast<unsigned char*>(codes + off) + cg * (NBQ / 8);
+          if constexpr (NBQ == 16) *reinterpret_cast<uint16_t*>(dst) = (uint16_t)bits;
+          else if constexpr (NBQ == 32) *reinterpret_cast<uint32_t*>(dst) = (uint32_t)bits;
+          else *reinterpret_cast<uint64_t*>(dst) = bits;
+        }
       }
     }
-    const int pages = BUILD_ROWS / dm.P;
-    for (int e = tid; e < pages * D; e += BUILD_THREADS) {
+    tc_fence_before();
+    __syncthreads();  // TMEM is free for the next tile; the queue is complete
+    #pragma unroll 1
+    for (int e = tid; e < min(*nfix, BT_FIXCAP); e += BT_THREADS) {
+      const int rr = fixq[e] >> 7, c = fixq[e] & 127;
+      const uint16_t v = bt_kexact(A, R + ((long long)h * D + c) * D, rr);
+      *reinterpret_cast<uint16_t*>(Ko + bt_koff(rr, c)) = v;
+    }
+    __syncthreads();  // the K' tile is complete
+    // ---- K' and V rows (coalesced; a thread's 4 V loads in flight), page min / max ----
+    {
+      long long offs[4];
+      uint4 vv[4];
+#pragma unroll
+      for (int i = 0; i < 4; ++i) {
+        const int e = tid + BT_THREADS * i, rr = e >> 4, c = e & 15, tt = t0 + rr;
+        offs[i] = (tt >= S0 && tt < L) ? kv_row(dm, table, b, h, tt, status) : -1;
+        if (offs[i] >= 0 && Vcache != V) vv[i] = ldg16(V + offs[i] + c * 8);
+      }
+#pragma unroll
+      for (int i = 0; i < 4; ++i) {
+        const int e = tid + BT_THREADS * i, rr = e >> 4, c = e & 15;
+        if (offs[i] >= 0) {
+          *reinterpret_cast<uint4*>(Krot + offs[i] + c * 8) = *reinterpret_cast<const uint4*>(Ko + bt_koff(rr, c * 8));
+          if (Vcache != V) *reinterpret_cast<uint4*>(Vcache + offs[i] + c * 8) = vv[i];
+        }
+      }
+    }
+    const int pages = BT_ROWS / dm.P;
+    #pragma unroll 1
+    for (int e = tid; e < pages * D; e += BT_THREADS) {
       const int pp = e / D, c = e % D;
       const int tp = t0 + pp * dm.P;
       const int r0 = max(0, S0 - tp), r1 = min(dm.P, L - tp);  // the page's rows built here
       if (r0 >= r1) continue;
       float lo = INFINITY, hi = -INFINITY;
-      for (int r = r0; r < r1; ++r) {
-        const float x = __bfloat162float(Ko[(pp * dm.P + r) * D + c]);
+      #pragma unroll 4
+      for (int rr = r0; rr < r1; ++rr) {
+        const float x = __bfloat162float(*reinterpret_cast<const __nv_bfloat16*>(Ko + bt_koff(pp * dm.P + rr, c)));
         lo = fminf(lo, x);
         hi = fmaxf(hi, x);
       }
@@ -228,7 +414,15 @@ build_cache_kernel(Dims dm, const __nv_bfloat16* K, const __nv_bfloat16* V, cons
         pmax[off + c] = __float2bfloat16_rn(hi);
       }
     }
+    // (the next tile's K-tile writes come after this tile's MMAs completed;
+    // its barrier orders the K' tile reads above before the next epilogue)
   }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  if (warp == 0)
+    asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" ::"r"(tmem), "r"(TCOLS) : "memory");
+  if (timed_out && tid == 0) set_status(status, HHR_ERR_TIMEOUT);
 }
 
 }  // namespace hhr

@@ -73,6 +73,7 @@ struct BuildArgs {
   uint64_t* codes;
   int* status;
   int max_rows;
+  long long wait_limit;  // SM clock cycles of the bounded wait for the tensor cores
   cudaStream_t stream;
 };
 cudaError_t launch_build(const BuildArgs& a);
