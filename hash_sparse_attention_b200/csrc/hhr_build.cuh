@@ -110,15 +110,25 @@ __device__ __forceinline__ void tc_ld16(uint32_t taddr, float (&v)[16]) {
   for (int i = 0; i < 16; ++i) v[i] = __uint_as_float(r[i]);
 }
 
-// Exact sign of the dot product of K-tile row r and W_h row j (both bf16 in
-// the canonical layout), summed in fp64 (the products are exact).
-static __device__ __noinline__ bool bt_sign64(const unsigned char* A, const unsigned char* Bw, int r, int j) {
-  double s = 0.0;
-  #pragma unroll 1
-  for (int k = 0; k < D; ++k)
-    s += (double)__bfloat162float(*reinterpret_cast<const __nv_bfloat16*>(A + bt_off(r, k))) *
-         (double)__bfloat162float(*reinterpret_cast<const __nv_bfloat16*>(Bw + bt_off(j, k)));
-  return s > 0.0;
+// fp64 partial dot product of K-tile row r and W_h row j (both bf16 in the
+// canonical layout) over k = 4 lane .. 4 lane + 3; the products are exact.
+__device__ __forceinline__ double bt_dot4(const unsigned char* A, const unsigned char* Bw, int r, int j, int lane) {
+  const uint2 a = *reinterpret_cast<const uint2*>(A + bt_off(r, 4 * lane));
+  const uint2 w = *reinterpret_cast<const uint2*>(Bw + bt_off(j, 4 * lane));
+  return (double)bf_lo(a.x) * bf_lo(w.x) + (double)bf_hi(a.x) * bf_hi(w.x) + (double)bf_lo(a.y) * bf_lo(w.y) +
+         (double)bf_hi(a.y) * bf_hi(w.y);
+}
+
+// The bf16 value nearest to s (ties to even), from the two bf16 values around
+// s: its truncation toward zero and the next one away from zero.
+__device__ __forceinline__ uint16_t bt_round_bf16(double s) {
+  const float f = (float)s;
+  uint32_t c0 = __float_as_uint(f) >> 16;
+  // ((float)s may have rounded away from zero past a bf16 value: step back)
+  if (fabs((double)__uint_as_float(c0 << 16)) > fabs(s)) c0 -= 1u;
+  const uint32_t c1 = c0 + 1u;
+  const double d0 = fabs(s - (double)__uint_as_float(c0 << 16)), d1 = fabs(s - (double)__uint_as_float(c1 << 16));
+  return (uint16_t)(d0 < d1 ? c0 : d1 < d0 ? c1 : ((c0 & 1u) ? c1 : c0));
 }
 
 // K'[r][i] exactly: the fp64 dot product of K-tile row r (bf16) with R_h row i
@@ -141,15 +151,62 @@ static __device__ __noinline__ uint16_t bt_kexact(const unsigned char* A, const 
              (double)rr[u];
     }
   }
-  // the two bf16 values around s: its truncation toward zero and the next one away from zero
-  const float f = (float)s;
-  uint32_t c0 = __float_as_uint(f) >> 16;
-  // ((float)s may have rounded away from zero past a bf16 value: step back)
-  if (fabs((double)__uint_as_float(c0 << 16)) > fabs(s)) c0 -= 1u;
-  const uint32_t c1 = c0 + 1u;
-  const double d0 = fabs(s - (double)__uint_as_float(c0 << 16)), d1 = fabs(s - (double)__uint_as_float(c1 << 16));
-  const uint32_t c = d0 < d1 ? c0 : d1 < d0 ? c1 : ((c0 & 1u) ? c1 : c0);
-  return (uint16_t)c;
+  return bt_round_bf16(s);
+}
+
+// The queued K' elements (row << 7 | column), four lanes per element: lane g
+// of a group sums k in [32 g, 32 g + 32) in fp64, the group adds its partial
+// sums by shuffles and the result is rounded once.  A lane takes two elements
+// per pass, their R loads in flight together.
+static __device__ __noinline__ void bt_fixups(const unsigned char* A, const float* __restrict__ Rh,
+                                              const uint16_t* fixq, int n, unsigned char* Ko, int warp, int lane) {
+  constexpr int PER = BT_THREADS / 4;  // elements per half pass
+  const int g = lane & 3;
+  #pragma unroll 1
+  for (int base = 8 * warp; base < n; base += 2 * PER) {  // (warp-uniform trip count)
+    int ent[2];
+    float4 x[2][8];
+#pragma unroll
+    for (int u = 0; u < 2; ++u) {
+      const int e = base + u * PER + (lane >> 2);
+      ent[u] = e < n ? (int)fixq[e] : -1;
+      const float4* Rp = reinterpret_cast<const float4*>(Rh + (ent[u] < 0 ? 0 : ent[u] & 127) * D + 32 * g);
+#pragma unroll
+      for (int v = 0; v < 8; ++v) x[u][v] = __ldg(Rp + v);
+    }
+#pragma unroll
+    for (int u = 0; u < 2; ++u) {
+      const int r = ent[u] < 0 ? 0 : ent[u] >> 7;
+      double s = 0.0;
+#pragma unroll
+      for (int v = 0; v < 4; ++v) {
+        float a[8];
+        unpack8(*reinterpret_cast<const uint4*>(A + bt_off(r, 32 * g + 8 * v)), a);
+        s += (double)a[0] * x[u][2 * v].x + (double)a[1] * x[u][2 * v].y + (double)a[2] * x[u][2 * v].z +
+             (double)a[3] * x[u][2 * v].w + (double)a[4] * x[u][2 * v + 1].x + (double)a[5] * x[u][2 * v + 1].y +
+             (double)a[6] * x[u][2 * v + 1].z + (double)a[7] * x[u][2 * v + 1].w;
+      }
+      s += __shfl_xor_sync(0xffffffffu, s, 1);
+      s += __shfl_xor_sync(0xffffffffu, s, 2);
+      if (ent[u] >= 0 && g == 0) *reinterpret_cast<uint16_t*>(Ko + bt_koff(r, ent[u] & 127)) = bt_round_bf16(s);
+    }
+  }
+}
+
+// Issue the copies of K tile rows t0 .. t0 + 127 into the canonical layout
+// (cp.async, one commit group); rows outside [S0, L) are zeros.
+__device__ __forceinline__ void bt_issue_k(const Dims& dm, const int* __restrict__ table, int b, int h, int t0,
+                                           int S0, int L, const __nv_bfloat16* K, unsigned char* A, int tid,
+                                           int* status) {
+#pragma unroll
+  for (int i = 0; i < 4; ++i) {
+    const int e = tid + BT_THREADS * i, rr = e >> 4, c = e & 15, t = t0 + rr;
+    unsigned char* dst = A + bt_off(rr, c * 8);
+    const long long off = (t >= S0 && t < L) ? kv_row(dm, table, b, h, t, status) : -1;
+    if (off >= 0) cp_async16(dst, K + off + c * 8);
+    else *reinterpret_cast<uint4*>(dst) = make_uint4(0u, 0u, 0u, 0u);
+  }
+  cp_async_commit();
 }
 
 template <int NB>
@@ -159,7 +216,6 @@ build_cache_kernel(Dims dm, const __nv_bfloat16* K, const __nv_bfloat16* V, cons
                    const int* __restrict__ seq_lens, const int* __restrict__ table, __nv_bfloat16* Krot,
                    __nv_bfloat16* Vcache, __nv_bfloat16* __restrict__ pmin, __nv_bfloat16* __restrict__ pmax,
                    uint64_t* __restrict__ codes, int* status, long long wait_limit) {
-  constexpr int WORDS = NB / 64;
   constexpr int TCOLS = NB <= 128 ? 256 : 512;  // TMEM columns: K' [0, 128), codes [128, 128 + NB)
   extern __shared__ __align__(1024) unsigned char smem[];
   unsigned char* Bh = smem + BuildSmem::rhi;
@@ -245,28 +301,12 @@ build_cache_kernel(Dims dm, const __nv_bfloat16* K, const __nv_bfloat16* V, cons
   const int r = 32 * q + lane;                  // the thread's row of the tile in the epilogue
   const uint32_t tl = tmem + ((uint32_t)(32 * q) << 16);
 
+  bt_issue_k(dm, table, b, h, row0, S0, L, K, A, tid, status);
   #pragma unroll 1
   for (int tile = 0; tile < BT_TILES; ++tile) {
     const int t0 = row0 + tile * BT_ROWS;
     if (t0 >= L) break;
-    // ---- the K tile; rows outside [S0, L) read as zeros (a thread's 4 loads in flight together) ----
-    {
-      uint4 v[4];
-#pragma unroll
-      for (int i = 0; i < 4; ++i) {
-        const int e = tid + BT_THREADS * i, rr = e >> 4, c = e & 15, t = t0 + rr;
-        v[i] = make_uint4(0u, 0u, 0u, 0u);
-        if (t >= S0 && t < L) {
-          const long long off = kv_row(dm, table, b, h, t, status);
-          if (off >= 0) v[i] = ldg16(K + off + c * 8);
-        }
-      }
-#pragma unroll
-      for (int i = 0; i < 4; ++i) {
-        const int e = tid + BT_THREADS * i;
-        *reinterpret_cast<uint4*>(A + bt_off(e >> 4, (e & 15) * 8)) = v[i];
-      }
-    }
+    cp_async_wait_all();  // this tile's K (issued before the previous tile's copy-out)
     if (tid == 0) *nfix = 0;
     fence_proxy_async();  // (the tensor cores read the tile through the async proxy)
     tc_fence_before();
@@ -339,18 +379,33 @@ build_cache_kernel(Dims dm, const __nv_bfloat16* K, const __nv_bfloat16* V, cons
     {
       constexpr int NBQ = NB / 4;  // bits per column group (16, 32 or 64)
       const float kg = kn * 6.103515625e-05f;  // 2^-14 |k|
-      uint64_t bits = 0ull;
+      uint64_t bits = 0ull, fb = 0ull;  // fb: bits whose sign fp32 cannot decide
 #pragma unroll
       for (int c0 = 0; c0 < NBQ; c0 += 16) {
         float v[16];
         tc_ld16(tl + 128 + cg * NBQ + c0, v);
 #pragma unroll
         for (int i = 0; i < 16; ++i) {
-          const int j = cg * NBQ + c0 + i;
-          bool sgn = v[i] > 0.f;
-          if (fabsf(v[i]) <= wn[j] * kg) sgn = bt_sign64(A, Bw, r, j);  // too close to zero for fp32
-          bits |= (uint64_t)sgn << (c0 + i);
+          const bool near0 = fabsf(v[i]) <= wn[cg * NBQ + c0 + i] * kg;
+          fb |= (uint64_t)near0 << (c0 + i);
+          bits |= (uint64_t)(v[i] > 0.f && !near0) << (c0 + i);
         }
+      }
+      // those signs from fp64, one bit at a time for the whole warp (each
+      // lane sums 4 of the 128 exact products)
+      unsigned any = __ballot_sync(0xffffffffu, fb != 0ull);
+      #pragma unroll 1
+      while (any) {
+        const int src = __ffs(any) - 1;
+        const int bit = __ffsll((long long)__shfl_sync(0xffffffffu, fb, src)) - 1;
+        double sd = bt_dot4(A, Bw, 32 * q + src, cg * NBQ + bit, lane);
+#pragma unroll
+        for (int o = 16; o >= 1; o >>= 1) sd += __shfl_xor_sync(0xffffffffu, sd, o);
+        if (lane == src) {
+          bits |= (uint64_t)(sd > 0.0) << bit;
+          fb &= fb - 1ull;
+        }
+        any = __ballot_sync(0xffffffffu, fb != 0ull);
       }
       if (live) {
         const long long off = code_row(dm, table, b, h, t, status);
@@ -364,13 +419,9 @@ build_cache_kernel(Dims dm, const __nv_bfloat16* K, const __nv_bfloat16* V, cons
     }
     tc_fence_before();
     __syncthreads();  // TMEM is free for the next tile; the queue is complete
-    #pragma unroll 1
-    for (int e = tid; e < min(*nfix, BT_FIXCAP); e += BT_THREADS) {
-      const int rr = fixq[e] >> 7, c = fixq[e] & 127;
-      const uint16_t v = bt_kexact(A, R + ((long long)h * D + c) * D, rr);
-      *reinterpret_cast<uint16_t*>(Ko + bt_koff(rr, c)) = v;
-    }
-    __syncthreads();  // the K' tile is complete
+    bt_fixups(A, Rh, fixq, min(*nfix, BT_FIXCAP), Ko, warp, lane);
+    __syncthreads();  // the K' tile is complete; nothing reads this K tile any more
+    if (tile + 1 < BT_TILES && t0 + BT_ROWS < L) bt_issue_k(dm, table, b, h, t0 + BT_ROWS, S0, L, K, A, tid, status);
     // ---- K' and V rows (coalesced; a thread's 4 V loads in flight), page min / max ----
     {
       long long offs[4];
@@ -417,6 +468,7 @@ build_cache_kernel(Dims dm, const __nv_bfloat16* K, const __nv_bfloat16* V, cons
     // (the next tile's K-tile writes come after this tile's MMAs completed;
     // its barrier orders the K' tile reads above before the next epilogue)
   }
+  cp_async_wait_all();
   tc_fence_before();
   __syncthreads();
   tc_fence_after();
