@@ -8,14 +8,15 @@
 // keeps the top-k, then exact attention runs over the kept keys.
 //
 // Per unit, CTA r of the group:
-//   1. copies the query heads and the first two of its 64-page metadata
-//      stages (cp.async; pages [p0, p1), five stages in flight), then computes
-//      q' = R_h q and the query sign codes on tensor cores (R_h and W_h of the
-//      first unit are copied to shared memory before the previous kernel on
-//      the stream has finished: programmatic dependent launch);
+//   1. starts the first two of its 64-page metadata stages (pages [p0, p1);
+//      TMA bulk copies completing on one mbarrier per stage, five stages in
+//      flight) and copies the query heads, then computes q' = R_h q and the
+//      query sign codes on tensor cores (R_h and W_h of the first unit are
+//      copied to shared memory before the previous kernel on the stream has
+//      finished: programmatic dependent launch);
 //   2. scans its pages: U = the page bound aggregated over the group's query
-//      heads (max, or sum).  Every thread consumes exactly the 16-byte pieces
-//      it copied, so the scan needs no CTA barrier;
+//      heads (max, or sum); a stage's slot is refilled once every thread is
+//      done with it, and every wait on a stage's barrier is bounded;
 //   3. group barrier; the page top-N on ALL the unit's bounds (read from
 //      L2), the same in every CTA: order-preserving keys in registers, a level
 //      over the keys' range, then the threshold bin's members refined 11 bits

@@ -67,9 +67,10 @@ def test_max_over_ranks_gloo_two_ranks():
     assert got == [(0, 2.0), (1, 2.0)]
 
 
-def test_build_report_counts_rows_bytes_and_fma():
-    """The cache-build line: median over layers after the first, fp32 FMA and
-    HBM ceilings from the unit counts (no GPU needed)."""
+def test_build_report_counts_rows_bytes_and_flops():
+    """The cache-build line: median over layers after the first, the HBM
+    ceiling from the bytes the build must move and the tensor-core ceiling
+    from the projection flops (no GPU needed)."""
     import bench
     from hash_sparse_attention_b200.synth import WORKLOADS
 
@@ -82,15 +83,21 @@ def test_build_report_counts_rows_bytes_and_fma():
 
     w = WORKLOADS["llama_32l_128k"]
     ev = [(Ev(0.0), Ev(9.0)), (Ev(0.0), Ev(4.0)), (Ev(0.0), Ev(2.0)), (Ev(0.0), Ev(3.0))]
-    r = bench.build_report(w, [{"lens": [131072]}], ev, {"sm_max_mhz": 2000.0}, 100, {"hbm_gbs": 1000.0})
+    r = bench.build_report(w, [{"lens": [131072]}], ev, {"sm_max_mhz": 2000.0}, 100,
+                           {"hbm_gbs": 1000.0, "bf16_tflops": 500.0, "source": "measured"})
     assert r["ms_per_layer"] == 3.0  # median of 4, 2, 3 (the first layer is left out)
     rows = 8 * 131072
     assert r["rows_per_layer"] == rows
-    assert r["fma_per_layer"] == rows * 128 * (128 + 128)
     pages = 8 * 131072 // 16
-    assert r["algorithmic_bytes_per_layer"] == rows * (512 + 16) + pages * 512 + 8 * (128 * 128 * 4 + 128 * 128 * 2)
-    assert abs(r["peak"] - 100 * 128 * 2000e6 / 1e12) < 1e-9
-    assert abs(r["frac"] - r["fma_per_layer"] / 3e-3 / (100 * 128 * 2000e6)) < 1e-12
+    nbytes = rows * (512 + 16) + pages * 512 + 8 * (128 * 128 * 4 + 128 * 128 * 2)
+    assert r["algorithmic_bytes_per_layer"] == nbytes
+    assert r["bound"] == "hbm" and r["peak"] == 1000.0
+    assert abs(r["achieved"] - nbytes / 3e-3 / 1e9) < 1e-6
+    assert abs(r["frac"] - r["achieved"] / 1000.0) < 1e-12
+    t = r["tensor"]
+    assert t["flops_per_layer"] == 2 * rows * 128 * (128 + 128)
+    assert t["issued_flops_per_layer"] == 2 * rows * 128 * (3 * 128 + 128)
+    assert abs(t["frac"] - t["flops_per_layer"] / 3e-3 / 1e12 / 500.0) < 1e-12
 
 
 def test_profiled_traffic_only_for_matching_sources_and_workload(tmp_path, monkeypatch):
