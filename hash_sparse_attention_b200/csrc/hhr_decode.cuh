@@ -1322,6 +1322,23 @@ __global__ void __launch_bounds__(SP_THREADS, 1) hhr_sparse_kernel(const __grid_
     const int ncs = nkp << dm.lgP;
     const bool conc = all_kept && wk.HB * 4 + 2 * ((ncs + S - 1) / S) <= 2 * SP_KLCAP;
     int j0 = 0, j1 = 0, mine = 0;
+    if (conc) {  // the scoring share's code rows go out ahead of the tile copies
+      if (!gw) {
+        int c0, c1;
+        share_of(ncs, S, r, c0, c1);
+        const int pa = c0 >> dm.lgP, pb = c1 > c0 ? ((c1 - 1) >> dm.lgP) + 1 : pa;
+        const int lines = (dm.P * WORDS * 8 + 127) >> 7;  // 128-byte lines of a page's code rows
+        #pragma unroll 1
+        for (int e = tid - TL_WARPS * 32; e < (pb - pa) * lines; e += SP_THREADS - TL_WARPS * 32) {
+          const int pg = kp[pa + e / lines];
+          const long long off = pg * dm.P < x.L ? code_row(dm, p.table, x.b, x.h, pg * dm.P, p.status) : -1;
+          if (off >= 0) prefetch_l2(p.codes + off + (e % lines) * 16);
+        }
+        bar_arrive(3, SP_THREADS);
+      } else {
+        bar_sync(3, SP_THREADS);
+      }
+    }
     if (all_kept) {
       share_of(keff, S, r, j0, j1);
       const int ntile = (j1 - j0 + TL_ROWS - 1) / TL_ROWS;

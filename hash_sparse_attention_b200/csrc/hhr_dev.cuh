@@ -133,6 +133,11 @@ __device__ __forceinline__ void split_bf16(float x, __nv_bfloat16& hi, __nv_bflo
 // Named barrier `id` over the first `n` threads that reach it (id 0 with the
 // whole block is __syncthreads).
 __device__ __forceinline__ void bar_sync(int id, int n) { asm volatile("bar.sync %0, %1;" ::"r"(id), "r"(n) : "memory"); }
+// arrive at named barrier id without waiting (the other n - 32 k threads wait in bar_sync)
+__device__ __forceinline__ void bar_arrive(int id, int n) {
+  asm volatile("bar.arrive %0, %1;" ::"r"(id), "r"(n) : "memory");
+}
+__device__ __forceinline__ void prefetch_l2(const void* p) { asm volatile("prefetch.global.L2 [%0];" ::"l"(p)); }
 
 // Exclusive prefix of v over the threads of a group of nw consecutive warps
 // (warps wbase .. wbase + nw - 1, nw <= 16, synchronised by named barrier
