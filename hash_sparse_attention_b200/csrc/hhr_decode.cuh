@@ -837,28 +837,35 @@ __device__ void tile_combine(unsigned char* sm, const float (&o)[16][4], float m
     }
   }
   __syncthreads();
+  // the warps' scale factors: thread 8 hh + w (hh < 8 heads, w < 8 warps)
+  float* scl = wsm + TL_WARPS * 8 * WS;  // [8 heads][8 warps]
+  if (tid < 64) {
+    const int hh = tid >> 3, w = tid & 7;
+    const float m = wsm[(w * 8 + hh) * WS + D];
+    float M = m;
+    M = fmaxf(M, __shfl_xor_sync(0xffffffffu, M, 1));
+    M = fmaxf(M, __shfl_xor_sync(0xffffffffu, M, 2));
+    M = fmaxf(M, __shfl_xor_sync(0xffffffffu, M, 4));
+    const float sc = M == -INFINITY ? 0.f : exp2f(m - M);  // 0 for a warp without rows
+    scl[tid] = sc;
+    const float lw = sc * wsm[(w * 8 + hh) * WS + D + 1];
+    float Ls = 0.f;  // in warp order
+#pragma unroll
+    for (int v = 0; v < TL_WARPS; ++v) Ls += __shfl_sync(0xffffffffu, lw, (lane & ~7) + v);
+    if (write && w == 0 && hh < G) {
+      part[G * D + hh] = M;
+      part[G * D + 8 + hh] = Ls;
+    }
+  }
+  __syncthreads();
   if (write) {
 #pragma unroll 1
     for (int e = tid; e < G * D; e += blockDim.x) {
       const int hh = e >> 7, c = e & (D - 1);
-      float M = -INFINITY;
+      float acc = 0.f;
 #pragma unroll
-      for (int w = 0; w < TL_WARPS; ++w) M = fmaxf(M, wsm[(w * 8 + hh) * WS + D]);
-      float acc = 0.f, Ls = 0.f;
-      if (M != -INFINITY) {
-#pragma unroll
-        for (int w = 0; w < TL_WARPS; ++w) {
-          const float* wr = wsm + (w * 8 + hh) * WS;
-          const float sc = exp2f(wr[D] - M);  // 0 for a warp without rows
-          acc = fmaf(sc, wr[c], acc);
-          Ls = fmaf(sc, wr[D + 1], Ls);
-        }
-      }
+      for (int w = 0; w < TL_WARPS; ++w) acc = fmaf(scl[hh * 8 + w], wsm[(w * 8 + hh) * WS + c], acc);
       part[e] = acc;
-      if (c == 0) {
-        part[G * D + hh] = M;
-        part[G * D + 8 + hh] = Ls;
-      }
     }
   }
   __syncthreads();
@@ -1149,10 +1156,14 @@ __device__ void sp_merge(const SpParams& p, unsigned char* sm, const SpUnit& x, 
     for (int i = tid; i < n16; i += SP_THREADS) cp_async16(sp + 4 * i, pt + 4 * i);
     cp_async_commit();
   }
-  if (warp < G) {  // warp h: the weights of head h
+  // warp h: the weights of head h, from the partials' (max, sum) pairs: in
+  // shared memory when every partial fits one pass, else read through L2
+  // (written by the other CTAs of the group)
+  auto weights = [&](const float* src, bool l2) {
+    auto ld = [&](long long i) { return l2 ? __ldcg(src + i) : src[i]; };
     float M = -INFINITY;
 #pragma unroll 1
-    for (int k = lane; k < n; k += 32) M = fmaxf(M, __ldcg(pt + (long long)k * PS + G * D + warp));
+    for (int k = lane; k < n; k += 32) M = fmaxf(M, ld((long long)k * PS + G * D + warp));
 #pragma unroll
     for (int o = 16; o >= 1; o >>= 1) M = fmaxf(M, __shfl_xor_sync(0xffffffffu, M, o));
     float tot = 0.f;
@@ -1161,17 +1172,19 @@ __device__ void sp_merge(const SpParams& p, unsigned char* sm, const SpUnit& x, 
       const int k = k0 + lane;
       float wl = 0.f;
       if (k < n) {
-        const float mk = __ldcg(pt + (long long)k * PS + G * D + warp);
+        const float mk = ld((long long)k * PS + G * D + warp);
         const float w = mk == -INFINITY ? 0.f : exp2f(mk - M);
         wbuf[k * 8 + warp] = w;
-        wl = w * __ldcg(pt + (long long)k * PS + G * D + 8 + warp);
+        wl = w * ld((long long)k * PS + G * D + 8 + warp);
       }
 #pragma unroll
       for (int o = 16; o >= 1; o >>= 1) wl += __shfl_xor_sync(0xffffffffu, wl, o);
       tot += wl;
     }
     if (lane == 0) inv[warp] = 1.f / tot;
-  }
+  };
+  const bool one_pass = n <= per;
+  if (!one_pass && warp < G) weights(pt, true);
   float acc0 = 0.f, acc1 = 0.f;  // elements tid and tid + 512 (G * 128 <= 1024)
 #pragma unroll 1
   for (int k0 = 0; k0 < n; k0 += per) {
@@ -1184,6 +1197,10 @@ __device__ void sp_merge(const SpParams& p, unsigned char* sm, const SpUnit& x, 
     }
     cp_async_wait_all();
     __syncthreads();
+    if (one_pass) {
+      if (warp < G) weights(sp, false);
+      __syncthreads();
+    }
 #pragma unroll 1
     for (int k = 0; k < nk; ++k) {
       const float* pk = sp + k * PS;
