@@ -193,6 +193,38 @@ static __device__ __noinline__ void bt_fixups(const unsigned char* A, const floa
   }
 }
 
+// The same recompute with R_h row c read back from its three staged bf16
+// terms (their fp32 sum is R_h's element exactly whenever the staging found
+// every split exact, which it checks), so that no global load is needed.
+static __device__ __noinline__ void bt_fixups_smem(const unsigned char* A, const unsigned char* Bh,
+                                                   const unsigned char* Bm, const unsigned char* Bl,
+                                                   const uint16_t* fixq, int n, unsigned char* Ko, int warp,
+                                                   int lane) {
+  constexpr int PER = BT_THREADS / 4;
+  const int g = lane & 3;
+  #pragma unroll 1
+  for (int base = 8 * warp; base < n; base += PER) {  // (warp-uniform trip count)
+    const int e = base + (lane >> 2);
+    const int ent = e < n ? (int)fixq[e] : 0;
+    const int r = ent >> 7, c = ent & 127;
+    double s = 0.0;
+#pragma unroll
+    for (int v = 0; v < 4; ++v) {
+      const int k = 32 * g + 8 * v;
+      float a[8], h[8], m[8], l[8];
+      unpack8(*reinterpret_cast<const uint4*>(A + bt_off(r, k)), a);
+      unpack8(*reinterpret_cast<const uint4*>(Bh + bt_off(c, k)), h);
+      unpack8(*reinterpret_cast<const uint4*>(Bm + bt_off(c, k)), m);
+      unpack8(*reinterpret_cast<const uint4*>(Bl + bt_off(c, k)), l);
+#pragma unroll
+      for (int u = 0; u < 8; ++u) s += (double)a[u] * (double)((h[u] + m[u]) + l[u]);
+    }
+    s += __shfl_xor_sync(0xffffffffu, s, 1);
+    s += __shfl_xor_sync(0xffffffffu, s, 2);
+    if (e < n && g == 0) *reinterpret_cast<uint16_t*>(Ko + bt_koff(r, c)) = bt_round_bf16(s);
+  }
+}
+
 // Issue the copies of K tile rows t0 .. t0 + 127 into the canonical layout
 // (cp.async, one commit group); rows outside [S0, L) are zeros.
 __device__ __forceinline__ void bt_issue_k(const Dims& dm, const int* __restrict__ table, int b, int h, int t0,
@@ -238,6 +270,7 @@ build_cache_kernel(Dims dm, const __nv_bfloat16* K, const __nv_bfloat16* V, cons
 
   // ---- stage R_h as bf16 hi + mid + lo and W_h (canonical layout), the norms |w_j| ----
   const float* Rh = R + (long long)h * D * D;
+  int inexact = 0;  // an element whose three terms do not add back to it in fp32
   #pragma unroll 4
   for (int e = tid; e < D * 16; e += BT_THREADS) {
     const int i = e >> 4, c = e & 15;
@@ -253,6 +286,8 @@ build_cache_kernel(Dims dm, const __nv_bfloat16* K, const __nv_bfloat16* V, cons
       const __nv_bfloat162 m2 = __floats2bfloat162_rn(r0, r1);
       const float2 mf = __bfloat1622float2(m2);
       const __nv_bfloat162 l2 = __floats2bfloat162_rn(r0 - mf.x, r1 - mf.y);
+      const float2 lf = __bfloat1622float2(l2);
+      if ((hf.x + mf.x) + lf.x != f[2 * q] || (hf.y + mf.y) + lf.y != f[2 * q + 1]) inexact = 1;
       hi[q] = *reinterpret_cast<const uint32_t*>(&h2);
       mi[q] = *reinterpret_cast<const uint32_t*>(&m2);
       lo[q] = *reinterpret_cast<const uint32_t*>(&l2);
@@ -267,7 +302,7 @@ build_cache_kernel(Dims dm, const __nv_bfloat16* K, const __nv_bfloat16* V, cons
     const int j = e >> 4, c = e & 15;
     *reinterpret_cast<uint4*>(Bw + bt_off(j, c * 8)) = ldg16(Wh + j * D + c * 8);
   }
-  __syncthreads();
+  const bool split_exact = !__syncthreads_or(inexact);
   #pragma unroll 1
   for (int j = tid; j < NB; j += BT_THREADS) {
     float sq = 0.f;
@@ -419,7 +454,8 @@ build_cache_kernel(Dims dm, const __nv_bfloat16* K, const __nv_bfloat16* V, cons
     }
     tc_fence_before();
     __syncthreads();  // TMEM is free for the next tile; the queue is complete
-    bt_fixups(A, Rh, fixq, min(*nfix, BT_FIXCAP), Ko, warp, lane);
+    if (split_exact) bt_fixups_smem(A, Bh, Bm, Bl, fixq, min(*nfix, BT_FIXCAP), Ko, warp, lane);
+    else bt_fixups(A, Rh, fixq, min(*nfix, BT_FIXCAP), Ko, warp, lane);
     __syncthreads();  // the K' tile is complete; nothing reads this K tile any more
     if (tile + 1 < BT_TILES && t0 + BT_ROWS < L) bt_issue_k(dm, table, b, h, t0 + BT_ROWS, S0, L, K, A, tid, status);
     // ---- K' and V rows (coalesced; a thread's 4 V loads in flight), page min / max ----
