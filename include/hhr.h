@@ -127,7 +127,11 @@ HHR_API void hhr_set_wait_limit(int64_t cycles);
  * two-level routing section); pages keep what their bound needs; LHP keys
  * get sign codes (paper page, Figure 2 caption: projection then sign).
  * For every sequence b, KV head h and row t < seq_lens[b]:
- *   Krot[t] = bf16_rne(R_h K[t])                 (fp32 accumulation)
+ *   Krot[t] = bf16_rne(R_h K[t])                 (the exact product rounded
+ *                                                 once: tensor-core fp32
+ *                                                 accumulation, elements near
+ *                                                 a rounding midpoint
+ *                                                 recomputed in fp64)
  *   codes[t] bit j = [ (W_h K[t])_j > 0 ]        (unrotated K; bit j in word
  *                                                 j/64 at position j%64; the
  *                                                 sign is exact: near-zero

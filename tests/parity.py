@@ -10,8 +10,7 @@ within tolerance where the selections agree.
 Tolerances and exemptions:
   * attention output: per query head max|o - o^| / max|o^| <= 2e-3
   * page bounds: |ub - ub^| <= 2e-3 * sum_i |q'_i| max(|mn_i|, |mx_i|)
-  * K': within one bf16 ulp of the fp64-rounded value plus the fp32
-    accumulation bound 2^-16 * sum_j |R_ij k_j|
+  * K': equal, bit for bit, to the oracle's bf16_rne(R_h k)
   * a hash bit is exempt when |fp64 projection| < 1e-5 |x|; a page is exempt
     when |U_p - thr| <= 1e-4 |thr| (thr = the N-th largest fp64 bound)
 """
@@ -122,11 +121,6 @@ def run_gpu(w: Workload, li: LayerInputs, max_keep: int | None = None, max_topk:
                   d, int(status.item()), Nmax, Kmax)
 
 
-def _bf16_ulp(x: np.ndarray) -> np.ndarray:
-    ax = np.maximum(np.abs(x), 2.0 ** -126)
-    return 2.0 ** (np.floor(np.log2(ax)) - 7)
-
-
 def rel_err(a: np.ndarray, ref: np.ndarray) -> float:
     den = np.abs(ref).max()
     return float(np.abs(a - ref).max() / den) if den > 0 else float(np.abs(a).max())
@@ -165,11 +159,9 @@ def check_build(w: Workload, li: LayerInputs, g: GpuRun, rep: Report, heads=None
             diff = Kp != Kp_ref
             rep.kprime_flips += int(diff.sum())
             rep.kprime_elems += diff.size
-            # fp32 accumulation: the unrounded value may be off by gamma_128 * sum|R_ij k_j|
-            # (about 2^-17 of it), then rounding to bf16 adds at most one ulp
-            acc_err = 2.0 ** -16 * (np.abs(Kx) @ np.abs(R32[h]).T)
-            assert np.all(np.abs(Kp - Kp_ref) <= _bf16_ulp(Kp_ref) * 1.0000001 + acc_err), \
-                "K' off by more than one bf16 ulp plus the fp32 accumulation bound"
+            # the build rounds the exact product once (elements near a rounding
+            # midpoint are recomputed in fp64), so K' equals the oracle's bit for bit
+            assert np.array_equal(Kp, Kp_ref), f"K' differs from bf16_rne(R_h k) in {int(diff.sum())} elements"
             # page metadata: stage-wise on the GPU's stored K'
             mn, mx = O.page_minmax(Kp, L, P)
             n = mn.shape[0]
@@ -184,8 +176,6 @@ def check_build(w: Workload, li: LayerInputs, g: GpuRun, rep: Report, heads=None
             assert not np.any(mism & ~exempt), f"key code mismatch outside the exempt band b{b} h{h}"
             rep.code_exempt_bits += int(exempt.sum())
             rep.code_exempt_mismatch += int((mism & exempt).sum())
-    if rep.kprime_elems:
-        assert rep.kprime_flips <= 1e-3 * rep.kprime_elems, f"too many K' rounding flips {rep.kprime_flips}"
 
 
 def _bits(words: np.ndarray, nb: int) -> np.ndarray:

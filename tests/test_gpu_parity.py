@@ -279,3 +279,18 @@ def test_group_aggregation_modes(G, page_agg, key_agg):
                page_agg=page_agg, key_agg=key_agg, seed=100 + G)
     li = make_layer(w)
     _run_and_check(w, li)
+
+
+def test_build_exact_when_the_rotation_split_is_inexact():
+    """K' stays the correctly rounded product when some entries of R_h are
+    fp32 subnormals, whose three bf16 terms do not add back to them: the
+    build's exact recompute then reads R_h from global memory instead of its
+    staged terms.  Other heads keep the staged path."""
+    _cuda()
+    w = scaled(WORKLOADS["llama_layer_32k"], context=3000, batch=1, seed=77)
+    li = make_layer(w)
+    R = li.R.clone()
+    R[0, 3, 7] = 1.0e-39   # subnormal: its bf16 split is inexact
+    R[0, 90, 11] = -3.3e-40
+    li.R = R
+    _run_and_check(w, li, e2e=False)
