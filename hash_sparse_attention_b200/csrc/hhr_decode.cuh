@@ -649,11 +649,11 @@ static __device__ __noinline__ int sp_psel(const SpParams& p, unsigned char* sm,
             const uint32_t key = v ? lk2[tid] : 0u;
             const int pg = v ? lp2[tid] : INT_MAX;
             int rank = 0;
-#pragma unroll 4
-            for (int o = 0; o < 32; ++o) {
+            #pragma unroll 1
+            for (int o = 0; o < cnt; ++o) {  // (cnt is the same in every lane)
               const uint32_t k2 = __shfl_sync(0xffffffffu, key, o);
               const int p2 = __shfl_sync(0xffffffffu, pg, o);
-              rank += (o < cnt) && (k2 > key || (k2 == key && p2 < pg));
+              rank += (k2 > key || (k2 == key && p2 < pg));
             }
             if (v && rank < need) atomicOr(&keep[pg >> 5], 1u << (pg & 31));
           }
