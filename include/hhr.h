@@ -214,7 +214,8 @@ HHR_API hhr_status hhr_workspace_init(void* workspace, size_t workspace_bytes, h
  * One kernel launch of at most one CTA per SM (the library checks on the host
  * that a CTA fits on an SM); the CTAs of a group that shares a (sequence, KV
  * head) wait for one another, so the launch expects the SMs it was sized for
- * (a kernel occupying SMs on another stream only delays it).  Every
+ * (a kernel occupying SMs on another stream delays it; one that holds them
+ * past the wait limit makes it end with HHR_ERR_TIMEOUT).  Every
  * device-side wait is bounded (hhr_set_wait_limit): on expiry the launch
  * records HHR_ERR_TIMEOUT in `device_status` and returns.  After any call
  * whose device status is not HHR_OK, zero the workspace again
